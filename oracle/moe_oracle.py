@@ -1,0 +1,300 @@
+"""fp64 CPU oracle for the DiT-MoE sparse expert layer (forward).
+
+TEST INFRASTRUCTURE.  This module is the checker, not the product: only the
+test suite, the smoke check and the benchmark's CPU-baseline leg may import
+it.  It shares no code with the CUDA path and imports nothing from it.
+
+Every function restates one step of the method as the pages define it, in
+plain numpy on float64, with a library primitive (matmul, exp, tanh, a
+stable sort) as a step where one fits and no blocking, fusion or reordering
+beyond the definition.  Sources, by page title and section:
+
+* "Scaling Diffusion Transformers to 16 Billion Parameters" (reading note)
+  - "MOE 回顾", eq. MoE(x): MoE(x) = sum_i g(x)_i e_i(x); g sparse with k of
+    E weights non-zero, so unused experts are not computed.
+  - "MOE-DIT", eq. MLP: MLP(x) = W2 gelu(W1 x); every expert is such an MLP.
+  - "MOE-DIT", shared-expert routing: n_s extra experts that every token is
+    assigned to, whatever the router says.
+  - "MOE-DIT", expert-level balance loss, eq. L_balance.
+* "DiT-MoE" hub page, section 1 "MoE Gate 路由机制": MoEGate with
+  weight (n_routed_experts, gating_dim), softmax scoring, top_k =
+  num_experts_per_tok, aux_loss_alpha.
+* "Scalable Diffusion Models with Transformers (DiT)", "DiT block 实现细节":
+  the core transformer uses the tanh approximation of GELU.
+* "Expert Race: A Flexible Routing Strategy for Scaling Diffusion
+  Transformer with Mixture of Experts", abstract: tokens and experts compete
+  together and the top candidates are selected.
+
+Readings where the pages are silent (each is listed in the design notes):
+g is the softmax score of a selected expert, not renormalised; shared
+experts are summed with weight 1; top-K order is descending score, ties to
+the lower expert id; Expert-Race takes the S = K*T largest of the T x E
+softmax scores, ties to the lower flat index t*E+i; the balance loss's T is
+every token of the call and its n is E; expert biases (nn.Linear) are applied
+inside e_i, before gating.
+
+Parity status: every function here is pinned by a CPU test (closed forms,
+brute force, library special cases, invariants, a hand-worked example).  The
+full-layer numeric output has no worked example on the pages, so beyond those
+pins it is "parity unpinned" against the pages themselves.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import numpy as np
+
+F64 = np.float64
+
+
+def as_f64(a):
+    return None if a is None else np.asarray(a, dtype=F64)
+
+
+# ---------------------------------------------------------------- router
+
+def gate_logits(x, wg, router_bias=None):
+    """l[t,i] = x_t . Wg[i] (+ b_i).
+
+    MoEGate keeps a weight of shape (n_routed_experts, gating_dim) and scores
+    hidden states against it ("DiT-MoE" hub page, section 1).  The router bias
+    is a synthetic load-skew device of the workloads, not on the pages.
+    """
+    l = as_f64(x) @ as_f64(wg).T
+    if router_bias is not None:
+        l = l + as_f64(router_bias)[None, :]
+    return l
+
+
+def softmax_scores(logits):
+    """P[t,i] = exp(l_i - m) / sum_j exp(l_j - m), m = max_j l_j.
+
+    MoEGate's scoring_func is 'softmax' (hub page, section 1); P(t,i) is the
+    probability of expert i for token t in the balance loss ("MOE-DIT").
+    """
+    l = as_f64(logits)
+    m = l.max(axis=1, keepdims=True)
+    e = np.exp(l - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def topk_route(P, K):
+    """Per token, the K largest scores, in descending score, ties to the lower id.
+
+    Returns (idx [T,K] int64, g [T,K] fp64) with g the selected scores themselves
+    (g sparse with K non-zeros, "MOE 回顾"; MoEGate picks top_k experts).
+    """
+    P = as_f64(P)
+    T, E = P.shape
+    idx = np.empty((T, K), dtype=np.int64)
+    for t in range(T):
+        # stable sort on -P keeps equal scores in ascending expert order
+        order = np.argsort(-P[t], kind="stable")
+        idx[t] = order[:K]
+    g = np.take_along_axis(P, idx, axis=1)
+    return idx, g
+
+
+def race_route(P, S):
+    """Expert-Race: the S largest entries of the flattened T x E score matrix.
+
+    Tokens and experts compete together and the top candidates win (Expert
+    Race abstract).  Ties go to the lower flat index t*E+i.  Each token keeps
+    its winners in descending score, ties to the lower expert id.
+    Returns (idx [T,E] int64 padded with -1, g [T,E] fp64 padded with 0,
+    n_sel [T] int64).
+    """
+    P = as_f64(P)
+    T, E = P.shape
+    flat = P.reshape(-1)
+    order = np.argsort(-flat, kind="stable")       # ties: ascending flat index
+    chosen = np.zeros(T * E, dtype=bool)
+    chosen[order[:S]] = True
+    chosen = chosen.reshape(T, E)
+    idx = np.full((T, E), -1, dtype=np.int64)
+    g = np.zeros((T, E), dtype=F64)
+    n_sel = chosen.sum(axis=1).astype(np.int64)
+    for t in range(T):
+        ids = np.nonzero(chosen[t])[0]
+        if ids.size:
+            o = ids[np.argsort(-P[t, ids], kind="stable")]
+            idx[t, :o.size] = o
+            g[t, :o.size] = P[t, o]
+    return idx, g, n_sel
+
+
+def expert_counts(idx, E):
+    """counts[i] = sum_t I(t,i): how many (token, expert) pairs chose expert i."""
+    idx = np.asarray(idx).reshape(-1)
+    idx = idx[idx >= 0]
+    return np.bincount(idx, minlength=E).astype(np.int64)
+
+
+def balance_loss(counts, P, K, alpha):
+    """L = alpha * sum_i (n/(K T) sum_t I(t,i)) * (1/T sum_t P(t,i)), n = E.
+
+    "MOE-DIT", expert-level balance loss; T is the number of tokens of the
+    call, K the experts per token, n the number of routed experts.
+    """
+    P = as_f64(P)
+    T, E = P.shape
+    f = (E / (K * T)) * np.asarray(counts, dtype=F64)
+    p = P.sum(axis=0) / T
+    return float(alpha * np.sum(f * p))
+
+
+# ---------------------------------------------------------------- experts
+
+def gelu_tanh(u):
+    """0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3))): the tanh GELU of the DiT core."""
+    u = as_f64(u)
+    return 0.5 * u * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (u + 0.044715 * u ** 3)))
+
+
+def gelu_erf(u):
+    """0.5 u (1 + erf(u / sqrt 2)): exact GELU (nn.GELU default), kept only as an option."""
+    u = as_f64(u)
+    erf = np.vectorize(math.erf, otypes=[F64])
+    return 0.5 * u * (1.0 + erf(u / math.sqrt(2.0)))
+
+
+def expert_mlp(x, w1, b1, w2, b2, act="tanh"):
+    """e(x) = W2 gelu(W1 x + b1) + b2 for a batch of rows x [n,D].
+
+    "MOE-DIT", eq. MLP: two linear layers with a GELU between; each expert is
+    such an MLP.  Weights are nn.Linear style: w1 [H,D], w2 [D,H].
+    """
+    sigma = gelu_tanh if act == "tanh" else gelu_erf
+    u = as_f64(x) @ as_f64(w1).T
+    if b1 is not None:
+        u = u + as_f64(b1)[None, :]
+    y = sigma(u) @ as_f64(w2).T
+    if b2 is not None:
+        y = y + as_f64(b2)[None, :]
+    return y
+
+
+# ---------------------------------------------------------------- layer
+
+def route(inp, K, routing="topk", alpha=0.01):
+    """Router half of the layer: logits, scores, selection, counts, balance loss."""
+    P = softmax_scores(gate_logits(inp["x"], inp["wg"], inp.get("router_bias")))
+    T, E = P.shape
+    if routing == "race":
+        idx, g, n_sel = race_route(P, K * T)
+    else:
+        idx, g = topk_route(P, K)
+        n_sel = np.full(T, K, dtype=np.int64)
+    counts = expert_counts(idx, E)
+    return {"P": P, "idx": idx, "g": g, "n_sel": n_sel, "counts": counts,
+            "aux": balance_loss(counts, P, K, alpha)}
+
+
+def _bias_row(b, j):
+    return None if b is None else b[j]
+
+
+def layer_output(inp, idx, g, n_sel=None, tokens=None, act="tanh"):
+    """MoE(x_t) = sum_{i in sel_t} g_{t,i} e_i(x_t) + sum_j s_j(x_t).
+
+    "MOE 回顾", eq. MoE(x), with the sparse g (only selected experts are
+    evaluated), plus the shared experts of "MOE-DIT" with weight 1.
+    ``idx``/``g`` hold each token's selection (-1 padded); ``tokens`` restricts
+    the evaluation to a subset of rows (the others are not computed).
+    """
+    x = as_f64(inp["x"])
+    T = x.shape[0]
+    tok = np.arange(T) if tokens is None else np.asarray(tokens)
+    idx = np.asarray(idx)[tok]
+    g = as_f64(g)[tok]
+    xs = x[tok]
+    out = np.zeros((tok.size, x.shape[1]), dtype=F64)
+    E = inp["w1"].shape[0]
+    for e in range(E):
+        rows, slots = np.nonzero(idx == e)
+        if rows.size == 0:
+            continue
+        y = expert_mlp(xs[rows], inp["w1"][e], _bias_row(inp.get("b1"), e),
+                       inp["w2"][e], _bias_row(inp.get("b2"), e), act)
+        np.add.at(out, rows, g[rows, slots][:, None] * y)
+    for j in range(inp["ws1"].shape[0]):
+        out += expert_mlp(xs, inp["ws1"][j], _bias_row(inp.get("bs1"), j),
+                          inp["ws2"][j], _bias_row(inp.get("bs2"), j), act)
+    return out
+
+
+def layer(inp, K, routing="topk", alpha=0.01, act="tanh"):
+    """Whole layer: route, evaluate the selected and the shared experts, combine."""
+    r = route(inp, K, routing, alpha)
+    r["out"] = layer_output(inp, r["idx"], r["g"], r["n_sel"], act=act)
+    return r
+
+
+def dense_masked_output(inp, g_dense, act="tanh"):
+    """MoE(x) = sum_{i=1..E} g(x)_i e_i(x) evaluated densely over all E experts.
+
+    The un-sparsified form of "MOE 回顾": every expert runs on every token and
+    is multiplied by a gate vector that is zero off the selection.
+    """
+    x = as_f64(inp["x"])
+    out = np.zeros_like(x)
+    for e in range(inp["w1"].shape[0]):
+        y = expert_mlp(x, inp["w1"][e], _bias_row(inp.get("b1"), e),
+                       inp["w2"][e], _bias_row(inp.get("b2"), e), act)
+        out += as_f64(g_dense)[:, e:e + 1] * y
+    for j in range(inp["ws1"].shape[0]):
+        out += expert_mlp(x, inp["ws1"][j], _bias_row(inp.get("bs1"), j),
+                          inp["ws2"][j], _bias_row(inp.get("bs2"), j), act)
+    return out
+
+
+def dense_gate(idx, g, T, E):
+    """Scatter a (-1 padded) selection into a dense [T,E] gate matrix."""
+    gd = np.zeros((T, E), dtype=F64)
+    idx = np.asarray(idx)
+    for t in range(T):
+        for k in range(idx.shape[1]):
+            if idx[t, k] >= 0:
+                gd[t, idx[t, k]] = g[t, k]
+    return gd
+
+
+# ---------------------------------------------------------------- permutation
+
+def canonical_permutation(idx, E, tile=128):
+    """Expert-contiguous order of the selected (token, expert) pairs.
+
+    Computing only the selected experts ("MOE 回顾": unused experts need not
+    be computed) means gathering each expert's tokens into one block.  The
+    canonical order: expert segments in ascending expert id, tokens ascending
+    inside a segment; segment i starts at padded_offsets[i], the sum of the
+    earlier segment lengths rounded up to ``tile`` rows.
+    Returns counts [E], offsets [E+1] (unpadded), padded_offsets [E+1],
+    pos [T,Kmax] (-1 where unselected) and row_token [R] (-1 on pad rows),
+    row_slot [R] (which of the token's slots the row serves, -1 on pad).
+    """
+    idx = np.asarray(idx)
+    T, Kmax = idx.shape
+    counts = expert_counts(idx, E)
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    padded = np.zeros(E + 1, dtype=np.int64)
+    padded[1:] = np.cumsum((counts + tile - 1) // tile * tile)
+    R = int(padded[-1])
+    pos = np.full((T, Kmax), -1, dtype=np.int64)
+    row_token = np.full(R, -1, dtype=np.int64)
+    row_slot = np.full(R, -1, dtype=np.int64)
+    fill = padded[:-1].copy()
+    for t in range(T):                      # ascending tokens inside each segment
+        for k in range(Kmax):
+            e = idx[t, k]
+            if e < 0:
+                continue
+            r = fill[e]
+            fill[e] += 1
+            pos[t, k] = r
+            row_token[r] = t
+            row_slot[r] = k
+    return {"counts": counts, "offsets": offsets, "padded_offsets": padded,
+            "pos": pos, "row_token": row_token, "row_slot": row_slot}

@@ -1,0 +1,363 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these compares the oracle with itself: each check is a closed form, a
+hand-worked example from tests/golden (with its citation), a brute force on a
+tiny input, a library routine for a special case, or an invariant.  The
+mutation tests at the end plant a plausible mistake in the oracle and check
+that some pin catches it.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from sparse_moe_layer_03_b200 import inputs as I
+from sparse_moe_layer_03_b200 import metrics as M
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_scores(T, E, seed):
+    rng = np.random.default_rng(seed)
+    return O.softmax_scores(rng.standard_normal((T, E)) * 2.0)
+
+
+# ------------------------------------------------------------------ softmax
+
+def test_softmax_rows_sum_to_one_and_argmax():
+    rng = np.random.default_rng(0)
+    l = rng.standard_normal((300, 16)) * 5
+    P = O.softmax_scores(l)
+    assert np.all(P >= 0)
+    assert np.max(np.abs(P.sum(1) - 1.0)) < 1e-12
+    assert np.array_equal(P.argmax(1), l.argmax(1))
+
+
+def test_softmax_matches_library_and_shift_invariance():
+    rng = np.random.default_rng(1)
+    l = rng.standard_normal((64, 8)) * 3
+    ref = torch.softmax(torch.from_numpy(l), dim=1).numpy()
+    assert np.max(np.abs(O.softmax_scores(l) - ref)) < 1e-14
+    assert np.max(np.abs(O.softmax_scores(l + 7.25) - O.softmax_scores(l))) < 1e-14
+
+
+def test_gate_logits_library():
+    rng = np.random.default_rng(2)
+    x, wg, b = rng.standard_normal((10, 12)), rng.standard_normal((4, 12)), rng.standard_normal(4)
+    ref = torch.nn.functional.linear(torch.from_numpy(x), torch.from_numpy(wg), torch.from_numpy(b))
+    assert np.allclose(O.gate_logits(x, wg, b), ref.numpy(), rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------------ top-K
+
+@pytest.mark.parametrize("K", [1, 2, 3, 8])
+def test_topk_equals_brute_force(K):
+    E = 8
+    P = _rand_scores(120, E, 3 + K)
+    idx, g = O.topk_route(P, K)
+    for t in range(P.shape[0]):
+        best = max(itertools.combinations(range(E), K), key=lambda c: sum(P[t, i] for i in c))
+        assert set(idx[t]) == set(best)
+        assert all(P[t, idx[t, k]] >= P[t, idx[t, k + 1]] for k in range(K - 1))
+        assert np.array_equal(g[t], P[t, idx[t]])
+    if K == E:
+        assert all(sorted(r) == list(range(E)) for r in idx.tolist())
+
+
+def test_topk_ties_take_lower_id():
+    P = np.array([[0.25, 0.25, 0.25, 0.25], [0.1, 0.4, 0.4, 0.1]])
+    idx, _ = O.topk_route(P, 2)
+    assert idx.tolist() == [[0, 1], [1, 2]]
+
+
+# ------------------------------------------------------------------ race
+
+def test_race_single_token_equals_topk():
+    P = _rand_scores(1, 16, 7)
+    idx, g, n = O.race_route(P, 2)
+    idk, gk = O.topk_route(P, 2)
+    assert n.tolist() == [2] and idx[0, :2].tolist() == idk[0].tolist()
+
+
+def test_race_all_selected_when_k_equals_e():
+    P = _rand_scores(9, 4, 8)
+    idx, g, n = O.race_route(P, 9 * 4)
+    assert n.tolist() == [4] * 9
+    assert all(sorted(r) == [0, 1, 2, 3] for r in idx.tolist())
+
+
+@pytest.mark.parametrize("T,E,K", [(4, 3, 1), (3, 4, 2), (5, 2, 1)])
+def test_race_brute_force_tiny(T, E, K):
+    P = _rand_scores(T, E, 10 * T + E)
+    S = K * T
+    idx, g, n = O.race_route(P, S)
+    flat = [(P[t, i], t, i) for t in range(T) for i in range(E)]
+    best = max(itertools.combinations(range(T * E), S), key=lambda c: sum(flat[f][0] for f in c))
+    want = {(flat[f][1], flat[f][2]) for f in best}
+    got = {(t, int(idx[t, k])) for t in range(T) for k in range(n[t])}
+    assert got == want and n.sum() == S
+    for t in range(T):
+        sel = idx[t, :n[t]]
+        assert all(P[t, sel[k]] >= P[t, sel[k + 1]] for k in range(len(sel) - 1))
+        assert np.all(idx[t, n[t]:] == -1)
+
+
+# ------------------------------------------------------------------ counts and loss
+
+def test_counts_sum_and_histogram():
+    P = _rand_scores(333, 8, 11)
+    idx, _ = O.topk_route(P, 2)
+    c = O.expert_counts(idx, 8)
+    assert c.sum() == 2 * 333
+    brute = [0] * 8
+    for row in idx.tolist():
+        for e in row:
+            brute[e] += 1
+    assert c.tolist() == brute
+
+
+def test_balance_loss_uniform_scores_gives_alpha():
+    # Wg = 0 and no bias: every P = 1/E, so p_i = 1/E and sum_i f_i = E -> L = alpha
+    T, D, E, K = 64, 16, 8, 2
+    x = np.random.default_rng(0).standard_normal((T, D))
+    r = O.route({"x": x, "wg": np.zeros((E, D))}, K, "topk", 0.05)
+    assert abs(r["aux"] - 0.05) < 1e-15
+    r = O.route({"x": x, "wg": np.zeros((E, D))}, K, "race", 0.05)
+    assert abs(r["aux"] - 0.05) < 1e-15
+
+
+def test_balance_loss_single_expert_gives_alpha():
+    x = np.random.default_rng(1).standard_normal((17, 8))
+    r = O.route({"x": x, "wg": np.random.default_rng(2).standard_normal((1, 8))}, 1, "topk", 0.01)
+    assert r["counts"].tolist() == [17] and abs(r["aux"] - 0.01) < 1e-16
+
+
+def test_balance_loss_uniform_counts_gives_alpha():
+    # hand-built router: token t points along expert (t mod E) -> counts all T*K/E
+    E, T = 4, 40
+    x = np.zeros((T, E))
+    for t in range(T):
+        x[t, t % E] = 3.0 + 0.01 * t
+    r = O.route({"x": x, "wg": np.eye(E)}, 1, "topk", 0.01)
+    assert r["counts"].tolist() == [T // E] * E
+    assert abs(r["aux"] - 0.01) < 1e-15
+
+
+def test_balance_loss_partial_sums():
+    P = _rand_scores(50, 8, 12)
+    idx, _ = O.topk_route(P, 2)
+    c = O.expert_counts(idx, 8)
+    f = 8 / (2 * 50) * c
+    assert abs(f.sum() - 8) < 1e-12 and abs(P.sum(0).sum() / 50 - 1) < 1e-12
+
+
+def _golden_x(a_list):
+    a = {"ln3": math.log(3.0), "-ln3": -math.log(3.0), "0": 0.0}
+    return np.array([[a[s], 0.0] for s in a_list])
+
+
+def test_worked_example_balance_and_race():
+    g = json.load(open(os.path.join(GOLDEN, "balance_worked_example.json")))
+    wg = np.array([[1.0, 0.0], [0.0, 0.0]])
+    for case in g["cases"]:
+        x = _golden_x(case["a"])
+        inp = {"x": x, "wg": wg}
+        for mode in ("topk", "race"):
+            r = O.route(inp, case["K"], mode, g["alpha"])
+            want = case[mode]
+            assert np.allclose(r["P"], case["P"], atol=1e-15)
+            assert r["idx"].tolist() == want["idx"], (case["name"], mode)
+            assert r["counts"].tolist() == want["counts"]
+            if mode == "race":
+                assert r["n_sel"].tolist() == want["n_sel"]
+            assert abs(r["aux"] - want["loss"]) < 1e-15
+
+
+# ------------------------------------------------------------------ experts
+
+def test_gelu_tanh_matches_library_and_identity():
+    u = np.linspace(-8, 8, 4001)
+    ref = torch.nn.functional.gelu(torch.from_numpy(u), approximate="tanh").numpy()
+    assert np.max(np.abs(O.gelu_tanh(u) - ref)) < 1e-14
+    assert np.max(np.abs(O.gelu_tanh(u) - O.gelu_tanh(-u) - u)) < 1e-13
+    assert O.gelu_tanh(np.array([0.0]))[0] == 0.0
+
+
+def test_gelu_erf_matches_library_and_differs_from_tanh():
+    u = np.linspace(-6, 6, 1201)
+    ref = torch.nn.functional.gelu(torch.from_numpy(u)).numpy()
+    assert np.max(np.abs(O.gelu_erf(u) - ref)) < 1e-14
+    assert np.max(np.abs(O.gelu_erf(u) - O.gelu_tanh(u))) > 1e-4
+
+
+def test_expert_mlp_matches_library():
+    rng = np.random.default_rng(5)
+    D, H = 24, 96
+    x = rng.standard_normal((13, D))
+    w1, b1 = rng.standard_normal((H, D)) / 5, rng.standard_normal(H)
+    w2, b2 = rng.standard_normal((D, H)) / 10, rng.standard_normal(D)
+    tt = lambda a: torch.from_numpy(a)
+    ref = torch.nn.functional.linear(
+        torch.nn.functional.gelu(torch.nn.functional.linear(tt(x), tt(w1), tt(b1)), approximate="tanh"),
+        tt(w2), tt(b2)).numpy()
+    assert np.max(np.abs(O.expert_mlp(x, w1, b1, w2, b2) - ref)) < 1e-12
+
+
+def _small_inputs(T=40, D=32, H=64, E=4, K=2, ns=2, bias=0.3, seed=9, routing="topk"):
+    w = I.small_workload(T, D, H, E, K, ns, "f32", routing, seed)
+    return w, I.make_inputs(w, bias_std=bias)
+
+
+def test_single_expert_reduces_to_dense_mlp():
+    w, inp = _small_inputs(E=1, K=1, ns=0)
+    r = O.layer(inp, 1)
+    tt = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    ref = torch.nn.functional.linear(
+        torch.nn.functional.gelu(torch.nn.functional.linear(tt(inp["x"]), tt(inp["w1"][0]), tt(inp["b1"][0])),
+                                 approximate="tanh"), tt(inp["w2"][0]), tt(inp["b2"][0])).numpy()
+    assert np.all(r["g"] == 1.0)
+    assert np.max(np.abs(r["out"] - ref)) < 1e-12
+
+
+@pytest.mark.parametrize("routing", ["topk", "race"])
+def test_sparse_equals_dense_masked(routing):
+    w, inp = _small_inputs(T=48, E=8, K=2, routing=routing)
+    r = O.layer(inp, 2, routing)
+    gd = O.dense_gate(r["idx"], r["g"], 48, 8)
+    dense = O.dense_masked_output(inp, gd)
+    assert np.max(np.abs(r["out"] - dense)) < 1e-12
+
+
+def test_shared_concat_identity():
+    w, inp = _small_inputs(E=2, ns=3)
+    x = torch.from_numpy(inp["x"].astype(np.float64))
+    w1c = torch.from_numpy(np.concatenate(list(inp["ws1"]), 0).astype(np.float64))
+    b1c = torch.from_numpy(np.concatenate(list(inp["bs1"]), 0).astype(np.float64))
+    w2c = torch.from_numpy(np.concatenate(list(inp["ws2"]), 1).astype(np.float64))
+    b2c = torch.from_numpy(inp["bs2"].astype(np.float64).sum(0))
+    cat = torch.nn.functional.linear(
+        torch.nn.functional.gelu(torch.nn.functional.linear(x, w1c, b1c), approximate="tanh"), w2c, b2c).numpy()
+    zero = dict(inp)
+    zero["w2"] = np.zeros_like(inp["w2"])
+    zero["b2"] = None
+    r = O.layer(zero, 2)
+    assert np.max(np.abs(r["out"] - cat)) < 1e-12
+
+
+def test_token_permutation_and_expert_relabelling():
+    w, inp = _small_inputs(T=30, E=6, K=2)
+    base = O.layer(inp, 2)["out"]
+    perm = np.random.default_rng(0).permutation(30)
+    p_inp = dict(inp)
+    p_inp["x"] = inp["x"][perm]
+    assert np.max(np.abs(O.layer(p_inp, 2)["out"] - base[perm])) < 1e-12
+    lab = np.random.default_rng(1).permutation(6)
+    r_inp = dict(inp)
+    for k in ("wg", "w1", "w2", "b1", "b2"):
+        r_inp[k] = inp[k][lab]
+    assert np.max(np.abs(O.layer(r_inp, 2)["out"] - base)) < 1e-12
+
+
+# ------------------------------------------------------------------ permutation
+
+@pytest.mark.parametrize("routing", ["topk", "race"])
+def test_canonical_permutation_properties(routing):
+    P = _rand_scores(300, 8, 21)
+    idx = O.topk_route(P, 2)[0] if routing == "topk" else O.race_route(P, 600)[0]
+    cp = O.canonical_permutation(idx, 8)
+    po = cp["padded_offsets"]
+    assert np.all(po % 128 == 0)
+    # independent construction: sort the (expert, token) pairs
+    t_of, k_of = np.nonzero(idx >= 0)
+    e_of = idx[t_of, k_of]
+    order = np.lexsort((t_of, e_of))
+    for e in range(8):
+        seg = cp["row_token"][po[e]:po[e] + cp["counts"][e]]
+        assert np.all(np.diff(seg) > 0)
+        assert set(seg.tolist()) == set(np.nonzero((idx == e).any(1))[0].tolist())
+        assert np.all(cp["row_token"][po[e] + cp["counts"][e]:po[e + 1]] == -1)
+    rows = cp["pos"][t_of[order], k_of[order]]
+    assert np.array_equal(cp["row_token"][rows], t_of[order])
+    assert np.array_equal(cp["offsets"][1:], np.cumsum(cp["counts"]))
+
+
+# ------------------------------------------------------------------ accounting and inputs
+
+def test_flop_convention_reproduces_dit_gflops():
+    g = json.load(open(os.path.join(GOLDEN, "dit_xl2_gflops.json")))
+    D, L, p, C = g["hidden"], g["depth"], g["patch"], g["latent_channels"]
+    H = g["mlp_ratio"] * D
+    for case in g["cases"]:
+        N = case["tokens"]
+        per_block = N * M.mlp_macs_per_token(D, H) + N * 4 * D * D + 2 * N * N * D + 6 * D * D
+        embed = N * p * p * C * D + g["frequency_embedding"] * D + D * D
+        final = N * D * p * p * 2 * C + 2 * D * D
+        gmacs = (L * per_block + embed + final) / 1e9
+        assert abs(gmacs / case["printed_gflops"] - 1) < 2e-3, gmacs
+
+
+def test_layer_flops_xl():
+    w = I.WORKLOADS["xl2_8e2a_512"]
+    f = M.gemm_flops(w.T, w.D, w.H, w.K, w.n_shared)
+    assert abs(f / 2.7831e12 - 1) < 1e-4
+
+
+def test_inputs_seeded_and_bf16_exact():
+    w = I.small_workload(20, 16, 32, 4, 2, 1, "bf16", seed=3)
+    a, b = I.make_inputs(w), I.make_inputs(w)
+    assert np.array_equal(a["w1"], b["w1"])
+    t = torch.from_numpy(np.random.default_rng(0).standard_normal(10000).astype(np.float32))
+    assert torch.equal(torch.from_numpy(I.round_to_bf16(t.numpy())), t.to(torch.bfloat16).float())
+    assert torch.equal(torch.from_numpy(a["x"]).to(torch.bfloat16).float(), torch.from_numpy(a["x"]))
+
+
+# ------------------------------------------------------------------ planted mistakes
+
+def test_planted_gelu_sign_is_caught(monkeypatch):
+    bad = lambda u: 0.5 * u * (1.0 - np.tanh(math.sqrt(2 / math.pi) * (u + 0.044715 * u ** 3)))
+    monkeypatch.setattr(O, "gelu_tanh", bad)
+    with pytest.raises(AssertionError):
+        test_gelu_tanh_matches_library_and_identity()
+
+
+def test_planted_loss_factor_is_caught(monkeypatch):
+    def bad(counts, P, K, alpha):
+        T, E = P.shape
+        return float(alpha * np.sum((1 / (K * T)) * counts * P.sum(0) / T))
+    monkeypatch.setattr(O, "balance_loss", bad)
+    with pytest.raises(AssertionError):
+        test_balance_loss_uniform_scores_gives_alpha()
+
+
+def test_planted_dropped_bias_is_caught(monkeypatch):
+    def bad(x, w1, b1, w2, b2, act="tanh"):
+        u = np.asarray(x, np.float64) @ np.asarray(w1, np.float64).T     # b1 dropped
+        y = O.gelu_tanh(u) @ np.asarray(w2, np.float64).T
+        return y if b2 is None else y + b2
+    monkeypatch.setattr(O, "expert_mlp", bad)
+    with pytest.raises(AssertionError):
+        test_expert_mlp_matches_library()
+
+
+def test_planted_race_tie_order_is_caught(monkeypatch):
+    def bad(P, S):
+        P = np.asarray(P, np.float64)
+        T, E = P.shape
+        order = np.lexsort((-np.arange(T * E), -P.reshape(-1)))   # ties to the higher flat index
+        chosen = np.zeros(T * E, bool)
+        chosen[order[:S]] = True
+        chosen = chosen.reshape(T, E)
+        idx = np.full((T, E), -1, np.int64)
+        for t in range(T):
+            ids = np.nonzero(chosen[t])[0]
+            idx[t, :ids.size] = ids[np.argsort(-P[t, ids], kind="stable")]
+        g = np.where(idx >= 0, np.take_along_axis(P, np.maximum(idx, 0), 1), 0.0)
+        return idx, g, chosen.sum(1)
+    monkeypatch.setattr(O, "race_route", bad)
+    with pytest.raises(AssertionError):
+        test_worked_example_balance_and_race()

@@ -1,0 +1,198 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) DiT-MoE sparse expert layer, forward.
+ *
+ * The layer (for every image-patch token x_t, width D):
+ *   logits  l[t,i] = x_t . Wg[i] (+ b_i)                 i = 0..E-1
+ *   scores  P[t,i] = softmax_i(l[t,:])
+ *   select  top-K experts per token (or Expert-Race: the S = K*T largest P
+ *           over the whole T x E matrix), gate g[t,i] = P[t,i] on the selection
+ *   output  MoE(x_t) = sum_{i in sel_t} g[t,i] e_i(x_t) + sum_{j<n_s} s_j(x_t)
+ *           e_i(x) = W2_i gelu_tanh(W1_i x + b1_i) + b2_i   (same form for s_j)
+ *   loss    L = alpha * sum_i (E/(K T)) counts_i * (1/T) sum_t P[t,i]
+ *
+ * Sources (page title, section):
+ *   "Scaling Diffusion Transformers to 16 Billion Parameters" (reading note):
+ *     "MOE 回顾" eq. MoE(x); "MOE-DIT" eq. MLP, shared-expert routing,
+ *     expert-level balance loss eq. L_balance.
+ *   "DiT-MoE" hub page, section 1 "MoE Gate 路由机制": MoEGate (weight
+ *     (n_routed_experts, gating_dim), softmax scoring, top_k, aux_loss_alpha).
+ *   "Scalable Diffusion Models with Transformers (DiT)", "DiT block 实现细节":
+ *     tanh-approximate GELU in the core transformer.
+ *   "Expert Race: A Flexible Routing Strategy for Scaling Diffusion
+ *     Transformer with Mixture of Experts", abstract: tokens and experts
+ *     compete together and the top candidates win.
+ *
+ * Conventions for every entry point:
+ *   - Every pointer argument named as a tensor is DEVICE memory owned by the
+ *     caller; the library never allocates, frees or keeps it.  Tensors are
+ *     row-major and contiguous; every tensor pointer must be 16-byte aligned.
+ *   - "act" tensors (x, x_perm, h_perm, h_sh, out) and weights/biases have the
+ *     storage type cfg->dtype (fp32 or bf16); scores, gates, y_perm, y_sh are
+ *     fp32; indices are int32.
+ *   - Weights follow nn.Linear (out x in): W1 [E,H,D], b1 [E,H], W2 [E,D,H],
+ *     b2 [E,D].  The n_s shared experts come stacked the same way: W1s
+ *     [n_s,H,D], b1s [n_s,H], W2s [n_s,D,H], b2s [n_s,D].  The kernels treat
+ *     W1s as one [n_s*H, D] layer and sum_j W2_j h_j + sum_j b2_j as one
+ *     K = n_s*H contraction, which is sum_j s_j(x) exactly.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream), never synchronise and never read device data on the
+ *     host.  Group sizes stay on the device.
+ *   - `ws` is caller-owned device scratch of at least moe_workspace_size(cfg)
+ *     bytes, 256-byte aligned.  Its first 256 bytes hold a status word that
+ *     kernels set on a device-detected error (bad index, a bounded wait that
+ *     ran out); moe_workspace_init() clears it and moe_check_status() reads it.
+ *     A workspace must not be shared by calls that may overlap on the GPU.
+ *   - Return value: MOE_OK, or a negative moe_status_t with a message
+ *     available from moe_last_error() (thread-local).  Argument errors are
+ *     detected on the host before anything is launched.
+ *   - T = 0 is valid: outputs are empty, counts are zeroed and aux_loss = 0.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1,  /* null / misaligned pointer, bad size, K > E ... */
+  MOE_ERR_UNSUPPORTED = -2,  /* valid but not built: D or H not a multiple of 64, E > 32 ... */
+  MOE_ERR_WORKSPACE = -3,    /* ws_bytes < moe_workspace_size(cfg) */
+  MOE_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed */
+  MOE_ERR_DEVICE_CHECK = -5, /* a kernel found a bad index (status word) */
+  MOE_ERR_TIMEOUT = -6       /* a kernel's bounded wait ran out (status word) */
+} moe_status_t;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+typedef enum { MOE_ROUTE_TOPK = 0, MOE_ROUTE_RACE = 1 } moe_routing_t;
+typedef enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SIMT = 1 } moe_gemm_impl_t;
+
+typedef struct {
+  int32_t T;         /* tokens in this call (batch x patch tokens), >= 0 */
+  int32_t D;         /* model width (MoEGate gating_dim), multiple of 64 */
+  int32_t H;         /* expert hidden width, multiple of 64 */
+  int32_t E;         /* routed experts (n_routed_experts), 1..32 */
+  int32_t K;         /* experts per token (top_k); race: S = K*T winners, 1..E */
+  int32_t n_shared;  /* shared experts n_s, 0..8 */
+  int32_t dtype;     /* moe_dtype_t: storage type of activations and weights */
+  int32_t routing;   /* moe_routing_t */
+  float alpha;       /* balance-loss factor (aux_loss_alpha) */
+  int32_t act;       /* 0 = gelu tanh form (DiT core), 1 = exact erf form */
+  int32_t gemm_impl; /* moe_gemm_impl_t: AUTO = tcgen05 for bf16, FFMA for fp32 */
+  int32_t reserved;  /* must be 0 */
+} moe_config_t;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int32_t moe_version(void);
+
+/* Message of the last failing call on this thread ("" if none). */
+const char* moe_last_error(void);
+
+/* Bytes of scratch `ws` that every call of this configuration needs (host only). */
+size_t moe_workspace_size(const moe_config_t* cfg);
+
+/* Row capacity R_max of the expert-contiguous buffers x_perm, h_perm, y_perm,
+ * row_token, row_gate: each expert segment starts on a 128-row boundary, so
+ * R_max = round_up(K*T + 127*E, 128).  Host only. */
+int64_t moe_max_rows(const moe_config_t* cfg);
+
+/* Zero the status word of `ws` (asynchronous on `stream`). */
+int moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read the status word of `ws`, clear it, and return
+ * MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT.  The only call that blocks. */
+int moe_check_status(void* ws, void* stream);
+
+/*
+ * moe_route -- router of the layer (MoEGate): gate logits, softmax, selection,
+ * per-expert counts and the expert-level balance loss.
+ *   x           [T,D] act      input tokens
+ *   wg          [E,D] act      gate weight
+ *   router_bias [E] fp32 or NULL   added to the logits
+ *   topk_idx    [T,Kmax] int32 out  Kmax = K (top-K) or E (race).  Each token's
+ *               experts in descending score, ties to the lower id; race pads
+ *               a token's unused slots with -1
+ *   topk_w      [T,Kmax] fp32 out   g = the selected softmax scores (not
+ *               renormalised); 0 on padded slots
+ *   n_sel       [T] int32 out or NULL  experts chosen per token (race:
+ *               required, 0..E; top-K: K for every token)
+ *   counts      [E] int32 out   sum_t I(t,i)
+ *   aux_loss    [1] fp32 out    L_balance with T = this call's tokens
+ * Race selection: the S = K*T largest scores of the flattened T x E matrix,
+ * ties to the lower flat index t*E+i, found by an exact radix select on the
+ * fp32 score bits.
+ */
+int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
+              int32_t* topk_idx, float* topk_w, int32_t* n_sel, int32_t* counts, float* aux_loss,
+              void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_dispatch -- permute tokens into expert-contiguous order (only the
+ * selected experts are computed, "MOE 回顾").  Expert i's rows occupy
+ * [P_i, P_i + counts_i) with P_i = sum_{j<i} round_up(counts_j, 128); tokens
+ * ascend inside a segment.  Deterministic (no order-dependent atomics).
+ *   x          [T,D] act          tokens
+ *   topk_idx   [T,Kmax] int32     from moe_route (-1 = unused slot)
+ *   topk_w     [T,Kmax] fp32      gates
+ *   n_sel      [T] int32 or NULL  NULL means K for every token (top-K)
+ *   offsets    [E+1] int32 out    unpadded exclusive scan of the counts
+ *   pos        [T,Kmax] int32 out row of (t, slot k) in the permuted buffers, -1 if unused
+ *   row_token  [R_max] int32 out  token of each row, -1 on padding rows
+ *   row_gate   [R_max] fp32 out   gate of each row, 0 on padding rows
+ *   x_perm     [R_max,D] act out  x_perm[pos[t,k]] = x[t]; padding rows untouched
+ * An index outside [0,E) is skipped and sets MOE_ERR_DEVICE_CHECK in ws.
+ */
+int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const float* topk_w,
+                 const int32_t* n_sel, int32_t* offsets, int32_t* pos, int32_t* row_token,
+                 float* row_gate, void* x_perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_gemm1 -- first expert layer with bias and GELU fused:
+ *   h_perm[r] = gelu(W1_{e(r)} x_perm[r] + b1_{e(r)})  for the rows of every
+ *               expert segment (e(r) read from `offsets` on the device)
+ *   h_sh[t]   = gelu(W1s x[t] + b1s)  (all n_s shared experts side by side)
+ *   offsets [E+1] int32 (moe_dispatch output); b1 [E,H] / b1s [n_s,H] may be NULL;
+ *   h_perm [R_max,H] act out; h_sh [T,n_s*H] act out (NULL when n_s = 0).
+ * bf16: one persistent tcgen05 kernel (TMA-fed, TMEM accumulators) runs the
+ * routed segments and the shared block together.  fp32: FFMA kernel.
+ */
+int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
+                     const void* x, const void* w1, const void* b1, const void* w1s, const void* b1s,
+                     void* h_perm, void* h_sh, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_gemm2 -- second expert layer with bias and gate scaling fused:
+ *   y_perm[r] = row_gate[r] * (W2_{e(r)} h_perm[r] + b2_{e(r)})   fp32 [R_max,D]
+ *   y_sh[t]   = sum_j (W2s_j h_sh[t, j*H:(j+1)*H] + b2s_j)         fp32 [T,D]
+ *   b2 [E,D] / b2s [n_s,D] may be NULL; y_sh NULL when n_s = 0.
+ */
+int moe_expert_gemm2(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm,
+                     const void* h_sh, const void* w2, const void* b2, const void* w2s,
+                     const void* b2s, const float* row_gate, float* y_perm, float* y_sh,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* moe_expert_mlp -- moe_expert_gemm1 followed by moe_expert_gemm2. */
+int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
+                   const void* x, const void* w1, const void* b1, const void* w2, const void* b2,
+                   const void* w1s, const void* b1s, const void* w2s, const void* b2s,
+                   const float* row_gate, void* h_perm, void* h_sh, float* y_perm, float* y_sh,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_combine -- MoE(x_t) = sum_{k < n_sel[t]} y_perm[pos[t,k]] + y_sh[t]
+ * (the gates are already applied in y_perm), summed in fp32 in slot order
+ * then the shared term, rounded once to the act type.
+ *   y_perm [R_max,D] fp32; y_sh [T,D] fp32 or NULL (n_s = 0);
+ *   pos [T,Kmax] int32; n_sel [T] or NULL (= K); out [T,D] act.
+ */
+int moe_combine(const moe_config_t* cfg, const float* y_perm, const float* y_sh,
+                const int32_t* pos, const int32_t* n_sel, void* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

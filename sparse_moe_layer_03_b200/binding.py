@@ -1,0 +1,153 @@
+"""ctypes binding of ``libmoe.so``: the C-ABI entry points under the same names.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  Tensors are passed as device pointers (``torch.Tensor.data_ptr()``)
+and the stream as a raw ``cudaStream_t``.  Importing this module loads the
+library and raises if it is missing: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, -1, -2, -3
+MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT = -4, -5, -6
+MOE_F32, MOE_BF16 = 0, 1
+MOE_ROUTE_TOPK, MOE_ROUTE_RACE = 0, 1
+MOE_GEMM_AUTO, MOE_GEMM_SIMT = 0, 1
+
+
+class MoeConfig(C.Structure):
+    _fields_ = [("T", C.c_int32), ("D", C.c_int32), ("H", C.c_int32), ("E", C.c_int32),
+                ("K", C.c_int32), ("n_shared", C.c_int32), ("dtype", C.c_int32),
+                ("routing", C.c_int32), ("alpha", C.c_float), ("act", C.c_int32),
+                ("gemm_impl", C.c_int32), ("reserved", C.c_int32)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"moe error {code}: {msg}")
+        self.code = code
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparse_moe_layer_03_b200.build` "
+                      "(the CUDA library is required; there is no CPU path)")
+lib = C.CDLL(LIB_PATH)
+
+_P = C.c_void_p
+_CFG = C.POINTER(MoeConfig)
+_SIGS = {
+    "moe_version": (C.c_int32, []),
+    "moe_last_error": (C.c_char_p, []),
+    "moe_workspace_size": (C.c_size_t, [_CFG]),
+    "moe_max_rows": (C.c_int64, [_CFG]),
+    "moe_workspace_init": (C.c_int, [_P, C.c_size_t, _P]),
+    "moe_check_status": (C.c_int, [_P, _P]),
+    "moe_route": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "moe_dispatch": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "moe_expert_gemm1": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "moe_expert_gemm2": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "moe_expert_mlp": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                 _P, C.c_size_t, _P]),
+    "moe_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def header_symbols(path: str = HEADER) -> list:
+    """Names of the functions that include/moe.h declares."""
+    text = open(path).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\*\s]+?\b(moe_\w+)\s*\(", text, re.M)))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _check(rc: int):
+    if rc != MOE_OK:
+        raise MoeError(rc, lib.moe_last_error().decode())
+
+
+def make_config(T, D, H, E, K, n_shared, dtype="bf16", routing="topk", alpha=0.01, act="tanh",
+                gemm_impl="auto") -> MoeConfig:
+    return MoeConfig(T, D, H, E, K, n_shared, MOE_BF16 if dtype == "bf16" else MOE_F32,
+                     MOE_ROUTE_RACE if routing == "race" else MOE_ROUTE_TOPK, alpha,
+                     1 if act == "erf" else 0, MOE_GEMM_SIMT if gemm_impl == "simt" else MOE_GEMM_AUTO, 0)
+
+
+def moe_version() -> int:
+    return lib.moe_version()
+
+
+def moe_workspace_size(cfg: MoeConfig) -> int:
+    n = lib.moe_workspace_size(C.byref(cfg))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, lib.moe_last_error().decode())
+    return n
+
+
+def moe_max_rows(cfg: MoeConfig) -> int:
+    n = lib.moe_max_rows(C.byref(cfg))
+    if n < 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, lib.moe_last_error().decode())
+    return n
+
+
+def moe_workspace_init(ws, ws_bytes, stream=0):
+    _check(lib.moe_workspace_init(_ptr(ws), ws_bytes, stream))
+
+
+def moe_check_status(ws, stream=0):
+    _check(lib.moe_check_status(_ptr(ws), stream))
+
+
+def moe_route(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, aux_loss, ws, ws_bytes, stream=0):
+    _check(lib.moe_route(C.byref(cfg), _ptr(x), _ptr(wg), _ptr(router_bias), _ptr(topk_idx), _ptr(topk_w),
+                         _ptr(n_sel), _ptr(counts), _ptr(aux_loss), _ptr(ws), ws_bytes, stream))
+
+
+def moe_dispatch(cfg, x, topk_idx, topk_w, n_sel, offsets, pos, row_token, row_gate, x_perm, ws, ws_bytes,
+                 stream=0):
+    _check(lib.moe_dispatch(C.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(topk_w), _ptr(n_sel), _ptr(offsets),
+                            _ptr(pos), _ptr(row_token), _ptr(row_gate), _ptr(x_perm), _ptr(ws), ws_bytes, stream))
+
+
+def moe_expert_gemm1(cfg, offsets, x_perm, x, w1, b1, w1s, b1s, h_perm, h_sh, ws, ws_bytes, stream=0):
+    _check(lib.moe_expert_gemm1(C.byref(cfg), _ptr(offsets), _ptr(x_perm), _ptr(x), _ptr(w1), _ptr(b1),
+                                _ptr(w1s), _ptr(b1s), _ptr(h_perm), _ptr(h_sh), _ptr(ws), ws_bytes, stream))
+
+
+def moe_expert_gemm2(cfg, offsets, h_perm, h_sh, w2, b2, w2s, b2s, row_gate, y_perm, y_sh, ws, ws_bytes,
+                     stream=0):
+    _check(lib.moe_expert_gemm2(C.byref(cfg), _ptr(offsets), _ptr(h_perm), _ptr(h_sh), _ptr(w2), _ptr(b2),
+                                _ptr(w2s), _ptr(b2s), _ptr(row_gate), _ptr(y_perm), _ptr(y_sh), _ptr(ws),
+                                ws_bytes, stream))
+
+
+def moe_expert_mlp(cfg, offsets, x_perm, x, w1, b1, w2, b2, w1s, b1s, w2s, b2s, row_gate, h_perm, h_sh, y_perm,
+                   y_sh, ws, ws_bytes, stream=0):
+    _check(lib.moe_expert_mlp(C.byref(cfg), _ptr(offsets), _ptr(x_perm), _ptr(x), _ptr(w1), _ptr(b1), _ptr(w2),
+                              _ptr(b2), _ptr(w1s), _ptr(b1s), _ptr(w2s), _ptr(b2s), _ptr(row_gate), _ptr(h_perm),
+                              _ptr(h_sh), _ptr(y_perm), _ptr(y_sh), _ptr(ws), ws_bytes, stream))
+
+
+def moe_combine(cfg, y_perm, y_sh, pos, n_sel, out, stream=0):
+    _check(lib.moe_combine(C.byref(cfg), _ptr(y_perm), _ptr(y_sh), _ptr(pos), _ptr(n_sel), _ptr(out), stream))
+
+
+def moe_last_error() -> str:
+    return lib.moe_last_error().decode()

@@ -1,0 +1,476 @@
+// C ABI of the layer: argument validation, workspace layout, TMA descriptor
+// encoding and kernel launches.  Every entry point is asynchronous on the
+// caller's stream; nothing is allocated; device data is never read on the host
+// (except in moe_check_status, which exists to do exactly that).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+int ok() {
+  g_last_error.clear();
+  return MOE_OK;
+}
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int elem_bytes(const moe_config_t* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
+
+constexpr int kMaxT = 262144;
+
+int validate(const moe_config_t* c) {
+  if (!c) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", c->T);
+  if (c->T > kMaxT) return fail(MOE_ERR_UNSUPPORTED, "T=%d above the supported %d", c->T, kMaxT);
+  if (c->D <= 0 || c->H <= 0) return fail(MOE_ERR_INVALID_ARG, "D=%d H=%d must be positive", c->D, c->H);
+  if (c->D % 64 || c->H % 64) return fail(MOE_ERR_UNSUPPORTED, "D=%d and H=%d must be multiples of 64", c->D, c->H);
+  if (c->E < 1 || c->E > 32) return fail(MOE_ERR_UNSUPPORTED, "E=%d outside 1..32", c->E);
+  if (c->K < 1 || c->K > c->E) return fail(MOE_ERR_INVALID_ARG, "K=%d outside 1..E=%d", c->K, c->E);
+  if (c->n_shared < 0 || c->n_shared > 8) return fail(MOE_ERR_UNSUPPORTED, "n_shared=%d outside 0..8", c->n_shared);
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype=%d", c->dtype);
+  if (c->routing != MOE_ROUTE_TOPK && c->routing != MOE_ROUTE_RACE) return fail(MOE_ERR_INVALID_ARG, "routing=%d", c->routing);
+  if (c->act != 0 && c->act != 1) return fail(MOE_ERR_INVALID_ARG, "act=%d", c->act);
+  if (c->gemm_impl != MOE_GEMM_AUTO && c->gemm_impl != MOE_GEMM_SIMT) return fail(MOE_ERR_INVALID_ARG, "gemm_impl=%d", c->gemm_impl);
+  if (c->reserved != 0) return fail(MOE_ERR_INVALID_ARG, "reserved field must be 0");
+  if ((size_t)c->E * c->D * 4 + 32 * 128 * 3 + 4096 > 227 * 1024)
+    return fail(MOE_ERR_UNSUPPORTED, "E*D=%d too large for the router's shared-memory gate", c->E * c->D);
+  return MOE_OK;
+}
+
+int kmax_of(const moe_config_t* c) { return c->routing == MOE_ROUTE_RACE ? c->E : c->K; }
+
+long long max_rows(const moe_config_t* c) {
+  const long long S = (long long)c->K * c->T;
+  return (long long)round_up((size_t)(S + 127ll * c->E), 128);
+}
+
+// dispatch chunking: at most 1024 chunks of >= 64 tokens (a multiple of 32)
+void chunking(int T, int* chunk, int* nchunks) {
+  int ch = (T + 1023) / 1024;
+  ch = (ch + 31) / 32 * 32;
+  if (ch < 64) ch = 64;
+  *chunk = ch;
+  *nchunks = (T + ch - 1) / ch;
+}
+
+struct WsLayout {
+  size_t status, tile_counts, tile_psum, P, hist, state, tile_eq, race_counts, chunk_base, total;
+};
+
+WsLayout ws_layout(const moe_config_t* c) {
+  WsLayout L{};
+  const size_t T = (size_t)c->T, E = (size_t)c->E;
+  const size_t max_route_tiles = (T + 31) / 32 + 1;
+  const size_t race_tiles = (T + 127) / 128 + 1;
+  int ch, nch;
+  chunking(c->T, &ch, &nch);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += round_up(bytes ? bytes : 1, 256); return o; };
+  L.status = take(256);
+  L.tile_counts = take(max_route_tiles * E * 4);
+  L.tile_psum = take(max_route_tiles * E * 4);
+  const bool race = c->routing == MOE_ROUTE_RACE;
+  L.P = take(race ? T * E * 4 : 0);
+  L.hist = take(race ? 4096 * 4 : 0);
+  L.state = take(race ? 16 : 0);
+  L.tile_eq = take(race ? race_tiles * 4 : 0);
+  L.race_counts = take(race ? race_tiles * E * 4 : 0);
+  L.chunk_base = take((size_t)(nch + 1) * E * 4);
+  L.total = off;
+  return L;
+}
+
+int check_ws(const moe_config_t* c, void* ws, size_t ws_bytes) {
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "ws is NULL");
+  if ((uintptr_t)ws & 255u) return fail(MOE_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+  const size_t need = ws_layout(c).total;
+  if (ws_bytes < need) return fail(MOE_ERR_WORKSPACE, "ws_bytes=%zu < %zu", ws_bytes, need);
+  return MOE_OK;
+}
+
+#define REQUIRE_PTR(p)                                                              \
+  do {                                                                              \
+    if (!(p)) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", #p);                   \
+    if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+  } while (0)
+#define OPTIONAL_PTR(p)                                                             \
+  do {                                                                              \
+    if ((p) && !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+int* status_ptr(void* ws) { return reinterpret_cast<int*>(ws); }
+template <typename T> T* ws_at(void* ws, size_t off) { return reinterpret_cast<T*>((uint8_t*)ws + off); }
+
+// ---------------------------------------------------------------- device info
+int num_sms_current() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major [rows, cols] tensor, 128-byte swizzled boxes of box_rows x (128 B)
+int make_tmap(CUtensorMap* m, const void* base, bool bf16, long long rows, long long cols, int box_rows,
+              const char* what) {
+  auto fn = encode_fn();
+  if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const int eb = bf16 ? 2 : 4;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * eb};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (CUresult %d)", what, (int)r);
+  return MOE_OK;
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+extern "C" {
+
+int32_t moe_version(void) { return 100; }
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+size_t moe_workspace_size(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return ws_layout(cfg).total;
+}
+
+int64_t moe_max_rows(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return -1;
+  return max_rows(cfg);
+}
+
+int moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < 256) return fail(MOE_ERR_INVALID_ARG, "ws is NULL or smaller than 256 bytes");
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_workspace_init");
+  return ok();
+}
+
+int moe_check_status(void* ws, void* stream) {
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "ws is NULL");
+  int h[2] = {0, 0};
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(h, ws, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "moe_check_status");
+  if (h[0] != 0) {
+    e = cudaMemsetAsync(ws, 0, 256, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (h[0] == 2 /* timeout */) return fail(MOE_ERR_TIMEOUT, "a kernel's bounded wait ran out (site %d)", h[1]);
+    return fail(MOE_ERR_DEVICE_CHECK, "a kernel found a bad index (site %d)", h[1]);
+  }
+  return ok();
+}
+
+int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
+              int32_t* topk_idx, float* topk_w, int32_t* n_sel, int32_t* counts, float* aux_loss,
+              void* ws, size_t ws_bytes, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  const bool race = cfg->routing == MOE_ROUTE_RACE;
+  REQUIRE_PTR(counts);
+  if (!aux_loss) return fail(MOE_ERR_INVALID_ARG, "aux_loss is NULL");
+  if ((rc = check_ws(cfg, ws, ws_bytes))) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  if (cfg->T == 0) {
+    if ((e = cudaMemsetAsync(counts, 0, cfg->E * sizeof(int32_t), s)) != cudaSuccess) return cuda_fail(e, "moe_route");
+    if ((e = cudaMemsetAsync(aux_loss, 0, sizeof(float), s)) != cudaSuccess) return cuda_fail(e, "moe_route");
+    return ok();
+  }
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(wg);
+  REQUIRE_PTR(topk_idx);
+  REQUIRE_PTR(topk_w);
+  OPTIONAL_PTR(router_bias);
+  OPTIONAL_PTR(n_sel);
+  if (race && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
+  const WsLayout L = ws_layout(cfg);
+  const int sms = num_sms_current();
+  // tile of tokens per CTA: spread T over the SMs, 32..256 rows, shared memory permitting
+  int tile = (int)round_up((size_t)((cfg->T + sms - 1) / sms), 32);
+  if (tile < 32) tile = 32;
+  if (tile > 256) tile = 256;
+  while (tile > 32 && route_smem_bytes(cfg->D, cfg->E, tile, cfg->dtype) > 227 * 1024) tile -= 32;
+  const int ntiles = (cfg->T + tile - 1) / tile;
+  CUtensorMap tm;
+  if ((rc = make_tmap(&tm, x, cfg->dtype == MOE_BF16, cfg->T, cfg->D, tile, "x"))) return rc;
+  RouteArgs ra{};
+  ra.x = x; ra.wg = wg; ra.bias = router_bias;
+  ra.T = cfg->T; ra.D = cfg->D; ra.E = cfg->E; ra.K = cfg->K; ra.bf16 = cfg->dtype == MOE_BF16;
+  ra.tile_rows = tile; ra.ntiles = ntiles; ra.grid = ntiles < sms ? ntiles : sms;
+  ra.topk_idx = topk_idx; ra.topk_w = topk_w; ra.n_sel = race ? nullptr : n_sel;
+  ra.P = race ? ws_at<float>(ws, L.P) : nullptr;
+  ra.tile_counts = ws_at<int32_t>(ws, L.tile_counts);
+  ra.tile_psum = ws_at<float>(ws, L.tile_psum);
+  ra.status = status_ptr(ws);
+  if ((e = launch_route(ra, &tm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
+  FinalizeArgs fa{};
+  fa.T = cfg->T; fa.E = cfg->E; fa.K = cfg->K; fa.alpha = cfg->alpha;
+  fa.counts = counts; fa.aux_loss = aux_loss;
+  fa.tile_psum = ra.tile_psum; fa.ntiles_psum = ntiles;
+  if (race) {
+    RaceArgs rr{};
+    rr.P = ra.P; rr.T = cfg->T; rr.E = cfg->E; rr.K = cfg->K;
+    rr.hist = ws_at<uint32_t>(ws, L.hist);
+    rr.state = ws_at<uint32_t>(ws, L.state);
+    rr.tile_eq = ws_at<uint32_t>(ws, L.tile_eq);
+    rr.ntiles = (cfg->T + 127) / 128;
+    rr.topk_idx = topk_idx; rr.topk_w = topk_w; rr.n_sel = n_sel;
+    rr.tile_counts = ws_at<int32_t>(ws, L.race_counts);
+    rr.status = status_ptr(ws);
+    if ((e = cudaMemsetAsync(rr.hist, 0, 4096 * 4, s)) != cudaSuccess) return cuda_fail(e, "moe_route");
+    if ((e = launch_race_select(rr, s)) != cudaSuccess) return cuda_fail(e, "race select kernels");
+    fa.tile_counts = rr.tile_counts; fa.ntiles_counts = rr.ntiles;
+  } else {
+    fa.tile_counts = ra.tile_counts; fa.ntiles_counts = ntiles;
+  }
+  if ((e = launch_route_finalize(fa, s)) != cudaSuccess) return cuda_fail(e, "route finalize kernel");
+  return ok();
+}
+
+int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const float* topk_w,
+                 const int32_t* n_sel, int32_t* offsets, int32_t* pos, int32_t* row_token,
+                 float* row_gate, void* x_perm, void* ws, size_t ws_bytes, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  const bool race = cfg->routing == MOE_ROUTE_RACE;
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(row_token);
+  REQUIRE_PTR(row_gate);
+  if ((rc = check_ws(cfg, ws, ws_bytes))) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  const long long R = max_rows(cfg);
+  if (cfg->T == 0) {
+    if ((e = cudaMemsetAsync(offsets, 0, (cfg->E + 1) * sizeof(int32_t), s)) != cudaSuccess) return cuda_fail(e, "moe_dispatch");
+    if ((e = cudaMemsetAsync(row_token, 0xFF, R * sizeof(int32_t), s)) != cudaSuccess) return cuda_fail(e, "moe_dispatch");
+    if ((e = cudaMemsetAsync(row_gate, 0, R * sizeof(float), s)) != cudaSuccess) return cuda_fail(e, "moe_dispatch");
+    return ok();
+  }
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(topk_idx);
+  REQUIRE_PTR(topk_w);
+  REQUIRE_PTR(pos);
+  REQUIRE_PTR(x_perm);
+  OPTIONAL_PTR(n_sel);
+  if (race && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
+  const WsLayout L = ws_layout(cfg);
+  DispatchArgs da{};
+  da.x = x; da.bf16 = cfg->dtype == MOE_BF16;
+  da.topk_idx = topk_idx; da.topk_w = topk_w; da.n_sel = n_sel;
+  da.T = cfg->T; da.D = cfg->D; da.E = cfg->E; da.K = cfg->K; da.Kmax = kmax_of(cfg);
+  chunking(cfg->T, &da.chunk, &da.nchunks);
+  da.r_max = R;
+  da.chunk_base = ws_at<int32_t>(ws, L.chunk_base);
+  da.offsets = offsets; da.pos = pos; da.row_token = row_token; da.row_gate = row_gate;
+  da.x_perm = x_perm;
+  da.status = status_ptr(ws);
+  if ((e = launch_dispatch(da, s)) != cudaSuccess) return cuda_fail(e, "dispatch kernels");
+  return ok();
+}
+
+namespace {
+
+// A0/B0: routed problem (A [rows0, K0], B [brows0, K0]); A1/B1: shared problem
+// (A [rows1, K1], B [brows1, bcols1]; bcols1 < K1 when B is a K-split stack)
+int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long rows0, const void* B0,
+             long long brows0, const void* A1, long long rows1, const void* B1, long long brows1, int K0,
+             int K1, int bcols1, void* ws, cudaStream_t s) {
+  (void)ws;
+  cudaError_t e;
+  const bool tc = cfg->dtype == MOE_BF16 && cfg->gemm_impl == MOE_GEMM_AUTO;
+  if (!tc) {
+    if ((e = launch_gemm_simt(g, s)) != cudaSuccess) return cuda_fail(e, "FFMA expert GEMM");
+    return ok();
+  }
+  const int bn = gemm_tc_pick_bn(g.p[0].N, g.nprob > 1 ? g.p[1].N : 0);
+  if (!bn) return fail(MOE_ERR_UNSUPPORTED, "no tile width divides N=%d", g.p[0].N);
+  CUtensorMap ta[2], tb[2];
+  int rc;
+  if ((rc = make_tmap(&ta[0], A0, true, rows0, K0, 128, "A0"))) return rc;
+  if ((rc = make_tmap(&tb[0], B0, true, brows0, K0, bn, "B0"))) return rc;
+  if (g.nprob > 1) {
+    if ((rc = make_tmap(&ta[1], A1, true, rows1, K1, 128, "A1"))) return rc;
+    if ((rc = make_tmap(&tb[1], B1, true, brows1, bcols1, bn, "B1"))) return rc;
+  } else {
+    ta[1] = ta[0];
+    tb[1] = tb[0];
+  }
+  if ((e = launch_gemm_tc(g, ta, tb, bn, num_sms_current(), s)) != cudaSuccess) return cuda_fail(e, "tcgen05 expert GEMM");
+  return ok();
+}
+
+}  // namespace
+
+int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
+                     const void* x, const void* w1, const void* b1, const void* w1s, const void* b1s,
+                     void* h_perm, void* h_sh, void* ws, size_t ws_bytes, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if ((rc = check_ws(cfg, ws, ws_bytes))) return rc;
+  if (cfg->T == 0) return ok();
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(x_perm);
+  REQUIRE_PTR(w1);
+  REQUIRE_PTR(h_perm);
+  OPTIONAL_PTR(b1);
+  const int ns = cfg->n_shared;
+  if (ns > 0) {
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(w1s);
+    REQUIRE_PTR(h_sh);
+    OPTIONAL_PTR(b1s);
+  }
+  const long long R = max_rows(cfg);
+  GemmArgs g{};
+  g.offsets = offsets; g.E = cfg->E; g.r_max = R; g.act = cfg->act; g.status = status_ptr(ws);
+  g.bf16 = cfg->dtype == MOE_BF16;
+  g.nprob = ns > 0 ? 2 : 1;
+  GemmProblem& p0 = g.p[0];
+  p0.routed = 1; p0.N = cfg->H; p0.K = cfg->D; p0.epi = 0;
+  p0.A = x_perm; p0.B = w1; p0.out = h_perm; p0.ld_out = cfg->H; p0.bias = b1; p0.bias_stride = cfg->H;
+  p0.bias_rows = 1;
+  if (ns > 0) {
+    // the n_s stacked W1 [n_s,H,D] are one [n_s*H, D] matrix; b1s [n_s,H] one [n_s*H] row
+    GemmProblem& p1 = g.p[1];
+    p1.routed = 0; p1.M = cfg->T; p1.N = ns * cfg->H; p1.K = cfg->D; p1.epi = 0;
+    p1.A = x; p1.B = w1s; p1.out = h_sh; p1.ld_out = (long long)ns * cfg->H; p1.bias = b1s; p1.bias_stride = 0;
+    p1.bias_rows = 1;
+  }
+  return run_gemm(cfg, g, x_perm, R, w1, (long long)cfg->E * cfg->H, x, cfg->T, w1s, (long long)ns * cfg->H,
+                  cfg->D, cfg->D, cfg->D, ws, (cudaStream_t)stream);
+}
+
+int moe_expert_gemm2(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm,
+                     const void* h_sh, const void* w2, const void* b2, const void* w2s,
+                     const void* b2s, const float* row_gate, float* y_perm, float* y_sh,
+                     void* ws, size_t ws_bytes, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if ((rc = check_ws(cfg, ws, ws_bytes))) return rc;
+  if (cfg->T == 0) return ok();
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(h_perm);
+  REQUIRE_PTR(w2);
+  REQUIRE_PTR(row_gate);
+  REQUIRE_PTR(y_perm);
+  OPTIONAL_PTR(b2);
+  const int ns = cfg->n_shared;
+  if (ns > 0) {
+    REQUIRE_PTR(h_sh);
+    REQUIRE_PTR(w2s);
+    REQUIRE_PTR(y_sh);
+    OPTIONAL_PTR(b2s);
+  }
+  const long long R = max_rows(cfg);
+  GemmArgs g{};
+  g.offsets = offsets; g.E = cfg->E; g.r_max = R; g.act = cfg->act; g.status = status_ptr(ws);
+  g.bf16 = cfg->dtype == MOE_BF16;
+  g.nprob = ns > 0 ? 2 : 1;
+  GemmProblem& p0 = g.p[0];
+  p0.routed = 1; p0.N = cfg->D; p0.K = cfg->H; p0.epi = 1;
+  p0.A = h_perm; p0.B = w2; p0.out = y_perm; p0.ld_out = cfg->D; p0.bias = b2; p0.bias_stride = cfg->D;
+  p0.bias_rows = 1;
+  p0.gate = row_gate;
+  if (ns > 0) {
+    // sum_j W2_j h_j over the n_s stacked W2 [n_s,D,H]: K = n_s*H walks the stack
+    // (ksplit = H); the n_s rows of b2s [n_s,D] are summed in the epilogue
+    GemmProblem& p1 = g.p[1];
+    p1.routed = 0; p1.M = cfg->T; p1.N = cfg->D; p1.K = ns * cfg->H; p1.epi = 1;
+    p1.A = h_sh; p1.B = w2s; p1.out = y_sh; p1.ld_out = cfg->D; p1.bias = b2s; p1.bias_stride = 0;
+    p1.bias_rows = ns; p1.ksplit = cfg->H;
+    p1.gate = nullptr;
+  }
+  return run_gemm(cfg, g, h_perm, R, w2, (long long)cfg->E * cfg->D, h_sh, cfg->T, w2s,
+                  (long long)ns * cfg->D, cfg->H, ns * cfg->H, cfg->H, ws, (cudaStream_t)stream);
+}
+
+int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
+                   const void* x, const void* w1, const void* b1, const void* w2, const void* b2,
+                   const void* w1s, const void* b1s, const void* w2s, const void* b2s,
+                   const float* row_gate, void* h_perm, void* h_sh, float* y_perm, float* y_sh,
+                   void* ws, size_t ws_bytes, void* stream) {
+  int rc = moe_expert_gemm1(cfg, offsets, x_perm, x, w1, b1, w1s, b1s, h_perm, h_sh, ws, ws_bytes, stream);
+  if (rc) return rc;
+  return moe_expert_gemm2(cfg, offsets, h_perm, h_sh, w2, b2, w2s, b2s, row_gate, y_perm, y_sh, ws, ws_bytes,
+                          stream);
+}
+
+int moe_combine(const moe_config_t* cfg, const float* y_perm, const float* y_sh,
+                const int32_t* pos, const int32_t* n_sel, void* out, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (cfg->T == 0) return ok();
+  REQUIRE_PTR(y_perm);
+  REQUIRE_PTR(pos);
+  REQUIRE_PTR(out);
+  OPTIONAL_PTR(n_sel);
+  if (cfg->n_shared > 0) REQUIRE_PTR(y_sh);
+  if (cfg->routing == MOE_ROUTE_RACE && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
+  CombineArgs ca{};
+  ca.y_perm = y_perm; ca.y_sh = cfg->n_shared > 0 ? y_sh : nullptr; ca.pos = pos; ca.n_sel = n_sel;
+  ca.out = out; ca.bf16 = cfg->dtype == MOE_BF16;
+  ca.T = cfg->T; ca.D = cfg->D; ca.K = cfg->K; ca.Kmax = kmax_of(cfg); ca.r_max = max_rows(cfg);
+  cudaError_t e = launch_combine(ca, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "combine kernel");
+  return ok();
+}
+
+}  // extern "C"

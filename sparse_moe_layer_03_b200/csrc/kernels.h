@@ -1,0 +1,101 @@
+// Internal launchers shared between the kernel files and the C-ABI layer.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---- route.cu
+struct RouteArgs {
+  const void* x;            // [T,D] act
+  const void* wg;           // [E,D] act
+  const float* bias;        // [E] or null
+  int T, D, E, K, bf16;
+  int tile_rows, ntiles, grid;
+  int32_t* topk_idx;        // top-K mode: [T,K]
+  float* topk_w;
+  int32_t* n_sel;           // may be null (top-K)
+  float* P;                 // race: [T,E] scores (scratch), else null
+  int32_t* tile_counts;     // [ntiles,E] (top-K)
+  float* tile_psum;         // [ntiles,E]
+  int* status;
+};
+cudaError_t launch_route(const RouteArgs& a, const CUtensorMap* tmap_x, cudaStream_t s);
+size_t route_smem_bytes(int D, int E, int tile_rows, int bf16);
+
+struct FinalizeArgs {
+  const int32_t* tile_counts; int ntiles_counts;
+  const float* tile_psum; int ntiles_psum;
+  int T, E, K; float alpha;
+  int32_t* counts; float* aux_loss;
+};
+cudaError_t launch_route_finalize(const FinalizeArgs& a, cudaStream_t s);
+
+struct RaceArgs {
+  const float* P;           // [T,E]
+  int T, E, K;
+  uint32_t* hist;           // [4096] scratch, zeroed by the caller before pass 0
+  uint32_t* state;          // [4] scratch: prefix, need, threshold bits, need_eq
+  uint32_t* tile_eq;        // [ntiles]
+  int ntiles;               // ceil(T/128)
+  int32_t* topk_idx;        // [T,E]
+  float* topk_w;            // [T,E]
+  int32_t* n_sel;           // [T]
+  int32_t* tile_counts;     // [ntiles,E]
+  int* status;
+};
+cudaError_t launch_race_select(const RaceArgs& a, cudaStream_t s);
+
+// ---- dispatch.cu
+struct DispatchArgs {
+  const void* x; int bf16;
+  const int32_t* topk_idx; const float* topk_w; const int32_t* n_sel;
+  int T, D, E, K, Kmax;
+  int chunk, nchunks;
+  long long r_max;
+  int32_t* chunk_base;      // [nchunks,E] scratch
+  int32_t* offsets;         // [E+1]
+  int32_t* pos; int32_t* row_token; float* row_gate;
+  void* x_perm;
+  int* status;
+};
+cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
+
+// ---- gemm (tcgen05 and FFMA)
+struct GemmProblem {
+  int routed;               // 1: rows grouped by expert segments (offsets), 0: dense rows
+  int M;                    // dense: rows; routed: unused (from offsets)
+  int N, K;                 // per-expert output width and reduction length
+  int epi;                  // 0: bias + GELU -> act store; 1: (bias) * gate -> fp32 store
+  const void* A;            // [rows,K] act (FFMA path; the TMA path uses tensor maps)
+  const void* B;            // [E*N or N, K] act
+  void* out; long long ld_out;
+  const void* bias; long long bias_stride;   // per-expert stride in elements, null = none
+  int bias_rows;            // bias rows summed per column (n_s for the shared GEMM2, else 1)
+  int ksplit;               // 0, or: B is [K/ksplit blocks][N][ksplit] (shared W2 stack)
+  const float* gate;        // per-row gate or null
+};
+struct GemmArgs {
+  GemmProblem p[2]; int nprob;
+  const int32_t* offsets; int E;
+  long long r_max;
+  int act;
+  int* status;
+  int bf16;
+};
+cudaError_t launch_gemm_tc(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, int bn,
+                           int num_sms, cudaStream_t s);
+int gemm_tc_pick_bn(int n0, int n1);
+cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t s);
+
+// ---- combine.cu
+struct CombineArgs {
+  const float* y_perm; const float* y_sh; const int32_t* pos; const int32_t* n_sel;
+  void* out; int bf16;
+  int T, D, K, Kmax;
+  long long r_max;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+}  // namespace moe

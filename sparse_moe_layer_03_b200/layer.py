@@ -1,0 +1,128 @@
+"""DiT-MoE sparse expert layer on one GPU: buffers plus the four C-ABI calls.
+
+``MoELayer`` owns the device buffers of one configuration (allocated once with
+torch, which is only the allocator and the stream provider here) and runs
+
+    moe_route -> moe_dispatch -> moe_expert_gemm1 -> moe_expert_gemm2 -> moe_combine
+
+on the current CUDA stream.  Nothing in this file computes any part of the
+layer: it moves arguments to the library.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+
+def _dev(a, dtype, device):
+    if a is None:
+        return None
+    t = torch.as_tensor(np.ascontiguousarray(a)) if isinstance(a, np.ndarray) else a
+    return t.to(device=device, dtype=dtype).contiguous()
+
+
+@dataclass
+class LayerShape:
+    T: int
+    D: int
+    H: int
+    E: int
+    K: int
+    n_shared: int
+    dtype: str = "bf16"
+    routing: str = "topk"
+    alpha: float = 0.01
+    act: str = "tanh"
+    gemm_impl: str = "auto"
+
+
+class MoELayer:
+    """Weights and buffers of one layer configuration on one CUDA device."""
+
+    def __init__(self, shape: LayerShape, params: dict, device="cuda:0"):
+        self.s = shape
+        self.device = torch.device(device)
+        self.cfg = B.make_config(shape.T, shape.D, shape.H, shape.E, shape.K, shape.n_shared, shape.dtype,
+                                 shape.routing, shape.alpha, shape.act, shape.gemm_impl)
+        self.act_dtype = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+        dt, dev = self.act_dtype, self.device
+        self.wg = _dev(params["wg"], dt, dev)
+        self.router_bias = _dev(params.get("router_bias"), torch.float32, dev)
+        self.w1 = _dev(params["w1"], dt, dev)
+        self.b1 = _dev(params.get("b1"), dt, dev)
+        self.w2 = _dev(params["w2"], dt, dev)
+        self.b2 = _dev(params.get("b2"), dt, dev)
+        ns = shape.n_shared
+        self.ws1 = _dev(params["ws1"], dt, dev) if ns else None
+        self.bs1 = _dev(params.get("bs1"), dt, dev) if ns else None
+        self.ws2 = _dev(params["ws2"], dt, dev) if ns else None
+        self.bs2 = _dev(params.get("bs2"), dt, dev) if ns else None
+        self._alloc(shape.T)
+
+    def _alloc(self, T: int):
+        s, dev, dt = self.s, self.device, self.act_dtype
+        self.cfg.T = T
+        kmax = s.E if s.routing == "race" else s.K
+        self.kmax = kmax
+        self.R = B.moe_max_rows(self.cfg)
+        self.ws_bytes = B.moe_workspace_size(self.cfg)
+        i32, f32 = torch.int32, torch.float32
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.topk_idx = torch.empty((T, kmax), dtype=i32, device=dev)
+        self.topk_w = torch.empty((T, kmax), dtype=f32, device=dev)
+        self.n_sel = torch.empty((T,), dtype=i32, device=dev)
+        self.counts = torch.empty((s.E,), dtype=i32, device=dev)
+        self.aux = torch.empty((1,), dtype=f32, device=dev)
+        self.offsets = torch.empty((s.E + 1,), dtype=i32, device=dev)
+        self.pos = torch.empty((T, kmax), dtype=i32, device=dev)
+        self.row_token = torch.empty((self.R,), dtype=i32, device=dev)
+        self.row_gate = torch.empty((self.R,), dtype=f32, device=dev)
+        self.x_perm = torch.empty((self.R, s.D), dtype=dt, device=dev)
+        self.h_perm = torch.empty((self.R, s.H), dtype=dt, device=dev)
+        self.y_perm = torch.empty((self.R, s.D), dtype=f32, device=dev)
+        ns = s.n_shared
+        self.h_sh = torch.empty((T, ns * s.H), dtype=dt, device=dev) if ns else None
+        self.y_sh = torch.empty((T, s.D), dtype=f32, device=dev) if ns else None
+        self.out = torch.empty((T, s.D), dtype=dt, device=dev)
+        B.moe_workspace_init(self.ws, self.ws_bytes, self.stream())
+
+    def stream(self) -> int:
+        return torch.cuda.current_stream(self.device).cuda_stream
+
+    # ------------------------------------------------------------ the four calls
+    def route(self, x: torch.Tensor):
+        B.moe_route(self.cfg, x, self.wg, self.router_bias, self.topk_idx, self.topk_w, self.n_sel, self.counts,
+                    self.aux, self.ws, self.ws_bytes, self.stream())
+
+    def dispatch(self, x: torch.Tensor):
+        B.moe_dispatch(self.cfg, x, self.topk_idx, self.topk_w, self.n_sel, self.offsets, self.pos,
+                       self.row_token, self.row_gate, self.x_perm, self.ws, self.ws_bytes, self.stream())
+
+    def gemm1(self, x: torch.Tensor):
+        B.moe_expert_gemm1(self.cfg, self.offsets, self.x_perm, x, self.w1, self.b1, self.ws1, self.bs1,
+                           self.h_perm, self.h_sh, self.ws, self.ws_bytes, self.stream())
+
+    def gemm2(self):
+        B.moe_expert_gemm2(self.cfg, self.offsets, self.h_perm, self.h_sh, self.w2, self.b2, self.ws2, self.bs2,
+                           self.row_gate, self.y_perm, self.y_sh, self.ws, self.ws_bytes, self.stream())
+
+    def combine(self):
+        B.moe_combine(self.cfg, self.y_perm, self.y_sh, self.pos, self.n_sel, self.out, self.stream())
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        """Whole layer on device-resident x [T,D]; returns the output buffer."""
+        assert x.shape == (self.cfg.T, self.s.D) and x.dtype == self.act_dtype and x.is_contiguous()
+        self.route(x)
+        self.dispatch(x)
+        self.gemm1(x)
+        self.gemm2()
+        self.combine()
+        return self.out
+
+    def check(self):
+        B.moe_check_status(self.ws, self.stream())

@@ -1,0 +1,63 @@
+"""The C-ABI library loads and exports every function include/moe.h declares.
+
+Runs without a GPU: only host-side entry points that touch no device memory
+are called (version, workspace sizing, row capacity, argument validation).
+"""
+import ctypes
+
+import pytest
+
+from sparse_moe_layer_03_b200 import binding as B
+
+
+def test_library_exports_every_declared_symbol():
+    names = B.header_symbols()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(B.lib, n), n
+    # and the binding wraps each of them under the same name
+    for n in names:
+        assert hasattr(B, n), n
+
+
+def test_version_and_sizes():
+    assert B.moe_version() == 100
+    cfg = B.make_config(32768, 1152, 4608, 8, 2, 2)
+    assert B.moe_max_rows(cfg) == 66560
+    assert B.moe_workspace_size(cfg) > 0
+    race = B.make_config(32768, 1152, 4608, 16, 2, 1, routing="race")
+    assert B.moe_workspace_size(race) > 32768 * 16 * 4
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("K", 9, B.MOE_ERR_INVALID_ARG), ("E", 33, B.MOE_ERR_UNSUPPORTED), ("D", 100, B.MOE_ERR_UNSUPPORTED),
+    ("T", -1, B.MOE_ERR_INVALID_ARG), ("n_shared", 9, B.MOE_ERR_UNSUPPORTED), ("dtype", 7, B.MOE_ERR_INVALID_ARG),
+    ("routing", 3, B.MOE_ERR_INVALID_ARG), ("reserved", 1, B.MOE_ERR_INVALID_ARG),
+])
+def test_invalid_config_is_rejected_on_host(field, value, code):
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    setattr(cfg, field, value)
+    assert B.lib.moe_workspace_size(ctypes.byref(cfg)) == 0
+    rc = B.lib.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None, 0, None)
+    assert rc == code
+    assert B.lib.moe_last_error()
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch():
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    n = B.moe_workspace_size(cfg)
+    fake = 1 << 40                          # never dereferenced: validation fails first
+    rc = B.lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, None, fake, n, None)
+    assert rc == B.MOE_ERR_INVALID_ARG and b"aux_loss" in B.lib.moe_last_error()
+    rc = B.lib.moe_route(ctypes.byref(cfg), fake + 8, fake, None, fake, fake, None, fake, fake, fake, n, None)
+    assert rc == B.MOE_ERR_INVALID_ARG and b"aligned" in B.lib.moe_last_error()
+    rc = B.lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, fake, fake, n - 256, None)
+    assert rc == B.MOE_ERR_WORKSPACE
+    rc = B.lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, fake, fake + 16, n, None)
+    assert rc == B.MOE_ERR_INVALID_ARG      # ws not 256-byte aligned
+    race = B.make_config(1024, 384, 1536, 8, 2, 2, routing="race")
+    n = B.moe_workspace_size(race)
+    rc = B.lib.moe_route(ctypes.byref(race), fake, fake, None, fake, fake, None, fake, fake, fake, n, None)
+    assert rc == B.MOE_ERR_INVALID_ARG and b"n_sel" in B.lib.moe_last_error()
+    rc = B.lib.moe_combine(ctypes.byref(race), fake, fake, fake, None, fake, None)
+    assert rc == B.MOE_ERR_INVALID_ARG

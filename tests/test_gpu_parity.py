@@ -1,0 +1,143 @@
+"""GPU parity: the CUDA layer, called through the C ABI, against the fp64 oracle.
+
+Small shapes (oracle in seconds) span several 128-row tiles and a ragged tail;
+the five named workloads run at full size in the launch configuration the
+benchmark times, with routing and permutation checked on every token and the
+output on sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+from sparse_moe_layer_03_b200 import inputs as I
+from tests import parity as PA
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(T, D, H, E, K, ns, dtype="bf16", routing="topk", seed=100, bias="none", bias_std=0.2):
+    w = I.small_workload(T, D, H, E, K, ns, dtype, routing, seed, bias)
+    return w, I.make_inputs(w, bias_std=bias_std)
+
+
+SMALL = [
+    # T, D, H, E, K, ns, dtype, routing
+    (1000, 256, 512, 8, 2, 2, "bf16", "topk"),
+    (1000, 256, 512, 8, 2, 2, "f32", "topk"),
+    (777, 384, 1536, 16, 2, 2, "bf16", "topk"),
+    (999, 128, 256, 4, 1, 0, "bf16", "topk"),
+    (1300, 192, 384, 8, 3, 1, "f32", "topk"),
+    (1000, 256, 512, 8, 2, 2, "bf16", "race"),
+    (513, 128, 256, 16, 2, 1, "f32", "race"),
+    (640, 64, 128, 32, 4, 2, "bf16", "topk"),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "T%d_D%d_H%d_E%d_K%d_ns%d_%s_%s" % c)
+def test_small_layer_parity(case):
+    w, inp = _small(*case)
+    rep = PA.full_check(w, inp)
+    assert rep["err"] <= PA.out_tol(w)
+
+
+def test_tensor_core_path_matches_ffma_path():
+    w, inp = _small(1000, 256, 512, 8, 2, 2, "bf16")
+    a = PA.full_check(w, inp, gemm_impl="auto")
+    b = PA.full_check(w, inp, gemm_impl="simt")
+    # both against the oracle already; against each other: same rounding points
+    assert PA.rel_err(a["res"]["out"], b["res"]["out"]) < 1e-2
+
+
+def test_erf_gelu_option():
+    w, inp = _small(300, 128, 256, 4, 2, 1, "f32")
+    rep = PA.full_check(w, inp, act="erf")
+    assert rep["err"] <= 1e-5
+
+
+def test_deterministic_repeat():
+    w, inp = _small(2000, 256, 512, 8, 2, 2, "bf16", routing="race")
+    L, x = PA.run_layer(w, inp)
+    valid = L.row_token >= 0          # padding rows of x_perm are never written
+    pick = lambda: (L.out, L.topk_idx, L.topk_w, L.pos, L.aux, L.counts, L.x_perm[valid], L.y_perm[valid])
+    first = [t.clone() for t in pick()]
+    for _ in range(2):
+        L.forward(x)
+        torch.cuda.synchronize()
+        for a, b in zip(first, pick()):
+            assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------ edge cases
+
+def test_empty_batch():
+    w, inp = _small(0, 128, 256, 8, 2, 1)
+    L, x = PA.run_layer(w, inp)
+    assert torch.all(L.counts == 0) and float(L.aux[0]) == 0.0
+    assert torch.all(L.offsets == 0) and torch.all(L.row_token == -1)
+
+
+def test_single_token_and_race_single_token():
+    for routing in ("topk", "race"):
+        w, inp = _small(1, 128, 256, 8, 2, 1, routing=routing)
+        PA.full_check(w, inp)
+
+
+def test_dense_mlp_special_case():
+    # E = 1, K = 1, n_s = 0: every token takes the one expert with g = 1
+    w, inp = _small(333, 128, 256, 1, 1, 0, "f32")
+    rep = PA.full_check(w, inp)
+    assert np.all(rep["res"]["topk_w"] == 1.0)
+
+
+def test_all_experts_selected():
+    w, inp = _small(500, 128, 256, 4, 4, 1, "bf16")
+    PA.full_check(w, inp)
+    w, inp = _small(300, 128, 256, 4, 4, 1, "bf16", routing="race")
+    rep = PA.full_check(w, inp)
+    assert np.all(rep["res"]["n_sel"] == 4)
+
+
+def test_skewed_experts_one_full_one_empty():
+    w, inp = _small(700, 128, 256, 8, 2, 1, "bf16")
+    inp = dict(inp)
+    b = np.zeros(8, np.float32)
+    b[3] = 40.0        # every token takes expert 3 first
+    b[5] = -40.0       # nobody ever takes expert 5
+    inp["router_bias"] = b
+    rep = PA.full_check(w, inp)
+    c = rep["res"]["counts"]
+    assert c[3] == 700 and c[5] == 0
+
+
+def test_uniform_router_gives_alpha():
+    # Wg = 0, no bias: all scores 1/E, ties broken by expert id, L = alpha exactly
+    w, inp = _small(512, 128, 256, 8, 2, 1, "bf16")
+    inp = dict(inp)
+    inp["wg"] = np.zeros_like(inp["wg"])
+    rep = PA.full_check(w, inp)
+    assert abs(float(rep["res"]["aux"][0]) - w.alpha) < 1e-7
+    assert np.all(rep["res"]["topk_idx"] == np.array([0, 1]))
+
+
+def test_planted_bad_index_reported_not_faulted():
+    from sparse_moe_layer_03_b200 import binding as B
+    w, inp = _small(256, 128, 256, 8, 2, 1, "bf16")
+    L, x = PA.run_layer(w, inp)
+    L.topk_idx[7, 1] = 8 + 3                    # out-of-range expert planted on the host side
+    L.dispatch(x)
+    with pytest.raises(B.MoeError) as ei:
+        L.check()
+    assert ei.value.code == B.MOE_ERR_DEVICE_CHECK
+    L.check()                                  # status cleared
+    assert int(L.pos[7, 1]) == -1
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+@pytest.mark.parametrize("key", I.WORKLOAD_ORDER)
+def test_named_workload_full_size(key):
+    w = I.WORKLOADS[key]
+    inp = I.make_inputs(w)
+    tokens = PA.sample_tokens(w.T, 256 if w.T > 4096 else w.T)
+    rep = PA.full_check(w, inp, tokens=tokens)
+    assert rep["err"] <= PA.out_tol(w)

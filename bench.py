@@ -1,0 +1,377 @@
+"""Benchmark of the DiT-MoE sparse expert layer forward on B200 (one process per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole layer (router, dispatch, expert GEMM1 with
+GELU, expert GEMM2 with gates, combine) over one batch of the workload, inputs
+resident in HBM.  Each step is timed on the device with CUDA events on the
+launching stream; L2 is flushed between steps by a 256 MB write outside the
+step's events.  With N > 1 (torchrun) every rank runs its own batch (weak
+scaling; the batches are independent, so there is no data-path collective),
+the timed region is bracketed by a barrier and a synchronize, and the max over
+ranks is reported.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+the method here) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from sparse_moe_layer_03_b200 import inputs as I  # noqa: E402
+from sparse_moe_layer_03_b200 import metrics as M  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec and TFLOP/s on 1 B200; % of bf16 peak and % HBM BW"
+DEFAULT_WORKLOAD = "xl2_8e2a_512"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"]}
+
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [s for s in sm if s is not None and s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_index_for(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ------------------------------------------------------------------ oracle timing (CPU baseline / reference arm)
+
+def oracle_rate(w: I.Workload, inp: dict, n_tokens: int):
+    """Time the fp64 oracle on a contiguous slice of the workload; returns tokens/s, seconds, cores."""
+    from oracle import moe_oracle as O
+    sl = {k: v for k, v in inp.items()}
+    sl["x"] = inp["x"][:n_tokens]
+    t0 = time.perf_counter()
+    O.layer(sl, w.K, w.routing, w.alpha)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    return n_tokens / dt, dt, cores
+
+
+def calibrated_tokens(w: I.Workload, inp: dict, target_s: float) -> int:
+    """Tokens of oracle work that take about target_s seconds on this host."""
+    rate, _, _ = oracle_rate(w, inp, 128)
+    return int(max(128, min(w.T, rate * target_s)))
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
+    import torch
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    # each rank draws its own batch (seed offset by rank); the weights are the workload's
+    inp = I.make_inputs(w)
+    if rank > 0:
+        inp["x"] = I.make_inputs(I.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}))["x"]
+    shape = LayerShape(w.T, w.D, w.H, w.E, w.K, w.n_shared, w.dtype, w.routing, w.alpha)
+    L = MoELayer(shape, inp, device)
+    dt = L.act_dtype
+    x_host = torch.as_tensor(inp["x"]).to(dt).pin_memory()
+    x = x_host.to(device, non_blocking=False)
+    out_host = torch.empty((w.T, w.D), dtype=dt).pin_memory()
+    aux_host = torch.empty((1,), dtype=torch.float32).pin_memory()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    stages = ["route", "dispatch", "gemm1", "gemm2", "combine"]
+    calls = {"route": lambda: L.route(x), "dispatch": lambda: L.dispatch(x), "gemm1": lambda: L.gemm1(x),
+             "gemm2": L.gemm2, "combine": L.combine}
+
+    def step(events):
+        for i, s in enumerate(stages):
+            events[i].record(stream)
+            calls[s]()
+        events[len(stages)].record(stream)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
+    wev = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+    for i in range(args.warmup):
+        flush.fill_(float(i))
+        step(wev)
+    torch.cuda.synchronize(device)
+    L.check()
+
+    barrier(world, device)
+    torch.cuda.synchronize(device)
+    with ClockSampler(gpu_index_for(local)) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))            # L2 flush outside the step's events
+            step(ev[i])
+        torch.cuda.synchronize(device)
+    barrier(world, device)
+    L.check()
+    clocks = clk.summary()
+
+    per_stage = {s: [] for s in stages}
+    totals = []
+    for i in range(args.steps):
+        for j, s in enumerate(stages):
+            per_stage[s].append(ev[i][j].elapsed_time(ev[i][j + 1]))
+        totals.append(ev[i][0].elapsed_time(ev[i][len(stages)]))
+    my_ms = sum(totals)
+    max_ms = reduce_max(my_ms, world, device)
+    ms_per_step = max_ms / args.steps
+
+    # ---- end to end through the public API: pinned host x in, host out + loss back
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        e2e_ev[i][0].record(stream)
+        x.copy_(x_host, non_blocking=True)
+        L.forward(x)
+        out_host.copy_(L.out, non_blocking=True)
+        aux_host.copy_(L.aux, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in e2e_ev), world, device) / args.steps
+
+    result = None
+    if rank == 0:
+        result = report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world, device)
+        dist.destroy_process_group()
+    return result
+
+
+def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> dict:
+    peaks, peak_kind = load_peaks()
+    elem = 2 if w.dtype == "bf16" else 4
+    race = w.routing == "race"
+    avg = {s: float(np.mean(v)) for s, v in per_stage.items()}
+    g1 = M.gemm1_flops(w.T, w.D, w.H, w.K, w.n_shared)
+    g2 = M.gemm2_flops(w.T, w.D, w.H, w.K, w.n_shared)
+    stage_work = {
+        "route": ("GB/s", M.route_bytes(w.T, w.D, w.E, w.K, elem, race)),
+        "dispatch": ("GB/s", M.dispatch_bytes(w.T, w.D, w.E, w.K, elem, race)),
+        "gemm1": ("TFLOP/s", g1),
+        "gemm2": ("TFLOP/s", g2),
+        "combine": ("GB/s", M.combine_bytes(w.T, w.D, w.K, w.n_shared, elem)),
+    }
+    hbm = peaks["hbm_gbs"]
+    tc_peak = peaks["bf16_tflops_sustained"]
+    stages_out = {}
+    for s, (unit, work) in stage_work.items():
+        ms = avg[s]
+        if unit == "GB/s":
+            a = work / (ms * 1e-3) / 1e9
+            stages_out[s] = {"ms": round(ms, 4), "GB/s": round(a, 1), "frac_hbm": round(a / hbm, 3)}
+        else:
+            a = work / (ms * 1e-3) / 1e12
+            stages_out[s] = {"ms": round(ms, 4), "TFLOP/s": round(a, 1), "frac_bf16": round(a / tc_peak, 3)}
+    dom = "gemm1" if avg["gemm1"] >= avg["gemm2"] else "gemm2"
+    dom_flops = g1 if dom == "gemm1" else g2
+    achieved = dom_flops / (avg[dom] * 1e-3) / 1e12
+    gemm_ms = avg["gemm1"] + avg["gemm2"]
+    mem_ms = avg["route"] + avg["dispatch"] + avg["combine"]
+    mem_bytes = sum(stage_work[s][1] for s in ("route", "dispatch", "combine"))
+    total_tokens = w.T * world
+    value = total_tokens / (ms_per_step * 1e-3)
+    ntok = calibrated_tokens(w, inp, 15.0)
+    rate, secs, cores = oracle_rate(w, inp, ntok)
+    h2d = w.T * w.D * elem
+    d2h = w.T * w.D * elem + 4
+    launches_per_step = (2 + (8 if race else 0)) + 2 + 1 + 1 + 1
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "D": w.D, "H": w.H, "E": w.E, "K": w.K, "n_shared": w.n_shared,
+                   "routing": w.routing, "batch": w.batch, "tokens_per_image": w.tokens_per_image,
+                   "global_batch_tokens": total_tokens, "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": "flushed between steps (256 MB write outside each step's events)"},
+        "layer_tflops": round(M.gemm_flops(w.T, w.D, w.H, w.K, w.n_shared) / (ms_per_step * 1e-3) / 1e12, 1),
+        "gemm_tflops": round((g1 + g2) / (gemm_ms * 1e-3) / 1e12, 1),
+        "gemm_frac_bf16": round((g1 + g2) / (gemm_ms * 1e-3) / 1e12 / tc_peak, 3),
+        "mem_stages_GBps": round(mem_bytes / (mem_ms * 1e-3) / 1e9, 1),
+        "mem_stages_frac_hbm": round(mem_bytes / (mem_ms * 1e-3) / 1e9 / hbm, 3),
+        "stages": stages_out,
+        "roofline": {"kernel": f"tcgen05 grouped expert GEMM ({dom}, one launch per step)", "bound": "tensor",
+                     "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / tc_peak, 3), "traffic": None,
+                     "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)"},
+        "cpu_baseline": {"value": round(rate, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{ntok} contiguous tokens of this workload through the whole fp64 oracle "
+                                   f"layer (router, selection, experts, combine); {secs:.1f} s"},
+        "e2e": {"value": round(total_tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def run_reference(args, w: I.Workload, rank: int, world: int) -> dict:
+    if rank != 0:
+        return None
+    inp = I.make_inputs(w)
+    ntok = calibrated_tokens(w, inp, 6.0)
+    times = []
+    cores = 1
+    for i in range(args.warmup + args.steps):
+        rate, secs, cores = oracle_rate(w, inp, ntok)
+        if i >= args.warmup:
+            times.append(secs)
+    secs = sum(times) / len(times)
+    value = ntok / secs
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "T": w.T, "D": w.D, "H": w.H, "E": w.E, "K": w.K,
+                       "n_shared": w.n_shared, "routing": w.routing},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step: {ntok} contiguous tokens of the workload through the whole "
+                                       f"fp64 oracle layer on the host cores"},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_env()
+    w = I.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        res = run_reference(args, w, rank, world)
+    else:
+        res = run_ours(args, w, rank, world, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -60,8 +60,9 @@ int validate(const moe_config_t* c) {
   if (c->act != 0 && c->act != 1) return fail(MOE_ERR_INVALID_ARG, "act=%d", c->act);
   if (c->gemm_impl != MOE_GEMM_AUTO && c->gemm_impl != MOE_GEMM_SIMT) return fail(MOE_ERR_INVALID_ARG, "gemm_impl=%d", c->gemm_impl);
   if (c->reserved != 0) return fail(MOE_ERR_INVALID_ARG, "reserved field must be 0");
-  if ((size_t)c->E * c->D * 4 + 32 * 128 * 3 + 4096 > 227 * 1024)
-    return fail(MOE_ERR_UNSUPPORTED, "E*D=%d too large for the router's shared-memory gate", c->E * c->D);
+  if (route_smem_total(c->D, c->E, 32, c->dtype == MOE_BF16) > 232448 ||
+      (c->dtype == MOE_BF16 && route_mma_stages(c->D, c->E) < 2))
+    return fail(MOE_ERR_UNSUPPORTED, "E=%d x D=%d too large for the router's shared memory", c->E, c->D);
   return MOE_OK;
 }
 
@@ -88,7 +89,8 @@ struct WsLayout {
 WsLayout ws_layout(const moe_config_t* c) {
   WsLayout L{};
   const size_t T = (size_t)c->T, E = (size_t)c->E;
-  const size_t max_route_tiles = (T + 31) / 32 + 1;
+  // partial rows: one per router CTA (<= one per 16 tokens) or per fp32 token tile (>= 32 rows)
+  const size_t max_route_tiles = (T + 15) / 16 + 1;
   const size_t race_tiles = (T + 127) / 128 + 1;
   int ch, nch;
   chunking(c->T, &ch, &nch);
@@ -243,29 +245,38 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   if (race && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
   const WsLayout L = ws_layout(cfg);
   const int sms = num_sms_current();
-  // tile of tokens per CTA: spread T over the SMs, 32..256 rows, shared memory permitting
-  int tile = (int)round_up((size_t)((cfg->T + sms - 1) / sms), 32);
-  if (tile < 32) tile = 32;
-  if (tile > 256) tile = 256;
-  while (tile > 32 && route_smem_bytes(cfg->D, cfg->E, tile, cfg->dtype) > 227 * 1024) tile -= 32;
+  int tile = 0, threads = 0;
+  const bool bf16 = cfg->dtype == MOE_BF16;
+  route_plan(cfg->T, cfg->D, cfg->E, bf16, sms, &tile, &threads);
   const int ntiles = (cfg->T + tile - 1) / tile;
+  const int grid = ntiles < sms ? ntiles : sms;
+  // partial sums: one row per CTA (bf16 kernel) or per token tile (fp32 kernel)
+  const int nparts = bf16 ? grid : ntiles;
   CUtensorMap tm;
-  if ((rc = make_tmap(&tm, x, cfg->dtype == MOE_BF16, cfg->T, cfg->D, tile, "x"))) return rc;
+  if ((rc = make_tmap(&tm, x, bf16, cfg->T, cfg->D, tile, "x"))) return rc;
   RouteArgs ra{};
   ra.x = x; ra.wg = wg; ra.bias = router_bias;
-  ra.T = cfg->T; ra.D = cfg->D; ra.E = cfg->E; ra.K = cfg->K; ra.bf16 = cfg->dtype == MOE_BF16;
-  ra.tile_rows = tile; ra.ntiles = ntiles; ra.grid = ntiles < sms ? ntiles : sms;
+  ra.T = cfg->T; ra.D = cfg->D; ra.E = cfg->E; ra.K = cfg->K; ra.bf16 = bf16;
+  ra.tile_rows = tile; ra.ntiles = ntiles; ra.grid = grid;
   ra.topk_idx = topk_idx; ra.topk_w = topk_w; ra.n_sel = race ? nullptr : n_sel;
   ra.P = race ? ws_at<float>(ws, L.P) : nullptr;
   ra.tile_counts = ws_at<int32_t>(ws, L.tile_counts);
   ra.tile_psum = ws_at<float>(ws, L.tile_psum);
   ra.status = status_ptr(ws);
-  if ((e = launch_route(ra, &tm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
   FinalizeArgs fa{};
   fa.T = cfg->T; fa.E = cfg->E; fa.K = cfg->K; fa.alpha = cfg->alpha;
   fa.counts = counts; fa.aux_loss = aux_loss;
-  fa.tile_psum = ra.tile_psum; fa.ntiles_psum = ntiles;
-  if (race) {
+  fa.tile_psum = ra.tile_psum; fa.ntiles_psum = nparts;
+  fa.tile_counts = ra.tile_counts; fa.ntiles_counts = nparts;
+  fa.ctr = ws_at<unsigned int>(ws, 64);
+  if (!race) {
+    // the router's last block finalizes counts and loss
+    if ((e = launch_route(ra, fa, &tm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
+    return ok();
+  }
+  FinalizeArgs none{};
+  if ((e = launch_route(ra, none, &tm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
+  {
     RaceArgs rr{};
     rr.P = ra.P; rr.T = cfg->T; rr.E = cfg->E; rr.K = cfg->K;
     rr.hist = ws_at<uint32_t>(ws, L.hist);
@@ -278,8 +289,6 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
     if ((e = cudaMemsetAsync(rr.hist, 0, 4096 * 4, s)) != cudaSuccess) return cuda_fail(e, "moe_route");
     if ((e = launch_race_select(rr, s)) != cudaSuccess) return cuda_fail(e, "race select kernels");
     fa.tile_counts = rr.tile_counts; fa.ntiles_counts = rr.ntiles;
-  } else {
-    fa.tile_counts = ra.tile_counts; fa.ntiles_counts = ntiles;
   }
   if ((e = launch_route_finalize(fa, s)) != cudaSuccess) return cuda_fail(e, "route finalize kernel");
   return ok();

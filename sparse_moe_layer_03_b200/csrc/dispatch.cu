@@ -7,92 +7,35 @@
 // from integer counts and prefix sums only (no order-dependent atomics), so
 // the permutation is deterministic and equals the canonical one bit for bit.
 //
-//   plan kernel   (1 block): per-chunk expert counts -> prefix over chunks ->
-//                 offsets, padded offsets, chunk bases; marks padding rows.
-//   gather kernel (1 block per chunk of tokens): ranks inside the chunk by warp
-//                 ballots, positions, then 16-byte row copies x -> x_perm.
+//   count kernel  (1 block per chunk of tokens): per-chunk expert counts.
+//   gather kernel (1 block per chunk): sums of the chunk counts give the
+//                 padded segment starts and the chunk's base in each segment;
+//                 ranks inside the chunk by warp ballots; positions; padding
+//                 rows marked; 16-byte row copies x -> x_perm.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
 
-constexpr int kPlanThreads = 1024;
 constexpr int kGatherThreads = 256;
 
-// exclusive scan of one value per thread over a 1024-thread block
-__device__ __forceinline__ int block_excl_scan_1024(int v, int* warp_tot, int& total) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_tot[w] = x;
+// per-chunk expert counts, expert-major: cnt[e * nchunks + c]
+__global__ void __launch_bounds__(kGatherThreads) dispatch_count_kernel(DispatchArgs a) {
+  __shared__ int cc[32];
+  const int tid = threadIdx.x, c = blockIdx.x, Kmax = a.Kmax;
+  if (tid < 32) cc[tid] = 0;
   __syncthreads();
-  if (w == 0) {
-    int t = warp_tot[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += y;
-    }
-    warp_tot[lane] = t;   // inclusive totals of warps
-  }
-  __syncthreads();
-  const int before = (w ? warp_tot[w - 1] : 0) + x - v;
-  total = warp_tot[31];
-  __syncthreads();
-  return before;
-}
-
-__global__ void __launch_bounds__(kPlanThreads) dispatch_plan_kernel(DispatchArgs a) {
-  extern __shared__ int cc[];   // [nchunks][E]
-  __shared__ int warp_tot[32];
-  __shared__ int tot[33], poff[33];
-  const int tid = threadIdx.x;
-  const int E = a.E, Kmax = a.Kmax;
-  for (int i = tid; i < a.nchunks * E; i += kPlanThreads) cc[i] = 0;
-  __syncthreads();
-  const long long npairs = (long long)a.T * Kmax;
-  for (long long i = tid; i < npairs; i += kPlanThreads) {
-    const int t = (int)(i / Kmax), k = (int)(i % Kmax);
+  const int t0 = c * a.chunk;
+  const int n = min(a.chunk, a.T - t0) * Kmax;
+  for (int i = tid; i < n; i += kGatherThreads) {
+    const int t = t0 + i / Kmax, k = i % Kmax;
     const int ns = a.n_sel ? a.n_sel[t] : a.K;
     if (k >= ns) continue;
-    const int e = a.topk_idx[i];
-    if (e >= 0 && e < E) atomicAdd(&cc[(t / a.chunk) * E + e], 1);
+    const int e = a.topk_idx[(size_t)t0 * Kmax + i];
+    if (e >= 0 && e < a.E) atomicAdd(&cc[e], 1);
   }
   __syncthreads();
-  for (int e = 0; e < E; ++e) {
-    const int v = tid < a.nchunks ? cc[tid * E + e] : 0;
-    int total;
-    const int before = block_excl_scan_1024(v, warp_tot, total);
-    if (tid < a.nchunks) cc[tid * E + e] = before;
-    if (tid == 0) tot[e] = total;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int u = 0, p = 0;
-    for (int e = 0; e < E; ++e) {
-      a.offsets[e] = u;
-      poff[e] = p;
-      u += tot[e];
-      p += (tot[e] + 127) / 128 * 128;
-    }
-    a.offsets[E] = u;
-    poff[E] = p;
-  }
-  __syncthreads();
-  for (int i = tid; i < a.nchunks * E; i += kPlanThreads) a.chunk_base[i] = poff[i % E] + cc[i];
-  // padding rows: inside each segment after its last token, and after the last segment
-  for (int e = 0; e <= E; ++e) {
-    const long long lo = e < E ? (long long)poff[e] + tot[e] : poff[E];
-    const long long hi = e < E ? (long long)poff[e + 1] : a.r_max;
-    for (long long r = lo + tid; r < hi; r += kPlanThreads) {
-      a.row_token[r] = -1;
-      a.row_gate[r] = 0.f;
-    }
-  }
+  if (tid < a.E) a.chunk_base[(size_t)tid * a.nchunks + c] = cc[tid];
 }
 
 template <typename T, int EMAX>
@@ -102,10 +45,51 @@ __global__ void __launch_bounds__(kGatherThreads) dispatch_gather_kernel(Dispatc
   int* sidx = sm;                     // [CH][Kmax] expert of each slot (-1 unused)
   int* spos = sm + CH * Kmax;         // [CH][Kmax] rank in warp, then row
   __shared__ int wcnt[kGatherThreads / 32][EMAX];
+  __shared__ int before_s[EMAX], total_s[EMAX], poff_s[EMAX + 1];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int c = blockIdx.x;
   const int t0 = c * CH;
 
+  // ---- segment starts and this chunk's base: sums over the chunk counts
+  for (int e = w; e < E; e += kGatherThreads / 32) {
+    const int* row = a.chunk_base + (size_t)e * a.nchunks;
+    int before = 0, total = 0;
+#pragma unroll 4
+    for (int j = lane; j < a.nchunks; j += 32) {
+      const int v = row[j];
+      total += v;
+      before += j < c ? v : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+    }
+    if (lane == 0) { total_s[e] = total; before_s[e] = before; }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int p = 0;
+    for (int e = 0; e < E; ++e) { poff_s[e] = p; p += (total_s[e] + 127) / 128 * 128; }
+    poff_s[E] = p;
+  }
+  __syncthreads();
+  if (c == 0 && tid <= E) {
+    int u = 0;
+    for (int e = 0; e < tid; ++e) u += total_s[e];
+    a.offsets[tid] = u;
+  }
+  // padding rows: segment e's tail (e < E) or the rows after the last segment (e = E)
+  for (int e = c; e <= E; e += gridDim.x) {
+    const long long lo = e < E ? (long long)poff_s[e] + total_s[e] : poff_s[E];
+    const long long hi = e < E ? (long long)poff_s[e + 1] : a.r_max;
+    for (long long r = lo + tid; r < hi; r += kGatherThreads) {
+      a.row_token[r] = -1;
+      a.row_gate[r] = 0.f;
+    }
+  }
+
+  // ---- slots of this chunk
   for (int i = tid; i < CH * Kmax; i += kGatherThreads) {
     const int l = i / Kmax, k = i % Kmax, t = t0 + l;
     int e = -1;
@@ -120,6 +104,7 @@ __global__ void __launch_bounds__(kGatherThreads) dispatch_gather_kernel(Dispatc
     spos[i] = -1;
   }
   __syncthreads();
+  // ---- rank of each token among the chunk's tokens of the same expert (token order)
   if (w < CH / 32) {
     const int l = w * 32 + lane;
     for (int e = 0; e < E; ++e) {
@@ -138,7 +123,7 @@ __global__ void __launch_bounds__(kGatherThreads) dispatch_gather_kernel(Dispatc
     const int e = sidx[i];
     int p = -1;
     if (e >= 0) {
-      int base = a.chunk_base[(size_t)c * E + e];
+      int base = poff_s[e] + before_s[e];
       for (int ww = 0; ww < l / 32; ++ww) base += wcnt[ww][e];
       p = base + spos[i];
       if (p < 0 || p >= a.r_max) { set_status(a.status, DEV_BAD_INDEX, 201); p = -1; }
@@ -151,7 +136,7 @@ __global__ void __launch_bounds__(kGatherThreads) dispatch_gather_kernel(Dispatc
     spos[i] = p;
   }
   __syncthreads();
-  // row copies: one warp per token, 16-byte vectors
+  // ---- row copies: one warp per token, 16-byte vectors
   const int nvec = a.D * (int)sizeof(T) / 16;
   const uint4* xv = reinterpret_cast<const uint4*>(a.x);
   uint4* xp = reinterpret_cast<uint4*>(a.x_perm);
@@ -195,12 +180,9 @@ static cudaError_t launch_gather_t(const DispatchArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)a.nchunks * a.E * sizeof(int);
-  cudaError_t err = cudaFuncSetAttribute(dispatch_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  dispatch_count_kernel<<<a.nchunks, kGatherThreads, 0, s>>>(a);
+  cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  dispatch_plan_kernel<<<1, kPlanThreads, smem, s>>>(a);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
   return a.bf16 ? launch_gather_t<__nv_bfloat16>(a, s) : launch_gather_t<float>(a, s);
 }
 

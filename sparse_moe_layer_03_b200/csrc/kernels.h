@@ -21,15 +21,20 @@ struct RouteArgs {
   float* tile_psum;         // [ntiles,E]
   int* status;
 };
-cudaError_t launch_route(const RouteArgs& a, const CUtensorMap* tmap_x, cudaStream_t s);
 size_t route_smem_bytes(int D, int E, int tile_rows, int bf16);
+size_t route_smem_total(int D, int E, int tile_rows, int bf16);
+int route_mma_stages(int D, int E);
+void route_plan(int T, int D, int E, int bf16, int sms, int* tile_rows, int* threads);
 
+// partial counts / score sums -> counts[E] and the balance loss
 struct FinalizeArgs {
   const int32_t* tile_counts; int ntiles_counts;
   const float* tile_psum; int ntiles_psum;
   int T, E, K; float alpha;
-  int32_t* counts; float* aux_loss;
+  int32_t* counts; float* aux_loss;   // counts == null: the router leaves finalizing to a later kernel
+  unsigned int* ctr;                  // blocks-done counter in ws (zero between calls)
 };
+cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tmap_x, cudaStream_t s);
 cudaError_t launch_route_finalize(const FinalizeArgs& a, cudaStream_t s);
 
 struct RaceArgs {

@@ -7,57 +7,361 @@
 // Parameters", "MOE-DIT" (balance loss eq. L_balance); "Expert Race" abstract
 // (tokens and experts compete jointly for the top candidates).
 //
-// The logits are memory-bound (E FMAs per element of x): x streams through
-// shared memory in 128-byte-swizzled column chunks fed by TMA, one or two
-// tokens per thread, the gate weight sits in shared memory as fp32 and is read
-// by broadcast.  Per-tile partial counts and score sums are reduced in a fixed
-// order, so the loss is bit-reproducible.
+// The logits are HBM-bound: x streams through shared memory once, in
+// 128-byte-swizzled column chunks fed by TMA.  bf16 inputs take their E dot
+// products on mma.sync (the FP32 pipe alone cannot keep up with HBM at E = 16);
+// fp32 inputs use FFMA.  Per-tile partial counts and score sums are reduced in
+// a fixed order, so the loss is bit-reproducible.
 #include <cuda.h>
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
 
-constexpr int kRouteThreads = 128;
-constexpr int kRouteStages = 3;
+constexpr int kRouteThreads = 128;     // FFMA kernel (fp32 inputs)
+constexpr int kRouteStages = 4;
 
-size_t route_smem_bytes(int D, int E, int tile_rows, int bf16) {
-  (void)bf16;
-  size_t wg = (size_t)E * D * sizeof(float);
-  wg = (wg + 1023) & ~(size_t)1023;
-  // align slack + gate + x stages + barriers (24 B) + counts (<= 128 B) + warp sums (<= 512 B)
-  return 1024 + wg + (size_t)kRouteStages * tile_rows * 128 + 1024;
+__host__ __device__ inline int route_emax(int E) { return E <= 8 ? 8 : (E <= 16 ? 16 : 32); }
+__host__ __device__ inline size_t align1k(size_t v) { return (v + 1023) & ~(size_t)1023; }
+
+// Shared-memory layout of both router kernels (bytes from the 1024-aligned base):
+//   gate weight | x stages (tile_rows x 128 B each) | logits (mma only) | barriers, counts, sums
+struct RouteSmem {
+  size_t wg, x, logits, misc, total;
+};
+__host__ __device__ inline RouteSmem route_layout(int D, int E, int tile_rows, int bf16) {
+  RouteSmem L;
+  const int em = route_emax(E);
+  L.wg = 0;
+  const size_t wg_bytes = bf16 ? (size_t)em * (D * 2 + 16) : (size_t)E * D * 4;
+  L.x = align1k(wg_bytes);
+  // the x stages double as the finalize scratch (2 x 32 x 33 x 8 bytes) at the end
+  const size_t xb = (size_t)kRouteStages * tile_rows * 128;
+  L.logits = L.x + (xb > 16896 ? xb : 16896);
+  L.misc = L.logits + (bf16 ? (size_t)tile_rows * em * 4 : 0);
+  // barriers (4 x 8 B) + counts (<= 32 x 4 B) + warp sums (8 x 32 x 4 B)
+  L.total = 1024 /*alignment slack*/ + L.misc + 2048;
+  return L;
 }
 
-template <typename T, int EMAX>
-__global__ void __launch_bounds__(kRouteThreads, 1)
-route_kernel(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a) {
+size_t route_smem_bytes(int D, int E, int tile_rows, int bf16) {
+  return route_layout(D, E, tile_rows, bf16).total;
+}
+
+// Per token: bias, softmax, then top-K selection (or the score row for
+// Expert-Race); score sums and counts accumulate for the balance loss.
+template <int EMAX>
+__device__ __forceinline__ void token_select(const float* logit, int tok, const RouteArgs& a, int* cnt_s,
+                                             float* psum) {
+  const int E = a.E;
+  float P[EMAX];
+  float m = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) {
+    if (e < E) {
+      float l = logit[e];
+      if (a.bias) l += a.bias[e];
+      P[e] = l;
+      m = fmaxf(m, l);
+    }
+  }
+  float z = 0.f;
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e)
+    if (e < E) { P[e] = expf(P[e] - m); z += P[e]; }
+  const float inv = 1.0f / z;
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e)
+    if (e < E) { P[e] = P[e] * inv; psum[e] += P[e]; }
+  if (a.P) {
+    float* prow = a.P + (size_t)tok * E;
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e)
+      if (e < E) prow[e] = P[e];
+    return;
+  }
+  uint32_t taken = 0;
+  for (int k = 0; k < a.K; ++k) {
+    float bp = -1.f;
+    int bi = -1;
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e)
+      if (e < E && !((taken >> e) & 1u) && P[e] > bp) { bp = P[e]; bi = e; }
+    if (bi >= 0) { taken |= 1u << bi; atomicAdd(&cnt_s[bi], 1); }
+    a.topk_idx[(size_t)tok * a.K + k] = bi;
+    a.topk_w[(size_t)tok * a.K + k] = bi >= 0 ? bp : 0.f;
+  }
+  if (a.n_sel) a.n_sel[tok] = a.K;
+}
+
+// Fixed-order reduction of the per-thread score sums (lanes, then warps) and
+// the tile's partial outputs.  Every thread of the block calls it.
+template <int EMAX>
+__device__ __forceinline__ void tile_partials(const float* psum, int tile, const RouteArgs& a, const int* cnt_s,
+                                              float* wsum_s) {
+  const int tid = threadIdx.x, w = tid >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) {
+    if (e < a.E) {
+      float v = psum[e];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if ((tid & 31) == 0) wsum_s[w * EMAX + e] = v;
+    }
+  }
+  __syncthreads();
+  if (tid < a.E) {
+    float v = 0.f;
+    for (int k = 0; k < nw; ++k) v += wsum_s[k * EMAX + tid];
+    a.tile_psum[(size_t)tile * a.E + tid] = v;
+    if (!a.P) a.tile_counts[(size_t)tile * a.E + tid] = cnt_s[tid];
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------- bf16: tensor-core logits
+// Work unit = a block of 16 consecutive tokens: their full rows (16 x D bf16,
+// one contiguous stretch of HBM, so DRAM pages are read whole) land in one
+// shared-memory buffer as D/64 TMA boxes of 16 rows x 128 bytes (128-byte
+// swizzle).  Every warp owns one buffer and runs its own pipeline over its
+// units with no block-wide barrier: wait for the rows, compute the 16 x E
+// logits with mma.sync m16n8k16 (A via ldmatrix from the swizzled buffer, B =
+// gate weight in shared memory with rows padded by 16 bytes), re-issue the
+// buffer for the next unit, then run softmax and selection (one lane per
+// token) while those rows load.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void mma_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+constexpr int kMmaRB = 16;        // tokens per work unit
+constexpr int kMmaMaxWarps = 8;
+
+// One TMA buffer (16 full rows) per warp; as many warps as buffers fit.
+struct MmaSmem {
+  size_t wg, x, logits, misc, total;
+  int warps;
+};
+__host__ __device__ inline MmaSmem mma_layout(int D, int E) {
+  MmaSmem L;
+  const int em = route_emax(E);
+  L.wg = 0;
+  L.x = align1k((size_t)em * (D * 2 + 16));
+  const size_t stage = (size_t)kMmaRB * D * 2;
+  const size_t per_warp_logits = (size_t)kMmaRB * em * 4;
+  const size_t fixed = L.x + 2048 /*misc*/ + 1024 /*align slack*/ + 1024 /*scratch margin*/;
+  int nw = (int)((232448 - fixed) / (stage + per_warp_logits));
+  L.warps = nw > kMmaMaxWarps ? kMmaMaxWarps : nw;
+  const size_t xb = (size_t)(L.warps > 0 ? L.warps : 0) * stage;
+  L.logits = L.x + (xb > 16896 ? xb : 16896);   // x buffers double as the finalize scratch
+  L.misc = L.logits + (size_t)(L.warps > 0 ? L.warps : 0) * per_warp_logits;
+  L.total = L.misc + 2048 + 1024;
+  return L;
+}
+
+// The last block to finish turns the per-block partials into counts and the loss.
+// scratch: 2 x 32 x 33 x 8 bytes of shared memory
+constexpr int kFinalizeScratch = 2 * 32 * 33 * 8;
+__device__ void finalize_counts_loss(const FinalizeArgs& a, uint8_t* scratch) {
+  auto cs = reinterpret_cast<long long(*)[33]>(scratch);
+  auto ps = reinterpret_cast<double(*)[33]>(scratch + 32 * 33 * 8);
+  const int tid = threadIdx.x, e = tid & 31, g = tid >> 5, ng = blockDim.x >> 5;
+  for (int k = g; k < 32; k += ng) { cs[k][e] = 0; ps[k][e] = 0.0; }
+  __syncthreads();
+  long long c = 0;
+  double p = 0.0;
+  if (e < a.E) {
+    for (int t = g; t < a.ntiles_counts; t += ng) c += __ldcg(a.tile_counts + (size_t)t * a.E + e);
+    for (int t = g; t < a.ntiles_psum; t += ng) p += (double)__ldcg(a.tile_psum + (size_t)t * a.E + e);
+  }
+  cs[g][e] = c;
+  ps[g][e] = p;
+  __syncthreads();
+  if (tid < 32) {
+    long long cc = 0;
+    double pp = 0.0;
+    for (int k = 0; k < 32; ++k) { cc += cs[k][tid]; pp += ps[k][tid]; }
+    double term = 0.0;
+    if (tid < a.E) {
+      a.counts[tid] = (int32_t)cc;
+      term = ((double)a.E / ((double)a.K * a.T)) * (double)cc * (pp / a.T);
+    }
+    for (int o = 16; o > 0; o >>= 1) term += __shfl_down_sync(0xffffffffu, term, o);
+    if (tid == 0) *a.aux_loss = (float)(a.alpha * term);
+  }
+}
+
+// Count this block as done; true for the block that finishes last (which then
+// also resets the counter for the next call).
+__device__ bool last_block_done(unsigned int* ctr) {
+  __shared__ bool last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned int prev = atomicAdd(ctr, 1u);
+    last = prev == gridDim.x - 1;
+    if (last) *ctr = 0u;
+  }
+  __syncthreads();
+  if (last) __threadfence();
+  return last;
+}
+
+template <int EMAX>
+__global__ void __launch_bounds__(kMmaMaxWarps * 32, 1)
+route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, FinalizeArgs fin) {
+  constexpr int NT = EMAX / 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const int E = a.E, D = a.D;
-  float* wg_s = reinterpret_cast<float*>(smem);
-  const size_t wg_bytes = (((size_t)E * D * 4) + 1023) & ~(size_t)1023;
-  uint8_t* xs = smem + wg_bytes;
-  const int stage_bytes = a.tile_rows * 128;
-  uint64_t* full = reinterpret_cast<uint64_t*>(xs + (size_t)kRouteStages * stage_bytes);
-  int* cnt_s = reinterpret_cast<int*>(full + kRouteStages);          // [EMAX]
-  float* wsum_s = reinterpret_cast<float*>(cnt_s + EMAX);             // [4][EMAX]
+  const MmaSmem L = mma_layout(a.D, a.E);
+  const int NW = blockDim.x >> 5;
+  const int E = a.E, D = a.D, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int wg_stride = D * 2 + 16;
+  const int nchunks = D / 64;
+  const int stage_bytes = kMmaRB * D * 2;
+  uint8_t* wg_s = smem + L.wg;
+  uint8_t* xs = smem + L.x;
+  float* logit_w = reinterpret_cast<float*>(smem + L.logits) + (size_t)w * kMmaRB * EMAX;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.misc);   // one barrier per warp
+  int* cnt_s = reinterpret_cast<int*>(full + kMmaMaxWarps);
+  float* wsum_s = reinterpret_cast<float*>(cnt_s + 32);
 
-  constexpr int CC = 128 / (int)sizeof(T);    // columns per 128-byte chunk
-  constexpr int VEC = 16 / (int)sizeof(T);    // elements per 16-byte vector
+  const int nunits = (a.T + kMmaRB - 1) / kMmaRB;
+  const int gw = blockIdx.x * NW + w, nwarps = gridDim.x * NW;
+  const int my_units = gw < nunits ? (nunits - gw + nwarps - 1) / nwarps : 0;
+  const uint32_t buf = smem_u32(xs + (size_t)w * stage_bytes);
+  const uint32_t bar = smem_u32(&full[w]);
+  auto issue = [&](int i) {              // lane 0: the 16 rows of unit i, all D/64 boxes
+    const int u = gw + i * nwarps;
+    mbar_arrive_expect_tx(bar, stage_bytes);
+    for (int c = 0; c < nchunks; ++c) tma_load_2d(buf + c * (kMmaRB * 128), &tmap_x, c * 64, u * kMmaRB, bar);
+  };
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    if (my_units > 0) issue(0);          // x streams in while the gate weight loads
+  }
+  if (tid < 32) cnt_s[tid] = 0;
+  {  // gate weight (bf16) -> padded rows; rows E..EMAX-1 are zero
+    const int vpr = D / 8;
+    const uint4* wv = reinterpret_cast<const uint4*>(a.wg);
+#pragma unroll 4
+    for (int i = tid; i < EMAX * vpr; i += blockDim.x) {
+      const int e = i / vpr, v = i % vpr;
+      const uint4 val = e < E ? __ldg(wv + (size_t)e * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(wg_s + (size_t)e * wg_stride + v * 16) = val;
+    }
+  }
+  __syncthreads();
+
+  const uint32_t wg_base = smem_u32(wg_s);
+  const int li = lane >> 3, lj = lane & 7;
+  float psum[EMAX];
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) psum[e] = 0.f;
+  bool ok = true;
+  for (int i = 0; i < my_units && ok; ++i) {
+    const int u = gw + i * nwarps;
+    ok = mbar_wait(bar, i & 1, nullptr, a.status, 100);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[nt][q] = 0.f;
+    for (int c = 0; c < nchunks; ++c) {
+      const uint32_t box = buf + c * (kMmaRB * 128);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        uint32_t b[NT][2];
+        const int kc = c * 64 + ks * 16 + (li & 1) * 8;
+#pragma unroll
+        for (int np = 0; np < NT; np += 2) {
+          if (np + 1 < NT) {
+            const int n = (np + (li >> 1)) * 8 + lj;
+            ldsm_x4(wg_base + n * wg_stride + kc * 2, b[np][0], b[np][1], b[np + 1][0], b[np + 1][1]);
+          } else {
+            ldsm_x2(wg_base + (np * 8 + lj) * wg_stride + kc * 2, b[np][0], b[np][1]);
+          }
+        }
+        const int row = (li & 1) * 8 + lj;
+        const int chunk = ks * 2 + (li >> 1);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_16816(acc[nt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
+      }
+    }
+    __syncwarp();                                  // every lane is done reading the buffer
+    if (lane == 0 && i + 1 < my_units) issue(i + 1);   // next rows load during the epilogue
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int row = lane >> 2, col = nt * 8 + (lane & 3) * 2;
+      logit_w[row * EMAX + col] = acc[nt][0];
+      logit_w[row * EMAX + col + 1] = acc[nt][1];
+      logit_w[(row + 8) * EMAX + col] = acc[nt][2];
+      logit_w[(row + 8) * EMAX + col + 1] = acc[nt][3];
+    }
+    __syncwarp();
+    if (lane < kMmaRB) {
+      const int tok = u * kMmaRB + lane;
+      if (tok < a.T) {
+        float l[EMAX];
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) l[e] = logit_w[lane * EMAX + e];
+        token_select<EMAX>(l, tok, a, cnt_s, psum);
+      }
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  tile_partials<EMAX>(psum, blockIdx.x, a, cnt_s, wsum_s);
+  if (!ok) set_status(a.status, DEV_TIMEOUT, 102);
+  if (fin.counts != nullptr && last_block_done(fin.ctr)) finalize_counts_loss(fin, xs);
+}
+
+// ---------------------------------------------------------------- fp32: FFMA logits
+// fp32 inputs keep true fp32 products (a 1e-5 bound rules out tf32 tensor
+// cores): one or two tokens per thread, the gate weight as fp32 in shared
+// memory read by broadcast.
+template <int EMAX>
+__global__ void __launch_bounds__(kRouteThreads, 1)
+route_kernel_ffma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, FinalizeArgs fin) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const RouteSmem L = route_layout(a.D, a.E, a.tile_rows, 0);
+  const int E = a.E, D = a.D, tid = threadIdx.x;
+  constexpr int CC = 32;     // fp32 columns per 128-byte chunk
   const int nchunks = D / CC;
-  const int tid = threadIdx.x;
-
-  // gate weight -> fp32 shared memory
-  const T* wg = reinterpret_cast<const T*>(a.wg);
-  for (int i = tid; i < E * D; i += kRouteThreads) wg_s[i] = Elem<T>::to_f(wg[i]);
+  float* wg_s = reinterpret_cast<float*>(smem + L.wg);
+  uint8_t* xs = smem + L.x;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.misc);
+  int* cnt_s = reinterpret_cast<int*>(full + kRouteStages);
+  float* wsum_s = reinterpret_cast<float*>(cnt_s + 32);
+  const int stage_bytes = a.tile_rows * 128;
+  {
+    const float4* wv = reinterpret_cast<const float4*>(a.wg);
+#pragma unroll 4
+    for (int i = tid; i < E * D / 4; i += kRouteThreads) reinterpret_cast<float4*>(wg_s)[i] = __ldg(wv + i);
+  }
   if (tid == 0) {
     for (int s = 0; s < kRouteStages; ++s) mbar_init(smem_u32(&full[s]), 1);
     fence_barrier_init();
     prefetch_tmap(&tmap_x);
   }
   __syncthreads();
-
   const int my_tiles = (a.ntiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
   const int items = my_tiles * nchunks;
   auto issue = [&](int item) {
@@ -70,199 +374,114 @@ route_kernel(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a) {
   };
   if (tid == 0)
     for (int i = 0; i < kRouteStages && i < items; ++i) issue(i);
-
   const int r0 = tid, r1 = tid + kRouteThreads;
   const bool has0 = r0 < a.tile_rows, has1 = r1 < a.tile_rows;
   float acc0[EMAX], acc1[EMAX];
-
   for (int it = 0; it < items; ++it) {
-    const int tl = it / nchunks;
     const int c = it % nchunks;
-    const int tile = blockIdx.x + tl * gridDim.x;
+    const int tile = blockIdx.x + (it / nchunks) * gridDim.x;
     if (c == 0) {
 #pragma unroll
       for (int e = 0; e < EMAX; ++e) { acc0[e] = 0.f; acc1[e] = 0.f; }
-      if (tid < EMAX) cnt_s[tid] = 0;
+      if (tid < 32) cnt_s[tid] = 0;
     }
     const int s = it % kRouteStages;
-    const bool ok = mbar_wait(smem_u32(&full[s]), (it / kRouteStages) & 1, nullptr, a.status, 100);
+    const bool ok = mbar_wait(smem_u32(&full[s]), (it / kRouteStages) & 1, nullptr, a.status, 101);
     const uint8_t* st = xs + (size_t)s * stage_bytes;
-#pragma unroll 2
     for (int j = 0; j < (ok ? 8 : 0); ++j) {
-      float f0[VEC], f1[VEC];
+      float f0[4] = {0.f, 0.f, 0.f, 0.f}, f1[4] = {0.f, 0.f, 0.f, 0.f};
       if (has0) {
-        const uint4 v = *reinterpret_cast<const uint4*>(st + r0 * 128 + ((j ^ (r0 & 7)) << 4));
-        if constexpr (sizeof(T) == 2) bf16x8_to_f32(v, f0);
-        else { f0[0] = __uint_as_float(v.x); f0[1] = __uint_as_float(v.y); f0[2] = __uint_as_float(v.z); f0[3] = __uint_as_float(v.w); }
+        const float4 v = *reinterpret_cast<const float4*>(st + r0 * 128 + ((j ^ (r0 & 7)) << 4));
+        f0[0] = v.x; f0[1] = v.y; f0[2] = v.z; f0[3] = v.w;
       }
       if (has1) {
-        const uint4 v = *reinterpret_cast<const uint4*>(st + r1 * 128 + ((j ^ (r1 & 7)) << 4));
-        if constexpr (sizeof(T) == 2) bf16x8_to_f32(v, f1);
-        else { f1[0] = __uint_as_float(v.x); f1[1] = __uint_as_float(v.y); f1[2] = __uint_as_float(v.z); f1[3] = __uint_as_float(v.w); }
-      } else {
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) f1[v] = 0.f;
+        const float4 v = *reinterpret_cast<const float4*>(st + r1 * 128 + ((j ^ (r1 & 7)) << 4));
+        f1[0] = v.x; f1[1] = v.y; f1[2] = v.z; f1[3] = v.w;
       }
-      const int col = c * CC + j * VEC;
+      const int col = c * CC + j * 4;
 #pragma unroll
       for (int e = 0; e < EMAX; ++e) {
         if (e < E) {
-          const float4* wp = reinterpret_cast<const float4*>(wg_s + (size_t)e * D + col);
-#pragma unroll
-          for (int q = 0; q < VEC / 4; ++q) {
-            const float4 w4 = wp[q];
-            acc0[e] = fmaf(f0[4 * q + 0], w4.x, acc0[e]);
-            acc0[e] = fmaf(f0[4 * q + 1], w4.y, acc0[e]);
-            acc0[e] = fmaf(f0[4 * q + 2], w4.z, acc0[e]);
-            acc0[e] = fmaf(f0[4 * q + 3], w4.w, acc0[e]);
-            acc1[e] = fmaf(f1[4 * q + 0], w4.x, acc1[e]);
-            acc1[e] = fmaf(f1[4 * q + 1], w4.y, acc1[e]);
-            acc1[e] = fmaf(f1[4 * q + 2], w4.z, acc1[e]);
-            acc1[e] = fmaf(f1[4 * q + 3], w4.w, acc1[e]);
-          }
+          const float4 w4 = *reinterpret_cast<const float4*>(wg_s + (size_t)e * D + col);
+          acc0[e] = fmaf(f0[0], w4.x, fmaf(f0[1], w4.y, fmaf(f0[2], w4.z, fmaf(f0[3], w4.w, 0.f)))) + acc0[e];
+          acc1[e] = fmaf(f1[0], w4.x, fmaf(f1[1], w4.y, fmaf(f1[2], w4.z, fmaf(f1[3], w4.w, 0.f)))) + acc1[e];
         }
       }
     }
-    // every thread is done with stage s; a timed-out wait ends the whole block
-    if (__syncthreads_or(!ok)) return;
+    if (__syncthreads_or(!ok)) { set_status(a.status, DEV_TIMEOUT, 103); break; }
     if (tid == 0 && it + kRouteStages < items) issue(it + kRouteStages);
-
     if (c == nchunks - 1) {
-      // ---- per-token softmax + selection for the (up to) two rows of this thread
       float psum[EMAX];
 #pragma unroll
       for (int e = 0; e < EMAX; ++e) psum[e] = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int r = half ? r1 : r0;
-        const bool has = half ? has1 : has0;
-        const int tok = tile * a.tile_rows + r;
-        if (!has || tok >= a.T) continue;
-        float P[EMAX];
-        float m = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-          if (e < E) {
-            float l = half ? acc1[e] : acc0[e];
-            if (a.bias) l += a.bias[e];
-            P[e] = l;
-            m = fmaxf(m, l);
-          }
-        }
-        float z = 0.f;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e)
-          if (e < E) { P[e] = expf(P[e] - m); z += P[e]; }
-        const float inv = 1.0f / z;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e)
-          if (e < E) { P[e] = P[e] * inv; psum[e] += P[e]; }
-        if (a.P) {
-          float* prow = a.P + (size_t)tok * E;
-#pragma unroll
-          for (int e = 0; e < EMAX; ++e)
-            if (e < E) prow[e] = P[e];
-        } else {
-          uint32_t taken = 0;
-          for (int k = 0; k < a.K; ++k) {
-            float bp = -1.f;
-            int bi = -1;
-#pragma unroll
-            for (int e = 0; e < EMAX; ++e)
-              if (e < E && !((taken >> e) & 1u) && P[e] > bp) { bp = P[e]; bi = e; }
-            if (bi >= 0) { taken |= 1u << bi; atomicAdd(&cnt_s[bi], 1); }
-            a.topk_idx[(size_t)tok * a.K + k] = bi;
-            a.topk_w[(size_t)tok * a.K + k] = bi >= 0 ? bp : 0.f;
-          }
-          if (a.n_sel) a.n_sel[tok] = a.K;
-        }
-      }
-      // ---- fixed-order reduction of the score sums: lanes, then warps
-      const int w = tid >> 5;
-#pragma unroll
-      for (int e = 0; e < EMAX; ++e) {
-        if (e < E) {
-          float v = psum[e];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-          if ((tid & 31) == 0) wsum_s[w * EMAX + e] = v;
-        }
-      }
-      __syncthreads();
-      if (tid < E) {
-        const float v = ((wsum_s[tid] + wsum_s[EMAX + tid]) + wsum_s[2 * EMAX + tid]) + wsum_s[3 * EMAX + tid];
-        a.tile_psum[(size_t)tile * E + tid] = v;
-        if (!a.P) a.tile_counts[(size_t)tile * E + tid] = cnt_s[tid];
-      }
-      __syncthreads();
+      const int tok0 = tile * a.tile_rows + r0, tok1 = tile * a.tile_rows + r1;
+      if (has0 && tok0 < a.T) token_select<EMAX>(acc0, tok0, a, cnt_s, psum);
+      if (has1 && tok1 < a.T) token_select<EMAX>(acc1, tok1, a, cnt_s, psum);
+      tile_partials<EMAX>(psum, tile, a, cnt_s, wsum_s);
     }
+  }
+  if (fin.counts != nullptr && last_block_done(fin.ctr)) finalize_counts_loss(fin, xs);
+}
+
+void route_plan(int T, int D, int E, int bf16, int sms, int* tile_rows, int* threads) {
+  if (bf16) {
+    *tile_rows = kMmaRB;
+    *threads = mma_layout(D, E).warps * 32;
+  } else {
+    int tile = (T + sms - 1) / sms;
+    tile = (tile + 31) / 32 * 32;
+    tile = tile < 32 ? 32 : (tile > 256 ? 256 : tile);
+    while (tile > 32 && route_smem_bytes(D, E, tile, 0) > 232448) tile -= 32;
+    *tile_rows = tile;
+    *threads = kRouteThreads;
   }
 }
 
-template <typename T>
-static cudaError_t launch_route_t(const RouteArgs& a, const CUtensorMap* tm, cudaStream_t s) {
-  const size_t smem = route_smem_bytes(a.D, a.E, a.tile_rows, a.bf16);
+size_t route_smem_total(int D, int E, int tile_rows, int bf16) {
+  return bf16 ? mma_layout(D, E).total : route_smem_bytes(D, E, tile_rows, 0);
+}
+
+int route_mma_stages(int D, int E) { return mma_layout(D, E).warps; }
+
+cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tm, cudaStream_t s) {
+  const size_t smem = route_smem_total(a.D, a.E, a.tile_rows, a.bf16);
   cudaError_t err;
-#define MOE_ROUTE_CASE(EM)                                                                     \
-  if (a.E <= EM) {                                                                             \
-    err = cudaFuncSetAttribute(route_kernel<T, EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                               (int)smem);                                                     \
-    if (err != cudaSuccess) return err;                                                        \
-    route_kernel<T, EM><<<a.grid, kRouteThreads, smem, s>>>(*tm, a);                           \
-    return cudaGetLastError();                                                                 \
+  if (a.bf16) {
+#define MOE_ROUTE_MMA(EM)                                                                               \
+  if (a.E <= EM) {                                                                                      \
+    err = cudaFuncSetAttribute(route_kernel_mma<EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    if (err != cudaSuccess) return err;                                                                 \
+    route_kernel_mma<EM><<<a.grid, mma_layout(a.D, a.E).warps * 32, smem, s>>>(*tm, a, fin);          \
+    return cudaGetLastError();                                                                          \
   }
-  MOE_ROUTE_CASE(8)
-  MOE_ROUTE_CASE(16)
-  MOE_ROUTE_CASE(32)
-#undef MOE_ROUTE_CASE
+    MOE_ROUTE_MMA(8)
+    MOE_ROUTE_MMA(16)
+    MOE_ROUTE_MMA(32)
+#undef MOE_ROUTE_MMA
+  } else {
+#define MOE_ROUTE_FFMA(EM)                                                                              \
+  if (a.E <= EM) {                                                                                      \
+    err = cudaFuncSetAttribute(route_kernel_ffma<EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+    if (err != cudaSuccess) return err;                                                                 \
+    route_kernel_ffma<EM><<<a.grid, kRouteThreads, smem, s>>>(*tm, a, fin);                             \
+    return cudaGetLastError();                                                                          \
+  }
+    MOE_ROUTE_FFMA(8)
+    MOE_ROUTE_FFMA(16)
+    MOE_ROUTE_FFMA(32)
+#undef MOE_ROUTE_FFMA
+  }
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_route(const RouteArgs& a, const CUtensorMap* tm, cudaStream_t s) {
-  return a.bf16 ? launch_route_t<__nv_bfloat16>(a, tm, s) : launch_route_t<float>(a, tm, s);
-}
-
-// ---------------------------------------------------------------- finalize
-// counts_i = sum over tiles; p_i = (1/T) sum over tiles (fp64, fixed order);
-// L = alpha * sum_i (E/(K T)) counts_i p_i.
-__global__ void __launch_bounds__(256) route_finalize_kernel(FinalizeArgs a) {
-  __shared__ double red[256];
-  __shared__ double loss_terms[32];
-  const int tid = threadIdx.x;
-  for (int e = 0; e < a.E; ++e) {
-    long long c = 0;
-    double p = 0.0;
-    for (int t = tid; t < a.ntiles_counts; t += 256) c += a.tile_counts[(size_t)t * a.E + e];
-    for (int t = tid; t < a.ntiles_psum; t += 256) p += (double)a.tile_psum[(size_t)t * a.E + e];
-    red[tid] = (double)c;
-    __syncthreads();
-    for (int o = 128; o > 0; o >>= 1) {
-      if (tid < o) red[tid] += red[tid + o];
-      __syncthreads();
-    }
-    const double cnt = red[0];
-    __syncthreads();
-    red[tid] = p;
-    __syncthreads();
-    for (int o = 128; o > 0; o >>= 1) {
-      if (tid < o) red[tid] += red[tid + o];
-      __syncthreads();
-    }
-    if (tid == 0) {
-      a.counts[e] = (int32_t)cnt;
-      loss_terms[e] = ((double)a.E / ((double)a.K * a.T)) * cnt * (red[0] / a.T);
-    }
-    __syncthreads();
-  }
-  if (tid == 0) {
-    double L = 0.0;
-    for (int e = 0; e < a.E; ++e) L += loss_terms[e];
-    *a.aux_loss = (float)(a.alpha * L);
-  }
+// ---------------------------------------------------------------- finalize (race path)
+__global__ void __launch_bounds__(1024) route_finalize_kernel(FinalizeArgs a) {
+  __shared__ __align__(16) uint8_t scratch[kFinalizeScratch];
+  finalize_counts_loss(a, scratch);
 }
 
 cudaError_t launch_route_finalize(const FinalizeArgs& a, cudaStream_t s) {
-  route_finalize_kernel<<<1, 256, 0, s>>>(a);
+  route_finalize_kernel<<<1, 1024, 0, s>>>(a);
   return cudaGetLastError();
 }
 

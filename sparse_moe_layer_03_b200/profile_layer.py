@@ -1,0 +1,41 @@
+"""Run the layer a few times on one workload, for profilers (ncu) to capture.
+
+    python -m sparse_moe_layer_03_b200.profile_layer --workload xl2_8e2a_512 [--tokens T] [--iters N]
+
+No timing and no checking: the seeded inputs of the workload (optionally cut
+to T tokens) go through N forward passes on cuda:0.  Each pass launches the
+layer's kernels in order: route (+ finalize; Expert-Race adds its select
+kernels), dispatch count, dispatch gather, GEMM1, GEMM2, combine.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import inputs as I
+from .layer import LayerShape, MoELayer
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="xl2_8e2a_512", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0, help="cut the workload to this many tokens")
+    ap.add_argument("--iters", type=int, default=2)
+    a = ap.parse_args(argv)
+    w = I.WORKLOADS[a.workload]
+    if a.tokens:
+        w = w.with_tokens(a.tokens)
+    inp = I.make_inputs(w)
+    shape = LayerShape(w.T, w.D, w.H, w.E, w.K, w.n_shared, w.dtype, w.routing, w.alpha)
+    L = MoELayer(shape, inp, "cuda:0")
+    x = torch.as_tensor(inp["x"]).to("cuda:0", L.act_dtype)
+    for _ in range(a.iters):
+        L.forward(x)
+    torch.cuda.synchronize()
+    L.check()
+    print(f"{w.name}: T={w.T} ran {a.iters} forward passes")
+
+
+if __name__ == "__main__":
+    main()

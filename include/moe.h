@@ -69,7 +69,11 @@ typedef enum {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
 typedef enum { MOE_ROUTE_TOPK = 0, MOE_ROUTE_RACE = 1 } moe_routing_t;
-typedef enum { MOE_GEMM_AUTO = 0, MOE_GEMM_SIMT = 1 } moe_gemm_impl_t;
+typedef enum {
+  MOE_GEMM_AUTO = 0, /* bf16: tcgen05 on CTA pairs (256-row tiles); fp32: FFMA */
+  MOE_GEMM_SIMT = 1, /* FFMA for both dtypes (second implementation, for checks) */
+  MOE_GEMM_TC1 = 2   /* bf16: tcgen05 on single CTAs (128-row tiles) */
+} moe_gemm_impl_t;
 
 typedef struct {
   int32_t T;         /* tokens in this call (batch x patch tokens), >= 0 */
@@ -82,7 +86,7 @@ typedef struct {
   int32_t routing;   /* moe_routing_t */
   float alpha;       /* balance-loss factor (aux_loss_alpha) */
   int32_t act;       /* 0 = gelu tanh form (DiT core), 1 = exact erf form */
-  int32_t gemm_impl; /* moe_gemm_impl_t: AUTO = tcgen05 for bf16, FFMA for fp32 */
+  int32_t gemm_impl; /* moe_gemm_impl_t */
   int32_t reserved;  /* must be 0 */
 } moe_config_t;
 
@@ -96,8 +100,8 @@ const char* moe_last_error(void);
 size_t moe_workspace_size(const moe_config_t* cfg);
 
 /* Row capacity R_max of the expert-contiguous buffers x_perm, h_perm, y_perm,
- * row_token, row_gate: each expert segment starts on a 128-row boundary, so
- * R_max = round_up(K*T + 127*E, 128).  Host only. */
+ * row_token, row_gate: each expert segment starts on a 256-row boundary, so
+ * R_max = round_up(K*T + 255*E, 256).  Host only. */
 int64_t moe_max_rows(const moe_config_t* cfg);
 
 /* Zero the status word of `ws` (asynchronous on `stream`). */
@@ -133,7 +137,7 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
 /*
  * moe_dispatch -- permute tokens into expert-contiguous order (only the
  * selected experts are computed, "MOE 回顾").  Expert i's rows occupy
- * [P_i, P_i + counts_i) with P_i = sum_{j<i} round_up(counts_j, 128); tokens
+ * [P_i, P_i + counts_i) with P_i = sum_{j<i} round_up(counts_j, 256); tokens
  * ascend inside a segment.  Deterministic (no order-dependent atomics).
  *   x          [T,D] act          tokens
  *   topk_idx   [T,Kmax] int32     from moe_route (-1 = unused slot)
@@ -157,8 +161,9 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx
  *   h_sh[t]   = gelu(W1s x[t] + b1s)  (all n_s shared experts side by side)
  *   offsets [E+1] int32 (moe_dispatch output); b1 [E,H] / b1s [n_s,H] may be NULL;
  *   h_perm [R_max,H] act out; h_sh [T,n_s*H] act out (NULL when n_s = 0).
- * bf16: one persistent tcgen05 kernel (TMA-fed, TMEM accumulators) runs the
- * routed segments and the shared block together.  fp32: FFMA kernel.
+ * bf16: one persistent tcgen05 kernel (TMA-fed, TMEM accumulators, 256-row
+ * tiles on CTA pairs) runs the routed segments and the shared block together.
+ * fp32: FFMA kernel.
  */
 int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
                      const void* x, const void* w1, const void* b1, const void* w1s, const void* b1s,

@@ -19,7 +19,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, -1, -2,
 MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT = -4, -5, -6
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ROUTE_TOPK, MOE_ROUTE_RACE = 0, 1
-MOE_GEMM_AUTO, MOE_GEMM_SIMT = 0, 1
+MOE_GEMM_AUTO, MOE_GEMM_SIMT, MOE_GEMM_TC1 = 0, 1, 2
 
 
 class MoeConfig(C.Structure):
@@ -86,7 +86,8 @@ def make_config(T, D, H, E, K, n_shared, dtype="bf16", routing="topk", alpha=0.0
                 gemm_impl="auto") -> MoeConfig:
     return MoeConfig(T, D, H, E, K, n_shared, MOE_BF16 if dtype == "bf16" else MOE_F32,
                      MOE_ROUTE_RACE if routing == "race" else MOE_ROUTE_TOPK, alpha,
-                     1 if act == "erf" else 0, MOE_GEMM_SIMT if gemm_impl == "simt" else MOE_GEMM_AUTO, 0)
+                     1 if act == "erf" else 0,
+                     {"auto": MOE_GEMM_AUTO, "simt": MOE_GEMM_SIMT, "tc1": MOE_GEMM_TC1}[gemm_impl], 0)
 
 
 def moe_version() -> int:

@@ -58,7 +58,7 @@ int validate(const moe_config_t* c) {
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype=%d", c->dtype);
   if (c->routing != MOE_ROUTE_TOPK && c->routing != MOE_ROUTE_RACE) return fail(MOE_ERR_INVALID_ARG, "routing=%d", c->routing);
   if (c->act != 0 && c->act != 1) return fail(MOE_ERR_INVALID_ARG, "act=%d", c->act);
-  if (c->gemm_impl != MOE_GEMM_AUTO && c->gemm_impl != MOE_GEMM_SIMT) return fail(MOE_ERR_INVALID_ARG, "gemm_impl=%d", c->gemm_impl);
+  if (c->gemm_impl < MOE_GEMM_AUTO || c->gemm_impl > MOE_GEMM_TC1) return fail(MOE_ERR_INVALID_ARG, "gemm_impl=%d", c->gemm_impl);
   if (c->reserved != 0) return fail(MOE_ERR_INVALID_ARG, "reserved field must be 0");
   if (route_smem_total(c->D, c->E, 32, c->dtype == MOE_BF16) > 232448 ||
       (c->dtype == MOE_BF16 && route_mma_stages(c->D, c->E) < 2))
@@ -70,7 +70,7 @@ int kmax_of(const moe_config_t* c) { return c->routing == MOE_ROUTE_RACE ? c->E 
 
 long long max_rows(const moe_config_t* c) {
   const long long S = (long long)c->K * c->T;
-  return (long long)round_up((size_t)(S + 127ll * c->E), 128);
+  return (long long)round_up((size_t)(S + (long long)(kSegAlign - 1) * c->E), kSegAlign);
 }
 
 // dispatch chunking: at most 1024 chunks of >= 64 tokens (a multiple of 32)
@@ -344,23 +344,41 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
              int K1, int bcols1, void* ws, cudaStream_t s) {
   (void)ws;
   cudaError_t e;
-  const bool tc = cfg->dtype == MOE_BF16 && cfg->gemm_impl == MOE_GEMM_AUTO;
+  const bool tc = cfg->dtype == MOE_BF16 && cfg->gemm_impl != MOE_GEMM_SIMT;
   if (!tc) {
     if ((e = launch_gemm_simt(g, s)) != cudaSuccess) return cuda_fail(e, "FFMA expert GEMM");
     return ok();
   }
-  const int bn = gemm_tc_pick_bn(g.p[0].N, g.nprob > 1 ? g.p[1].N : 0);
+  const bool pair = cfg->gemm_impl == MOE_GEMM_AUTO;     // 2-SM tiles unless the 1-SM kernel is asked for
+  const int n1 = g.nprob > 1 ? g.p[1].N : 0;
+  const int bn = pair ? gemm_pair_pick_bn(g.p[0].N, n1) : gemm_tc_pick_bn(g.p[0].N, n1);
   if (!bn) return fail(MOE_ERR_UNSUPPORTED, "no tile width divides N=%d", g.p[0].N);
+  // boxes: A rows per CTA = 128; B rows per CTA = bn (1 SM) or bn/2 (2 SMs)
+  const int brows_box = pair ? bn / 2 : bn;
   CUtensorMap ta[2], tb[2];
   int rc;
   if ((rc = make_tmap(&ta[0], A0, true, rows0, K0, 128, "A0"))) return rc;
-  if ((rc = make_tmap(&tb[0], B0, true, brows0, K0, bn, "B0"))) return rc;
+  if ((rc = make_tmap(&tb[0], B0, true, brows0, K0, brows_box, "B0"))) return rc;
   if (g.nprob > 1) {
     if ((rc = make_tmap(&ta[1], A1, true, rows1, K1, 128, "A1"))) return rc;
-    if ((rc = make_tmap(&tb[1], B1, true, brows1, bcols1, bn, "B1"))) return rc;
+    if ((rc = make_tmap(&tb[1], B1, true, brows1, bcols1, brows_box, "B1"))) return rc;
   } else {
     ta[1] = ta[0];
     tb[1] = tb[0];
+  }
+  if (pair) {
+    // output boxes for the TMA-store epilogue: 32 rows x 128 bytes (bf16 h or fp32 y)
+    CUtensorMap to[2];
+    const bool out_bf16 = g.p[0].epi == 0;
+    if ((rc = make_tmap(&to[0], g.p[0].out, out_bf16, rows0, g.p[0].N, 32, "out0"))) return rc;
+    if (g.nprob > 1) {
+      if ((rc = make_tmap(&to[1], g.p[1].out, out_bf16, rows1, g.p[1].N, 32, "out1"))) return rc;
+    } else {
+      to[1] = to[0];
+    }
+    if ((e = launch_gemm_pair(g, ta, tb, to, bn, num_sms_current(), s)) != cudaSuccess)
+      return cuda_fail(e, "tcgen05 CTA-pair expert GEMM");
+    return ok();
   }
   if ((e = launch_gemm_tc(g, ta, tb, bn, num_sms_current(), s)) != cudaSuccess) return cuda_fail(e, "tcgen05 expert GEMM");
   return ok();

@@ -3,7 +3,7 @@
 // Parameters", "MOE 回顾": with a sparse g, unused experts need not be run).
 //
 // Layout: expert i owns rows [P_i, P_i + counts_i), P_i = sum_{j<i}
-// round_up(counts_j, 128), tokens ascending inside a segment.  Positions come
+// round_up(counts_j, 256), tokens ascending inside a segment.  Positions come
 // from integer counts and prefix sums only (no order-dependent atomics), so
 // the permutation is deterministic and equals the canonical one bit for bit.
 //
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kGatherThreads) dispatch_gather_kernel(Dispatc
   __syncthreads();
   if (tid == 0) {
     int p = 0;
-    for (int e = 0; e < E; ++e) { poff_s[e] = p; p += (total_s[e] + 127) / 128 * 128; }
+    for (int e = 0; e < E; ++e) { poff_s[e] = p; p += (total_s[e] + kSegAlign - 1) / kSegAlign * kSegAlign; }
     poff_s[E] = p;
   }
   __syncthreads();

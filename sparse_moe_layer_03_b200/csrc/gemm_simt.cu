@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
         int c = a.offsets[e + 1] - a.offsets[e];
         if (c < 0) { c = 0; bad = 1; }
         cnt[e] = c;
-        p += (c + 127) / 128 * 128;
+        p += (c + kSegAlign - 1) / kSegAlign * kSegAlign;
         poff[e + 1] = p;
       }
       if ((long long)p > a.r_max) bad = 1;

@@ -117,7 +117,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ 
       int c = a.offsets ? a.offsets[e + 1] - a.offsets[e] : 0;
       if (c < 0) { c = 0; bad = true; }
       pl.cnt[e] = c;
-      p += (c + kBM - 1) / kBM * kBM;
+      p += (c + kSegAlign - 1) / kSegAlign * kSegAlign;
       pl.poff[e + 1] = p;
     }
     if ((long long)p > a.r_max) { bad = true; }

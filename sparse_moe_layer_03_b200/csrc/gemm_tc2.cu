@@ -1,0 +1,379 @@
+// Grouped expert GEMM on CTA pairs: tcgen05.mma.cta_group::2 (sm_100a).
+//
+// The same problems and epilogues as the single-CTA kernel (expert MLP =
+// W2 gelu(W1 x), "Scaling Diffusion Transformers to 16 Billion Parameters",
+// "MOE-DIT" eq. MLP), but every output tile is 256 x BN and belongs to a pair
+// of CTAs on the two SMs of a TPC (a cluster of 2).  Each CTA loads its own
+// 128 rows of A and its own BN/2 rows of B, so per FLOP each SM pulls 2/3 of
+// the operand bytes of a 128 x 256 single-CTA tile; the pair's tensor cores
+// read the peer's half through the CTA pair, and each CTA's TMEM receives its
+// 128 rows of the 256 x BN accumulator.  No TMA load uses cluster multicast.
+//
+// Roles per CTA (6 warps): warp 0 = TMA producer (both CTAs; loads complete on
+// the leader's barrier); warp 1 = TMEM allocation (both) and the MMA issuer
+// (leader only); warps 2-5 = epilogue (both CTAs, one per TMEM lane quadrant),
+// storing through TMA.  (More epilogue warps measured slower: the GEMMs run
+// at the power cap, where extra epilogue activity costs clock.)
+// Synchronisation: the leader's MMA thread commits MMA completion to the
+// "stage empty" and "accumulator full" barriers of both CTAs (one commit per
+// CTA, by shared::cluster address); every epilogue warp of both CTAs arrives
+// on the leader's "accumulator empty" barrier; both CTAs' TMA loads complete
+// on the leader's "stage full" barrier.  All waits are bounded.
+#include <cuda.h>
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kPairBM = 256;            // rows of a pair tile (128 per CTA)
+constexpr int kPairBK = 64;             // bf16 elements per 128-byte swizzle row
+constexpr int kPairEpiWarps = 4;          // one per TMEM lane quadrant
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
+constexpr int kPairSmemLimit = 232448;
+
+template <int BN>
+struct PairCfg {
+  static constexpr int A_BYTES = 128 * kPairBK * 2;
+  static constexpr int B_BYTES = (BN / 2) * kPairBK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  // epilogue staging: two 32 rows x 128 bytes buffers per epilogue warp for TMA stores
+  static constexpr int EPI_BYTES = kPairEpiWarps * 2 * 4096;
+  // keep 4 KB of the 227 KB for barriers, the 1 KB alignment slack and static shared memory
+  static constexpr int FIT = (kPairSmemLimit - 4096 - EPI_BYTES) / STAGE;
+  static constexpr int STAGES = FIT > 8 ? 8 : FIT;
+  static constexpr int SMEM = STAGES * STAGE + EPI_BYTES + 2048;
+  static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+};
+
+struct PairPlan {
+  int poff[33];
+  int cnt[32];
+  int ntiles[2];
+  int nn[2];
+  int total;
+};
+
+struct PairTile {
+  int p, row0, valid, brow, n0, e, nk;
+};
+
+template <int BN>
+__device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, const GemmArgs& a) {
+  PairTile ti;
+  int t = tile;
+  ti.p = 0;
+  if (t >= pl.ntiles[0]) { t -= pl.ntiles[0]; ti.p = 1; }
+  const GemmProblem& pr = a.p[ti.p];
+  const int mt = t / pl.nn[ti.p], nt = t % pl.nn[ti.p];
+  ti.row0 = mt * kPairBM;
+  ti.n0 = nt * BN;
+  ti.nk = pr.K / kPairBK;
+  if (pr.routed) {
+    int e = 0;
+    while (e < a.E - 1 && ti.row0 >= pl.poff[e + 1]) ++e;
+    ti.e = e;
+    const int v = pl.poff[e] + pl.cnt[e] - ti.row0;
+    ti.valid = v < kPairBM ? v : kPairBM;
+    ti.brow = e * pr.N + ti.n0;
+  } else {
+    ti.e = 0;
+    const int v = pr.M - ti.row0;
+    ti.valid = v < kPairBM ? v : kPairBM;
+    ti.brow = ti.n0;
+  }
+  return ti;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kPairThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
+                 const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
+                 const __grid_constant__ CUtensorMap to0, const __grid_constant__ CUtensorMap to1, GemmArgs a) {
+  using C = PairCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* stage_base = smem;
+  uint8_t* epi_base = smem + C::STAGES * C::STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_base + C::EPI_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ PairPlan pl;
+
+  const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();          // 0 = leader of the pair
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);             // leader: its producer's expect_tx arrive
+      mbar_init(smem_u32(&empty[s]), 1);            // one MMA-completion commit per phase
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&acc_full[i]), 1);
+      mbar_init(smem_u32(&acc_empty[i]), 2 * kPairEpiWarps);   // leader: every epilogue warp of both CTAs
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    bool bad = false;
+    int p = 0;
+    pl.poff[0] = 0;
+    for (int e = 0; e < a.E; ++e) {
+      int c = a.offsets ? a.offsets[e + 1] - a.offsets[e] : 0;
+      if (c < 0) { c = 0; bad = true; }
+      pl.cnt[e] = c;
+      p += (c + kSegAlign - 1) / kSegAlign * kSegAlign;
+      pl.poff[e + 1] = p;
+    }
+    if ((long long)p > a.r_max) bad = true;
+    for (int q = 0; q < 2; ++q) {
+      if (q >= a.nprob) { pl.ntiles[q] = 0; pl.nn[q] = 1; continue; }
+      const GemmProblem& pr = a.p[q];
+      pl.nn[q] = pr.N / BN;
+      const int mt = pr.routed ? (bad ? 0 : p / kPairBM) : (pr.M + kPairBM - 1) / kPairBM;
+      pl.ntiles[q] = mt * pl.nn[q];
+    }
+    pl.total = pl.ntiles[0] + pl.ntiles[1];
+    if (bad && rank == 0 && cid == 0) set_status(a.status, DEV_BAD_INDEX, 500);
+    prefetch_tmap(&ta0);
+    prefetch_tmap(&tb0);
+    prefetch_tmap(&ta1);
+    prefetch_tmap(&tb1);
+    prefetch_tmap(&to0);
+    prefetch_tmap(&to1);
+  }
+  if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                   // both CTAs' barriers exist before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t idesc = idesc_bf16_f32(kPairBM, BN);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_last();
+      const uint64_t pol_a = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = cid; tile < pl.total; tile += ncl) {
+        const PairTile ti = pair_decode<BN>(tile, pl, a);
+        const CUtensorMap* tA = ti.p ? &ta1 : &ta0;
+        const CUtensorMap* tB = ti.p ? &tb1 : &tb0;
+        const int ksplit = a.p[ti.p].ksplit;
+        const int nrows = a.p[ti.p].N;
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.status, 501)) goto done;
+          const uint32_t fb_local = smem_u32(&full[stage]);
+          const uint32_t fb_leader = map_to_cta(fb_local, 0);
+          if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::STAGE);   // both CTAs' bytes
+          uint8_t* sa = stage_base + stage * C::STAGE;
+          const int bx = ksplit ? (kb * kPairBK) % ksplit : kb * kPairBK;
+          const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (BN / 2);
+          tma_load_2d_pair(smem_u32(sa), tA, kb * kPairBK, ti.row0 + (int)rank * 128, fb_leader, pol_a);
+          tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tB, bx, by, fb_leader, pol_w);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool issued_any = false;
+      for (int tile = cid; tile < pl.total; tile += ncl, ++local) {
+        const PairTile ti = pair_decode<BN>(tile, pl, a);
+        const int acc = local & 1;
+        const uint32_t accph = (local >> 1) & 1;
+        if (!mbar_wait(smem_u32(&acc_empty[acc]), accph ^ 1u, abort_flag, a.status, 502)) goto mma_out;
+        tc_fence_after();
+        const uint32_t d = tmem_base + acc * BN;
+        for (int kb = 0; kb < ti.nk; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)) goto mma_out;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * C::STAGE);
+          const uint64_t adesc = smem_desc_sw128(sa);
+          const uint64_t bdesc = smem_desc_sw128(sa + C::A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kPairBK / 16; ++kk)
+            umma_bf16_pair(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+          issued_any = true;
+          // stage free in both CTAs once these MMAs finish
+          const uint32_t eb = smem_u32(&empty[stage]);
+          umma_commit_pair(eb);
+          umma_commit_pair(map_to_cta(eb, 1));
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        const uint32_t fb = smem_u32(&acc_full[acc]);   // accumulator ready in both CTAs
+        umma_commit_pair(fb);
+        umma_commit_pair(map_to_cta(fb, 1));
+      }
+    mma_out:
+      if (issued_any) {
+        umma_commit_pair(smem_u32(drain));
+        mbar_wait(smem_u32(drain), 0, nullptr, a.status, 504);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    // Each warp owns 32 TMEM lanes = 32 rows of this CTA's half.  Per 128-byte
+    // column box it loads the accumulator, applies the epilogue, writes the
+    // 32 x 128-byte box into a swizzled shared buffer and hands it to a TMA
+    // store (two buffers per warp, so a store overlaps the next box).
+    const int q = warp & 3;
+    const int r = q * 32 + lane;                   // row inside this CTA's 128-row half
+    const uint32_t acc_empty_leader0 = map_to_cta(smem_u32(&acc_empty[0]), 0);
+    const uint32_t acc_empty_leader1 = map_to_cta(smem_u32(&acc_empty[1]), 0);
+    const uint32_t sbuf = smem_u32(epi_base + (warp - 2) * 8192);
+    int nstore = 0;
+    int local = 0;
+    for (int tile = cid; tile < pl.total; tile += ncl, ++local) {
+      const PairTile ti = pair_decode<BN>(tile, pl, a);
+      const GemmProblem& pr = a.p[ti.p];
+      const CUtensorMap* tO = ti.p ? &to1 : &to0;
+      const int acc = local & 1;
+      const uint32_t accph = (local >> 1) & 1;
+      if (!mbar_wait(smem_u32(&acc_full[acc]), accph, abort_flag, a.status, 505)) break;
+      tc_fence_after();
+      const int valid_here = ti.valid - (int)rank * 128;
+      const bool rv = r < valid_here;
+      const long long grow = (long long)ti.row0 + (int)rank * 128 + r;
+      const int box_row = ti.row0 + (int)rank * 128 + q * 32;
+      const float gate = (pr.gate != nullptr && rv) ? pr.gate[grow] : 1.0f;
+      const __nv_bfloat16* bias =
+          pr.bias ? reinterpret_cast<const __nv_bfloat16*>(pr.bias) + (long long)ti.e * pr.bias_stride : nullptr;
+      const int box_cols = pr.epi == 0 ? 64 : 32;          // 128 bytes of bf16 or fp32
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += box_cols) {
+        uint4 o[8];
+        uint32_t vv[2][32];
+        tmem_ld_32x32b_x32(tbase + c0, vv[0]);
+        if (box_cols == 64) tmem_ld_32x32b_x32(tbase + c0 + 32, vv[1]);
+        tmem_ld_wait();                              // both halves in flight before one wait
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (half * 32 >= box_cols) break;
+          const int cc = c0 + half * 32;
+          const uint32_t* v = vv[half];
+          const int col0 = ti.n0 + cc;
+          float b[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) b[j] = 0.f;
+          if (bias) {
+            for (int br = 0; br < pr.bias_rows; ++br) {
+              const uint4* bp = reinterpret_cast<const uint4*>(bias + (long long)br * pr.N + col0);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                float t8[8];
+                bf16x8_to_f32(__ldg(bp + u), t8);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) b[8 * u + j] += t8[j];
+              }
+            }
+          }
+          if (pr.epi == 0) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint32_t* ow = reinterpret_cast<uint32_t*>(&o[half * 4 + u]);
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const int j = 8 * u + 2 * h;
+                ow[h] = pack_bf16x2(gelu_act<true>(__uint_as_float(v[j]) + b[j], a.act),
+                                    gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], a.act));
+              }
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int j = 4 * u;
+              float4 f = make_float4((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate,
+                                     (__uint_as_float(v[j + 2]) + b[j + 2]) * gate,
+                                     (__uint_as_float(v[j + 3]) + b[j + 3]) * gate);
+              o[u] = *reinterpret_cast<uint4*>(&f);
+            }
+          }
+        }
+        // stage the 32 x 128-byte box (128-byte swizzle) and store it with TMA; rows past the
+        // segment's tokens are padding rows of the permuted buffers (or clipped past T)
+        const uint32_t buf = sbuf + (nstore & 1) * 4096;
+        if (lane == 0) bulk_wait_read_le1();   // the store that last used this buffer has read it
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + lane * 128 + ((j ^ (lane & 7)) << 4)),
+                       "r"(o[j].x), "r"(o[j].y), "r"(o[j].z), "r"(o[j].w)
+                       : "memory");
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tO, buf, ti.n0 + c0, box_row);
+          bulk_commit();
+        }
+        ++nstore;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
+    }
+    if (lane == 0) bulk_wait_all();            // stores done before the CTA may exit
+  }
+done:
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                   // no CTA leaves while its peer may still use it
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+}
+
+template <int BN>
+static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb,
+                                  const CUtensorMap* to, int grid, cudaStream_t s) {
+  using C = PairCfg<BN>;
+  cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN>, ta[0], tb[0], ta[1], tb[1], to[0], to[1], a);
+}
+
+int gemm_pair_pick_bn(int n0, int n1) {
+  const int cands[4] = {256, 192, 128, 64};
+  for (int i = 0; i < 4; ++i) {
+    const int bn = cands[i];
+    if (n0 % bn == 0 && (n1 == 0 || n1 % bn == 0)) return bn;
+  }
+  return 0;
+}
+
+cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, const CUtensorMap* to,
+                             int bn, int num_sms, cudaStream_t s) {
+  const int grid = num_sms & ~1;
+  switch (bn) {
+    case 256: return launch_pair_bn<256>(a, ta, tb, to, grid, s);
+    case 192: return launch_pair_bn<192>(a, ta, tb, to, grid, s);
+    case 128: return launch_pair_bn<128>(a, ta, tb, to, grid, s);
+    case 64: return launch_pair_bn<64>(a, ta, tb, to, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace moe

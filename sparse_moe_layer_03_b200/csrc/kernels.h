@@ -6,6 +6,9 @@
 
 namespace moe {
 
+// every expert segment of the permuted buffers starts on a multiple of this many rows
+constexpr int kSegAlign = 256;
+
 // ---- route.cu
 struct RouteArgs {
   const void* x;            // [T,D] act
@@ -92,6 +95,9 @@ struct GemmArgs {
 cudaError_t launch_gemm_tc(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, int bn,
                            int num_sms, cudaStream_t s);
 int gemm_tc_pick_bn(int n0, int n1);
+cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, const CUtensorMap* to,
+                             int bn, int num_sms, cudaStream_t s);
+int gemm_pair_pick_bn(int n0, int n1);
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t s);
 
 // ---- combine.cu

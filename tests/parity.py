@@ -20,6 +20,7 @@ from oracle import moe_oracle as O
 from sparse_moe_layer_03_b200.inputs import Workload
 
 TIE = 1e-4
+SEG_ALIGN = 256      # expert segments of the permuted buffers start on multiples of this
 
 
 def out_tol(w: Workload) -> float:
@@ -120,7 +121,7 @@ def gpu_selection(r: dict) -> np.ndarray:
 
 def check_permutation(w: Workload, L, r: dict, x_dev: torch.Tensor, rows_to_check: int = 4096):
     idx = gpu_selection(r)
-    cp = O.canonical_permutation(idx, w.E)
+    cp = O.canonical_permutation(idx, w.E, tile=SEG_ALIGN)
     assert np.array_equal(r["offsets"].astype(np.int64), cp["offsets"])
     assert np.array_equal(r["pos"].astype(np.int64), cp["pos"])
     Rv = int(cp["padded_offsets"][-1])

@@ -23,7 +23,7 @@ def test_library_exports_every_declared_symbol():
 def test_version_and_sizes():
     assert B.moe_version() == 100
     cfg = B.make_config(32768, 1152, 4608, 8, 2, 2)
-    assert B.moe_max_rows(cfg) == 66560
+    assert B.moe_max_rows(cfg) == 67584     # round_up(65536 + 255*8, 256)
     assert B.moe_workspace_size(cfg) > 0
     race = B.make_config(32768, 1152, 4608, 16, 2, 1, routing="race")
     assert B.moe_workspace_size(race) > 32768 * 16 * 4

@@ -40,12 +40,21 @@ def test_small_layer_parity(case):
     assert rep["err"] <= PA.out_tol(w)
 
 
-def test_tensor_core_path_matches_ffma_path():
+@pytest.mark.parametrize("impl", ["auto", "tc1"])
+def test_tensor_core_paths_match_ffma_path(impl):
+    # auto = tcgen05 on CTA pairs (256-row tiles), tc1 = tcgen05 on single CTAs
     w, inp = _small(1000, 256, 512, 8, 2, 2, "bf16")
-    a = PA.full_check(w, inp, gemm_impl="auto")
+    a = PA.full_check(w, inp, gemm_impl=impl)
     b = PA.full_check(w, inp, gemm_impl="simt")
     # both against the oracle already; against each other: same rounding points
     assert PA.rel_err(a["res"]["out"], b["res"]["out"]) < 1e-2
+
+
+@pytest.mark.parametrize("impl", ["tc1", "simt"])
+def test_other_gemm_paths_full_size_xl(impl):
+    w = I.WORKLOADS["xl2_8e2a_512"]
+    inp = I.make_inputs(w)
+    PA.full_check(w, inp, gemm_impl=impl, tokens=PA.sample_tokens(w.T, 128))
 
 
 def test_erf_gelu_option():

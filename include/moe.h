@@ -197,6 +197,30 @@ int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* 
 int moe_combine(const moe_config_t* cfg, const float* y_perm, const float* y_sh,
                 const int32_t* pos, const int32_t* n_sel, void* out, void* stream);
 
+/*
+ * moe_route_static -- moe_route for callers that cannot allocate device memory.
+ * (No counterpart on the pages: this is a deployment convenience.)
+ *
+ * Same arguments, results and errors as moe_route, minus the workspace: the
+ * router's scratch comes from a fixed 4 MiB array built into the library
+ * (reserved on every GPU that loads it, until the process exits), so a caller
+ * whose framework gives it no allocator, or that must not call cudaMalloc
+ * after start-up, needs none.
+ *   - Configurations whose scratch (moe_workspace_size) exceeds 4 MiB are
+ *     rejected with MOE_ERR_WORKSPACE and a message; nothing is launched.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.  The call allocates nothing itself.
+ *   - All calls share the one array: calls that may overlap on the GPU (other
+ *     streams, other threads) race and must be serialised by the caller.  Each
+ *     call clears the array's status word and counters itself; device-detected
+ *     errors are not reported back (there is no workspace to pass to
+ *     moe_check_status).
+ */
+int moe_route_static(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
+                     int32_t* topk_idx, float* topk_w, int32_t* n_sel, int32_t* counts, float* aux_loss,
+                     void* stream);
+
 #ifdef __cplusplus
 }
 #endif

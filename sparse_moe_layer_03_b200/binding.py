@@ -56,6 +56,7 @@ _SIGS = {
     "moe_expert_mlp": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                  _P, C.c_size_t, _P]),
     "moe_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
+    "moe_route_static": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -152,3 +153,9 @@ def moe_combine(cfg, y_perm, y_sh, pos, n_sel, out, stream=0):
 
 def moe_last_error() -> str:
     return lib.moe_last_error().decode()
+
+
+def moe_route_static(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, aux_loss, stream=0):
+    """moe_route without a workspace: scratch comes from the library's built-in 4 MiB array."""
+    _check(lib.moe_route_static(C.byref(cfg), _ptr(x), _ptr(wg), _ptr(router_bias), _ptr(topk_idx), _ptr(topk_w),
+                                _ptr(n_sel), _ptr(counts), _ptr(aux_loss), stream))

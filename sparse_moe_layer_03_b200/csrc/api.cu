@@ -180,6 +180,8 @@ int make_tmap(CUtensorMap* m, const void* base, bool bf16, long long rows, long 
 
 }  // namespace
 
+void moe::set_last_error_message(const char* msg) { g_last_error = msg ? msg : ""; }
+
 // ====================================================================== ABI
 extern "C" {
 

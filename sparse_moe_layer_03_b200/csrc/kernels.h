@@ -6,6 +6,9 @@
 
 namespace moe {
 
+// message returned by moe_last_error() on this thread
+void set_last_error_message(const char* msg);
+
 // every expert segment of the permuted buffers starts on a multiple of this many rows
 constexpr int kSegAlign = 256;
 

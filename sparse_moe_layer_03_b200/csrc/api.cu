@@ -178,6 +178,23 @@ int make_tmap(CUtensorMap* m, const void* base, bool bf16, long long rows, long 
   return MOE_OK;
 }
 
+// x [rows, cols] bf16 seen as 3-D {64 columns, rows, cols/64 blocks}: one box brings
+// `box_rows` whole rows as cols/64 swizzled 128-byte blocks, block-major.  Returns
+// false when the driver does not accept the layout (the caller then uses 2-D boxes).
+bool make_tmap_rows3d(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)(rows > 0 ? rows : 1), (cuuint64_t)(cols / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)(cols / 64)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (cols / 64 > 256) return false;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 void moe::set_last_error_message(const char* msg) { g_last_error = msg ? msg : ""; }
@@ -255,8 +272,11 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   // partial sums: one row per CTA (bf16 kernel) or per token tile (fp32 kernel)
   const int nparts = bf16 ? grid : ntiles;
   CUtensorMap tm;
-  if ((rc = make_tmap(&tm, x, bf16, cfg->T, cfg->D, tile, "x"))) return rc;
+  int tmap3d = 0;
+  if (bf16 && make_tmap_rows3d(&tm, x, cfg->T, cfg->D, tile)) tmap3d = 1;
+  else if ((rc = make_tmap(&tm, x, bf16, cfg->T, cfg->D, tile, "x"))) return rc;
   RouteArgs ra{};
+  ra.tmap3d = tmap3d;
   ra.x = x; ra.wg = wg; ra.bias = router_bias;
   ra.T = cfg->T; ra.D = cfg->D; ra.E = cfg->E; ra.K = cfg->K; ra.bf16 = bf16;
   ra.tile_rows = tile; ra.ntiles = ntiles; ra.grid = grid;

@@ -19,6 +19,7 @@ struct RouteArgs {
   const float* bias;        // [E] or null
   int T, D, E, K, bf16;
   int tile_rows, ntiles, grid;
+  int tmap3d;               // bf16 router: 1 = one 3-D box {64, 16 rows, D/64} per unit, 0 = D/64 2-D boxes
   int32_t* topk_idx;        // top-K mode: [T,K]
   float* topk_w;
   int32_t* n_sel;           // may be null (top-K)

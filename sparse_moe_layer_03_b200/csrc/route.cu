@@ -122,13 +122,13 @@ __device__ __forceinline__ void tile_partials(const float* psum, int tile, const
 // ---------------------------------------------------------------- bf16: tensor-core logits
 // Work unit = a block of 16 consecutive tokens: their full rows (16 x D bf16,
 // one contiguous stretch of HBM, so DRAM pages are read whole) land in one
-// shared-memory buffer as D/64 TMA boxes of 16 rows x 128 bytes (128-byte
-// swizzle).  Every warp owns one buffer and runs its own pipeline over its
-// units with no block-wide barrier: wait for the rows, compute the 16 x E
-// logits with mma.sync m16n8k16 (A via ldmatrix from the swizzled buffer, B =
-// gate weight in shared memory with rows padded by 16 bytes), re-issue the
-// buffer for the next unit, then run softmax and selection (one lane per
-// token) while those rows load.
+// shared-memory stage as D/64 TMA boxes of 16 rows x 128 bytes (128-byte
+// swizzle).  One producer thread keeps a ring of stages in flight; four
+// consumer warps take units in turn: wait for the rows, compute the 16 x E
+// logits with mma.sync m16n8k16 (A via ldmatrix from the swizzled stage, B =
+// gate weight in shared memory with rows padded by 16 bytes), free the stage,
+// then run softmax and selection (one lane per token).  No block-wide barrier
+// inside the loop.
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
@@ -146,12 +146,17 @@ __device__ __forceinline__ void mma_16816(float* d, uint32_t a0, uint32_t a1, ui
 }
 
 constexpr int kMmaRB = 16;        // tokens per work unit
-constexpr int kMmaMaxWarps = 8;
+constexpr int kMmaConsumers = 4;  // consumer warps; warp 0 is the TMA producer
+// Consumer warp c owns stage c: it waits on that stage's phases strictly in order.
+// (Stages shared round-robin by several consumers would let a warp wait on a phase two
+// ahead of the barrier, where the parity test passes early.)
+constexpr int kMmaStages = kMmaConsumers;
+constexpr int kMmaMaxStages = kMmaStages;
 
-// One TMA buffer (16 full rows) per warp; as many warps as buffers fit.
+// A ring of stages (16 full rows each) fed by one producer thread.
 struct MmaSmem {
   size_t wg, x, logits, misc, total;
-  int warps;
+  int stages;
 };
 __host__ __device__ inline MmaSmem mma_layout(int D, int E) {
   MmaSmem L;
@@ -159,43 +164,63 @@ __host__ __device__ inline MmaSmem mma_layout(int D, int E) {
   L.wg = 0;
   L.x = align1k((size_t)em * (D * 2 + 16));
   const size_t stage = (size_t)kMmaRB * D * 2;
-  const size_t per_warp_logits = (size_t)kMmaRB * em * 4;
-  const size_t fixed = L.x + 2048 /*misc*/ + 1024 /*align slack*/ + 1024 /*scratch margin*/;
-  int nw = (int)((232448 - fixed) / (stage + per_warp_logits));
-  L.warps = nw > kMmaMaxWarps ? kMmaMaxWarps : nw;
-  const size_t xb = (size_t)(L.warps > 0 ? L.warps : 0) * stage;
-  L.logits = L.x + (xb > 16896 ? xb : 16896);   // x buffers double as the finalize scratch
-  L.misc = L.logits + (size_t)(L.warps > 0 ? L.warps : 0) * per_warp_logits;
+  const size_t logits = (size_t)kMmaConsumers * kMmaRB * em * 4;
+  const size_t fixed = L.x + logits + 2048 /*misc*/ + 1024 /*align slack*/ + 1024 /*scratch margin*/;
+  const int st = (int)((232448 - fixed) / stage);
+  L.stages = st >= kMmaStages ? kMmaStages : 0;   // 0: does not fit (rejected by validation)
+  const size_t xb = (size_t)(L.stages > 0 ? L.stages : 0) * stage;
+  L.logits = L.x + (xb > 16896 ? xb : 16896);   // x stages double as the finalize scratch
+  L.misc = L.logits + logits;
   L.total = L.misc + 2048 + 1024;
   return L;
 }
 
 // The last block to finish turns the per-block partials into counts and the loss.
-// scratch: 2 x 32 x 33 x 8 bytes of shared memory
-constexpr int kFinalizeScratch = 2 * 32 * 33 * 8;
+// Every thread loads its tiles' partials for all experts at once (no chain of
+// dependent loads), then fixed-order shuffle trees and a fixed warp order make
+// the result bit-reproducible.  scratch: 2 x 32 x 32 x 8 bytes of shared memory.
+constexpr int kFinalizeScratch = 2 * 32 * 32 * 8;
+template <int EMAX>
 __device__ void finalize_counts_loss(const FinalizeArgs& a, uint8_t* scratch) {
-  auto cs = reinterpret_cast<long long(*)[33]>(scratch);
-  auto ps = reinterpret_cast<double(*)[33]>(scratch + 32 * 33 * 8);
-  const int tid = threadIdx.x, e = tid & 31, g = tid >> 5, ng = blockDim.x >> 5;
-  for (int k = g; k < 32; k += ng) { cs[k][e] = 0; ps[k][e] = 0.0; }
-  __syncthreads();
-  long long c = 0;
-  double p = 0.0;
-  if (e < a.E) {
-    for (int t = g; t < a.ntiles_counts; t += ng) c += __ldcg(a.tile_counts + (size_t)t * a.E + e);
-    for (int t = g; t < a.ntiles_psum; t += ng) p += (double)__ldcg(a.tile_psum + (size_t)t * a.E + e);
+  auto wc = reinterpret_cast<long long(*)[32]>(scratch);
+  auto wp = reinterpret_cast<double(*)[32]>(scratch + 32 * 32 * 8);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  const int E = a.E;
+  long long c[EMAX];
+  double p[EMAX];
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) { c[e] = 0; p[e] = 0.0; }
+  const int nt = a.ntiles_counts > a.ntiles_psum ? a.ntiles_counts : a.ntiles_psum;
+  for (int t = tid; t < nt; t += blockDim.x) {
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+      if (e < E) {
+        if (t < a.ntiles_counts) c[e] += __ldcg(a.tile_counts + (size_t)t * E + e);
+        if (t < a.ntiles_psum) p[e] += (double)__ldcg(a.tile_psum + (size_t)t * E + e);
+      }
+    }
   }
-  cs[g][e] = c;
-  ps[g][e] = p;
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) {
+    if (e < E) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        c[e] += __shfl_xor_sync(0xffffffffu, c[e], o);
+        p[e] += __shfl_xor_sync(0xffffffffu, p[e], o);
+      }
+      if (lane == 0) { wc[w][e] = c[e]; wp[w][e] = p[e]; }
+    }
+  }
   __syncthreads();
   if (tid < 32) {
     long long cc = 0;
     double pp = 0.0;
-    for (int k = 0; k < 32; ++k) { cc += cs[k][tid]; pp += ps[k][tid]; }
+    if (tid < E)
+      for (int k = 0; k < nw; ++k) { cc += wc[k][tid]; pp += wp[k][tid]; }
     double term = 0.0;
-    if (tid < a.E) {
+    if (tid < E) {
       a.counts[tid] = (int32_t)cc;
-      term = ((double)a.E / ((double)a.K * a.T)) * (double)cc * (pp / a.T);
+      term = ((double)E / ((double)a.K * a.T)) * (double)cc * (pp / a.T);
     }
     for (int o = 16; o > 0; o >>= 1) term += __shfl_down_sync(0xffffffffu, term, o);
     if (tid == 0) *a.aux_loss = (float)(a.alpha * term);
@@ -219,38 +244,46 @@ __device__ bool last_block_done(unsigned int* ctr) {
 }
 
 template <int EMAX>
-__global__ void __launch_bounds__(kMmaMaxWarps * 32, 1)
+__global__ void __launch_bounds__((kMmaConsumers + 1) * 32, 1)
 route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, FinalizeArgs fin) {
   constexpr int NT = EMAX / 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const MmaSmem L = mma_layout(a.D, a.E);
-  const int NW = blockDim.x >> 5;
+  const int S = L.stages;
   const int E = a.E, D = a.D, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int wg_stride = D * 2 + 16;
   const int nchunks = D / 64;
   const int stage_bytes = kMmaRB * D * 2;
   uint8_t* wg_s = smem + L.wg;
   uint8_t* xs = smem + L.x;
-  float* logit_w = reinterpret_cast<float*>(smem + L.logits) + (size_t)w * kMmaRB * EMAX;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.misc);   // one barrier per warp
-  int* cnt_s = reinterpret_cast<int*>(full + kMmaMaxWarps);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.misc);
+  uint64_t* empty = full + kMmaMaxStages;
+  int* cnt_s = reinterpret_cast<int*>(empty + kMmaMaxStages);
   float* wsum_s = reinterpret_cast<float*>(cnt_s + 32);
 
   const int nunits = (a.T + kMmaRB - 1) / kMmaRB;
-  const int gw = blockIdx.x * NW + w, nwarps = gridDim.x * NW;
-  const int my_units = gw < nunits ? (nunits - gw + nwarps - 1) / nwarps : 0;
-  const uint32_t buf = smem_u32(xs + (size_t)w * stage_bytes);
-  const uint32_t bar = smem_u32(&full[w]);
-  auto issue = [&](int i) {              // lane 0: the 16 rows of unit i, all D/64 boxes
-    const int u = gw + i * nwarps;
+  const int my_units = (nunits - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  auto issue = [&](int i) {              // thread 0: the 16 rows of this CTA's i-th unit, all D/64 boxes
+    const int u = blockIdx.x + i * gridDim.x;
+    const int s = i % S;
+    const uint32_t bar = smem_u32(&full[s]);
     mbar_arrive_expect_tx(bar, stage_bytes);
-    for (int c = 0; c < nchunks; ++c) tma_load_2d(buf + c * (kMmaRB * 128), &tmap_x, c * 64, u * kMmaRB, bar);
+    const uint32_t dst = smem_u32(xs + (size_t)s * stage_bytes);
+    if (a.tmap3d) {
+      // one box: 64 columns x 16 rows x all D/64 column blocks, laid out [block][row][128 B]
+      tma_load_3d(dst, &tmap_x, 0, u * kMmaRB, 0, bar);
+    } else {
+      for (int c = 0; c < nchunks; ++c) tma_load_2d(dst + c * (kMmaRB * 128), &tmap_x, c * 64, u * kMmaRB, bar);
+    }
   };
-  if (lane == 0) {
-    mbar_init(bar, 1);
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);   // the consumer warp that finished the stage's MMAs
+    }
     fence_barrier_init();
-    if (my_units > 0) issue(0);          // x streams in while the gate weight loads
+    for (int i = 0; i < S && i < my_units; ++i) issue(i);   // x streams in while the gate loads
   }
   if (tid < 32) cnt_s[tid] = 0;
   {  // gate weight (bf16) -> padded rows; rows E..EMAX-1 are zero
@@ -265,71 +298,95 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
   }
   __syncthreads();
 
-  const uint32_t wg_base = smem_u32(wg_s);
-  const int li = lane >> 3, lj = lane & 7;
   float psum[EMAX];
 #pragma unroll
   for (int e = 0; e < EMAX; ++e) psum[e] = 0.f;
   bool ok = true;
-  for (int i = 0; i < my_units && ok; ++i) {
-    const int u = gw + i * nwarps;
-    ok = mbar_wait(bar, i & 1, nullptr, a.status, 100);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) break;
-    float acc[NT][4];
+  if (w == 0) {
+    // ------------------------------------------------ producer: refill each stage once it is free
+    if (lane == 0) {
+      for (int i = S; i < my_units; ++i) {
+        const int s = i % S;
+        if (!mbar_wait(smem_u32(&empty[s]), ((i / S) - 1) & 1, nullptr, a.status, 104)) { ok = false; break; }
+        issue(i);
+      }
+    }
+  } else {
+    // ------------------------------------------------ consumers: units i = cw, cw + 4, ...
+    const int cw = w - 1;
+    float* logit_w = reinterpret_cast<float*>(smem + L.logits) + (size_t)cw * kMmaRB * EMAX;
+    const uint32_t wg_base = smem_u32(wg_s);
+    const int li = lane >> 3, lj = lane & 7;
+    for (int i = cw; i < my_units; i += kMmaConsumers) {
+      const int u = blockIdx.x + i * gridDim.x;
+      const int s = i % S;                           // == cw: this warp's own stage
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[s]), (i / S) & 1, nullptr, a.status, 100));
+      if (!ok) break;
+      const uint32_t buf = smem_u32(xs + (size_t)s * stage_bytes);
+      // four independent accumulator chains (one per k16 step of a 64-column block) keep
+      // several mma.sync in flight instead of one long dependent chain
+      float acc4[4][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+      for (int g = 0; g < 4; ++g)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[nt][q] = 0.f;
-    for (int c = 0; c < nchunks; ++c) {
-      const uint32_t box = buf + c * (kMmaRB * 128);
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        uint32_t b[NT][2];
-        const int kc = c * 64 + ks * 16 + (li & 1) * 8;
+          for (int q = 0; q < 4; ++q) acc4[g][nt][q] = 0.f;
+      for (int c = 0; c < nchunks; ++c) {
+        const uint32_t box = buf + c * (kMmaRB * 128);
 #pragma unroll
-        for (int np = 0; np < NT; np += 2) {
-          if (np + 1 < NT) {
-            const int n = (np + (li >> 1)) * 8 + lj;
-            ldsm_x4(wg_base + n * wg_stride + kc * 2, b[np][0], b[np][1], b[np + 1][0], b[np + 1][1]);
-          } else {
-            ldsm_x2(wg_base + (np * 8 + lj) * wg_stride + kc * 2, b[np][0], b[np][1]);
+        for (int ks = 0; ks < 4; ++ks) {
+          uint32_t b[NT][2];
+          const int kc = c * 64 + ks * 16 + (li & 1) * 8;
+#pragma unroll
+          for (int np = 0; np < NT; np += 2) {
+            if (np + 1 < NT) {
+              const int n = (np + (li >> 1)) * 8 + lj;
+              ldsm_x4(wg_base + n * wg_stride + kc * 2, b[np][0], b[np][1], b[np + 1][0], b[np + 1][1]);
+            } else {
+              ldsm_x2(wg_base + (np * 8 + lj) * wg_stride + kc * 2, b[np][0], b[np][1]);
+            }
           }
+          const int row = (li & 1) * 8 + lj;
+          const int chunk = ks * 2 + (li >> 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_16816(acc4[ks][nt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
         }
-        const int row = (li & 1) * 8 + lj;
-        const int chunk = ks * 2 + (li >> 1);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_16816(acc[nt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
       }
-    }
-    __syncwarp();                                  // every lane is done reading the buffer
-    if (lane == 0 && i + 1 < my_units) issue(i + 1);   // next rows load during the epilogue
+      float acc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int row = lane >> 2, col = nt * 8 + (lane & 3) * 2;
-      logit_w[row * EMAX + col] = acc[nt][0];
-      logit_w[row * EMAX + col + 1] = acc[nt][1];
-      logit_w[(row + 8) * EMAX + col] = acc[nt][2];
-      logit_w[(row + 8) * EMAX + col + 1] = acc[nt][3];
-    }
-    __syncwarp();
-    if (lane < kMmaRB) {
-      const int tok = u * kMmaRB + lane;
-      if (tok < a.T) {
-        float l[EMAX];
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) l[e] = logit_w[lane * EMAX + e];
-        token_select<EMAX>(l, tok, a, cnt_s, psum);
+        for (int q = 0; q < 4; ++q) acc[nt][q] = (acc4[0][nt][q] + acc4[1][nt][q]) + (acc4[2][nt][q] + acc4[3][nt][q]);
+      __syncwarp();                                  // every lane is done reading the stage
+      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));  // the producer may refill it now
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int row = lane >> 2, col = nt * 8 + (lane & 3) * 2;
+        logit_w[row * EMAX + col] = acc[nt][0];
+        logit_w[row * EMAX + col + 1] = acc[nt][1];
+        logit_w[(row + 8) * EMAX + col] = acc[nt][2];
+        logit_w[(row + 8) * EMAX + col + 1] = acc[nt][3];
       }
+      __syncwarp();
+      if (lane < kMmaRB) {
+        const int tok = u * kMmaRB + lane;
+        if (tok < a.T) {
+          float l[EMAX];
+#pragma unroll
+          for (int e = 0; e < EMAX; ++e) l[e] = logit_w[lane * EMAX + e];
+          token_select<EMAX>(l, tok, a, cnt_s, psum);
+        }
+      }
+      __syncwarp();
     }
-    __syncwarp();
   }
   __syncthreads();
   tile_partials<EMAX>(psum, blockIdx.x, a, cnt_s, wsum_s);
   if (!ok) set_status(a.status, DEV_TIMEOUT, 102);
-  if (fin.counts != nullptr && last_block_done(fin.ctr)) finalize_counts_loss(fin, xs);
+  if (fin.counts != nullptr && last_block_done(fin.ctr)) finalize_counts_loss<EMAX>(fin, xs);
 }
 
 // ---------------------------------------------------------------- fp32: FFMA logits
@@ -420,13 +477,13 @@ route_kernel_ffma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Final
       tile_partials<EMAX>(psum, tile, a, cnt_s, wsum_s);
     }
   }
-  if (fin.counts != nullptr && last_block_done(fin.ctr)) finalize_counts_loss(fin, xs);
+  if (fin.counts != nullptr && last_block_done(fin.ctr)) finalize_counts_loss<EMAX>(fin, xs);
 }
 
 void route_plan(int T, int D, int E, int bf16, int sms, int* tile_rows, int* threads) {
   if (bf16) {
     *tile_rows = kMmaRB;
-    *threads = mma_layout(D, E).warps * 32;
+    *threads = (kMmaConsumers + 1) * 32;
   } else {
     int tile = (T + sms - 1) / sms;
     tile = (tile + 31) / 32 * 32;
@@ -441,7 +498,7 @@ size_t route_smem_total(int D, int E, int tile_rows, int bf16) {
   return bf16 ? mma_layout(D, E).total : route_smem_bytes(D, E, tile_rows, 0);
 }
 
-int route_mma_stages(int D, int E) { return mma_layout(D, E).warps; }
+int route_mma_stages(int D, int E) { return mma_layout(D, E).stages; }
 
 cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tm, cudaStream_t s) {
   const size_t smem = route_smem_total(a.D, a.E, a.tile_rows, a.bf16);
@@ -451,7 +508,7 @@ cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUte
   if (a.E <= EM) {                                                                                      \
     err = cudaFuncSetAttribute(route_kernel_mma<EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (err != cudaSuccess) return err;                                                                 \
-    route_kernel_mma<EM><<<a.grid, mma_layout(a.D, a.E).warps * 32, smem, s>>>(*tm, a, fin);          \
+    route_kernel_mma<EM><<<a.grid, (kMmaConsumers + 1) * 32, smem, s>>>(*tm, a, fin);                   \
     return cudaGetLastError();                                                                          \
   }
     MOE_ROUTE_MMA(8)
@@ -475,13 +532,16 @@ cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUte
 }
 
 // ---------------------------------------------------------------- finalize (race path)
-__global__ void __launch_bounds__(1024) route_finalize_kernel(FinalizeArgs a) {
+template <int EMAX>
+__global__ void __launch_bounds__(256) route_finalize_kernel(FinalizeArgs a) {
   __shared__ __align__(16) uint8_t scratch[kFinalizeScratch];
-  finalize_counts_loss(a, scratch);
+  finalize_counts_loss<EMAX>(a, scratch);
 }
 
 cudaError_t launch_route_finalize(const FinalizeArgs& a, cudaStream_t s) {
-  route_finalize_kernel<<<1, 1024, 0, s>>>(a);
+  if (a.E <= 8) route_finalize_kernel<8><<<1, 256, 0, s>>>(a);
+  else if (a.E <= 16) route_finalize_kernel<16><<<1, 256, 0, s>>>(a);
+  else route_finalize_kernel<32><<<1, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -26,9 +26,9 @@
  *   - Every pointer argument named as a tensor is DEVICE memory owned by the
  *     caller; the library never allocates, frees or keeps it.  Tensors are
  *     row-major and contiguous; every tensor pointer must be 16-byte aligned.
- *   - "act" tensors (x, x_perm, h_perm, h_sh, out) and weights/biases have the
- *     storage type cfg->dtype (fp32 or bf16); scores, gates, y_perm, y_sh are
- *     fp32; indices are int32.
+ *   - "act" tensors (x, x_perm, h_perm, h_sh, y_perm, y_sh, out) and
+ *     weights/biases have the storage type cfg->dtype (fp32 or bf16); scores and
+ *     gates are fp32; indices are int32.  Every sum runs in fp32.
  *   - Weights follow nn.Linear (out x in): W1 [E,H,D], b1 [E,H], W2 [E,D,H],
  *     b2 [E,D].  The n_s shared experts come stacked the same way: W1s
  *     [n_s,H,D], b1s [n_s,H], W2s [n_s,D,H], b2s [n_s,D].  The kernels treat
@@ -171,30 +171,31 @@ int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void
 
 /*
  * moe_expert_gemm2 -- second expert layer with bias and gate scaling fused:
- *   y_perm[r] = row_gate[r] * (W2_{e(r)} h_perm[r] + b2_{e(r)})   fp32 [R_max,D]
- *   y_sh[t]   = sum_j (W2s_j h_sh[t, j*H:(j+1)*H] + b2s_j)         fp32 [T,D]
+ *   y_perm[r] = row_gate[r] * (W2_{e(r)} h_perm[r] + b2_{e(r)})   act [R_max,D]
+ *   y_sh[t]   = sum_j (W2s_j h_sh[t, j*H:(j+1)*H] + b2s_j)         act [T,D]
+ *   (fp32 accumulation and epilogue; one rounding to the act type on store)
  *   b2 [E,D] / b2s [n_s,D] may be NULL; y_sh NULL when n_s = 0.
  */
 int moe_expert_gemm2(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm,
                      const void* h_sh, const void* w2, const void* b2, const void* w2s,
-                     const void* b2s, const float* row_gate, float* y_perm, float* y_sh,
+                     const void* b2s, const float* row_gate, void* y_perm, void* y_sh,
                      void* ws, size_t ws_bytes, void* stream);
 
 /* moe_expert_mlp -- moe_expert_gemm1 followed by moe_expert_gemm2. */
 int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
                    const void* x, const void* w1, const void* b1, const void* w2, const void* b2,
                    const void* w1s, const void* b1s, const void* w2s, const void* b2s,
-                   const float* row_gate, void* h_perm, void* h_sh, float* y_perm, float* y_sh,
+                   const float* row_gate, void* h_perm, void* h_sh, void* y_perm, void* y_sh,
                    void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_combine -- MoE(x_t) = sum_{k < n_sel[t]} y_perm[pos[t,k]] + y_sh[t]
  * (the gates are already applied in y_perm), summed in fp32 in slot order
  * then the shared term, rounded once to the act type.
- *   y_perm [R_max,D] fp32; y_sh [T,D] fp32 or NULL (n_s = 0);
+ *   y_perm [R_max,D] act; y_sh [T,D] act or NULL (n_s = 0);
  *   pos [T,Kmax] int32; n_sel [T] or NULL (= K); out [T,D] act.
  */
-int moe_combine(const moe_config_t* cfg, const float* y_perm, const float* y_sh,
+int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,
                 const int32_t* pos, const int32_t* n_sel, void* out, void* stream);
 
 /*

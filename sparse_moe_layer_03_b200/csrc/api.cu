@@ -61,7 +61,7 @@ int validate(const moe_config_t* c) {
   if (c->gemm_impl < MOE_GEMM_AUTO || c->gemm_impl > MOE_GEMM_TC1) return fail(MOE_ERR_INVALID_ARG, "gemm_impl=%d", c->gemm_impl);
   if (c->reserved != 0) return fail(MOE_ERR_INVALID_ARG, "reserved field must be 0");
   if (route_smem_total(c->D, c->E, 32, c->dtype == MOE_BF16) > 232448 ||
-      (c->dtype == MOE_BF16 && route_mma_stages(c->D, c->E) < 2))
+      (c->dtype == MOE_BF16 && route_mma_stages(c->D, c->E) < 1))
     return fail(MOE_ERR_UNSUPPORTED, "E=%d x D=%d too large for the router's shared memory", c->E, c->D);
   return MOE_OK;
 }
@@ -179,16 +179,18 @@ int make_tmap(CUtensorMap* m, const void* base, bool bf16, long long rows, long 
 }
 
 // x [rows, cols] bf16 seen as 3-D {64 columns, rows, cols/64 blocks}: one box brings
-// `box_rows` whole rows as cols/64 swizzled 128-byte blocks, block-major.  Returns
-// false when the driver does not accept the layout (the caller then uses 2-D boxes).
+// `box_rows` rows x ceil(cols/128) swizzled 128-byte blocks (half of each row),
+// block-major.  Returns false when the driver does not accept the layout (the
+// caller then uses 2-D boxes).
 bool make_tmap_rows3d(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)(rows > 0 ? rows : 1), (cuuint64_t)(cols / 64)};
   cuuint64_t strides[2] = {(cuuint64_t)cols * 2, 128};
-  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)(cols / 64)};
+  const cuuint32_t blocks = (cuuint32_t)((cols / 64 + 1) / 2);    // one box = half of a row block
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, blocks};
   cuuint32_t estr[3] = {1, 1, 1};
-  if (cols / 64 > 256) return false;
+  if (blocks > 256) return false;
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -391,7 +393,7 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
   if (pair) {
     // output boxes for the TMA-store epilogue: 32 rows x 128 bytes (bf16 h or fp32 y)
     CUtensorMap to[2];
-    const bool out_bf16 = g.p[0].epi == 0;
+    const bool out_bf16 = g.bf16 != 0;          // h and y are both in the act dtype
     if ((rc = make_tmap(&to[0], g.p[0].out, out_bf16, rows0, g.p[0].N, 32, "out0"))) return rc;
     if (g.nprob > 1) {
       if ((rc = make_tmap(&to[1], g.p[1].out, out_bf16, rows1, g.p[1].N, 32, "out1"))) return rc;
@@ -449,7 +451,7 @@ int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void
 
 int moe_expert_gemm2(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm,
                      const void* h_sh, const void* w2, const void* b2, const void* w2s,
-                     const void* b2s, const float* row_gate, float* y_perm, float* y_sh,
+                     const void* b2s, const float* row_gate, void* y_perm, void* y_sh,
                      void* ws, size_t ws_bytes, void* stream) {
   int rc = validate(cfg);
   if (rc) return rc;
@@ -494,7 +496,7 @@ int moe_expert_gemm2(const moe_config_t* cfg, const int32_t* offsets, const void
 int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
                    const void* x, const void* w1, const void* b1, const void* w2, const void* b2,
                    const void* w1s, const void* b1s, const void* w2s, const void* b2s,
-                   const float* row_gate, void* h_perm, void* h_sh, float* y_perm, float* y_sh,
+                   const float* row_gate, void* h_perm, void* h_sh, void* y_perm, void* y_sh,
                    void* ws, size_t ws_bytes, void* stream) {
   int rc = moe_expert_gemm1(cfg, offsets, x_perm, x, w1, b1, w1s, b1s, h_perm, h_sh, ws, ws_bytes, stream);
   if (rc) return rc;
@@ -502,7 +504,7 @@ int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* 
                           stream);
 }
 
-int moe_combine(const moe_config_t* cfg, const float* y_perm, const float* y_sh,
+int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,
                 const int32_t* pos, const int32_t* n_sel, void* out, void* stream) {
   int rc = validate(cfg);
   if (rc) return rc;

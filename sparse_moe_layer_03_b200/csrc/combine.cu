@@ -11,13 +11,23 @@ namespace moe {
 
 constexpr int kCombineThreads = 256;
 
+// 8 consecutive elements as fp32
+template <typename T> __device__ __forceinline__ void load8(const T* p, size_t i, float* f);
+template <> __device__ __forceinline__ void load8<float>(const float* p, size_t i, float* f) {
+  const float4 a = reinterpret_cast<const float4*>(p)[2 * i], b = reinterpret_cast<const float4*>(p)[2 * i + 1];
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+template <> __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, size_t i, float* f) {
+  bf16x8_to_f32(reinterpret_cast<const uint4*>(p)[i], f);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * (kCombineThreads / 32);
-  const int n4 = a.D / 4;
-  const float4* yp = reinterpret_cast<const float4*>(a.y_perm);
-  const float4* ys = reinterpret_cast<const float4*>(a.y_sh);
+  const int n8 = a.D / 8;
+  const T* yp = reinterpret_cast<const T*>(a.y_perm);
+  const T* ys = reinterpret_cast<const T*>(a.y_sh);
   for (int t = blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5); t < a.T; t += nwarps) {
     int ns = a.n_sel ? a.n_sel[t] : a.K;
     ns = ns < 0 ? 0 : (ns > a.Kmax ? a.Kmax : ns);
@@ -26,24 +36,32 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
       const int p = a.pos[(size_t)t * a.Kmax + k];
       rows[k] = (p >= 0 && p < a.r_max) ? p : -1;
     }
-    for (int v = lane; v < n4; v += 32) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int v = lane; v < n8; v += 32) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int k = 0; k < ns; ++k) {
         if (rows[k] < 0) continue;
-        const float4 y = yp[(size_t)rows[k] * n4 + v];
-        acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w;
+        float y[8];
+        load8<T>(yp, (size_t)rows[k] * n8 + v, y);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] += y[q];
       }
       if (ys) {
-        const float4 y = ys[(size_t)t * n4 + v];
-        acc.x += y.x; acc.y += y.y; acc.z += y.z; acc.w += y.w;
+        float y[8];
+        load8<T>(ys, (size_t)t * n8 + v, y);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] += y[q];
       }
       if constexpr (sizeof(T) == 2) {
-        uint2 o;
-        o.x = pack_bf16x2(acc.x, acc.y);
-        o.y = pack_bf16x2(acc.z, acc.w);
-        reinterpret_cast<uint2*>(a.out)[(size_t)t * n4 + v] = o;
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        reinterpret_cast<uint4*>(a.out)[(size_t)t * n8 + v] = o;
       } else {
-        reinterpret_cast<float4*>(a.out)[(size_t)t * n4 + v] = acc;
+        float4* o = reinterpret_cast<float4*>(a.out) + (size_t)t * 2 * n8 + 2 * v;
+        o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
       }
     }
   }

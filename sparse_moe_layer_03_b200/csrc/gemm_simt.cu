@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
       if (pr.epi == 0)
         reinterpret_cast<T*>(pr.out)[grow * pr.ld_out + n] = Elem<T>::from_f(gelu_act<false>(u, a.act));
       else
-        reinterpret_cast<float*>(pr.out)[grow * pr.ld_out + n] = u * gate;
+        reinterpret_cast<T*>(pr.out)[grow * pr.ld_out + n] = Elem<T>::from_f(u * gate);
     }
   }
 }

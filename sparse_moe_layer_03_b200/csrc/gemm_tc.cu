@@ -8,7 +8,7 @@
 // GELU per "Scalable Diffusion Models with Transformers", DiT block details),
 // each expert a pair of these GEMMs:
 //   GEMM1 epilogue: + b1, GELU, round to bf16           -> h
-//   GEMM2 epilogue: + b2, times the row's gate (routed)  -> y (fp32)
+//   GEMM2 epilogue: + b2, times the row's gate (routed)  -> y (bf16)
 //
 // CTA = 6 warps: warp 0 issues TMA loads (128-byte swizzled K-major tiles) into
 // a ring of shared-memory stages; warp 1 allocates TMEM and one thread issues
@@ -146,7 +146,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ 
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_last();
-      const uint64_t pol_a = policy_evict_first();
+      // A tiles are reused by every column tile of their row block (consecutive tiles, run
+      // side by side): keep them in L2 normally; evict-first sent them back to DRAM 3.5x
+      const uint64_t pol_a = policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       for (int tile = blockIdx.x; tile < pl.total; tile += gridDim.x) {
@@ -245,29 +247,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ 
           }
         }
         if (rv) {
-          if (pr.epi == 0) {
-            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ld_out + col0);
+          // GEMM1: gelu(acc + b1); GEMM2: gate * (acc + b2); both rounded once to bf16
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ld_out + col0);
+          uint4 o[4];
+          uint32_t* ow = reinterpret_cast<uint32_t*>(o);
+          const int mode = pr.epi == 0 ? (a.act == 1 ? 1 : 0) : 2;
+          if (mode == 0) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 o;
-              uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+            for (int j = 0; j < 32; j += 2)
+              ow[j / 2] = pack_bf16x2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 0),
+                                      gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], 0));
+          } else if (mode == 1) {
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const int j = 8 * u + 2 * h;
-                ow[h] = pack_bf16x2(gelu_act<true>(__uint_as_float(v[j]) + b[j], a.act),
-                                    gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], a.act));
-              }
-              dst[u] = o;
-            }
+            for (int j = 0; j < 32; j += 2)
+              ow[j / 2] = pack_bf16x2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 1),
+                                      gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], 1));
           } else {
-            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(pr.out) + grow * pr.ld_out + col0);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int j = 4 * u;
-              dst[u] = make_float4((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate,
-                                   (__uint_as_float(v[j + 2]) + b[j + 2]) * gate, (__uint_as_float(v[j + 3]) + b[j + 3]) * gate);
-            }
+            for (int j = 0; j < 32; j += 2)
+              ow[j / 2] = pack_bf16x2((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate);
           }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) dst[u] = o[u];
         }
       }
       tc_fence_before();

@@ -79,7 +79,7 @@ struct GemmProblem {
   int routed;               // 1: rows grouped by expert segments (offsets), 0: dense rows
   int M;                    // dense: rows; routed: unused (from offsets)
   int N, K;                 // per-expert output width and reduction length
-  int epi;                  // 0: bias + GELU -> act store; 1: (bias) * gate -> fp32 store
+  int epi;                  // 0: bias + GELU -> act store; 1: (bias) * gate -> act store
   const void* A;            // [rows,K] act (FFMA path; the TMA path uses tensor maps)
   const void* B;            // [E*N or N, K] act
   void* out; long long ld_out;
@@ -106,7 +106,7 @@ cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t s);
 
 // ---- combine.cu
 struct CombineArgs {
-  const float* y_perm; const float* y_sh; const int32_t* pos; const int32_t* n_sel;
+  const void* y_perm; const void* y_sh; const int32_t* pos; const int32_t* n_sel;   // act dtype
   void* out; int bf16;
   int T, D, K, Kmax;
   long long r_max;

@@ -122,13 +122,14 @@ __device__ __forceinline__ void tile_partials(const float* psum, int tile, const
 // ---------------------------------------------------------------- bf16: tensor-core logits
 // Work unit = a block of 16 consecutive tokens: their full rows (16 x D bf16,
 // one contiguous stretch of HBM, so DRAM pages are read whole) land in one
-// shared-memory stage as D/64 TMA boxes of 16 rows x 128 bytes (128-byte
-// swizzle).  One producer thread keeps a ring of stages in flight; four
-// consumer warps take units in turn: wait for the rows, compute the 16 x E
-// logits with mma.sync m16n8k16 (A via ldmatrix from the swizzled stage, B =
-// gate weight in shared memory with rows padded by 16 bytes), free the stage,
-// then run softmax and selection (one lane per token).  No block-wide barrier
-// inside the loop.
+// pair of shared-memory stages (one per half of the row, each one 3-D TMA box of
+// 64-column blocks x 16 rows, 128-byte swizzle).  One producer thread keeps the
+// stages in flight; each consumer warp owns two stages and takes every NC-th
+// row block: wait for a half, compute its part of the 16 x E logits with
+// mma.sync m16n8k16 (A via ldmatrix from the swizzled stage, B = gate weight in
+// shared memory with rows padded by 16 bytes), free that stage (the next load
+// overlaps the other half's MMAs), then run softmax and selection (one lane
+// per token).  No block-wide barrier inside the loop.
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
@@ -145,32 +146,34 @@ __device__ __forceinline__ void mma_16816(float* d, uint32_t a0, uint32_t a1, ui
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-constexpr int kMmaRB = 16;        // tokens per work unit
-constexpr int kMmaConsumers = 4;  // consumer warps; warp 0 is the TMA producer
-// Consumer warp c owns stage c: it waits on that stage's phases strictly in order.
-// (Stages shared round-robin by several consumers would let a warp wait on a phase two
-// ahead of the barrier, where the parity test passes early.)
-constexpr int kMmaStages = kMmaConsumers;
-constexpr int kMmaMaxStages = kMmaStages;
+constexpr int kMmaRB = 16;        // tokens per row block
+constexpr int kMmaMaxConsumers = 4;
 
-// A ring of stages (16 full rows each) fed by one producer thread.
+// A row block is loaded as two halves (column blocks [0, hc) and [hc, 2hc), hc =
+// ceil(D/128)), each into its own stage; consumer warp c owns stages 2c and 2c+1
+// and waits on their phases strictly in order.  As many consumers (<= 4) as the
+// shared memory allows.
 struct MmaSmem {
   size_t wg, x, logits, misc, total;
-  int stages;
+  int consumers, hc;
 };
 __host__ __device__ inline MmaSmem mma_layout(int D, int E) {
   MmaSmem L;
   const int em = route_emax(E);
+  L.hc = (D / 64 + 1) / 2;
   L.wg = 0;
   L.x = align1k((size_t)em * (D * 2 + 16));
-  const size_t stage = (size_t)kMmaRB * D * 2;
-  const size_t logits = (size_t)kMmaConsumers * kMmaRB * em * 4;
-  const size_t fixed = L.x + logits + 2048 /*misc*/ + 1024 /*align slack*/ + 1024 /*scratch margin*/;
-  const int st = (int)((232448 - fixed) / stage);
-  L.stages = st >= kMmaStages ? kMmaStages : 0;   // 0: does not fit (rejected by validation)
-  const size_t xb = (size_t)(L.stages > 0 ? L.stages : 0) * stage;
+  const size_t stage = (size_t)kMmaRB * L.hc * 128;
+  L.consumers = 0;
+  for (int nc = kMmaMaxConsumers; nc >= 1; --nc) {
+    const size_t xb = 2 * nc * stage;
+    const size_t total = L.x + (xb > 16896 ? xb : 16896) + (size_t)nc * kMmaRB * em * 4 + 2048 + 1024;
+    if (total + 1024 <= 232448) { L.consumers = nc; break; }
+  }
+  const int nc = L.consumers > 0 ? L.consumers : 1;
+  const size_t xb = 2 * nc * stage;
   L.logits = L.x + (xb > 16896 ? xb : 16896);   // x stages double as the finalize scratch
-  L.misc = L.logits + logits;
+  L.misc = L.logits + (size_t)nc * kMmaRB * em * 4;
   L.total = L.misc + 2048 + 1024;
   return L;
 }
@@ -244,46 +247,50 @@ __device__ bool last_block_done(unsigned int* ctr) {
 }
 
 template <int EMAX>
-__global__ void __launch_bounds__((kMmaConsumers + 1) * 32, 1)
+__global__ void __launch_bounds__((kMmaMaxConsumers + 1) * 32, 1)
 route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, FinalizeArgs fin) {
   constexpr int NT = EMAX / 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const MmaSmem L = mma_layout(a.D, a.E);
-  const int S = L.stages;
+  const int NC = L.consumers, hc = L.hc;
   const int E = a.E, D = a.D, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int wg_stride = D * 2 + 16;
   const int nchunks = D / 64;
-  const int stage_bytes = kMmaRB * D * 2;
+  const int stage_bytes = kMmaRB * hc * 128;
   uint8_t* wg_s = smem + L.wg;
   uint8_t* xs = smem + L.x;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.misc);
-  uint64_t* empty = full + kMmaMaxStages;
-  int* cnt_s = reinterpret_cast<int*>(empty + kMmaMaxStages);
+  uint64_t* empty = full + 2 * kMmaMaxConsumers;
+  int* cnt_s = reinterpret_cast<int*>(empty + 2 * kMmaMaxConsumers);
   float* wsum_s = reinterpret_cast<float*>(cnt_s + 32);
 
-  const int nunits = (a.T + kMmaRB - 1) / kMmaRB;
-  const int my_units = (nunits - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-  auto issue = [&](int i) {              // thread 0: the 16 rows of this CTA's i-th unit, all D/64 boxes
-    const int u = blockIdx.x + i * gridDim.x;
-    const int s = i % S;
-    const uint32_t bar = smem_u32(&full[s]);
-    mbar_arrive_expect_tx(bar, stage_bytes);
-    const uint32_t dst = smem_u32(xs + (size_t)s * stage_bytes);
+  const int nrb = (a.T + kMmaRB - 1) / kMmaRB;
+  const int my_rb = (nrb - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  // thread 0: half h of this CTA's j-th row block into stage 2 (j mod NC) + h
+  auto issue = [&](int j, int h) {
+    const int rb = blockIdx.x + j * gridDim.x;
+    const int st = 2 * (j % NC) + h;
+    const int z0 = h * hc;
+    const int nb = (nchunks - z0) < hc ? (nchunks - z0) : hc;     // blocks inside D
+    const uint32_t bar = smem_u32(&full[st]);
+    const uint32_t dst = smem_u32(xs + (size_t)st * stage_bytes);
     if (a.tmap3d) {
-      // one box: 64 columns x 16 rows x all D/64 column blocks, laid out [block][row][128 B]
-      tma_load_3d(dst, &tmap_x, 0, u * kMmaRB, 0, bar);
+      // one box of hc blocks; blocks past D come back zero-filled and count as bytes
+      mbar_arrive_expect_tx(bar, stage_bytes);
+      tma_load_3d(dst, &tmap_x, 0, rb * kMmaRB, z0, bar);
     } else {
-      for (int c = 0; c < nchunks; ++c) tma_load_2d(dst + c * (kMmaRB * 128), &tmap_x, c * 64, u * kMmaRB, bar);
+      mbar_arrive_expect_tx(bar, (uint32_t)nb * kMmaRB * 128);
+      for (int c = 0; c < nb; ++c) tma_load_2d(dst + c * (kMmaRB * 128), &tmap_x, (z0 + c) * 64, rb * kMmaRB, bar);
     }
   };
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 1);   // the consumer warp that finished the stage's MMAs
+    for (int st = 0; st < 2 * NC; ++st) {
+      mbar_init(smem_u32(&full[st]), 1);
+      mbar_init(smem_u32(&empty[st]), 1);   // the owning consumer warp, after its MMAs
     }
     fence_barrier_init();
-    for (int i = 0; i < S && i < my_units; ++i) issue(i);   // x streams in while the gate loads
+    for (int j = 0; j < NC && j < my_rb; ++j) { issue(j, 0); issue(j, 1); }   // x streams in while Wg loads
   }
   if (tid < 32) cnt_s[tid] = 0;
   {  // gate weight (bf16) -> padded rows; rows E..EMAX-1 are zero
@@ -305,26 +312,25 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
   if (w == 0) {
     // ------------------------------------------------ producer: refill each stage once it is free
     if (lane == 0) {
-      for (int i = S; i < my_units; ++i) {
-        const int s = i % S;
-        if (!mbar_wait(smem_u32(&empty[s]), ((i / S) - 1) & 1, nullptr, a.status, 104)) { ok = false; break; }
-        issue(i);
+      for (int j = NC; j < my_rb && ok; ++j) {
+        const int k = j / NC;
+        for (int h = 0; h < 2; ++h) {
+          const int st = 2 * (j % NC) + h;
+          if (!mbar_wait(smem_u32(&empty[st]), (k - 1) & 1, nullptr, a.status, 104)) { ok = false; break; }
+          issue(j, h);
+        }
       }
     }
-  } else {
-    // ------------------------------------------------ consumers: units i = cw, cw + 4, ...
+  } else if (w <= NC) {
+    // ------------------------------------------------ consumer warp cw: row blocks j = cw, cw + NC, ...
     const int cw = w - 1;
     float* logit_w = reinterpret_cast<float*>(smem + L.logits) + (size_t)cw * kMmaRB * EMAX;
     const uint32_t wg_base = smem_u32(wg_s);
     const int li = lane >> 3, lj = lane & 7;
-    for (int i = cw; i < my_units; i += kMmaConsumers) {
-      const int u = blockIdx.x + i * gridDim.x;
-      const int s = i % S;                           // == cw: this warp's own stage
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[s]), (i / S) & 1, nullptr, a.status, 100));
-      if (!ok) break;
-      const uint32_t buf = smem_u32(xs + (size_t)s * stage_bytes);
-      // four independent accumulator chains (one per k16 step of a 64-column block) keep
-      // several mma.sync in flight instead of one long dependent chain
+    for (int j = cw; j < my_rb; j += NC) {
+      const int rb = blockIdx.x + j * gridDim.x;
+      const uint32_t parity = (j / NC) & 1;
+      // four independent accumulator chains (one per k16 step of a 64-column block)
       float acc4[4][NT][4];
 #pragma unroll
       for (int g = 0; g < 4; ++g)
@@ -332,36 +338,46 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int q = 0; q < 4; ++q) acc4[g][nt][q] = 0.f;
-      for (int c = 0; c < nchunks; ++c) {
-        const uint32_t box = buf + c * (kMmaRB * 128);
+      for (int h = 0; h < 2 && ok; ++h) {
+        const int st = 2 * cw + h;
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), parity, nullptr, a.status, 100));
+        if (!ok) break;
+        const uint32_t buf = smem_u32(xs + (size_t)st * stage_bytes);
+        const int z0 = h * hc;
+        const int nb = (nchunks - z0) < hc ? (nchunks - z0) : hc;
+        for (int cb = 0; cb < nb; ++cb) {
+          const int c = z0 + cb;                       // global 64-column block
+          const uint32_t box = buf + cb * (kMmaRB * 128);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          uint32_t b[NT][2];
-          const int kc = c * 64 + ks * 16 + (li & 1) * 8;
+          for (int ks = 0; ks < 4; ++ks) {
+            uint32_t b[NT][2];
+            const int kc = c * 64 + ks * 16 + (li & 1) * 8;
 #pragma unroll
-          for (int np = 0; np < NT; np += 2) {
-            if (np + 1 < NT) {
-              const int n = (np + (li >> 1)) * 8 + lj;
-              ldsm_x4(wg_base + n * wg_stride + kc * 2, b[np][0], b[np][1], b[np + 1][0], b[np + 1][1]);
-            } else {
-              ldsm_x2(wg_base + (np * 8 + lj) * wg_stride + kc * 2, b[np][0], b[np][1]);
+            for (int np = 0; np < NT; np += 2) {
+              if (np + 1 < NT) {
+                const int n = (np + (li >> 1)) * 8 + lj;
+                ldsm_x4(wg_base + n * wg_stride + kc * 2, b[np][0], b[np][1], b[np + 1][0], b[np + 1][1]);
+              } else {
+                ldsm_x2(wg_base + (np * 8 + lj) * wg_stride + kc * 2, b[np][0], b[np][1]);
+              }
             }
-          }
-          const int row = (li & 1) * 8 + lj;
-          const int chunk = ks * 2 + (li >> 1);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
+            const int row = (li & 1) * 8 + lj;
+            const int chunk = ks * 2 + (li >> 1);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_16816(acc4[ks][nt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
+            for (int nt = 0; nt < NT; ++nt) mma_16816(acc4[ks][nt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
+          }
         }
+        __syncwarp();                                // every lane is done reading the stage
+        if (lane == 0) mbar_arrive(smem_u32(&empty[st]));   // the producer may refill it now
       }
+      if (!ok) break;
       float acc[NT][4];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[nt][q] = (acc4[0][nt][q] + acc4[1][nt][q]) + (acc4[2][nt][q] + acc4[3][nt][q]);
-      __syncwarp();                                  // every lane is done reading the stage
-      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));  // the producer may refill it now
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int row = lane >> 2, col = nt * 8 + (lane & 3) * 2;
@@ -372,7 +388,7 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
       }
       __syncwarp();
       if (lane < kMmaRB) {
-        const int tok = u * kMmaRB + lane;
+        const int tok = rb * kMmaRB + lane;
         if (tok < a.T) {
           float l[EMAX];
 #pragma unroll
@@ -483,7 +499,7 @@ route_kernel_ffma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Final
 void route_plan(int T, int D, int E, int bf16, int sms, int* tile_rows, int* threads) {
   if (bf16) {
     *tile_rows = kMmaRB;
-    *threads = (kMmaConsumers + 1) * 32;
+    *threads = (mma_layout(D, E).consumers + 1) * 32;
   } else {
     int tile = (T + sms - 1) / sms;
     tile = (tile + 31) / 32 * 32;
@@ -498,7 +514,7 @@ size_t route_smem_total(int D, int E, int tile_rows, int bf16) {
   return bf16 ? mma_layout(D, E).total : route_smem_bytes(D, E, tile_rows, 0);
 }
 
-int route_mma_stages(int D, int E) { return mma_layout(D, E).stages; }
+int route_mma_stages(int D, int E) { return mma_layout(D, E).consumers; }
 
 cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tm, cudaStream_t s) {
   const size_t smem = route_smem_total(a.D, a.E, a.tile_rows, a.bf16);
@@ -508,7 +524,7 @@ cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUte
   if (a.E <= EM) {                                                                                      \
     err = cudaFuncSetAttribute(route_kernel_mma<EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (err != cudaSuccess) return err;                                                                 \
-    route_kernel_mma<EM><<<a.grid, (kMmaConsumers + 1) * 32, smem, s>>>(*tm, a, fin);                   \
+    route_kernel_mma<EM><<<a.grid, (mma_layout(a.D, a.E).consumers + 1) * 32, smem, s>>>(*tm, a, fin);    \
     return cudaGetLastError();                                                                          \
   }
     MOE_ROUTE_MMA(8)

@@ -84,10 +84,10 @@ class MoELayer:
         self.row_gate = torch.empty((self.R,), dtype=f32, device=dev)
         self.x_perm = torch.empty((self.R, s.D), dtype=dt, device=dev)
         self.h_perm = torch.empty((self.R, s.H), dtype=dt, device=dev)
-        self.y_perm = torch.empty((self.R, s.D), dtype=f32, device=dev)
+        self.y_perm = torch.empty((self.R, s.D), dtype=dt, device=dev)
         ns = s.n_shared
         self.h_sh = torch.empty((T, ns * s.H), dtype=dt, device=dev) if ns else None
-        self.y_sh = torch.empty((T, s.D), dtype=f32, device=dev) if ns else None
+        self.y_sh = torch.empty((T, s.D), dtype=dt, device=dev) if ns else None
         self.out = torch.empty((T, s.D), dtype=dt, device=dev)
         B.moe_workspace_init(self.ws, self.ws_bytes, self.stream())
 

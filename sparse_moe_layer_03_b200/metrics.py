@@ -44,9 +44,10 @@ def dispatch_bytes(T, D, E, K, elem, race=False):
     return T * D * elem + S * D * elem + T * kmax * 4 * 2 + S * 8
 
 
-def combine_bytes(T, D, K, n_shared, elem, y_elem=4):
+def combine_bytes(T, D, K, n_shared, elem, y_elem=None):
     """Routed rows and the shared row read, output written, positions read."""
     S = K * T
+    y_elem = elem if y_elem is None else y_elem      # expert outputs are stored in the act dtype
     b = S * D * y_elem + T * D * elem + T * K * 4
     if n_shared > 0:
         b += T * D * y_elem

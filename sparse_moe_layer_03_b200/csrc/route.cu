@@ -123,13 +123,14 @@ __device__ __forceinline__ void tile_partials(const float* psum, int tile, const
 // Work unit = a block of 16 consecutive tokens: their full rows (16 x D bf16,
 // one contiguous stretch of HBM, so DRAM pages are read whole) land in one
 // pair of shared-memory stages (one per half of the row, each one 3-D TMA box of
-// 64-column blocks x 16 rows, 128-byte swizzle).  One producer thread keeps the
-// stages in flight; each consumer warp owns two stages and takes every NC-th
-// row block: wait for a half, compute its part of the 16 x E logits with
-// mma.sync m16n8k16 (A via ldmatrix from the swizzled stage, B = gate weight in
-// shared memory with rows padded by 16 bytes), free that stage (the next load
-// overlaps the other half's MMAs), then run softmax and selection (one lane
-// per token).  No block-wide barrier inside the loop.
+// 64-column blocks x 16 rows, 128-byte swizzle).  Each warp owns two stages,
+// takes every NC-th row block and issues its own loads: wait for a half,
+// compute its part of the 16 x E logits with mma.sync m16n8k16 (A via ldmatrix
+// from the swizzled stage, B = gate weight in shared memory with rows padded by
+// 16 bytes), refill that stage with the next row block's half (the load
+// overlaps the other half's MMAs and the epilogue), then run softmax and
+// selection (one lane per token).  No block-wide barrier inside the loop and no
+// warp waits on another warp's progress.
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
@@ -147,12 +148,12 @@ __device__ __forceinline__ void mma_16816(float* d, uint32_t a0, uint32_t a1, ui
 }
 
 constexpr int kMmaRB = 16;        // tokens per row block
-constexpr int kMmaMaxConsumers = 4;
+constexpr int kMmaMaxConsumers = 6;
 
 // A row block is loaded as two halves (column blocks [0, hc) and [hc, 2hc), hc =
-// ceil(D/128)), each into its own stage; consumer warp c owns stages 2c and 2c+1
-// and waits on their phases strictly in order.  As many consumers (<= 4) as the
-// shared memory allows.
+// ceil(D/128)), each into its own stage; warp c owns stages 2c and 2c+1, issues
+// their loads itself and waits on their phases strictly in order.  As many warps
+// (<= 6) as the shared memory allows.
 struct MmaSmem {
   size_t wg, x, logits, misc, total;
   int consumers, hc;
@@ -247,7 +248,7 @@ __device__ bool last_block_done(unsigned int* ctr) {
 }
 
 template <int EMAX>
-__global__ void __launch_bounds__((kMmaMaxConsumers + 1) * 32, 1)
+__global__ void __launch_bounds__(kMmaMaxConsumers * 32, 1)
 route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, FinalizeArgs fin) {
   constexpr int NT = EMAX / 8;
   extern __shared__ uint8_t smem_raw[];
@@ -261,16 +262,15 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
   uint8_t* wg_s = smem + L.wg;
   uint8_t* xs = smem + L.x;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.misc);
-  uint64_t* empty = full + 2 * kMmaMaxConsumers;
-  int* cnt_s = reinterpret_cast<int*>(empty + 2 * kMmaMaxConsumers);
+  int* cnt_s = reinterpret_cast<int*>(full + 2 * kMmaMaxConsumers);
   float* wsum_s = reinterpret_cast<float*>(cnt_s + 32);
 
   const int nrb = (a.T + kMmaRB - 1) / kMmaRB;
   const int my_rb = (nrb - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-  // thread 0: half h of this CTA's j-th row block into stage 2 (j mod NC) + h
+  // lane 0 of warp w: half h of this CTA's j-th row block into the warp's stage 2w + h
   auto issue = [&](int j, int h) {
     const int rb = blockIdx.x + j * gridDim.x;
-    const int st = 2 * (j % NC) + h;
+    const int st = 2 * w + h;
     const int z0 = h * hc;
     const int nb = (nchunks - z0) < hc ? (nchunks - z0) : hc;     // blocks inside D
     const uint32_t bar = smem_u32(&full[st]);
@@ -284,13 +284,11 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
       for (int c = 0; c < nb; ++c) tma_load_2d(dst + c * (kMmaRB * 128), &tmap_x, (z0 + c) * 64, rb * kMmaRB, bar);
     }
   };
-  if (tid == 0) {
-    for (int st = 0; st < 2 * NC; ++st) {
-      mbar_init(smem_u32(&full[st]), 1);
-      mbar_init(smem_u32(&empty[st]), 1);   // the owning consumer warp, after its MMAs
-    }
+  if (lane == 0) {
+    mbar_init(smem_u32(&full[2 * w]), 1);
+    mbar_init(smem_u32(&full[2 * w + 1]), 1);
     fence_barrier_init();
-    for (int j = 0; j < NC && j < my_rb; ++j) { issue(j, 0); issue(j, 1); }   // x streams in while Wg loads
+    if (w < my_rb) { issue(w, 0); issue(w, 1); }   // x streams in while the gate weight loads
   }
   if (tid < 32) cnt_s[tid] = 0;
   {  // gate weight (bf16) -> padded rows; rows E..EMAX-1 are zero
@@ -309,95 +307,81 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
 #pragma unroll
   for (int e = 0; e < EMAX; ++e) psum[e] = 0.f;
   bool ok = true;
-  if (w == 0) {
-    // ------------------------------------------------ producer: refill each stage once it is free
-    if (lane == 0) {
-      for (int j = NC; j < my_rb && ok; ++j) {
-        const int k = j / NC;
-        for (int h = 0; h < 2; ++h) {
-          const int st = 2 * (j % NC) + h;
-          if (!mbar_wait(smem_u32(&empty[st]), (k - 1) & 1, nullptr, a.status, 104)) { ok = false; break; }
-          issue(j, h);
-        }
-      }
-    }
-  } else if (w <= NC) {
-    // ------------------------------------------------ consumer warp cw: row blocks j = cw, cw + NC, ...
-    const int cw = w - 1;
-    float* logit_w = reinterpret_cast<float*>(smem + L.logits) + (size_t)cw * kMmaRB * EMAX;
-    const uint32_t wg_base = smem_u32(wg_s);
-    const int li = lane >> 3, lj = lane & 7;
-    for (int j = cw; j < my_rb; j += NC) {
-      const int rb = blockIdx.x + j * gridDim.x;
-      const uint32_t parity = (j / NC) & 1;
-      // four independent accumulator chains (one per k16 step of a 64-column block)
-      float acc4[4][NT][4];
+  float* logit_w = reinterpret_cast<float*>(smem + L.logits) + (size_t)w * kMmaRB * EMAX;
+  const uint32_t wg_base = smem_u32(wg_s);
+  const int li = lane >> 3, lj = lane & 7;
+  for (int j = w, k = 0; j < my_rb; j += NC, ++k) {
+    const int rb = blockIdx.x + j * gridDim.x;
+    // four independent accumulator chains (one per k16 step of a 64-column block)
+    float acc4[4][NT][4];
 #pragma unroll
-      for (int g = 0; g < 4; ++g)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc4[g][nt][q] = 0.f;
-      for (int h = 0; h < 2 && ok; ++h) {
-        const int st = 2 * cw + h;
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), parity, nullptr, a.status, 100));
-        if (!ok) break;
-        const uint32_t buf = smem_u32(xs + (size_t)st * stage_bytes);
-        const int z0 = h * hc;
-        const int nb = (nchunks - z0) < hc ? (nchunks - z0) : hc;
-        for (int cb = 0; cb < nb; ++cb) {
-          const int c = z0 + cb;                       // global 64-column block
-          const uint32_t box = buf + cb * (kMmaRB * 128);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            uint32_t b[NT][2];
-            const int kc = c * 64 + ks * 16 + (li & 1) * 8;
-#pragma unroll
-            for (int np = 0; np < NT; np += 2) {
-              if (np + 1 < NT) {
-                const int n = (np + (li >> 1)) * 8 + lj;
-                ldsm_x4(wg_base + n * wg_stride + kc * 2, b[np][0], b[np][1], b[np + 1][0], b[np + 1][1]);
-              } else {
-                ldsm_x2(wg_base + (np * 8 + lj) * wg_stride + kc * 2, b[np][0], b[np][1]);
-              }
-            }
-            const int row = (li & 1) * 8 + lj;
-            const int chunk = ks * 2 + (li >> 1);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_16816(acc4[ks][nt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
-          }
-        }
-        __syncwarp();                                // every lane is done reading the stage
-        if (lane == 0) mbar_arrive(smem_u32(&empty[st]));   // the producer may refill it now
-      }
-      if (!ok) break;
-      float acc[NT][4];
+    for (int g = 0; g < 4; ++g)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc[nt][q] = (acc4[0][nt][q] + acc4[1][nt][q]) + (acc4[2][nt][q] + acc4[3][nt][q]);
+        for (int q = 0; q < 4; ++q) acc4[g][nt][q] = 0.f;
+    for (int h = 0; h < 2; ++h) {
+      const int st = 2 * w + h;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), k & 1, nullptr, a.status, 100));
+      if (!ok) break;
+      const uint32_t buf = smem_u32(xs + (size_t)st * stage_bytes);
+      const int z0 = h * hc;
+      const int nb = (nchunks - z0) < hc ? (nchunks - z0) : hc;
+      for (int cb = 0; cb < nb; ++cb) {
+        const int c = z0 + cb;                       // global 64-column block
+        const uint32_t box = buf + cb * (kMmaRB * 128);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int row = lane >> 2, col = nt * 8 + (lane & 3) * 2;
-        logit_w[row * EMAX + col] = acc[nt][0];
-        logit_w[row * EMAX + col + 1] = acc[nt][1];
-        logit_w[(row + 8) * EMAX + col] = acc[nt][2];
-        logit_w[(row + 8) * EMAX + col + 1] = acc[nt][3];
-      }
-      __syncwarp();
-      if (lane < kMmaRB) {
-        const int tok = rb * kMmaRB + lane;
-        if (tok < a.T) {
-          float l[EMAX];
+        for (int ks = 0; ks < 4; ++ks) {
+          uint32_t b[NT][2];
+          const int kc = c * 64 + ks * 16 + (li & 1) * 8;
 #pragma unroll
-          for (int e = 0; e < EMAX; ++e) l[e] = logit_w[lane * EMAX + e];
-          token_select<EMAX>(l, tok, a, cnt_s, psum);
+          for (int np = 0; np < NT; np += 2) {
+            if (np + 1 < NT) {
+              const int n = (np + (li >> 1)) * 8 + lj;
+              ldsm_x4(wg_base + n * wg_stride + kc * 2, b[np][0], b[np][1], b[np + 1][0], b[np + 1][1]);
+            } else {
+              ldsm_x2(wg_base + (np * 8 + lj) * wg_stride + kc * 2, b[np][0], b[np][1]);
+            }
+          }
+          const int row = (li & 1) * 8 + lj;
+          const int chunk = ks * 2 + (li >> 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma_16816(acc4[ks][nt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
         }
       }
-      __syncwarp();
+      __syncwarp();                                  // every lane is done reading the stage
+      if (lane == 0 && j + NC < my_rb) {             // refill it with the next row block's half
+        fence_async_shared();
+        issue(j + NC, h);
+      }
     }
+    if (!ok) break;
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[nt][q] = (acc4[0][nt][q] + acc4[1][nt][q]) + (acc4[2][nt][q] + acc4[3][nt][q]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int row = lane >> 2, col = nt * 8 + (lane & 3) * 2;
+      logit_w[row * EMAX + col] = acc[nt][0];
+      logit_w[row * EMAX + col + 1] = acc[nt][1];
+      logit_w[(row + 8) * EMAX + col] = acc[nt][2];
+      logit_w[(row + 8) * EMAX + col + 1] = acc[nt][3];
+    }
+    __syncwarp();
+    if (lane < kMmaRB) {
+      const int tok = rb * kMmaRB + lane;
+      if (tok < a.T) {
+        float l[EMAX];
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) l[e] = logit_w[lane * EMAX + e];
+        token_select<EMAX>(l, tok, a, cnt_s, psum);
+      }
+    }
+    __syncwarp();
   }
   __syncthreads();
   tile_partials<EMAX>(psum, blockIdx.x, a, cnt_s, wsum_s);
@@ -499,7 +483,7 @@ route_kernel_ffma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Final
 void route_plan(int T, int D, int E, int bf16, int sms, int* tile_rows, int* threads) {
   if (bf16) {
     *tile_rows = kMmaRB;
-    *threads = (mma_layout(D, E).consumers + 1) * 32;
+    *threads = mma_layout(D, E).consumers * 32;
   } else {
     int tile = (T + sms - 1) / sms;
     tile = (tile + 31) / 32 * 32;
@@ -524,7 +508,7 @@ cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUte
   if (a.E <= EM) {                                                                                      \
     err = cudaFuncSetAttribute(route_kernel_mma<EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (err != cudaSuccess) return err;                                                                 \
-    route_kernel_mma<EM><<<a.grid, (mma_layout(a.D, a.E).consumers + 1) * 32, smem, s>>>(*tm, a, fin);    \
+    route_kernel_mma<EM><<<a.grid, mma_layout(a.D, a.E).consumers * 32, smem, s>>>(*tm, a, fin);          \
     return cudaGetLastError();                                                                          \
   }
     MOE_ROUTE_MMA(8)

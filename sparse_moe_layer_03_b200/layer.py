@@ -126,3 +126,56 @@ class MoELayer:
 
     def check(self):
         B.moe_check_status(self.ws, self.stream())
+
+    # ------------------------------------------------------------ serving from host memory
+    def forward_host_pipelined(self, x_host, out_host, aux_host=None):
+        """Run the layer over a sequence of host batches, overlapping transfers with compute.
+
+        ``x_host`` / ``out_host`` are lists of pinned host tensors [T, D] (act dtype);
+        ``aux_host`` an optional list of pinned fp32 [1] tensors for each batch's balance
+        loss.  Batch i+1's host-to-device copy and batch i-1's device-to-host copy run on
+        their own streams while batch i computes (two device input and output buffers).
+        Returns when every copy back has finished.
+        """
+        n = len(x_host)
+        dev = self.device
+        if not hasattr(self, "_pipe"):
+            self._pipe = {
+                "x": [torch.empty((self.cfg.T, self.s.D), dtype=self.act_dtype, device=dev) for _ in range(2)],
+                "out": [torch.empty((self.cfg.T, self.s.D), dtype=self.act_dtype, device=dev) for _ in range(2)],
+                "aux": [torch.empty((1,), dtype=torch.float32, device=dev) for _ in range(2)],
+                "h2d": torch.cuda.Stream(dev), "d2h": torch.cuda.Stream(dev),
+            }
+        P = self._pipe
+        comp = torch.cuda.current_stream(dev)
+        loaded = [torch.cuda.Event() for _ in range(n)]
+        computed = [torch.cuda.Event() for _ in range(n)]
+        drained = [torch.cuda.Event() for _ in range(n)]
+        consumed = [torch.cuda.Event() for _ in range(n)]
+
+        def load(i):
+            with torch.cuda.stream(P["h2d"]):
+                if i >= 2:
+                    P["h2d"].wait_event(consumed[i - 2])      # buffer i%2 free again
+                P["x"][i % 2].copy_(x_host[i], non_blocking=True)
+                loaded[i].record(P["h2d"])
+
+        load(0)
+        for i in range(n):
+            if i + 1 < n:
+                load(i + 1)
+            comp.wait_event(loaded[i])
+            if i >= 2:
+                comp.wait_event(drained[i - 2])               # output buffer i%2 copied out
+            self.forward(P["x"][i % 2])
+            consumed[i].record(comp)
+            P["out"][i % 2].copy_(self.out)
+            P["aux"][i % 2].copy_(self.aux)
+            computed[i].record(comp)
+            with torch.cuda.stream(P["d2h"]):
+                P["d2h"].wait_event(computed[i])
+                out_host[i].copy_(P["out"][i % 2], non_blocking=True)
+                if aux_host is not None:
+                    aux_host[i].copy_(P["aux"][i % 2], non_blocking=True)
+                drained[i].record(P["d2h"])
+        drained[n - 1].synchronize()

@@ -30,6 +30,8 @@ SMALL = [
     (1000, 256, 512, 8, 2, 2, "bf16", "race"),
     (513, 128, 256, 16, 2, 1, "f32", "race"),
     (640, 64, 128, 32, 4, 2, "bf16", "topk"),
+    (1111, 192, 384, 8, 2, 1, "bf16", "topk"),     # odd number of 64-column blocks in the router
+    (900, 320, 640, 16, 3, 2, "bf16", "race"),
 ]
 
 
@@ -150,3 +152,19 @@ def test_named_workload_full_size(key):
     tokens = PA.sample_tokens(w.T, 256 if w.T > 4096 else w.T)
     rep = PA.full_check(w, inp, tokens=tokens)
     assert rep["err"] <= PA.out_tol(w)
+
+
+def test_pipelined_host_batches_match_device_forward():
+    # three different batches through the copy/compute-overlapped host path
+    w, inp = _small(700, 256, 512, 8, 2, 2, "bf16")
+    L, x = PA.run_layer(w, inp)
+    xs = [torch.randn((700, 256), generator=torch.Generator().manual_seed(i)).to(torch.bfloat16).pin_memory()
+          for i in range(3)]
+    outs = [torch.empty((700, 256), dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    auxs = [torch.empty((1,), dtype=torch.float32).pin_memory() for _ in range(3)]
+    L.forward_host_pipelined(xs, outs, auxs)
+    for i in range(3):
+        ref = L.forward(xs[i].to("cuda:0")).cpu()
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i], ref)
+        assert float(auxs[i][0]) == float(L.aux[0].cpu())

@@ -144,6 +144,58 @@ def balance_loss(counts, P, K, alpha):
     return float(alpha * np.sum(f * p))
 
 
+def balance_loss_per_sequence(idx, P, K, alpha, seq_len):
+    """Mean over images of L_balance with T read as one image's patch count.
+
+    "MOE-DIT", eq. L_balance calls T "the length of the image-patch
+    sequence".  A call holding B = T_call / seq_len images of seq_len tokens
+    each then has one loss per image, counts and score means taken over that
+    image's tokens only; this returns their mean.  seq_len = T_call gives
+    balance_loss over the whole call.
+    """
+    P = as_f64(P)
+    T, E = P.shape
+    if seq_len <= 0 or T % seq_len:
+        raise ValueError("seq_len must divide the token count")
+    idx = np.asarray(idx).reshape(T, -1)
+    per_image = []
+    for b in range(T // seq_len):
+        rows = slice(b * seq_len, (b + 1) * seq_len)
+        per_image.append(balance_loss(expert_counts(idx[rows], E), P[rows], K, alpha))
+    return float(np.mean(per_image))
+
+
+def expert_frequency(idx, E, labels, n_labels):
+    """hist[b, i] = number of selected pairs (t, i) whose token carries label b.
+
+    "Scaling Diffusion Transformers to 16 Billion Parameters", expert
+    specialisation analysis: expert-selection frequency counted by image
+    class, by spatial position and by denoising timestep.  labels[t] is the
+    label of token t: its patch position inside the image, or the class or
+    timestep of the image it belongs to.
+    """
+    idx = np.asarray(idx)
+    T = idx.shape[0]
+    idx = idx.reshape(T, -1)
+    labels = np.asarray(labels).reshape(T)
+    hist = np.zeros((n_labels, E), dtype=np.int64)
+    for t in range(T):
+        for i in idx[t]:
+            if i >= 0:
+                hist[labels[t], i] += 1
+    return hist
+
+
+def position_labels(T, seq_len):
+    """Label of token t by its patch position inside its image: t mod seq_len."""
+    return np.arange(T) % seq_len
+
+
+def image_labels(T, seq_len, per_image):
+    """Label of token t from the label of the image holding it (class or timestep)."""
+    return np.repeat(np.asarray(per_image), seq_len)[:T]
+
+
 # ---------------------------------------------------------------- experts
 
 def gelu_tanh(u):

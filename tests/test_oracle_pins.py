@@ -178,6 +178,69 @@ def test_worked_example_balance_and_race():
             assert abs(r["aux"] - want["loss"]) < 1e-15
 
 
+def test_worked_example_per_image_loss_and_frequencies():
+    g = json.load(open(os.path.join(GOLDEN, "balance_per_image_example.json")))
+    inp = {"x": _golden_x(g["a"]), "wg": np.array([[1.0, 0.0], [0.0, 0.0]])}
+    L, K, alpha = g["seq_len"], g["K"], g["alpha"]
+    for mode in ("topk", "race"):
+        r = O.route(inp, K, mode, alpha)
+        assert np.allclose(r["P"], g["P"], atol=1e-15)
+        idx = r["idx"][:, :1] if mode == "race" else r["idx"]
+        assert idx.tolist() == g["idx"], mode
+        assert abs(O.balance_loss_per_sequence(r["idx"], r["P"], K, alpha, L) - g["per_image"]["loss"]) < 1e-15
+        assert abs(r["aux"] - g["whole_call"]["loss"]) < 1e-15
+        T = r["P"].shape[0]
+        hp = O.expert_frequency(r["idx"], 2, O.position_labels(T, L), L)
+        assert hp.tolist() == g["position_hist"]["hist"]
+        ih = g["image_hist"]
+        hi = O.expert_frequency(r["idx"], 2, O.image_labels(T, L, ih["image_labels"]), ih["n_labels"])
+        want = np.zeros((ih["n_labels"], 2), dtype=np.int64)
+        for row, v in ih["rows"].items():
+            want[int(row)] = v
+        assert np.array_equal(hi, want)
+
+
+def test_per_image_loss_closed_forms():
+    # one image spanning the call is the whole-call loss
+    P = _rand_scores(48, 8, 21)
+    idx, _ = O.topk_route(P, 2)
+    whole = O.balance_loss(O.expert_counts(idx, 8), P, 2, 0.01)
+    assert abs(O.balance_loss_per_sequence(idx, P, 2, 0.01, 48) - whole) < 1e-15
+    # uniform scores: every image's loss is alpha, whatever the selection
+    Pu = np.full((64, 8), 1 / 8)
+    idx_u, _ = O.topk_route(Pu, 2)
+    assert abs(O.balance_loss_per_sequence(idx_u, Pu, 2, 0.01, 16) - 0.01) < 1e-15
+    # every image routes each expert equally often: alpha again, whatever the scores
+    E, K, L = 4, 1, 8
+    idx_b = np.tile(np.arange(E).repeat(L // E), 3).reshape(-1, 1)
+    Pb = _rand_scores(3 * L, E, 22)
+    assert abs(O.balance_loss_per_sequence(idx_b, Pb, K, 0.05, L) - 0.05) < 1e-15
+    with pytest.raises(ValueError):
+        O.balance_loss_per_sequence(idx, P, 2, 0.01, 5)
+
+
+@pytest.mark.parametrize("routing", ["topk", "race"])
+def test_frequency_marginals_and_relabelling(routing):
+    P = _rand_scores(96, 8, 23)
+    if routing == "race":
+        idx, _, _ = O.race_route(P, 2 * 96)
+    else:
+        idx, _ = O.topk_route(P, 2)
+    counts = O.expert_counts(idx, 8)
+    hp = O.expert_frequency(idx, 8, O.position_labels(96, 32), 32)
+    assert np.array_equal(hp.sum(0), counts)
+    img = [5, 0, 2]
+    hi = O.expert_frequency(idx, 8, O.image_labels(96, 32, img), 6)
+    assert np.array_equal(hi.sum(0), counts)
+    assert hi[1].sum() == 0 and hi[3].sum() == 0 and hi[4].sum() == 0
+    for b, lab in enumerate(img):   # an image's row is its own selection histogram
+        assert np.array_equal(hi[lab], O.expert_counts(idx[b * 32:(b + 1) * 32], 8))
+    # renaming the labels permutes the rows
+    perm = np.array([3, 1, 0, 2, 5, 4])
+    hi2 = O.expert_frequency(idx, 8, perm[O.image_labels(96, 32, img)], 6)
+    assert np.array_equal(hi2[perm], hi)
+
+
 # ------------------------------------------------------------------ experts
 
 def test_gelu_tanh_matches_library_and_identity():
@@ -361,3 +424,20 @@ def test_planted_race_tie_order_is_caught(monkeypatch):
     monkeypatch.setattr(O, "race_route", bad)
     with pytest.raises(AssertionError):
         test_worked_example_balance_and_race()
+
+
+def test_planted_per_image_token_count_is_caught(monkeypatch):
+    # a per-image loss that keeps the whole call's T in f and p
+    def wrong(idx, P, K, alpha, seq_len):
+        P = np.asarray(P, dtype=np.float64)
+        T, E = P.shape
+        idx = np.asarray(idx).reshape(T, -1)
+        out = []
+        for b in range(T // seq_len):
+            rows = slice(b * seq_len, (b + 1) * seq_len)
+            c = O.expert_counts(idx[rows], E)
+            out.append(alpha * np.sum((E / (K * T)) * c * P[rows].sum(0) / T))
+        return float(np.mean(out))
+    monkeypatch.setattr(O, "balance_loss_per_sequence", wrong)
+    with pytest.raises(AssertionError):
+        test_worked_example_per_image_loss_and_frequencies()

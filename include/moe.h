@@ -87,7 +87,10 @@ typedef struct {
   float alpha;       /* balance-loss factor (aux_loss_alpha) */
   int32_t act;       /* 0 = gelu tanh form (DiT core), 1 = exact erf form */
   int32_t gemm_impl; /* moe_gemm_impl_t */
-  int32_t reserved;  /* must be 0 */
+  int32_t seq_len;   /* tokens per image for the balance loss: 0 = the whole call is one
+                        sequence; L > 0 (L divides T) = mean over the T/L images of the loss
+                        taken over each image's tokens ("MOE-DIT": T in L_balance is the
+                        length of the image-patch sequence) */
 } moe_config_t;
 
 /* Library version (major*10000 + minor*100 + patch). */
@@ -125,7 +128,8 @@ int moe_check_status(void* ws, void* stream);
  *   n_sel       [T] int32 out or NULL  experts chosen per token (race:
  *               required, 0..E; top-K: K for every token)
  *   counts      [E] int32 out   sum_t I(t,i)
- *   aux_loss    [1] fp32 out    L_balance with T = this call's tokens
+ *   aux_loss    [1] fp32 out    L_balance with T = this call's tokens (seq_len = 0), or the
+ *               mean over images of L_balance with T = seq_len tokens per image
  * Race selection: the S = K*T largest scores of the flattened T x E matrix,
  * ties to the lower flat index t*E+i, found by an exact radix select on the
  * fp32 score bits.
@@ -221,6 +225,27 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,
 int moe_route_static(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
                      int32_t* topk_idx, float* topk_w, int32_t* n_sel, int32_t* counts, float* aux_loss,
                      void* stream);
+
+/*
+ * moe_expert_frequency -- expert-selection frequency per label, the statistic of
+ * the expert specialisation analysis ("Scaling Diffusion Transformers to 16
+ * Billion Parameters": selection frequency by image class, spatial position
+ * and denoising timestep).
+ *   topk_idx    [T,Kmax] int32   selection from moe_route (-1 = unused slot)
+ *   n_sel       [T] int32 or NULL  (race: required)
+ *   seq_len     tokens per image, >= 1, dividing T
+ *   seq_labels  [T/seq_len] int32 or NULL: the label of each image (its class,
+ *               or its timestep or timestep bucket).  NULL labels every token
+ *               by its patch position t mod seq_len.
+ *   n_labels    rows of hist (NULL seq_labels: must equal seq_len)
+ *   hist        [n_labels,E] int32 out: hist[b*E+i] = number of selected pairs
+ *               (t,i) whose token carries label b.  Overwritten.
+ *   ws          status word only (a label outside [0, n_labels) or an expert
+ *               id >= E is skipped and reported through moe_check_status)
+ * Integer counts: the result does not depend on the order of the atomics.
+ */
+int moe_expert_frequency(const moe_config_t* cfg, const int32_t* topk_idx, const int32_t* n_sel, int32_t seq_len,
+                         const int32_t* seq_labels, int32_t n_labels, int32_t* hist, void* ws, void* stream);
 
 #ifdef __cplusplus
 }

@@ -59,7 +59,9 @@ int validate(const moe_config_t* c) {
   if (c->routing != MOE_ROUTE_TOPK && c->routing != MOE_ROUTE_RACE) return fail(MOE_ERR_INVALID_ARG, "routing=%d", c->routing);
   if (c->act != 0 && c->act != 1) return fail(MOE_ERR_INVALID_ARG, "act=%d", c->act);
   if (c->gemm_impl < MOE_GEMM_AUTO || c->gemm_impl > MOE_GEMM_TC1) return fail(MOE_ERR_INVALID_ARG, "gemm_impl=%d", c->gemm_impl);
-  if (c->reserved != 0) return fail(MOE_ERR_INVALID_ARG, "reserved field must be 0");
+  if (c->seq_len < 0) return fail(MOE_ERR_INVALID_ARG, "seq_len=%d < 0", c->seq_len);
+  if (c->seq_len > 0 && c->T % c->seq_len)
+    return fail(MOE_ERR_INVALID_ARG, "seq_len=%d does not divide T=%d", c->seq_len, c->T);
   if (route_smem_total(c->D, c->E, 32, c->dtype == MOE_BF16) > 232448 ||
       (c->dtype == MOE_BF16 && route_mma_stages(c->D, c->E) < 1))
     return fail(MOE_ERR_UNSUPPORTED, "E=%d x D=%d too large for the router's shared memory", c->E, c->D);
@@ -73,17 +75,13 @@ long long max_rows(const moe_config_t* c) {
   return (long long)round_up((size_t)(S + (long long)(kSegAlign - 1) * c->E), kSegAlign);
 }
 
-// dispatch chunking: at most 1024 chunks of >= 64 tokens (a multiple of 32)
-void chunking(int T, int* chunk, int* nchunks) {
-  int ch = (T + 1023) / 1024;
-  ch = (ch + 31) / 32 * 32;
-  if (ch < 64) ch = 64;
-  *chunk = ch;
-  *nchunks = (T + ch - 1) / ch;
-}
+// dispatch: groups of 256 tokens (counts and ranks), 64 tokens per gather block
+constexpr int kDispatchGroup = 256;
+constexpr int kGatherTokens = 64;
+int ngroups_of(int T) { return (T + kDispatchGroup - 1) / kDispatchGroup; }
 
 struct WsLayout {
-  size_t status, tile_counts, tile_psum, P, hist, state, tile_eq, race_counts, chunk_base, total;
+  size_t status, tile_counts, tile_psum, P, seq_loss, race_sync, race_loc, race_counts, group_base, total;
 };
 
 WsLayout ws_layout(const moe_config_t* c) {
@@ -91,21 +89,19 @@ WsLayout ws_layout(const moe_config_t* c) {
   const size_t T = (size_t)c->T, E = (size_t)c->E;
   // partial rows: one per router CTA (<= one per 16 tokens) or per fp32 token tile (>= 32 rows)
   const size_t max_route_tiles = (T + 15) / 16 + 1;
-  const size_t race_tiles = (T + 127) / 128 + 1;
-  int ch, nch;
-  chunking(c->T, &ch, &nch);
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off += round_up(bytes ? bytes : 1, 256); return o; };
   L.status = take(256);
   L.tile_counts = take(max_route_tiles * E * 4);
   L.tile_psum = take(max_route_tiles * E * 4);
   const bool race = c->routing == MOE_ROUTE_RACE;
-  L.P = take(race ? T * E * 4 : 0);
-  L.hist = take(race ? 4096 * 4 : 0);
-  L.state = take(race ? 16 : 0);
-  L.tile_eq = take(race ? race_tiles * 4 : 0);
-  L.race_counts = take(race ? race_tiles * E * 4 : 0);
-  L.chunk_base = take((size_t)(nch + 1) * E * 4);
+  const bool per_image = c->seq_len > 0;
+  L.P = take(race || per_image ? T * E * 4 : 0);
+  L.seq_loss = take(per_image ? (T / (size_t)c->seq_len) * 8 : 0);
+  L.race_sync = take(race ? (size_t)kRaceSyncWords * 4 : 0);
+  L.race_loc = take(race ? (size_t)kRaceMaxCtas * 256 * 4 : 0);
+  L.race_counts = take(race ? (size_t)kRaceMaxCtas * E * 4 : 0);
+  L.group_base = take((size_t)ngroups_of(c->T) * E * 4);
   L.total = off;
   return L;
 }
@@ -283,7 +279,16 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   ra.T = cfg->T; ra.D = cfg->D; ra.E = cfg->E; ra.K = cfg->K; ra.bf16 = bf16;
   ra.tile_rows = tile; ra.ntiles = ntiles; ra.grid = grid;
   ra.topk_idx = topk_idx; ra.topk_w = topk_w; ra.n_sel = race ? nullptr : n_sel;
-  ra.P = race ? ws_at<float>(ws, L.P) : nullptr;
+  const bool per_image = cfg->seq_len > 0;
+  ra.P = race || per_image ? ws_at<float>(ws, L.P) : nullptr;
+  ra.race = race;
+  SeqLossArgs sl{};
+  sl.P = ra.P; sl.topk_idx = topk_idx; sl.n_sel = n_sel;
+  sl.T = cfg->T; sl.E = cfg->E; sl.K = cfg->K; sl.Kmax = kmax_of(cfg); sl.L = cfg->seq_len;
+  sl.alpha = cfg->alpha;
+  sl.seq_loss = per_image ? ws_at<double>(ws, L.seq_loss) : nullptr;
+  sl.ctr = ws_at<unsigned int>(ws, 192);
+  sl.aux_loss = aux_loss;
   ra.tile_counts = ws_at<int32_t>(ws, L.tile_counts);
   ra.tile_psum = ws_at<float>(ws, L.tile_psum);
   ra.status = status_ptr(ws);
@@ -296,25 +301,55 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   if (!race) {
     // the router's last block finalizes counts and loss
     if ((e = launch_route(ra, fa, &tm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
+    if (per_image && (e = launch_seq_loss(sl, s)) != cudaSuccess) return cuda_fail(e, "per-image loss kernel");
     return ok();
   }
+  // Expert-Race: the router writes the score matrix (and clears the selection's
+  // scratch); one cooperative launch selects and finalizes.
+  ra.zero = ws_at<uint32_t>(ws, L.race_sync);
+  ra.nzero = kRaceSyncWords;
   FinalizeArgs none{};
   if ((e = launch_route(ra, none, &tm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
-  {
-    RaceArgs rr{};
-    rr.P = ra.P; rr.T = cfg->T; rr.E = cfg->E; rr.K = cfg->K;
-    rr.hist = ws_at<uint32_t>(ws, L.hist);
-    rr.state = ws_at<uint32_t>(ws, L.state);
-    rr.tile_eq = ws_at<uint32_t>(ws, L.tile_eq);
-    rr.ntiles = (cfg->T + 127) / 128;
-    rr.topk_idx = topk_idx; rr.topk_w = topk_w; rr.n_sel = n_sel;
-    rr.tile_counts = ws_at<int32_t>(ws, L.race_counts);
-    rr.status = status_ptr(ws);
-    if ((e = cudaMemsetAsync(rr.hist, 0, 4096 * 4, s)) != cudaSuccess) return cuda_fail(e, "moe_route");
-    if ((e = launch_race_select(rr, s)) != cudaSuccess) return cuda_fail(e, "race select kernels");
-    fa.tile_counts = rr.tile_counts; fa.ntiles_counts = rr.ntiles;
+  RaceArgs rr{};
+  rr.P = ra.P; rr.T = cfg->T; rr.E = cfg->E; rr.K = cfg->K;
+  rr.sync = ra.zero;
+  rr.loc = ws_at<uint32_t>(ws, L.race_loc);
+  rr.grid = race_plan(cfg->T, sms, &rr.tpc);
+  rr.topk_idx = topk_idx; rr.topk_w = topk_w; rr.n_sel = n_sel;
+  rr.tile_counts = ws_at<int32_t>(ws, L.race_counts);
+  rr.status = status_ptr(ws);
+  fa.tile_counts = rr.tile_counts; fa.ntiles_counts = rr.grid;
+  if ((e = launch_race_select(rr, fa, s)) != cudaSuccess) return cuda_fail(e, "Expert-Race select kernel");
+  if (per_image && (e = launch_seq_loss(sl, s)) != cudaSuccess) return cuda_fail(e, "per-image loss kernel");
+  return ok();
+}
+
+int moe_expert_frequency(const moe_config_t* cfg, const int32_t* topk_idx, const int32_t* n_sel, int32_t seq_len,
+                         const int32_t* seq_labels, int32_t n_labels, int32_t* hist, void* ws, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (seq_len < 1) return fail(MOE_ERR_INVALID_ARG, "seq_len=%d < 1", seq_len);
+  if (cfg->T % seq_len) return fail(MOE_ERR_INVALID_ARG, "seq_len=%d does not divide T=%d", seq_len, cfg->T);
+  if (n_labels < 1 || (long long)n_labels * cfg->E > (1ll << 30))
+    return fail(MOE_ERR_INVALID_ARG, "n_labels=%d outside 1..2^30/E", n_labels);
+  if (!seq_labels && n_labels != seq_len)
+    return fail(MOE_ERR_INVALID_ARG, "position labels need n_labels == seq_len (%d != %d)", n_labels, seq_len);
+  REQUIRE_PTR(hist);
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "ws is NULL");
+  if ((uintptr_t)ws & 255u) return fail(MOE_ERR_INVALID_ARG, "ws must be 256-byte aligned");
+  if (cfg->T > 0) {
+    REQUIRE_PTR(topk_idx);
+    OPTIONAL_PTR(n_sel);
+    OPTIONAL_PTR(seq_labels);
+    if (cfg->routing == MOE_ROUTE_RACE && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
   }
-  if ((e = launch_route_finalize(fa, s)) != cudaSuccess) return cuda_fail(e, "route finalize kernel");
+  FreqArgs fa{};
+  fa.topk_idx = topk_idx; fa.n_sel = n_sel;
+  fa.T = cfg->T; fa.E = cfg->E; fa.K = cfg->K; fa.Kmax = kmax_of(cfg); fa.L = seq_len;
+  fa.labels = seq_labels; fa.n_labels = n_labels; fa.hist = hist;
+  fa.status = status_ptr(ws);
+  cudaError_t e = launch_frequency(fa, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "frequency kernel");
   return ok();
 }
 
@@ -349,9 +384,11 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx
   da.x = x; da.bf16 = cfg->dtype == MOE_BF16;
   da.topk_idx = topk_idx; da.topk_w = topk_w; da.n_sel = n_sel;
   da.T = cfg->T; da.D = cfg->D; da.E = cfg->E; da.K = cfg->K; da.Kmax = kmax_of(cfg);
-  chunking(cfg->T, &da.chunk, &da.nchunks);
+  da.ngroups = ngroups_of(cfg->T);
+  da.tpb = kGatherTokens;
   da.r_max = R;
-  da.chunk_base = ws_at<int32_t>(ws, L.chunk_base);
+  da.group_base = ws_at<int32_t>(ws, L.group_base);
+  da.ctr = ws_at<unsigned int>(ws, 128);
   da.offsets = offsets; da.pos = pos; da.row_token = row_token; da.row_gate = row_gate;
   da.x_perm = x_perm;
   da.status = status_ptr(ws);

@@ -7,158 +7,248 @@
 // from integer counts and prefix sums only (no order-dependent atomics), so
 // the permutation is deterministic and equals the canonical one bit for bit.
 //
-//   count kernel  (1 block per chunk of tokens): per-chunk expert counts.
-//   gather kernel (1 block per chunk): sums of the chunk counts give the
-//                 padded segment starts and the chunk's base in each segment;
-//                 ranks inside the chunk by warp ballots; positions; padding
-//                 rows marked; 16-byte row copies x -> x_perm.
+//   count kernel  (one block per group of 256 tokens): the group's count per
+//                 expert, and each slot's rank among the group's slots of the
+//                 same expert (warp ballots), parked in `pos`.  The block that
+//                 finishes last scans the group counts into each group's first
+//                 row in every segment, writes the offsets and marks the
+//                 padding rows.
+//   gather kernel (64 tokens per block): one thread per slot turns ranks into
+//                 rows (group base + rank) and writes pos, row_token and
+//                 row_gate; then one warp per token loads the row and stores
+//                 it once per selected expert with 16-byte vectors (each
+//                 warp's first row loads while the rows are worked out).
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
 
-constexpr int kGatherThreads = 256;
+constexpr int kDispatchThreads = 256;
+constexpr int kGroup = kDispatchThreads;      // tokens per group: one count block, one token per thread
 
-// per-chunk expert counts, expert-major: cnt[e * nchunks + c]
-__global__ void __launch_bounds__(kGatherThreads) dispatch_count_kernel(DispatchArgs a) {
-  __shared__ int cc[32];
-  const int tid = threadIdx.x, c = blockIdx.x, Kmax = a.Kmax;
-  if (tid < 32) cc[tid] = 0;
-  __syncthreads();
-  const int t0 = c * a.chunk;
-  const int n = min(a.chunk, a.T - t0) * Kmax;
-  for (int i = tid; i < n; i += kGatherThreads) {
-    const int t = t0 + i / Kmax, k = i % Kmax;
-    const int ns = a.n_sel ? a.n_sel[t] : a.K;
-    if (k >= ns) continue;
-    const int e = a.topk_idx[(size_t)t0 * Kmax + i];
-    if (e >= 0 && e < a.E) atomicAdd(&cc[e], 1);
-  }
-  __syncthreads();
-  if (tid < a.E) a.chunk_base[(size_t)tid * a.nchunks + c] = cc[tid];
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
 }
 
-template <typename T, int EMAX>
-__global__ void __launch_bounds__(kGatherThreads) dispatch_gather_kernel(DispatchArgs a) {
-  extern __shared__ int sm[];
-  const int Kmax = a.Kmax, E = a.E, CH = a.chunk;
-  int* sidx = sm;                     // [CH][Kmax] expert of each slot (-1 unused)
-  int* spos = sm + CH * Kmax;         // [CH][Kmax] rank in warp, then row
-  __shared__ int wcnt[kGatherThreads / 32][EMAX];
-  __shared__ int before_s[EMAX], total_s[EMAX], poff_s[EMAX + 1];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int c = blockIdx.x;
-  const int t0 = c * CH;
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
 
-  // ---- segment starts and this chunk's base: sums over the chunk counts
-  for (int e = w; e < E; e += kGatherThreads / 32) {
-    const int* row = a.chunk_base + (size_t)e * a.nchunks;
-    int before = 0, total = 0;
-#pragma unroll 4
-    for (int j = lane; j < a.nchunks; j += 32) {
-      const int v = row[j];
-      total += v;
-      before += j < c ? v : 0;
+// Segment bases from the group counts; run by the last block of the count kernel.
+// cnt[e * ngroups + g] (counts in, first row of group g in segment e out).
+// Warp w takes experts w, w + 8, ...; its lanes read 32 consecutive groups per
+// load (coalesced), eight loads in flight.
+__device__ void dispatch_scan_groups(const DispatchArgs& a) {
+  __shared__ int total_s[32], poff_s[33];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, NW = kDispatchThreads / 32;
+  const int E = a.E, ng = a.ngroups;
+  int32_t* cnt = a.group_base;
+  // 1. per-expert totals
+  for (int e = w; e < E; e += NW) {
+    const int32_t* row = cnt + (size_t)e * ng;
+    int sum = 0;
+    for (int g0 = 0; g0 < ng; g0 += 8 * 32) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int g = g0 + u * 32 + lane;
+        v[u] = g < ng ? __ldcg(row + g) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += v[u];
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      total += __shfl_xor_sync(0xffffffffu, total, o);
-      before += __shfl_xor_sync(0xffffffffu, before, o);
-    }
-    if (lane == 0) { total_s[e] = total; before_s[e] = before; }
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) total_s[e] = sum;
   }
   __syncthreads();
   if (tid == 0) {
-    int p = 0;
-    for (int e = 0; e < E; ++e) { poff_s[e] = p; p += (total_s[e] + kSegAlign - 1) / kSegAlign * kSegAlign; }
+    int p = 0, u = 0;
+    for (int e = 0; e < E; ++e) {
+      poff_s[e] = p;
+      a.offsets[e] = u;
+      u += total_s[e];
+      p += (total_s[e] + kSegAlign - 1) / kSegAlign * kSegAlign;
+    }
     poff_s[E] = p;
+    a.offsets[E] = u;
   }
   __syncthreads();
-  if (c == 0 && tid <= E) {
-    int u = 0;
-    for (int e = 0; e < tid; ++e) u += total_s[e];
-    a.offsets[tid] = u;
+  // 2. exclusive scan over the groups of each segment, from the segment's start
+  for (int e = w; e < E; e += NW) {
+    int32_t* row = cnt + (size_t)e * ng;
+    int carry = poff_s[e];
+    for (int g0 = 0; g0 < ng; g0 += 8 * 32) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int g = g0 + u * 32 + lane;
+        v[u] = g < ng ? __ldcg(row + g) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int g = g0 + u * 32 + lane;
+        const int incl = warp_incl_scan(v[u], lane);
+        if (g < ng) row[g] = carry + incl - v[u];
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
   }
-  // padding rows: segment e's tail (e < E) or the rows after the last segment (e = E)
-  for (int e = c; e <= E; e += gridDim.x) {
+  // 3. padding rows: segment e's tail (e < E) or the rows after the last segment (e = E)
+  for (int e = 0; e <= E; ++e) {
     const long long lo = e < E ? (long long)poff_s[e] + total_s[e] : poff_s[E];
     const long long hi = e < E ? (long long)poff_s[e + 1] : a.r_max;
-    for (long long r = lo + tid; r < hi; r += kGatherThreads) {
+    for (long long r = lo + tid; r < hi; r += kDispatchThreads) {
       a.row_token[r] = -1;
       a.row_gate[r] = 0.f;
     }
   }
+}
 
-  // ---- slots of this chunk
-  for (int i = tid; i < CH * Kmax; i += kGatherThreads) {
-    const int l = i / Kmax, k = i % Kmax, t = t0 + l;
+// One group of kGroup tokens per block, one token per thread: the group's count
+// per expert, and each slot's rank among the group's slots of the same expert
+// (rank inside the warp from a ballot, plus the counts of the earlier warps).
+template <int EMAX>
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_count_kernel(DispatchArgs a) {
+  constexpr int NW = kDispatchThreads / 32;
+  __shared__ uint32_t bal[NW][EMAX];
+  __shared__ int wbase[NW][EMAX];
+  __shared__ bool last;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int g = blockIdx.x;
+  const int Kmax = a.Kmax, E = a.E;
+  const int t = g * kGroup + tid;
+  const bool valid = t < a.T;
+  const int ns = valid ? (a.n_sel ? a.n_sel[t] : a.K) : 0;
+  int ek[EMAX];
+  uint32_t m = 0;
+#pragma unroll
+  for (int k = 0; k < EMAX; ++k) {
     int e = -1;
-    if (t < a.T) {
-      const int ns = a.n_sel ? a.n_sel[t] : a.K;
-      if (k < ns) {
-        e = a.topk_idx[(size_t)t * Kmax + k];
-        if (e >= E) { set_status(a.status, DEV_BAD_INDEX, 200); e = -1; }
-      }
+    if (k < Kmax && k < ns) {
+      e = a.topk_idx[(size_t)t * Kmax + k];
+      if (e >= E) { set_status(a.status, DEV_BAD_INDEX, 200); e = -1; }
+      else if (e >= 0 && ((m >> e) & 1u)) { set_status(a.status, DEV_BAD_INDEX, 202); e = -1; }   // repeated expert
+      if (e >= 0) m |= 1u << e;
     }
-    sidx[i] = e < 0 ? -1 : e;
-    spos[i] = -1;
+    ek[k] = e < 0 ? -1 : e;
   }
-  __syncthreads();
-  // ---- rank of each token among the chunk's tokens of the same expert (token order)
-  if (w < CH / 32) {
-    const int l = w * 32 + lane;
-    for (int e = 0; e < E; ++e) {
-      int slot = -1;
-      for (int k = 0; k < Kmax; ++k)
-        if (sidx[l * Kmax + k] == e) slot = k;
-      const unsigned mask = __ballot_sync(0xffffffffu, slot >= 0);
-      if (slot >= 0) spos[l * Kmax + slot] = __popc(mask & ((1u << lane) - 1u));
-      if (lane == 0) wcnt[w][e] = __popc(mask);
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) {
+    if (e < E) {
+      const uint32_t b = __ballot_sync(0xffffffffu, (m >> e) & 1u);
+      if (lane == 0) bal[w][e] = b;
     }
   }
   __syncthreads();
-  for (int i = tid; i < CH * Kmax; i += kGatherThreads) {
-    const int l = i / Kmax, k = i % Kmax, t = t0 + l;
-    if (t >= a.T) continue;
-    const int e = sidx[i];
+  if (tid < E) {
+    int run = 0;
+#pragma unroll
+    for (int v = 0; v < NW; ++v) {
+      wbase[v][tid] = run;
+      run += __popc(bal[v][tid]);
+    }
+    a.group_base[(size_t)tid * a.ngroups + g] = run;
+  }
+  __syncthreads();
+  const uint32_t lt = lanemask_lt();
+#pragma unroll
+  for (int k = 0; k < EMAX; ++k)
+    if (k < Kmax && valid)
+      a.pos[(size_t)t * Kmax + k] = ek[k] >= 0 ? wbase[w][ek[k]] + __popc(bal[w][ek[k]] & lt) : -1;
+  // the last block to finish turns the counts into segment bases
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned int prev = atomicAdd(a.ctr, 1u);
+    last = prev == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  dispatch_scan_groups(a);
+  if (tid == 0) *a.ctr = 0u;                            // ready for the next call
+}
+
+// One row copy: P x 32 lanes x 16 bytes covers up to P*32 vectors of the row.
+template <int P>
+__device__ __forceinline__ void load_row(const uint4* src, int nvec, int lane, uint4* buf) {
+#pragma unroll
+  for (int u = 0; u < P; ++u) {
+    const int v = u * 32 + lane;
+    if (v < nvec) buf[u] = src[v];
+  }
+}
+template <int P>
+__device__ __forceinline__ void store_row(uint4* dst, int nvec, int lane, const uint4* buf) {
+#pragma unroll
+  for (int u = 0; u < P; ++u) {
+    const int v = u * 32 + lane;
+    if (v < nvec) dst[v] = buf[u];
+  }
+}
+
+// Gather block: tokens [t0, t0 + tpb).  Phase 1, one thread per slot, all
+// slots of the block at once: row = group base + rank inside the group; writes
+// pos, row_token, row_gate and keeps the row in shared memory.  Phase 2, one
+// warp per token: row loads, then one store of the row per selected slot.  Each
+// warp's first row is already loading while phase 1 runs.
+template <typename T, int P>
+__device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int Kmax = a.Kmax;
+  const int nvec = a.D * (int)sizeof(T) / 16;
+  const int t0 = blockIdx.x * a.tpb;
+  const int nt = min(a.tpb, a.T - t0);
+  const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+  uint4* xp = reinterpret_cast<uint4*>(a.x_perm);
+  uint4 buf[P > 0 ? P : 1];
+  if (P > 0 && w < nt) load_row<P>(xv + (size_t)(t0 + w) * nvec, nvec, lane, buf);
+
+  for (int i = tid; i < nt * Kmax; i += kDispatchThreads) {
+    const int t = t0 + i / Kmax, k = i % Kmax;
+    const size_t slot = (size_t)t0 * Kmax + i;
+    const int ns = a.n_sel ? a.n_sel[t] : a.K;
     int p = -1;
-    if (e >= 0) {
-      int base = poff_s[e] + before_s[e];
-      for (int ww = 0; ww < l / 32; ++ww) base += wcnt[ww][e];
-      p = base + spos[i];
-      if (p < 0 || p >= a.r_max) { set_status(a.status, DEV_BAD_INDEX, 201); p = -1; }
-      else {
-        a.row_token[p] = t;
-        a.row_gate[p] = a.topk_w[(size_t)t * Kmax + k];
+    if (k < ns) {
+      const int e = a.topk_idx[slot];
+      const int r = a.pos[slot];
+      if (e >= 0 && e < a.E && r >= 0) {
+        p = a.group_base[(size_t)e * a.ngroups + t / kGroup] + r;
+        if (p < 0 || p >= a.r_max) { set_status(a.status, DEV_BAD_INDEX, 201); p = -1; }
+        else {
+          a.row_token[p] = t;
+          a.row_gate[p] = a.topk_w[slot];
+        }
       }
     }
-    a.pos[(size_t)t * Kmax + k] = p;
+    a.pos[slot] = p;
     spos[i] = p;
   }
   __syncthreads();
-  // ---- row copies: one warp per token, 16-byte vectors
-  const int nvec = a.D * (int)sizeof(T) / 16;
-  const uint4* xv = reinterpret_cast<const uint4*>(a.x);
-  uint4* xp = reinterpret_cast<uint4*>(a.x_perm);
-  for (int l = w; l < CH; l += kGatherThreads / 32) {
-    const int t = t0 + l;
-    if (t >= a.T) break;
-    const uint4* src = xv + (size_t)t * nvec;
-    for (int v0 = 0; v0 < nvec; v0 += 32 * 4) {
-      uint4 buf[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int v = v0 + u * 32 + lane;
-        if (v < nvec) buf[u] = src[v];
-      }
+
+  for (int l = w; l < nt; l += kDispatchThreads / 32) {
+    const uint4* src = xv + (size_t)(t0 + l) * nvec;
+    if (P > 0) {
+      if (l != w) load_row<P>(src, nvec, lane, buf);
       for (int k = 0; k < Kmax; ++k) {
         const int p = spos[l * Kmax + k];
-        if (p < 0) continue;
-        uint4* dst = xp + (size_t)p * nvec;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int v = v0 + u * 32 + lane;
-          if (v < nvec) dst[v] = buf[u];
+        if (p >= 0) store_row<P>(xp + (size_t)p * nvec, nvec, lane, buf);
+      }
+    } else {
+      for (int v0 = 0; v0 < nvec; v0 += 8 * 32) {      // wide rows: pieces of 8 vectors per lane
+        uint4 piece[8];
+        load_row<8>(src + v0, nvec - v0, lane, piece);
+        for (int k = 0; k < Kmax; ++k) {
+          const int p = spos[l * Kmax + k];
+          if (p >= 0) store_row<8>(xp + (size_t)p * nvec + v0, nvec - v0, lane, piece);
         }
       }
     }
@@ -166,24 +256,26 @@ __global__ void __launch_bounds__(kGatherThreads) dispatch_gather_kernel(Dispatc
 }
 
 template <typename T>
-static cudaError_t launch_gather_t(const DispatchArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)2 * a.chunk * a.Kmax * sizeof(int);
-  cudaError_t err = cudaSuccess;
-  if (a.E <= 8) err = cudaFuncSetAttribute(dispatch_gather_kernel<T, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  else if (a.E <= 16) err = cudaFuncSetAttribute(dispatch_gather_kernel<T, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  else err = cudaFuncSetAttribute(dispatch_gather_kernel<T, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  if (a.E <= 8) dispatch_gather_kernel<T, 8><<<a.nchunks, kGatherThreads, smem, s>>>(a);
-  else if (a.E <= 16) dispatch_gather_kernel<T, 16><<<a.nchunks, kGatherThreads, smem, s>>>(a);
-  else dispatch_gather_kernel<T, 32><<<a.nchunks, kGatherThreads, smem, s>>>(a);
-  return cudaGetLastError();
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(DispatchArgs a) {
+  extern __shared__ int spos[];                       // [tpb * Kmax] rows of the block's slots
+  const int nvec = a.D * (int)sizeof(T) / 16;
+  if (nvec <= 4 * 32) gather_block<T, 4>(a, spos);
+  else if (nvec <= 8 * 32) gather_block<T, 8>(a, spos);
+  else gather_block<T, 0>(a, spos);
 }
 
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
-  dispatch_count_kernel<<<a.nchunks, kGatherThreads, 0, s>>>(a);
+  const int cgrid = a.ngroups;
+  if (a.E <= 8) dispatch_count_kernel<8><<<cgrid, kDispatchThreads, 0, s>>>(a);
+  else if (a.E <= 16) dispatch_count_kernel<16><<<cgrid, kDispatchThreads, 0, s>>>(a);
+  else dispatch_count_kernel<32><<<cgrid, kDispatchThreads, 0, s>>>(a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  return a.bf16 ? launch_gather_t<__nv_bfloat16>(a, s) : launch_gather_t<float>(a, s);
+  const int ggrid = (a.T + a.tpb - 1) / a.tpb;
+  const size_t smem = (size_t)a.tpb * a.Kmax * sizeof(int);
+  if (a.bf16) dispatch_gather_kernel<__nv_bfloat16><<<ggrid, kDispatchThreads, smem, s>>>(a);
+  else dispatch_gather_kernel<float><<<ggrid, kDispatchThreads, smem, s>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace moe

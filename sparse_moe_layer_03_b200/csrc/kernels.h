@@ -23,9 +23,12 @@ struct RouteArgs {
   int32_t* topk_idx;        // top-K mode: [T,K]
   float* topk_w;
   int32_t* n_sel;           // may be null (top-K)
-  float* P;                 // race: [T,E] scores (scratch), else null
+  float* P;                 // [T,E] scores (scratch) for Expert-Race or per-image losses, else null
+  int race;                 // 1: P only, the selection happens later
   int32_t* tile_counts;     // [ntiles,E] (top-K)
   float* tile_psum;         // [ntiles,E]
+  uint32_t* zero;           // block 0 clears zero[0, nzero) first (the Expert-Race scratch), or null
+  int nzero;
   int* status;
 };
 size_t route_smem_bytes(int D, int E, int tile_rows, int bf16);
@@ -42,31 +45,62 @@ struct FinalizeArgs {
   unsigned int* ctr;                  // blocks-done counter in ws (zero between calls)
 };
 cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tmap_x, cudaStream_t s);
-cudaError_t launch_route_finalize(const FinalizeArgs& a, cudaStream_t s);
 
+// per-image balance loss (seq_len > 0): overwrites aux_loss with the mean over images
+struct SeqLossArgs {
+  const float* P;               // [T,E] scores
+  const int32_t* topk_idx;      // [T,Kmax]
+  const int32_t* n_sel;         // [T] or null
+  int T, E, K, Kmax, L;
+  float alpha;
+  double* seq_loss;             // [T/L] scratch
+  unsigned int* ctr;            // blocks-done counter in ws (zero between calls)
+  float* aux_loss;
+};
+cudaError_t launch_seq_loss(const SeqLossArgs& a, cudaStream_t s);
+
+// ---- stats.cu: expert-selection frequency per label
+struct FreqArgs {
+  const int32_t* topk_idx; const int32_t* n_sel;
+  int T, E, K, Kmax, L;
+  const int32_t* labels;        // [T/L] or null (label = t mod L)
+  int n_labels;
+  int32_t* hist;                // [n_labels,E]
+  int* status;
+};
+cudaError_t launch_frequency(const FreqArgs& a, cudaStream_t s);
+
+// Expert-Race selection: one cooperative launch of `grid` CTAs (at most one per
+// SM), CTA r owning tokens [r*tpc, (r+1)*tpc)
+constexpr int kRaceMaxCtas = 256;
+constexpr int kRaceSyncWords = 4096 + 4096 + 256 + 16;   // digit histograms 1..3, grid-barrier counter
 struct RaceArgs {
-  const float* P;           // [T,E]
+  const float* P;           // [T,E] scores
   int T, E, K;
-  uint32_t* hist;           // [4096] scratch, zeroed by the caller before pass 0
-  uint32_t* state;          // [4] scratch: prefix, need, threshold bits, need_eq
-  uint32_t* tile_eq;        // [ntiles]
-  int ntiles;               // ceil(T/128)
+  uint32_t* sync;           // [kRaceSyncWords], zero on entry (the router clears it)
+  uint32_t* loc;            // [grid,256] per-CTA histograms of the last digit
+  int grid, tpc;            // CTAs; tokens per CTA (a multiple of 4)
   int32_t* topk_idx;        // [T,E]
   float* topk_w;            // [T,E]
   int32_t* n_sel;           // [T]
-  int32_t* tile_counts;     // [ntiles,E]
+  int32_t* tile_counts;     // [grid,E]
   int* status;
 };
-cudaError_t launch_race_select(const RaceArgs& a, cudaStream_t s);
+// CTAs for T tokens on `sms` SMs; *tpc = tokens per CTA
+int race_plan(int T, int sms, int* tpc);
+// selection, per-CTA counts, then the last CTA turns counts and score sums into counts[E] and the loss
+cudaError_t launch_race_select(const RaceArgs& a, const FinalizeArgs& fin, cudaStream_t s);
 
 // ---- dispatch.cu
 struct DispatchArgs {
   const void* x; int bf16;
   const int32_t* topk_idx; const float* topk_w; const int32_t* n_sel;
   int T, D, E, K, Kmax;
-  int chunk, nchunks;
+  int ngroups;              // ceil(T/256): groups of 256 tokens
+  int tpb;                  // tokens per gather block
   long long r_max;
-  int32_t* chunk_base;      // [nchunks,E] scratch
+  int32_t* group_base;      // [E,ngroups] scratch: counts, then each group's first row in every segment
+  unsigned int* ctr;        // blocks-done counter in ws (zero between calls)
   int32_t* offsets;         // [E+1]
   int32_t* pos; int32_t* row_token; float* row_gate;
   void* x_perm;

@@ -73,12 +73,12 @@ __device__ __forceinline__ void token_select(const float* logit, int tok, const 
 #pragma unroll
   for (int e = 0; e < EMAX; ++e)
     if (e < E) { P[e] = P[e] * inv; psum[e] += P[e]; }
-  if (a.P) {
+  if (a.P) {      // score row: Expert-Race selects from it; per-image losses read it
     float* prow = a.P + (size_t)tok * E;
 #pragma unroll
     for (int e = 0; e < EMAX; ++e)
       if (e < E) prow[e] = P[e];
-    return;
+    if (a.race) return;
   }
   uint32_t taken = 0;
   for (int k = 0; k < a.K; ++k) {
@@ -114,7 +114,7 @@ __device__ __forceinline__ void tile_partials(const float* psum, int tile, const
     float v = 0.f;
     for (int k = 0; k < nw; ++k) v += wsum_s[k * EMAX + tid];
     a.tile_psum[(size_t)tile * a.E + tid] = v;
-    if (!a.P) a.tile_counts[(size_t)tile * a.E + tid] = cnt_s[tid];
+    if (!a.race) a.tile_counts[(size_t)tile * a.E + tid] = cnt_s[tid];
   }
   __syncthreads();
 }
@@ -180,51 +180,37 @@ __host__ __device__ inline MmaSmem mma_layout(int D, int E) {
 }
 
 // The last block to finish turns the per-block partials into counts and the loss.
-// Every thread loads its tiles' partials for all experts at once (no chain of
-// dependent loads), then fixed-order shuffle trees and a fixed warp order make
-// the result bit-reproducible.  scratch: 2 x 32 x 32 x 8 bytes of shared memory.
+// Warp w reduces experts w, w + nwarps, ...: its lanes stride over the tiles
+// (independent loads), then a fixed xor tree; a fixed expert order for the
+// loss.  Bit-reproducible.  scratch: 2 x 32 x 8 bytes of shared memory.
 constexpr int kFinalizeScratch = 2 * 32 * 32 * 8;
 template <int EMAX>
 __device__ void finalize_counts_loss(const FinalizeArgs& a, uint8_t* scratch) {
-  auto wc = reinterpret_cast<long long(*)[32]>(scratch);
-  auto wp = reinterpret_cast<double(*)[32]>(scratch + 32 * 32 * 8);
+  long long* wc = reinterpret_cast<long long*>(scratch);
+  double* wp = reinterpret_cast<double*>(scratch + 32 * 8);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
   const int E = a.E;
-  long long c[EMAX];
-  double p[EMAX];
+  for (int e = w; e < E; e += nw) {
+    long long c = 0;
+    double p = 0.0;
+#pragma unroll 4
+    for (int t = lane; t < a.ntiles_counts; t += 32) c += __ldcg(a.tile_counts + (size_t)t * E + e);
+#pragma unroll 4
+    for (int t = lane; t < a.ntiles_psum; t += 32) p += (double)__ldcg(a.tile_psum + (size_t)t * E + e);
 #pragma unroll
-  for (int e = 0; e < EMAX; ++e) { c[e] = 0; p[e] = 0.0; }
-  const int nt = a.ntiles_counts > a.ntiles_psum ? a.ntiles_counts : a.ntiles_psum;
-  for (int t = tid; t < nt; t += blockDim.x) {
-#pragma unroll
-    for (int e = 0; e < EMAX; ++e) {
-      if (e < E) {
-        if (t < a.ntiles_counts) c[e] += __ldcg(a.tile_counts + (size_t)t * E + e);
-        if (t < a.ntiles_psum) p[e] += (double)__ldcg(a.tile_psum + (size_t)t * E + e);
-      }
+    for (int o = 16; o > 0; o >>= 1) {
+      c += __shfl_xor_sync(0xffffffffu, c, o);
+      p += __shfl_xor_sync(0xffffffffu, p, o);
     }
-  }
-#pragma unroll
-  for (int e = 0; e < EMAX; ++e) {
-    if (e < E) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        c[e] += __shfl_xor_sync(0xffffffffu, c[e], o);
-        p[e] += __shfl_xor_sync(0xffffffffu, p[e], o);
-      }
-      if (lane == 0) { wc[w][e] = c[e]; wp[w][e] = p[e]; }
-    }
+    if (lane == 0) { wc[e] = c; wp[e] = p; }
   }
   __syncthreads();
   if (tid < 32) {
-    long long cc = 0;
-    double pp = 0.0;
-    if (tid < E)
-      for (int k = 0; k < nw; ++k) { cc += wc[k][tid]; pp += wp[k][tid]; }
     double term = 0.0;
     if (tid < E) {
+      const long long cc = wc[tid];
       a.counts[tid] = (int32_t)cc;
-      term = ((double)E / ((double)a.K * a.T)) * (double)cc * (pp / a.T);
+      term = ((double)E / ((double)a.K * a.T)) * (double)cc * (wp[tid] / a.T);
     }
     for (int o = 16; o > 0; o >>= 1) term += __shfl_down_sync(0xffffffffu, term, o);
     if (tid == 0) *a.aux_loss = (float)(a.alpha * term);
@@ -291,6 +277,8 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
     if (w < my_rb) { issue(w, 0); issue(w, 1); }   // x streams in while the gate weight loads
   }
   if (tid < 32) cnt_s[tid] = 0;
+  if (blockIdx.x == 0 && a.zero)
+    for (int i = tid; i < a.nzero; i += blockDim.x) a.zero[i] = 0u;
   {  // gate weight (bf16) -> padded rows; rows E..EMAX-1 are zero
     const int vpr = D / 8;
     const uint4* wv = reinterpret_cast<const uint4*>(a.wg);
@@ -408,6 +396,8 @@ route_kernel_ffma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Final
   int* cnt_s = reinterpret_cast<int*>(full + kRouteStages);
   float* wsum_s = reinterpret_cast<float*>(cnt_s + 32);
   const int stage_bytes = a.tile_rows * 128;
+  if (blockIdx.x == 0 && a.zero)
+    for (int i = tid; i < a.nzero; i += blockDim.x) a.zero[i] = 0u;
   {
     const float4* wv = reinterpret_cast<const float4*>(a.wg);
 #pragma unroll 4
@@ -531,153 +521,265 @@ cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUte
   return cudaErrorInvalidValue;
 }
 
-// ---------------------------------------------------------------- finalize (race path)
+// ---------------------------------------------------------------- per-image balance loss
+// Block b takes image b's tokens [b*L, (b+1)*L): the counts of their selected
+// experts and their score sums per expert (fp64, fixed reduction order), then
+// the image's L_balance with T = L.  The last block averages the images'
+// losses, in a fixed order.
+constexpr int kSeqThreads = 256;
+
 template <int EMAX>
-__global__ void __launch_bounds__(256) route_finalize_kernel(FinalizeArgs a) {
-  __shared__ __align__(16) uint8_t scratch[kFinalizeScratch];
-  finalize_counts_loss<EMAX>(a, scratch);
+__global__ void __launch_bounds__(kSeqThreads) seq_loss_kernel(SeqLossArgs a) {
+  __shared__ double wp[kSeqThreads / 32][EMAX];
+  __shared__ int cnt_s[EMAX];
+  __shared__ bool last;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, E = a.E, L = a.L;
+  const int b = blockIdx.x;
+  if (tid < EMAX) cnt_s[tid] = 0;
+  __syncthreads();
+  double p[EMAX];
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) p[e] = 0.0;
+  for (int t = b * L + tid; t < (b + 1) * L; t += kSeqThreads) {
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e)
+      if (e < E) p[e] += (double)__ldcg(a.P + (size_t)t * E + e);
+    const int ns = a.n_sel ? a.n_sel[t] : a.K;
+    for (int k = 0; k < a.Kmax && k < ns; ++k) {
+      const int e = a.topk_idx[(size_t)t * a.Kmax + k];
+      if (e >= 0 && e < E) atomicAdd(&cnt_s[e], 1);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) {
+    if (e < E) {
+      double v = p[e];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) wp[w][e] = v;
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    double term = 0.0;
+    if (tid < E) {
+      double ps = 0.0;
+      for (int k = 0; k < kSeqThreads / 32; ++k) ps += wp[k][tid];
+      term = ((double)E / ((double)a.K * L)) * (double)cnt_s[tid] * (ps / L);
+    }
+    for (int o = 16; o > 0; o >>= 1) term += __shfl_down_sync(0xffffffffu, term, o);
+    if (tid == 0) a.seq_loss[b] = a.alpha * term;
+  }
+  // the last block: mean over images
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) last = atomicAdd(a.ctr, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const int nseq = gridDim.x;
+  double s = 0.0;
+  for (int i = tid; i < nseq; i += kSeqThreads) s += __ldcg(a.seq_loss + i);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) wp[w][0] = s;
+  __syncthreads();
+  if (tid == 0) {
+    double tot = 0.0;
+    for (int k = 0; k < kSeqThreads / 32; ++k) tot += wp[k][0];
+    *a.aux_loss = (float)(tot / nseq);
+    *a.ctr = 0u;
+  }
 }
 
-cudaError_t launch_route_finalize(const FinalizeArgs& a, cudaStream_t s) {
-  if (a.E <= 8) route_finalize_kernel<8><<<1, 256, 0, s>>>(a);
-  else if (a.E <= 16) route_finalize_kernel<16><<<1, 256, 0, s>>>(a);
-  else route_finalize_kernel<32><<<1, 256, 0, s>>>(a);
+cudaError_t launch_seq_loss(const SeqLossArgs& a, cudaStream_t s) {
+  const int nseq = a.T / a.L;
+  if (a.E <= 8) seq_loss_kernel<8><<<nseq, kSeqThreads, 0, s>>>(a);
+  else if (a.E <= 16) seq_loss_kernel<16><<<nseq, kSeqThreads, 0, s>>>(a);
+  else seq_loss_kernel<32><<<nseq, kSeqThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------- Expert-Race
-// Exact radix select of the S-th largest score over the T x E matrix on the
-// fp32 bit patterns (scores are >= 0, so the unsigned order of the bits is the
-// numeric order): 12 + 12 + 8 bits.  state[0] = prefix so far, state[1] =
-// winners still needed inside the current bin, state[2] = threshold bits,
-// state[3] = winners to take among the entries equal to the threshold.
-constexpr int kRaceTile = 128;
+// Exact radix select of the S-th largest score of the T x E matrix on the fp32
+// bit patterns (scores are >= 0, so the unsigned order of the bits is the
+// numeric order), digits of 12, 12 and 8 bits, followed by the selection, all in
+// one cooperative launch with one CTA per SM.  CTA r owns a contiguous range of
+// tokens, hence of flat indices t*E+i.  Per digit: a shared-memory histogram of
+// the CTA's range, added into a global one; a grid barrier; then every CTA
+// finds the bin that holds the needed rank on its own (the same integers
+// everywhere give the same answer), so one barrier per digit suffices.  The
+// last digit's histogram of CTA r is also stored: its threshold bin counts the
+// CTA's entries equal to the threshold, which gives every CTA the number of
+// equal entries before its range (ties go to the lower flat index) without a
+// fourth barrier.  Each token's score row for the selection is loaded before
+// the last barrier.
+constexpr int kRaceThreads = 512;
 
-__global__ void __launch_bounds__(256) race_hist_kernel(const uint32_t* __restrict__ bits, long long n,
-                                                       int pass, const uint32_t* __restrict__ state,
-                                                       uint32_t* __restrict__ hist) {
-  __shared__ uint32_t h[4096];
-  for (int i = threadIdx.x; i < 4096; i += 256) h[i] = 0;
-  __syncthreads();
-  const uint32_t prefix = pass ? state[0] : 0u;
-  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += (long long)gridDim.x * 256) {
-    const uint32_t b = bits[i];
-    if (pass == 0) atomicAdd(&h[b >> 20], 1u);
-    else if (pass == 1) { if ((b >> 20) == prefix) atomicAdd(&h[(b >> 8) & 0xFFFu], 1u); }
-    else { if ((b >> 8) == prefix) atomicAdd(&h[b & 0xFFu], 1u); }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 4096; i += 256)
-    if (h[i]) atomicAdd(&hist[i], h[i]);
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
-// one block of 1024 threads: pick the bin holding the needed rank, from the top
-__global__ void __launch_bounds__(1024) race_find_kernel(uint32_t* hist, uint32_t* state, int pass,
-                                                         uint32_t S) {
-  __shared__ uint32_t part[1024];
-  const int nb = pass == 2 ? 256 : 4096;
-  const int per = nb / 1024 > 0 ? nb / 1024 : 1;
-  const int tid = threadIdx.x;
-  const uint32_t need = pass ? state[1] : S;
-  // thread i owns bins (from the top) [i*per, i*per+per) when i*per < nb
-  uint32_t local = 0;
-  if (tid * per < nb)
-    for (int j = 0; j < per; ++j) local += hist[nb - 1 - (tid * per + j)];
-  part[tid] = local;
-  __syncthreads();
-  // inclusive scan (Hillis-Steele) over 1024 partial sums
-  for (int o = 1; o < 1024; o <<= 1) {
-    const uint32_t v = tid >= o ? part[tid - o] : 0u;
-    __syncthreads();
-    part[tid] += v;
-    __syncthreads();
-  }
-  uint32_t above = tid ? part[tid - 1] : 0u;
-  if (tid * per < nb) {
-    for (int j = 0; j < per; ++j) {
-      const int bin = nb - 1 - (tid * per + j);
-      const uint32_t h = hist[bin];
-      if (above < need && above + h >= need) {
-        const uint32_t prefix = pass == 0 ? (uint32_t)bin
-                              : pass == 1 ? ((state[0] << 12) | (uint32_t)bin)
-                                          : ((state[0] << 8) | (uint32_t)bin);
-        state[0] = prefix;
-        state[1] = need - above;
-        if (pass == 2) { state[2] = prefix; state[3] = need - above; }
-      }
-      above += h;
-    }
-  }
-  __syncthreads();
-  for (int i = tid; i < 4096; i += 1024) hist[i] = 0;   // ready for the next pass
-}
-
-// entries equal to the threshold, per tile of 128 tokens
-__global__ void __launch_bounds__(kRaceTile) race_count_eq_kernel(const uint32_t* __restrict__ bits,
-                                                                 int T, int E, const uint32_t* state,
-                                                                 uint32_t* tile_eq) {
-  __shared__ uint32_t wsum[kRaceTile / 32];
-  const uint32_t thr = state[2];
-  const int t = blockIdx.x * kRaceTile + threadIdx.x;
-  uint32_t c = 0;
-  if (t < T)
-    for (int e = 0; e < E; ++e) c += bits[(size_t)t * E + e] == thr;
-  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = c;
+// Barrier over all CTAs of a cooperative launch: arrive on a counter that only
+// grows during the launch, then wait until it reaches `target`.  The wait is
+// bounded: on expiry the status word records `where` and the CTA goes on (its
+// outputs are then invalid, which the status reports).
+__device__ void grid_barrier(uint32_t* ctr, uint32_t target, int* status, int where) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    uint32_t s = 0;
-    for (int w = 0; w < kRaceTile / 32; ++w) s += wsum[w];
-    tile_eq[blockIdx.x] = s;
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    const uint64_t t0 = global_ns();
+    while (ld_acquire_gpu(ctr) < target) {
+      if (global_ns() - t0 > kWaitLimitNs) {
+        set_status(status, DEV_TIMEOUT, where);
+        break;
+      }
+      __nanosleep(32);
+    }
+    __threadfence();
   }
+  __syncthreads();
 }
 
-template <int EMAX>
-__global__ void __launch_bounds__(kRaceTile) race_select_kernel(RaceArgs a) {
-  __shared__ uint32_t scan[kRaceTile];
-  __shared__ int cnt_s[EMAX];
-  __shared__ uint32_t base_s;
-  const int tid = threadIdx.x;
-  const int E = a.E;
-  const uint32_t thr = a.state[2], need_eq = a.state[3];
-  if (tid < EMAX) cnt_s[tid] = 0;
-  if (tid == 0) {
-    uint32_t b = 0;
-    for (int i = 0; i < (int)blockIdx.x; ++i) b += a.tile_eq[i];
-    base_s = b;
+// Exclusive prefix sum of v over the block (kRaceThreads threads); *total gets the sum.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
+  constexpr int NW = kRaceThreads / 32;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  const int t = blockIdx.x * kRaceTile + tid;
-  const uint32_t* bits = reinterpret_cast<const uint32_t*>(a.P);
-  uint32_t v[EMAX];
-  uint32_t my_eq = 0;
+  if (lane == 31) wsum[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    uint32_t y = lane < NW ? wsum[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t z = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) y += z;
+    }
+    if (lane < NW) wsum[lane] = y;
+  }
+  __syncthreads();
+  const uint32_t before = (w ? wsum[w - 1] : 0u) + x - v;
+  *total = wsum[NW - 1];
+  __syncthreads();
+  return before;
+}
+
+// The bin of the merged histogram h[nb] (global, counted from the top) that
+// holds rank `need`, and the rank inside it: out[0], out[1] for every thread.
+__device__ void race_find_bin(const uint32_t* h, int nb, uint32_t need, uint32_t* wsum, uint32_t* out) {
+  const int per = nb / kRaceThreads > 0 ? nb / kRaceThreads : 1;    // 8 (4096 bins) or 1 (256)
+  const int tid = threadIdx.x;
+  if (tid == 0) { out[0] = 0u; out[1] = need; }
+  uint32_t c[8];
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int i = tid * per + j;
+    c[j] = (j < per && i < nb) ? __ldcg(h + nb - 1 - i) : 0u;
+    local += c[j];
+  }
+  uint32_t total;
+  uint32_t above = block_excl_scan(local, wsum, &total);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < per) {
+      if (above < need && above + c[j] >= need) { out[0] = (uint32_t)(nb - 1 - (tid * per + j)); out[1] = need - above; }
+      above += c[j];
+    }
+  }
+  __syncthreads();
+}
+
+template <int DIGIT>
+__device__ __forceinline__ void race_count(uint32_t* h, uint32_t b, uint32_t prefix) {
+  if (DIGIT == 0) atomicAdd(&h[b >> 20], 1u);
+  else if (DIGIT == 1) { if ((b >> 20) == prefix) atomicAdd(&h[(b >> 8) & 0xFFFu], 1u); }
+  else { if ((b >> 8) == prefix) atomicAdd(&h[b & 0xFFu], 1u); }
+}
+
+// shared-memory histogram of digit DIGIT over bits[e0, e1) (e0 a multiple of 4)
+template <int DIGIT>
+__device__ void race_local_hist(const uint32_t* bits, long long e0, long long e1, uint32_t prefix, uint32_t* h) {
+  const long long n4 = (e1 - e0) >> 2;
+  const uint4* v4 = reinterpret_cast<const uint4*>(bits + e0);
+  for (long long i = threadIdx.x; i < n4; i += kRaceThreads) {
+    const uint4 q = __ldcg(v4 + i);
+    race_count<DIGIT>(h, q.x, prefix);
+    race_count<DIGIT>(h, q.y, prefix);
+    race_count<DIGIT>(h, q.z, prefix);
+    race_count<DIGIT>(h, q.w, prefix);
+  }
+  for (long long i = e0 + n4 * 4 + threadIdx.x; i < e1; i += kRaceThreads) race_count<DIGIT>(h, __ldcg(bits + i), prefix);
+}
+
+// Winners of token t among its scores v[] against the threshold (`valid` false:
+// no token, but the lane still takes part in the warp's ballots); `rank` counts
+// the entries equal to the threshold before them in flat order.  The token's
+// row (winners in descending score, ties to the lower expert id, then -1 / 0
+// padding) is built in registers and written with 16-byte stores when E is a
+// multiple of 4 and at most 16.
+template <int EMAX>
+__device__ __forceinline__ void race_emit(const RaceArgs& a, int t, bool valid, const uint32_t* v, uint32_t thr,
+                                          uint32_t need_eq, uint32_t rank, int* cnt_s) {
+  const int E = a.E;
+  uint32_t win = 0;
 #pragma unroll
   for (int e = 0; e < EMAX; ++e) {
-    v[e] = (t < a.T && e < E) ? bits[(size_t)t * E + e] : 0u;
-    my_eq += (t < a.T && e < E && v[e] == thr) ? 1u : 0u;
+    if (valid && e < E) {
+      bool sel = v[e] > thr;
+      if (v[e] == thr) { sel = rank < need_eq; ++rank; }
+      if (sel) win |= 1u << e;
+    }
   }
-  scan[tid] = my_eq;
-  __syncthreads();
-  for (int o = 1; o < kRaceTile; o <<= 1) {
-    const uint32_t x = tid >= o ? scan[tid - o] : 0u;
-    __syncthreads();
-    scan[tid] += x;
-    __syncthreads();
-  }
-  const bool valid = t < a.T;
-  if (valid) {
-    uint32_t rank = base_s + scan[tid] - my_eq;   // equal entries before this token
-    uint32_t chosen = 0;
+  // per-expert counts: one shared atomic per warp and expert
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int e = 0; e < EMAX; ++e) {
-      if (e < E) {
-        bool sel = v[e] > thr;
-        if (v[e] == thr) { sel = rank < need_eq; ++rank; }
-        if (sel) chosen |= 1u << e;
+  for (int e = 0; e < EMAX; ++e) {
+    if (e < E) {
+      const int c = __popc(__ballot_sync(0xffffffffu, (win >> e) & 1u));
+      if (lane == 0 && c) atomicAdd(&cnt_s[e], c);
+    }
+  }
+  if (!valid) return;
+  const int n = __popc(win);
+  int32_t* ri = a.topk_idx + (size_t)t * E;
+  float* rw = a.topk_w + (size_t)t * E;
+  if (EMAX <= 16 && (E & 3) == 0) {
+    // the row in registers (constant indices only), then 16-byte stores
+    int oi[EMAX];
+    uint32_t ow[EMAX];
+#pragma unroll
+    for (int k = 0; k < EMAX; ++k) { oi[k] = -1; ow[k] = 0u; }
+    uint32_t left = win;
+    for (int m = 0; left; ++m) {
+      uint32_t bv = 0;
+      int bi = -1;
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e)
+        if (((left >> e) & 1u) && (bi < 0 || v[e] > bv)) { bv = v[e]; bi = e; }
+      left &= ~(1u << bi);
+#pragma unroll
+      for (int k = 0; k < EMAX; ++k)
+        if (k == m) { oi[k] = bi; ow[k] = bv; }
+    }
+#pragma unroll
+    for (int k = 0; k < EMAX; k += 4) {
+      if (k < E) {
+        *reinterpret_cast<int4*>(ri + k) = make_int4(oi[k], oi[k + 1], oi[k + 2], oi[k + 3]);
+        *reinterpret_cast<uint4*>(rw + k) = make_uint4(ow[k], ow[k + 1], ow[k + 2], ow[k + 3]);
       }
     }
-    // winners of this token in descending score, ties to the lower expert id
-    int n = 0;
-    uint32_t left = chosen;
+  } else {
+    int m = 0;
+    uint32_t left = win;
     while (left) {
       uint32_t bv = 0;
       int bi = -1;
@@ -685,37 +787,128 @@ __global__ void __launch_bounds__(kRaceTile) race_select_kernel(RaceArgs a) {
       for (int e = 0; e < EMAX; ++e)
         if (((left >> e) & 1u) && (bi < 0 || v[e] > bv)) { bv = v[e]; bi = e; }
       left &= ~(1u << bi);
-      a.topk_idx[(size_t)t * E + n] = bi;
-      a.topk_w[(size_t)t * E + n] = __uint_as_float(bv);
-      atomicAdd(&cnt_s[bi], 1);
-      ++n;
+      ri[m] = bi;
+      rw[m] = __uint_as_float(bv);
+      ++m;
     }
-    for (int k = n; k < E; ++k) {
-      a.topk_idx[(size_t)t * E + k] = -1;
-      a.topk_w[(size_t)t * E + k] = 0.f;
+    for (int k = m; k < E; ++k) {
+      ri[k] = -1;
+      rw[k] = 0.f;
     }
-    a.n_sel[t] = n;
   }
-  __syncthreads();
-  if (tid < E) a.tile_counts[(size_t)blockIdx.x * E + tid] = cnt_s[tid];
+  a.n_sel[t] = n;
 }
 
-cudaError_t launch_race_select(const RaceArgs& a, cudaStream_t s) {
-  const long long n = (long long)a.T * a.E;
-  const uint32_t S = (uint32_t)((long long)a.K * a.T);
+template <int EMAX>
+__global__ void __launch_bounds__(kRaceThreads, 1) race_select_kernel(RaceArgs a, FinalizeArgs fin) {
+  __shared__ __align__(16) uint32_t h[4096];     // also the finalize scratch (16 KB) at the end
+  __shared__ uint32_t wsum[32];
+  __shared__ uint32_t found[2];
+  __shared__ int cnt_s[EMAX];
+  const int tid = threadIdx.x, r = blockIdx.x, E = a.E;
+  const uint32_t G = gridDim.x;
   const uint32_t* bits = reinterpret_cast<const uint32_t*>(a.P);
-  int hist_grid = (int)((n + 256 * 8 - 1) / (256 * 8));
-  if (hist_grid > 1184) hist_grid = 1184;
-  if (hist_grid < 1) hist_grid = 1;
-  for (int pass = 0; pass < 3; ++pass) {
-    race_hist_kernel<<<hist_grid, 256, 0, s>>>(bits, n, pass, a.state, a.hist);
-    race_find_kernel<<<1, 1024, 0, s>>>(a.hist, a.state, pass, S);
+  uint32_t* g0 = a.sync;
+  uint32_t* g1 = a.sync + 4096;
+  uint32_t* g2 = a.sync + 8192;
+  uint32_t* bar = a.sync + 8448;
+  const int t0 = min(a.T, r * a.tpc), t1 = min(a.T, t0 + a.tpc);
+  const long long e0 = (long long)t0 * E, e1 = (long long)t1 * E;
+  const uint32_t S = (uint32_t)a.K * (uint32_t)a.T;
+
+  // digit 1: bits 31..20
+  for (int i = tid; i < 4096; i += kRaceThreads) h[i] = 0u;
+  if (tid < EMAX) cnt_s[tid] = 0;
+  __syncthreads();
+  race_local_hist<0>(bits, e0, e1, 0u, h);
+  __syncthreads();
+  for (int i = tid; i < 4096; i += kRaceThreads)
+    if (h[i]) atomicAdd(&g0[i], h[i]);
+  grid_barrier(bar, G, a.status, 300);
+  race_find_bin(g0, 4096, S, wsum, found);
+  uint32_t prefix = found[0], need = found[1];
+
+  // digit 2: bits 19..8 among the entries whose top 12 bits equal the prefix
+  for (int i = tid; i < 4096; i += kRaceThreads) h[i] = 0u;
+  __syncthreads();
+  race_local_hist<1>(bits, e0, e1, prefix, h);
+  __syncthreads();
+  for (int i = tid; i < 4096; i += kRaceThreads)
+    if (h[i]) atomicAdd(&g1[i], h[i]);
+  grid_barrier(bar, 2 * G, a.status, 301);
+  race_find_bin(g1, 4096, need, wsum, found);
+  prefix = (prefix << 12) | found[0];
+  need = found[1];
+
+  // digit 3: bits 7..0; this CTA's histogram is also kept for the tie ranks
+  for (int i = tid; i < 256; i += kRaceThreads) h[i] = 0u;
+  __syncthreads();
+  race_local_hist<2>(bits, e0, e1, prefix, h);
+  __syncthreads();
+  for (int i = tid; i < 256; i += kRaceThreads) {
+    a.loc[(size_t)r * 256 + i] = h[i];
+    if (h[i]) atomicAdd(&g2[i], h[i]);
   }
-  race_count_eq_kernel<<<a.ntiles, kRaceTile, 0, s>>>(bits, a.T, a.E, a.state, a.tile_eq);
-  if (a.E <= 8) race_select_kernel<8><<<a.ntiles, kRaceTile, 0, s>>>(a);
-  else if (a.E <= 16) race_select_kernel<16><<<a.ntiles, kRaceTile, 0, s>>>(a);
-  else race_select_kernel<32><<<a.ntiles, kRaceTile, 0, s>>>(a);
-  return cudaGetLastError();
+  // the score rows of this CTA's first round of tokens load across the barrier
+  uint32_t v[EMAX];
+  {
+    const int t = t0 + tid;
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) v[e] = (t < t1 && e < E) ? __ldcg(bits + (size_t)t * E + e) : 0u;
+  }
+  grid_barrier(bar, 3 * G, a.status, 302);
+  race_find_bin(g2, 256, need, wsum, found);
+  const uint32_t thr = (prefix << 8) | found[0];   // the S-th largest score's bits
+  const uint32_t need_eq = found[1];                // entries equal to it that are selected
+
+  // entries equal to the threshold in the ranges of CTAs 0..r-1
+  uint32_t carry;
+  {
+    uint32_t c = 0;
+    for (int q = tid; q < r; q += kRaceThreads) c += __ldcg(a.loc + (size_t)q * 256 + (thr & 0xFFu));
+    block_excl_scan(c, wsum, &carry);
+  }
+
+  // selection, kRaceThreads tokens at a time (one per thread), in token order
+  for (int tb = t0; tb < t1; tb += kRaceThreads) {
+    const int t = tb + tid;
+    const bool valid = t < t1;
+    if (tb != t0) {
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e) v[e] = (valid && e < E) ? __ldcg(bits + (size_t)t * E + e) : 0u;
+    }
+    uint32_t my_eq = 0;
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) my_eq += (valid && e < E && v[e] == thr) ? 1u : 0u;
+    uint32_t round_eq;
+    const uint32_t rank = carry + block_excl_scan(my_eq, wsum, &round_eq);
+    carry += round_eq;
+    race_emit<EMAX>(a, t, valid, v, thr, need_eq, rank, cnt_s);
+  }
+  __syncthreads();
+  if (tid < E) a.tile_counts[(size_t)r * E + tid] = cnt_s[tid];
+  if (last_block_done(fin.ctr)) finalize_counts_loss<EMAX>(fin, reinterpret_cast<uint8_t*>(h));
+}
+
+int race_plan(int T, int sms, int* tpc) {
+  int g = sms < kRaceMaxCtas ? sms : kRaceMaxCtas;
+  const int by4 = (T + 3) / 4;
+  if (g > by4) g = by4;
+  if (g < 1) g = 1;
+  int per = (T + g - 1) / g;
+  per = (per + 3) / 4 * 4;         // a multiple of 4 tokens keeps every range's start 16-byte aligned
+  *tpc = per;
+  return (T + per - 1) / per;
+}
+
+cudaError_t launch_race_select(const RaceArgs& a, const FinalizeArgs& fin, cudaStream_t s) {
+  RaceArgs ra = a;
+  FinalizeArgs fa = fin;
+  void* args[] = {(void*)&ra, (void*)&fa};
+  const dim3 grid((unsigned)a.grid), block(kRaceThreads);
+  if (a.E <= 8) return cudaLaunchCooperativeKernel((const void*)race_select_kernel<8>, grid, block, args, 0, s);
+  if (a.E <= 16) return cudaLaunchCooperativeKernel((const void*)race_select_kernel<16>, grid, block, args, 0, s);
+  return cudaLaunchCooperativeKernel((const void*)race_select_kernel<32>, grid, block, args, 0, s);
 }
 
 }  // namespace moe

@@ -1,0 +1,47 @@
+// Expert-selection frequency per label: the statistic behind the expert
+// specialisation heat maps of "Scaling Diffusion Transformers to 16 Billion
+// Parameters" (selection frequency by image class, by spatial position and by
+// denoising timestep).  One thread per token; each slot's (label, expert)
+// key is merged across the warp (match.any) before one global atomic per
+// distinct key.  Integer counts, so the order of the atomics does not matter.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+constexpr int kFreqThreads = 256;
+
+__global__ void __launch_bounds__(kFreqThreads) frequency_kernel(FreqArgs a) {
+  const int t = blockIdx.x * kFreqThreads + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const bool valid = t < a.T;
+  int label = -1;
+  if (valid) {
+    label = a.labels ? a.labels[t / a.L] : t % a.L;
+    if (label < 0 || label >= a.n_labels) {
+      set_status(a.status, DEV_BAD_INDEX, 400);
+      label = -1;
+    }
+  }
+  const int ns = label >= 0 ? (a.n_sel ? a.n_sel[t] : a.K) : 0;
+  for (int k = 0; k < a.Kmax; ++k) {     // the same trip count in every lane
+    int key = -1;
+    if (k < ns) {
+      const int e = a.topk_idx[(size_t)t * a.Kmax + k];
+      if (e >= a.E) set_status(a.status, DEV_BAD_INDEX, 401);
+      else if (e >= 0) key = label * a.E + e;
+    }
+    const unsigned same = __match_any_sync(0xffffffffu, key);
+    if (key >= 0 && lane == __ffs(same) - 1) atomicAdd(&a.hist[key], __popc(same));
+  }
+}
+
+cudaError_t launch_frequency(const FreqArgs& a, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(a.hist, 0, (size_t)a.n_labels * a.E * sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
+  if (a.T == 0) return cudaSuccess;
+  frequency_kernel<<<(a.T + kFreqThreads - 1) / kFreqThreads, kFreqThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

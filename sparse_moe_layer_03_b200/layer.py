@@ -39,6 +39,7 @@ class LayerShape:
     alpha: float = 0.01
     act: str = "tanh"
     gemm_impl: str = "auto"
+    seq_len: int = 0          # tokens per image for the balance loss (0 = the whole call)
 
 
 class MoELayer:
@@ -48,7 +49,7 @@ class MoELayer:
         self.s = shape
         self.device = torch.device(device)
         self.cfg = B.make_config(shape.T, shape.D, shape.H, shape.E, shape.K, shape.n_shared, shape.dtype,
-                                 shape.routing, shape.alpha, shape.act, shape.gemm_impl)
+                                 shape.routing, shape.alpha, shape.act, shape.gemm_impl, shape.seq_len)
         self.act_dtype = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
         dt, dev = self.act_dtype, self.device
         self.wg = _dev(params["wg"], dt, dev)
@@ -123,6 +124,16 @@ class MoELayer:
         self.gemm2()
         self.combine()
         return self.out
+
+    def expert_frequency(self, seq_len: int, seq_labels: Optional[torch.Tensor] = None,
+                         n_labels: Optional[int] = None) -> torch.Tensor:
+        """Counts [n_labels, E] of the last routing's selections per label: per patch position
+        (t mod seq_len) without labels, else per image label (class or timestep)."""
+        n = seq_len if seq_labels is None else int(n_labels)
+        hist = torch.empty((n, self.s.E), dtype=torch.int32, device=self.device)
+        B.moe_expert_frequency(self.cfg, self.topk_idx, self.n_sel, seq_len, seq_labels, n, hist, self.ws,
+                               self.stream())
+        return hist
 
     def check(self):
         B.moe_check_status(self.ws, self.stream())

@@ -32,7 +32,7 @@ def test_version_and_sizes():
 @pytest.mark.parametrize("field,value,code", [
     ("K", 9, B.MOE_ERR_INVALID_ARG), ("E", 33, B.MOE_ERR_UNSUPPORTED), ("D", 100, B.MOE_ERR_UNSUPPORTED),
     ("T", -1, B.MOE_ERR_INVALID_ARG), ("n_shared", 9, B.MOE_ERR_UNSUPPORTED), ("dtype", 7, B.MOE_ERR_INVALID_ARG),
-    ("routing", 3, B.MOE_ERR_INVALID_ARG), ("reserved", 1, B.MOE_ERR_INVALID_ARG),
+    ("routing", 3, B.MOE_ERR_INVALID_ARG), ("seq_len", -1, B.MOE_ERR_INVALID_ARG), ("seq_len", 7, B.MOE_ERR_INVALID_ARG),
 ])
 def test_invalid_config_is_rejected_on_host(field, value, code):
     cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
@@ -61,3 +61,23 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
     assert rc == B.MOE_ERR_INVALID_ARG and b"n_sel" in B.lib.moe_last_error()
     rc = B.lib.moe_combine(ctypes.byref(race), fake, fake, fake, None, fake, None)
     assert rc == B.MOE_ERR_INVALID_ARG
+
+
+def test_frequency_arguments_rejected_before_launch():
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    fake = 1 << 40                          # never dereferenced: validation fails first
+    f = B.lib.moe_expert_frequency
+    cases = [
+        (0, None, 0, fake, b"seq_len"),          # seq_len < 1
+        (100, None, 100, fake, b"divide"),        # 100 does not divide 1024
+        (256, None, 255, fake, b"n_labels"),      # position labels need n_labels == seq_len
+        (256, fake, 0, fake, b"n_labels"),        # no rows
+        (256, None, 256, None, b"hist"),          # no output
+    ]
+    for seq_len, labels, n_labels, hist, word in cases:
+        rc = f(ctypes.byref(cfg), fake, None, seq_len, labels, n_labels, hist, fake, None)
+        assert rc == B.MOE_ERR_INVALID_ARG, (seq_len, n_labels)
+        assert word in B.lib.moe_last_error()
+    race = B.make_config(1024, 384, 1536, 8, 2, 2, routing="race")
+    rc = f(ctypes.byref(race), fake, None, 256, None, 256, fake, fake, None)
+    assert rc == B.MOE_ERR_INVALID_ARG and b"n_sel" in B.lib.moe_last_error()

@@ -1,0 +1,103 @@
+"""GPU parity of the per-image balance loss and of the expert-selection frequencies.
+
+Both are checked against the oracle evaluated on the GPU's own selection: the
+loss to the same relative tolerance as the whole-call loss, the frequencies
+bit for bit (integer counts).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from sparse_moe_layer_03_b200 import binding as B
+from sparse_moe_layer_03_b200 import inputs as I
+from tests import parity as PA
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(w, inp, seq_len):
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    shape = LayerShape(w.T, w.D, w.H, w.E, w.K, w.n_shared, w.dtype, w.routing, w.alpha, seq_len=seq_len)
+    L = MoELayer(shape, inp, "cuda:0")
+    x = torch.as_tensor(inp["x"]).to(device="cuda:0", dtype=L.act_dtype).contiguous()
+    L.forward(x)
+    torch.cuda.synchronize()
+    L.check()
+    return L, PA.fetch(L)
+
+
+def _check_loss(w, inp, L, r, seq_len):
+    P = O.softmax_scores(O.gate_logits(inp["x"], inp["wg"], inp.get("router_bias")))
+    PA.check_routing(w, P, r)
+    idx = PA.gpu_selection(r)
+    assert np.array_equal(r["counts"].astype(np.int64), O.expert_counts(idx, w.E))
+    ref = O.balance_loss_per_sequence(idx, P, w.K, w.alpha, seq_len)
+    got = float(r["aux"][0])
+    assert abs(got - ref) <= PA.aux_tol(w) * abs(ref), (got, ref)
+    return idx
+
+
+CASES = [  # T, D, H, E, K, n_s, dtype, routing, seq_len
+    (1024, 128, 256, 8, 2, 1, "bf16", "topk", 256),
+    (1024, 128, 256, 16, 2, 1, "bf16", "race", 256),
+    (960, 64, 128, 8, 1, 0, "f32", "topk", 64),
+    (960, 64, 128, 8, 3, 0, "f32", "race", 320),
+    (600, 192, 384, 32, 4, 2, "bf16", "topk", 1),      # one token per image
+    (600, 192, 384, 4, 2, 0, "bf16", "race", 600),     # one image: the whole-call loss
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "T%d_D%d_E%d_K%d_%s_%s_L%d" % (c[0], c[1], c[3], c[4], c[6], c[7], c[8]))
+def test_per_image_loss_and_frequencies(case):
+    T, D, H, E, K, ns, dt, routing, L_img = case
+    w = I.small_workload(T, D, H, E, K, ns, dt, routing, seed=31 + T + E)
+    inp = I.make_inputs(w)
+    L, r = _run(w, inp, L_img)
+    idx = _check_loss(w, inp, L, r, L_img)
+    if L_img == T:
+        assert abs(float(r["aux"][0]) - O.balance_loss(O.expert_counts(idx, E), O.softmax_scores(
+            O.gate_logits(inp["x"], inp["wg"], inp.get("router_bias"))), K, w.alpha)) <= 1e-4 * float(r["aux"][0])
+    # per patch position
+    hp = L.expert_frequency(L_img).cpu().numpy()
+    assert np.array_equal(hp, O.expert_frequency(idx, E, O.position_labels(T, L_img), L_img))
+    # per image label (a class out of 1000, or a timestep out of 250 DDPM steps)
+    nimg = T // L_img
+    rng = np.random.default_rng(5)
+    for n_labels in (1000, 250):
+        lab = rng.integers(0, n_labels, nimg).astype(np.int32)
+        hl = L.expert_frequency(L_img, torch.as_tensor(lab, device="cuda:0"), n_labels).cpu().numpy()
+        assert np.array_equal(hl, O.expert_frequency(idx, E, O.image_labels(T, L_img, lab), n_labels))
+    L.check()
+
+
+@pytest.mark.parametrize("key", ["xl2_8e2a_512", "xl_race_16e"])
+def test_per_image_loss_full_size(key):
+    # 512x512 images: 1024 patch tokens each, 32 images per call
+    w = I.WORKLOADS[key]
+    inp = I.make_inputs(w)
+    L, r = _run(w, inp, 1024)
+    idx = _check_loss(w, inp, L, r, 1024)
+    hp = L.expert_frequency(1024).cpu().numpy()
+    assert np.array_equal(hp, O.expert_frequency(idx, w.E, O.position_labels(w.T, 1024), 1024))
+    lab = (np.arange(32) * 7 % 250).astype(np.int32)
+    hl = L.expert_frequency(1024, torch.as_tensor(lab, device="cuda:0"), 250).cpu().numpy()
+    assert np.array_equal(hl, O.expert_frequency(idx, w.E, O.image_labels(w.T, 1024, lab), 250))
+
+
+def test_label_out_of_range_is_reported_not_faulted():
+    w = I.small_workload(512, 64, 128, 8, 2, 0, "bf16", "topk", seed=3)
+    inp = I.make_inputs(w)
+    L, r = _run(w, inp, 128)
+    lab = torch.tensor([0, 5, 12, 1], dtype=torch.int32, device="cuda:0")   # 12 is outside 0..9
+    hist = L.expert_frequency(128, lab, 10)
+    torch.cuda.synchronize()
+    with pytest.raises(B.MoeError) as ei:
+        L.check()
+    assert ei.value.code == B.MOE_ERR_DEVICE_CHECK
+    idx = PA.gpu_selection(r)
+    tok_lab = O.image_labels(512, 128, [0, 5, 12, 1])
+    keep = tok_lab < 10
+    want = O.expert_frequency(idx[keep], 8, tok_lab[keep], 10)
+    assert np.array_equal(hist.cpu().numpy(), want)      # the image with the bad label is skipped
+    L.check()                                            # the status word was cleared

@@ -42,6 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM read + write bytes of one launch of each expert GEMM at the default workload (ncu, one pass,
 # full size; profiles/gemm_pair_dram_xl2_8e2a_512.md).  Set to None whenever the kernel changes.
 MEASURED_TRAFFIC = {("xl2_8e2a_512", "gemm1"): 1_509_157_000, ("xl2_8e2a_512", "gemm2"): 1_594_224_000}
+# (the GEMM2 launch with the combine folded in has not been captured yet: its traffic is reported as null)
 
 
 def load_peaks():
@@ -193,7 +194,8 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     inp = I.make_inputs(w)
     if rank > 0:
         inp["x"] = I.make_inputs(I.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}))["x"]
-    shape = LayerShape(w.T, w.D, w.H, w.E, w.K, w.n_shared, w.dtype, w.routing, w.alpha)
+    shape = LayerShape(w.T, w.D, w.H, w.E, w.K, w.n_shared, w.dtype, w.routing, w.alpha,
+                       fuse_combine=args.fuse_combine == "on")
     L = MoELayer(shape, inp, device)
     dt = L.act_dtype
     x_host = torch.as_tensor(inp["x"]).to(dt).pin_memory()
@@ -203,9 +205,11 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
-    stages = ["route", "dispatch", "gemm1", "gemm2", "combine"]
+    # with the combine folded into GEMM2 (bf16, n_s >= 1) the step has four stages
+    stages = (["route", "dispatch", "gemm1", "gemm2_combine"] if L.fused
+              else ["route", "dispatch", "gemm1", "gemm2", "combine"])
     calls = {"route": lambda: L.route(x), "dispatch": lambda: L.dispatch(x), "gemm1": lambda: L.gemm1(x),
-             "gemm2": L.gemm2, "combine": L.combine}
+             "gemm2": L.gemm2, "combine": L.combine, "gemm2_combine": L.gemm2_combine}
 
     def step(events):
         for i, s in enumerate(stages):
@@ -283,13 +287,19 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
     avg = {s: float(np.mean(v)) for s, v in per_stage.items()}
     g1 = M.gemm1_flops(w.T, w.D, w.H, w.K, w.n_shared)
     g2 = M.gemm2_flops(w.T, w.D, w.H, w.K, w.n_shared)
+    fused = "gemm2_combine" in avg
     stage_work = {
         "route": ("GB/s", M.route_bytes(w.T, w.D, w.E, w.K, elem, race)),
         "dispatch": ("GB/s", M.dispatch_bytes(w.T, w.D, w.E, w.K, elem, race)),
         "gemm1": ("TFLOP/s", g1),
-        "gemm2": ("TFLOP/s", g2),
-        "combine": ("GB/s", M.combine_bytes(w.T, w.D, w.K, w.n_shared, elem)),
     }
+    if fused:
+        stage_work["gemm2_combine"] = ("TFLOP/s", g2)
+    else:
+        stage_work["gemm2"] = ("TFLOP/s", g2)
+        stage_work["combine"] = ("GB/s", M.combine_bytes(w.T, w.D, w.K, w.n_shared, elem))
+    g2_stage = "gemm2_combine" if fused else "gemm2"
+    mem_stages = ("route", "dispatch") if fused else ("route", "dispatch", "combine")
     hbm = peaks["hbm_gbs"]
     tc_peak = peaks["bf16_tflops_sustained"]
     tc_burst = peaks["bf16_tflops"]
@@ -302,12 +312,12 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
         else:
             a = work / (ms * 1e-3) / 1e12
             stages_out[s] = {"ms": round(ms, 4), "TFLOP/s": round(a, 1), "frac_bf16": round(a / tc_peak, 3)}
-    dom = "gemm1" if avg["gemm1"] >= avg["gemm2"] else "gemm2"
+    dom = "gemm1" if avg["gemm1"] >= avg[g2_stage] else g2_stage
     dom_flops = g1 if dom == "gemm1" else g2
     achieved = dom_flops / (avg[dom] * 1e-3) / 1e12
-    gemm_ms = avg["gemm1"] + avg["gemm2"]
-    mem_ms = avg["route"] + avg["dispatch"] + avg["combine"]
-    mem_bytes = sum(stage_work[s][1] for s in ("route", "dispatch", "combine"))
+    gemm_ms = avg["gemm1"] + avg[g2_stage]
+    mem_ms = sum(avg[s] for s in mem_stages)
+    mem_bytes = sum(stage_work[s][1] for s in mem_stages)
     total_tokens = w.T * world
     value = total_tokens / (ms_per_step * 1e-3)
     ntok = calibrated_tokens(w, inp, 15.0)
@@ -315,8 +325,8 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
     h2d = w.T * w.D * elem
     d2h = w.T * w.D * elem + 4
     # route (finalize fused; race: + one cooperative select-and-finalize launch), dispatch count +
-    # gather, GEMM1, GEMM2, combine
-    launches_per_step = (1 + (1 if race else 0)) + 2 + 1 + 1 + 1
+    # gather, GEMM1, GEMM2 (+ combine unless folded into GEMM2)
+    launches_per_step = (1 + (1 if race else 0)) + 2 + 1 + 1 + (0 if fused else 1)
     return {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
@@ -332,7 +342,8 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
         "mem_stages_GBps": round(mem_bytes / (mem_ms * 1e-3) / 1e9, 1),
         "mem_stages_frac_hbm": round(mem_bytes / (mem_ms * 1e-3) / 1e9 / hbm, 3),
         "stages": stages_out,
-        "roofline": {"kernel": f"tcgen05 CTA-pair grouped expert GEMM ({dom}, one launch per step)",
+        "roofline": {"kernel": f"tcgen05 CTA-pair grouped expert GEMM ({dom}, one launch per step"
+                               + (", combine folded into the shared experts' tiles)" if dom == "gemm2_combine" else ")"),
                      "bound": "tensor", "achieved": round(achieved, 1), "peak": tc_burst, "unit": "TFLOP/s",
                      "frac": round(achieved / tc_burst, 3),
                      "traffic": MEASURED_TRAFFIC.get((args.workload, dom)),
@@ -384,6 +395,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(I.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--fuse-combine", default="on", choices=["on", "off"],
+                    help="fold the combine into the shared experts' GEMM2 (bf16, n_s >= 1)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

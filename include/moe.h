@@ -107,7 +107,8 @@ size_t moe_workspace_size(const moe_config_t* cfg);
  * R_max = round_up(K*T + 255*E, 256).  Host only. */
 int64_t moe_max_rows(const moe_config_t* cfg);
 
-/* Zero the status word of `ws` (asynchronous on `stream`). */
+/* Zero the first 256 bytes of `ws`: the status word and the blocks-done counters the
+ * kernels use between launches (asynchronous on `stream`).  Once before first use. */
 int moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, read the status word of `ws`, clear it, and return
@@ -191,6 +192,28 @@ int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* 
                    const void* w1s, const void* b1s, const void* w2s, const void* b2s,
                    const float* row_gate, void* h_perm, void* h_sh, void* y_perm, void* y_sh,
                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_gemm2_combine -- moe_expert_gemm2 and moe_combine in one launch:
+ * the shared experts' GEMM2 tiles add each token's routed rows y_perm[pos[t,k]]
+ * (slot order, fp32) to their own output and write `out` directly, so the
+ * shared output never goes to memory.  The routed tiles of the same launch
+ * write y_perm first; the shared tiles' epilogue waits (bounded) until every
+ * routed tile is stored.
+ *   Arguments as moe_expert_gemm2 (no y_sh), plus pos [T,Kmax] and n_sel [T]
+ *   (or NULL for top-K) from moe_dispatch / moe_route, and out [T,D] act.
+ *   out[t] = sum_k y_perm[pos[t,k]] + sum_j (W2s_j h_sh_j + b2s_j), rounded once.
+ * Only for bf16 with gemm_impl AUTO and n_shared >= 1 (MOE_ERR_UNSUPPORTED
+ * otherwise: call moe_expert_gemm2 and moe_combine).  Uses the words at byte
+ * offsets 224 and 228 of ws, which must be zero on entry (moe_workspace_init;
+ * each launch leaves them zero).  All CTAs of the launch must be resident at
+ * once (one per SM, as launched); a wait that runs out reports MOE_ERR_TIMEOUT
+ * through moe_check_status.
+ */
+int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm, const void* h_sh,
+                             const void* w2, const void* b2, const void* w2s, const void* b2s, const float* row_gate,
+                             const int32_t* pos, const int32_t* n_sel, void* y_perm, void* out, void* ws,
+                             size_t ws_bytes, void* stream);
 
 /*
  * moe_combine -- MoE(x_t) = sum_{k < n_sel[t]} y_perm[pos[t,k]] + y_sh[t]

@@ -58,6 +58,8 @@ _SIGS = {
     "moe_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
     "moe_route_static": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_frequency": (C.c_int, [_CFG, _P, _P, C.c_int32, _P, C.c_int32, _P, _P, _P]),
+    "moe_expert_gemm2_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t,
+                                           _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -166,3 +168,11 @@ def moe_expert_frequency(cfg, topk_idx, n_sel, seq_len, seq_labels, n_labels, hi
     """Expert-selection counts per label: patch position (seq_labels None) or each image's label."""
     _check(lib.moe_expert_frequency(C.byref(cfg), _ptr(topk_idx), _ptr(n_sel), seq_len, _ptr(seq_labels),
                                     n_labels, _ptr(hist), _ptr(ws), stream))
+
+
+def moe_expert_gemm2_combine(cfg, offsets, h_perm, h_sh, w2, b2, w2s, b2s, row_gate, pos, n_sel, y_perm, out, ws,
+                             ws_bytes, stream=0):
+    """GEMM2 with the combine folded into the shared experts' tiles: writes out [T,D] directly."""
+    _check(lib.moe_expert_gemm2_combine(C.byref(cfg), _ptr(offsets), _ptr(h_perm), _ptr(h_sh), _ptr(w2), _ptr(b2),
+                                        _ptr(w2s), _ptr(b2s), _ptr(row_gate), _ptr(pos), _ptr(n_sel), _ptr(y_perm),
+                                        _ptr(out), _ptr(ws), ws_bytes, stream))

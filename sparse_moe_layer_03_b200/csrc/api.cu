@@ -530,6 +530,55 @@ int moe_expert_gemm2(const moe_config_t* cfg, const int32_t* offsets, const void
                   (long long)ns * cfg->D, cfg->H, ns * cfg->H, cfg->H, ws, (cudaStream_t)stream);
 }
 
+int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm,
+                             const void* h_sh, const void* w2, const void* b2, const void* w2s,
+                             const void* b2s, const float* row_gate, const int32_t* pos, const int32_t* n_sel,
+                             void* y_perm, void* out, void* ws, size_t ws_bytes, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (cfg->dtype != MOE_BF16 || cfg->gemm_impl != MOE_GEMM_AUTO || cfg->n_shared < 1)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "the combine folds into the shared experts' GEMM2 only for bf16, gemm_impl AUTO and n_shared >= 1; "
+                "use moe_expert_gemm2 + moe_combine");
+  if ((rc = check_ws(cfg, ws, ws_bytes))) return rc;
+  if (cfg->T == 0) return ok();
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(h_perm);
+  REQUIRE_PTR(w2);
+  REQUIRE_PTR(row_gate);
+  REQUIRE_PTR(y_perm);
+  REQUIRE_PTR(h_sh);
+  REQUIRE_PTR(w2s);
+  REQUIRE_PTR(pos);
+  REQUIRE_PTR(out);
+  OPTIONAL_PTR(b2);
+  OPTIONAL_PTR(b2s);
+  OPTIONAL_PTR(n_sel);
+  if (cfg->routing == MOE_ROUTE_RACE && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
+  const int ns = cfg->n_shared;
+  const long long R = max_rows(cfg);
+  GemmArgs g{};
+  g.offsets = offsets; g.E = cfg->E; g.r_max = R; g.act = cfg->act; g.status = status_ptr(ws);
+  g.bf16 = 1;
+  g.nprob = 2;
+  GemmProblem& p0 = g.p[0];
+  p0.routed = 1; p0.N = cfg->D; p0.K = cfg->H; p0.epi = 1;
+  p0.A = h_perm; p0.B = w2; p0.out = y_perm; p0.ld_out = cfg->D; p0.bias = b2; p0.bias_stride = cfg->D;
+  p0.bias_rows = 1;
+  p0.gate = row_gate;
+  GemmProblem& p1 = g.p[1];
+  p1.routed = 0; p1.M = cfg->T; p1.N = cfg->D; p1.K = ns * cfg->H; p1.epi = 2;
+  p1.A = h_sh; p1.B = w2s; p1.out = out; p1.ld_out = cfg->D; p1.bias = b2s; p1.bias_stride = 0;
+  p1.bias_rows = ns; p1.ksplit = cfg->H;
+  p1.gate = nullptr;
+  g.pos = pos; g.n_sel = n_sel; g.kmax = kmax_of(cfg); g.kdef = cfg->K;
+  g.y_routed = y_perm;
+  g.done_ctr = ws_at<unsigned int>(ws, 224);
+  g.exit_ctr = ws_at<unsigned int>(ws, 228);
+  return run_gemm(cfg, g, h_perm, R, w2, (long long)cfg->E * cfg->D, h_sh, cfg->T, w2s,
+                  (long long)ns * cfg->D, cfg->H, ns * cfg->H, cfg->H, ws, (cudaStream_t)stream);
+}
+
 int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
                    const void* x, const void* w1, const void* b1, const void* w2, const void* b2,
                    const void* w1s, const void* b1s, const void* w2s, const void* b2s,

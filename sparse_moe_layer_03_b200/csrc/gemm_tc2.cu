@@ -236,6 +236,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     const uint32_t acc_empty_leader0 = map_to_cta(smem_u32(&acc_empty[0]), 0);
     const uint32_t acc_empty_leader1 = map_to_cta(smem_u32(&acc_empty[1]), 0);
     const uint32_t sbuf = smem_u32(epi_base + (warp - 2) * 8192);
+    // combine folded into the shared tiles: every epilogue warp of both CTAs counts each routed tile
+    const bool count_routed = a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr;
+    const unsigned int done_target = (unsigned int)pl.ntiles[0] * 2u * kPairEpiWarps;
+    bool routed_done = false;
     int nstore = 0;
     int local = 0;
     for (int tile = cid; tile < pl.total; tile += ncl, ++local) {
@@ -254,7 +258,29 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       const __nv_bfloat16* bias =
           pr.bias ? reinterpret_cast<const __nv_bfloat16*>(pr.bias) + (long long)ti.e * pr.bias_stride : nullptr;
       constexpr int box_cols = 64;                          // 128 bytes of bf16 (h and y)
-      const int mode = pr.epi == 0 ? (a.act == 1 ? 1 : 0) : 2;   // tanh GELU, erf GELU, gate
+      // tanh GELU, erf GELU, gate, or the combine (routed rows + shared output)
+      const int mode = pr.epi == 0 ? (a.act == 1 ? 1 : 0) : (pr.epi == 2 ? 3 : 2);
+      int ns = 0;
+      const int32_t* prow = nullptr;
+      if (mode == 3) {
+        if (!routed_done) {
+          // every routed tile of this launch has its y rows stored (bounded wait)
+          if (lane == 0) {
+            const uint64_t t0 = global_ns();
+            while (ld_acquire_gpu_u32(a.done_ctr) < done_target) {
+              if (global_ns() - t0 > kWaitLimitNs) { set_status(a.status, DEV_TIMEOUT, 506); break; }
+              __nanosleep(64);
+            }
+          }
+          __syncwarp();
+          routed_done = true;
+        }
+        if (rv) {
+          ns = a.n_sel ? a.n_sel[grow] : a.kdef;
+          ns = ns < 0 ? 0 : (ns > a.kmax ? a.kmax : ns);
+          prow = a.pos + grow * a.kmax;
+        }
+      }
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += box_cols) {
@@ -297,10 +323,31 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
             for (int j = 0; j < 32; j += 2)
               ow[j / 2] = pack_bf16x2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 1),
                                       gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], 1));
-          } else {
+          } else if (mode == 2) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
               ow[j / 2] = pack_bf16x2((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate);
+          } else {
+            // out = sum over the token's slots of its routed rows (slot order), plus the shared output
+            float y[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) y[j] = 0.f;
+            for (int k = 0; k < ns; ++k) {
+              const int pr_row = __ldcg(prow + k);
+              if (pr_row < 0 || pr_row >= a.r_max) continue;
+              const uint4* yp = reinterpret_cast<const uint4*>(
+                  reinterpret_cast<const __nv_bfloat16*>(a.y_routed) + (long long)pr_row * pr.N + col0);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                float t8[8];
+                bf16x8_to_f32(__ldcg(yp + u), t8);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) y[8 * u + j] += t8[j];
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 2)
+              ow[j / 2] = pack_bf16x2(y[j] + (__uint_as_float(v[j]) + b[j]), y[j + 1] + (__uint_as_float(v[j + 1]) + b[j + 1]));
           }
         }
         // stage the 32 x 128-byte box (128-byte swizzle) and store it with TMA; rows past the
@@ -324,6 +371,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
+      if (count_routed && ti.p == 0 && lane == 0) {
+        // this warp's rows of a routed tile are in global memory: count them for the combine
+        bulk_wait_all();
+        fence_proxy_async_all();
+        __threadfence();
+        atomicAdd(a.done_ctr, 1u);
+      }
     }
     if (lane == 0) bulk_wait_all();            // stores done before the CTA may exit
   }
@@ -333,6 +387,14 @@ done:
   cluster_sync();                                   // no CTA leaves while its peer may still use it
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  if (threadIdx.x == 0 && a.exit_ctr != nullptr && a.nprob > 1 && a.p[1].epi == 2) {
+    // the last CTA out resets the combine counters for the next launch (all reads are done)
+    if (atomicAdd(a.exit_ctr, 1u) == gridDim.x - 1) {
+      *a.done_ctr = 0u;
+      *a.exit_ctr = 0u;
+      __threadfence();
+    }
+  }
 }
 
 template <int BN>

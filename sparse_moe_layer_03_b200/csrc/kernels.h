@@ -113,7 +113,8 @@ struct GemmProblem {
   int routed;               // 1: rows grouped by expert segments (offsets), 0: dense rows
   int M;                    // dense: rows; routed: unused (from offsets)
   int N, K;                 // per-expert output width and reduction length
-  int epi;                  // 0: bias + GELU -> act store; 1: (bias) * gate -> act store
+  int epi;                  // 0: bias + GELU -> act store; 1: (bias) * gate -> act store;
+                            // 2 (dense rows, CTA-pair kernel only): out = sum_k y_routed[pos[t,k]] + (acc + bias)
   const void* A;            // [rows,K] act (FFMA path; the TMA path uses tensor maps)
   const void* B;            // [E*N or N, K] act
   void* out; long long ld_out;
@@ -129,6 +130,15 @@ struct GemmArgs {
   int act;
   int* status;
   int bf16;
+  // combine folded into the shared-expert epilogue (epi 2 on problem 1): the routed
+  // tiles of the same launch write y_routed; each epilogue warp counts its finished
+  // routed tiles in done_ctr, and the shared tiles wait for all of them
+  const int32_t* pos;       // [T,kmax] rows of y_routed per token slot (-1 unused)
+  const int32_t* n_sel;     // [T] or null (then kdef slots per token)
+  int kmax, kdef;
+  const void* y_routed;     // [r_max, N] act
+  unsigned int* done_ctr;   // zero on entry; the launch's last CTA resets both counters
+  unsigned int* exit_ctr;
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, int bn,
                            int num_sms, cudaStream_t s);

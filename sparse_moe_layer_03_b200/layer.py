@@ -40,6 +40,7 @@ class LayerShape:
     act: str = "tanh"
     gemm_impl: str = "auto"
     seq_len: int = 0          # tokens per image for the balance loss (0 = the whole call)
+    fuse_combine: bool = True  # fold the combine into the shared experts' GEMM2 where supported
 
 
 class MoELayer:
@@ -87,8 +88,10 @@ class MoELayer:
         self.h_perm = torch.empty((self.R, s.H), dtype=dt, device=dev)
         self.y_perm = torch.empty((self.R, s.D), dtype=dt, device=dev)
         ns = s.n_shared
+        # the combine folds into the shared experts' GEMM2 for bf16 on the CTA-pair GEMM with n_s >= 1
+        self.fused = bool(s.fuse_combine and ns > 0 and s.dtype == "bf16" and s.gemm_impl == "auto")
         self.h_sh = torch.empty((T, ns * s.H), dtype=dt, device=dev) if ns else None
-        self.y_sh = torch.empty((T, s.D), dtype=dt, device=dev) if ns else None
+        self.y_sh = torch.empty((T, s.D), dtype=dt, device=dev) if ns and not self.fused else None
         self.out = torch.empty((T, s.D), dtype=dt, device=dev)
         B.moe_workspace_init(self.ws, self.ws_bytes, self.stream())
 
@@ -115,14 +118,22 @@ class MoELayer:
     def combine(self):
         B.moe_combine(self.cfg, self.y_perm, self.y_sh, self.pos, self.n_sel, self.out, self.stream())
 
+    def gemm2_combine(self):
+        B.moe_expert_gemm2_combine(self.cfg, self.offsets, self.h_perm, self.h_sh, self.w2, self.b2, self.ws2,
+                                   self.bs2, self.row_gate, self.pos, self.n_sel, self.y_perm, self.out, self.ws,
+                                   self.ws_bytes, self.stream())
+
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         """Whole layer on device-resident x [T,D]; returns the output buffer."""
         assert x.shape == (self.cfg.T, self.s.D) and x.dtype == self.act_dtype and x.is_contiguous()
         self.route(x)
         self.dispatch(x)
         self.gemm1(x)
-        self.gemm2()
-        self.combine()
+        if self.fused:
+            self.gemm2_combine()
+        else:
+            self.gemm2()
+            self.combine()
         return self.out
 
     def expert_frequency(self, seq_len: int, seq_labels: Optional[torch.Tensor] = None,

@@ -81,3 +81,18 @@ def test_frequency_arguments_rejected_before_launch():
     race = B.make_config(1024, 384, 1536, 8, 2, 2, routing="race")
     rc = f(ctypes.byref(race), fake, None, 256, None, 256, fake, fake, None)
     assert rc == B.MOE_ERR_INVALID_ARG and b"n_sel" in B.lib.moe_last_error()
+
+
+def test_fused_combine_refuses_unsupported_configs_before_launch():
+    fake = 1 << 40
+    f = B.lib.moe_expert_gemm2_combine
+    for cfg, why in [(B.make_config(1024, 384, 1536, 8, 2, 2, dtype="f32"), b"bf16"),
+                     (B.make_config(1024, 384, 1536, 8, 2, 0), b"n_shared"),
+                     (B.make_config(1024, 384, 1536, 8, 2, 2, gemm_impl="tc1"), b"AUTO")]:
+        n = B.moe_workspace_size(cfg)
+        rc = f(ctypes.byref(cfg), fake, fake, fake, fake, None, fake, None, fake, fake, None, fake, fake, fake, n, None)
+        assert rc == B.MOE_ERR_UNSUPPORTED and why in B.lib.moe_last_error()
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    n = B.moe_workspace_size(cfg)
+    rc = f(ctypes.byref(cfg), fake, fake, fake, fake, None, fake, None, fake, None, None, fake, fake, fake, n, None)
+    assert rc == B.MOE_ERR_INVALID_ARG and b"pos" in B.lib.moe_last_error()

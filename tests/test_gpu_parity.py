@@ -10,6 +10,7 @@ import pytest
 import torch
 
 from sparse_moe_layer_03_b200 import inputs as I
+from oracle import moe_oracle as O
 from tests import parity as PA
 
 pytestmark = pytest.mark.gpu
@@ -168,3 +169,35 @@ def test_pipelined_host_batches_match_device_forward():
         torch.cuda.synchronize()
         assert torch.equal(outs[i], ref)
         assert float(auxs[i][0]) == float(L.aux[0].cpu())
+
+
+FUSED_CASES = [  # T, D, H, E, K, n_s, routing
+    (600, 192, 384, 8, 2, 1, "topk"),
+    (1111, 128, 256, 16, 2, 2, "race"),
+    (300, 64, 128, 4, 4, 3, "topk"),        # every token takes every expert
+]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "T%d_D%d_E%d_K%d_ns%d_%s" % (c[0], c[1], c[3], c[4], c[5], c[6]))
+def test_combine_folded_into_gemm2_matches_separate_combine(case):
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    T, D, H, E, K, ns, routing = case
+    w = I.small_workload(T, D, H, E, K, ns, "bf16", routing, seed=77 + T)
+    inp = I.make_inputs(w, bias_std=0.3)
+    outs = {}
+    for fuse in (True, False):
+        shape = LayerShape(T, D, H, E, K, ns, "bf16", routing, w.alpha, fuse_combine=fuse)
+        L = MoELayer(shape, inp, "cuda:0")
+        assert L.fused == fuse
+        x = torch.as_tensor(inp["x"]).to(device="cuda:0", dtype=L.act_dtype).contiguous()
+        for _ in range(2):                   # the second call checks the counters were left at zero
+            L.forward(x)
+        torch.cuda.synchronize()
+        L.check()
+        r = PA.fetch(L)
+        P = O.softmax_scores(O.gate_logits(inp["x"], inp["wg"], inp.get("router_bias")))
+        PA.check_routing(w, P, r)
+        PA.check_output(w, inp, P, r)
+        outs[fuse] = r["out"]
+    # the folded path skips one bf16 rounding of the shared output: at most a couple of bf16 ulps apart
+    assert PA.rel_err(outs[True], outs[False]) < 2e-2

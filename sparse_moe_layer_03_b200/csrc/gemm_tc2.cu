@@ -2,12 +2,13 @@
 //
 // The same problems and epilogues as the single-CTA kernel (expert MLP =
 // W2 gelu(W1 x), "Scaling Diffusion Transformers to 16 Billion Parameters",
-// "MOE-DIT" eq. MLP), but every output tile is 256 x BN and belongs to a pair
+// "MOE-DIT" eq. MLP), but every output tile is 256 x BN (BN = 256, and one
+// narrower tile per row block when BN does not divide N) and belongs to a pair
 // of CTAs on the two SMs of a TPC (a cluster of 2).  Each CTA loads its own
-// 128 rows of A and its own BN/2 rows of B, so per FLOP each SM pulls 2/3 of
-// the operand bytes of a 128 x 256 single-CTA tile; the pair's tensor cores
-// read the peer's half through the CTA pair, and each CTA's TMEM receives its
-// 128 rows of the 256 x BN accumulator.  No TMA load uses cluster multicast.
+// 128 rows of A and its own half of the tile's B rows, so per FLOP each SM
+// pulls 2/3 of the operand bytes of a 128 x 256 single-CTA tile; the pair's
+// tensor cores read the peer's half through the CTA pair, and each CTA's TMEM
+// receives its 128 rows of the accumulator.  No TMA load uses cluster multicast.
 //
 // Roles per CTA (6 warps): warp 0 = TMA producer (both CTAs; loads complete on
 // the leader's barrier); warp 1 = TMEM allocation (both) and the MMA issuer
@@ -50,12 +51,14 @@ struct PairPlan {
   int poff[33];
   int cnt[32];
   int ntiles[2];
-  int nn[2];
+  int nn[2];          // column tiles per row block: nfull of width BN, then one of width nrem if nrem > 0
+  int nfull[2];
+  int nrem[2];
   int total;
 };
 
 struct PairTile {
-  int p, row0, valid, brow, n0, e, nk;
+  int p, row0, valid, brow, n0, width, e, nk;
 };
 
 template <int BN>
@@ -68,6 +71,7 @@ __device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, co
   const int mt = t / pl.nn[ti.p], nt = t % pl.nn[ti.p];
   ti.row0 = mt * kPairBM;
   ti.n0 = nt * BN;
+  ti.width = nt < pl.nfull[ti.p] ? BN : pl.nrem[ti.p];
   ti.nk = pr.K / kPairBK;
   if (pr.routed) {
     int e = 0;
@@ -132,9 +136,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     }
     if ((long long)p > a.r_max) bad = true;
     for (int q = 0; q < 2; ++q) {
-      if (q >= a.nprob) { pl.ntiles[q] = 0; pl.nn[q] = 1; continue; }
+      if (q >= a.nprob) { pl.ntiles[q] = 0; pl.nn[q] = 1; pl.nfull[q] = 1; pl.nrem[q] = 0; continue; }
       const GemmProblem& pr = a.p[q];
-      pl.nn[q] = pr.N / BN;
+      pl.nfull[q] = pr.N / BN;
+      pl.nrem[q] = pr.N % BN;
+      pl.nn[q] = pl.nfull[q] + (pl.nrem[q] ? 1 : 0);
       const int mt = pr.routed ? (bad ? 0 : p / kPairBM) : (pr.M + kPairBM - 1) / kPairBM;
       pl.ntiles[q] = mt * pl.nn[q];
     }
@@ -153,7 +159,6 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
   cluster_sync();                                   // both CTAs' barriers exist before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t idesc = idesc_bf16_f32(kPairBM, BN);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -177,7 +182,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::STAGE);   // both CTAs' bytes
           uint8_t* sa = stage_base + stage * C::STAGE;
           const int bx = ksplit ? (kb * kPairBK) % ksplit : kb * kPairBK;
-          const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (BN / 2);
+          // each CTA holds half of the tile's B rows (a narrower tile's box also brings rows it does not use)
+          const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (ti.width / 2);
           tma_load_2d_pair(smem_u32(sa), tA, kb * kPairBK, ti.row0 + (int)rank * 128, fb_leader, pol_a);
           tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tB, bx, by, fb_leader, pol_w);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -198,6 +204,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         if (!mbar_wait(smem_u32(&acc_empty[acc]), accph ^ 1u, abort_flag, a.status, 502)) goto mma_out;
         tc_fence_after();
         const uint32_t d = tmem_base + acc * BN;
+        const uint32_t idesc = idesc_bf16_f32(kPairBM, ti.width);
         for (int kb = 0; kb < ti.nk; ++kb) {
           if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)) goto mma_out;
           tc_fence_after();
@@ -283,7 +290,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       }
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += box_cols) {
+      for (int c0 = 0; c0 < ti.width; c0 += box_cols) {
         uint4 o[8];
         uint32_t vv[2][32];
         tmem_ld_32x32b_x32(tbase + c0, vv[0]);
@@ -418,25 +425,19 @@ static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, cons
   return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN>, ta[0], tb[0], ta[1], tb[1], to[0], to[1], a);
 }
 
+// Tiles are 256 columns wide, with one narrower tile (a multiple of 64 columns)
+// for the rest of a row block: N = 1152 runs as 4 x 256 + 128, so each A row
+// block is read 4.5 times instead of 6 (192-wide tiles).
 int gemm_pair_pick_bn(int n0, int n1) {
-  const int cands[4] = {256, 192, 128, 64};
-  for (int i = 0; i < 4; ++i) {
-    const int bn = cands[i];
-    if (n0 % bn == 0 && (n1 == 0 || n1 % bn == 0)) return bn;
-  }
+  if (n0 % 64 == 0 && (n1 == 0 || n1 % 64 == 0)) return 256;
   return 0;
 }
 
 cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, const CUtensorMap* to,
                              int bn, int num_sms, cudaStream_t s) {
   const int grid = num_sms & ~1;
-  switch (bn) {
-    case 256: return launch_pair_bn<256>(a, ta, tb, to, grid, s);
-    case 192: return launch_pair_bn<192>(a, ta, tb, to, grid, s);
-    case 128: return launch_pair_bn<128>(a, ta, tb, to, grid, s);
-    case 64: return launch_pair_bn<64>(a, ta, tb, to, grid, s);
-    default: return cudaErrorInvalidValue;
-  }
+  if (bn != 256) return cudaErrorInvalidValue;
+  return launch_pair_bn<256>(a, ta, tb, to, grid, s);
 }
 
 }  // namespace moe

@@ -67,7 +67,7 @@ typedef enum {
   MOE_ERR_TIMEOUT = -6       /* a kernel's bounded wait ran out (status word) */
 } moe_status_t;
 
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_F16 = 2 } moe_dtype_t;
 typedef enum { MOE_ROUTE_TOPK = 0, MOE_ROUTE_RACE = 1 } moe_routing_t;
 typedef enum {
   MOE_GEMM_AUTO = 0, /* bf16: tcgen05 on CTA pairs (256-row tiles); fp32: FFMA */

@@ -17,7 +17,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "moe.h")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, -1, -2, -3
 MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT = -4, -5, -6
-MOE_F32, MOE_BF16 = 0, 1
+MOE_F32, MOE_BF16, MOE_F16 = 0, 1, 2
 MOE_ROUTE_TOPK, MOE_ROUTE_RACE = 0, 1
 MOE_GEMM_AUTO, MOE_GEMM_SIMT, MOE_GEMM_TC1 = 0, 1, 2
 
@@ -88,7 +88,7 @@ def _check(rc: int):
 
 def make_config(T, D, H, E, K, n_shared, dtype="bf16", routing="topk", alpha=0.01, act="tanh",
                 gemm_impl="auto", seq_len=0) -> MoeConfig:
-    return MoeConfig(T, D, H, E, K, n_shared, MOE_BF16 if dtype == "bf16" else MOE_F32,
+    return MoeConfig(T, D, H, E, K, n_shared, {"f32": MOE_F32, "bf16": MOE_BF16, "f16": MOE_F16}[dtype],
                      MOE_ROUTE_RACE if routing == "race" else MOE_ROUTE_TOPK, alpha,
                      1 if act == "erf" else 0,
                      {"auto": MOE_GEMM_AUTO, "simt": MOE_GEMM_SIMT, "tc1": MOE_GEMM_TC1}[gemm_impl], seq_len)

@@ -42,7 +42,9 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-int elem_bytes(const moe_config_t* c) { return c->dtype == MOE_BF16 ? 2 : 4; }
+// bf16 and fp16 share every 16-bit path; only conversions and MMA operand formats differ
+bool is16(const moe_config_t* c) { return c->dtype == MOE_BF16 || c->dtype == MOE_F16; }
+int elem_bytes(const moe_config_t* c) { return is16(c) ? 2 : 4; }
 
 constexpr int kMaxT = 262144;
 
@@ -55,15 +57,15 @@ int validate(const moe_config_t* c) {
   if (c->E < 1 || c->E > 32) return fail(MOE_ERR_UNSUPPORTED, "E=%d outside 1..32", c->E);
   if (c->K < 1 || c->K > c->E) return fail(MOE_ERR_INVALID_ARG, "K=%d outside 1..E=%d", c->K, c->E);
   if (c->n_shared < 0 || c->n_shared > 8) return fail(MOE_ERR_UNSUPPORTED, "n_shared=%d outside 0..8", c->n_shared);
-  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return fail(MOE_ERR_INVALID_ARG, "dtype=%d", c->dtype);
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16 && c->dtype != MOE_F16) return fail(MOE_ERR_INVALID_ARG, "dtype=%d", c->dtype);
   if (c->routing != MOE_ROUTE_TOPK && c->routing != MOE_ROUTE_RACE) return fail(MOE_ERR_INVALID_ARG, "routing=%d", c->routing);
   if (c->act != 0 && c->act != 1) return fail(MOE_ERR_INVALID_ARG, "act=%d", c->act);
   if (c->gemm_impl < MOE_GEMM_AUTO || c->gemm_impl > MOE_GEMM_TC1) return fail(MOE_ERR_INVALID_ARG, "gemm_impl=%d", c->gemm_impl);
   if (c->seq_len < 0) return fail(MOE_ERR_INVALID_ARG, "seq_len=%d < 0", c->seq_len);
   if (c->seq_len > 0 && c->T % c->seq_len)
     return fail(MOE_ERR_INVALID_ARG, "seq_len=%d does not divide T=%d", c->seq_len, c->T);
-  if (route_smem_total(c->D, c->E, 32, c->dtype == MOE_BF16) > 232448 ||
-      (c->dtype == MOE_BF16 && route_mma_stages(c->D, c->E) < 1))
+  if (route_smem_total(c->D, c->E, 32, is16(c)) > 232448 ||
+      (is16(c) && route_mma_stages(c->D, c->E) < 1))
     return fail(MOE_ERR_UNSUPPORTED, "E=%d x D=%d too large for the router's shared memory", c->E, c->D);
   return MOE_OK;
 }
@@ -157,16 +159,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D row-major [rows, cols] tensor, 128-byte swizzled boxes of box_rows x (128 B)
-int make_tmap(CUtensorMap* m, const void* base, bool bf16, long long rows, long long cols, int box_rows,
+int make_tmap(CUtensorMap* m, const void* base, int dtype, long long rows, long long cols, int box_rows,
               const char* what) {
   auto fn = encode_fn();
   if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  const int eb = bf16 ? 2 : 4;
+  const int eb = dtype == MOE_F32 ? 4 : 2;
+  const CUtensorMapDataType ty = dtype == MOE_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : dtype == MOE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
   cuuint64_t strides[1] = {(cuuint64_t)cols * eb};
   cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+  CUresult r = fn(m, ty, 2,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -174,11 +179,11 @@ int make_tmap(CUtensorMap* m, const void* base, bool bf16, long long rows, long 
   return MOE_OK;
 }
 
-// x [rows, cols] bf16 seen as 3-D {64 columns, rows, cols/64 blocks}: one box brings
+// x [rows, cols] 16-bit seen as 3-D {64 columns, rows, cols/64 blocks}: one box brings
 // `box_rows` rows x ceil(cols/128) swizzled 128-byte blocks (half of each row),
 // block-major.  Returns false when the driver does not accept the layout (the
 // caller then uses 2-D boxes).
-bool make_tmap_rows3d(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
+bool make_tmap_rows3d(CUtensorMap* m, const void* base, int dtype, long long rows, long long cols, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)(rows > 0 ? rows : 1), (cuuint64_t)(cols / 64)};
@@ -187,7 +192,8 @@ bool make_tmap_rows3d(CUtensorMap* m, const void* base, long long rows, long lon
   cuuint32_t box[3] = {64, (cuuint32_t)box_rows, blocks};
   cuuint32_t estr[3] = {1, 1, 1};
   if (blocks > 256) return false;
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(m, dtype == MOE_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -263,20 +269,20 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   const WsLayout L = ws_layout(cfg);
   const int sms = num_sms_current();
   int tile = 0, threads = 0;
-  const bool bf16 = cfg->dtype == MOE_BF16;
-  route_plan(cfg->T, cfg->D, cfg->E, bf16, sms, &tile, &threads);
+  const bool b16 = is16(cfg);
+  route_plan(cfg->T, cfg->D, cfg->E, b16, sms, &tile, &threads);
   const int ntiles = (cfg->T + tile - 1) / tile;
   const int grid = ntiles < sms ? ntiles : sms;
-  // partial sums: one row per CTA (bf16 kernel) or per token tile (fp32 kernel)
-  const int nparts = bf16 ? grid : ntiles;
+  // partial sums: one row per CTA (16-bit kernel) or per token tile (fp32 kernel)
+  const int nparts = b16 ? grid : ntiles;
   CUtensorMap tm;
   int tmap3d = 0;
-  if (bf16 && make_tmap_rows3d(&tm, x, cfg->T, cfg->D, tile)) tmap3d = 1;
-  else if ((rc = make_tmap(&tm, x, bf16, cfg->T, cfg->D, tile, "x"))) return rc;
+  if (b16 && make_tmap_rows3d(&tm, x, cfg->dtype, cfg->T, cfg->D, tile)) tmap3d = 1;
+  else if ((rc = make_tmap(&tm, x, cfg->dtype, cfg->T, cfg->D, tile, "x"))) return rc;
   RouteArgs ra{};
   ra.tmap3d = tmap3d;
   ra.x = x; ra.wg = wg; ra.bias = router_bias;
-  ra.T = cfg->T; ra.D = cfg->D; ra.E = cfg->E; ra.K = cfg->K; ra.bf16 = bf16;
+  ra.T = cfg->T; ra.D = cfg->D; ra.E = cfg->E; ra.K = cfg->K; ra.b16 = b16; ra.f16 = cfg->dtype == MOE_F16;
   ra.tile_rows = tile; ra.ntiles = ntiles; ra.grid = grid;
   ra.topk_idx = topk_idx; ra.topk_w = topk_w; ra.n_sel = race ? nullptr : n_sel;
   const bool per_image = cfg->seq_len > 0;
@@ -381,7 +387,7 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx
   if (race && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
   const WsLayout L = ws_layout(cfg);
   DispatchArgs da{};
-  da.x = x; da.bf16 = cfg->dtype == MOE_BF16;
+  da.x = x; da.b16 = is16(cfg);
   da.topk_idx = topk_idx; da.topk_w = topk_w; da.n_sel = n_sel;
   da.T = cfg->T; da.D = cfg->D; da.E = cfg->E; da.K = cfg->K; da.Kmax = kmax_of(cfg);
   da.ngroups = ngroups_of(cfg->T);
@@ -405,7 +411,7 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
              int K1, int bcols1, void* ws, cudaStream_t s) {
   (void)ws;
   cudaError_t e;
-  const bool tc = cfg->dtype == MOE_BF16 && cfg->gemm_impl != MOE_GEMM_SIMT;
+  const bool tc = is16(cfg) && cfg->gemm_impl != MOE_GEMM_SIMT;
   if (!tc) {
     if ((e = launch_gemm_simt(g, s)) != cudaSuccess) return cuda_fail(e, "FFMA expert GEMM");
     return ok();
@@ -418,22 +424,21 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
   const int brows_box = pair ? bn / 2 : bn;
   CUtensorMap ta[2], tb[2];
   int rc;
-  if ((rc = make_tmap(&ta[0], A0, true, rows0, K0, 128, "A0"))) return rc;
-  if ((rc = make_tmap(&tb[0], B0, true, brows0, K0, brows_box, "B0"))) return rc;
+  if ((rc = make_tmap(&ta[0], A0, cfg->dtype, rows0, K0, 128, "A0"))) return rc;
+  if ((rc = make_tmap(&tb[0], B0, cfg->dtype, brows0, K0, brows_box, "B0"))) return rc;
   if (g.nprob > 1) {
-    if ((rc = make_tmap(&ta[1], A1, true, rows1, K1, 128, "A1"))) return rc;
-    if ((rc = make_tmap(&tb[1], B1, true, brows1, bcols1, brows_box, "B1"))) return rc;
+    if ((rc = make_tmap(&ta[1], A1, cfg->dtype, rows1, K1, 128, "A1"))) return rc;
+    if ((rc = make_tmap(&tb[1], B1, cfg->dtype, brows1, bcols1, brows_box, "B1"))) return rc;
   } else {
     ta[1] = ta[0];
     tb[1] = tb[0];
   }
   if (pair) {
-    // output boxes for the TMA-store epilogue: 32 rows x 128 bytes (bf16 h or fp32 y)
+    // output boxes for the TMA-store epilogue: 32 rows x 128 bytes of h or y (act dtype)
     CUtensorMap to[2];
-    const bool out_bf16 = g.bf16 != 0;          // h and y are both in the act dtype
-    if ((rc = make_tmap(&to[0], g.p[0].out, out_bf16, rows0, g.p[0].N, 32, "out0"))) return rc;
+    if ((rc = make_tmap(&to[0], g.p[0].out, cfg->dtype, rows0, g.p[0].N, 32, "out0"))) return rc;
     if (g.nprob > 1) {
-      if ((rc = make_tmap(&to[1], g.p[1].out, out_bf16, rows1, g.p[1].N, 32, "out1"))) return rc;
+      if ((rc = make_tmap(&to[1], g.p[1].out, cfg->dtype, rows1, g.p[1].N, 32, "out1"))) return rc;
     } else {
       to[1] = to[0];
     }
@@ -469,7 +474,7 @@ int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void
   const long long R = max_rows(cfg);
   GemmArgs g{};
   g.offsets = offsets; g.E = cfg->E; g.r_max = R; g.act = cfg->act; g.status = status_ptr(ws);
-  g.bf16 = cfg->dtype == MOE_BF16;
+  g.b16 = is16(cfg); g.f16 = cfg->dtype == MOE_F16;
   g.nprob = ns > 0 ? 2 : 1;
   GemmProblem& p0 = g.p[0];
   p0.routed = 1; p0.N = cfg->H; p0.K = cfg->D; p0.epi = 0;
@@ -510,7 +515,7 @@ int moe_expert_gemm2(const moe_config_t* cfg, const int32_t* offsets, const void
   const long long R = max_rows(cfg);
   GemmArgs g{};
   g.offsets = offsets; g.E = cfg->E; g.r_max = R; g.act = cfg->act; g.status = status_ptr(ws);
-  g.bf16 = cfg->dtype == MOE_BF16;
+  g.b16 = is16(cfg); g.f16 = cfg->dtype == MOE_F16;
   g.nprob = ns > 0 ? 2 : 1;
   GemmProblem& p0 = g.p[0];
   p0.routed = 1; p0.N = cfg->D; p0.K = cfg->H; p0.epi = 1;
@@ -536,9 +541,9 @@ int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, co
                              void* y_perm, void* out, void* ws, size_t ws_bytes, void* stream) {
   int rc = validate(cfg);
   if (rc) return rc;
-  if (cfg->dtype != MOE_BF16 || cfg->gemm_impl != MOE_GEMM_AUTO || cfg->n_shared < 1)
+  if (!is16(cfg) || cfg->gemm_impl != MOE_GEMM_AUTO || cfg->n_shared < 1)
     return fail(MOE_ERR_UNSUPPORTED,
-                "the combine folds into the shared experts' GEMM2 only for bf16, gemm_impl AUTO and n_shared >= 1; "
+                "the combine folds into the shared experts' GEMM2 only for bf16 or fp16, gemm_impl AUTO and n_shared >= 1; "
                 "use moe_expert_gemm2 + moe_combine");
   if ((rc = check_ws(cfg, ws, ws_bytes))) return rc;
   if (cfg->T == 0) return ok();
@@ -559,7 +564,7 @@ int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, co
   const long long R = max_rows(cfg);
   GemmArgs g{};
   g.offsets = offsets; g.E = cfg->E; g.r_max = R; g.act = cfg->act; g.status = status_ptr(ws);
-  g.bf16 = 1;
+  g.b16 = 1; g.f16 = cfg->dtype == MOE_F16;
   g.nprob = 2;
   GemmProblem& p0 = g.p[0];
   p0.routed = 1; p0.N = cfg->D; p0.K = cfg->H; p0.epi = 1;
@@ -603,7 +608,7 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,
   if (cfg->routing == MOE_ROUTE_RACE && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
   CombineArgs ca{};
   ca.y_perm = y_perm; ca.y_sh = cfg->n_shared > 0 ? y_sh : nullptr; ca.pos = pos; ca.n_sel = n_sel;
-  ca.out = out; ca.bf16 = cfg->dtype == MOE_BF16;
+  ca.out = out; ca.b16 = is16(cfg); ca.f16 = cfg->dtype == MOE_F16;
   ca.T = cfg->T; ca.D = cfg->D; ca.K = cfg->K; ca.Kmax = kmax_of(cfg); ca.r_max = max_rows(cfg);
   cudaError_t e = launch_combine(ca, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel");

@@ -3,7 +3,7 @@
 // eq. MoE(x) and "MOE-DIT" shared experts).  The gates were applied in the
 // second expert GEMM's epilogue, so this is an un-permute and a sum: fp32 in
 // slot order k = 0..n_sel-1, then the shared term, rounded once.
-// HBM-bound: one warp per token, 16-byte loads of fp32 rows.
+// HBM-bound: one warp per token, 16-byte loads.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -20,6 +20,11 @@ template <> __device__ __forceinline__ void load8<float>(const float* p, size_t 
 template <> __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, size_t i, float* f) {
   bf16x8_to_f32(reinterpret_cast<const uint4*>(p)[i], f);
 }
+template <> __device__ __forceinline__ void load8<__half>(const __half* p, size_t i, float* f) {
+  f16x8_to_f32(reinterpret_cast<const uint4*>(p)[i], f);
+}
+__device__ __forceinline__ uint32_t pack2(const __nv_bfloat16*, float lo, float hi) { return pack_bf16x2(lo, hi); }
+__device__ __forceinline__ uint32_t pack2(const __half*, float lo, float hi) { return pack_f16x2(lo, hi); }
 
 template <typename T>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
@@ -52,11 +57,12 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
         for (int q = 0; q < 8; ++q) acc[q] += y[q];
       }
       if constexpr (sizeof(T) == 2) {
+        const T* tag = nullptr;
         uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
+        o.x = pack2(tag, acc[0], acc[1]);
+        o.y = pack2(tag, acc[2], acc[3]);
+        o.z = pack2(tag, acc[4], acc[5]);
+        o.w = pack2(tag, acc[6], acc[7]);
         reinterpret_cast<uint4*>(a.out)[(size_t)t * n8 + v] = o;
       } else {
         float4* o = reinterpret_cast<float4*>(a.out) + (size_t)t * 2 * n8 + 2 * v;
@@ -70,7 +76,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
   int grid = (a.T + 7) / 8;
   if (grid > 148 * 16) grid = 148 * 16;
-  if (a.bf16) combine_kernel<__nv_bfloat16><<<grid, kCombineThreads, 0, s>>>(a);
+  if (a.b16 && a.f16) combine_kernel<__half><<<grid, kCombineThreads, 0, s>>>(a);
+  else if (a.b16) combine_kernel<__nv_bfloat16><<<grid, kCombineThreads, 0, s>>>(a);
   else combine_kernel<float><<<grid, kCombineThreads, 0, s>>>(a);
   return cudaGetLastError();
 }

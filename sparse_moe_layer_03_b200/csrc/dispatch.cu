@@ -273,7 +273,7 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   const int ggrid = (a.T + a.tpb - 1) / a.tpb;
   const size_t smem = (size_t)a.tpb * a.Kmax * sizeof(int);
-  if (a.bf16) dispatch_gather_kernel<__nv_bfloat16><<<ggrid, kDispatchThreads, smem, s>>>(a);
+  if (a.b16) dispatch_gather_kernel<uint16_t><<<ggrid, kDispatchThreads, smem, s>>>(a);
   else dispatch_gather_kernel<float><<<ggrid, kDispatchThreads, smem, s>>>(a);
   return cudaGetLastError();
 }

@@ -4,7 +4,7 @@
 // cannot meet, so fp32 inputs run here in true fp32.  The same problems and
 // epilogues as the tcgen05 kernel (bias + GELU for the first expert layer,
 // bias times gate for the second), 64 x 64 output tiles, 4 x 4 per thread.
-// It also accepts bf16 inputs, which gives a second GPU implementation to
+// It also accepts bf16 and fp16 inputs, which gives a second GPU implementation to
 // cross-check the tensor-core path.
 #include "common.cuh"
 #include "kernels.h"
@@ -120,7 +120,8 @@ cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t s) {
   }
   if (maxm == 0 || maxn == 0) return cudaSuccess;
   dim3 grid((maxn + kSBN - 1) / kSBN, (unsigned)((maxm + kSBM - 1) / kSBM), a.nprob);
-  if (a.bf16) gemm_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
+  if (a.b16 && a.f16) gemm_simt_kernel<__half><<<grid, 256, 0, s>>>(a);
+  else if (a.b16) gemm_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
   else gemm_simt_kernel<float><<<grid, 256, 0, s>>>(a);
   return cudaGetLastError();
 }

@@ -7,8 +7,8 @@
 // Diffusion Transformers to 16 Billion Parameters", "MOE-DIT" eq. MLP; tanh
 // GELU per "Scalable Diffusion Models with Transformers", DiT block details),
 // each expert a pair of these GEMMs:
-//   GEMM1 epilogue: + b1, GELU, round to bf16           -> h
-//   GEMM2 epilogue: + b2, times the row's gate (routed)  -> y (bf16)
+//   GEMM1 epilogue: + b1, GELU, round to 16 bits        -> h
+//   GEMM2 epilogue: + b2, times the row's gate (routed)  -> y (16 bits)
 //
 // CTA = 6 warps: warp 0 issues TMA loads (128-byte swizzled K-major tiles) into
 // a ring of shared-memory stages; warp 1 allocates TMEM and one thread issues
@@ -23,7 +23,7 @@
 namespace moe {
 
 constexpr int kBM = 128;
-constexpr int kBK = 64;                 // bf16 elements in one 128-byte swizzle row
+constexpr int kBK = 64;                 // 16-bit elements in one 128-byte swizzle row
 constexpr int kTcThreads = 192;
 constexpr int kSmemLimit = 232448;      // 227 KB opt-in dynamic shared memory per block
 
@@ -77,7 +77,7 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const TilePlan& pl, co
   return ti;
 }
 
-template <int BN>
+template <int BN, typename S>
 __global__ void __launch_bounds__(kTcThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
                const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
@@ -140,7 +140,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const uint32_t idesc = idesc_bf16_f32(kBM, BN);
+  const uint32_t idesc = idesc_f16kind_f32(kBM, BN, S::kFmt);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -193,7 +193,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ 
           const uint64_t bdesc = smem_desc_sw128(sa + C::A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_bf16(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+            umma_kindf16(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
           issued_any = true;
           umma_commit(smem_u32(&empty[stage]));
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -223,8 +223,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ 
       const bool rv = r < ti.valid;
       const long long grow = (long long)ti.row0 + r;
       const float gate = (pr.gate != nullptr && rv) ? pr.gate[grow] : 1.0f;
-      const __nv_bfloat16* bias =
-          pr.bias ? reinterpret_cast<const __nv_bfloat16*>(pr.bias) + (long long)ti.e * pr.bias_stride : nullptr;
+      const uint16_t* bias =
+          pr.bias ? reinterpret_cast<const uint16_t*>(pr.bias) + (long long)ti.e * pr.bias_stride : nullptr;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
@@ -240,32 +240,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ 
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               float t8[8];
-              bf16x8_to_f32(__ldg(bp + u), t8);
+              S::x8_to_f32(__ldg(bp + u), t8);
 #pragma unroll
               for (int j = 0; j < 8; ++j) b[8 * u + j] += t8[j];
             }
           }
         }
         if (rv) {
-          // GEMM1: gelu(acc + b1); GEMM2: gate * (acc + b2); both rounded once to bf16
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ld_out + col0);
+          // GEMM1: gelu(acc + b1); GEMM2: gate * (acc + b2); both rounded once to 16 bits
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(pr.out) + grow * pr.ld_out + col0);
           uint4 o[4];
           uint32_t* ow = reinterpret_cast<uint32_t*>(o);
           const int mode = pr.epi == 0 ? (a.act == 1 ? 1 : 0) : 2;
           if (mode == 0) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = pack_bf16x2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 0),
+              ow[j / 2] = S::pack2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 0),
                                       gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], 0));
           } else if (mode == 1) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = pack_bf16x2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 1),
+              ow[j / 2] = S::pack2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 1),
                                       gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], 1));
           } else {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = pack_bf16x2((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate);
+              ow[j / 2] = S::pack2((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate);
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) dst[u] = o[u];
@@ -291,14 +291,19 @@ int gemm_tc_pick_bn(int n0, int n1) {
   return 0;
 }
 
+template <int BN, typename S>
+static cudaError_t launch_bn_t(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, int grid,
+                               cudaStream_t s) {
+  using C = TcCfg<BN>;
+  cudaError_t err = cudaFuncSetAttribute(gemm_tc_kernel<BN, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (err != cudaSuccess) return err;
+  gemm_tc_kernel<BN, S><<<grid, kTcThreads, C::SMEM, s>>>(ta[0], tb[0], ta[1], tb[1], a);
+  return cudaGetLastError();
+}
 template <int BN>
 static cudaError_t launch_bn(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, int grid,
                              cudaStream_t s) {
-  using C = TcCfg<BN>;
-  cudaError_t err = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  if (err != cudaSuccess) return err;
-  gemm_tc_kernel<BN><<<grid, kTcThreads, C::SMEM, s>>>(ta[0], tb[0], ta[1], tb[1], a);
-  return cudaGetLastError();
+  return a.f16 ? launch_bn_t<BN, StoreF16>(a, ta, tb, grid, s) : launch_bn_t<BN, StoreBF16>(a, ta, tb, grid, s);
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, int bn,

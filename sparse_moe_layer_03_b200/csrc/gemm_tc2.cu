@@ -27,7 +27,7 @@
 namespace moe {
 
 constexpr int kPairBM = 256;            // rows of a pair tile (128 per CTA)
-constexpr int kPairBK = 64;             // bf16 elements per 128-byte swizzle row
+constexpr int kPairBK = 64;             // 16-bit elements per 128-byte swizzle row
 constexpr int kPairEpiWarps = 4;          // one per TMEM lane quadrant
 constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
 constexpr int kPairSmemLimit = 232448;
@@ -89,7 +89,7 @@ __device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, co
   return ti;
 }
 
-template <int BN>
+template <int BN, typename S>
 __global__ void __launch_bounds__(kPairThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
                  const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
@@ -204,7 +204,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         if (!mbar_wait(smem_u32(&acc_empty[acc]), accph ^ 1u, abort_flag, a.status, 502)) goto mma_out;
         tc_fence_after();
         const uint32_t d = tmem_base + acc * BN;
-        const uint32_t idesc = idesc_bf16_f32(kPairBM, ti.width);
+        const uint32_t idesc = idesc_f16kind_f32(kPairBM, ti.width, S::kFmt);
         for (int kb = 0; kb < ti.nk; ++kb) {
           if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)) goto mma_out;
           tc_fence_after();
@@ -213,7 +213,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           const uint64_t bdesc = smem_desc_sw128(sa + C::A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < kPairBK / 16; ++kk)
-            umma_bf16_pair(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+            umma_kindf16_pair(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
           issued_any = true;
           // stage free in both CTAs once these MMAs finish
           const uint32_t eb = smem_u32(&empty[stage]);
@@ -262,9 +262,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       const long long grow = (long long)ti.row0 + (int)rank * 128 + r;
       const int box_row = ti.row0 + (int)rank * 128 + q * 32;
       const float gate = (pr.gate != nullptr && rv) ? pr.gate[grow] : 1.0f;
-      const __nv_bfloat16* bias =
-          pr.bias ? reinterpret_cast<const __nv_bfloat16*>(pr.bias) + (long long)ti.e * pr.bias_stride : nullptr;
-      constexpr int box_cols = 64;                          // 128 bytes of bf16 (h and y)
+      const uint16_t* bias =
+          pr.bias ? reinterpret_cast<const uint16_t*>(pr.bias) + (long long)ti.e * pr.bias_stride : nullptr;
+      constexpr int box_cols = 64;                          // 128 bytes of 16-bit h or y
       // tanh GELU, erf GELU, gate, or the combine (routed rows + shared output)
       const int mode = pr.epi == 0 ? (a.act == 1 ? 1 : 0) : (pr.epi == 2 ? 3 : 2);
       int ns = 0;
@@ -311,29 +311,29 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
                 float t8[8];
-                bf16x8_to_f32(__ldg(bp + u), t8);
+                S::x8_to_f32(__ldg(bp + u), t8);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) b[8 * u + j] += t8[j];
               }
             }
           }
-          // GEMM1: gelu(acc + b1); GEMM2: gate * (acc + b2); both rounded once to bf16.  The
+          // GEMM1: gelu(acc + b1); GEMM2: gate * (acc + b2); both rounded once to 16 bits.  The
           // mode is uniform per tile, so each element loop holds one form only.
           uint32_t* ow = reinterpret_cast<uint32_t*>(&o[half * 4]);
           if (mode == 0) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = pack_bf16x2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 0),
+              ow[j / 2] = S::pack2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 0),
                                       gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], 0));
           } else if (mode == 1) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = pack_bf16x2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 1),
+              ow[j / 2] = S::pack2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 1),
                                       gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], 1));
           } else if (mode == 2) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = pack_bf16x2((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate);
+              ow[j / 2] = S::pack2((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate);
           } else {
             // out = sum over the token's slots of its routed rows (slot order), plus the shared output
             float y[32];
@@ -343,18 +343,18 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
               const int pr_row = __ldcg(prow + k);
               if (pr_row < 0 || pr_row >= a.r_max) continue;
               const uint4* yp = reinterpret_cast<const uint4*>(
-                  reinterpret_cast<const __nv_bfloat16*>(a.y_routed) + (long long)pr_row * pr.N + col0);
+                  reinterpret_cast<const uint16_t*>(a.y_routed) + (long long)pr_row * pr.N + col0);
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
                 float t8[8];
-                bf16x8_to_f32(__ldcg(yp + u), t8);
+                S::x8_to_f32(__ldcg(yp + u), t8);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) y[8 * u + j] += t8[j];
               }
             }
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = pack_bf16x2(y[j] + (__uint_as_float(v[j]) + b[j]), y[j + 1] + (__uint_as_float(v[j + 1]) + b[j + 1]));
+              ow[j / 2] = S::pack2(y[j] + (__uint_as_float(v[j]) + b[j]), y[j + 1] + (__uint_as_float(v[j + 1]) + b[j + 1]));
           }
         }
         // stage the 32 x 128-byte box (128-byte swizzle) and store it with TMA; rows past the
@@ -404,11 +404,11 @@ done:
   }
 }
 
-template <int BN>
+template <int BN, typename S>
 static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb,
                                   const CUtensorMap* to, int grid, cudaStream_t s) {
   using C = PairCfg<BN>;
-  cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<BN, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
@@ -422,7 +422,7 @@ static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN>, ta[0], tb[0], ta[1], tb[1], to[0], to[1], a);
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, S>, ta[0], tb[0], ta[1], tb[1], to[0], to[1], a);
 }
 
 // Tiles are 256 columns wide, with one narrower tile (a multiple of 64 columns)
@@ -437,7 +437,7 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUt
                              int bn, int num_sms, cudaStream_t s) {
   const int grid = num_sms & ~1;
   if (bn != 256) return cudaErrorInvalidValue;
-  return launch_pair_bn<256>(a, ta, tb, to, grid, s);
+  return a.f16 ? launch_pair_bn<256, StoreF16>(a, ta, tb, to, grid, s) : launch_pair_bn<256, StoreBF16>(a, ta, tb, to, grid, s);
 }
 
 }  // namespace moe

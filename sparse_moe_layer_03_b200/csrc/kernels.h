@@ -17,9 +17,10 @@ struct RouteArgs {
   const void* x;            // [T,D] act
   const void* wg;           // [E,D] act
   const float* bias;        // [E] or null
-  int T, D, E, K, bf16;
+  int T, D, E, K;
+  int b16, f16;             // 16-bit storage (bf16 or fp16); fp16
   int tile_rows, ntiles, grid;
-  int tmap3d;               // bf16 router: 1 = one 3-D box {64, 16 rows, D/64} per unit, 0 = D/64 2-D boxes
+  int tmap3d;               // 16-bit router: 1 = one 3-D box {64, 16 rows, D/64} per unit, 0 = D/64 2-D boxes
   int32_t* topk_idx;        // top-K mode: [T,K]
   float* topk_w;
   int32_t* n_sel;           // may be null (top-K)
@@ -31,10 +32,10 @@ struct RouteArgs {
   int nzero;
   int* status;
 };
-size_t route_smem_bytes(int D, int E, int tile_rows, int bf16);
-size_t route_smem_total(int D, int E, int tile_rows, int bf16);
+size_t route_smem_bytes(int D, int E, int tile_rows, int b16);
+size_t route_smem_total(int D, int E, int tile_rows, int b16);
 int route_mma_stages(int D, int E);
-void route_plan(int T, int D, int E, int bf16, int sms, int* tile_rows, int* threads);
+void route_plan(int T, int D, int E, int b16, int sms, int* tile_rows, int* threads);
 
 // partial counts / score sums -> counts[E] and the balance loss
 struct FinalizeArgs {
@@ -93,7 +94,7 @@ cudaError_t launch_race_select(const RaceArgs& a, const FinalizeArgs& fin, cudaS
 
 // ---- dispatch.cu
 struct DispatchArgs {
-  const void* x; int bf16;
+  const void* x; int b16;   // 16-bit storage (rows are copied as bytes)
   const int32_t* topk_idx; const float* topk_w; const int32_t* n_sel;
   int T, D, E, K, Kmax;
   int ngroups;              // ceil(T/256): groups of 256 tokens
@@ -129,7 +130,7 @@ struct GemmArgs {
   long long r_max;
   int act;
   int* status;
-  int bf16;
+  int b16, f16;             // 16-bit storage (bf16 or fp16); fp16
   // combine folded into the shared-expert epilogue (epi 2 on problem 1): the routed
   // tiles of the same launch write y_routed; each epilogue warp counts its finished
   // routed tiles in done_ctr, and the shared tiles wait for all of them
@@ -151,7 +152,7 @@ cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t s);
 // ---- combine.cu
 struct CombineArgs {
   const void* y_perm; const void* y_sh; const int32_t* pos; const int32_t* n_sel;   // act dtype
-  void* out; int bf16;
+  void* out; int b16, f16;
   int T, D, K, Kmax;
   long long r_max;
 };

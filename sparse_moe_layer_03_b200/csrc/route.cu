@@ -8,7 +8,7 @@
 // (tokens and experts compete jointly for the top candidates).
 //
 // The logits are HBM-bound: x streams through shared memory once, in
-// 128-byte-swizzled column chunks fed by TMA.  bf16 inputs take their E dot
+// 128-byte-swizzled column chunks fed by TMA.  bf16 and fp16 inputs take their E dot
 // products on mma.sync (the FP32 pipe alone cannot keep up with HBM at E = 16);
 // fp32 inputs use FFMA.  Per-tile partial counts and score sums are reduced in
 // a fixed order, so the loss is bit-reproducible.
@@ -29,23 +29,23 @@ __host__ __device__ inline size_t align1k(size_t v) { return (v + 1023) & ~(size
 struct RouteSmem {
   size_t wg, x, logits, misc, total;
 };
-__host__ __device__ inline RouteSmem route_layout(int D, int E, int tile_rows, int bf16) {
+__host__ __device__ inline RouteSmem route_layout(int D, int E, int tile_rows, int b16) {
   RouteSmem L;
   const int em = route_emax(E);
   L.wg = 0;
-  const size_t wg_bytes = bf16 ? (size_t)em * (D * 2 + 16) : (size_t)E * D * 4;
+  const size_t wg_bytes = b16 ? (size_t)em * (D * 2 + 16) : (size_t)E * D * 4;
   L.x = align1k(wg_bytes);
   // the x stages double as the finalize scratch (2 x 32 x 33 x 8 bytes) at the end
   const size_t xb = (size_t)kRouteStages * tile_rows * 128;
   L.logits = L.x + (xb > 16896 ? xb : 16896);
-  L.misc = L.logits + (bf16 ? (size_t)tile_rows * em * 4 : 0);
+  L.misc = L.logits + (b16 ? (size_t)tile_rows * em * 4 : 0);
   // barriers (4 x 8 B) + counts (<= 32 x 4 B) + warp sums (8 x 32 x 4 B)
   L.total = 1024 /*alignment slack*/ + L.misc + 2048;
   return L;
 }
 
-size_t route_smem_bytes(int D, int E, int tile_rows, int bf16) {
-  return route_layout(D, E, tile_rows, bf16).total;
+size_t route_smem_bytes(int D, int E, int tile_rows, int b16) {
+  return route_layout(D, E, tile_rows, b16).total;
 }
 
 // Per token: bias, softmax, then top-K selection (or the score row for
@@ -119,8 +119,8 @@ __device__ __forceinline__ void tile_partials(const float* psum, int tile, const
   __syncthreads();
 }
 
-// ---------------------------------------------------------------- bf16: tensor-core logits
-// Work unit = a block of 16 consecutive tokens: their full rows (16 x D bf16,
+// ---------------------------------------------------------------- 16-bit: tensor-core logits
+// Work unit = a block of 16 consecutive tokens: their full rows (16 x D 16-bit,
 // one contiguous stretch of HBM, so DRAM pages are read whole) land in one
 // pair of shared-memory stages (one per half of the row, each one 3-D TMA box of
 // 64-column blocks x 16 rows, 128-byte swizzle).  Each warp owns two stages,
@@ -138,13 +138,23 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
 __device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
 }
+// d += a * b on 16 x 8 x 16 tiles, fp32 accumulate; F16 selects fp16 operands, else bf16
+template <bool F16>
 __device__ __forceinline__ void mma_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  if (F16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
 }
 
 constexpr int kMmaRB = 16;        // tokens per row block
@@ -233,7 +243,7 @@ __device__ bool last_block_done(unsigned int* ctr) {
   return last;
 }
 
-template <int EMAX>
+template <int EMAX, bool F16>
 __global__ void __launch_bounds__(kMmaMaxConsumers * 32, 1)
 route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, FinalizeArgs fin) {
   constexpr int NT = EMAX / 8;
@@ -279,7 +289,7 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
   if (tid < 32) cnt_s[tid] = 0;
   if (blockIdx.x == 0 && a.zero)
     for (int i = tid; i < a.nzero; i += blockDim.x) a.zero[i] = 0u;
-  {  // gate weight (bf16) -> padded rows; rows E..EMAX-1 are zero
+  {  // gate weight (16-bit) -> padded rows; rows E..EMAX-1 are zero
     const int vpr = D / 8;
     const uint4* wv = reinterpret_cast<const uint4*>(a.wg);
 #pragma unroll 4
@@ -336,7 +346,7 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
           uint32_t a0, a1, a2, a3;
           ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) mma_16816(acc4[ks][nt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
+          for (int nt = 0; nt < NT; ++nt) mma_16816<F16>(acc4[ks][nt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
         }
       }
       __syncwarp();                                  // every lane is done reading the stage
@@ -470,8 +480,8 @@ route_kernel_ffma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Final
   if (fin.counts != nullptr && last_block_done(fin.ctr)) finalize_counts_loss<EMAX>(fin, xs);
 }
 
-void route_plan(int T, int D, int E, int bf16, int sms, int* tile_rows, int* threads) {
-  if (bf16) {
+void route_plan(int T, int D, int E, int b16, int sms, int* tile_rows, int* threads) {
+  if (b16) {
     *tile_rows = kMmaRB;
     *threads = mma_layout(D, E).consumers * 32;
   } else {
@@ -484,26 +494,29 @@ void route_plan(int T, int D, int E, int bf16, int sms, int* tile_rows, int* thr
   }
 }
 
-size_t route_smem_total(int D, int E, int tile_rows, int bf16) {
-  return bf16 ? mma_layout(D, E).total : route_smem_bytes(D, E, tile_rows, 0);
+size_t route_smem_total(int D, int E, int tile_rows, int b16) {
+  return b16 ? mma_layout(D, E).total : route_smem_bytes(D, E, tile_rows, 0);
 }
 
 int route_mma_stages(int D, int E) { return mma_layout(D, E).consumers; }
 
 cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tm, cudaStream_t s) {
-  const size_t smem = route_smem_total(a.D, a.E, a.tile_rows, a.bf16);
+  const size_t smem = route_smem_total(a.D, a.E, a.tile_rows, a.b16);
   cudaError_t err;
-  if (a.bf16) {
-#define MOE_ROUTE_MMA(EM)                                                                               \
-  if (a.E <= EM) {                                                                                      \
-    err = cudaFuncSetAttribute(route_kernel_mma<EM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
+  if (a.b16) {
+#define MOE_ROUTE_MMA(EM, F)                                                                            \
+  if (a.E <= EM && (a.f16 != 0) == F) {                                                                 \
+    err = cudaFuncSetAttribute(route_kernel_mma<EM, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (err != cudaSuccess) return err;                                                                 \
-    route_kernel_mma<EM><<<a.grid, mma_layout(a.D, a.E).consumers * 32, smem, s>>>(*tm, a, fin);          \
+    route_kernel_mma<EM, F><<<a.grid, mma_layout(a.D, a.E).consumers * 32, smem, s>>>(*tm, a, fin);       \
     return cudaGetLastError();                                                                          \
   }
-    MOE_ROUTE_MMA(8)
-    MOE_ROUTE_MMA(16)
-    MOE_ROUTE_MMA(32)
+    MOE_ROUTE_MMA(8, false)
+    MOE_ROUTE_MMA(16, false)
+    MOE_ROUTE_MMA(32, false)
+    MOE_ROUTE_MMA(8, true)
+    MOE_ROUTE_MMA(16, true)
+    MOE_ROUTE_MMA(32, true)
 #undef MOE_ROUTE_MMA
   } else {
 #define MOE_ROUTE_FFMA(EM)                                                                              \

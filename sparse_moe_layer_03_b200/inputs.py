@@ -9,7 +9,7 @@ Recipe (the same for every workload):
 
 * ``numpy.random.Generator(PCG64(seed))``; every array is drawn as fp64
   standard normals, scaled by its standard deviation, cast to fp32, and for
-  bf16 workloads rounded to the nearest bf16 value (ties to even).  The
+  bf16 (fp16) workloads rounded to the nearest bf16 (fp16) value, ties to even.  The
   returned arrays are fp32 whose values are exactly representable in the
   workload's storage type, so both sides read identical numbers.
 * Draw order: x, Wg, W1 (E,H,D), W2 (E,D,H), shared W1 (n_s,H,D), shared
@@ -45,7 +45,7 @@ class Workload:
     E: int            # routed experts
     K: int            # experts per token (race: average, S = K*T)
     n_shared: int     # shared experts every token visits
-    dtype: str        # "f32" or "bf16" (storage type of activations and weights)
+    dtype: str        # "f32", "bf16" or "f16" (storage type of activations and weights)
     routing: str      # "topk" or "race"
     alpha: float      # balance-loss factor
     seed: int
@@ -92,9 +92,18 @@ def bf16_bits(a: np.ndarray) -> np.ndarray:
     return (a.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
 
 
+def round_to_f16(a: np.ndarray) -> np.ndarray:
+    """Round fp32 values to the nearest fp16 value (IEEE round to nearest even); returns fp32."""
+    return np.ascontiguousarray(a, dtype=np.float32).astype(np.float16).astype(np.float32)
+
+
 def _store(a: np.ndarray, dtype: str) -> np.ndarray:
     a = a.astype(np.float32)
-    return round_to_bf16(a) if dtype == "bf16" else a
+    if dtype == "bf16":
+        return round_to_bf16(a)
+    if dtype == "f16":
+        return round_to_f16(a)
+    return a
 
 
 def make_inputs(w: Workload, bias_std: float = 0.0, x_only_tokens: Optional[int] = None) -> dict:

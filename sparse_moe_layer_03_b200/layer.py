@@ -51,7 +51,7 @@ class MoELayer:
         self.device = torch.device(device)
         self.cfg = B.make_config(shape.T, shape.D, shape.H, shape.E, shape.K, shape.n_shared, shape.dtype,
                                  shape.routing, shape.alpha, shape.act, shape.gemm_impl, shape.seq_len)
-        self.act_dtype = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+        self.act_dtype = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[shape.dtype]
         dt, dev = self.act_dtype, self.device
         self.wg = _dev(params["wg"], dt, dev)
         self.router_bias = _dev(params.get("router_bias"), torch.float32, dev)
@@ -88,8 +88,8 @@ class MoELayer:
         self.h_perm = torch.empty((self.R, s.H), dtype=dt, device=dev)
         self.y_perm = torch.empty((self.R, s.D), dtype=dt, device=dev)
         ns = s.n_shared
-        # the combine folds into the shared experts' GEMM2 for bf16 on the CTA-pair GEMM with n_s >= 1
-        self.fused = bool(s.fuse_combine and ns > 0 and s.dtype == "bf16" and s.gemm_impl == "auto")
+        # the combine folds into the shared experts' GEMM2 for 16-bit types on the CTA-pair GEMM with n_s >= 1
+        self.fused = bool(s.fuse_combine and ns > 0 and s.dtype in ("bf16", "f16") and s.gemm_impl == "auto")
         self.h_sh = torch.empty((T, ns * s.H), dtype=dt, device=dev) if ns else None
         self.y_sh = torch.empty((T, s.D), dtype=dt, device=dev) if ns and not self.fused else None
         self.out = torch.empty((T, s.D), dtype=dt, device=dev)
@@ -161,6 +161,7 @@ class MoELayer:
         """
         n = len(x_host)
         dev = self.device
+        own_out, own_aux = self.out, self.aux
         if not hasattr(self, "_pipe"):
             self._pipe = {
                 "x": [torch.empty((self.cfg.T, self.s.D), dtype=self.act_dtype, device=dev) for _ in range(2)],
@@ -183,16 +184,23 @@ class MoELayer:
                 loaded[i].record(P["h2d"])
 
         load(0)
+        try:
+            self._pipeline(n, P, comp, load, loaded, computed, drained, consumed, out_host, aux_host)
+        finally:
+            self.out, self.aux = own_out, own_aux
+        drained[n - 1].synchronize()
+
+    def _pipeline(self, n, P, comp, load, loaded, computed, drained, consumed, out_host, aux_host):
         for i in range(n):
             if i + 1 < n:
                 load(i + 1)
             comp.wait_event(loaded[i])
             if i >= 2:
                 comp.wait_event(drained[i - 2])               # output buffer i%2 copied out
+            # the layer writes straight into this batch's output buffers
+            self.out, self.aux = P["out"][i % 2], P["aux"][i % 2]
             self.forward(P["x"][i % 2])
             consumed[i].record(comp)
-            P["out"][i % 2].copy_(self.out)
-            P["aux"][i % 2].copy_(self.aux)
             computed[i].record(comp)
             with torch.cuda.stream(P["d2h"]):
                 P["d2h"].wait_event(computed[i])
@@ -200,4 +208,3 @@ class MoELayer:
                 if aux_host is not None:
                     aux_host[i].copy_(P["aux"][i % 2], non_blocking=True)
                 drained[i].record(P["d2h"])
-        drained[n - 1].synchronize()

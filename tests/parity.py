@@ -8,8 +8,8 @@ Rules (from the method's workload description):
   for bit with the oracle's canonical permutation of the GPU's own selection;
 * the output is compared with the oracle evaluated on the GPU's selection
   (so a tie flip costs no output tolerance): normwise max relative error
-  max|y - y_ref| / max|y_ref| <= 1e-5 (fp32) and <= 2e-2 (bf16);
-* the balance loss to 1e-5 (fp32) / 1e-4 (bf16) relative.
+  max|y - y_ref| / max|y_ref| <= 1e-5 (fp32), <= 2e-2 (bf16), <= 5e-3 (fp16);
+* the balance loss to 1e-5 (fp32) / 1e-4 (bf16, fp16) relative.
 """
 from __future__ import annotations
 
@@ -24,7 +24,9 @@ SEG_ALIGN = 256      # expert segments of the permuted buffers start on multiple
 
 
 def out_tol(w: Workload) -> float:
-    return 1e-5 if w.dtype == "f32" else 2e-2
+    # fp16 carries 3 more mantissa bits than bf16 (unit roundoff 2^-11 against 2^-8), so the same
+    # few roundings (h, y, out) sit 8x lower; 5e-3 keeps the bf16 bound's margin of about 4
+    return {"f32": 1e-5, "bf16": 2e-2, "f16": 5e-3}[w.dtype]
 
 
 def aux_tol(w: Workload) -> float:

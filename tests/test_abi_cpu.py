@@ -27,6 +27,8 @@ def test_version_and_sizes():
     assert B.moe_workspace_size(cfg) > 0
     race = B.make_config(32768, 1152, 4608, 16, 2, 1, routing="race")
     assert B.moe_workspace_size(race) > 32768 * 16 * 4
+    f16 = B.make_config(32768, 1152, 4608, 8, 2, 2, dtype="f16")
+    assert B.moe_workspace_size(f16) == B.moe_workspace_size(cfg)
 
 
 @pytest.mark.parametrize("field,value,code", [

@@ -33,6 +33,9 @@ SMALL = [
     (640, 64, 128, 32, 4, 2, "bf16", "topk"),
     (1111, 192, 384, 8, 2, 1, "bf16", "topk"),     # odd number of 64-column blocks in the router
     (900, 320, 640, 16, 3, 2, "bf16", "race"),
+    (1000, 256, 512, 8, 2, 2, "f16", "topk"),     # fp16 storage (DiT inference default)
+    (900, 320, 640, 16, 3, 2, "f16", "race"),
+    (999, 128, 256, 4, 1, 0, "f16", "topk"),       # no shared experts: separate combine
 ]
 
 
@@ -201,3 +204,18 @@ def test_combine_folded_into_gemm2_matches_separate_combine(case):
         outs[fuse] = r["out"]
     # the folded path skips one bf16 rounding of the shared output: at most a couple of bf16 ulps apart
     assert PA.rel_err(outs[True], outs[False]) < 2e-2
+
+
+@pytest.mark.parametrize("impl", ["tc1", "simt"])
+def test_f16_other_gemm_paths(impl):
+    w = I.small_workload(777, 384, 1536, 16, 2, 2, "f16", "topk", seed=21)
+    inp = I.make_inputs(w, bias_std=0.25)
+    PA.full_check(w, inp, gemm_impl=impl)
+
+
+def test_f16_full_size_xl():
+    # the XL/2-8E2A layer with fp16 storage: all output tokens sampled against the oracle
+    import dataclasses
+    w = dataclasses.replace(I.WORKLOADS["xl2_8e2a_512"], dtype="f16", name="DiT-MoE-XL/2-8E2A layer at 512x512, fp16")
+    inp = I.make_inputs(w)
+    PA.full_check(w, inp, tokens=PA.sample_tokens(w.T, 512))

@@ -196,6 +196,46 @@ def image_labels(T, seq_len, per_image):
     return np.repeat(np.asarray(per_image), seq_len)[:T]
 
 
+# ---------------------------------------------------------------- adaLN-Zero around the layer
+
+def layer_norm(x, eps=1e-5):
+    """(x - mean) / sqrt(var + eps) over the last dimension, biased variance, no affine.
+
+    "Diffusion Transformer (DiT) 技术全景解析" 2.2.3 (AdaLN): the adaptive norm
+    normalises with a plain layer_norm over the feature dimension (library
+    default epsilon) before the conditional scale and shift.
+    """
+    x = as_f64(x)
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps)
+
+
+def adaln(x, gamma, beta, img_len, eps=1e-5):
+    """gamma_b * LayerNorm(x_t) + beta_b for token t of image b = t // img_len.
+
+    "Diffusion Transformer (DiT) 技术全景解析" 2.2.3: gamma and beta are
+    regressed from the conditioning per sample and broadcast over its tokens.
+    """
+    x = as_f64(x)
+    T = x.shape[0]
+    b = np.arange(T) // img_len
+    return as_f64(gamma)[b] * layer_norm(x, eps) + as_f64(beta)[b]
+
+
+def gated_residual(x_res, y, alpha, img_len):
+    """x_res_t + alpha_b * y_t: the adaLN-Zero gate on a residual branch.
+
+    "Scalable Diffusion Models with Transformers (DiT)", DiT block details
+    (adaLN-Zero): a per-dimension scale alpha, regressed per sample, multiplies
+    the branch before each residual connection; zero alpha makes the block the
+    identity.
+    """
+    x_res = as_f64(x_res)
+    b = np.arange(x_res.shape[0]) // img_len
+    return x_res + as_f64(alpha)[b] * as_f64(y)
+
+
 # ---------------------------------------------------------------- experts
 
 def gelu_tanh(u):

@@ -241,6 +241,41 @@ def test_frequency_marginals_and_relabelling(routing):
     assert np.array_equal(hi2[perm], hi)
 
 
+# ------------------------------------------------------------------ adaLN-Zero
+
+def test_layer_norm_matches_library_and_moments():
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((64, 96)) * 3 + 1.5
+    ref = torch.nn.functional.layer_norm(torch.from_numpy(x), (96,)).numpy()
+    assert np.max(np.abs(O.layer_norm(x) - ref)) < 1e-12
+    y = O.layer_norm(x, eps=0.0)
+    assert np.max(np.abs(y.mean(1))) < 1e-12 and np.max(np.abs(y.var(1) - 1)) < 1e-12
+
+
+def test_adaln_special_cases():
+    rng = np.random.default_rng(42)
+    x = rng.standard_normal((48, 32))
+    ones, zeros = np.ones((3, 32)), np.zeros((3, 32))
+    assert np.max(np.abs(O.adaln(x, ones, zeros, 16) - O.layer_norm(x))) < 1e-15
+    g, b = rng.standard_normal((3, 32)), rng.standard_normal((3, 32))
+    m = O.adaln(x, g, b, 16)
+    for i in range(3):   # each image uses its own gamma and beta
+        rows = slice(16 * i, 16 * i + 16)
+        ref = torch.nn.functional.layer_norm(torch.from_numpy(x[rows]), (32,), weight=torch.from_numpy(g[i]),
+                                             bias=torch.from_numpy(b[i])).numpy()
+        assert np.max(np.abs(m[rows] - ref)) < 1e-12
+
+
+def test_gated_residual_identity_at_zero_gate():
+    rng = np.random.default_rng(43)
+    x, y = rng.standard_normal((40, 24)), rng.standard_normal((40, 24))
+    assert np.array_equal(O.gated_residual(x, y, np.zeros((5, 24)), 8), x)          # adaLN-Zero at init
+    assert np.max(np.abs(O.gated_residual(np.zeros_like(x), y, np.ones((5, 24)), 8) - y)) == 0
+    a = rng.standard_normal((5, 24))
+    out = O.gated_residual(x, y, a, 8)
+    assert np.max(np.abs(out[17] - (x[17] + a[2] * y[17]))) < 1e-15                 # token 17 is in image 2
+
+
 # ------------------------------------------------------------------ experts
 
 def test_gelu_tanh_matches_library_and_identity():

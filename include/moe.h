@@ -93,6 +93,17 @@ typedef struct {
                         length of the image-patch sequence) */
 } moe_config_t;
 
+/* The adaLN-Zero residual connection around the layer, applied where the
+ * combine writes `out` ("Scalable Diffusion Models with Transformers (DiT)",
+ * DiT block details: a per-sample, per-dimension gate alpha scales each branch
+ * before its residual connection):
+ *     out[t] = x_res[t] + alpha[t / img_len] * MoE(x)[t]   (fp32, rounded once) */
+typedef struct {
+  const void* x_res;   /* [T,D] act: the residual stream entering the block */
+  const void* alpha;   /* [T/img_len, D] act: the gate of each image */
+  int32_t img_len;     /* tokens per image, >= 1, dividing T */
+} moe_residual_t;
+
 /* Library version (major*10000 + minor*100 + patch). */
 int32_t moe_version(void);
 
@@ -202,8 +213,9 @@ int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* 
  * routed tile is stored.
  *   Arguments as moe_expert_gemm2 (no y_sh), plus pos [T,Kmax] and n_sel [T]
  *   (or NULL for top-K) from moe_dispatch / moe_route, and out [T,D] act.
- *   out[t] = sum_k y_perm[pos[t,k]] + sum_j (W2s_j h_sh_j + b2s_j), rounded once.
- * Only for bf16 with gemm_impl AUTO and n_shared >= 1 (MOE_ERR_UNSUPPORTED
+ *   out[t] = sum_k y_perm[pos[t,k]] + sum_j (W2s_j h_sh_j + b2s_j), rounded once;
+ *   with `res` (or NULL), out[t] = x_res[t] + alpha[t/img_len] * (that sum).
+ * Only for bf16 or fp16 with gemm_impl AUTO and n_shared >= 1 (MOE_ERR_UNSUPPORTED
  * otherwise: call moe_expert_gemm2 and moe_combine).  Uses the words at byte
  * offsets 224 and 228 of ws, which must be zero on entry (moe_workspace_init;
  * each launch leaves them zero).  All CTAs of the launch must be resident at
@@ -212,18 +224,20 @@ int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* 
  */
 int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm, const void* h_sh,
                              const void* w2, const void* b2, const void* w2s, const void* b2s, const float* row_gate,
-                             const int32_t* pos, const int32_t* n_sel, void* y_perm, void* out, void* ws,
-                             size_t ws_bytes, void* stream);
+                             const int32_t* pos, const int32_t* n_sel, void* y_perm, const moe_residual_t* res,
+                             void* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_combine -- MoE(x_t) = sum_{k < n_sel[t]} y_perm[pos[t,k]] + y_sh[t]
  * (the gates are already applied in y_perm), summed in fp32 in slot order
  * then the shared term, rounded once to the act type.
  *   y_perm [R_max,D] act; y_sh [T,D] act or NULL (n_s = 0);
- *   pos [T,Kmax] int32; n_sel [T] or NULL (= K); out [T,D] act.
+ *   pos [T,Kmax] int32; n_sel [T] or NULL (= K); out [T,D] act;
+ *   res: the adaLN-Zero residual (out[t] = x_res[t] + alpha[t/img_len] * MoE(x_t)),
+ *   or NULL for MoE(x) alone.
  */
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,
-                const int32_t* pos, const int32_t* n_sel, void* out, void* stream);
+                const int32_t* pos, const int32_t* n_sel, const moe_residual_t* res, void* out, void* stream);
 
 /*
  * moe_route_static -- moe_route for callers that cannot allocate device memory.

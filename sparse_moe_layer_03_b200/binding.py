@@ -29,6 +29,21 @@ class MoeConfig(C.Structure):
                 ("gemm_impl", C.c_int32), ("seq_len", C.c_int32)]
 
 
+class MoeResidual(C.Structure):
+    _fields_ = [("x_res", C.c_void_p), ("alpha", C.c_void_p), ("img_len", C.c_int32)]
+
+
+def make_residual(x_res, alpha, img_len):
+    """adaLN-Zero residual for the combine: out = x_res + alpha[image] * MoE(x); None for MoE(x) alone."""
+    if x_res is None:
+        return None
+    return MoeResidual(_ptr(x_res), _ptr(alpha), img_len)
+
+
+def _res_ref(r):
+    return None if r is None else C.byref(r)
+
+
 class MoeError(RuntimeError):
     def __init__(self, code: int, msg: str):
         super().__init__(f"moe error {code}: {msg}")
@@ -55,11 +70,11 @@ _SIGS = {
     "moe_expert_gemm2": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_expert_mlp": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                  _P, C.c_size_t, _P]),
-    "moe_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
+    "moe_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
     "moe_route_static": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_frequency": (C.c_int, [_CFG, _P, _P, C.c_int32, _P, C.c_int32, _P, _P, _P]),
-    "moe_expert_gemm2_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t,
-                                           _P]),
+    "moe_expert_gemm2_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                           C.c_size_t, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -150,8 +165,9 @@ def moe_expert_mlp(cfg, offsets, x_perm, x, w1, b1, w2, b2, w1s, b1s, w2s, b2s, 
                               _ptr(h_sh), _ptr(y_perm), _ptr(y_sh), _ptr(ws), ws_bytes, stream))
 
 
-def moe_combine(cfg, y_perm, y_sh, pos, n_sel, out, stream=0):
-    _check(lib.moe_combine(C.byref(cfg), _ptr(y_perm), _ptr(y_sh), _ptr(pos), _ptr(n_sel), _ptr(out), stream))
+def moe_combine(cfg, y_perm, y_sh, pos, n_sel, out, stream=0, res=None):
+    _check(lib.moe_combine(C.byref(cfg), _ptr(y_perm), _ptr(y_sh), _ptr(pos), _ptr(n_sel), _res_ref(res), _ptr(out),
+                           stream))
 
 
 def moe_last_error() -> str:
@@ -171,8 +187,8 @@ def moe_expert_frequency(cfg, topk_idx, n_sel, seq_len, seq_labels, n_labels, hi
 
 
 def moe_expert_gemm2_combine(cfg, offsets, h_perm, h_sh, w2, b2, w2s, b2s, row_gate, pos, n_sel, y_perm, out, ws,
-                             ws_bytes, stream=0):
+                             ws_bytes, stream=0, res=None):
     """GEMM2 with the combine folded into the shared experts' tiles: writes out [T,D] directly."""
     _check(lib.moe_expert_gemm2_combine(C.byref(cfg), _ptr(offsets), _ptr(h_perm), _ptr(h_sh), _ptr(w2), _ptr(b2),
                                         _ptr(w2s), _ptr(b2s), _ptr(row_gate), _ptr(pos), _ptr(n_sel), _ptr(y_perm),
-                                        _ptr(out), _ptr(ws), ws_bytes, stream))
+                                        _res_ref(res), _ptr(out), _ptr(ws), ws_bytes, stream))

@@ -404,6 +404,21 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx
 
 namespace {
 
+// adaLN-Zero residual argument: both pointers 16-byte aligned, img_len dividing T
+int check_residual(const moe_config_t* cfg, const moe_residual_t* res) {
+  if (!res) return MOE_OK;
+  if (!res->x_res || !res->alpha) return fail(MOE_ERR_INVALID_ARG, "res->x_res and res->alpha must be set");
+  if (!aligned16(res->x_res) || !aligned16(res->alpha))
+    return fail(MOE_ERR_INVALID_ARG, "res->x_res and res->alpha must be 16-byte aligned");
+  if (res->img_len < 1 || cfg->T % res->img_len)
+    return fail(MOE_ERR_INVALID_ARG, "res->img_len=%d does not divide T=%d", res->img_len, cfg->T);
+  return MOE_OK;
+}
+
+}  // namespace
+
+namespace {
+
 // A0/B0: routed problem (A [rows0, K0], B [brows0, K0]); A1/B1: shared problem
 // (A [rows1, K1], B [brows1, bcols1]; bcols1 < K1 when B is a K-split stack)
 int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long rows0, const void* B0,
@@ -538,7 +553,8 @@ int moe_expert_gemm2(const moe_config_t* cfg, const int32_t* offsets, const void
 int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm,
                              const void* h_sh, const void* w2, const void* b2, const void* w2s,
                              const void* b2s, const float* row_gate, const int32_t* pos, const int32_t* n_sel,
-                             void* y_perm, void* out, void* ws, size_t ws_bytes, void* stream) {
+                             void* y_perm, const moe_residual_t* res, void* out, void* ws, size_t ws_bytes,
+                             void* stream) {
   int rc = validate(cfg);
   if (rc) return rc;
   if (!is16(cfg) || cfg->gemm_impl != MOE_GEMM_AUTO || cfg->n_shared < 1)
@@ -560,6 +576,7 @@ int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, co
   OPTIONAL_PTR(b2s);
   OPTIONAL_PTR(n_sel);
   if (cfg->routing == MOE_ROUTE_RACE && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
+  if ((rc = check_residual(cfg, res))) return rc;
   const int ns = cfg->n_shared;
   const long long R = max_rows(cfg);
   GemmArgs g{};
@@ -580,6 +597,7 @@ int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, co
   g.y_routed = y_perm;
   g.done_ctr = ws_at<unsigned int>(ws, 224);
   g.exit_ctr = ws_at<unsigned int>(ws, 228);
+  if (res) { g.x_res = res->x_res; g.alpha = res->alpha; g.img_len = res->img_len; }
   return run_gemm(cfg, g, h_perm, R, w2, (long long)cfg->E * cfg->D, h_sh, cfg->T, w2s,
                   (long long)ns * cfg->D, cfg->H, ns * cfg->H, cfg->H, ws, (cudaStream_t)stream);
 }
@@ -596,7 +614,7 @@ int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* 
 }
 
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,
-                const int32_t* pos, const int32_t* n_sel, void* out, void* stream) {
+                const int32_t* pos, const int32_t* n_sel, const moe_residual_t* res, void* out, void* stream) {
   int rc = validate(cfg);
   if (rc) return rc;
   if (cfg->T == 0) return ok();
@@ -606,10 +624,12 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,
   OPTIONAL_PTR(n_sel);
   if (cfg->n_shared > 0) REQUIRE_PTR(y_sh);
   if (cfg->routing == MOE_ROUTE_RACE && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
+  if ((rc = check_residual(cfg, res))) return rc;
   CombineArgs ca{};
   ca.y_perm = y_perm; ca.y_sh = cfg->n_shared > 0 ? y_sh : nullptr; ca.pos = pos; ca.n_sel = n_sel;
   ca.out = out; ca.b16 = is16(cfg); ca.f16 = cfg->dtype == MOE_F16;
   ca.T = cfg->T; ca.D = cfg->D; ca.K = cfg->K; ca.Kmax = kmax_of(cfg); ca.r_max = max_rows(cfg);
+  if (res) { ca.x_res = res->x_res; ca.alpha = res->alpha; ca.img_len = res->img_len; }
   cudaError_t e = launch_combine(ca, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "combine kernel");
   return ok();

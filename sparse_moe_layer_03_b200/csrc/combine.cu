@@ -2,7 +2,9 @@
 // ("Scaling Diffusion Transformers to 16 Billion Parameters", "MOE 回顾"
 // eq. MoE(x) and "MOE-DIT" shared experts).  The gates were applied in the
 // second expert GEMM's epilogue, so this is an un-permute and a sum: fp32 in
-// slot order k = 0..n_sel-1, then the shared term, rounded once.
+// slot order k = 0..n_sel-1, then the shared term; with the adaLN-Zero residual
+// ("Scalable Diffusion Models with Transformers (DiT)", DiT block details)
+// out = x_res + alpha_image * that sum; rounded once.
 // HBM-bound: one warp per token, 16-byte loads.
 #include "common.cuh"
 #include "kernels.h"
@@ -33,6 +35,8 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
   const int n8 = a.D / 8;
   const T* yp = reinterpret_cast<const T*>(a.y_perm);
   const T* ys = reinterpret_cast<const T*>(a.y_sh);
+  const T* xr = reinterpret_cast<const T*>(a.x_res);
+  const T* al = reinterpret_cast<const T*>(a.alpha);
   for (int t = blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5); t < a.T; t += nwarps) {
     int ns = a.n_sel ? a.n_sel[t] : a.K;
     ns = ns < 0 ? 0 : (ns > a.Kmax ? a.Kmax : ns);
@@ -55,6 +59,13 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
         load8<T>(ys, (size_t)t * n8 + v, y);
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] += y[q];
+      }
+      if (xr) {   // adaLN-Zero: the residual plus the image's gate times the layer output
+        float r[8], g[8];
+        load8<T>(xr, (size_t)t * n8 + v, r);
+        load8<T>(al, (size_t)(t / a.img_len) * n8 + v, g);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = r[q] + g[q] * acc[q];
       }
       if constexpr (sizeof(T) == 2) {
         const T* tag = nullptr;

@@ -353,8 +353,24 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
               }
             }
 #pragma unroll
-            for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = S::pack2(y[j] + (__uint_as_float(v[j]) + b[j]), y[j + 1] + (__uint_as_float(v[j + 1]) + b[j + 1]));
+            for (int j = 0; j < 32; ++j) y[j] += __uint_as_float(v[j]) + b[j];
+            if (a.x_res != nullptr && rv) {
+              // adaLN-Zero residual: x_res + alpha[image] * (layer output)
+              const uint4* xp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.x_res) +
+                                                               grow * pr.N + col0);
+              const uint4* ap = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.alpha) +
+                                                               (grow / a.img_len) * pr.N + col0);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                float r8[8], g8[8];
+                S::x8_to_f32(__ldg(xp + u), r8);
+                S::x8_to_f32(__ldg(ap + u), g8);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) y[8 * u + j] = r8[j] + g8[j] * y[8 * u + j];
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) ow[j / 2] = S::pack2(y[j], y[j + 1]);
           }
         }
         // stage the 32 x 128-byte box (128-byte swizzle) and store it with TMA; rows past the

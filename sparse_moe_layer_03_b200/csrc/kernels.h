@@ -140,6 +140,9 @@ struct GemmArgs {
   const void* y_routed;     // [r_max, N] act
   unsigned int* done_ctr;   // zero on entry; the launch's last CTA resets both counters
   unsigned int* exit_ctr;
+  const void* x_res;        // adaLN-Zero residual in the epi-2 output: x_res + alpha[t / img_len] * sum, or null
+  const void* alpha;
+  int img_len;
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, int bn,
                            int num_sms, cudaStream_t s);
@@ -155,6 +158,9 @@ struct CombineArgs {
   void* out; int b16, f16;
   int T, D, K, Kmax;
   long long r_max;
+  const void* x_res;        // adaLN-Zero residual: out = x_res + alpha[t / img_len] * MoE, or null
+  const void* alpha;
+  int img_len;
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 

@@ -115,25 +115,35 @@ class MoELayer:
         B.moe_expert_gemm2(self.cfg, self.offsets, self.h_perm, self.h_sh, self.w2, self.b2, self.ws2, self.bs2,
                            self.row_gate, self.y_perm, self.y_sh, self.ws, self.ws_bytes, self.stream())
 
-    def combine(self):
-        B.moe_combine(self.cfg, self.y_perm, self.y_sh, self.pos, self.n_sel, self.out, self.stream())
+    def combine(self, res=None):
+        B.moe_combine(self.cfg, self.y_perm, self.y_sh, self.pos, self.n_sel, self.out, self.stream(), res=res)
 
-    def gemm2_combine(self):
+    def gemm2_combine(self, res=None):
         B.moe_expert_gemm2_combine(self.cfg, self.offsets, self.h_perm, self.h_sh, self.w2, self.b2, self.ws2,
                                    self.bs2, self.row_gate, self.pos, self.n_sel, self.y_perm, self.out, self.ws,
-                                   self.ws_bytes, self.stream())
+                                   self.ws_bytes, self.stream(), res=res)
 
-    def forward(self, x: torch.Tensor) -> torch.Tensor:
-        """Whole layer on device-resident x [T,D]; returns the output buffer."""
+    def forward(self, x: torch.Tensor, x_res: Optional[torch.Tensor] = None, alpha: Optional[torch.Tensor] = None,
+                img_len: Optional[int] = None) -> torch.Tensor:
+        """Whole layer on device-resident x [T,D]; returns the output buffer.
+
+        With ``x_res`` [T,D] and ``alpha`` [T/img_len, D] (act dtype) the output is the adaLN-Zero
+        residual x_res + alpha[image] * MoE(x), applied where the combine writes it.
+        """
         assert x.shape == (self.cfg.T, self.s.D) and x.dtype == self.act_dtype and x.is_contiguous()
+        res = None
+        if x_res is not None:
+            assert x_res.shape == x.shape and x_res.dtype == x.dtype and x_res.is_contiguous()
+            assert alpha.dtype == x.dtype and alpha.is_contiguous() and alpha.shape == (self.cfg.T // img_len, self.s.D)
+            res = B.make_residual(x_res, alpha, img_len)
         self.route(x)
         self.dispatch(x)
         self.gemm1(x)
         if self.fused:
-            self.gemm2_combine()
+            self.gemm2_combine(res)
         else:
             self.gemm2()
-            self.combine()
+            self.combine(res)
         return self.out
 
     def expert_frequency(self, seq_len: int, seq_labels: Optional[torch.Tensor] = None,

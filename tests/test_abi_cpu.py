@@ -61,8 +61,14 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
     n = B.moe_workspace_size(race)
     rc = B.lib.moe_route(ctypes.byref(race), fake, fake, None, fake, fake, None, fake, fake, fake, n, None)
     assert rc == B.MOE_ERR_INVALID_ARG and b"n_sel" in B.lib.moe_last_error()
-    rc = B.lib.moe_combine(ctypes.byref(race), fake, fake, fake, None, fake, None)
+    rc = B.lib.moe_combine(ctypes.byref(race), fake, fake, fake, None, None, fake, None)
     assert rc == B.MOE_ERR_INVALID_ARG
+    # adaLN-Zero residual: img_len must divide T, pointers set and aligned
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    for res, word in [(B.MoeResidual(fake, fake, 300), b"img_len"), (B.MoeResidual(fake, None, 256), b"alpha"),
+                      (B.MoeResidual(fake + 2, fake, 256), b"aligned")]:
+        rc = B.lib.moe_combine(ctypes.byref(cfg), fake, fake, fake, None, ctypes.byref(res), fake, None)
+        assert rc == B.MOE_ERR_INVALID_ARG and word in B.lib.moe_last_error()
 
 
 def test_frequency_arguments_rejected_before_launch():
@@ -92,9 +98,31 @@ def test_fused_combine_refuses_unsupported_configs_before_launch():
                      (B.make_config(1024, 384, 1536, 8, 2, 0), b"n_shared"),
                      (B.make_config(1024, 384, 1536, 8, 2, 2, gemm_impl="tc1"), b"AUTO")]:
         n = B.moe_workspace_size(cfg)
-        rc = f(ctypes.byref(cfg), fake, fake, fake, fake, None, fake, None, fake, fake, None, fake, fake, fake, n, None)
+        rc = f(ctypes.byref(cfg), fake, fake, fake, fake, None, fake, None, fake, fake, None, fake, None, fake, fake, n,
+               None)
         assert rc == B.MOE_ERR_UNSUPPORTED and why in B.lib.moe_last_error()
     cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
     n = B.moe_workspace_size(cfg)
-    rc = f(ctypes.byref(cfg), fake, fake, fake, fake, None, fake, None, fake, None, None, fake, fake, fake, n, None)
+    rc = f(ctypes.byref(cfg), fake, fake, fake, fake, None, fake, None, fake, None, None, fake, None, fake, fake, n, None)
     assert rc == B.MOE_ERR_INVALID_ARG and b"pos" in B.lib.moe_last_error()
+
+
+def test_python_wrappers_reach_the_library():
+    # every wrapper marshals its arguments and reaches the C ABI (which then fails without a GPU,
+    # or on the fake pointers, with its own error code rather than a Python TypeError)
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    n = B.moe_workspace_size(cfg)
+    f = 1 << 40
+    res = B.make_residual(f, f, 256)
+    calls = [
+        lambda: B.moe_route(cfg, f, f, None, f, f, f, f, f, f, n),
+        lambda: B.moe_dispatch(cfg, f, f, f, f, f, f, f, f, f, f, n),
+        lambda: B.moe_expert_gemm1(cfg, f, f, f, f, None, f, None, f, f, f, n),
+        lambda: B.moe_expert_gemm2(cfg, f, f, f, f, None, f, None, f, f, f, f, n),
+        lambda: B.moe_expert_gemm2_combine(cfg, f, f, f, f, None, f, None, f, f, None, f, f, f, n, res=res),
+        lambda: B.moe_combine(cfg, f, f, f, None, f, res=res),
+        lambda: B.moe_expert_frequency(cfg, f, None, 256, None, 256, f, f),
+    ]
+    for c in calls:
+        with pytest.raises(B.MoeError):
+            c()

@@ -219,3 +219,42 @@ def test_f16_full_size_xl():
     w = dataclasses.replace(I.WORKLOADS["xl2_8e2a_512"], dtype="f16", name="DiT-MoE-XL/2-8E2A layer at 512x512, fp16")
     inp = I.make_inputs(w)
     PA.full_check(w, inp, tokens=PA.sample_tokens(w.T, 512))
+
+
+RESIDUAL_CASES = [  # T, D, H, E, K, n_s, dtype, routing, img_len, fuse
+    (1024, 256, 512, 8, 2, 2, "bf16", "topk", 256, True),
+    (1024, 256, 512, 8, 2, 2, "bf16", "topk", 256, False),
+    (900, 320, 640, 16, 3, 1, "bf16", "race", 300, True),
+    (999, 128, 256, 4, 1, 0, "bf16", "topk", 333, True),     # n_s = 0: the separate combine applies it
+    (1000, 256, 512, 8, 2, 2, "f16", "topk", 250, True),
+]
+
+
+@pytest.mark.parametrize("case", RESIDUAL_CASES,
+                         ids=lambda c: "T%d_E%d_K%d_ns%d_%s_%s_L%d_%s" % (c[0], c[3], c[4], c[5], c[6], c[7], c[8],
+                                                                         "fused" if c[9] else "separate"))
+def test_adaln_zero_residual_in_combine(case):
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    T, D, H, E, K, ns, dt, routing, L_img, fuse = case
+    w = I.small_workload(T, D, H, E, K, ns, dt, routing, seed=5 + T + E)
+    inp = I.make_inputs(w, bias_std=0.2)
+    rng = np.random.default_rng(T)
+    x_res = I._store(rng.standard_normal((T, D)), dt)
+    alpha = I._store(rng.standard_normal((T // L_img, D)) * 0.5, dt)
+    L = MoELayer(LayerShape(T, D, H, E, K, ns, dt, routing, w.alpha, fuse_combine=fuse), inp, "cuda:0")
+    dev = lambda a: torch.as_tensor(a).to(device="cuda:0", dtype=L.act_dtype).contiguous()
+    L.forward(dev(inp["x"]), dev(x_res), dev(alpha), L_img)
+    torch.cuda.synchronize()
+    L.check()
+    r = PA.fetch(L)
+    P = O.softmax_scores(O.gate_logits(inp["x"], inp["wg"], inp.get("router_bias")))
+    PA.check_routing(w, P, r)
+    idx = PA.gpu_selection(r)
+    g = np.where(idx >= 0, np.take_along_axis(P, np.maximum(idx, 0), axis=1), 0.0)
+    ref = O.gated_residual(x_res, O.layer_output(inp, idx, g), alpha, L_img)
+    err = PA.rel_err(r["out"], ref)
+    assert err <= PA.out_tol(w), err
+    # a zero gate leaves the residual stream unchanged (adaLN-Zero at initialisation)
+    L.forward(dev(inp["x"]), dev(x_res), torch.zeros_like(dev(alpha)), L_img)
+    torch.cuda.synchronize()
+    assert torch.equal(L.out, dev(x_res))

@@ -181,6 +181,7 @@ def calibrated_tokens(w: I.Workload, inp: dict, target_s: float) -> int:
 
 def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     import torch
+    from sparse_moe_layer_03_b200 import binding as B
     from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
 
     device = torch.device("cuda", local)
@@ -208,8 +209,20 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     # with the combine folded into GEMM2 (bf16, n_s >= 1) the step has four stages
     stages = (["route", "dispatch", "gemm1", "gemm2_combine"] if L.fused
               else ["route", "dispatch", "gemm1", "gemm2", "combine"])
-    calls = {"route": lambda: L.route(x), "dispatch": lambda: L.dispatch(x), "gemm1": lambda: L.gemm1(x),
-             "gemm2": L.gemm2, "combine": L.combine, "gemm2_combine": L.gemm2_combine}
+    mod = res = None
+    x_in = x
+    if args.adaln == "on":
+        # per-image adaLN parameters (the synthetic conditioning of the workload's images)
+        g = torch.Generator().manual_seed(w.seed + 77)
+        nimg = w.T // w.tokens_per_image
+        per_img = lambda scale, shift: (torch.randn((nimg, w.D), generator=g) * scale + shift).to(dt).to(device)
+        gamma, beta, alpha = per_img(0.3, 1.0), per_img(0.3, 0.0), per_img(0.5, 0.0)
+        L.x_mod = torch.empty_like(x)
+        mod = B.make_adaln(gamma, beta, w.tokens_per_image, 1e-5, L.x_mod)
+        res = B.make_residual(x, alpha, w.tokens_per_image)
+        x_in = L.x_mod
+    calls = {"route": lambda: L.route(x, mod), "dispatch": lambda: L.dispatch(x_in), "gemm1": lambda: L.gemm1(x_in),
+             "gemm2": L.gemm2, "combine": lambda: L.combine(res), "gemm2_combine": lambda: L.gemm2_combine(res)}
 
     def step(events):
         for i, s in enumerate(stages):
@@ -334,6 +347,8 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
         "config": {"workload": w.name, "T": w.T, "D": w.D, "H": w.H, "E": w.E, "K": w.K, "n_shared": w.n_shared,
                    "routing": w.routing, "batch": w.batch, "tokens_per_image": w.tokens_per_image,
                    "global_batch_tokens": total_tokens, "parallelism": f"dp{world}" if world > 1 else "single",
+                   "adaln": ("modulation in the router and the gated residual in the combine (e2e: the plain "
+                             "layer)") if args.adaln == "on" else "off",
                    "l2": "flushed between steps (256 MB write, then a 0.2 ms GPU sleep so the host is ahead; both "
                          "outside each step's events)"},
         "layer_tflops": round(M.gemm_flops(w.T, w.D, w.H, w.K, w.n_shared) / (ms_per_step * 1e-3) / 1e12, 1),
@@ -397,6 +412,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--fuse-combine", default="on", choices=["on", "off"],
                     help="fold the combine into the shared experts' GEMM2 (bf16, n_s >= 1)")
+    ap.add_argument("--adaln", default="off", choices=["on", "off"],
+                    help="time the layer inside its DiT block: adaLN modulation in the router and the "
+                         "adaLN-Zero gated residual in the combine (per-image gamma, beta, alpha)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -104,6 +104,21 @@ typedef struct {
   int32_t img_len;     /* tokens per image, >= 1, dividing T */
 } moe_residual_t;
 
+/* adaLN modulation of the layer input, applied inside moe_route
+ * ("Diffusion Transformer (DiT) 技术全景解析" 2.2.3, AdaLN: a plain layer_norm
+ * over the features, then a per-sample scale gamma and shift beta):
+ *     m[t] = gamma[t / img_len] * (x[t] - mean) / sqrt(var + eps) + beta[t / img_len]
+ * The router routes on m and writes it to x_mod, rounded to the act type;
+ * moe_dispatch and the shared experts' GEMM1 then take x_mod as their x.
+ * 16-bit types only. */
+typedef struct {
+  const void* gamma;   /* [T/img_len, D] act */
+  const void* beta;    /* [T/img_len, D] act */
+  int32_t img_len;     /* tokens per image, >= 1, dividing T */
+  float eps;           /* > 0; the pages' layer_norm uses the library default 1e-5 */
+  void* x_mod;         /* [T, D] act out: m */
+} moe_adaln_t;
+
 /* Library version (major*10000 + minor*100 + patch). */
 int32_t moe_version(void);
 
@@ -142,13 +157,14 @@ int moe_check_status(void* ws, void* stream);
  *   counts      [E] int32 out   sum_t I(t,i)
  *   aux_loss    [1] fp32 out    L_balance with T = this call's tokens (seq_len = 0), or the
  *               mean over images of L_balance with T = seq_len tokens per image
+ *   mod         adaLN modulation of x before routing (see moe_adaln_t), or NULL
  * Race selection: the S = K*T largest scores of the flattened T x E matrix,
  * ties to the lower flat index t*E+i, found by an exact radix select on the
  * fp32 score bits.
  */
 int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
               int32_t* topk_idx, float* topk_w, int32_t* n_sel, int32_t* counts, float* aux_loss,
-              void* ws, size_t ws_bytes, void* stream);
+              const moe_adaln_t* mod, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_dispatch -- permute tokens into expert-contiguous order (only the
@@ -243,7 +259,8 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,
  * moe_route_static -- moe_route for callers that cannot allocate device memory.
  * (No counterpart on the pages: this is a deployment convenience.)
  *
- * Same arguments, results and errors as moe_route, minus the workspace: the
+ * Same arguments, results and errors as moe_route, minus the workspace and the
+ * adaLN modulation (it routes on x as given): the
  * router's scratch comes from a fixed 4 MiB array built into the library
  * (reserved on every GPU that loads it, until the process exits), so a caller
  * whose framework gives it no allocator, or that must not call cudaMalloc

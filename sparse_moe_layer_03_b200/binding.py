@@ -29,6 +29,18 @@ class MoeConfig(C.Structure):
                 ("gemm_impl", C.c_int32), ("seq_len", C.c_int32)]
 
 
+class MoeAdaln(C.Structure):
+    _fields_ = [("gamma", C.c_void_p), ("beta", C.c_void_p), ("img_len", C.c_int32), ("eps", C.c_float),
+                ("x_mod", C.c_void_p)]
+
+
+def make_adaln(gamma, beta, img_len, eps, x_mod):
+    """adaLN modulation done by the router: x_mod = gamma[image] * LayerNorm(x) + beta[image]; None for none."""
+    if gamma is None:
+        return None
+    return MoeAdaln(_ptr(gamma), _ptr(beta), img_len, eps, _ptr(x_mod))
+
+
 class MoeResidual(C.Structure):
     _fields_ = [("x_res", C.c_void_p), ("alpha", C.c_void_p), ("img_len", C.c_int32)]
 
@@ -64,7 +76,7 @@ _SIGS = {
     "moe_max_rows": (C.c_int64, [_CFG]),
     "moe_workspace_init": (C.c_int, [_P, C.c_size_t, _P]),
     "moe_check_status": (C.c_int, [_P, _P]),
-    "moe_route": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "moe_route": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_dispatch": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_expert_gemm1": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_expert_gemm2": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
@@ -135,9 +147,9 @@ def moe_check_status(ws, stream=0):
     _check(lib.moe_check_status(_ptr(ws), stream))
 
 
-def moe_route(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, aux_loss, ws, ws_bytes, stream=0):
+def moe_route(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, aux_loss, ws, ws_bytes, stream=0, mod=None):
     _check(lib.moe_route(C.byref(cfg), _ptr(x), _ptr(wg), _ptr(router_bias), _ptr(topk_idx), _ptr(topk_w),
-                         _ptr(n_sel), _ptr(counts), _ptr(aux_loss), _ptr(ws), ws_bytes, stream))
+                         _ptr(n_sel), _ptr(counts), _ptr(aux_loss), _res_ref(mod), _ptr(ws), ws_bytes, stream))
 
 
 def moe_dispatch(cfg, x, topk_idx, topk_w, n_sel, offsets, pos, row_token, row_gate, x_perm, ws, ws_bytes,

@@ -245,7 +245,7 @@ int moe_check_status(void* ws, void* stream) {
 
 int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
               int32_t* topk_idx, float* topk_w, int32_t* n_sel, int32_t* counts, float* aux_loss,
-              void* ws, size_t ws_bytes, void* stream) {
+              const moe_adaln_t* mod, void* ws, size_t ws_bytes, void* stream) {
   int rc = validate(cfg);
   if (rc) return rc;
   const bool race = cfg->routing == MOE_ROUTE_RACE;
@@ -266,6 +266,15 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   OPTIONAL_PTR(router_bias);
   OPTIONAL_PTR(n_sel);
   if (race && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
+  if (mod) {
+    if (!is16(cfg)) return fail(MOE_ERR_UNSUPPORTED, "adaLN modulation in the router needs a 16-bit act type");
+    REQUIRE_PTR(mod->gamma);
+    REQUIRE_PTR(mod->beta);
+    REQUIRE_PTR(mod->x_mod);
+    if (mod->img_len < 1 || cfg->T % mod->img_len)
+      return fail(MOE_ERR_INVALID_ARG, "mod->img_len=%d does not divide T=%d", mod->img_len, cfg->T);
+    if (!(mod->eps > 0.f) || mod->eps > 1.f) return fail(MOE_ERR_INVALID_ARG, "mod->eps=%g outside (0, 1]", mod->eps);
+  }
   const WsLayout L = ws_layout(cfg);
   const int sms = num_sms_current();
   int tile = 0, threads = 0;
@@ -275,10 +284,20 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   const int grid = ntiles < sms ? ntiles : sms;
   // partial sums: one row per CTA (16-bit kernel) or per token tile (fp32 kernel)
   const int nparts = b16 ? grid : ntiles;
-  CUtensorMap tm;
+  CUtensorMap tm, tmm;
   int tmap3d = 0;
   if (b16 && make_tmap_rows3d(&tm, x, cfg->dtype, cfg->T, cfg->D, tile)) tmap3d = 1;
   else if ((rc = make_tmap(&tm, x, cfg->dtype, cfg->T, cfg->D, tile, "x"))) return rc;
+  // the modulated rows go out with the same box geometry as x comes in
+  tmm = tm;
+  if (mod) {
+    if (tmap3d) {
+      if (!make_tmap_rows3d(&tmm, mod->x_mod, cfg->dtype, cfg->T, cfg->D, tile))
+        return fail(MOE_ERR_CUDA, "tensor map for mod->x_mod failed");
+    } else if ((rc = make_tmap(&tmm, mod->x_mod, cfg->dtype, cfg->T, cfg->D, tile, "x_mod"))) {
+      return rc;
+    }
+  }
   RouteArgs ra{};
   ra.tmap3d = tmap3d;
   ra.x = x; ra.wg = wg; ra.bias = router_bias;
@@ -298,6 +317,7 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   ra.tile_counts = ws_at<int32_t>(ws, L.tile_counts);
   ra.tile_psum = ws_at<float>(ws, L.tile_psum);
   ra.status = status_ptr(ws);
+  if (mod) { ra.gamma = mod->gamma; ra.beta = mod->beta; ra.img_len = mod->img_len; ra.eps = mod->eps; }
   FinalizeArgs fa{};
   fa.T = cfg->T; fa.E = cfg->E; fa.K = cfg->K; fa.alpha = cfg->alpha;
   fa.counts = counts; fa.aux_loss = aux_loss;
@@ -306,7 +326,7 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   fa.ctr = ws_at<unsigned int>(ws, 64);
   if (!race) {
     // the router's last block finalizes counts and loss
-    if ((e = launch_route(ra, fa, &tm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
+    if ((e = launch_route(ra, fa, &tm, &tmm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
     if (per_image && (e = launch_seq_loss(sl, s)) != cudaSuccess) return cuda_fail(e, "per-image loss kernel");
     return ok();
   }
@@ -315,7 +335,7 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   ra.zero = ws_at<uint32_t>(ws, L.race_sync);
   ra.nzero = kRaceSyncWords;
   FinalizeArgs none{};
-  if ((e = launch_route(ra, none, &tm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
+  if ((e = launch_route(ra, none, &tm, &tmm, s)) != cudaSuccess) return cuda_fail(e, "route kernel");
   RaceArgs rr{};
   rr.P = ra.P; rr.T = cfg->T; rr.E = cfg->E; rr.K = cfg->K;
   rr.sync = ra.zero;

@@ -30,6 +30,12 @@ struct RouteArgs {
   float* tile_psum;         // [ntiles,E]
   uint32_t* zero;           // block 0 clears zero[0, nzero) first (the Expert-Race scratch), or null
   int nzero;
+  // adaLN modulation (16-bit router only): the router routes on
+  // m = gamma[t / img_len] * LayerNorm(x_t) + beta[t / img_len] and stores m through tmap_m
+  const void* gamma;        // [T/img_len, D] act, or null (route on x itself)
+  const void* beta;
+  int img_len;
+  float eps;
   int* status;
 };
 size_t route_smem_bytes(int D, int E, int tile_rows, int b16);
@@ -45,7 +51,8 @@ struct FinalizeArgs {
   int32_t* counts; float* aux_loss;   // counts == null: the router leaves finalizing to a later kernel
   unsigned int* ctr;                  // blocks-done counter in ws (zero between calls)
 };
-cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tmap_x, cudaStream_t s);
+cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tmap_x,
+                         const CUtensorMap* tmap_m, cudaStream_t s);
 
 // per-image balance loss (seq_len > 0): overwrites aux_loss with the mean over images
 struct SeqLossArgs {

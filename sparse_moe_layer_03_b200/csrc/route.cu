@@ -13,6 +13,7 @@
 // fp32 inputs use FFMA.  Per-tile partial counts and score sums are reduced in
 // a fixed order, so the loss is bit-reproducible.
 #include <cuda.h>
+#include <type_traits>
 #include "common.cuh"
 #include "kernels.h"
 
@@ -189,6 +190,81 @@ __host__ __device__ inline MmaSmem mma_layout(int D, int E) {
   return L;
 }
 
+// adaLN modulation of one row block held in a warp's two stages, in place:
+// m = gamma_b * (x - mean) / sqrt(var + eps) + beta_b for token t of image
+// b = t / img_len ("Diffusion Transformer (DiT) 技术全景解析" 2.2.3, AdaLN: a
+// plain layer_norm over the features, then the per-sample scale and shift).
+// Lane l takes row l % 16 of half l / 16 (two lanes per row); the row's mean
+// and then its sum of squared deviations are formed over both halves (two
+// passes over shared memory), and each 16-byte chunk is rewritten with its
+// logical columns read through the 128-byte swizzle.
+template <bool F16>
+__device__ __forceinline__ void route_modulate(const RouteArgs& a, uint8_t* xs, int stage_bytes, int w, int hc,
+                                               int nchunks, int rb, int lane) {
+  using S = typename std::conditional<F16, StoreF16, StoreBF16>::type;
+  const int r = lane & 15, p = lane >> 4;
+  const int z0 = p * hc;
+  const int nb = (nchunks - z0) < hc ? (nchunks - z0) : hc;
+  const uint32_t base = smem_u32(xs + (size_t)(2 * w + p) * stage_bytes) + r * 128;
+  const int D = a.D;
+  float s = 0.f;
+  for (int cb = 0; cb < nb; ++cb) {
+#pragma unroll
+    for (int pj = 0; pj < 8; ++pj) {
+      uint4 v;
+      asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "r"(base + cb * (kMmaRB * 128) + pj * 16));
+      float f[8];
+      S::x8_to_f32(v, f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) s += f[q];
+    }
+  }
+  s += __shfl_xor_sync(0xffffffffu, s, 16);
+  const float mu = s / (float)D;
+  float ss = 0.f;
+  for (int cb = 0; cb < nb; ++cb) {
+#pragma unroll
+    for (int pj = 0; pj < 8; ++pj) {
+      uint4 v;
+      asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "r"(base + cb * (kMmaRB * 128) + pj * 16));
+      float f[8];
+      S::x8_to_f32(v, f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ss += (f[q] - mu) * (f[q] - mu);
+    }
+  }
+  ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+  const float rstd = rsqrtf(ss / (float)D + a.eps);
+  const int tok = rb * kMmaRB + r;
+  if (tok >= a.T) return;                           // rows past T stay zero (the store clips them)
+  const int img = tok / a.img_len;
+  const uint4* gp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.gamma) + (size_t)img * D);
+  const uint4* bp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.beta) + (size_t)img * D);
+  for (int cb = 0; cb < nb; ++cb) {
+#pragma unroll
+    for (int pj = 0; pj < 8; ++pj) {
+      const uint32_t addr = base + cb * (kMmaRB * 128) + pj * 16;
+      const int c8 = (z0 + cb) * 8 + (pj ^ (r & 7));   // logical 8-column chunk of this row
+      uint4 v;
+      asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "r"(addr));
+      float f[8], g[8], b[8];
+      S::x8_to_f32(v, f);
+      S::x8_to_f32(__ldg(gp + c8), g);
+      S::x8_to_f32(__ldg(bp + c8), b);
+      uint4 o;
+      o.x = S::pack2(g[0] * ((f[0] - mu) * rstd) + b[0], g[1] * ((f[1] - mu) * rstd) + b[1]);
+      o.y = S::pack2(g[2] * ((f[2] - mu) * rstd) + b[2], g[3] * ((f[3] - mu) * rstd) + b[3]);
+      o.z = S::pack2(g[4] * ((f[4] - mu) * rstd) + b[4], g[5] * ((f[5] - mu) * rstd) + b[5]);
+      o.w = S::pack2(g[6] * ((f[6] - mu) * rstd) + b[6], g[7] * ((f[7] - mu) * rstd) + b[7]);
+      asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w)
+                   : "memory");
+    }
+  }
+}
+
 // The last block to finish turns the per-block partials into counts and the loss.
 // Warp w reduces experts w, w + nwarps, ...: its lanes stride over the tiles
 // (independent loads), then a fixed xor tree; a fixed expert order for the
@@ -245,7 +321,8 @@ __device__ bool last_block_done(unsigned int* ctr) {
 
 template <int EMAX, bool F16>
 __global__ void __launch_bounds__(kMmaMaxConsumers * 32, 1)
-route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, FinalizeArgs fin) {
+route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_m, RouteArgs a,
+                 FinalizeArgs fin) {
   constexpr int NT = EMAX / 8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -305,6 +382,7 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
 #pragma unroll
   for (int e = 0; e < EMAX; ++e) psum[e] = 0.f;
   bool ok = true;
+  const bool modulate = a.gamma != nullptr;
   float* logit_w = reinterpret_cast<float*>(smem + L.logits) + (size_t)w * kMmaRB * EMAX;
   const uint32_t wg_base = smem_u32(wg_s);
   const int li = lane >> 3, lj = lane & 7;
@@ -318,9 +396,30 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc4[g][nt][q] = 0.f;
+    if (modulate) {
+      // both halves of the row block, then m in place; m goes out to x_mod while the MMAs read it
+      for (int h = 0; h < 2 && ok; ++h)
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[2 * w + h]), k & 1, nullptr, a.status, 103));
+      if (!ok) break;
+      route_modulate<F16>(a, xs, stage_bytes, w, hc, nchunks, rb, lane);
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t src = smem_u32(xs + (size_t)(2 * w + h) * stage_bytes);
+          if (a.tmap3d) {
+            tma_store_3d(&tmap_m, src, 0, rb * kMmaRB, h * hc);
+          } else {
+            const int nbh = (nchunks - h * hc) < hc ? (nchunks - h * hc) : hc;
+            for (int c = 0; c < nbh; ++c) tma_store_2d(&tmap_m, src + c * (kMmaRB * 128), (h * hc + c) * 64, rb * kMmaRB);
+          }
+        }
+        bulk_commit();
+      }
+    }
     for (int h = 0; h < 2; ++h) {
       const int st = 2 * w + h;
-      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), k & 1, nullptr, a.status, 100));
+      if (!modulate) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), k & 1, nullptr, a.status, 100));
       if (!ok) break;
       const uint32_t buf = smem_u32(xs + (size_t)st * stage_bytes);
       const int z0 = h * hc;
@@ -351,6 +450,7 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
       }
       __syncwarp();                                  // every lane is done reading the stage
       if (lane == 0 && j + NC < my_rb) {             // refill it with the next row block's half
+        if (modulate) bulk_wait_read_all();          // the x_mod store has read the stage
         fence_async_shared();
         issue(j + NC, h);
       }
@@ -381,6 +481,7 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Finali
     }
     __syncwarp();
   }
+  if (modulate && lane == 0) bulk_wait_all();       // x_mod stores complete before the stages are reused
   __syncthreads();
   tile_partials<EMAX>(psum, blockIdx.x, a, cnt_s, wsum_s);
   if (!ok) set_status(a.status, DEV_TIMEOUT, 102);
@@ -500,7 +601,8 @@ size_t route_smem_total(int D, int E, int tile_rows, int b16) {
 
 int route_mma_stages(int D, int E) { return mma_layout(D, E).consumers; }
 
-cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tm, cudaStream_t s) {
+cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tm, const CUtensorMap* tmm,
+                         cudaStream_t s) {
   const size_t smem = route_smem_total(a.D, a.E, a.tile_rows, a.b16);
   cudaError_t err;
   if (a.b16) {
@@ -508,7 +610,7 @@ cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUte
   if (a.E <= EM && (a.f16 != 0) == F) {                                                                 \
     err = cudaFuncSetAttribute(route_kernel_mma<EM, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (err != cudaSuccess) return err;                                                                 \
-    route_kernel_mma<EM, F><<<a.grid, mma_layout(a.D, a.E).consumers * 32, smem, s>>>(*tm, a, fin);       \
+    route_kernel_mma<EM, F><<<a.grid, mma_layout(a.D, a.E).consumers * 32, smem, s>>>(*tm, *tmm, a, fin); \
     return cudaGetLastError();                                                                          \
   }
     MOE_ROUTE_MMA(8, false)

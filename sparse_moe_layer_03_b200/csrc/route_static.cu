@@ -71,7 +71,7 @@ extern "C" int moe_route_static(const moe_config_t* cfg, const void* x, const vo
                                 float* aux_loss, void* stream) {
   const size_t need = moe_workspace_size(cfg);
   if (need == 0)   // invalid configuration: moe_route reports the same code and message, launching nothing
-    return moe_route(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, aux_loss, nullptr, 0, stream);
+    return moe_route(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, aux_loss, nullptr, nullptr, 0, stream);
   if (need > kStaticScratchBytes) {
     char msg[200];
     snprintf(msg, sizeof(msg),
@@ -87,6 +87,6 @@ extern "C" int moe_route_static(const moe_config_t* cfg, const void* x, const vo
   // status word and blocks-done counter must start at zero on every call
   rc = moe_workspace_init(ws, kStaticScratchBytes, stream);
   if (rc != MOE_OK) return rc;
-  return moe_route(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, aux_loss, ws, kStaticScratchBytes,
-                   stream);
+  return moe_route(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, aux_loss, nullptr, ws,
+                   kStaticScratchBytes, stream);
 }

@@ -99,9 +99,9 @@ class MoELayer:
         return torch.cuda.current_stream(self.device).cuda_stream
 
     # ------------------------------------------------------------ the four calls
-    def route(self, x: torch.Tensor):
+    def route(self, x: torch.Tensor, mod=None):
         B.moe_route(self.cfg, x, self.wg, self.router_bias, self.topk_idx, self.topk_w, self.n_sel, self.counts,
-                    self.aux, self.ws, self.ws_bytes, self.stream())
+                    self.aux, self.ws, self.ws_bytes, self.stream(), mod=mod)
 
     def dispatch(self, x: torch.Tensor):
         B.moe_dispatch(self.cfg, x, self.topk_idx, self.topk_w, self.n_sel, self.offsets, self.pos,
@@ -124,21 +124,35 @@ class MoELayer:
                                    self.ws_bytes, self.stream(), res=res)
 
     def forward(self, x: torch.Tensor, x_res: Optional[torch.Tensor] = None, alpha: Optional[torch.Tensor] = None,
-                img_len: Optional[int] = None) -> torch.Tensor:
+                img_len: Optional[int] = None, gamma: Optional[torch.Tensor] = None,
+                beta: Optional[torch.Tensor] = None, eps: float = 1e-5) -> torch.Tensor:
         """Whole layer on device-resident x [T,D]; returns the output buffer.
 
-        With ``x_res`` [T,D] and ``alpha`` [T/img_len, D] (act dtype) the output is the adaLN-Zero
-        residual x_res + alpha[image] * MoE(x), applied where the combine writes it.
+        adaLN-Zero around the layer (all per-image tensors [T/img_len, D], act dtype):
+        ``gamma``/``beta`` make the router route on m = gamma * LayerNorm(x) + beta (written to
+        ``self.x_mod``, which dispatch and the shared GEMM1 then read); ``alpha`` makes the output
+        x_res + alpha * MoE(m), with x_res = x unless given.
         """
         assert x.shape == (self.cfg.T, self.s.D) and x.dtype == self.act_dtype and x.is_contiguous()
+        per_image = (self.cfg.T // img_len, self.s.D) if img_len else None
+        mod = None
+        x_in = x
+        if gamma is not None:
+            for t in (gamma, beta):
+                assert t.dtype == x.dtype and t.is_contiguous() and t.shape == per_image
+            if getattr(self, "x_mod", None) is None or self.x_mod.shape != x.shape:
+                self.x_mod = torch.empty_like(x)
+            mod = B.make_adaln(gamma, beta, img_len, eps, self.x_mod)
+            x_in = self.x_mod
         res = None
-        if x_res is not None:
+        if alpha is not None:
+            x_res = x if x_res is None else x_res
             assert x_res.shape == x.shape and x_res.dtype == x.dtype and x_res.is_contiguous()
-            assert alpha.dtype == x.dtype and alpha.is_contiguous() and alpha.shape == (self.cfg.T // img_len, self.s.D)
+            assert alpha.dtype == x.dtype and alpha.is_contiguous() and alpha.shape == per_image
             res = B.make_residual(x_res, alpha, img_len)
-        self.route(x)
-        self.dispatch(x)
-        self.gemm1(x)
+        self.route(x, mod)
+        self.dispatch(x_in)
+        self.gemm1(x_in)
         if self.fused:
             self.gemm2_combine(res)
         else:

@@ -40,7 +40,7 @@ def test_invalid_config_is_rejected_on_host(field, value, code):
     cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
     setattr(cfg, field, value)
     assert B.lib.moe_workspace_size(ctypes.byref(cfg)) == 0
-    rc = B.lib.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None, 0, None)
+    rc = B.lib.moe_route(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None, None, 0, None)
     assert rc == code
     assert B.lib.moe_last_error()
 
@@ -49,17 +49,17 @@ def test_null_and_misaligned_pointers_rejected_before_launch():
     cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
     n = B.moe_workspace_size(cfg)
     fake = 1 << 40                          # never dereferenced: validation fails first
-    rc = B.lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, None, fake, n, None)
+    rc = B.lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, None, None, fake, n, None)
     assert rc == B.MOE_ERR_INVALID_ARG and b"aux_loss" in B.lib.moe_last_error()
-    rc = B.lib.moe_route(ctypes.byref(cfg), fake + 8, fake, None, fake, fake, None, fake, fake, fake, n, None)
+    rc = B.lib.moe_route(ctypes.byref(cfg), fake + 8, fake, None, fake, fake, None, fake, fake, None, fake, n, None)
     assert rc == B.MOE_ERR_INVALID_ARG and b"aligned" in B.lib.moe_last_error()
-    rc = B.lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, fake, fake, n - 256, None)
+    rc = B.lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, fake, None, fake, n - 256, None)
     assert rc == B.MOE_ERR_WORKSPACE
-    rc = B.lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, fake, fake + 16, n, None)
+    rc = B.lib.moe_route(ctypes.byref(cfg), fake, fake, None, fake, fake, None, fake, fake, None, fake + 16, n, None)
     assert rc == B.MOE_ERR_INVALID_ARG      # ws not 256-byte aligned
     race = B.make_config(1024, 384, 1536, 8, 2, 2, routing="race")
     n = B.moe_workspace_size(race)
-    rc = B.lib.moe_route(ctypes.byref(race), fake, fake, None, fake, fake, None, fake, fake, fake, n, None)
+    rc = B.lib.moe_route(ctypes.byref(race), fake, fake, None, fake, fake, None, fake, fake, None, fake, n, None)
     assert rc == B.MOE_ERR_INVALID_ARG and b"n_sel" in B.lib.moe_last_error()
     rc = B.lib.moe_combine(ctypes.byref(race), fake, fake, fake, None, None, fake, None)
     assert rc == B.MOE_ERR_INVALID_ARG
@@ -126,3 +126,20 @@ def test_python_wrappers_reach_the_library():
     for c in calls:
         with pytest.raises(B.MoeError):
             c()
+
+
+
+def test_modulation_arguments_rejected_before_launch():
+    fake = 1 << 40
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    n = B.moe_workspace_size(cfg)
+    f32 = B.make_config(1024, 384, 1536, 8, 2, 2, dtype="f32")
+    nf = B.moe_workspace_size(f32)
+    cases = [(cfg, n, B.MoeAdaln(fake, fake, 300, 1e-5, fake), B.MOE_ERR_INVALID_ARG, b"img_len"),
+             (cfg, n, B.MoeAdaln(fake, fake, 256, 0.0, fake), B.MOE_ERR_INVALID_ARG, b"eps"),
+             (cfg, n, B.MoeAdaln(fake, fake, 256, 1e-5, None), B.MOE_ERR_INVALID_ARG, b"x_mod"),
+             (f32, nf, B.MoeAdaln(fake, fake, 256, 1e-5, fake), B.MOE_ERR_UNSUPPORTED, b"16-bit")]
+    for c, nb, mod, code, word in cases:
+        rc = B.lib.moe_route(ctypes.byref(c), fake, fake, None, fake, fake, None, fake, fake, ctypes.byref(mod),
+                             fake, nb, None)
+        assert rc == code and word in B.lib.moe_last_error(), B.lib.moe_last_error()

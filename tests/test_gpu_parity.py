@@ -258,3 +258,55 @@ def test_adaln_zero_residual_in_combine(case):
     L.forward(dev(inp["x"]), dev(x_res), torch.zeros_like(dev(alpha)), L_img)
     torch.cuda.synchronize()
     assert torch.equal(L.out, dev(x_res))
+
+
+ADALN_CASES = [  # T, D, H, E, K, n_s, dtype, routing, img_len, gate
+    (1024, 256, 512, 8, 2, 2, "bf16", "topk", 256, True),
+    (1024, 384, 1536, 16, 2, 1, "bf16", "race", 512, True),
+    (1000, 192, 384, 8, 2, 1, "bf16", "topk", 40, False),     # img_len not a multiple of 16; odd 64-column blocks
+    (1024, 256, 512, 8, 2, 2, "f16", "topk", 128, True),
+]
+
+
+@pytest.mark.parametrize("case", ADALN_CASES,
+                         ids=lambda c: "T%d_D%d_E%d_%s_%s_L%d_%s" % (c[0], c[1], c[3], c[6], c[7], c[8],
+                                                                     "gate" if c[9] else "nogate"))
+def test_adaln_modulation_in_router(case):
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    T, D, H, E, K, ns, dt, routing, L_img, gate = case
+    w = I.small_workload(T, D, H, E, K, ns, dt, routing, seed=9 + T + D)
+    inp = I.make_inputs(w)
+    rng = np.random.default_rng(D)
+    nimg = T // L_img
+    x = I._store(rng.standard_normal((T, D)) * 2.0 + 0.5, dt)          # a residual stream with an offset
+    gamma = I._store(1.0 + 0.3 * rng.standard_normal((nimg, D)), dt)
+    beta = I._store(0.3 * rng.standard_normal((nimg, D)), dt)
+    alpha = I._store(0.5 * rng.standard_normal((nimg, D)), dt) if gate else None
+    L = MoELayer(LayerShape(T, D, H, E, K, ns, dt, routing, w.alpha), inp, "cuda:0")
+    dev = lambda a: torch.as_tensor(a).to(device="cuda:0", dtype=L.act_dtype).contiguous()
+    L.forward(dev(x), alpha=dev(alpha) if gate else None, img_len=L_img, gamma=dev(gamma), beta=dev(beta))
+    torch.cuda.synchronize()
+    L.check()
+    # m as the layer stores it: the oracle's adaLN rounded to the act type; the GPU's fp32 statistics may
+    # land a value on the other side of a rounding boundary, so one unit in the last place is allowed
+    m = I._store(O.adaln(x, gamma, beta, L_img).astype(np.float32), dt)
+    got = L.x_mod.float().cpu().numpy()
+    ulp = np.abs(m) * (2.0 ** (-7 if dt == "bf16" else -10)) + 1e-30
+    # where gamma * LayerNorm(x) and beta nearly cancel, the fp32 row statistics (mean, variance over
+    # D values, error about D * 2^-24 relative) matter against a small m: allow 2^-16 of the terms' size
+    b = np.arange(T) // L_img
+    terms = np.abs(gamma[b] * O.layer_norm(x)) + np.abs(beta[b])
+    assert np.all(np.abs(got - m) <= ulp * 1.01 + terms * 2.0 ** -16)
+    assert np.mean(got == m) > 0.99
+    # routing and output on the layer's own m
+    inp_m = dict(inp, x=got.astype(np.float64))
+    r = PA.fetch(L)
+    P = O.softmax_scores(O.gate_logits(inp_m["x"], inp["wg"], inp.get("router_bias")))
+    w_m = w
+    PA.check_routing(w_m, P, r)
+    idx = PA.gpu_selection(r)
+    g = np.where(idx >= 0, np.take_along_axis(P, np.maximum(idx, 0), axis=1), 0.0)
+    y = O.layer_output(inp_m, idx, g)
+    ref = O.gated_residual(x, y, alpha, L_img) if gate else y
+    err = PA.rel_err(r["out"], ref)
+    assert err <= PA.out_tol(w), err

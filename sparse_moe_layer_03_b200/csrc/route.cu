@@ -194,10 +194,13 @@ __host__ __device__ inline MmaSmem mma_layout(int D, int E) {
 // m = gamma_b * (x - mean) / sqrt(var + eps) + beta_b for token t of image
 // b = t / img_len ("Diffusion Transformer (DiT) 技术全景解析" 2.2.3, AdaLN: a
 // plain layer_norm over the features, then the per-sample scale and shift).
-// Lane l takes row l % 16 of half l / 16 (two lanes per row); the row's mean
-// and then its sum of squared deviations are formed over both halves (two
-// passes over shared memory), and each 16-byte chunk is rewritten with its
-// logical columns read through the 128-byte swizzle.
+// Lane l takes row l % 16 of half l / 16 (two lanes per row).  The statistics
+// take one pass over shared memory: sums of x - x0 and its square, shifted by
+// the row's first value x0 (so the variance does not cancel when the mean is
+// large).  The rewrite applies m = x * a_c + (beta_c - a_c * mean) with
+// a_c = gamma_c * rstd, reading each chunk's logical columns through the
+// 128-byte swizzle.  Lane (r, p) starts at 16-byte chunk r + 4p of its row, so
+// the 32 lanes spread over the 8 chunk positions (4 wavefronts per access).
 template <bool F16>
 __device__ __forceinline__ void route_modulate(const RouteArgs& a, uint8_t* xs, int stage_bytes, int w, int hc,
                                                int nchunks, int rb, int lane) {
@@ -206,37 +209,44 @@ __device__ __forceinline__ void route_modulate(const RouteArgs& a, uint8_t* xs, 
   const int z0 = p * hc;
   const int nb = (nchunks - z0) < hc ? (nchunks - z0) : hc;
   const uint32_t base = smem_u32(xs + (size_t)(2 * w + p) * stage_bytes) + r * 128;
+  const int rot = (r + 4 * p) & 7;
   const int D = a.D;
-  float s = 0.f;
+  // the row's first value (logical column 0 lives in half 0, block 0, physical chunk r % 8)
+  float x0;
+  {
+    uint32_t v0;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v0)
+                 : "r"(smem_u32(xs + (size_t)(2 * w) * stage_bytes) + r * 128 + ((0 ^ (r & 7)) << 4)));
+    const uint4 q = make_uint4(v0, 0u, 0u, 0u);
+    float f[8];
+    S::x8_to_f32(q, f);
+    x0 = f[0];
+  }
+  float s1 = 0.f, s2 = 0.f;
   for (int cb = 0; cb < nb; ++cb) {
 #pragma unroll
-    for (int pj = 0; pj < 8; ++pj) {
+    for (int q = 0; q < 8; ++q) {
+      const int pj = (q + rot) & 7;
       uint4 v;
       asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                    : "r"(base + cb * (kMmaRB * 128) + pj * 16));
       float f[8];
       S::x8_to_f32(v, f);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) s += f[q];
+      for (int e = 0; e < 8; ++e) {
+        const float d = f[e] - x0;
+        s1 += d;
+        s2 = fmaf(d, d, s2);
+      }
     }
   }
-  s += __shfl_xor_sync(0xffffffffu, s, 16);
-  const float mu = s / (float)D;
-  float ss = 0.f;
-  for (int cb = 0; cb < nb; ++cb) {
-#pragma unroll
-    for (int pj = 0; pj < 8; ++pj) {
-      uint4 v;
-      asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                   : "r"(base + cb * (kMmaRB * 128) + pj * 16));
-      float f[8];
-      S::x8_to_f32(v, f);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) ss += (f[q] - mu) * (f[q] - mu);
-    }
-  }
-  ss += __shfl_xor_sync(0xffffffffu, ss, 16);
-  const float rstd = rsqrtf(ss / (float)D + a.eps);
+  s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+  s2 += __shfl_xor_sync(0xffffffffu, s2, 16);
+  const float inv_d = 1.0f / (float)D;
+  const float dm = s1 * inv_d;                                   // mean - x0
+  const float var = fmaxf(s2 * inv_d - dm * dm, 0.f);
+  const float mu = x0 + dm;
+  const float rstd = rsqrtf(var + a.eps);
   const int tok = rb * kMmaRB + r;
   if (tok >= a.T) return;                           // rows past T stay zero (the store clips them)
   const int img = tok / a.img_len;
@@ -244,7 +254,8 @@ __device__ __forceinline__ void route_modulate(const RouteArgs& a, uint8_t* xs, 
   const uint4* bp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.beta) + (size_t)img * D);
   for (int cb = 0; cb < nb; ++cb) {
 #pragma unroll
-    for (int pj = 0; pj < 8; ++pj) {
+    for (int q = 0; q < 8; ++q) {
+      const int pj = (q + rot) & 7;
       const uint32_t addr = base + cb * (kMmaRB * 128) + pj * 16;
       const int c8 = (z0 + cb) * 8 + (pj ^ (r & 7));   // logical 8-column chunk of this row
       uint4 v;
@@ -254,11 +265,17 @@ __device__ __forceinline__ void route_modulate(const RouteArgs& a, uint8_t* xs, 
       S::x8_to_f32(v, f);
       S::x8_to_f32(__ldg(gp + c8), g);
       S::x8_to_f32(__ldg(bp + c8), b);
+      float m[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float ac = g[e] * rstd;
+        m[e] = fmaf(f[e], ac, fmaf(-ac, mu, b[e]));
+      }
       uint4 o;
-      o.x = S::pack2(g[0] * ((f[0] - mu) * rstd) + b[0], g[1] * ((f[1] - mu) * rstd) + b[1]);
-      o.y = S::pack2(g[2] * ((f[2] - mu) * rstd) + b[2], g[3] * ((f[3] - mu) * rstd) + b[3]);
-      o.z = S::pack2(g[4] * ((f[4] - mu) * rstd) + b[4], g[5] * ((f[5] - mu) * rstd) + b[5]);
-      o.w = S::pack2(g[6] * ((f[6] - mu) * rstd) + b[6], g[7] * ((f[7] - mu) * rstd) + b[7]);
+      o.x = S::pack2(m[0], m[1]);
+      o.y = S::pack2(m[2], m[3]);
+      o.z = S::pack2(m[4], m[5]);
+      o.w = S::pack2(m[6], m[7]);
       asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(o.x), "r"(o.y), "r"(o.z), "r"(o.w)
                    : "memory");
     }

@@ -179,7 +179,9 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
  *   pos        [T,Kmax] int32 out row of (t, slot k) in the permuted buffers, -1 if unused
  *   row_token  [R_max] int32 out  token of each row, -1 on padding rows
  *   row_gate   [R_max] fp32 out   gate of each row, 0 on padding rows
- *   x_perm     [R_max,D] act out  x_perm[pos[t,k]] = x[t]; padding rows untouched
+ *   x_perm     [R_max,D] act out  x_perm[pos[t,k]] = x[t]; padding rows untouched.  NULL:
+ *              write the positions only (x may then be NULL too), for
+ *              moe_expert_gemm1_gather, which reads the rows of x itself
  * An index outside [0,E) is skipped and sets MOE_ERR_DEVICE_CHECK in ws.
  */
 int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx, const float* topk_w,
@@ -200,6 +202,19 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx
 int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
                      const void* x, const void* w1, const void* b1, const void* w1s, const void* b1s,
                      void* h_perm, void* h_sh, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_gemm1_gather -- moe_expert_gemm1 without x_perm: each routed row
+ * r of the expert-contiguous layout is row row_token[r] of x, brought into
+ * shared memory by TMA tile::gather4 (four rows per load) inside the GEMM, so
+ * the dispatch writes positions only and the permuted copy of x never exists.
+ * Padding rows (row_token -1) read row 0; their h rows are never used.
+ *   row_token [R_max] int32 from moe_dispatch; other arguments as moe_expert_gemm1.
+ * Only for bf16 or fp16 with gemm_impl AUTO (MOE_ERR_UNSUPPORTED otherwise).
+ */
+int moe_expert_gemm1_gather(const moe_config_t* cfg, const int32_t* offsets, const int32_t* row_token, const void* x,
+                            const void* w1, const void* b1, const void* w1s, const void* b1s, void* h_perm,
+                            void* h_sh, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_expert_gemm2 -- second expert layer with bias and gate scaling fused:

@@ -79,6 +79,7 @@ _SIGS = {
     "moe_route": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_dispatch": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_expert_gemm1": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
+    "moe_expert_gemm1_gather": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_expert_gemm2": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_expert_mlp": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                  _P, C.c_size_t, _P]),
@@ -161,6 +162,12 @@ def moe_dispatch(cfg, x, topk_idx, topk_w, n_sel, offsets, pos, row_token, row_g
 def moe_expert_gemm1(cfg, offsets, x_perm, x, w1, b1, w1s, b1s, h_perm, h_sh, ws, ws_bytes, stream=0):
     _check(lib.moe_expert_gemm1(C.byref(cfg), _ptr(offsets), _ptr(x_perm), _ptr(x), _ptr(w1), _ptr(b1),
                                 _ptr(w1s), _ptr(b1s), _ptr(h_perm), _ptr(h_sh), _ptr(ws), ws_bytes, stream))
+
+
+def moe_expert_gemm1_gather(cfg, offsets, row_token, x, w1, b1, w1s, b1s, h_perm, h_sh, ws, ws_bytes, stream=0):
+    """GEMM1 reading its routed rows straight from x (TMA gather4 by row_token): no x_perm."""
+    _check(lib.moe_expert_gemm1_gather(C.byref(cfg), _ptr(offsets), _ptr(row_token), _ptr(x), _ptr(w1), _ptr(b1),
+                                       _ptr(w1s), _ptr(b1s), _ptr(h_perm), _ptr(h_sh), _ptr(ws), ws_bytes, stream))
 
 
 def moe_expert_gemm2(cfg, offsets, h_perm, h_sh, w2, b2, w2s, b2s, row_gate, y_perm, y_sh, ws, ws_bytes,

@@ -398,11 +398,11 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx
     if ((e = cudaMemsetAsync(row_gate, 0, R * sizeof(float), s)) != cudaSuccess) return cuda_fail(e, "moe_dispatch");
     return ok();
   }
-  REQUIRE_PTR(x);
+  if (x_perm) REQUIRE_PTR(x);           // without x_perm only positions are written (GEMM1 gathers the rows)
   REQUIRE_PTR(topk_idx);
   REQUIRE_PTR(topk_w);
   REQUIRE_PTR(pos);
-  REQUIRE_PTR(x_perm);
+  OPTIONAL_PTR(x_perm);
   OPTIONAL_PTR(n_sel);
   if (race && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
   const WsLayout L = ws_layout(cfg);
@@ -459,7 +459,13 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
   const int brows_box = pair ? bn / 2 : bn;
   CUtensorMap ta[2], tb[2];
   int rc;
-  if ((rc = make_tmap(&ta[0], A0, cfg->dtype, rows0, K0, 128, "A0"))) return rc;
+  if (g.p[0].gather_rows) {
+    // gathered A rows: one-row boxes (tile::gather4 brings four rows per load)
+    if (!pair) return fail(MOE_ERR_UNSUPPORTED, "row gathering needs the CTA-pair GEMM");
+    if ((rc = make_tmap(&ta[0], A0, cfg->dtype, rows0, K0, 1, "A0 (gathered rows)"))) return rc;
+  } else if ((rc = make_tmap(&ta[0], A0, cfg->dtype, rows0, K0, 128, "A0"))) {
+    return rc;
+  }
   if ((rc = make_tmap(&tb[0], B0, cfg->dtype, brows0, K0, brows_box, "B0"))) return rc;
   if (g.nprob > 1) {
     if ((rc = make_tmap(&ta[1], A1, cfg->dtype, rows1, K1, 128, "A1"))) return rc;
@@ -471,7 +477,9 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
   if (pair) {
     // output boxes for the TMA-store epilogue: 32 rows x 128 bytes of h or y (act dtype)
     CUtensorMap to[2];
-    if ((rc = make_tmap(&to[0], g.p[0].out, cfg->dtype, rows0, g.p[0].N, 32, "out0"))) return rc;
+    // the routed output has the permuted layout's R_max rows, whatever the A tensor's row count
+    const long long orows0 = g.p[0].routed ? g.r_max : rows0;
+    if ((rc = make_tmap(&to[0], g.p[0].out, cfg->dtype, orows0, g.p[0].N, 32, "out0"))) return rc;
     if (g.nprob > 1) {
       if ((rc = make_tmap(&to[1], g.p[1].out, cfg->dtype, rows1, g.p[1].N, 32, "out1"))) return rc;
     } else {
@@ -487,15 +495,40 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
 
 }  // namespace
 
+static int expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm, const int32_t* row_token,
+                        const void* x, const void* w1, const void* b1, const void* w1s, const void* b1s,
+                        void* h_perm, void* h_sh, void* ws, size_t ws_bytes, void* stream);
+
 int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
                      const void* x, const void* w1, const void* b1, const void* w1s, const void* b1s,
                      void* h_perm, void* h_sh, void* ws, size_t ws_bytes, void* stream) {
+  return expert_gemm1(cfg, offsets, x_perm, nullptr, x, w1, b1, w1s, b1s, h_perm, h_sh, ws, ws_bytes, stream);
+}
+
+int moe_expert_gemm1_gather(const moe_config_t* cfg, const int32_t* offsets, const int32_t* row_token,
+                            const void* x, const void* w1, const void* b1, const void* w1s, const void* b1s,
+                            void* h_perm, void* h_sh, void* ws, size_t ws_bytes, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (!is16(cfg) || cfg->gemm_impl != MOE_GEMM_AUTO)
+    return fail(MOE_ERR_UNSUPPORTED, "GEMM1 gathers its rows only for bf16 or fp16 with gemm_impl AUTO; "
+                                     "use moe_dispatch with x_perm and moe_expert_gemm1");
+  if (cfg->T > 0) {
+    REQUIRE_PTR(row_token);
+    REQUIRE_PTR(x);
+  }
+  return expert_gemm1(cfg, offsets, nullptr, row_token, x, w1, b1, w1s, b1s, h_perm, h_sh, ws, ws_bytes, stream);
+}
+
+static int expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm, const int32_t* row_token,
+                        const void* x, const void* w1, const void* b1, const void* w1s, const void* b1s,
+                        void* h_perm, void* h_sh, void* ws, size_t ws_bytes, void* stream) {
   int rc = validate(cfg);
   if (rc) return rc;
   if ((rc = check_ws(cfg, ws, ws_bytes))) return rc;
   if (cfg->T == 0) return ok();
   REQUIRE_PTR(offsets);
-  REQUIRE_PTR(x_perm);
+  if (!row_token) REQUIRE_PTR(x_perm);
   REQUIRE_PTR(w1);
   REQUIRE_PTR(h_perm);
   OPTIONAL_PTR(b1);
@@ -513,8 +546,11 @@ int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void
   g.nprob = ns > 0 ? 2 : 1;
   GemmProblem& p0 = g.p[0];
   p0.routed = 1; p0.N = cfg->H; p0.K = cfg->D; p0.epi = 0;
-  p0.A = x_perm; p0.B = w1; p0.out = h_perm; p0.ld_out = cfg->H; p0.bias = b1; p0.bias_stride = cfg->H;
+  p0.A = row_token ? x : x_perm; p0.B = w1; p0.out = h_perm; p0.ld_out = cfg->H; p0.bias = b1;
+  p0.bias_stride = cfg->H;
   p0.bias_rows = 1;
+  p0.gather_rows = row_token;
+  p0.gather_nrows = cfg->T;
   if (ns > 0) {
     // the n_s stacked W1 [n_s,H,D] are one [n_s*H, D] matrix; b1s [n_s,H] one [n_s*H] row
     GemmProblem& p1 = g.p[1];
@@ -522,8 +558,8 @@ int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void
     p1.A = x; p1.B = w1s; p1.out = h_sh; p1.ld_out = (long long)ns * cfg->H; p1.bias = b1s; p1.bias_stride = 0;
     p1.bias_rows = 1;
   }
-  return run_gemm(cfg, g, x_perm, R, w1, (long long)cfg->E * cfg->H, x, cfg->T, w1s, (long long)ns * cfg->H,
-                  cfg->D, cfg->D, cfg->D, ws, (cudaStream_t)stream);
+  return run_gemm(cfg, g, row_token ? x : x_perm, row_token ? (long long)cfg->T : R, w1, (long long)cfg->E * cfg->H,
+                  x, cfg->T, w1s, (long long)ns * cfg->H, cfg->D, cfg->D, cfg->D, ws, (cudaStream_t)stream);
 }
 
 int moe_expert_gemm2(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm,

@@ -210,7 +210,8 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos) {
   const uint4* xv = reinterpret_cast<const uint4*>(a.x);
   uint4* xp = reinterpret_cast<uint4*>(a.x_perm);
   uint4 buf[P > 0 ? P : 1];
-  if (P > 0 && w < nt) load_row<P>(xv + (size_t)(t0 + w) * nvec, nvec, lane, buf);
+  const bool copy = a.x_perm != nullptr;               // else positions only
+  if (P > 0 && copy && w < nt) load_row<P>(xv + (size_t)(t0 + w) * nvec, nvec, lane, buf);
 
   for (int i = tid; i < nt * Kmax; i += kDispatchThreads) {
     const int t = t0 + i / Kmax, k = i % Kmax;
@@ -232,6 +233,7 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos) {
     a.pos[slot] = p;
     spos[i] = p;
   }
+  if (!copy) return;
   __syncthreads();
 
   for (int l = w; l < nt; l += kDispatchThreads / 32) {

@@ -162,34 +162,60 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      const uint64_t pol_w = policy_evict_last();
-      // A tiles are reused by every column tile of their row block (consecutive tiles, run
-      // side by side): keep them in L2 normally; evict-first sent them back to DRAM 3.5x
-      const uint64_t pol_a = policy_evict_normal();
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int tile = cid; tile < pl.total; tile += ncl) {
-        const PairTile ti = pair_decode<BN>(tile, pl, a);
-        const CUtensorMap* tA = ti.p ? &ta1 : &ta0;
-        const CUtensorMap* tB = ti.p ? &tb1 : &tb0;
-        const int ksplit = a.p[ti.p].ksplit;
-        const int nrows = a.p[ti.p].N;
-        for (int kb = 0; kb < ti.nk; ++kb) {
-          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.status, 501)) goto done;
-          const uint32_t fb_local = smem_u32(&full[stage]);
-          const uint32_t fb_leader = map_to_cta(fb_local, 0);
+    // Lane 0 loads the tiles.  When the routed problem gathers its A rows, every lane also
+    // issues one tile::gather4 per stage for 4 of this CTA's 128 rows (indices held for the
+    // whole tile), after lane 0 has seen the stage free and posted the expected bytes.
+    const uint64_t pol_w = policy_evict_last();
+    // A tiles are reused by every column tile of their row block (consecutive tiles, run
+    // side by side): keep them in L2 normally; evict-first sent them back to DRAM 3.5x
+    const uint64_t pol_a = policy_evict_normal();
+    int stage = 0;
+    uint32_t phase = 0;
+    bool alive = true;
+    for (int tile = cid; tile < pl.total && alive; tile += ncl) {
+      const PairTile ti = pair_decode<BN>(tile, pl, a);
+      const GemmProblem& pr = a.p[ti.p];
+      const CUtensorMap* tA = ti.p ? &ta1 : &ta0;
+      const CUtensorMap* tB = ti.p ? &tb1 : &tb0;
+      const int ksplit = pr.ksplit;
+      const int nrows = pr.N;
+      const bool gather = pr.gather_rows != nullptr;      // uniform across the warp
+      int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
+      if (gather) {
+        const long long r0 = (long long)ti.row0 + (int)rank * 128 + lane * 4;
+        int g[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int v = __ldg(pr.gather_rows + r0 + u);
+          g[u] = (v >= 0 && v < pr.gather_nrows) ? v : 0;   // padding rows read row 0; never used
+        }
+        g0 = g[0]; g1 = g[1]; g2 = g[2]; g3 = g[3];
+      }
+      for (int kb = 0; kb < ti.nk; ++kb) {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.status, 501) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { alive = false; break; }
+        const uint32_t fb_local = smem_u32(&full[stage]);
+        const uint32_t fb_leader = map_to_cta(fb_local, 0);
+        uint8_t* sa = stage_base + stage * C::STAGE;
+        if (lane == 0) {
           if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::STAGE);   // both CTAs' bytes
-          uint8_t* sa = stage_base + stage * C::STAGE;
           const int bx = ksplit ? (kb * kPairBK) % ksplit : kb * kPairBK;
           // each CTA holds half of the tile's B rows (a narrower tile's box also brings rows it does not use)
           const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (ti.width / 2);
-          tma_load_2d_pair(smem_u32(sa), tA, kb * kPairBK, ti.row0 + (int)rank * 128, fb_leader, pol_a);
+          if (!gather) tma_load_2d_pair(smem_u32(sa), tA, kb * kPairBK, ti.row0 + (int)rank * 128, fb_leader, pol_a);
           tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tB, bx, by, fb_leader, pol_w);
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
+        if (gather) {
+          __syncwarp();
+          tma_gather4_pair(smem_u32(sa) + lane * 4 * 128, tA, kb * kPairBK, g0, g1, g2, g3, fb_leader, pol_a);
+        }
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       }
     }
+    __syncwarp();
+    if (!alive) goto done;
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && rank == 0) {

@@ -111,7 +111,7 @@ struct DispatchArgs {
   unsigned int* ctr;        // blocks-done counter in ws (zero between calls)
   int32_t* offsets;         // [E+1]
   int32_t* pos; int32_t* row_token; float* row_gate;
-  void* x_perm;
+  void* x_perm;             // null: positions only (GEMM1 gathers the rows itself)
   int* status;
 };
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
@@ -130,6 +130,10 @@ struct GemmProblem {
   int bias_rows;            // bias rows summed per column (n_s for the shared GEMM2, else 1)
   int ksplit;               // 0, or: B is [K/ksplit blocks][N][ksplit] (shared W2 stack)
   const float* gate;        // per-row gate or null
+  // routed problem on the CTA-pair kernel: A row r is row gather_rows[r] of the A tensor (rows
+  // < 0 read row 0), loaded with TMA tile::gather4 (the A tensor map's box is one row high)
+  const int32_t* gather_rows;
+  int gather_nrows;         // rows of the A tensor
 };
 struct GemmArgs {
   GemmProblem p[2]; int nprob;

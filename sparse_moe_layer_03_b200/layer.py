@@ -41,6 +41,8 @@ class LayerShape:
     gemm_impl: str = "auto"
     seq_len: int = 0          # tokens per image for the balance loss (0 = the whole call)
     fuse_combine: bool = True  # fold the combine into the shared experts' GEMM2 where supported
+    gather_rows: bool = False  # GEMM1 gathers its routed rows from x by TMA gather4 (no x_perm); measured
+                               # slower at XL (GEMM1 2.37 ms against 1.11 ms): off by default
 
 
 class MoELayer:
@@ -84,7 +86,9 @@ class MoELayer:
         self.pos = torch.empty((T, kmax), dtype=i32, device=dev)
         self.row_token = torch.empty((self.R,), dtype=i32, device=dev)
         self.row_gate = torch.empty((self.R,), dtype=f32, device=dev)
-        self.x_perm = torch.empty((self.R, s.D), dtype=dt, device=dev)
+        # GEMM1 reads the routed rows of x itself (TMA gather4) on the 16-bit CTA-pair path: no x_perm
+        self.gathered = bool(s.gather_rows and s.dtype in ("bf16", "f16") and s.gemm_impl == "auto")
+        self.x_perm = None if self.gathered else torch.empty((self.R, s.D), dtype=dt, device=dev)
         self.h_perm = torch.empty((self.R, s.H), dtype=dt, device=dev)
         self.y_perm = torch.empty((self.R, s.D), dtype=dt, device=dev)
         ns = s.n_shared
@@ -108,6 +112,10 @@ class MoELayer:
                        self.row_token, self.row_gate, self.x_perm, self.ws, self.ws_bytes, self.stream())
 
     def gemm1(self, x: torch.Tensor):
+        if self.gathered:
+            B.moe_expert_gemm1_gather(self.cfg, self.offsets, self.row_token, x, self.w1, self.b1, self.ws1,
+                                      self.bs1, self.h_perm, self.h_sh, self.ws, self.ws_bytes, self.stream())
+            return
         B.moe_expert_gemm1(self.cfg, self.offsets, self.x_perm, x, self.w1, self.b1, self.ws1, self.bs1,
                            self.h_perm, self.h_sh, self.ws, self.ws_bytes, self.stream())
 

@@ -73,7 +73,7 @@ def test_deterministic_repeat():
     w, inp = _small(2000, 256, 512, 8, 2, 2, "bf16", routing="race")
     L, x = PA.run_layer(w, inp)
     valid = L.row_token >= 0          # padding rows of x_perm are never written
-    pick = lambda: (L.out, L.topk_idx, L.topk_w, L.pos, L.aux, L.counts, L.x_perm[valid], L.y_perm[valid])
+    pick = lambda: (L.out, L.topk_idx, L.topk_w, L.pos, L.aux, L.counts, L.h_perm[valid], L.y_perm[valid])
     first = [t.clone() for t in pick()]
     for _ in range(2):
         L.forward(x)
@@ -310,3 +310,25 @@ def test_adaln_modulation_in_router(case):
     ref = O.gated_residual(x, y, alpha, L_img) if gate else y
     err = PA.rel_err(r["out"], ref)
     assert err <= PA.out_tol(w), err
+
+
+
+@pytest.mark.parametrize("routing", ["topk", "race"])
+def test_gathered_gemm1_rows_equal_permuted_copy(routing):
+    # GEMM1 reading its rows from x by TMA gather4 computes bit for bit what it computes on x_perm
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    w = I.small_workload(1500, 384, 768, 16 if routing == "race" else 8, 2, 2, "bf16", routing, seed=61)
+    inp = I.make_inputs(w, bias_std=0.2)
+    res = {}
+    for gather in (True, False):
+        L = MoELayer(LayerShape(w.T, w.D, w.H, w.E, w.K, w.n_shared, "bf16", routing, w.alpha, gather_rows=gather),
+                     inp, "cuda:0")
+        assert L.gathered == gather and (L.x_perm is None) == gather
+        x = torch.as_tensor(inp["x"]).to(device="cuda:0", dtype=L.act_dtype).contiguous()
+        L.forward(x)
+        torch.cuda.synchronize()
+        L.check()
+        valid = L.row_token >= 0
+        res[gather] = (L.h_perm[valid].clone(), L.out.clone())
+    assert torch.equal(res[True][0], res[False][0])
+    assert torch.equal(res[True][1], res[False][1])

@@ -196,6 +196,28 @@ def image_labels(T, seq_len, per_image):
     return np.repeat(np.asarray(per_image), seq_len)[:T]
 
 
+# ---------------------------------------------------------------- balance loss backward
+
+def balance_loss_grad_logits(P, counts, K, alpha):
+    """dL_balance / dl[t,i] for the logits l of the router (counts held constant).
+
+    "MOE-DIT", eq. L_balance: L = alpha sum_i f_i p_i with f_i = (n/(K T))
+    counts_i from the discrete selection (no gradient) and p_i = (1/T) sum_t
+    P[t,i], so dL/dP[t,i] = alpha f_i / T =: c_i for every token.  Through the
+    softmax: dl[t,i] = P[t,i] (c_i - sum_j P[t,j] c_j).
+    """
+    P = as_f64(P)
+    T, E = P.shape
+    c = alpha * (E / (K * T)) * np.asarray(counts, dtype=F64) / T
+    return P * (c[None, :] - (P @ c)[:, None])
+
+
+def router_backward(x, wg, dlogits):
+    """Gradients of l = x Wg^T + b: dWg = dl^T x [E,D], db = sum_t dl [E], dx = dl Wg [T,D]."""
+    x, wg, dl = as_f64(x), as_f64(wg), as_f64(dlogits)
+    return dl.T @ x, dl.sum(axis=0), dl @ wg
+
+
 # ---------------------------------------------------------------- adaLN-Zero around the layer
 
 def layer_norm(x, eps=1e-5):

@@ -241,6 +241,42 @@ def test_frequency_marginals_and_relabelling(routing):
     assert np.array_equal(hi2[perm], hi)
 
 
+# ------------------------------------------------------------------ balance loss backward
+
+@pytest.mark.parametrize("routing", ["topk", "race"])
+def test_balance_loss_gradient_matches_autograd(routing):
+    # torch autograd (float64) differentiates the loss written with library ops; the counts come
+    # from the discrete selection and carry no gradient
+    rng = np.random.default_rng(51)
+    T, D, E, K, alpha = 40, 24, 8, 2, 0.01
+    x = rng.standard_normal((T, D))
+    wg = rng.standard_normal((E, D)) / np.sqrt(D)
+    b = rng.standard_normal(E) * 0.3
+    inp = {"x": x, "wg": wg, "router_bias": b}
+    r = O.route(inp, K, routing, alpha)
+    xt = torch.tensor(x, requires_grad=True)
+    wt = torch.tensor(wg, requires_grad=True)
+    bt = torch.tensor(b, requires_grad=True)
+    Pt = torch.softmax(torch.nn.functional.linear(xt, wt, bt), dim=1)
+    counts = torch.tensor(r["counts"], dtype=torch.float64)
+    loss = alpha * torch.sum((E / (K * T)) * counts * Pt.mean(0))
+    loss.backward()
+    assert abs(loss.item() - r["aux"]) < 1e-15
+    dl = O.balance_loss_grad_logits(r["P"], r["counts"], K, alpha)
+    dwg, db, dx = O.router_backward(x, wg, dl)
+    assert np.max(np.abs(dwg - wt.grad.numpy())) < 1e-15
+    assert np.max(np.abs(db - bt.grad.numpy())) < 1e-15
+    assert np.max(np.abs(dx - xt.grad.numpy())) < 1e-15
+
+
+def test_balance_loss_gradient_vanishes_for_uniform_counts():
+    # with every expert equally loaded, L = alpha sum_i p_i = alpha whatever the scores: zero gradient
+    P = _rand_scores(32, 4, 52)
+    dl = O.balance_loss_grad_logits(P, np.full(4, 16), 2, 0.05)
+    assert np.max(np.abs(dl)) < 1e-18
+    assert np.max(np.abs(dl.sum(1))) < 1e-18   # every row of a softmax gradient sums to zero
+
+
 # ------------------------------------------------------------------ adaLN-Zero
 
 def test_layer_norm_matches_library_and_moments():

@@ -283,9 +283,37 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     torch.cuda.synchronize(device)
     e2e_ms = reduce_max(e0.elapsed_time(e1), world, device) / args.steps
 
+    # the balance loss's gradient through the router (not part of the forward step): timed on its own
+    bwd_ms = None
+    if w.routing in ("topk", "race"):
+        bws = torch.empty(B.moe_backward_workspace_size(L.cfg), dtype=torch.uint8, device=device)
+        dwg = torch.empty((w.E, w.D), dtype=torch.float32, device=device)
+        dbias = torch.empty((w.E,), dtype=torch.float32, device=device)
+        dx = torch.empty_like(x)
+        run_bwd = lambda: B.moe_balance_loss_backward(L.cfg, x, L.wg, L.router_bias, L.counts, 1.0, dwg, dbias, dx,
+                                                      bws, bws.numel(), L.stream())
+        for _ in range(3):
+            run_bwd()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        times = []
+        for i in range(5):
+            flush_l2(i)
+            b0.record(stream)
+            run_bwd()
+            b1.record(stream)
+            torch.cuda.synchronize(device)
+            times.append(b0.elapsed_time(b1))
+        bwd_ms = float(np.median(times))
+
     result = None
     if rank == 0:
         result = report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp)
+        if bwd_ms is not None:
+            elem = 2 if w.dtype in ("bf16", "f16") else 4
+            moved = 2 * w.T * w.D * elem + w.E * w.D * (elem + 4)
+            result["balance_backward"] = {"ms": round(bwd_ms, 4), "GB/s": round(moved / (bwd_ms * 1e-3) / 1e9, 1),
+                                          "what": "moe_balance_loss_backward (dWg, db, dx of the balance loss), "
+                                                  "timed separately; x read and dx written once"}
     if world > 1:
         import torch.distributed as dist
         barrier(world, device)

@@ -296,6 +296,24 @@ int moe_route_static(const moe_config_t* cfg, const void* x, const void* wg, con
                      void* stream);
 
 /*
+ * moe_balance_loss_backward -- gradient of the expert-level balance loss with
+ * respect to the router ("MOE-DIT", eq. L_balance; the counts come from the
+ * discrete selection and carry no gradient): dL/dP[t,i] = alpha f_i / T, back
+ * through the softmax to the logits, then through l = x Wg^T + b.
+ *   x, wg, router_bias   as given to moe_route (the logits are recomputed in fp32)
+ *   counts      [E] int32 from moe_route
+ *   grad_scale  dObjective/dL_balance (1 for the loss alone)
+ *   dwg         [E,D] fp32 out; dbias [E] fp32 out or NULL; dx [T,D] act out or NULL
+ *   bws         scratch of moe_backward_workspace_size(cfg) bytes, 256-byte aligned
+ * Whole-call loss only (seq_len = 0; MOE_ERR_UNSUPPORTED otherwise).  The sums
+ * run in a fixed order: bit-reproducible.
+ */
+size_t moe_backward_workspace_size(const moe_config_t* cfg);
+int moe_balance_loss_backward(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
+                              const int32_t* counts, float grad_scale, float* dwg, float* dbias, void* dx,
+                              void* bws, size_t bws_bytes, void* stream);
+
+/*
  * moe_expert_frequency -- expert-selection frequency per label, the statistic of
  * the expert specialisation analysis ("Scaling Diffusion Transformers to 16
  * Billion Parameters": selection frequency by image class, spatial position

@@ -86,6 +86,8 @@ _SIGS = {
     "moe_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
     "moe_route_static": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_frequency": (C.c_int, [_CFG, _P, _P, C.c_int32, _P, C.c_int32, _P, _P, _P]),
+    "moe_backward_workspace_size": (C.c_size_t, [_CFG]),
+    "moe_balance_loss_backward": (C.c_int, [_CFG, _P, _P, _P, _P, C.c_float, _P, _P, _P, _P, C.c_size_t, _P]),
     "moe_expert_gemm2_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            C.c_size_t, _P]),
 }
@@ -211,3 +213,16 @@ def moe_expert_gemm2_combine(cfg, offsets, h_perm, h_sh, w2, b2, w2s, b2s, row_g
     _check(lib.moe_expert_gemm2_combine(C.byref(cfg), _ptr(offsets), _ptr(h_perm), _ptr(h_sh), _ptr(w2), _ptr(b2),
                                         _ptr(w2s), _ptr(b2s), _ptr(row_gate), _ptr(pos), _ptr(n_sel), _ptr(y_perm),
                                         _res_ref(res), _ptr(out), _ptr(ws), ws_bytes, stream))
+
+
+def moe_backward_workspace_size(cfg) -> int:
+    n = lib.moe_backward_workspace_size(C.byref(cfg))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, lib.moe_last_error().decode())
+    return n
+
+
+def moe_balance_loss_backward(cfg, x, wg, router_bias, counts, grad_scale, dwg, dbias, dx, bws, bws_bytes, stream=0):
+    """Gradient of the balance loss through the router: dWg [E,D], db [E] (fp32) and dx [T,D] (act)."""
+    _check(lib.moe_balance_loss_backward(C.byref(cfg), _ptr(x), _ptr(wg), _ptr(router_bias), _ptr(counts),
+                                         grad_scale, _ptr(dwg), _ptr(dbias), _ptr(dx), _ptr(bws), bws_bytes, stream))

@@ -350,6 +350,71 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   return ok();
 }
 
+namespace {
+struct BwdLayout { size_t dl, db_part, partials, total; };
+BwdLayout bwd_layout(const moe_config_t* c) {
+  BwdLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += round_up(bytes ? bytes : 1, 256); return o; };
+  L.dl = take((size_t)c->T * c->E * sizeof(float));
+  L.db_part = take((size_t)kBwdMaxBlocks * c->E * sizeof(float));
+  L.partials = take((size_t)balance_grad_chunks(c->T) * c->E * c->D * sizeof(float));
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+size_t moe_backward_workspace_size(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return bwd_layout(cfg).total;
+}
+
+int moe_balance_loss_backward(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
+                              const int32_t* counts, float grad_scale, float* dwg, float* dbias, void* dx,
+                              void* bws, size_t bws_bytes, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (cfg->seq_len > 0)
+    return fail(MOE_ERR_UNSUPPORTED, "the balance-loss backward covers the whole-call loss (seq_len = 0)");
+  if ((size_t)cfg->E * cfg->D * elem_bytes(cfg) > 232448)
+    return fail(MOE_ERR_UNSUPPORTED, "E=%d x D=%d: the gate weight does not fit the backward's shared memory", cfg->E,
+                cfg->D);
+  REQUIRE_PTR(dwg);
+  OPTIONAL_PTR(dbias);
+  if (!bws) return fail(MOE_ERR_INVALID_ARG, "bws is NULL");
+  if ((uintptr_t)bws & 255u) return fail(MOE_ERR_INVALID_ARG, "bws must be 256-byte aligned");
+  if (bws_bytes < moe_backward_workspace_size(cfg))
+    return fail(MOE_ERR_WORKSPACE, "bws_bytes=%zu < %zu", bws_bytes, moe_backward_workspace_size(cfg));
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  if (cfg->T == 0) {
+    if ((e = cudaMemsetAsync(dwg, 0, (size_t)cfg->E * cfg->D * sizeof(float), s)) != cudaSuccess) return cuda_fail(e, "backward");
+    if (dbias && (e = cudaMemsetAsync(dbias, 0, cfg->E * sizeof(float), s)) != cudaSuccess) return cuda_fail(e, "backward");
+    return ok();
+  }
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(wg);
+  REQUIRE_PTR(counts);
+  OPTIONAL_PTR(router_bias);
+  OPTIONAL_PTR(dx);
+  BalanceGradArgs a{};
+  a.x = x; a.wg = wg; a.bias = router_bias; a.counts = counts;
+  a.T = cfg->T; a.D = cfg->D; a.E = cfg->E; a.K = cfg->K; a.dtype = cfg->dtype;
+  a.alpha = cfg->alpha; a.scale = grad_scale;
+  const BwdLayout BL = bwd_layout(cfg);
+  a.dx = dx; a.dwg = dwg; a.dbias = dbias;
+  a.dl = ws_at<float>(bws, BL.dl);
+  a.db_part = ws_at<float>(bws, BL.db_part);
+  a.partials = ws_at<float>(bws, BL.partials);
+  // 8 tokens per block (one per warp) at a time: enough blocks to keep every SM's memory pipe busy
+  int blocks = num_sms_current() * 4;
+  if (blocks > kBwdMaxBlocks) blocks = kBwdMaxBlocks;
+  const int need = (cfg->T + 7) / 8;
+  if (blocks > need) blocks = need;
+  if ((e = launch_balance_grad(a, blocks, s)) != cudaSuccess) return cuda_fail(e, "balance-loss backward kernels");
+  return ok();
+}
+
 int moe_expert_frequency(const moe_config_t* cfg, const int32_t* topk_idx, const int32_t* n_sel, int32_t seq_len,
                          const int32_t* seq_labels, int32_t n_labels, int32_t* hist, void* ws, void* stream) {
   int rc = validate(cfg);

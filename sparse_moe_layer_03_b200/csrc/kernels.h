@@ -67,6 +67,24 @@ struct SeqLossArgs {
 };
 cudaError_t launch_seq_loss(const SeqLossArgs& a, cudaStream_t s);
 
+// ---- backward.cu: the balance loss's gradient through the router
+struct BalanceGradArgs {
+  const void* x; const void* wg; const float* bias;   // x [T,D], wg [E,D] act; bias [E] or null
+  const int32_t* counts;                              // [E] from the forward selection
+  int T, D, E, K;
+  int dtype;                                          // moe_dtype_t of x and wg (and dx)
+  float alpha, scale;                                 // scale = dObjective / dL_balance
+  void* dx;                                           // [T,D] act or null
+  float* dwg;                                         // [E,D]
+  float* dbias;                                       // [E] or null
+  float* dl;                                          // [T,E] scratch: dL/dlogits
+  float* db_part;                                     // [blocks,E] scratch
+  float* partials;                                    // [chunks,E,D] scratch
+};
+constexpr int kBwdMaxBlocks = 1024;
+int balance_grad_chunks(int T);
+cudaError_t launch_balance_grad(const BalanceGradArgs& a, int blocks, cudaStream_t s);
+
 // ---- stats.cu: expert-selection frequency per label
 struct FreqArgs {
   const int32_t* topk_idx; const int32_t* n_sel;

@@ -143,3 +143,18 @@ def test_modulation_arguments_rejected_before_launch():
         rc = B.lib.moe_route(ctypes.byref(c), fake, fake, None, fake, fake, None, fake, fake, ctypes.byref(mod),
                              fake, nb, None)
         assert rc == code and word in B.lib.moe_last_error(), B.lib.moe_last_error()
+
+
+def test_balance_backward_arguments_rejected_before_launch():
+    fake = 1 << 40
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    n = B.moe_backward_workspace_size(cfg)
+    assert n >= 8 * 385 * 4
+    f = B.lib.moe_balance_loss_backward
+    assert f(ctypes.byref(cfg), fake, fake, None, fake, ctypes.c_float(1.0), None, None, None, fake, n, None) == \
+        B.MOE_ERR_INVALID_ARG
+    assert f(ctypes.byref(cfg), fake, fake, None, fake, ctypes.c_float(1.0), fake, None, None, fake, n - 4, None) == \
+        B.MOE_ERR_WORKSPACE
+    per_image = B.make_config(1024, 384, 1536, 8, 2, 2, seq_len=256)
+    assert f(ctypes.byref(per_image), fake, fake, None, fake, ctypes.c_float(1.0), fake, None, None, fake, n, None) == \
+        B.MOE_ERR_UNSUPPORTED

@@ -101,3 +101,43 @@ def test_label_out_of_range_is_reported_not_faulted():
     want = O.expert_frequency(idx[keep], 8, tok_lab[keep], 10)
     assert np.array_equal(hist.cpu().numpy(), want)      # the image with the bad label is skipped
     L.check()                                            # the status word was cleared
+
+
+BWD_CASES = [  # T, D, E, K, dtype, routing
+    (1000, 256, 8, 2, "bf16", "topk"),
+    (1024, 384, 16, 2, "bf16", "race"),
+    (777, 128, 4, 1, "f32", "topk"),
+    (600, 192, 32, 4, "f16", "topk"),
+    (32768, 1152, 8, 2, "bf16", "topk"),       # XL/2-8E2A router
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "T%d_D%d_E%d_K%d_%s_%s" % c)
+def test_balance_loss_backward(case):
+    T, D, E, K, dt, routing = case
+    w = I.small_workload(T, D, 2 * D, E, K, 0, dt, routing, seed=3 + T + E, router_bias="normal")
+    inp = I.make_inputs(w)
+    L, r = _run(w, inp, 0)
+    dev = L.device
+    bws = torch.empty(B.moe_backward_workspace_size(L.cfg), dtype=torch.uint8, device=dev)
+    outs = []
+    for _ in range(2):
+        dwg = torch.empty((E, D), dtype=torch.float32, device=dev)
+        db = torch.empty((E,), dtype=torch.float32, device=dev)
+        dx = torch.empty((T, D), dtype=L.act_dtype, device=dev)
+        x = torch.as_tensor(inp["x"]).to(device=dev, dtype=L.act_dtype).contiguous()
+        B.moe_balance_loss_backward(L.cfg, x, L.wg, L.router_bias, L.counts, 1.0, dwg, db, dx, bws, bws.numel(),
+                                    L.stream())
+        torch.cuda.synchronize()
+        outs.append((dwg.cpu().numpy(), db.cpu().numpy(), dx.float().cpu().numpy()))
+    for a, b in zip(outs[0], outs[1]):
+        assert np.array_equal(a, b)                     # fixed summation order
+    P = O.softmax_scores(O.gate_logits(inp["x"], inp["wg"], inp.get("router_bias")))
+    dl = O.balance_loss_grad_logits(P, r["counts"], K, w.alpha)
+    ref_dwg, ref_db, ref_dx = O.router_backward(inp["x"], inp["wg"], dl)
+    dwg, db, dx = outs[0]
+    # fp32 logits against fp64 and fp32 sums: the gradient is a difference of nearby terms
+    # (P (c - P.c)), so it is held to 1e-3 of its largest entry; dx is also rounded to the act type
+    assert PA.rel_err(dwg, ref_dwg) < 1e-3
+    assert PA.rel_err(db, ref_db) < 1e-3
+    assert PA.rel_err(dx, ref_dx) < (1e-3 if dt == "f32" else 1e-2)

@@ -8,7 +8,8 @@
 // 128 rows of A and its own half of the tile's B rows, so per FLOP each SM
 // pulls 2/3 of the operand bytes of a 128 x 256 single-CTA tile; the pair's
 // tensor cores read the peer's half through the CTA pair, and each CTA's TMEM
-// receives its 128 rows of the accumulator.  No TMA load uses cluster multicast.
+// receives its 128 rows of the accumulator.  Every TMA load fills one CTA's own
+// shared memory (nothing is broadcast to several CTAs).
 //
 // Roles per CTA (6 warps): warp 0 = TMA producer (both CTAs; loads complete on
 // the leader's barrier); warp 1 = TMEM allocation (both) and the MMA issuer

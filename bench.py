@@ -204,6 +204,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     out_host = torch.empty((w.T, w.D), dtype=dt).pin_memory()
     aux_host = torch.empty((1,), dtype=torch.float32).pin_memory()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    flush_clean = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
 
     # with the combine folded into GEMM2 (bf16, n_s >= 1) the step has four stages
@@ -233,9 +234,12 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
     wev = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
     def flush_l2(i):
-        # write a buffer larger than L2, then idle the GPU briefly so the host has enqueued the
+        # write a buffer larger than L2; then read another one as large, so the written lines
+        # go back to DRAM here and not inside the next stage's events (a write-back L2 keeps
+        # them dirty until evicted); then idle the GPU briefly so the host has enqueued the
         # whole step before the GPU reaches it (every stage is then timed as device time alone)
         flush.fill_(float(i))
+        flush_clean.sum()
         torch.cuda._sleep(SPACER_CYCLES)
 
     for i in range(args.warmup):
@@ -377,7 +381,8 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
                    "global_batch_tokens": total_tokens, "parallelism": f"dp{world}" if world > 1 else "single",
                    "adaln": ("modulation in the router and the gated residual in the combine (e2e: the plain "
                              "layer)") if args.adaln == "on" else "off",
-                   "l2": "flushed between steps (256 MB write, then a 0.2 ms GPU sleep so the host is ahead; both "
+                   "l2": "flushed between steps (256 MB written, then another 256 MB read so the written lines "
+                         "return to DRAM before the step, then a 0.2 ms GPU sleep so the host is ahead; all "
                          "outside each step's events)"},
         "layer_tflops": round(M.gemm_flops(w.T, w.D, w.H, w.K, w.n_shared) / (ms_per_step * 1e-3) / 1e12, 1),
         "gemm_tflops": round((g1 + g2) / (gemm_ms * 1e-3) / 1e12, 1),

@@ -168,6 +168,25 @@ class MoELayer:
             self.combine(res)
         return self.out
 
+    def capture(self, x: torch.Tensor, **kwargs) -> "torch.cuda.CUDAGraph":
+        """Record one forward on the fixed input buffer ``x`` into a CUDA graph.
+
+        ``graph.replay()`` then reruns the whole layer with one launch from the host
+        (whatever is in ``x`` at replay time).  Every counter the kernels keep in the
+        workspace between launches is reset by the kernels themselves, so replays need
+        no host work in between.
+        """
+        self.forward(x, **kwargs)                 # warm: lazy buffers, kernel attributes
+        torch.cuda.synchronize(self.device)
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                self.forward(x, **kwargs)
+        torch.cuda.current_stream(self.device).wait_stream(side)
+        return graph
+
     def expert_frequency(self, seq_len: int, seq_labels: Optional[torch.Tensor] = None,
                          n_labels: Optional[int] = None) -> torch.Tensor:
         """Counts [n_labels, E] of the last routing's selections per label: per patch position

@@ -332,3 +332,31 @@ def test_gathered_gemm1_rows_equal_permuted_copy(routing):
         res[gather] = (L.h_perm[valid].clone(), L.out.clone())
     assert torch.equal(res[True][0], res[False][0])
     assert torch.equal(res[True][1], res[False][1])
+
+
+@pytest.mark.parametrize("routing", ["topk", "race"])
+def test_forward_captured_in_a_cuda_graph(routing):
+    # one graph launch reruns the whole layer; replays match the eager forward bit for bit
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    w = I.small_workload(2048, 384, 768, 16 if routing == "race" else 8, 2, 2, "bf16", routing, seed=71)
+    inp = I.make_inputs(w, bias_std=0.2)
+    L = MoELayer(LayerShape(w.T, w.D, w.H, w.E, w.K, w.n_shared, "bf16", routing, w.alpha), inp, "cuda:0")
+    x = torch.as_tensor(inp["x"]).to(device="cuda:0", dtype=L.act_dtype).contiguous()
+    eager = L.forward(x).clone()
+    eager_aux = L.aux.clone()
+    g = L.capture(x)
+    for _ in range(3):
+        L.out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(L.out, eager) and torch.equal(L.aux, eager_aux)
+    L.check()
+    # a new input in the captured buffer is routed afresh
+    x2 = torch.as_tensor(I.make_inputs(I.small_workload(2048, 384, 768, w.E, 2, 2, "bf16", routing, seed=72))["x"])
+    x.copy_(x2.to(device="cuda:0", dtype=L.act_dtype))
+    g.replay()
+    torch.cuda.synchronize()
+    fresh = L.forward(x).clone()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(L.out, fresh)

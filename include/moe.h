@@ -27,8 +27,9 @@
  *     caller; the library never allocates, frees or keeps it.  Tensors are
  *     row-major and contiguous; every tensor pointer must be 16-byte aligned.
  *   - "act" tensors (x, x_perm, h_perm, h_sh, y_perm, y_sh, out) and
- *     weights/biases have the storage type cfg->dtype (fp32 or bf16); scores and
- *     gates are fp32; indices are int32.  Every sum runs in fp32.
+ *     weights/biases have the storage type cfg->dtype (fp32, bf16 or fp16);
+ *     scores, gates and gradients are fp32; indices are int32.  Every sum runs
+ *     in fp32 (fp64 where the balance loss is finalised).
  *   - Weights follow nn.Linear (out x in): W1 [E,H,D], b1 [E,H], W2 [E,D,H],
  *     b2 [E,D].  The n_s shared experts come stacked the same way: W1s
  *     [n_s,H,D], b1s [n_s,H], W2s [n_s,D,H], b2s [n_s,D].  The kernels treat
@@ -40,7 +41,8 @@
  *   - `ws` is caller-owned device scratch of at least moe_workspace_size(cfg)
  *     bytes, 256-byte aligned.  Its first 256 bytes hold a status word that
  *     kernels set on a device-detected error (bad index, a bounded wait that
- *     ran out); moe_workspace_init() clears it and moe_check_status() reads it.
+ *     ran out) and the blocks-done counters kernels use between launches;
+ *     moe_workspace_init() clears them and moe_check_status() reads the status.
  *     A workspace must not be shared by calls that may overlap on the GPU.
  *   - Return value: MOE_OK, or a negative moe_status_t with a message
  *     available from moe_last_error() (thread-local).  Argument errors are
@@ -70,9 +72,9 @@ typedef enum {
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_F16 = 2 } moe_dtype_t;
 typedef enum { MOE_ROUTE_TOPK = 0, MOE_ROUTE_RACE = 1 } moe_routing_t;
 typedef enum {
-  MOE_GEMM_AUTO = 0, /* bf16: tcgen05 on CTA pairs (256-row tiles); fp32: FFMA */
-  MOE_GEMM_SIMT = 1, /* FFMA for both dtypes (second implementation, for checks) */
-  MOE_GEMM_TC1 = 2   /* bf16: tcgen05 on single CTAs (128-row tiles) */
+  MOE_GEMM_AUTO = 0, /* bf16 / fp16: tcgen05 on CTA pairs (256-row tiles); fp32: FFMA */
+  MOE_GEMM_SIMT = 1, /* FFMA for every dtype (a second implementation, for checks) */
+  MOE_GEMM_TC1 = 2   /* bf16 / fp16: tcgen05 on single CTAs (128-row tiles) */
 } moe_gemm_impl_t;
 
 typedef struct {
@@ -195,9 +197,10 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx
  *   h_sh[t]   = gelu(W1s x[t] + b1s)  (all n_s shared experts side by side)
  *   offsets [E+1] int32 (moe_dispatch output); b1 [E,H] / b1s [n_s,H] may be NULL;
  *   h_perm [R_max,H] act out; h_sh [T,n_s*H] act out (NULL when n_s = 0).
- * bf16: one persistent tcgen05 kernel (TMA-fed, TMEM accumulators, 256-row
- * tiles on CTA pairs) runs the routed segments and the shared block together.
- * fp32: FFMA kernel.
+ * bf16 / fp16: one persistent tcgen05 kernel (TMA-fed, TMEM accumulators,
+ * 256 x 256 tiles on CTA pairs, one narrower column tile per row block where
+ * 256 does not divide the width) runs the routed segments and the shared block
+ * together.  fp32: FFMA kernel.
  */
 int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void* x_perm,
                      const void* x, const void* w1, const void* b1, const void* w1s, const void* b1s,

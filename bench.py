@@ -41,8 +41,8 @@ SPACER_CYCLES = 400_000          # ~0.2 ms of GPU sleep after each flush, outsid
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM read + write bytes of one launch of each expert GEMM at the default workload (ncu, one pass,
 # full size; profiles/gemm_pair_dram_xl2_8e2a_512.md).  Set to None whenever the kernel changes.
-MEASURED_TRAFFIC = {("xl2_8e2a_512", "gemm1"): 344_317_184 + 1_172_789_248,
-                    ("xl2_8e2a_512", "gemm2_combine"): 1_993_010_944 + 221_332_736}
+MEASURED_TRAFFIC = {("xl2_8e2a_512", "gemm1"): 341_693_440 + 1_172_227_840,
+                    ("xl2_8e2a_512", "gemm2_combine"): 1_612_760_064 + 221_111_808}
 
 
 def load_peaks():

@@ -20,7 +20,13 @@ beyond the definition.  Sources, by page title and section:
   weight (n_routed_experts, gating_dim), softmax scoring, top_k =
   num_experts_per_tok, aux_loss_alpha.
 * "Scalable Diffusion Models with Transformers (DiT)", "DiT block 实现细节":
-  the core transformer uses the tanh approximation of GELU.
+  the core transformer uses the tanh approximation of GELU; adaLN-Zero
+  scales each residual branch by a per-sample gate alpha.
+* "Diffusion Transformer (DiT) 技术全景解析" 2.2.3 (AdaLN): a plain
+  layer_norm over the features, then a per-sample scale and shift.
+* "Scaling Diffusion Transformers to 16 Billion Parameters", expert
+  specialisation analysis: expert-selection frequency by class, spatial
+  position and denoising step.
 * "Expert Race: A Flexible Routing Strategy for Scaling Diffusion
   Transformer with Mixture of Experts", abstract: tokens and experts compete
   together and the top candidates are selected.

@@ -1,0 +1,52 @@
+"""The JSON line bench.py prints: every key the benchmark contract names, with the right types.
+
+report() is fed synthetic stage times (no GPU); the oracle timing is replaced by a
+stub so the test stays fast.
+"""
+import argparse
+import json
+
+import pytest
+
+import bench
+from sparse_moe_layer_03_b200 import inputs as I
+
+
+@pytest.mark.parametrize("fused", [True, False])
+def test_report_has_the_contract_keys(monkeypatch, fused):
+    monkeypatch.setattr(bench, "calibrated_tokens", lambda w, inp, s: 128)
+    monkeypatch.setattr(bench, "oracle_rate", lambda w, inp, n: (700.0, 0.18, 8))
+    w = I.WORKLOADS["xl2_8e2a_512"]
+    args = argparse.Namespace(steps=20, warmup=5, workload="xl2_8e2a_512", adaln="off", fuse_combine="on")
+    stages = {"route": [0.03] * 20, "dispatch": [0.05] * 20, "gemm1": [1.1] * 20}
+    if fused:
+        stages["gemm2_combine"] = [1.12] * 20
+    else:
+        stages.update(gemm2=[1.08] * 20, combine=[0.06] * 20)
+    clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 5}
+    r = bench.report(args, w, None, stages, 2.3, 2.5, clocks, 1, {})
+    line = json.loads(json.dumps(r))                     # one JSON-serialisable object
+    for k, t in [("metric", str), ("value", float), ("unit", str), ("n_gpus", int), ("steps", int),
+                 ("warmup", int), ("ms_per_step", float), ("higher_is_better", bool), ("scaling", str),
+                 ("dtype", str), ("data", str), ("config", dict), ("roofline", dict), ("cpu_baseline", dict),
+                 ("e2e", dict), ("gpu_launches", int), ("clocks", dict)]:
+        assert isinstance(line[k], t), k
+    assert line["metric"] == bench.METRIC and line["unit"] == "tokens/s" and line["scaling"] == "weak"
+    assert line["vs_baseline"] is None
+    assert abs(line["value"] - w.T / 2.3e-3) < 1.0
+    assert line["config"]["workload"] == w.name
+    rf = line["roofline"]
+    assert rf["bound"] == "tensor" and rf["unit"] == "TFLOP/s" and abs(rf["frac"] - rf["achieved"] / rf["peak"]) < 1e-3
+    assert "traffic" in rf
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 8 and cb["unit"] == "tokens/s" and cb["sample"]
+    e2e = line["e2e"]
+    assert e2e["unit"] == "tokens/s" and e2e["h2d_bytes_per_step"] == w.T * w.D * 2
+    assert e2e["d2h_bytes_per_step"] == w.T * w.D * 2 + 4
+    assert line["gpu_launches"] == (5 if fused else 6) * 20
+    assert set(line["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
+
+
+def test_warmup_below_three_is_refused():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2", "--steps", "1"])

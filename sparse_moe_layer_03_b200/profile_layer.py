@@ -4,8 +4,10 @@
 
 No timing and no checking: the seeded inputs of the workload (optionally cut
 to T tokens) go through N forward passes on cuda:0.  Each pass launches the
-layer's kernels in order: route (+ finalize; Expert-Race adds its select
-kernels), dispatch count, dispatch gather, GEMM1, GEMM2, combine.
+layer's kernels in order: route (its last CTA finalizes counts and loss;
+Expert-Race adds one select kernel), dispatch count, dispatch gather, GEMM1,
+and GEMM2 with the combine folded in (16-bit types with shared experts; else
+GEMM2 and a combine kernel).
 """
 from __future__ import annotations
 

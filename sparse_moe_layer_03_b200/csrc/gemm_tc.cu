@@ -1,7 +1,7 @@
 // Grouped expert GEMM on the 5th-generation tensor cores (tcgen05, sm_100a).
 //
 // One persistent launch computes every 128 x BN output tile of up to two
-// problems: the routed experts (rows grouped in 128-aligned expert segments,
+// problems: the routed experts (rows grouped in 256-aligned expert segments,
 // segment bounds read on the device from the dispatch offsets) and the shared
 // experts (dense rows, packed weights).  Expert MLP = W2 gelu(W1 x) ("Scaling
 // Diffusion Transformers to 16 Billion Parameters", "MOE-DIT" eq. MLP; tanh

@@ -7,11 +7,14 @@
 // Parameters", "MOE-DIT" (balance loss eq. L_balance); "Expert Race" abstract
 // (tokens and experts compete jointly for the top candidates).
 //
-// The logits are HBM-bound: x streams through shared memory once, in
-// 128-byte-swizzled column chunks fed by TMA.  bf16 and fp16 inputs take their E dot
-// products on mma.sync (the FP32 pipe alone cannot keep up with HBM at E = 16);
-// fp32 inputs use FFMA.  Per-tile partial counts and score sums are reduced in
-// a fixed order, so the loss is bit-reproducible.
+// The logits are HBM-bound: x streams through shared memory once, in blocks of
+// 16 whole rows brought by TMA (3-D boxes of 64-column blocks, 128-byte swizzle).
+// bf16 and fp16 inputs take their E dot products on mma.sync (the FP32 pipe
+// alone cannot keep up with HBM at E = 16); fp32 inputs use FFMA.  Per-tile
+// partial counts and score sums are reduced in a fixed order, so the loss is
+// bit-reproducible.  Also here: the adaLN modulation of the rows in shared
+// memory before the logits, the per-image balance loss, and the Expert-Race
+// selection (one cooperative kernel after the router).
 #include <cuda.h>
 #include <type_traits>
 #include "common.cuh"

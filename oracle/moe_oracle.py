@@ -224,6 +224,91 @@ def router_backward(x, wg, dlogits):
     return dl.T @ x, dl.sum(axis=0), dl @ wg
 
 
+# ---------------------------------------------------------------- layer backward
+
+def gelu_tanh_grad(u):
+    """d/du of the tanh GELU: 0.5 (1 + th) + 0.5 u (1 - th^2) c (1 + 3 * 0.044715 u^2),
+    th = tanh(c (u + 0.044715 u^3)), c = sqrt(2/pi)."""
+    u = as_f64(u)
+    c = math.sqrt(2.0 / math.pi)
+    th = np.tanh(c * (u + 0.044715 * u ** 3))
+    return 0.5 * (1.0 + th) + 0.5 * u * (1.0 - th * th) * c * (1.0 + 3.0 * 0.044715 * u * u)
+
+
+def _expert_backward(x, w1, b1, w2, b2, dz):
+    """Rows x [n,D] through e(x) = W2 gelu(W1 x + b1) + b2, given dz = dJ/de [n,D]:
+    returns z = e(x) and the gradients (dx, dW1, db1, dW2, db2)."""
+    u = as_f64(x) @ as_f64(w1).T
+    if b1 is not None:
+        u = u + as_f64(b1)[None, :]
+    h = gelu_tanh(u)
+    z = h @ as_f64(w2).T
+    if b2 is not None:
+        z = z + as_f64(b2)[None, :]
+    dw2 = dz.T @ h
+    db2 = dz.sum(axis=0)
+    du = (dz @ as_f64(w2)) * gelu_tanh_grad(u)
+    dw1 = du.T @ as_f64(x)
+    db1 = du.sum(axis=0)
+    dx = du @ as_f64(w1)
+    return z, dx, dw1, db1, dw2, db2
+
+
+def layer_backward(inp, idx, dout, K, alpha, aux_scale=1.0):
+    """Gradients of J = <dout, MoE(x)> + aux_scale * L_balance for the tanh-GELU layer.
+
+    The selection idx (-1 padded) and the counts are discrete (no gradient);
+    the gates g[t,i] = P[t,i] of the selected experts carry the routing
+    gradient: dP[t,i] = <dout_t, e_i(x_t)> on the selection plus the balance
+    loss's alpha f_i / T on every entry ("MOE 回顾" eq. MoE(x), "MOE-DIT" eq.
+    MLP and eq. L_balance), then back through the softmax and l = x Wg^T + b.
+    Returns a dict of dx, dwg, dbias, dw1, db1, dw2, db2, dws1, dbs1, dws2, dbs2.
+    """
+    x = as_f64(inp["x"])
+    dout = as_f64(dout)
+    T, D = x.shape
+    E = inp["w1"].shape[0]
+    P = softmax_scores(gate_logits(x, inp["wg"], inp.get("router_bias")))
+    idx = np.asarray(idx).reshape(T, -1)
+    grads = {k: np.zeros_like(as_f64(inp[w])) for k, w in
+             (("dw1", "w1"), ("dw2", "w2"), ("dws1", "ws1"), ("dws2", "ws2"))}
+    H = inp["w1"].shape[1]
+    grads["db1"] = np.zeros((E, H))
+    grads["db2"] = np.zeros((E, D))
+    ns = inp["ws1"].shape[0]
+    grads["dbs1"] = np.zeros((ns, H))
+    grads["dbs2"] = np.zeros((ns, D))
+    dx = np.zeros((T, D))
+    dP = np.zeros((T, E))
+    for e in range(E):
+        rows, slots = np.nonzero(idx == e)
+        if rows.size == 0:
+            continue
+        g = P[rows, e][:, None]
+        z, dxe, dw1, db1, dw2, db2 = _expert_backward(x[rows], inp["w1"][e], _bias_row(inp.get("b1"), e),
+                                                      inp["w2"][e], _bias_row(inp.get("b2"), e), g * dout[rows])
+        np.add.at(dx, rows, dxe)
+        grads["dw1"][e] += dw1
+        grads["db1"][e] += db1
+        grads["dw2"][e] += dw2
+        grads["db2"][e] += db2
+        dP[rows, e] += np.sum(dout[rows] * z, axis=1)
+    for j in range(ns):
+        _, dxj, dw1, db1, dw2, db2 = _expert_backward(x, inp["ws1"][j], _bias_row(inp.get("bs1"), j),
+                                                      inp["ws2"][j], _bias_row(inp.get("bs2"), j), dout)
+        dx += dxj
+        grads["dws1"][j] += dw1
+        grads["dbs1"][j] += db1
+        grads["dws2"][j] += dw2
+        grads["dbs2"][j] += db2
+    counts = expert_counts(idx, E)
+    dP += aux_scale * alpha * (E / (K * T)) * counts[None, :].astype(F64) / T
+    dl = P * (dP - np.sum(P * dP, axis=1, keepdims=True))
+    dwg, dbias, dxr = router_backward(x, inp["wg"], dl)
+    grads.update(dx=dx + dxr, dwg=dwg, dbias=dbias)
+    return grads
+
+
 # ---------------------------------------------------------------- adaLN-Zero around the layer
 
 def layer_norm(x, eps=1e-5):

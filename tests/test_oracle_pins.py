@@ -269,6 +269,52 @@ def test_balance_loss_gradient_matches_autograd(routing):
     assert np.max(np.abs(dx - xt.grad.numpy())) < 1e-15
 
 
+def test_gelu_tanh_grad_matches_autograd():
+    u = torch.linspace(-6, 6, 2001, dtype=torch.float64, requires_grad=True)
+    torch.nn.functional.gelu(u, approximate="tanh").sum().backward()
+    assert np.max(np.abs(O.gelu_tanh_grad(u.detach().numpy()) - u.grad.numpy())) < 1e-14
+
+
+@pytest.mark.parametrize("routing", ["topk", "race"])
+def test_layer_backward_matches_autograd(routing):
+    # the whole layer written with library ops in float64, the selection held fixed
+    rng = np.random.default_rng(53)
+    T, D, H, E, K, ns, alpha, lam = 24, 16, 32, 4, 2, 2, 0.05, 0.7
+    inp = {"x": rng.standard_normal((T, D)), "wg": rng.standard_normal((E, D)) / 4,
+           "router_bias": rng.standard_normal(E) * 0.2,
+           "w1": rng.standard_normal((E, H, D)) / 4, "b1": rng.standard_normal((E, H)) * 0.1,
+           "w2": rng.standard_normal((E, D, H)) / 6, "b2": rng.standard_normal((E, D)) * 0.1,
+           "ws1": rng.standard_normal((ns, H, D)) / 4, "bs1": rng.standard_normal((ns, H)) * 0.1,
+           "ws2": rng.standard_normal((ns, D, H)) / 6, "bs2": rng.standard_normal((ns, D)) * 0.1}
+    r = O.route(inp, K, routing, alpha)
+    idx = r["idx"]
+    dout = rng.standard_normal((T, D))
+    got = O.layer_backward(inp, idx, dout, K, alpha, aux_scale=lam)
+    t = {k: torch.tensor(v, requires_grad=True) for k, v in inp.items()}
+    F = torch.nn.functional
+    P = torch.softmax(F.linear(t["x"], t["wg"], t["router_bias"]), dim=1)
+    out = torch.zeros(T, D, dtype=torch.float64)
+    for e in range(E):
+        rows, slots = np.nonzero(idx == e)
+        if rows.size == 0:
+            continue
+        rr = torch.as_tensor(rows)
+        y = F.linear(F.gelu(F.linear(t["x"][rr], t["w1"][e], t["b1"][e]), approximate="tanh"), t["w2"][e], t["b2"][e])
+        out = out.index_add(0, rr, P[rr, e][:, None] * y)
+    for j in range(ns):
+        out = out + F.linear(F.gelu(F.linear(t["x"], t["ws1"][j], t["bs1"][j]), approximate="tanh"), t["ws2"][j],
+                             t["bs2"][j])
+    counts = torch.tensor(O.expert_counts(idx, E), dtype=torch.float64)
+    loss = alpha * torch.sum((E / (K * T)) * counts * P.mean(0))
+    J = (torch.tensor(dout) * out).sum() + lam * loss
+    J.backward()
+    pairs = [("dx", "x"), ("dwg", "wg"), ("dbias", "router_bias"), ("dw1", "w1"), ("db1", "b1"), ("dw2", "w2"),
+             ("db2", "b2"), ("dws1", "ws1"), ("dbs1", "bs1"), ("dws2", "ws2"), ("dbs2", "bs2")]
+    for g, k in pairs:
+        ref = t[k].grad.numpy()
+        assert np.max(np.abs(got[g] - ref)) <= 1e-12 * max(1.0, np.max(np.abs(ref))), g
+
+
 def test_balance_loss_gradient_vanishes_for_uniform_counts():
     # with every expert equally loaded, L = alpha sum_i p_i = alpha whatever the scores: zero gradient
     P = _rand_scores(32, 4, 52)
@@ -512,3 +558,13 @@ def test_planted_per_image_token_count_is_caught(monkeypatch):
     monkeypatch.setattr(O, "balance_loss_per_sequence", wrong)
     with pytest.raises(AssertionError):
         test_worked_example_per_image_loss_and_frequencies()
+
+
+def test_planted_gelu_derivative_is_caught(monkeypatch):
+    # a GELU derivative missing the tanh-slope term
+    def wrong(u):
+        c = math.sqrt(2.0 / math.pi)
+        return 0.5 * (1.0 + np.tanh(c * (u + 0.044715 * u ** 3)))
+    monkeypatch.setattr(O, "gelu_tanh_grad", wrong)
+    with pytest.raises(AssertionError):
+        test_layer_backward_matches_autograd("topk")

@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for the DiT-MoE sparse expert layer (forward).
+"""fp64 CPU oracle for the DiT-MoE sparse expert layer: the forward, the
+adaLN pieces around it, per-image statistics, and the backward.
 
 TEST INFRASTRUCTURE.  This module is the checker, not the product: only the
 test suite, the smoke check and the benchmark's CPU-baseline leg may import
@@ -37,10 +38,14 @@ experts are summed with weight 1; top-K order is descending score, ties to
 the lower expert id; Expert-Race takes the S = K*T largest of the T x E
 softmax scores, ties to the lower flat index t*E+i; the balance loss's T is
 every token of the call and its n is E; expert biases (nn.Linear) are applied
-inside e_i, before gating.
+inside e_i, before gating.  For the backward: the selection and the counts
+are discrete and carry no gradient; the gates g = P of the selected experts
+and the balance loss's p_i carry it back through the softmax.
 
 Parity status: every function here is pinned by a CPU test (closed forms,
-brute force, library special cases, invariants, a hand-worked example).  The
+brute force, library special cases, invariants, a hand-worked example; the
+backward functions against float64 torch autograd through the layer written
+with torch library ops, the selection held fixed).  The
 full-layer numeric output has no worked example on the pages, so beyond those
 pins it is "parity unpinned" against the pages themselves.
 """

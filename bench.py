@@ -182,7 +182,7 @@ def calibrated_tokens(w: I.Workload, inp: dict, target_s: float) -> int:
 def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     import torch
     from sparse_moe_layer_03_b200 import binding as B
-    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer, global_balance_loss
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -222,8 +222,12 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
         mod = B.make_adaln(gamma, beta, w.tokens_per_image, 1e-5, L.x_mod)
         res = B.make_residual(x, alpha, w.tokens_per_image)
         x_in = L.x_mod
+    if args.global_aux == "on":
+        # the balance loss of the whole batch over every rank: statistics, one all-reduce of 2E values, loss
+        stages.insert(1, "balance_exchange")
     calls = {"route": lambda: L.route(x, mod), "dispatch": lambda: L.dispatch(x_in), "gemm1": lambda: L.gemm1(x_in),
-             "gemm2": L.gemm2, "combine": lambda: L.combine(res), "gemm2_combine": lambda: L.gemm2_combine(res)}
+             "gemm2": L.gemm2, "combine": lambda: L.combine(res), "gemm2_combine": lambda: L.gemm2_combine(res),
+             "balance_exchange": lambda: global_balance_loss(L)}
 
     def step(events):
         for i, s in enumerate(stages):
@@ -327,7 +331,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
 
 def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> dict:
     peaks, peak_kind = load_peaks()
-    elem = 2 if w.dtype == "bf16" else 4
+    elem = 2 if w.dtype in ("bf16", "f16") else 4
     race = w.routing == "race"
     avg = {s: float(np.mean(v)) for s, v in per_stage.items()}
     g1 = M.gemm1_flops(w.T, w.D, w.H, w.K, w.n_shared)
@@ -357,6 +361,11 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
         else:
             a = work / (ms * 1e-3) / 1e12
             stages_out[s] = {"ms": round(ms, 4), "TFLOP/s": round(a, 1), "frac_bf16": round(a / tc_peak, 3)}
+    if "balance_exchange" in avg:
+        stages_out["balance_exchange"] = {
+            "ms": round(avg["balance_exchange"], 4),
+            "what": "moe_balance_stats, an all-reduce of the 2E statistics over the ranks (NCCL; none at one "
+                    "process), moe_balance_loss_from_stats"}
     dom = "gemm1" if avg["gemm1"] >= avg[g2_stage] else g2_stage
     dom_flops = g1 if dom == "gemm1" else g2
     achieved = dom_flops / (avg[dom] * 1e-3) / 1e12
@@ -372,6 +381,8 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
     # route (finalize fused; race: + one cooperative select-and-finalize launch), dispatch count +
     # gather, GEMM1, GEMM2 (+ combine unless folded into GEMM2)
     launches_per_step = (1 + (1 if race else 0)) + 2 + 1 + 1 + (0 if fused else 1)
+    if "balance_exchange" in avg:
+        launches_per_step += 2                  # statistics and loss kernels (the all-reduce is NCCL's)
     return {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
@@ -381,6 +392,8 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
                    "global_batch_tokens": total_tokens, "parallelism": f"dp{world}" if world > 1 else "single",
                    "adaln": ("modulation in the router and the gated residual in the combine (e2e: the plain "
                              "layer)") if args.adaln == "on" else "off",
+                   "balance_loss": ("whole batch over all ranks (one all-reduce of 2E statistics per step; e2e: "
+                                    "per rank)") if args.global_aux == "on" else "per rank (this rank's batch)",
                    "l2": "flushed between steps (256 MB written, then another 256 MB read so the written lines "
                          "return to DRAM before the step, then a 0.2 ms GPU sleep so the host is ahead; all "
                          "outside each step's events)"},
@@ -448,6 +461,9 @@ def main(argv=None):
     ap.add_argument("--adaln", default="off", choices=["on", "off"],
                     help="time the layer inside its DiT block: adaLN modulation in the router and the "
                          "adaLN-Zero gated residual in the combine (per-image gamma, beta, alpha)")
+    ap.add_argument("--global-aux", default="off", choices=["on", "off"],
+                    help="balance loss of the whole batch over every rank (statistics all-reduced each step) "
+                         "instead of each rank's own")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -299,6 +299,39 @@ int moe_route_static(const moe_config_t* cfg, const void* x, const void* wg, con
                      void* stream);
 
 /*
+ * moe_balance_stats -- the statistics the balance loss is made of, for a loss
+ * over a batch split between ranks (or between calls).  "MOE-DIT", eq.
+ * L_balance: L = alpha sum_i f_i p_i with f_i = (E/(K T)) counts_i and
+ * p_i = (1/T) sum_t P[t,i] depends on the batch only through counts_i and
+ * s_i = sum_t P[t,i], and both add over disjoint parts of the batch.
+ *   counts      [E] int32   from the last moe_route on this ws
+ *   ws          the workspace that moe_route call used (its score sums stay there
+ *               until the next moe_route on it)
+ *   stats       [2E] fp64 out: counts_0..counts_{E-1}, then s_0..s_{E-1}
+ *               (s_i summed in fp64 in the router's fixed order)
+ * Sum stats over the ranks (one all-reduce of 2E values, e.g. NCCL over
+ * NVLink), then moe_balance_loss_from_stats.  A call that routed zero tokens
+ * gives zeros.  Not available after moe_route_static (no workspace).
+ */
+int moe_balance_stats(const moe_config_t* cfg, const int32_t* counts, const void* ws, size_t ws_bytes, double* stats,
+                      void* stream);
+
+/*
+ * moe_balance_loss_from_stats -- L_balance of a batch from its summed
+ * statistics: alpha sum_i (E/(K T_total)) stats[i] (stats[E+i] / T_total),
+ * accumulated in fp64 in a fixed order, written as fp32.
+ *   stats       [2E] fp64   moe_balance_stats of every part, summed
+ *   T_total     tokens of the whole batch (the parts' T added); 0 gives 0
+ *   aux_loss    [1] fp32 out
+ * cfg supplies E, K and alpha.  With Expert-Race routing, K T_total is the
+ * batch's number of selected pairs, as in the per-call loss.  This is the
+ * whole-batch loss (seq_len is ignored): the per-image loss of seq_len > 0 is
+ * a mean over images and is not a function of these sums.
+ */
+int moe_balance_loss_from_stats(const moe_config_t* cfg, const double* stats, long long T_total, float* aux_loss,
+                                void* stream);
+
+/*
  * moe_balance_loss_backward -- gradient of the expert-level balance loss with
  * respect to the router ("MOE-DIT", eq. L_balance; the counts come from the
  * discrete selection and carry no gradient): dL/dP[t,i] = alpha f_i / T, back

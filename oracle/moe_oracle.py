@@ -155,6 +155,21 @@ def balance_loss(counts, P, K, alpha):
     return float(alpha * np.sum(f * p))
 
 
+def balance_stats(idx, P, E):
+    """[counts_0..counts_{E-1}, s_0..s_{E-1}] with s_i = sum_t P(t,i): the two per-expert
+    token sums eq. L_balance ("MOE-DIT") is made of; both add over disjoint token sets."""
+    return np.concatenate([expert_counts(idx, E).astype(F64), as_f64(P).sum(axis=0)])
+
+
+def balance_loss_from_stats(stats, K, T, alpha):
+    """L_balance of T tokens from their statistics: alpha sum_i (n/(K T)) counts_i (s_i / T)."""
+    stats = as_f64(stats)
+    E = stats.size // 2
+    if T == 0:
+        return 0.0
+    return float(alpha * np.sum((E / (K * T)) * stats[:E] * (stats[E:] / T)))
+
+
 def balance_loss_per_sequence(idx, P, K, alpha, seq_len):
     """Mean over images of L_balance with T read as one image's patch count.
 

@@ -88,6 +88,8 @@ _SIGS = {
     "moe_expert_frequency": (C.c_int, [_CFG, _P, _P, C.c_int32, _P, C.c_int32, _P, _P, _P]),
     "moe_backward_workspace_size": (C.c_size_t, [_CFG]),
     "moe_balance_loss_backward": (C.c_int, [_CFG, _P, _P, _P, _P, C.c_float, _P, _P, _P, _P, C.c_size_t, _P]),
+    "moe_balance_stats": (C.c_int, [_CFG, _P, _P, C.c_size_t, _P, _P]),
+    "moe_balance_loss_from_stats": (C.c_int, [_CFG, _P, C.c_longlong, _P, _P]),
     "moe_expert_gemm2_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            C.c_size_t, _P]),
 }
@@ -220,6 +222,16 @@ def moe_backward_workspace_size(cfg) -> int:
     if n == 0:
         raise MoeError(MOE_ERR_INVALID_ARG, lib.moe_last_error().decode())
     return n
+
+
+def moe_balance_stats(cfg, counts, ws, ws_bytes, stats, stream=0):
+    """[counts, score sums] of the last moe_route on ws, as [2E] fp64 (summable over ranks)."""
+    _check(lib.moe_balance_stats(C.byref(cfg), _ptr(counts), _ptr(ws), ws_bytes, _ptr(stats), stream))
+
+
+def moe_balance_loss_from_stats(cfg, stats, T_total, aux_loss, stream=0):
+    """Balance loss of a whole batch from its summed [2E] statistics and its token count."""
+    _check(lib.moe_balance_loss_from_stats(C.byref(cfg), _ptr(stats), int(T_total), _ptr(aux_loss), stream))
 
 
 def moe_balance_loss_backward(cfg, x, wg, router_bias, counts, grad_scale, dwg, dbias, dx, bws, bws_bytes, stream=0):

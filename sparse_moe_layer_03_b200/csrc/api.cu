@@ -83,7 +83,7 @@ constexpr int kGatherTokens = 64;
 int ngroups_of(int T) { return (T + kDispatchGroup - 1) / kDispatchGroup; }
 
 struct WsLayout {
-  size_t status, tile_counts, tile_psum, P, seq_loss, race_sync, race_loc, race_counts, group_base, total;
+  size_t status, tile_counts, tile_psum, score_sum, P, seq_loss, race_sync, race_loc, race_counts, group_base, total;
 };
 
 WsLayout ws_layout(const moe_config_t* c) {
@@ -96,6 +96,7 @@ WsLayout ws_layout(const moe_config_t* c) {
   L.status = take(256);
   L.tile_counts = take(max_route_tiles * E * 4);
   L.tile_psum = take(max_route_tiles * E * 4);
+  L.score_sum = take(E * 8);
   const bool race = c->routing == MOE_ROUTE_RACE;
   const bool per_image = c->seq_len > 0;
   L.P = take(race || per_image ? T * E * 4 : 0);
@@ -257,6 +258,9 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   if (cfg->T == 0) {
     if ((e = cudaMemsetAsync(counts, 0, cfg->E * sizeof(int32_t), s)) != cudaSuccess) return cuda_fail(e, "moe_route");
     if ((e = cudaMemsetAsync(aux_loss, 0, sizeof(float), s)) != cudaSuccess) return cuda_fail(e, "moe_route");
+    if ((e = cudaMemsetAsync(ws_at<double>(ws, ws_layout(cfg).score_sum), 0, cfg->E * sizeof(double), s)) !=
+        cudaSuccess)
+      return cuda_fail(e, "moe_route");
     return ok();
   }
   REQUIRE_PTR(x);
@@ -321,6 +325,7 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   FinalizeArgs fa{};
   fa.T = cfg->T; fa.E = cfg->E; fa.K = cfg->K; fa.alpha = cfg->alpha;
   fa.counts = counts; fa.aux_loss = aux_loss;
+  fa.score_sum = ws_at<double>(ws, L.score_sum);
   fa.tile_psum = ra.tile_psum; fa.ntiles_psum = nparts;
   fa.tile_counts = ra.tile_counts; fa.ntiles_counts = nparts;
   fa.ctr = ws_at<unsigned int>(ws, 64);
@@ -347,6 +352,32 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   fa.tile_counts = rr.tile_counts; fa.ntiles_counts = rr.grid;
   if ((e = launch_race_select(rr, fa, s)) != cudaSuccess) return cuda_fail(e, "Expert-Race select kernel");
   if (per_image && (e = launch_seq_loss(sl, s)) != cudaSuccess) return cuda_fail(e, "per-image loss kernel");
+  return ok();
+}
+
+int moe_balance_stats(const moe_config_t* cfg, const int32_t* counts, const void* ws, size_t ws_bytes, double* stats,
+                      void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  REQUIRE_PTR(counts);
+  REQUIRE_PTR(stats);
+  if ((rc = check_ws(cfg, const_cast<void*>(ws), ws_bytes))) return rc;
+  const double* ssum = ws_at<double>(const_cast<void*>(ws), ws_layout(cfg).score_sum);
+  cudaError_t e = launch_balance_stats(counts, ssum, cfg->E, stats, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "balance statistics kernel");
+  return ok();
+}
+
+int moe_balance_loss_from_stats(const moe_config_t* cfg, const double* stats, long long T_total, float* aux_loss,
+                                void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  REQUIRE_PTR(stats);
+  if (!aux_loss) return fail(MOE_ERR_INVALID_ARG, "aux_loss is NULL");
+  if (T_total < 0) return fail(MOE_ERR_INVALID_ARG, "T_total=%lld < 0", T_total);
+  cudaError_t e = launch_balance_loss_from_stats(stats, cfg->E, cfg->K, T_total, cfg->alpha, aux_loss,
+                                                 (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "balance loss kernel");
   return ok();
 }
 

@@ -49,10 +49,17 @@ struct FinalizeArgs {
   const float* tile_psum; int ntiles_psum;
   int T, E, K; float alpha;
   int32_t* counts; float* aux_loss;   // counts == null: the router leaves finalizing to a later kernel
+  double* score_sum;                  // [E] sum_t P[t,i] of the call (fp64) out, or null
   unsigned int* ctr;                  // blocks-done counter in ws (zero between calls)
 };
 cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tmap_x,
                          const CUtensorMap* tmap_m, cudaStream_t s);
+
+// balance-loss statistics of a call ([counts, score sums], fp64) and the loss from
+// statistics summed over several calls or ranks
+cudaError_t launch_balance_stats(const int32_t* counts, const double* score_sum, int E, double* stats, cudaStream_t s);
+cudaError_t launch_balance_loss_from_stats(const double* stats, int E, int K, long long T_total, float alpha,
+                                           float* aux_loss, cudaStream_t s);
 
 // per-image balance loss (seq_len > 0): overwrites aux_loss with the mean over images
 struct SeqLossArgs {

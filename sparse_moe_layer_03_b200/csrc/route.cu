@@ -285,7 +285,8 @@ __device__ __forceinline__ void route_modulate(const RouteArgs& a, uint8_t* xs, 
   }
 }
 
-// The last block to finish turns the per-block partials into counts and the loss.
+// The last block to finish turns the per-block partials into counts and the loss
+// (and, where asked, leaves the per-expert score sums for cross-call statistics).
 // Warp w reduces experts w, w + nwarps, ...: its lanes stride over the tiles
 // (independent loads), then a fixed xor tree; a fixed expert order for the
 // loss.  Bit-reproducible.  scratch: 2 x 32 x 8 bytes of shared memory.
@@ -316,6 +317,7 @@ __device__ void finalize_counts_loss(const FinalizeArgs& a, uint8_t* scratch) {
     if (tid < E) {
       const long long cc = wc[tid];
       a.counts[tid] = (int32_t)cc;
+      if (a.score_sum) a.score_sum[tid] = wp[tid];
       term = ((double)E / ((double)a.K * a.T)) * (double)cc * (wp[tid] / a.T);
     }
     for (int o = 16; o > 0; o >>= 1) term += __shfl_down_sync(0xffffffffu, term, o);

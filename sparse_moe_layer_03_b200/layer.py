@@ -26,6 +26,23 @@ def _dev(a, dtype, device):
     return t.to(device=device, dtype=dtype).contiguous()
 
 
+def global_balance_loss(layer, group=None):
+    """The cross-rank exchange of a data-parallel layer: each rank's [counts, score sums]
+    are summed by one all-reduce of 2E values, and every rank then computes the loss of
+    the whole batch.  Every rank must route the same number of tokens (T_total = T x world
+    size) and call this in the same order as the other collectives."""
+    import torch.distributed as dist
+    if layer.s.seq_len:
+        raise ValueError("the cross-rank loss is the whole-batch loss; seq_len must be 0")
+    stats = layer.balance_stats(getattr(layer, "_stats", None))
+    layer._stats = stats
+    world = 1
+    if dist.is_available() and dist.is_initialized():
+        dist.all_reduce(stats, op=dist.ReduceOp.SUM, group=group)
+        world = dist.get_world_size(group)
+    return layer.balance_loss_from_stats(stats, layer.cfg.T * world)
+
+
 @dataclass
 class LayerShape:
     T: int
@@ -196,6 +213,25 @@ class MoELayer:
         B.moe_expert_frequency(self.cfg, self.topk_idx, self.n_sel, seq_len, seq_labels, n, hist, self.ws,
                                self.stream())
         return hist
+
+    def balance_stats(self, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """[2E] fp64 statistics of the last routing: per-expert counts, then score sums."""
+        if out is None:
+            out = torch.empty((2 * self.s.E,), dtype=torch.float64, device=self.device)
+        B.moe_balance_stats(self.cfg, self.counts, self.ws, self.ws_bytes, out, self.stream())
+        return out
+
+    def balance_loss_from_stats(self, stats: torch.Tensor, T_total: int) -> torch.Tensor:
+        """Overwrite ``self.aux`` with the balance loss of a batch of T_total tokens whose
+        statistics (summed over its parts) are ``stats``."""
+        B.moe_balance_loss_from_stats(self.cfg, stats, T_total, self.aux, self.stream())
+        return self.aux
+
+    def global_balance_loss(self, group=None) -> torch.Tensor:
+        """Balance loss over the batch of every rank of ``group``: one all-reduce of the 2E
+        statistics (NCCL on GPUs), then the loss with T = the tokens of all ranks.
+        Overwrites ``self.aux`` on every rank with the same value."""
+        return global_balance_loss(self, group)
 
     def check(self):
         B.moe_check_status(self.ws, self.stream())

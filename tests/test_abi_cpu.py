@@ -122,6 +122,8 @@ def test_python_wrappers_reach_the_library():
         lambda: B.moe_expert_gemm2_combine(cfg, f, f, f, f, None, f, None, f, f, None, f, f, f, n, res=res),
         lambda: B.moe_combine(cfg, f, f, f, None, f, res=res),
         lambda: B.moe_expert_frequency(cfg, f, None, 256, None, 256, f, f),
+        lambda: B.moe_balance_stats(cfg, f, f, n, f),
+        lambda: B.moe_balance_loss_from_stats(cfg, f, 2048, f),
     ]
     for c in calls:
         with pytest.raises(B.MoeError):
@@ -158,3 +160,22 @@ def test_balance_backward_arguments_rejected_before_launch():
     per_image = B.make_config(1024, 384, 1536, 8, 2, 2, seq_len=256)
     assert f(ctypes.byref(per_image), fake, fake, None, fake, ctypes.c_float(1.0), fake, None, None, fake, n, None) == \
         B.MOE_ERR_UNSUPPORTED
+
+
+def test_balance_statistics_arguments_rejected_before_launch():
+    fake = 1 << 40
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    n = B.moe_workspace_size(cfg)
+    st = B.lib.moe_balance_stats
+    assert st(ctypes.byref(cfg), fake, fake, n, None, None) == B.MOE_ERR_INVALID_ARG
+    assert b"stats" in B.lib.moe_last_error()
+    assert st(ctypes.byref(cfg), None, fake, n, fake, None) == B.MOE_ERR_INVALID_ARG
+    assert st(ctypes.byref(cfg), fake, fake, n - 8, fake, None) == B.MOE_ERR_WORKSPACE
+    lf = B.lib.moe_balance_loss_from_stats
+    assert lf(ctypes.byref(cfg), fake, -1, fake, None) == B.MOE_ERR_INVALID_ARG
+    assert b"T_total" in B.lib.moe_last_error()
+    assert lf(ctypes.byref(cfg), fake, 1024, None, None) == B.MOE_ERR_INVALID_ARG
+    assert lf(ctypes.byref(cfg), None, 1024, fake, None) == B.MOE_ERR_INVALID_ARG
+    bad = B.make_config(1024, 384, 1536, 8, 9, 2)          # K > E
+    assert lf(ctypes.byref(bad), fake, 1024, fake, None) == B.MOE_ERR_INVALID_ARG
+

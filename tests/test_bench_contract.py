@@ -12,13 +12,16 @@ import bench
 from sparse_moe_layer_03_b200 import inputs as I
 
 
-@pytest.mark.parametrize("fused", [True, False])
-def test_report_has_the_contract_keys(monkeypatch, fused):
+@pytest.mark.parametrize("fused,exchange", [(True, False), (False, False), (True, True)])
+def test_report_has_the_contract_keys(monkeypatch, fused, exchange):
     monkeypatch.setattr(bench, "calibrated_tokens", lambda w, inp, s: 128)
     monkeypatch.setattr(bench, "oracle_rate", lambda w, inp, n: (700.0, 0.18, 8))
     w = I.WORKLOADS["xl2_8e2a_512"]
-    args = argparse.Namespace(steps=20, warmup=5, workload="xl2_8e2a_512", adaln="off", fuse_combine="on")
+    args = argparse.Namespace(steps=20, warmup=5, workload="xl2_8e2a_512", adaln="off", fuse_combine="on",
+                              global_aux="on" if exchange else "off")
     stages = {"route": [0.03] * 20, "dispatch": [0.05] * 20, "gemm1": [1.1] * 20}
+    if exchange:
+        stages["balance_exchange"] = [0.01] * 20
     if fused:
         stages["gemm2_combine"] = [1.12] * 20
     else:
@@ -43,7 +46,9 @@ def test_report_has_the_contract_keys(monkeypatch, fused):
     e2e = line["e2e"]
     assert e2e["unit"] == "tokens/s" and e2e["h2d_bytes_per_step"] == w.T * w.D * 2
     assert e2e["d2h_bytes_per_step"] == w.T * w.D * 2 + 4
-    assert line["gpu_launches"] == (5 if fused else 6) * 20
+    assert line["gpu_launches"] == ((5 if fused else 6) + (2 if exchange else 0)) * 20
+    assert ("balance_exchange" in line["stages"]) == exchange
+    assert line["config"]["balance_loss"].startswith("whole batch" if exchange else "per rank")
     assert set(line["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
 
 

@@ -141,3 +141,67 @@ def test_balance_loss_backward(case):
     assert PA.rel_err(dwg, ref_dwg) < 1e-3
     assert PA.rel_err(db, ref_db) < 1e-3
     assert PA.rel_err(dx, ref_dx) < (1e-3 if dt == "f32" else 1e-2)
+
+
+STATS_CASES = [  # T (two halves of T/2), D, E, K, dtype, routing
+    (2048, 128, 8, 2, "bf16", "topk"),
+    (2048, 128, 16, 2, "bf16", "race"),
+    (1000, 64, 8, 1, "f32", "topk"),
+    (1200, 192, 4, 2, "f16", "topk"),
+]
+
+
+@pytest.mark.parametrize("case", STATS_CASES, ids=lambda c: "T%d_D%d_E%d_K%d_%s_%s" % c)
+def test_balance_stats_and_loss_of_two_calls(case):
+    # one layer routes the two halves of a batch in two calls (as two ranks would); the sum of
+    # their statistics gives the loss of the whole batch under the union of the two selections
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    T, D, E, K, dt, routing = case
+    Th = T // 2
+    w = I.small_workload(T, D, 2 * D, E, K, 0, dt, routing, seed=11 + T + E, router_bias="normal")
+    inp = I.make_inputs(w)
+    L = MoELayer(LayerShape(Th, D, 2 * D, E, K, 0, dt, routing, w.alpha), inp, "cuda:0")
+    xs = torch.as_tensor(inp["x"]).to(device="cuda:0", dtype=L.act_dtype).contiguous()
+    stats, sels, own = [], [], []
+    for h in range(2):
+        L.route(xs[h * Th:(h + 1) * Th].contiguous())
+        st = L.balance_stats().clone()
+        own.append(L.aux.clone())
+        L.balance_loss_from_stats(st, Th)                # one call's statistics: that call's own loss
+        torch.cuda.synchronize()
+        L.check()
+        assert torch.equal(L.aux, own[-1])              # same terms, same order
+        r = PA.fetch(L)
+        idx = PA.gpu_selection(r)
+        half = slice(h * Th, (h + 1) * Th)
+        P = O.softmax_scores(O.gate_logits(inp["x"][half], inp["wg"], inp.get("router_bias")))
+        PA.check_routing(w, P, r)
+        got = st.cpu().numpy()
+        assert np.array_equal(got[:E], r["counts"].astype(np.float64))
+        assert np.max(np.abs(got[E:] - P.sum(axis=0))) <= 1e-5 * Th
+        stats.append(st)
+        sels.append((idx, P))
+    total = stats[0] + stats[1]
+    L.balance_loss_from_stats(total, T)
+    torch.cuda.synchronize()
+    idx = np.concatenate([s[0] for s in sels])
+    P = np.concatenate([s[1] for s in sels])
+    ref = O.balance_loss_from_stats(O.balance_stats(idx, P, E), K, T, w.alpha)
+    got = float(L.aux[0])
+    assert abs(got - ref) <= PA.aux_tol(w) * abs(ref), (got, ref)
+    if routing == "topk":                               # per-token selection: the whole batch's own loss
+        assert abs(ref - O.balance_loss(O.expert_counts(idx, E), P, K, w.alpha)) <= 1e-12 * ref
+    L.check()
+
+
+def test_balance_stats_of_an_empty_call():
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    w = I.small_workload(0, 128, 256, 8, 2, 0, "bf16", "topk", seed=5)
+    inp = I.make_inputs(w)
+    L = MoELayer(LayerShape(0, 128, 256, 8, 2, 0, "bf16", "topk", w.alpha), inp, "cuda:0")
+    L.route(torch.empty((0, 128), dtype=torch.bfloat16, device="cuda:0"))
+    st = L.balance_stats()
+    L.balance_loss_from_stats(st, 0)
+    torch.cuda.synchronize()
+    assert torch.all(st == 0) and float(L.aux[0]) == 0.0
+    L.check()

@@ -178,6 +178,49 @@ def test_worked_example_balance_and_race():
             assert abs(r["aux"] - want["loss"]) < 1e-15
 
 
+def test_balance_stats_of_parts_give_the_whole_batch_loss():
+    # counts and score sums add over disjoint token sets, so the loss from summed statistics
+    # of the parts is the loss of the whole batch: the hand-worked values, then a random case
+    g = json.load(open(os.path.join(GOLDEN, "balance_worked_example.json")))
+    wg = np.array([[1.0, 0.0], [0.0, 0.0]])
+    for case in g["cases"]:
+        r = O.route({"x": _golden_x(case["a"]), "wg": wg}, case["K"], "topk", g["alpha"])
+        parts = [slice(0, 2), slice(2, 4)]
+        st = sum(O.balance_stats(r["idx"][p], r["P"][p], 2) for p in parts)
+        assert abs(O.balance_loss_from_stats(st, case["K"], 4, g["alpha"]) - case["topk"]["loss"]) < 1e-15
+    rng = np.random.default_rng(61)
+    T, E, K, alpha = 97, 8, 2, 0.01
+    P = O.softmax_scores(rng.standard_normal((T, E)) * 1.5 + np.linspace(-1, 1, E))
+    idx, _ = O.topk_route(P, K)
+    whole = O.balance_loss(O.expert_counts(idx, E), P, K, alpha)
+    cuts = [0, 13, 60, 97]
+    st = sum(O.balance_stats(idx[a:b], P[a:b], E) for a, b in zip(cuts[:-1], cuts[1:]))
+    assert abs(O.balance_loss_from_stats(st, K, T, alpha) - whole) <= 1e-15 * abs(whole) * 10
+    assert np.array_equal(st[:E], O.expert_counts(idx, E))
+    assert O.balance_loss_from_stats(np.zeros(2 * E), K, 0, alpha) == 0.0
+
+
+def test_balance_stats_uniform_scores_give_alpha_for_any_split():
+    # uniform P: every p_i = 1/E and sum_i f_i = E, so L = alpha whatever the selection or split
+    T, E, K, alpha = 30, 4, 2, 0.05
+    P = np.full((T, E), 1.0 / E)
+    idx, _ = O.topk_route(P, K)
+    st = O.balance_stats(idx[:7], P[:7], E) + O.balance_stats(idx[7:], P[7:], E)
+    assert abs(O.balance_loss_from_stats(st, K, T, alpha) - alpha) < 1e-15
+
+
+def test_planted_mean_of_rank_losses_is_caught():
+    # averaging the parts' own losses is not the whole-batch loss: worked case A split in two
+    # halves gives 1.5 alpha and 1.0 alpha (mean 1.25 alpha) against 1.125 alpha for the batch
+    g = json.load(open(os.path.join(GOLDEN, "balance_worked_example.json")))
+    case = g["cases"][0]
+    r = O.route({"x": _golden_x(case["a"]), "wg": np.array([[1.0, 0.0], [0.0, 0.0]])}, 1, "topk", g["alpha"])
+    halves = [O.balance_loss(O.expert_counts(r["idx"][p], 2), r["P"][p], 1, g["alpha"])
+              for p in (slice(0, 2), slice(2, 4))]
+    assert abs(halves[0] - 1.5 * g["alpha"]) < 1e-15 and abs(halves[1] - g["alpha"]) < 1e-15
+    assert abs(np.mean(halves) - case["topk"]["loss"]) > 0.1 * g["alpha"]
+
+
 def test_worked_example_per_image_loss_and_frequencies():
     g = json.load(open(os.path.join(GOLDEN, "balance_per_image_example.json")))
     inp = {"x": _golden_x(g["a"]), "wg": np.array([[1.0, 0.0], [0.0, 0.0]])}

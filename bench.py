@@ -17,6 +17,7 @@ the method here) on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -196,7 +197,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     if rank > 0:
         inp["x"] = I.make_inputs(I.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}))["x"]
     shape = LayerShape(w.T, w.D, w.H, w.E, w.K, w.n_shared, w.dtype, w.routing, w.alpha,
-                       fuse_combine=args.fuse_combine == "on")
+                       seq_len=getattr(args, "seq_len", 0), fuse_combine=args.fuse_combine == "on")
     L = MoELayer(shape, inp, device)
     dt = L.act_dtype
     x_host = torch.as_tensor(inp["x"]).to(dt).pin_memory()
@@ -313,9 +314,32 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
             times.append(b0.elapsed_time(b1))
         bwd_ms = float(np.median(times))
 
+    # expert-selection frequency per patch position of the last routing (not part of the step): on its own
+    freq_ms = None
+    if w.tokens_per_image and w.T % w.tokens_per_image == 0:
+        for _ in range(3):
+            L.expert_frequency(w.tokens_per_image)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        times = []
+        for i in range(5):
+            flush_l2(i)
+            f0.record(stream)
+            L.expert_frequency(w.tokens_per_image)
+            f1.record(stream)
+            torch.cuda.synchronize(device)
+            times.append(f0.elapsed_time(f1))
+        freq_ms = float(np.median(times))
+        L.check()
+
     result = None
     if rank == 0:
         result = report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp)
+        if freq_ms is not None:
+            kmax = w.E if w.routing == "race" else w.K
+            moved = w.T * kmax * 4 + (w.T * 4 if w.routing == "race" else 0) + w.tokens_per_image * w.E * 4
+            result["expert_frequency"] = {"ms": round(freq_ms, 4), "GB/s": round(moved / (freq_ms * 1e-3) / 1e9, 1),
+                                          "what": "moe_expert_frequency per patch position (selection read once, "
+                                                  "[positions, E] counts written), timed separately"}
         if bwd_ms is not None:
             elem = 2 if w.dtype in ("bf16", "f16") else 4
             moved = 2 * w.T * w.D * elem + w.E * w.D * (elem + 4)
@@ -381,6 +405,8 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
     # route (finalize fused; race: + one cooperative select-and-finalize launch), dispatch count +
     # gather, GEMM1, GEMM2 (+ combine unless folded into GEMM2)
     launches_per_step = (1 + (1 if race else 0)) + 2 + 1 + 1 + (0 if fused else 1)
+    if getattr(args, "seq_len", 0):
+        launches_per_step += 1                  # the per-image loss kernel after the router
     if "balance_exchange" in avg:
         launches_per_step += 2                  # statistics and loss kernels (the all-reduce is NCCL's)
     return {
@@ -393,7 +419,10 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
                    "adaln": ("modulation in the router and the gated residual in the combine (e2e: the plain "
                              "layer)") if args.adaln == "on" else "off",
                    "balance_loss": ("whole batch over all ranks (one all-reduce of 2E statistics per step; e2e: "
-                                    "per rank)") if args.global_aux == "on" else "per rank (this rank's batch)",
+                                    "per rank)") if args.global_aux == "on" else
+                                   (f"per rank, mean over images of {args.seq_len} tokens (router stores P; "
+                                    f"one more launch)" if getattr(args, "seq_len", 0) else
+                                    "per rank (this rank's batch)"),
                    "l2": "flushed between steps (256 MB written, then another 256 MB read so the written lines "
                          "return to DRAM before the step, then a 0.2 ms GPU sleep so the host is ahead; all "
                          "outside each step's events)"},
@@ -407,10 +436,12 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
                                + (", combine folded into the shared experts' tiles)" if dom == "gemm2_combine" else ")"),
                      "bound": "tensor", "achieved": round(achieved, 1), "peak": tc_burst, "unit": "TFLOP/s",
                      "frac": round(achieved / tc_burst, 3),
-                     "traffic": MEASURED_TRAFFIC.get((args.workload, dom)),
+                     "traffic": MEASURED_TRAFFIC.get((args.workload, dom)) if w.dtype == "bf16" else None,
                      "peak_source": f"{peak_kind} bf16_tflops (burst: the timed region is short and the "
                                     f"sampled SM clock stays at its maximum); vs sustained "
-                                    f"{tc_peak}: {round(achieved / tc_peak, 3)}"},
+                                    f"{tc_peak}: {round(achieved / tc_peak, 3)}"
+                                    + ("; fp16 takes the bf16 figure (equal nominal dense rates)"
+                                       if w.dtype == "f16" else "")},
         "cpu_baseline": {"value": round(rate, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": f"{ntok} contiguous tokens of this workload through the whole fp64 oracle "
                                    f"layer (router, selection, experts, combine); {secs:.1f} s"},
@@ -464,11 +495,24 @@ def main(argv=None):
     ap.add_argument("--global-aux", default="off", choices=["on", "off"],
                     help="balance loss of the whole batch over every rank (statistics all-reduced each step) "
                          "instead of each rank's own")
+    ap.add_argument("--dtype", default=None, choices=["bf16", "f16"],
+                    help="storage type of activations and weights (default: the workload's); f16 is the "
+                         "pages' inference type")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="balance loss per image of this many tokens, averaged over the images (0: over the "
+                         "whole call)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.global_aux == "on" and args.seq_len:
+        ap.error("--global-aux gives the whole-batch loss; it does not combine with --seq-len")
     rank, world, local = dist_env()
     w = I.WORKLOADS[args.workload]
+    if args.seq_len and (args.seq_len < 0 or w.T % args.seq_len):
+        ap.error(f"--seq-len must divide T={w.T}")
+    if args.dtype and args.dtype != w.dtype:
+        base = w.name[: -len(", " + w.dtype)] if w.name.endswith(", " + w.dtype) else w.name
+        w = dataclasses.replace(w, dtype=args.dtype, name=f"{base}, {args.dtype}")
     if args.impl == "reference":
         res = run_reference(args, w, rank, world)
     else:

@@ -55,3 +55,28 @@ def test_report_has_the_contract_keys(monkeypatch, fused, exchange):
 def test_warmup_below_three_is_refused():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2", "--steps", "1"])
+
+
+def test_report_fp16_and_per_image_loss(monkeypatch):
+    import dataclasses
+    monkeypatch.setattr(bench, "calibrated_tokens", lambda w, inp, s: 128)
+    monkeypatch.setattr(bench, "oracle_rate", lambda w, inp, n: (700.0, 0.18, 8))
+    w = dataclasses.replace(I.WORKLOADS["xl2_8e2a_512"], dtype="f16")
+    args = argparse.Namespace(steps=10, warmup=3, workload="xl2_8e2a_512", adaln="off", fuse_combine="on",
+                              global_aux="off", seq_len=1024, dtype="f16")
+    stages = {"route": [0.04] * 10, "dispatch": [0.05] * 10, "gemm1": [1.1] * 10, "gemm2_combine": [1.12] * 10}
+    clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 5}
+    line = json.loads(json.dumps(bench.report(args, w, None, stages, 2.31, 2.5, clocks, 1, {})))
+    assert line["dtype"] == "f16"
+    assert line["roofline"]["traffic"] is None                 # DRAM counters were taken on the bf16 build
+    assert "fp16" in line["roofline"]["peak_source"]
+    assert line["gpu_launches"] == (5 + 1) * 10                 # + the per-image loss kernel
+    assert "mean over images of 1024" in line["config"]["balance_loss"]
+    assert line["e2e"]["h2d_bytes_per_step"] == w.T * w.D * 2
+
+
+def test_bench_refuses_inconsistent_loss_options():
+    with pytest.raises(SystemExit):
+        bench.main(["--global-aux", "on", "--seq-len", "1024"])
+    with pytest.raises(SystemExit):
+        bench.main(["--seq-len", "1000"])

@@ -294,7 +294,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
 
     # the balance loss's gradient through the router (not part of the forward step): timed on its own
     bwd_ms = None
-    if w.routing in ("topk", "race"):
+    if w.routing in ("topk", "race") and not getattr(args, "seq_len", 0):   # covers the whole-call loss only
         bws = torch.empty(B.moe_backward_workspace_size(L.cfg), dtype=torch.uint8, device=device)
         dwg = torch.empty((w.E, w.D), dtype=torch.float32, device=device)
         dbias = torch.empty((w.E,), dtype=torch.float32, device=device)

@@ -57,6 +57,13 @@ int main(void) {
                                 moe_workspace_size(&f32), 0) == MOE_ERR_UNSUPPORTED, "gather: fp32");
   CHECK(strlen(moe_last_error()) > 0, "message on failure");
 
+  /* the balance-loss statistics and the loss from summed statistics */
+  double* fd = (double*)fake;
+  CHECK(moe_balance_stats(&cfg, fi, fake, ws, 0, 0) == MOE_ERR_INVALID_ARG, "stats: stats NULL");
+  CHECK(moe_balance_stats(&cfg, fi, fake, ws - 256, fd, 0) == MOE_ERR_WORKSPACE, "stats: workspace too small");
+  CHECK(moe_balance_loss_from_stats(&cfg, fd, -1, ff, 0) == MOE_ERR_INVALID_ARG, "loss from stats: T_total < 0");
+  CHECK(moe_balance_loss_from_stats(&cfg, fd, 65536, 0, 0) == MOE_ERR_INVALID_ARG, "loss from stats: aux NULL");
+
   if (failures == 0) printf("c abi ok\n");
   return failures == 0 ? 0 : 1;
 }

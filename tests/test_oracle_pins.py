@@ -456,6 +456,19 @@ def test_sparse_equals_dense_masked(routing):
     assert np.max(np.abs(r["out"] - dense)) < 1e-12
 
 
+@pytest.mark.parametrize("routing", ["topk", "race"])
+def test_layer_output_on_a_token_subset_equals_those_rows(routing):
+    # the sampled full-size parity checks evaluate the oracle on a subset of tokens: the subset's
+    # rows must be the full evaluation's rows, in the order asked, repeats included
+    w, inp = _small_inputs(T=48, E=8, K=2, routing=routing)
+    r = O.layer(inp, 2, routing)
+    for tok in ([0], [47, 3, 19, 3], list(range(0, 48, 5)), []):
+        tok = np.asarray(tok, dtype=np.int64)
+        sub = O.layer_output(inp, r["idx"], r["g"], tokens=tok)
+        assert sub.shape == (len(tok), inp["x"].shape[1])
+        assert np.max(np.abs(sub - r["out"][tok]), initial=0.0) < 1e-13
+
+
 def test_shared_concat_identity():
     w, inp = _small_inputs(E=2, ns=3)
     x = torch.from_numpy(inp["x"].astype(np.float64))

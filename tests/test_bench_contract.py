@@ -80,3 +80,18 @@ def test_bench_refuses_inconsistent_loss_options():
         bench.main(["--global-aux", "on", "--seq-len", "1024"])
     with pytest.raises(SystemExit):
         bench.main(["--seq-len", "1000"])
+
+
+def test_reference_arm_line_on_the_host(monkeypatch):
+    # the reference arm is the oracle on the host cores: it runs here as it does on the GPU machine
+    monkeypatch.setattr(bench, "calibrated_tokens", lambda w, inp, s: 64)
+    w = I.WORKLOADS["s2_8e2a_f32"]
+    args = argparse.Namespace(steps=1, warmup=3)
+    line = json.loads(json.dumps(bench.run_reference(args, w, 0, 1)))
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "tokens/s"
+    assert line["value"] > 0 and line["steps"] == 1 and line["warmup"] == 3
+    assert line["config"]["workload"] == w.name
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and "64" in cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}

@@ -1,4 +1,5 @@
-"""B200-native DiT-MoE sparse expert layer (forward): C-ABI library + thin binding.
+"""B200-native DiT-MoE sparse expert layer (forward, with the balance loss's
+statistics and gradient): C-ABI library + thin binding.
 
 ``inputs`` (seeded synthetic workloads) and ``metrics`` (work accounting) load
 without a GPU.  The compute entry points live in ``binding`` (ctypes over

@@ -1,5 +1,6 @@
 /*
- * moe.h -- C ABI of the B200 (sm_100a) DiT-MoE sparse expert layer, forward.
+ * moe.h -- C ABI of the B200 (sm_100a) DiT-MoE sparse expert layer: the
+ * forward, the balance loss's statistics over ranks and its gradient.
  *
  * The layer (for every image-patch token x_t, width D):
  *   logits  l[t,i] = x_t . Wg[i] (+ b_i)                 i = 0..E-1

@@ -42,6 +42,8 @@ SPACER_CYCLES = 400_000          # ~0.2 ms of GPU sleep after each flush, outsid
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM read + write bytes of one launch of each expert GEMM at the default workload (ncu, one pass,
 # full size; profiles/gemm_pair_dram_xl2_8e2a_512.md).  Set to None whenever the kernel changes.
+NOMINAL_BF16_TFLOPS = 2250.0     # dense bf16 tensor rate, vendor figure
+NOMINAL_HBM_GBS = 8000.0         # HBM3e bandwidth named by the workload's targets
 MEASURED_TRAFFIC = {("xl2_8e2a_512", "gemm1"): 341_693_440 + 1_172_227_840,
                     ("xl2_8e2a_512", "gemm2_combine"): 1_612_760_064 + 221_111_808}
 
@@ -431,6 +433,10 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
         "gemm_frac_bf16": round((g1 + g2) / (gemm_ms * 1e-3) / 1e12 / tc_peak, 3),
         "mem_stages_GBps": round(mem_bytes / (mem_ms * 1e-3) / 1e9, 1),
         "mem_stages_frac_hbm": round(mem_bytes / (mem_ms * 1e-3) / 1e9 / hbm, 3),
+        "vs_nominal": {"gemm_frac": round((g1 + g2) / (gemm_ms * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS, 3),
+                       "mem_stages_frac": round(mem_bytes / (mem_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 3),
+                       "denominators": f"{NOMINAL_BF16_TFLOPS} TFLOP/s dense bf16, {NOMINAL_HBM_GBS} GB/s HBM "
+                                       "(nominal B200 figures; the fractions above use the measured peaks)"},
         "stages": stages_out,
         "roofline": {"kernel": f"tcgen05 CTA-pair grouped expert GEMM ({dom}, one launch per step"
                                + (", combine folded into the shared experts' tiles)" if dom == "gemm2_combine" else ")"),

@@ -50,6 +50,9 @@ def test_report_has_the_contract_keys(monkeypatch, fused, exchange):
     assert ("balance_exchange" in line["stages"]) == exchange
     assert line["config"]["balance_loss"].startswith("whole batch" if exchange else "per rank")
     assert set(line["clocks"]) >= {"sm_mhz", "sm_max_mhz", "reasons"}
+    nom = line["vs_nominal"]
+    assert abs(nom["gemm_frac"] - line["gemm_tflops"] / 2250.0) < 2e-3
+    assert abs(nom["mem_stages_frac"] - line["mem_stages_GBps"] / 8000.0) < 2e-3
 
 
 def test_warmup_below_three_is_refused():

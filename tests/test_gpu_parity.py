@@ -1,9 +1,10 @@
 """GPU parity: the CUDA layer, called through the C ABI, against the fp64 oracle.
 
-Small shapes (oracle in seconds) span several 128-row tiles and a ragged tail;
+Small shapes (oracle in seconds) span several 256-row tiles and a ragged tail;
 the five named workloads run at full size in the launch configuration the
-benchmark times, with routing and permutation checked on every token and the
-output on sampled tokens.
+benchmark times, with routing, permutation and output checked on every token.
+Other GEMM paths at full size are checked on 2048 sampled tokens, which put
+about 16 rows into every 256-row tile of each GEMM.
 """
 import numpy as np
 import pytest
@@ -60,7 +61,7 @@ def test_tensor_core_paths_match_ffma_path(impl):
 def test_other_gemm_paths_full_size_xl(impl):
     w = I.WORKLOADS["xl2_8e2a_512"]
     inp = I.make_inputs(w)
-    PA.full_check(w, inp, gemm_impl=impl, tokens=PA.sample_tokens(w.T, 128))
+    PA.full_check(w, inp, gemm_impl=impl, tokens=PA.sample_tokens(w.T, 2048))
 
 
 def test_erf_gelu_option():
@@ -151,10 +152,10 @@ def test_planted_bad_index_reported_not_faulted():
 
 @pytest.mark.parametrize("key", I.WORKLOAD_ORDER)
 def test_named_workload_full_size(key):
+    # every output token of the workload against the oracle (about 40 s of oracle at XL)
     w = I.WORKLOADS[key]
     inp = I.make_inputs(w)
-    tokens = PA.sample_tokens(w.T, 256 if w.T > 4096 else w.T)
-    rep = PA.full_check(w, inp, tokens=tokens)
+    rep = PA.full_check(w, inp)
     assert rep["err"] <= PA.out_tol(w)
 
 
@@ -199,7 +200,7 @@ def test_combine_folded_into_gemm2_matches_separate_combine(case):
         L.check()
         r = PA.fetch(L)
         P = O.softmax_scores(O.gate_logits(inp["x"], inp["wg"], inp.get("router_bias")))
-        PA.check_routing(w, P, r)
+        PA.check_routing(w, P, r, inp)
         PA.check_output(w, inp, P, r)
         outs[fuse] = r["out"]
     # the folded path skips one bf16 rounding of the shared output: at most a couple of bf16 ulps apart
@@ -214,11 +215,11 @@ def test_f16_other_gemm_paths(impl):
 
 
 def test_f16_full_size_xl():
-    # the XL/2-8E2A layer with fp16 storage: all output tokens sampled against the oracle
+    # the XL/2-8E2A layer with fp16 storage: every output token against the oracle
     import dataclasses
     w = dataclasses.replace(I.WORKLOADS["xl2_8e2a_512"], dtype="f16", name="DiT-MoE-XL/2-8E2A layer at 512x512, fp16")
     inp = I.make_inputs(w)
-    PA.full_check(w, inp, tokens=PA.sample_tokens(w.T, 512))
+    PA.full_check(w, inp)
 
 
 RESIDUAL_CASES = [  # T, D, H, E, K, n_s, dtype, routing, img_len, fuse
@@ -248,7 +249,7 @@ def test_adaln_zero_residual_in_combine(case):
     L.check()
     r = PA.fetch(L)
     P = O.softmax_scores(O.gate_logits(inp["x"], inp["wg"], inp.get("router_bias")))
-    PA.check_routing(w, P, r)
+    PA.check_routing(w, P, r, inp)
     idx = PA.gpu_selection(r)
     g = np.where(idx >= 0, np.take_along_axis(P, np.maximum(idx, 0), axis=1), 0.0)
     ref = O.gated_residual(x_res, O.layer_output(inp, idx, g), alpha, L_img)
@@ -302,8 +303,7 @@ def test_adaln_modulation_in_router(case):
     inp_m = dict(inp, x=got.astype(np.float64))
     r = PA.fetch(L)
     P = O.softmax_scores(O.gate_logits(inp_m["x"], inp["wg"], inp.get("router_bias")))
-    w_m = w
-    PA.check_routing(w_m, P, r)
+    PA.check_routing(w, P, r, inp_m)
     idx = PA.gpu_selection(r)
     g = np.where(idx >= 0, np.take_along_axis(P, np.maximum(idx, 0), axis=1), 0.0)
     y = O.layer_output(inp_m, idx, g)
@@ -311,6 +311,24 @@ def test_adaln_modulation_in_router(case):
     err = PA.rel_err(r["out"], ref)
     assert err <= PA.out_tol(w), err
 
+
+
+@pytest.mark.parametrize("routing", ["topk", "race"])
+def test_gathered_gemm1_rows_against_oracle(routing):
+    # GEMM1 reading its routed rows straight from x (no x_perm): routing, positions and output
+    # against the oracle
+    w = I.small_workload(1500, 384, 768, 16 if routing == "race" else 8, 2, 2, "bf16", routing, seed=63)
+    inp = I.make_inputs(w, bias_std=0.2)
+    rep = PA.full_check(w, inp, gather_rows=True)
+    assert rep["layer"].gathered and rep["layer"].x_perm is None
+    assert rep["err"] <= PA.out_tol(w)
+
+
+def test_gathered_gemm1_full_size_xl():
+    w = I.WORKLOADS["xl2_8e2a_512"]
+    inp = I.make_inputs(w)
+    rep = PA.full_check(w, inp, gather_rows=True, tokens=PA.sample_tokens(w.T, 2048))
+    assert rep["layer"].gathered
 
 
 @pytest.mark.parametrize("routing", ["topk", "race"])
@@ -360,3 +378,38 @@ def test_forward_captured_in_a_cuda_graph(routing):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(L.out, fresh)
+
+
+MLP_CASES = [  # T, D, H, E, K, n_s, dtype, routing
+    (1000, 256, 512, 8, 2, 2, "bf16", "topk"),
+    (900, 320, 640, 16, 3, 1, "bf16", "race"),
+    (700, 256, 512, 8, 2, 1, "f32", "topk"),
+    (999, 128, 256, 4, 1, 0, "f16", "topk"),
+]
+
+
+@pytest.mark.parametrize("case", MLP_CASES, ids=lambda c: "T%d_D%d_E%d_K%d_ns%d_%s_%s" % (c[0], c[1], c[3], c[4], c[5],
+                                                                                         c[6], c[7]))
+def test_expert_mlp_call_then_combine(case):
+    # moe_expert_mlp (GEMM1 then GEMM2 in one call) and moe_combine, called through the C ABI into
+    # buffers of their own after the layer's route and dispatch, against the oracle
+    from sparse_moe_layer_03_b200 import binding as B
+    T, D, H, E, K, ns, dt, routing = case
+    w = I.small_workload(T, D, H, E, K, ns, dt, routing, seed=31 + T)
+    inp = I.make_inputs(w, bias_std=0.2)
+    L, x = PA.run_layer(w, inp)
+    r = PA.fetch(L)
+    h_perm = torch.zeros_like(L.h_perm)
+    y_perm = torch.zeros_like(L.y_perm)
+    h_sh = torch.zeros((T, ns * H), dtype=L.act_dtype, device=x.device) if ns else None
+    y_sh = torch.zeros((T, D), dtype=L.act_dtype, device=x.device) if ns else None
+    out = torch.zeros_like(L.out)
+    B.moe_expert_mlp(L.cfg, L.offsets, L.x_perm, x, L.w1, L.b1, L.w2, L.b2, L.ws1, L.bs1, L.ws2, L.bs2, L.row_gate,
+                     h_perm, h_sh, y_perm, y_sh, L.ws, L.ws_bytes, L.stream())
+    B.moe_combine(L.cfg, y_perm, y_sh, L.pos, L.n_sel, out, L.stream())
+    torch.cuda.synchronize()
+    L.check()
+    r["out"] = out.float().cpu().numpy()
+    P = O.softmax_scores(O.gate_logits(inp["x"], inp["wg"], inp.get("router_bias")))
+    err = PA.check_output(w, inp, P, r)
+    assert err <= PA.out_tol(w)

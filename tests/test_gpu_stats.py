@@ -29,7 +29,7 @@ def _run(w, inp, seq_len):
 
 def _check_loss(w, inp, L, r, seq_len):
     P = O.softmax_scores(O.gate_logits(inp["x"], inp["wg"], inp.get("router_bias")))
-    PA.check_routing(w, P, r)
+    PA.check_routing(w, P, r, inp)
     idx = PA.gpu_selection(r)
     assert np.array_equal(r["counts"].astype(np.int64), O.expert_counts(idx, w.E))
     ref = O.balance_loss_per_sequence(idx, P, w.K, w.alpha, seq_len)
@@ -175,7 +175,7 @@ def test_balance_stats_and_loss_of_two_calls(case):
         idx = PA.gpu_selection(r)
         half = slice(h * Th, (h + 1) * Th)
         P = O.softmax_scores(O.gate_logits(inp["x"][half], inp["wg"], inp.get("router_bias")))
-        PA.check_routing(w, P, r)
+        PA.check_routing(w, P, r, dict(inp, x=inp["x"][half]))
         got = st.cpu().numpy()
         assert np.array_equal(got[:E], r["counts"].astype(np.float64))
         assert np.max(np.abs(got[E:] - P.sum(axis=0))) <= 1e-5 * Th

@@ -94,6 +94,9 @@ typedef struct {
                         sequence; L > 0 (L divides T) = mean over the T/L images of the loss
                         taken over each image's tokens ("MOE-DIT": T in L_balance is the
                         length of the image-patch sequence) */
+  int32_t gemm_pairs; /* CTA pairs (two SMs each) the tensor-core expert GEMMs may occupy at
+                         once: 0 = as many as the device holds; a smaller value leaves SMs free
+                         for work on other streams.  The result does not depend on it. */
 } moe_config_t;
 
 /* The adaLN-Zero residual connection around the layer, applied where the
@@ -136,8 +139,21 @@ size_t moe_workspace_size(const moe_config_t* cfg);
  * R_max = round_up(K*T + 255*E, 256).  Host only. */
 int64_t moe_max_rows(const moe_config_t* cfg);
 
-/* Zero the first 256 bytes of `ws`: the status word and the blocks-done counters the
- * kernels use between launches (asynchronous on `stream`).  Once before first use. */
+/* Zero the first 256 bytes of `ws`: the status word and the counters the kernels keep
+ * between launches (asynchronous on `stream`).  Once before first use.
+ * Layout of those bytes: status word and error site (0, 4); blocks-done counters of the
+ * router (64), the dispatch (128) and the per-image loss (192); the fused GEMM2's count of
+ * finished routed tiles (224); the CTA-pair GEMM's exit and tile-claim counters (228, 232).
+ * Every kernel leaves its counters at zero when it ends.
+ * Bytes 240..247 are two test words that only the host writes (zero in normal use); they let a
+ * test make a bounded wait run out without faulting anything:
+ *   word at 240, bit 0: the routed tiles of moe_expert_gemm2_combine do not report themselves
+ *                       done, so the shared tiles' wait for them cannot end;
+ *                bit 1: each grid barrier of the Expert-Race selection waits for one arrival
+ *                       more than the launch makes;
+ *   word at 244: limit of those two waits in microseconds (0 = the default of 1 s).
+ * A wait that runs out records MOE_ERR_TIMEOUT for moe_check_status; the kernel then finishes
+ * with invalid outputs, and the next call (with the words cleared) is unaffected. */
 int moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronise `stream`, read the status word of `ws`, clear it, and return
@@ -251,11 +267,13 @@ int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* 
  *   out[t] = sum_k y_perm[pos[t,k]] + sum_j (W2s_j h_sh_j + b2s_j), rounded once;
  *   with `res` (or NULL), out[t] = x_res[t] + alpha[t/img_len] * (that sum).
  * Only for bf16 or fp16 with gemm_impl AUTO and n_shared >= 1 (MOE_ERR_UNSUPPORTED
- * otherwise: call moe_expert_gemm2 and moe_combine).  Uses the words at byte
- * offsets 224 and 228 of ws, which must be zero on entry (moe_workspace_init;
- * each launch leaves them zero).  All CTAs of the launch must be resident at
- * once (one per SM, as launched); a wait that runs out reports MOE_ERR_TIMEOUT
- * through moe_check_status.
+ * otherwise: call moe_expert_gemm2 and moe_combine).  Uses the counters at byte
+ * offsets 224..235 of ws, which must be zero on entry (moe_workspace_init; each
+ * launch leaves them zero).  Tiles are claimed in increasing order, routed ones
+ * first, so the shared tiles only ever wait for routed tiles that running CTA
+ * pairs hold: the wait ends however few pairs the device runs at once (other
+ * streams' kernels included).  A wait that runs out (1 s) reports
+ * MOE_ERR_TIMEOUT through moe_check_status.
  */
 int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, const void* h_perm, const void* h_sh,
                              const void* w2, const void* b2, const void* w2s, const void* b2s, const float* row_gate,
@@ -291,13 +309,19 @@ int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,
  *     stream capture.  The call allocates nothing itself.
  *   - All calls share the one array: calls that may overlap on the GPU (other
  *     streams, other threads) race and must be serialised by the caller.  Each
- *     call clears the array's status word and counters itself; device-detected
- *     errors are not reported back (there is no workspace to pass to
- *     moe_check_status).
+ *     call clears the array's counters itself.  Device-detected errors (a
+ *     bounded wait that ran out, for instance) stay in the array's status word
+ *     until moe_route_static_check_status reads them.
  */
 int moe_route_static(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
                      int32_t* topk_idx, float* topk_w, int32_t* n_sel, int32_t* counts, float* aux_loss,
                      void* stream);
+
+/* moe_check_status for the built-in array of moe_route_static on the current
+ * device: synchronise `stream`, read the first error the router's kernels
+ * recorded since the last check (MOE_OK, MOE_ERR_DEVICE_CHECK or
+ * MOE_ERR_TIMEOUT) and clear it.  Blocks; allocates nothing. */
+int moe_route_static_check_status(void* stream);
 
 /*
  * moe_balance_stats -- the statistics the balance loss is made of, for a loss

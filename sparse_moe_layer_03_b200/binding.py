@@ -26,7 +26,7 @@ class MoeConfig(C.Structure):
     _fields_ = [("T", C.c_int32), ("D", C.c_int32), ("H", C.c_int32), ("E", C.c_int32),
                 ("K", C.c_int32), ("n_shared", C.c_int32), ("dtype", C.c_int32),
                 ("routing", C.c_int32), ("alpha", C.c_float), ("act", C.c_int32),
-                ("gemm_impl", C.c_int32), ("seq_len", C.c_int32)]
+                ("gemm_impl", C.c_int32), ("seq_len", C.c_int32), ("gemm_pairs", C.c_int32)]
 
 
 class MoeAdaln(C.Structure):
@@ -85,6 +85,7 @@ _SIGS = {
                                  _P, C.c_size_t, _P]),
     "moe_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
     "moe_route_static": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "moe_route_static_check_status": (C.c_int, [_P]),
     "moe_expert_frequency": (C.c_int, [_CFG, _P, _P, C.c_int32, _P, C.c_int32, _P, _P, _P]),
     "moe_backward_workspace_size": (C.c_size_t, [_CFG]),
     "moe_balance_loss_backward": (C.c_int, [_CFG, _P, _P, _P, _P, C.c_float, _P, _P, _P, _P, C.c_size_t, _P]),
@@ -119,11 +120,12 @@ def _check(rc: int):
 
 
 def make_config(T, D, H, E, K, n_shared, dtype="bf16", routing="topk", alpha=0.01, act="tanh",
-                gemm_impl="auto", seq_len=0) -> MoeConfig:
+                gemm_impl="auto", seq_len=0, gemm_pairs=0) -> MoeConfig:
     return MoeConfig(T, D, H, E, K, n_shared, {"f32": MOE_F32, "bf16": MOE_BF16, "f16": MOE_F16}[dtype],
                      MOE_ROUTE_RACE if routing == "race" else MOE_ROUTE_TOPK, alpha,
                      1 if act == "erf" else 0,
-                     {"auto": MOE_GEMM_AUTO, "simt": MOE_GEMM_SIMT, "tc1": MOE_GEMM_TC1}[gemm_impl], seq_len)
+                     {"auto": MOE_GEMM_AUTO, "simt": MOE_GEMM_SIMT, "tc1": MOE_GEMM_TC1}[gemm_impl], seq_len,
+                     gemm_pairs)
 
 
 def moe_version() -> int:
@@ -201,6 +203,11 @@ def moe_route_static(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, a
     """moe_route without a workspace: scratch comes from the library's built-in 4 MiB array."""
     _check(lib.moe_route_static(C.byref(cfg), _ptr(x), _ptr(wg), _ptr(router_bias), _ptr(topk_idx), _ptr(topk_w),
                                 _ptr(n_sel), _ptr(counts), _ptr(aux_loss), stream))
+
+
+def moe_route_static_check_status(stream=0):
+    """Read and clear the first device-detected error of moe_route_static's calls (blocks)."""
+    _check(lib.moe_route_static_check_status(stream))
 
 
 def moe_expert_frequency(cfg, topk_idx, n_sel, seq_len, seq_labels, n_labels, hist, ws, stream=0):

@@ -62,6 +62,7 @@ int validate(const moe_config_t* c) {
   if (c->act != 0 && c->act != 1) return fail(MOE_ERR_INVALID_ARG, "act=%d", c->act);
   if (c->gemm_impl < MOE_GEMM_AUTO || c->gemm_impl > MOE_GEMM_TC1) return fail(MOE_ERR_INVALID_ARG, "gemm_impl=%d", c->gemm_impl);
   if (c->seq_len < 0) return fail(MOE_ERR_INVALID_ARG, "seq_len=%d < 0", c->seq_len);
+  if (c->gemm_pairs < 0) return fail(MOE_ERR_INVALID_ARG, "gemm_pairs=%d < 0", c->gemm_pairs);
   if (c->seq_len > 0 && c->T % c->seq_len)
     return fail(MOE_ERR_INVALID_ARG, "seq_len=%d does not divide T=%d", c->seq_len, c->T);
   if (route_smem_total(c->D, c->E, 32, is16(c)) > 232448 ||
@@ -126,6 +127,12 @@ int check_ws(const moe_config_t* c, void* ws, size_t ws_bytes) {
   do {                                                                              \
     if ((p) && !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
   } while (0)
+
+// words of the workspace's first 256 bytes (besides the status word at 0): blocks-done counters
+// of the router (64), the dispatch count (128) and the per-image loss (192); the fused GEMM2's
+// routed-tile count (224); the CTA-pair GEMM's exit counter (228) and tile claim counter (232);
+// two test words written only by the host (240: flags, 244: wait limit in microseconds)
+constexpr size_t kWsDoneCtr = 224, kWsExitCtr = 228, kWsSchedCtr = 232, kWsTestWords = 240;
 
 int* status_ptr(void* ws) { return reinterpret_cast<int*>(ws); }
 template <typename T> T* ws_at(void* ws, size_t off) { return reinterpret_cast<T*>((uint8_t*)ws + off); }
@@ -349,6 +356,7 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   rr.topk_idx = topk_idx; rr.topk_w = topk_w; rr.n_sel = n_sel;
   rr.tile_counts = ws_at<int32_t>(ws, L.race_counts);
   rr.status = status_ptr(ws);
+  rr.test = ws_at<const uint32_t>(ws, kWsTestWords);
   fa.tile_counts = rr.tile_counts; fa.ntiles_counts = rr.grid;
   if ((e = launch_race_select(rr, fa, s)) != cudaSuccess) return cuda_fail(e, "Expert-Race select kernel");
   if (per_image && (e = launch_seq_loss(sl, s)) != cudaSuccess) return cuda_fail(e, "per-image loss kernel");
@@ -540,7 +548,6 @@ namespace {
 int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long rows0, const void* B0,
              long long brows0, const void* A1, long long rows1, const void* B1, long long brows1, int K0,
              int K1, int bcols1, void* ws, cudaStream_t s) {
-  (void)ws;
   cudaError_t e;
   const bool tc = is16(cfg) && cfg->gemm_impl != MOE_GEMM_SIMT;
   if (!tc) {
@@ -581,7 +588,11 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
     } else {
       to[1] = to[0];
     }
-    if ((e = launch_gemm_pair(g, ta, tb, to, bn, num_sms_current(), s)) != cudaSuccess)
+    // tile claim counter, exit counter and test words of the workspace header
+    g.sched_ctr = ws_at<unsigned int>(ws, kWsSchedCtr);
+    g.exit_ctr = ws_at<unsigned int>(ws, kWsExitCtr);
+    g.test = ws_at<const uint32_t>(ws, kWsTestWords);
+    if ((e = launch_gemm_pair(g, ta, tb, to, bn, num_sms_current(), cfg->gemm_pairs, s)) != cudaSuccess)
       return cuda_fail(e, "tcgen05 CTA-pair expert GEMM");
     return ok();
   }
@@ -747,8 +758,7 @@ int moe_expert_gemm2_combine(const moe_config_t* cfg, const int32_t* offsets, co
   p1.gate = nullptr;
   g.pos = pos; g.n_sel = n_sel; g.kmax = kmax_of(cfg); g.kdef = cfg->K;
   g.y_routed = y_perm;
-  g.done_ctr = ws_at<unsigned int>(ws, 224);
-  g.exit_ctr = ws_at<unsigned int>(ws, 228);
+  g.done_ctr = ws_at<unsigned int>(ws, kWsDoneCtr);
   if (res) { g.x_res = res->x_res; g.alpha = res->alpha; g.img_len = res->img_len; }
   return run_gemm(cfg, g, h_perm, R, w2, (long long)cfg->E * cfg->D, h_sh, cfg->T, w2s,
                   (long long)ns * cfg->D, cfg->H, ns * cfg->H, cfg->H, ws, (cudaStream_t)stream);

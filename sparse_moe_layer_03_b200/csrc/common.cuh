@@ -332,6 +332,15 @@ __device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const void* tmap,
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar), "l"(policy)
       : "memory");
 }
+// arrive on an mbarrier of any CTA of the cluster, releasing this thread's earlier writes
+// (shared::cluster stores included) at cluster scope
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// 32-bit store into the shared memory of any CTA of the cluster (shared::cluster address)
+__device__ __forceinline__ void st_shared_cluster_s32(uint32_t addr, int v) {
+  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 // remote arrive.expect_tx on a shared::cluster mbarrier address
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)

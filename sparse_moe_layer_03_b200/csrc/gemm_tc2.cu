@@ -21,7 +21,18 @@
 // CTA, by shared::cluster address); every epilogue warp of both CTAs arrives
 // on the leader's "accumulator empty" barrier; both CTAs' TMA loads complete
 // on the leader's "stage full" barrier.  All waits are bounded.
+//
+// Scheduling: persistent pairs claim tiles in increasing order from a counter
+// in global memory (the leader's producer claims one tile ahead and hands each
+// id to the other roles of both CTAs through a small ring in shared memory).
+// Routed tiles are numbered before shared ones, so when the combine is folded
+// into the shared tiles, a shared tile can only wait for routed tiles that
+// resident pairs have already claimed: no wait depends on a pair that is not
+// running, however many pairs the device holds at once.
 #include <cuda.h>
+
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,6 +43,8 @@ constexpr int kPairBK = 64;             // 16-bit elements per 128-byte swizzle 
 constexpr int kPairEpiWarps = 4;          // one per TMEM lane quadrant
 constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
 constexpr int kPairSmemLimit = 232448;
+constexpr int kSchedSlots = 4;                                  // tile ids handed out ahead
+constexpr int kSchedConsumers = 2 + 2 * kPairEpiWarps;          // peer producer, MMA issuer, epilogue warps
 
 template <int BN>
 struct PairCfg {
@@ -90,6 +103,38 @@ __device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, co
   return ti;
 }
 
+// Next tile id of a consumer role (lane 0): wait for the ring slot, read it, and release the
+// slot on the leader.  -1: no tile left (or a wait ran out, recorded in the status word).
+__device__ __forceinline__ int sched_take(uint64_t* sfull, uint64_t* sempty, volatile int* stile, uint32_t& n,
+                                          volatile int* abort_flag, int* status, int where) {
+  const uint32_t slot = n % kSchedSlots, ph = (n / kSchedSlots) & 1u;
+  ++n;
+  if (!mbar_wait_cluster(smem_u32(&sfull[slot]), ph, abort_flag, status, where)) return -1;
+  const int t = stile[slot];
+  mbar_arrive_release_cluster(map_to_cta(smem_u32(&sempty[slot]), 0));
+  return t;
+}
+
+// Leader producer (lane 0): hand tile id t (-1 = none left) to both CTAs' ring once the slot
+// is free.  False when the wait ran out.
+__device__ __forceinline__ bool sched_publish(uint64_t* sfull, uint64_t* sempty, volatile int* stile, uint32_t& n,
+                                              int t, volatile int* abort_flag, int* status) {
+  const uint32_t slot = n % kSchedSlots, ph = (n / kSchedSlots) & 1u;
+  ++n;
+  if (!mbar_wait_cluster(smem_u32(&sempty[slot]), ph ^ 1u, abort_flag, status, 507)) return false;
+  stile[slot] = t;
+  st_shared_cluster_s32(map_to_cta(smem_u32((const void*)&stile[slot]), 1), t);
+  mbar_arrive(smem_u32(&sfull[slot]));
+  mbar_arrive_release_cluster(map_to_cta(smem_u32(&sfull[slot]), 1));
+  return true;
+}
+
+// Claim the next tile of the launch (-1 when every tile is taken).
+__device__ __forceinline__ int sched_claim(unsigned int* ctr, int total) {
+  const int t = (int)atomicAdd(ctr, 1u);
+  return t < total ? t : -1;
+}
+
 template <int BN, typename S>
 __global__ void __launch_bounds__(kPairThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
@@ -105,13 +150,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
   uint64_t* acc_full = empty + C::STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sched_full = drain + 1;
+  uint64_t* sched_empty = sched_full + kSchedSlots;
+  volatile int* sched_tile = reinterpret_cast<volatile int*>(sched_empty + kSchedSlots);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sched_empty + kSchedSlots) + kSchedSlots;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   __shared__ PairPlan pl;
 
   const int warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();          // 0 = leader of the pair
-  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -123,6 +170,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       mbar_init(smem_u32(&acc_empty[i]), 2 * kPairEpiWarps);   // leader: every epilogue warp of both CTAs
     }
     mbar_init(smem_u32(drain), 1);
+    for (int i = 0; i < kSchedSlots; ++i) {
+      mbar_init(smem_u32(&sched_full[i]), 1);                  // the leader producer's hand-over
+      mbar_init(smem_u32(&sched_empty[i]), kSchedConsumers);  // leader: every consumer role of the pair
+    }
     *abort_flag = 0;
     fence_barrier_init();
     bool bad = false;
@@ -146,7 +197,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       pl.ntiles[q] = mt * pl.nn[q];
     }
     pl.total = pl.ntiles[0] + pl.ntiles[1];
-    if (bad && rank == 0 && cid == 0) set_status(a.status, DEV_BAD_INDEX, 500);
+    if (bad && rank == 0 && blockIdx.x == 0) set_status(a.status, DEV_BAD_INDEX, 500);
     prefetch_tmap(&ta0);
     prefetch_tmap(&tb0);
     prefetch_tmap(&ta1);
@@ -173,7 +224,25 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     int stage = 0;
     uint32_t phase = 0;
     bool alive = true;
-    for (int tile = cid; tile < pl.total && alive; tile += ncl) {
+    uint32_t sn = 0;
+    int next = (rank == 0 && lane == 0) ? sched_claim(a.sched_ctr, pl.total) : -1;
+    while (alive) {
+      // the leader hands its claimed tile to both CTAs and claims the one after it while the
+      // loads go out; the peer takes the tile from its ring
+      int tile = -1, ok = 1;
+      if (lane == 0) {
+        if (rank == 0) {
+          tile = next;
+          ok = sched_publish(sched_full, sched_empty, sched_tile, sn, tile, abort_flag, a.status) ? 1 : 0;
+          if (ok && tile >= 0) next = sched_claim(a.sched_ctr, pl.total);
+        } else {
+          tile = sched_take(sched_full, sched_empty, sched_tile, sn, abort_flag, a.status, 508);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      if (!ok) { alive = false; break; }
+      if (tile < 0) break;
       const PairTile ti = pair_decode<BN>(tile, pl, a);
       const GemmProblem& pr = a.p[ti.p];
       const CUtensorMap* tA = ti.p ? &ta1 : &ta0;
@@ -222,9 +291,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int local = 0;
       bool issued_any = false;
-      for (int tile = cid; tile < pl.total; tile += ncl, ++local) {
+      uint32_t sn = 0;
+      for (int local = 0;; ++local) {
+        const int tile = sched_take(sched_full, sched_empty, sched_tile, sn, abort_flag, a.status, 509);
+        if (tile < 0) break;
         const PairTile ti = pair_decode<BN>(tile, pl, a);
         const int acc = local & 1;
         const uint32_t accph = (local >> 1) & 1;
@@ -273,10 +344,19 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     // combine folded into the shared tiles: every epilogue warp of both CTAs counts each routed tile
     const bool count_routed = a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr;
     const unsigned int done_target = (unsigned int)pl.ntiles[0] * 2u * kPairEpiWarps;
+    // test words (host-written, zero in normal use): bit 0 of word 0 makes the routed tiles skip
+    // their count, so the shared tiles' wait cannot end; word 1 shortens that wait to microseconds
+    const uint32_t tflags = (count_routed && a.test != nullptr) ? __ldcg(a.test) : 0u;
+    const uint32_t tlimit_us = (count_routed && a.test != nullptr) ? __ldcg(a.test + 1) : 0u;
+    const uint64_t done_limit = tlimit_us ? (uint64_t)tlimit_us * 1000ull : kWaitLimitNs;
     bool routed_done = false;
     int nstore = 0;
-    int local = 0;
-    for (int tile = cid; tile < pl.total; tile += ncl, ++local) {
+    uint32_t sn = 0;
+    for (int local = 0;; ++local) {
+      int tile = 0;
+      if (lane == 0) tile = sched_take(sched_full, sched_empty, sched_tile, sn, abort_flag, a.status, 510);
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      if (tile < 0) break;
       const PairTile ti = pair_decode<BN>(tile, pl, a);
       const GemmProblem& pr = a.p[ti.p];
       const CUtensorMap* tO = ti.p ? &to1 : &to0;
@@ -302,7 +382,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           if (lane == 0) {
             const uint64_t t0 = global_ns();
             while (ld_acquire_gpu_u32(a.done_ctr) < done_target) {
-              if (global_ns() - t0 > kWaitLimitNs) { set_status(a.status, DEV_TIMEOUT, 506); break; }
+              if (global_ns() - t0 > done_limit) { set_status(a.status, DEV_TIMEOUT, 506); break; }
               __nanosleep(64);
             }
           }
@@ -421,12 +501,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
-      if (count_routed && ti.p == 0 && lane == 0) {
+      if (count_routed && ti.p == 0 && lane == 0 && !(tflags & 1u)) {
         // this warp's rows of a routed tile are in global memory: count them for the combine
         bulk_wait_all();
         fence_proxy_async_all();
         __threadfence();
         atomicAdd(a.done_ctr, 1u);
+        __threadfence();                           // the count lands before this CTA reports its exit
       }
     }
     if (lane == 0) bulk_wait_all();            // stores done before the CTA may exit
@@ -437,10 +518,13 @@ done:
   cluster_sync();                                   // no CTA leaves while its peer may still use it
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
-  if (threadIdx.x == 0 && a.exit_ctr != nullptr && a.nprob > 1 && a.p[1].epi == 2) {
-    // the last CTA out resets the combine counters for the next launch (all reads are done)
+  if (threadIdx.x == 0) {
+    // the last CTA out resets the tile counter and the combine count for the next launch (every
+    // claim of every CTA has returned before its exit is counted)
+    __threadfence();
     if (atomicAdd(a.exit_ctr, 1u) == gridDim.x - 1) {
-      *a.done_ctr = 0u;
+      *a.sched_ctr = 0u;
+      if (a.done_ctr != nullptr) *a.done_ctr = 0u;
       *a.exit_ctr = 0u;
       __threadfence();
     }
@@ -449,12 +533,12 @@ done:
 
 template <int BN, typename S>
 static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb,
-                                  const CUtensorMap* to, int grid, cudaStream_t s) {
+                                  const CUtensorMap* to, int num_sms, int max_pairs, cudaStream_t s) {
   using C = PairCfg<BN>;
   cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<BN, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.gridDim = dim3(num_sms & ~1, 1, 1);
   cfg.blockDim = dim3(kPairThreads, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
@@ -465,6 +549,27 @@ static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // pairs the device can hold at once (one per TPC normally; fewer on a partitioned device):
+  // asked once per device, then at most that many are launched
+  static std::mutex mu;
+  static int fit[kMaxDevicesCached] = {0};
+  int dev = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  int pairs = 0;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < kMaxDevicesCached && fit[dev] > 0) {
+      pairs = fit[dev];
+    } else {
+      err = cudaOccupancyMaxActiveClusters(&pairs, gemm_pair_kernel<BN, S>, &cfg);
+      if (err != cudaSuccess) return err;
+      if (pairs < 1) return cudaErrorInvalidConfiguration;
+      if (dev >= 0 && dev < kMaxDevicesCached) fit[dev] = pairs;
+    }
+  }
+  const int grid = pair_grid(num_sms, pairs, max_pairs);
+  if (grid < 2) return cudaErrorInvalidConfiguration;
+  cfg.gridDim = dim3(grid, 1, 1);
   return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, S>, ta[0], tb[0], ta[1], tb[1], to[0], to[1], a);
 }
 
@@ -477,10 +582,10 @@ int gemm_pair_pick_bn(int n0, int n1) {
 }
 
 cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, const CUtensorMap* to,
-                             int bn, int num_sms, cudaStream_t s) {
-  const int grid = num_sms & ~1;
+                             int bn, int num_sms, int max_pairs, cudaStream_t s) {
   if (bn != 256) return cudaErrorInvalidValue;
-  return a.f16 ? launch_pair_bn<256, StoreF16>(a, ta, tb, to, grid, s) : launch_pair_bn<256, StoreBF16>(a, ta, tb, to, grid, s);
+  return a.f16 ? launch_pair_bn<256, StoreF16>(a, ta, tb, to, num_sms, max_pairs, s)
+               : launch_pair_bn<256, StoreBF16>(a, ta, tb, to, num_sms, max_pairs, s);
 }
 
 }  // namespace moe

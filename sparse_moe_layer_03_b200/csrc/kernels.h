@@ -12,6 +12,18 @@ void set_last_error_message(const char* msg);
 // every expert segment of the permuted buffers starts on a multiple of this many rows
 constexpr int kSegAlign = 256;
 
+// per-device values cached by the launchers (devices 0 .. kMaxDevicesCached-1)
+constexpr int kMaxDevicesCached = 64;
+
+// CTAs of a CTA-pair GEMM launch: one pair per two SMs, at most `fit` pairs (what the device
+// holds at once) and at most `max_pairs` (0 = no limit of the caller's)
+inline int pair_grid(int num_sms, int fit, int max_pairs) {
+  int pairs = num_sms / 2;
+  if (fit < pairs) pairs = fit;
+  if (max_pairs > 0 && max_pairs < pairs) pairs = max_pairs;
+  return pairs > 0 ? 2 * pairs : 0;
+}
+
 // ---- route.cu
 struct RouteArgs {
   const void* x;            // [T,D] act
@@ -118,6 +130,7 @@ struct RaceArgs {
   int32_t* n_sel;           // [T]
   int32_t* tile_counts;     // [grid,E]
   int* status;
+  const uint32_t* test;     // two host-written test words (flags, wait limit in us) or null
 };
 // CTAs for T tokens on `sms` SMs; *tpc = tokens per CTA
 int race_plan(int T, int sms, int* tpc);
@@ -170,12 +183,14 @@ struct GemmArgs {
   // combine folded into the shared-expert epilogue (epi 2 on problem 1): the routed
   // tiles of the same launch write y_routed; each epilogue warp counts its finished
   // routed tiles in done_ctr, and the shared tiles wait for all of them
+  unsigned int* sched_ctr;  // CTA-pair kernel: tile claim counter, zero on entry; the last CTA resets it
+  unsigned int* exit_ctr;   // CTAs that finished (the last one resets the counters)
+  const uint32_t* test;     // two host-written test words (flags, wait limit in us) or null
   const int32_t* pos;       // [T,kmax] rows of y_routed per token slot (-1 unused)
   const int32_t* n_sel;     // [T] or null (then kdef slots per token)
   int kmax, kdef;
   const void* y_routed;     // [r_max, N] act
-  unsigned int* done_ctr;   // zero on entry; the launch's last CTA resets both counters
-  unsigned int* exit_ctr;
+  unsigned int* done_ctr;   // zero on entry; the launch's last CTA resets it
   const void* x_res;        // adaLN-Zero residual in the epi-2 output: x_res + alpha[t / img_len] * sum, or null
   const void* alpha;
   int img_len;
@@ -184,7 +199,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, const CUtensorMap* ta, const CUten
                            int num_sms, cudaStream_t s);
 int gemm_tc_pick_bn(int n0, int n1);
 cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, const CUtensorMap* to,
-                             int bn, int num_sms, cudaStream_t s);
+                             int bn, int num_sms, int max_pairs, cudaStream_t s);
 int gemm_pair_pick_bn(int n0, int n1);
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t s);
 

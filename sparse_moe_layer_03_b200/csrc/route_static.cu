@@ -15,8 +15,9 @@
 // on the first call made on that device.  Every call shares the array: calls
 // that may run at the same time on the GPU (different streams, or threads) race
 // and must be serialised by the caller.  The array keeps the last call's
-// contents; the part that must start at zero (status word and blocks-done
-// counter) is cleared by each call.
+// contents; the counters that must start at zero are cleared by each call.
+// The status word is not: like a workspace's, it keeps the first error a
+// kernel found until moe_route_static_check_status reads and clears it.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -84,9 +85,22 @@ extern "C" int moe_route_static(const moe_config_t* cfg, const void* x, const vo
   void* ws = nullptr;
   int rc = scratch_for_current_device(&ws);
   if (rc != MOE_OK) return rc;
-  // status word and blocks-done counter must start at zero on every call
-  rc = moe_workspace_init(ws, kStaticScratchBytes, stream);
-  if (rc != MOE_OK) return rc;
+  // the counters after the status word (and its error site) start at zero on every call; the
+  // status word itself keeps an earlier call's error until it is read
+  cudaError_t e = cudaMemsetAsync(static_cast<unsigned char*>(ws) + 8, 0, 248, (cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    char msg[160];
+    snprintf(msg, sizeof(msg), "moe_route_static: clearing the counters failed (%s)", cudaGetErrorString(e));
+    moe::set_last_error_message(msg);
+    return MOE_ERR_CUDA;
+  }
   return moe_route(cfg, x, wg, router_bias, topk_idx, topk_w, n_sel, counts, aux_loss, nullptr, ws,
                    kStaticScratchBytes, stream);
+}
+
+extern "C" int moe_route_static_check_status(void* stream) {
+  void* ws = nullptr;
+  const int rc = scratch_for_current_device(&ws);
+  if (rc != MOE_OK) return rc;
+  return moe_check_status(ws, stream);
 }

@@ -60,6 +60,7 @@ class LayerShape:
     fuse_combine: bool = True  # fold the combine into the shared experts' GEMM2 where supported
     gather_rows: bool = False  # GEMM1 gathers its routed rows from x by TMA gather4 (no x_perm); measured
                                # slower at XL (GEMM1 2.37 ms against 1.11 ms): off by default
+    gemm_pairs: int = 0        # CTA pairs the tensor-core GEMMs may occupy at once (0 = as many as fit)
 
 
 class MoELayer:
@@ -69,7 +70,8 @@ class MoELayer:
         self.s = shape
         self.device = torch.device(device)
         self.cfg = B.make_config(shape.T, shape.D, shape.H, shape.E, shape.K, shape.n_shared, shape.dtype,
-                                 shape.routing, shape.alpha, shape.act, shape.gemm_impl, shape.seq_len)
+                                 shape.routing, shape.alpha, shape.act, shape.gemm_impl, shape.seq_len,
+                                 shape.gemm_pairs)
         self.act_dtype = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[shape.dtype]
         dt, dev = self.act_dtype, self.device
         self.wg = _dev(params["wg"], dt, dev)

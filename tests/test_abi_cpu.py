@@ -179,3 +179,15 @@ def test_balance_statistics_arguments_rejected_before_launch():
     bad = B.make_config(1024, 384, 1536, 8, 9, 2)          # K > E
     assert lf(ctypes.byref(bad), fake, 1024, fake, None) == B.MOE_ERR_INVALID_ARG
 
+
+
+def test_negative_gemm_pairs_rejected():
+    fake = 1 << 40
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2, gemm_pairs=-1)
+    assert B.lib.moe_workspace_size(ctypes.byref(cfg)) == 0
+    assert b"gemm_pairs" in B.lib.moe_last_error()
+    ok = B.make_config(1024, 384, 1536, 8, 2, 2, gemm_pairs=3)
+    assert B.lib.moe_workspace_size(ctypes.byref(ok)) > 0
+    f = B.lib.moe_expert_gemm1
+    assert f(ctypes.byref(cfg), fake, fake, fake, fake, None, fake, None, fake, fake, fake, 1 << 20, None) == \
+        B.MOE_ERR_INVALID_ARG

@@ -21,8 +21,8 @@ from sparse_moe_layer_03_b200 import inputs as I
 pytestmark = pytest.mark.gpu
 
 
-def _route_both(w, inp, dev="cuda:0"):
-    cfg = B.make_config(w.T, w.D, w.H, w.E, w.K, w.n_shared, w.dtype, w.routing, w.alpha)
+def _route_both(w, inp, dev="cuda:0", seq_len=0):
+    cfg = B.make_config(w.T, w.D, w.H, w.E, w.K, w.n_shared, w.dtype, w.routing, w.alpha, seq_len=seq_len)
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     x = torch.as_tensor(inp["x"]).to(dev, dt)
     wg = torch.as_tensor(inp["wg"]).to(dev, dt)
@@ -47,15 +47,19 @@ def _route_both(w, inp, dev="cuda:0"):
         B.moe_route_static(cfg, x, wg, bias, *o, stream)
         runs.append(o)
     torch.cuda.synchronize()
+    B.moe_route_static_check_status(stream)   # no device-detected error in either call
+    B.moe_check_status(ws, stream)
     return ref, runs
 
 
-@pytest.mark.parametrize("key,T", [("xl2_8e2a_512", 4096), ("s2_8e2a_f32", 512), ("xl_race_16e", 3000),
-                                   ("xl2_8e2a_512", 32768)])
-def test_static_scratch_router_matches_workspace_router(key, T):
+@pytest.mark.parametrize("key,T,seq_len", [("xl2_8e2a_512", 4096, 0), ("s2_8e2a_f32", 512, 0),
+                                           ("xl_race_16e", 3000, 0), ("xl2_8e2a_512", 32768, 0),
+                                           ("xl2_8e2a_512", 8192, 1024)])
+def test_static_scratch_router_matches_workspace_router(key, T, seq_len):
+    # seq_len > 0: per-image losses, whose T x E score matrix also lives in the scratch
     w = I.WORKLOADS[key].with_tokens(T)
     inp = I.make_inputs(w)
-    ref, runs = _route_both(w, inp)
+    ref, runs = _route_both(w, inp, seq_len=seq_len)
     for o in runs:
         assert torch.equal(o[0], ref[0])                               # topk_idx: exact
         assert torch.allclose(o[1], ref[1], rtol=0, atol=1e-6)         # gates
@@ -71,3 +75,10 @@ def test_static_scratch_rejects_oversized_config_without_launching():
     rc = B.lib.moe_route_static(ctypes.byref(cfg), None, None, None, None, None, None, None, None, None)
     assert rc == B.MOE_ERR_WORKSPACE
     assert b"4194304" in B.lib.moe_last_error()
+    # per-image losses keep the T x E score matrix in the scratch too: top-K at E = 8 then fits
+    # about 113k tokens, not the 262144 of the whole-call loss
+    ok = B.make_config(65536, 1152, 4608, 8, 2, 2, seq_len=1024)
+    big = B.make_config(131072, 1152, 4608, 8, 2, 2, seq_len=1024)
+    assert B.moe_workspace_size(ok) <= 4194304 < B.moe_workspace_size(big)
+    rc = B.lib.moe_route_static(ctypes.byref(big), None, None, None, None, None, None, None, None, None)
+    assert rc == B.MOE_ERR_WORKSPACE

@@ -11,6 +11,11 @@ scaling; the batches are independent, so there is no data-path collective),
 the timed region is bracketed by a barrier and a synchronize, and the max over
 ranks is reported.  Rank 0 prints one JSON line.
 
+The line's headline is the XL/2-8E2A workload; the key ``workloads`` adds the
+device time of the other four workloads of the method (fewer steps, same
+timing rules).  ``--gpus N`` without torchrun relaunches itself under
+torch.distributed.run with N ranks on 127.0.0.1.
+
 --impl reference times the fp64 CPU oracle (the only other implementation of
 the method here) on a bounded sample of the same workload.
 """
@@ -18,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import dataclasses
+import hashlib
 import json
 import os
 import statistics
@@ -40,12 +46,30 @@ DEFAULT_WORKLOAD = "xl2_8e2a_512"
 L2_FLUSH_BYTES = 256 << 20
 SPACER_CYCLES = 400_000          # ~0.2 ms of GPU sleep after each flush, outside the timed events
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM read + write bytes of one launch of each expert GEMM at the default workload (ncu, one pass,
-# full size; profiles/gemm_pair_dram_xl2_8e2a_512.md).  Set to None whenever the kernel changes.
 NOMINAL_BF16_TFLOPS = 2250.0     # dense bf16 tensor rate, vendor figure
 NOMINAL_HBM_GBS = 8000.0         # HBM3e bandwidth named by the workload's targets
-MEASURED_TRAFFIC = {("xl2_8e2a_512", "gemm1"): 341_693_440 + 1_172_227_840,
-                    ("xl2_8e2a_512", "gemm2_combine"): 1_612_760_064 + 221_111_808}
+# DRAM read + write bytes of one launch of each expert GEMM at the default workload (ncu, one pass,
+# full size), valid only for the GEMM sources they were measured on: GEMM_SOURCES hashed to
+# TRAFFIC_SOURCES_SHA.  Any change to those files makes the reported traffic null until re-measured.
+GEMM_SOURCES = ("sparse_moe_layer_03_b200/csrc/gemm_tc2.cu", "sparse_moe_layer_03_b200/csrc/common.cuh")
+TRAFFIC_SOURCES_SHA = ""
+MEASURED_TRAFFIC = {}
+EXTRA_STEPS = 10                 # timed steps of each other workload in the ``workloads`` key
+
+
+def gemm_sources_sha() -> str:
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, stage: str):
+    """ncu DRAM bytes of one launch, or None when the GEMM sources changed since the capture."""
+    if not TRAFFIC_SOURCES_SHA or gemm_sources_sha() != TRAFFIC_SOURCES_SHA:
+        return None
+    return MEASURED_TRAFFIC.get((workload, stage))
 
 
 def load_peaks():
@@ -182,6 +206,70 @@ def calibrated_tokens(w: I.Workload, inp: dict, target_s: float) -> int:
 
 # ------------------------------------------------------------------ our arm
 
+def time_steps(stages, calls, stream, steps, flush_l2):
+    """Run `steps` steps (each stage between CUDA events on `stream`, L2 flushed before every
+    step outside the events); returns per-stage ms lists and per-step totals."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(steps)]
+    for i in range(steps):
+        flush_l2(i)
+        for j, st in enumerate(stages):
+            ev[i][j].record(stream)
+            calls[st]()
+        ev[i][len(stages)].record(stream)
+    torch.cuda.synchronize()
+    per_stage = {st: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)] for j, st in enumerate(stages)}
+    totals = [ev[i][0].elapsed_time(ev[i][len(stages)]) for i in range(steps)]
+    return per_stage, totals
+
+
+def other_workloads(args, device, world, flush_l2) -> dict:
+    """Device time of every workload besides the headline one, on this rank (max over ranks)."""
+    import torch
+    from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
+    peaks, _ = load_peaks()
+    out = {}
+    for key in I.WORKLOAD_ORDER:
+        if key == args.workload:
+            continue
+        w = I.WORKLOADS[key]
+        inp = I.make_inputs(w)
+        L = MoELayer(LayerShape(w.T, w.D, w.H, w.E, w.K, w.n_shared, w.dtype, w.routing, w.alpha), inp, device)
+        x = torch.as_tensor(inp["x"]).to(device=device, dtype=L.act_dtype)
+        stages = ["route", "dispatch", "gemm1"] + (["gemm2_combine"] if L.fused else ["gemm2", "combine"])
+        calls = {"route": lambda: L.route(x), "dispatch": lambda: L.dispatch(x), "gemm1": lambda: L.gemm1(x),
+                 "gemm2": L.gemm2, "combine": L.combine, "gemm2_combine": L.gemm2_combine}
+        stream = torch.cuda.current_stream(device)
+        time_steps(stages, calls, stream, max(3, args.warmup), flush_l2)
+        steps = min(args.steps, EXTRA_STEPS)
+        per_stage, totals = time_steps(stages, calls, stream, steps, flush_l2)
+        L.check()
+        ms = reduce_max(sum(totals), world, device) / steps
+        elem = 2 if w.dtype in ("bf16", "f16") else 4
+        race = w.routing == "race"
+        avg = {st: float(np.mean(v)) for st, v in per_stage.items()}
+        g1 = M.gemm1_flops(w.T, w.D, w.H, w.K, w.n_shared)
+        g2 = M.gemm2_flops(w.T, w.D, w.H, w.K, w.n_shared)
+        work = {"route": ("GB/s", M.route_bytes(w.T, w.D, w.E, w.K, elem, race)),
+                "dispatch": ("GB/s", M.dispatch_bytes(w.T, w.D, w.E, w.K, elem, race)),
+                "gemm1": ("TFLOP/s", g1), "gemm2": ("TFLOP/s", g2), "gemm2_combine": ("TFLOP/s", g2),
+                "combine": ("GB/s", M.combine_bytes(w.T, w.D, w.K, w.n_shared, elem))}
+        st_out = {}
+        for st in stages:
+            unit, amount = work[st]
+            rate = amount / (avg[st] * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+            frac = rate / (peaks["hbm_gbs"] if unit == "GB/s" else peaks["bf16_tflops"])
+            st_out[st] = {"ms": round(avg[st], 4), unit: round(rate, 1),
+                          ("frac_hbm" if unit == "GB/s" else "frac_bf16"): round(frac, 3)}
+        out[key] = {"workload": w.name, "dtype": w.dtype, "T": w.T, "steps": steps,
+                    "ms_per_step": round(ms, 4), "tokens/s": round(w.T * world / (ms * 1e-3), 1),
+                    "layer_tflops": round(M.gemm_flops(w.T, w.D, w.H, w.K, w.n_shared) / (ms * 1e-3) / 1e12, 1),
+                    "stages": st_out}
+        del L, x, inp
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
     import torch
     from sparse_moe_layer_03_b200 import binding as B
@@ -232,14 +320,6 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
              "gemm2": L.gemm2, "combine": lambda: L.combine(res), "gemm2_combine": lambda: L.gemm2_combine(res),
              "balance_exchange": lambda: global_balance_loss(L)}
 
-    def step(events):
-        for i, s in enumerate(stages):
-            events[i].record(stream)
-            calls[s]()
-        events[len(stages)].record(stream)
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(args.steps)]
-    wev = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
     def flush_l2(i):
         # write a buffer larger than L2; then read another one as large, so the written lines
         # go back to DRAM here and not inside the next stage's events (a write-back L2 keeps
@@ -249,29 +329,16 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
         flush_clean.sum()
         torch.cuda._sleep(SPACER_CYCLES)
 
-    for i in range(args.warmup):
-        flush_l2(i)
-        step(wev)
-    torch.cuda.synchronize(device)
+    time_steps(stages, calls, stream, args.warmup, flush_l2)
     L.check()
 
     barrier(world, device)
     torch.cuda.synchronize(device)
     with ClockSampler(gpu_index_for(local)) as clk:
-        for i in range(args.steps):
-            flush_l2(i)                      # outside the step's events
-            step(ev[i])
-        torch.cuda.synchronize(device)
+        per_stage, totals = time_steps(stages, calls, stream, args.steps, flush_l2)
     barrier(world, device)
     L.check()
     clocks = clk.summary()
-
-    per_stage = {s: [] for s in stages}
-    totals = []
-    for i in range(args.steps):
-        for j, s in enumerate(stages):
-            per_stage[s].append(ev[i][j].elapsed_time(ev[i][j + 1]))
-        totals.append(ev[i][0].elapsed_time(ev[i][len(stages)]))
     my_ms = sum(totals)
     max_ms = reduce_max(my_ms, world, device)
     ms_per_step = max_ms / args.steps
@@ -333,9 +400,13 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
         freq_ms = float(np.median(times))
         L.check()
 
+    others = other_workloads(args, device, world, flush_l2) if args.other_workloads == "on" else None
+
     result = None
     if rank == 0:
         result = report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp)
+        if others is not None:
+            result["workloads"] = others
         if freq_ms is not None:
             kmax = w.E if w.routing == "race" else w.K
             moved = w.T * kmax * 4 + (w.T * 4 if w.routing == "race" else 0) + w.tokens_per_image * w.E * 4
@@ -442,7 +513,7 @@ def report(args, w, L, per_stage, ms_per_step, e2e_ms, clocks, world, inp) -> di
                                + (", combine folded into the shared experts' tiles)" if dom == "gemm2_combine" else ")"),
                      "bound": "tensor", "achieved": round(achieved, 1), "peak": tc_burst, "unit": "TFLOP/s",
                      "frac": round(achieved / tc_burst, 3),
-                     "traffic": MEASURED_TRAFFIC.get((args.workload, dom)) if w.dtype == "bf16" else None,
+                     "traffic": measured_traffic(args.workload, dom) if w.dtype == "bf16" else None,
                      "peak_source": f"{peak_kind} bf16_tflops (burst: the timed region is short and the "
                                     f"sampled SM clock stays at its maximum); vs sustained "
                                     f"{tc_peak}: {round(achieved / tc_peak, 3)}"
@@ -486,6 +557,18 @@ def run_reference(args, w: I.Workload, rank: int, world: int) -> dict:
             "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def relaunch(n: int, argv: list):
+    """Start this script under torch.distributed.run with n ranks (one per GPU) on 127.0.0.1 and
+    exit with its status; rank 0 prints the line."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    sys.exit(subprocess.call(cmd))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -507,12 +590,21 @@ def main(argv=None):
     ap.add_argument("--seq-len", type=int, default=0,
                     help="balance loss per image of this many tokens, averaged over the images (0: over the "
                          "whole call)")
+    ap.add_argument("--other-workloads", default="on", choices=["on", "off"],
+                    help="also time the method's other workloads (key `workloads` of the line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.global_aux == "on" and args.seq_len:
         ap.error("--global-aux gives the whole-batch loss; it does not combine with --seq-len")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        relaunch(args.gpus, sys.argv[1:] if argv is None else list(argv))
+        return
     rank, world, local = dist_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but the launcher started {world} rank(s)")
     w = I.WORKLOADS[args.workload]
     if args.seq_len and (args.seq_len < 0 or w.T % args.seq_len):
         ap.error(f"--seq-len must divide T={w.T}")

@@ -98,3 +98,35 @@ def test_reference_arm_line_on_the_host(monkeypatch):
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and "64" in cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_gpus_mismatch_with_launcher_is_refused(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    with pytest.raises(SystemExit):
+        bench.main(["--gpus", "2", "--steps", "1", "--warmup", "3"])
+
+
+def test_gpus_without_launcher_relaunches_under_torchrun(monkeypatch):
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    seen = {}
+
+    def fake_call(cmd):
+        seen["cmd"] = cmd
+        return 0
+    monkeypatch.setattr(bench.subprocess, "call", fake_call)
+    with pytest.raises(SystemExit) as ei:
+        bench.main(["--gpus", "4", "--steps", "7", "--warmup", "3"])
+    assert ei.value.code == 0
+    cmd = seen["cmd"]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"] and "--nproc-per-node=4" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-6:] == ["--gpus", "4", "--steps", "7", "--warmup", "3"]
+
+
+def test_traffic_is_null_once_the_gemm_sources_change(monkeypatch):
+    key = ("xl2_8e2a_512", "gemm1")
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", {key: 123})
+    monkeypatch.setattr(bench, "TRAFFIC_SOURCES_SHA", bench.gemm_sources_sha())
+    assert bench.measured_traffic(*key) == 123
+    monkeypatch.setattr(bench, "TRAFFIC_SOURCES_SHA", "0" * 16)
+    assert bench.measured_traffic(*key) is None

@@ -198,7 +198,8 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
  *   pos        [T,Kmax] int32 out row of (t, slot k) in the permuted buffers, -1 if unused
  *   row_token  [R_max] int32 out  token of each row, -1 on padding rows
  *   row_gate   [R_max] fp32 out   gate of each row, 0 on padding rows
- *   x_perm     [R_max,D] act out  x_perm[pos[t,k]] = x[t]; padding rows untouched.  NULL:
+ *   x_perm     [R_max,D] act out  x_perm[pos[t,k]] = x[t]; the padding rows of each expert
+ *              segment are written with zeros (rows after the last segment are untouched).  NULL:
  *              write the positions only (x may then be NULL too), for
  *              moe_expert_gemm1_gather, which reads the rows of x itself
  * An index outside [0,E) is skipped and sets MOE_ERR_DEVICE_CHECK in ws.
@@ -373,6 +374,79 @@ size_t moe_backward_workspace_size(const moe_config_t* cfg);
 int moe_balance_loss_backward(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
                               const int32_t* counts, float grad_scale, float* dwg, float* dbias, void* dx,
                               void* bws, size_t bws_bytes, void* stream);
+
+/*
+ * The expert MLPs' backward ("Scaling Diffusion Transformers to 16 Billion
+ * Parameters": the DiT-MoE models are trained; "MOE 回顾" eq. MoE(x) and
+ * "MOE-DIT" eq. MLP give the forward it differentiates).  For an objective J
+ * with dout = dJ/dMoE(x):
+ *   dZ_r  = g_r dout[t_r]                    (each routed row r of token t_r)
+ *   dH_r  = dZ_r W2_e,  dU_r = dH_r * gelu'(u_r),  u_r = W1_e x_r + b1_e
+ *   dW2_e = sum_r dZ_r^T gelu(u_r),  db2_e = sum_r dZ_r
+ *   dW1_e = sum_r dU_r^T x_r,        db1_e = sum_r dU_r
+ *   dgate[t,k] = dJ/dg = <dout_t, e_i(x_t)> for the token's k-th selected expert i
+ *   dx_t  = sum_k (dU W1)[pos[t,k]] + the shared experts' part (weight 1, same forms)
+ * The selection is discrete (no gradient through it); moe_router_backward takes
+ * dgate the rest of the way to Wg, the router bias and x.
+ */
+typedef struct {
+  const void* w1; const void* b1;     /* [E,H,D] act, [E,H] act or NULL */
+  const void* w2; const void* b2;     /* [E,D,H], [E,D] or NULL */
+  const void* w1s; const void* b1s;   /* [n_s,H,D], [n_s,H] or NULL (n_s = 0: NULL) */
+  const void* w2s; const void* b2s;   /* [n_s,D,H], [n_s,D] or NULL */
+} moe_expert_weights_t;
+
+typedef struct {                      /* fp32, the weights' shapes; overwritten.  Bias gradients may be NULL */
+  float* dw1; float* db1; float* dw2; float* db2;
+  float* dws1; float* dbs1; float* dws2; float* dbs2;
+} moe_expert_grads_t;
+
+/* Scratch of moe_expert_backward: dout and g*dout in permuted order, the
+ * pre-activations (overwritten by dU), dx per routed row, the gates' row dots
+ * and column-sum partials.  Host only. */
+size_t moe_expert_backward_workspace_size(const moe_config_t* cfg);
+
+/*
+ * moe_expert_backward -- gradients of the expert MLPs, of their input and of the gates.
+ *   x, x_perm, offsets, pos, topk_idx, n_sel, row_token, row_gate: the forward's
+ *               input and its moe_route / moe_dispatch outputs (x_perm's padding
+ *               rows are the zeros moe_dispatch writes)
+ *   wts         the forward's expert weights
+ *   h_perm, h_sh  the forward's moe_expert_gemm1 outputs (gelu(u) per row)
+ *   dout        [T,D] act: dJ/dMoE(x)
+ *   grads       fp32 weight gradients out (see moe_expert_grads_t)
+ *   dgate       [T,Kmax] fp32 out: dJ/dg per selected slot, 0 on unused slots
+ *   dx          [T,D] act out: the experts' part of dJ/dx
+ *   ws          the forward's workspace (status word and GEMM counters)
+ *   bws         scratch of moe_expert_backward_workspace_size(cfg) bytes, 256-byte aligned
+ * Every GEMM runs on the CTA-pair tensor cores (the weights and the weight
+ * gradients' operands are read MN-major by TMA, no transposed copies): the
+ * pre-activations again, dU with the GELU derivative and the gates' row dots in
+ * its epilogue, dx with the combine folded in, and dW2, dW1 reducing over each
+ * expert's rows.  bf16 or fp16 with gemm_impl AUTO and act = 0 only
+ * (MOE_ERR_UNSUPPORTED otherwise).  Sums of the bias gradients run in a fixed order.
+ */
+int moe_expert_backward(const moe_config_t* cfg, const void* x, const void* x_perm, const int32_t* offsets,
+                        const int32_t* pos, const int32_t* topk_idx, const int32_t* n_sel, const int32_t* row_token,
+                        const float* row_gate, const moe_expert_weights_t* wts, const void* h_perm, const void* h_sh,
+                        const void* dout, const moe_expert_grads_t* grads, float* dgate, void* dx, void* ws,
+                        size_t ws_bytes, void* bws, size_t bws_bytes, void* stream);
+
+/*
+ * moe_router_backward -- the router's part of the layer's backward: dJ/dP =
+ * aux_scale * (the balance loss's alpha f_i / T on every score) + dgate on the
+ * selected slots, back through the softmax and l = x Wg^T + b.
+ *   x, wg, router_bias, counts, topk_idx, n_sel  as in the forward
+ *   dgate       [T,Kmax] fp32 from moe_expert_backward, or NULL (balance loss only)
+ *   dwg [E,D] fp32 out; dbias [E] fp32 out or NULL; dx [T,D] act or NULL
+ *   dx_accumulate  1: dx += the router's part (dx holds the experts' part), 0: dx = it
+ *   bws         scratch of moe_backward_workspace_size(cfg) bytes
+ * Whole-call balance loss only (seq_len = 0).  Fixed-order sums: bit-reproducible.
+ */
+int moe_router_backward(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
+                        const int32_t* counts, const int32_t* topk_idx, const int32_t* n_sel, const float* dgate,
+                        float aux_scale, float* dwg, float* dbias, void* dx, int32_t dx_accumulate, void* bws,
+                        size_t bws_bytes, void* stream);
 
 /*
  * moe_expert_frequency -- expert-selection frequency per label, the statistic of

@@ -56,6 +56,22 @@ def _res_ref(r):
     return None if r is None else C.byref(r)
 
 
+class MoeExpertWeights(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("w1", "b1", "w2", "b2", "w1s", "b1s", "w2s", "b2s")]
+
+
+class MoeExpertGrads(C.Structure):
+    _fields_ = [(n, C.c_void_p) for n in ("dw1", "db1", "dw2", "db2", "dws1", "dbs1", "dws2", "dbs2")]
+
+
+def make_expert_weights(w1, b1, w2, b2, w1s, b1s, w2s, b2s):
+    return MoeExpertWeights(*[_ptr(t) for t in (w1, b1, w2, b2, w1s, b1s, w2s, b2s)])
+
+
+def make_expert_grads(dw1, db1, dw2, db2, dws1, dbs1, dws2, dbs2):
+    return MoeExpertGrads(*[_ptr(t) for t in (dw1, db1, dw2, db2, dws1, dbs1, dws2, dbs2)])
+
+
 class MoeError(RuntimeError):
     def __init__(self, code: int, msg: str):
         super().__init__(f"moe error {code}: {msg}")
@@ -93,6 +109,11 @@ _SIGS = {
     "moe_balance_loss_from_stats": (C.c_int, [_CFG, _P, C.c_longlong, _P, _P]),
     "moe_expert_gemm2_combine": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            C.c_size_t, _P]),
+    "moe_expert_backward_workspace_size": (C.c_size_t, [_CFG]),
+    "moe_expert_backward": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P, C.POINTER(MoeExpertWeights), _P, _P,
+                                      _P, C.POINTER(MoeExpertGrads), _P, _P, _P, C.c_size_t, _P, C.c_size_t, _P]),
+    "moe_router_backward": (C.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, C.c_float, _P, _P, _P, C.c_int32, _P,
+                                      C.c_size_t, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -245,3 +266,27 @@ def moe_balance_loss_backward(cfg, x, wg, router_bias, counts, grad_scale, dwg, 
     """Gradient of the balance loss through the router: dWg [E,D], db [E] (fp32) and dx [T,D] (act)."""
     _check(lib.moe_balance_loss_backward(C.byref(cfg), _ptr(x), _ptr(wg), _ptr(router_bias), _ptr(counts),
                                          grad_scale, _ptr(dwg), _ptr(dbias), _ptr(dx), _ptr(bws), bws_bytes, stream))
+
+
+def moe_expert_backward_workspace_size(cfg) -> int:
+    n = lib.moe_expert_backward_workspace_size(C.byref(cfg))
+    if n == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, lib.moe_last_error().decode())
+    return n
+
+
+def moe_expert_backward(cfg, x, x_perm, offsets, pos, topk_idx, n_sel, row_token, row_gate, weights, h_perm, h_sh,
+                        dout, grads, dgate, dx, ws, ws_bytes, bws, bws_bytes, stream=0):
+    """Gradients of the expert MLPs (weights, biases), of the gates and the experts' part of dx."""
+    _check(lib.moe_expert_backward(C.byref(cfg), _ptr(x), _ptr(x_perm), _ptr(offsets), _ptr(pos), _ptr(topk_idx),
+                                   _ptr(n_sel), _ptr(row_token), _ptr(row_gate), C.byref(weights), _ptr(h_perm),
+                                   _ptr(h_sh), _ptr(dout), C.byref(grads), _ptr(dgate), _ptr(dx), _ptr(ws), ws_bytes,
+                                   _ptr(bws), bws_bytes, stream))
+
+
+def moe_router_backward(cfg, x, wg, router_bias, counts, topk_idx, n_sel, dgate, aux_scale, dwg, dbias, dx,
+                        dx_accumulate, bws, bws_bytes, stream=0):
+    """The router's gradients (dWg, db, dx) from the gates' gradient and the balance loss."""
+    _check(lib.moe_router_backward(C.byref(cfg), _ptr(x), _ptr(wg), _ptr(router_bias), _ptr(counts), _ptr(topk_idx),
+                                   _ptr(n_sel), _ptr(dgate), aux_scale, _ptr(dwg), _ptr(dbias), _ptr(dx),
+                                   int(dx_accumulate), _ptr(bws), bws_bytes, stream))

@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
 SOURCES = ["api.cu", "route.cu", "dispatch.cu", "gemm_tc.cu", "gemm_tc2.cu", "gemm_simt.cu", "combine.cu",
-           "route_static.cu", "stats.cu", "backward.cu"]
+           "route_static.cu", "stats.cu", "backward.cu", "expert_backward.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I" + os.path.join(ROOT, "include")]

@@ -397,7 +397,12 @@ BwdLayout bwd_layout(const moe_config_t* c) {
   auto take = [&](size_t bytes) { size_t o = off; off += round_up(bytes ? bytes : 1, 256); return o; };
   L.dl = take((size_t)c->T * c->E * sizeof(float));
   L.db_part = take((size_t)kBwdMaxBlocks * c->E * sizeof(float));
-  L.partials = take((size_t)balance_grad_chunks(c->T) * c->E * c->D * sizeof(float));
+  // partial rows: one per chunk of tokens (three-kernel path) or per CTA of the one-pass kernel
+  int pass_tpc = 0;
+  const size_t pass_rows = (size_t)router_bwd_pass_grid(c->T, num_sms_current(), &pass_tpc);
+  const size_t chunks = (size_t)balance_grad_chunks(c->T);
+  const size_t nparts = chunks > pass_rows ? chunks : pass_rows;
+  L.partials = take(nparts * c->E * c->D * sizeof(float));
   L.total = off;
   return L;
 }
@@ -408,9 +413,13 @@ size_t moe_backward_workspace_size(const moe_config_t* cfg) {
   return bwd_layout(cfg).total;
 }
 
-int moe_balance_loss_backward(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
-                              const int32_t* counts, float grad_scale, float* dwg, float* dbias, void* dx,
-                              void* bws, size_t bws_bytes, void* stream) {
+namespace {
+// The router's backward: dJ/dP = the balance loss's term (times aux_scale) on every score plus
+// dgate on the selected slots (or none), through the softmax and l = x Wg^T + b.
+int router_backward(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
+                    const int32_t* counts, const int32_t* topk_idx, const int32_t* n_sel, const float* dgate,
+                    float aux_scale, float* dwg, float* dbias, void* dx, int dx_accumulate, void* bws,
+                    size_t bws_bytes, void* stream) {
   int rc = validate(cfg);
   if (rc) return rc;
   if (cfg->seq_len > 0)
@@ -424,6 +433,7 @@ int moe_balance_loss_backward(const moe_config_t* cfg, const void* x, const void
   if ((uintptr_t)bws & 255u) return fail(MOE_ERR_INVALID_ARG, "bws must be 256-byte aligned");
   if (bws_bytes < moe_backward_workspace_size(cfg))
     return fail(MOE_ERR_WORKSPACE, "bws_bytes=%zu < %zu", bws_bytes, moe_backward_workspace_size(cfg));
+  if (dx_accumulate && !dx) return fail(MOE_ERR_INVALID_ARG, "dx_accumulate needs dx");
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
   if (cfg->T == 0) {
@@ -436,22 +446,38 @@ int moe_balance_loss_backward(const moe_config_t* cfg, const void* x, const void
   REQUIRE_PTR(counts);
   OPTIONAL_PTR(router_bias);
   OPTIONAL_PTR(dx);
+  if (dgate) {
+    REQUIRE_PTR(topk_idx);
+    OPTIONAL_PTR(n_sel);
+    if (cfg->routing == MOE_ROUTE_RACE && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
+  }
   BalanceGradArgs a{};
   a.x = x; a.wg = wg; a.bias = router_bias; a.counts = counts;
   a.T = cfg->T; a.D = cfg->D; a.E = cfg->E; a.K = cfg->K; a.dtype = cfg->dtype;
-  a.alpha = cfg->alpha; a.scale = grad_scale;
+  a.alpha = cfg->alpha; a.scale = aux_scale;
+  a.dgate = dgate; a.topk_idx = topk_idx; a.n_sel = n_sel; a.Kmax = kmax_of(cfg); a.dx_accumulate = dx_accumulate;
   const BwdLayout BL = bwd_layout(cfg);
   a.dx = dx; a.dwg = dwg; a.dbias = dbias;
   a.dl = ws_at<float>(bws, BL.dl);
   a.db_part = ws_at<float>(bws, BL.db_part);
   a.partials = ws_at<float>(bws, BL.partials);
+  if (router_bwd_pass_fits(cfg->D, cfg->E, cfg->dtype, cfg->T, num_sms_current()))
+    a.pass_grid = router_bwd_pass_grid(cfg->T, num_sms_current(), &a.pass_tpc);
   // 8 tokens per block (one per warp) at a time: enough blocks to keep every SM's memory pipe busy
   int blocks = num_sms_current() * 4;
   if (blocks > kBwdMaxBlocks) blocks = kBwdMaxBlocks;
   const int need = (cfg->T + 7) / 8;
   if (blocks > need) blocks = need;
-  if ((e = launch_balance_grad(a, blocks, s)) != cudaSuccess) return cuda_fail(e, "balance-loss backward kernels");
+  if ((e = launch_balance_grad(a, blocks, s)) != cudaSuccess) return cuda_fail(e, "router backward kernels");
   return ok();
+}
+}  // namespace
+
+int moe_balance_loss_backward(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
+                              const int32_t* counts, float grad_scale, float* dwg, float* dbias, void* dx,
+                              void* bws, size_t bws_bytes, void* stream) {
+  return router_backward(cfg, x, wg, router_bias, counts, nullptr, nullptr, nullptr, grad_scale, dwg, dbias, dx, 0,
+                         bws, bws_bytes, stream);
 }
 
 int moe_expert_frequency(const moe_config_t* cfg, const int32_t* topk_idx, const int32_t* n_sel, int32_t seq_len,
@@ -598,6 +624,75 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
   }
   if ((e = launch_gemm_tc(g, ta, tb, bn, num_sms_current(), s)) != cudaSuccess) return cuda_fail(e, "tcgen05 expert GEMM");
   return ok();
+}
+
+}  // namespace
+
+namespace {
+
+// 3-D fp32 tensor [z, rows, cols] (row-major), boxes of 32 rows x 32 columns (128 bytes, swizzled)
+int make_tmap_f32_3d(CUtensorMap* m, void* base, long long z, long long rows, long long cols, const char* what) {
+  auto fn = encode_fn();
+  if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1), (cuuint64_t)(z > 0 ? z : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 4, (cuuint64_t)(rows * cols * 4)};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "tensor map for %s failed (CUresult %d)", what, (int)r);
+  return MOE_OK;
+}
+
+// One operand of a CTA-pair problem as a 2-D [rows, cols] 16-bit tensor: K-major operands are
+// read in boxes of 64 columns (K) x box_rows rows, MN-major ones in boxes of 64 x 64.
+struct OperandMap { const void* base; long long rows, cols; int box_rows; };
+// The output: 16-bit [rows, cols] in 32-row boxes of 64 columns, or fp32 [z, rows, cols].
+struct OutputMap { void* base; int f32; long long z, rows, cols; };
+
+int launch_pair_problems(const moe_config_t* cfg, GemmArgs& g, const OperandMap* A, const OperandMap* B,
+                         const OutputMap* O, void* ws, cudaStream_t s) {
+  CUtensorMap ta[2], tb[2], to[2];
+  int rc;
+  for (int q = 0; q < 2; ++q) {
+    const int k = q < g.nprob ? q : 0;
+    if ((rc = make_tmap(&ta[q], A[k].base, cfg->dtype, A[k].rows, A[k].cols, A[k].box_rows, "A"))) return rc;
+    if ((rc = make_tmap(&tb[q], B[k].base, cfg->dtype, B[k].rows, B[k].cols, B[k].box_rows, "B"))) return rc;
+    if (O[k].f32) {
+      if ((rc = make_tmap_f32_3d(&to[q], O[k].base, O[k].z, O[k].rows, O[k].cols, "out"))) return rc;
+    } else if ((rc = make_tmap(&to[q], O[k].base, cfg->dtype, O[k].rows, O[k].cols, 32, "out"))) {
+      return rc;
+    }
+  }
+  g.sched_ctr = ws_at<unsigned int>(ws, kWsSchedCtr);
+  g.exit_ctr = ws_at<unsigned int>(ws, kWsExitCtr);
+  g.test = ws_at<const uint32_t>(ws, kWsTestWords);
+  const cudaError_t e = launch_gemm_pair(g, ta, tb, to, 256, num_sms_current(), cfg->gemm_pairs, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tcgen05 CTA-pair GEMM (backward)");
+  return MOE_OK;
+}
+
+// Scratch of the expert backward (bytes from the start of bws).
+struct EbLayout { size_t dout_perm, dz_perm, du_perm, du_sh, dx_perm, dg, partial, total; int dg_stride; };
+EbLayout eb_layout(const moe_config_t* c) {
+  EbLayout L{};
+  const size_t R = (size_t)max_rows(c), T = (size_t)c->T, D = (size_t)c->D, H = (size_t)c->H;
+  const size_t ns = (size_t)c->n_shared, eb = 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += round_up(bytes ? bytes : 1, 256); return o; };
+  L.dout_perm = take(R * D * eb);
+  L.dz_perm = take(R * D * eb);
+  L.du_perm = take(R * H * eb);
+  L.du_sh = take(T * ns * H * eb);
+  L.dx_perm = take(R * D * eb);
+  L.dg_stride = (int)((H + 255) / 256);
+  L.dg = take(R * (size_t)L.dg_stride * 4);
+  size_t cmax = D > H ? D : H;
+  if (ns * H > cmax) cmax = ns * H;
+  const size_t rmax = R > T ? R : T;
+  L.partial = take((size_t)colsum_chunks((long long)rmax) * cmax * 4);
+  L.total = off;
+  return L;
 }
 
 }  // namespace
@@ -773,6 +868,216 @@ int moe_expert_mlp(const moe_config_t* cfg, const int32_t* offsets, const void* 
   if (rc) return rc;
   return moe_expert_gemm2(cfg, offsets, h_perm, h_sh, w2, b2, w2s, b2s, row_gate, y_perm, y_sh, ws, ws_bytes,
                           stream);
+}
+
+size_t moe_expert_backward_workspace_size(const moe_config_t* cfg) {
+  if (validate(cfg) != MOE_OK) return 0;
+  return eb_layout(cfg).total;
+}
+
+int moe_expert_backward(const moe_config_t* cfg, const void* x, const void* x_perm, const int32_t* offsets,
+                        const int32_t* pos, const int32_t* topk_idx, const int32_t* n_sel, const int32_t* row_token,
+                        const float* row_gate, const moe_expert_weights_t* wts, const void* h_perm, const void* h_sh,
+                        const void* dout, const moe_expert_grads_t* grads, float* dgate, void* dx, void* ws,
+                        size_t ws_bytes, void* bws, size_t bws_bytes, void* stream) {
+  int rc = validate(cfg);
+  if (rc) return rc;
+  if (!is16(cfg) || cfg->gemm_impl != MOE_GEMM_AUTO)
+    return fail(MOE_ERR_UNSUPPORTED, "the expert backward runs on the CTA-pair tensor-core GEMM: bf16 or fp16 with "
+                                     "gemm_impl AUTO");
+  if (cfg->act != 0) return fail(MOE_ERR_UNSUPPORTED, "the expert backward covers the tanh-form GELU (act = 0)");
+  if (!wts || !grads) return fail(MOE_ERR_INVALID_ARG, "wts and grads must be given");
+  if ((rc = check_ws(cfg, ws, ws_bytes))) return rc;
+  if (!bws) return fail(MOE_ERR_INVALID_ARG, "bws is NULL");
+  if ((uintptr_t)bws & 255u) return fail(MOE_ERR_INVALID_ARG, "bws must be 256-byte aligned");
+  const EbLayout L = eb_layout(cfg);
+  if (bws_bytes < L.total) return fail(MOE_ERR_WORKSPACE, "bws_bytes=%zu < %zu", bws_bytes, L.total);
+  const int ns = cfg->n_shared;
+  REQUIRE_PTR(grads->dw1);
+  REQUIRE_PTR(grads->dw2);
+  OPTIONAL_PTR(grads->db1);
+  OPTIONAL_PTR(grads->db2);
+  if (ns > 0) {
+    REQUIRE_PTR(grads->dws1);
+    REQUIRE_PTR(grads->dws2);
+    OPTIONAL_PTR(grads->dbs1);
+    OPTIONAL_PTR(grads->dbs2);
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  const long long T = cfg->T, D = cfg->D, H = cfg->H, E = cfg->E, R = max_rows(cfg);
+  if (T == 0) {   // no token: zero gradients
+    struct { float* p; size_t n; } z[] = {{grads->dw1, (size_t)(E * H * D)}, {grads->db1, (size_t)(E * H)},
+                                          {grads->dw2, (size_t)(E * D * H)}, {grads->db2, (size_t)(E * D)},
+                                          {grads->dws1, (size_t)(ns * H * D)}, {grads->dbs1, (size_t)(ns * H)},
+                                          {grads->dws2, (size_t)(ns * D * H)}, {grads->dbs2, (size_t)(ns * D)}};
+    for (auto& q : z)
+      if (q.p && q.n && (e = cudaMemsetAsync(q.p, 0, q.n * 4, s)) != cudaSuccess) return cuda_fail(e, "moe_expert_backward");
+    return ok();
+  }
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(x_perm);
+  REQUIRE_PTR(offsets);
+  REQUIRE_PTR(pos);
+  REQUIRE_PTR(topk_idx);
+  OPTIONAL_PTR(n_sel);
+  REQUIRE_PTR(row_token);
+  REQUIRE_PTR(row_gate);
+  REQUIRE_PTR(wts->w1);
+  REQUIRE_PTR(wts->w2);
+  OPTIONAL_PTR(wts->b1);
+  OPTIONAL_PTR(wts->b2);
+  REQUIRE_PTR(h_perm);
+  REQUIRE_PTR(dout);
+  REQUIRE_PTR(dgate);
+  REQUIRE_PTR(dx);
+  if (ns > 0) {
+    REQUIRE_PTR(wts->w1s);
+    REQUIRE_PTR(wts->w2s);
+    OPTIONAL_PTR(wts->b1s);
+    REQUIRE_PTR(h_sh);
+  }
+  if (cfg->routing == MOE_ROUTE_RACE && !n_sel) return fail(MOE_ERR_INVALID_ARG, "n_sel is required for Expert-Race routing");
+  const int f16 = cfg->dtype == MOE_F16;
+  const int kmax = kmax_of(cfg);
+  uint8_t* b = static_cast<uint8_t*>(bws);
+  void* dout_perm = b + L.dout_perm;
+  void* dz_perm = b + L.dz_perm;
+  void* du_perm = b + L.du_perm;
+  void* du_sh = b + L.du_sh;
+  void* dx_perm = b + L.dx_perm;
+  float* dg = reinterpret_cast<float*>(b + L.dg);
+  float* partial = reinterpret_cast<float*>(b + L.partial);
+  int* status = status_ptr(ws);
+
+  // 1. dY in permuted order, as given and times the row's gate
+  ExpertBwdArgs ea{};
+  ea.dout = dout; ea.row_token = row_token; ea.row_gate = row_gate; ea.rows = R;
+  ea.T = (int)T; ea.D = (int)D; ea.E = (int)E; ea.K = cfg->K; ea.Kmax = kmax; ea.f16 = f16;
+  ea.dout_perm = dout_perm; ea.dz_perm = dz_perm;
+  ea.pos = pos; ea.topk_idx = topk_idx; ea.n_sel = n_sel; ea.dg = dg; ea.dg_stride = L.dg_stride;
+  ea.b2 = wts->b2; ea.dgate = dgate;
+  if ((e = launch_bwd_gather(ea, s)) != cudaSuccess) return cuda_fail(e, "backward gather");
+
+  auto base_args = [&](int nprob) {
+    GemmArgs g{};
+    g.offsets = offsets; g.E = (int)E; g.r_max = R; g.act = 0; g.status = status;
+    g.b16 = 1; g.f16 = f16; g.nprob = nprob;
+    return g;
+  };
+  const int np = ns > 0 ? 2 : 1;
+  // 2. the pre-activations again: u = x W1^T + b1 (routed rows and shared block), into the dU buffers
+  {
+    GemmArgs g = base_args(np);
+    GemmProblem& p0 = g.p[0];
+    p0.routed = 1; p0.N = (int)H; p0.K = (int)D; p0.epi = 1; p0.out = du_perm; p0.ld_out = H;
+    p0.bias = wts->b1; p0.bias_stride = H; p0.bias_rows = 1;
+    GemmProblem& p1 = g.p[1];
+    if (ns > 0) {
+      p1.routed = 0; p1.M = (int)T; p1.N = ns * (int)H; p1.K = (int)D; p1.epi = 1; p1.out = du_sh;
+      p1.ld_out = ns * H; p1.bias = wts->b1s; p1.bias_stride = 0; p1.bias_rows = 1;
+    }
+    const OperandMap A[2] = {{x_perm, R, D, 128}, {x, T, D, 128}};
+    const OperandMap B[2] = {{wts->w1, E * H, D, 128}, {wts->w1s, (long long)ns * H, D, 128}};
+    const OutputMap O[2] = {{du_perm, 0, 1, R, H}, {du_sh, 0, 1, T, (long long)ns * H}};
+    if ((rc = launch_pair_problems(cfg, g, A, B, O, ws, s))) return rc;
+  }
+  // 3. dU = gate * (dY W2) * gelu'(u), written over u; the row dots sum (dY W2) gelu(u) per column
+  //    tile give the gates' gradient
+  {
+    GemmArgs g = base_args(np);
+    GemmProblem& p0 = g.p[0];
+    p0.routed = 1; p0.N = (int)H; p0.K = (int)D; p0.epi = 4; p0.out = du_perm; p0.ld_out = H;
+    p0.b_mn = 1; p0.aux = du_perm; p0.gate = row_gate; p0.dg = dg; p0.dg_stride = L.dg_stride;
+    GemmProblem& p1 = g.p[1];
+    if (ns > 0) {
+      p1.routed = 0; p1.M = (int)T; p1.N = ns * (int)H; p1.K = (int)D; p1.epi = 4; p1.out = du_sh;
+      p1.ld_out = ns * H; p1.b_mn = 1; p1.b_split = (int)H; p1.aux = du_sh;
+    }
+    const OperandMap A[2] = {{dout_perm, R, D, 128}, {dout, T, D, 128}};
+    const OperandMap B[2] = {{wts->w2, E * D, H, 64}, {wts->w2s, (long long)ns * D, H, 64}};
+    const OutputMap O[2] = {{du_perm, 0, 1, R, H}, {du_sh, 0, 1, T, (long long)ns * H}};
+    if ((rc = launch_pair_problems(cfg, g, A, B, O, ws, s))) return rc;
+  }
+  // 4. dx = sum over the token's slots of (dU W1)[pos] + dU_sh W1s (combine folded into the shared tiles)
+  {
+    GemmArgs g = base_args(np);
+    GemmProblem& p0 = g.p[0];
+    p0.routed = 1; p0.N = (int)D; p0.K = (int)H; p0.epi = 1; p0.out = dx_perm; p0.ld_out = D; p0.b_mn = 1;
+    p0.bias_rows = 1;
+    GemmProblem& p1 = g.p[1];
+    if (ns > 0) {
+      p1.routed = 0; p1.M = (int)T; p1.N = (int)D; p1.K = ns * (int)H; p1.epi = 2; p1.out = dx; p1.ld_out = D;
+      p1.b_mn = 1; p1.bias_rows = 1;
+      g.pos = pos; g.n_sel = n_sel; g.kmax = kmax; g.kdef = cfg->K;
+      g.y_routed = dx_perm;
+      g.done_ctr = ws_at<unsigned int>(ws, kWsDoneCtr);
+    }
+    const OperandMap A[2] = {{du_perm, R, H, 128}, {du_sh, T, (long long)ns * H, 128}};
+    const OperandMap B[2] = {{wts->w1, E * H, D, 64}, {wts->w1s, (long long)ns * H, D, 64}};
+    const OutputMap O[2] = {{dx_perm, 0, 1, R, D}, {dx, 0, 1, T, D}};
+    if ((rc = launch_pair_problems(cfg, g, A, B, O, ws, s))) return rc;
+    if (ns == 0) {
+      CombineArgs ca{};
+      ca.y_perm = dx_perm; ca.y_sh = nullptr; ca.pos = pos; ca.n_sel = n_sel; ca.out = dx; ca.b16 = 1; ca.f16 = f16;
+      ca.T = (int)T; ca.D = (int)D; ca.K = cfg->K; ca.Kmax = kmax; ca.r_max = R;
+      if ((e = launch_combine(ca, s)) != cudaSuccess) return cuda_fail(e, "backward combine");
+    }
+  }
+  // 5. dW2 = sum over the expert's rows of (g dY)^T h; dW2s_j = dY^T h_sh_j
+  {
+    GemmArgs g = base_args(np);
+    GemmProblem& p0 = g.p[0];
+    p0.routed = 1; p0.kgrouped = 1; p0.M = (int)D; p0.N = (int)H; p0.K = 0; p0.a_mn = 1; p0.b_mn = 1;
+    p0.out_f32 = 1; p0.out = grads->dw2;
+    GemmProblem& p1 = g.p[1];
+    if (ns > 0) {
+      p1.routed = 0; p1.kgrouped = 1; p1.M = (int)D; p1.N = ns * (int)H; p1.K = (int)T; p1.a_mn = 1; p1.b_mn = 1;
+      p1.out_f32 = 1; p1.out_split = (int)H; p1.out = grads->dws2;
+    }
+    const OperandMap A[2] = {{dz_perm, R, D, 64}, {dout, T, D, 64}};
+    const OperandMap B[2] = {{h_perm, R, H, 64}, {h_sh, T, (long long)ns * H, 64}};
+    const OutputMap O[2] = {{grads->dw2, 1, E, D, H}, {grads->dws2, 1, ns, D, H}};
+    if ((rc = launch_pair_problems(cfg, g, A, B, O, ws, s))) return rc;
+  }
+  // 6. dW1 = sum over the expert's rows of dU^T x_perm; dW1s = dU_sh^T x
+  {
+    GemmArgs g = base_args(np);
+    GemmProblem& p0 = g.p[0];
+    p0.routed = 1; p0.kgrouped = 1; p0.M = (int)H; p0.N = (int)D; p0.K = 0; p0.a_mn = 1; p0.b_mn = 1;
+    p0.out_f32 = 1; p0.out = grads->dw1;
+    GemmProblem& p1 = g.p[1];
+    if (ns > 0) {
+      p1.routed = 0; p1.kgrouped = 1; p1.M = ns * (int)H; p1.N = (int)D; p1.K = (int)T; p1.a_mn = 1; p1.b_mn = 1;
+      p1.out_f32 = 1; p1.out = grads->dws1;
+    }
+    const OperandMap A[2] = {{du_perm, R, H, 64}, {du_sh, T, (long long)ns * H, 64}};
+    const OperandMap B[2] = {{x_perm, R, D, 64}, {x, T, D, 64}};
+    const OutputMap O[2] = {{grads->dw1, 1, E, H, D}, {grads->dws1, 1, 1, (long long)ns * H, D}};
+    if ((rc = launch_pair_problems(cfg, g, A, B, O, ws, s))) return rc;
+  }
+  // 7. bias gradients: column sums of g dY and dU over each expert's rows, of dY and dU_sh over all tokens
+  if (grads->db2 && (e = launch_colsum(dz_perm, R, (int)D, offsets, (int)E, 1, partial, grads->db2, f16, s)) != cudaSuccess)
+    return cuda_fail(e, "db2 column sums");
+  if (grads->db1 && (e = launch_colsum(du_perm, R, (int)H, offsets, (int)E, 1, partial, grads->db1, f16, s)) != cudaSuccess)
+    return cuda_fail(e, "db1 column sums");
+  if (ns > 0 && grads->dbs2 &&
+      (e = launch_colsum(dout, T, (int)D, nullptr, 1, ns, partial, grads->dbs2, f16, s)) != cudaSuccess)
+    return cuda_fail(e, "dbs2 column sums");
+  if (ns > 0 && grads->dbs1 &&
+      (e = launch_colsum(du_sh, T, ns * (int)H, nullptr, 1, 1, partial, grads->dbs1, f16, s)) != cudaSuccess)
+    return cuda_fail(e, "dbs1 column sums");
+  // 8. the gates' gradient per selected slot
+  if ((e = launch_dgate(ea, s)) != cudaSuccess) return cuda_fail(e, "gate gradient");
+  return ok();
+}
+
+int moe_router_backward(const moe_config_t* cfg, const void* x, const void* wg, const float* router_bias,
+                        const int32_t* counts, const int32_t* topk_idx, const int32_t* n_sel, const float* dgate,
+                        float aux_scale, float* dwg, float* dbias, void* dx, int32_t dx_accumulate, void* bws,
+                        size_t bws_bytes, void* stream) {
+  return router_backward(cfg, x, wg, router_bias, counts, topk_idx, n_sel, dgate, aux_scale, dwg, dbias, dx,
+                         dx_accumulate, bws, bws_bytes, stream);
 }
 
 int moe_combine(const moe_config_t* cfg, const void* y_perm, const void* y_sh,

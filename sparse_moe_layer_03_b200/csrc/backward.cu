@@ -1,20 +1,22 @@
-// Backward of the expert-level balance loss through the router
-// ("Scaling Diffusion Transformers to 16 Billion Parameters", "MOE-DIT",
-// eq. L_balance).  L = alpha sum_i f_i p_i with f_i = (E/(K T)) counts_i from
-// the discrete selection (no gradient) and p_i = (1/T) sum_t P[t,i], so
-// dL/dP[t,i] = alpha f_i / T = c_i for every token, and through the softmax
-//     dl[t,i] = P[t,i] (c_i - sum_j P[t,j] c_j).
-// The router's linear map l = x Wg^T + b then gives dWg = dl^T x, db = sum_t dl
+// Backward of the router: the expert-level balance loss ("Scaling Diffusion
+// Transformers to 16 Billion Parameters", "MOE-DIT", eq. L_balance) and, for the
+// whole layer's backward, the gates' gradient.  L = alpha sum_i f_i p_i with
+// f_i = (E/(K T)) counts_i from the discrete selection (no gradient) and
+// p_i = (1/T) sum_t P[t,i], so dL/dP[t,i] = alpha f_i / T = c_i for every token;
+// the gates g = P on the selected slots add dgate there.  Through the softmax
+//     dl[t,i] = P[t,i] (dP[t,i] - sum_j P[t,j] dP[t,j]),
+// and the router's linear map l = x Wg^T + b gives dWg = dl^T x, db = sum_t dl
 // and dx = dl Wg.
 //
-// token kernel (one warp per token, the gate weight in shared memory): the row
-//   of x in 16-byte vectors, E partial dot products per lane and a fixed xor
-//   tree, softmax and dl (every lane), the dx row, dl written out, and the
-//   block's db partial (warps in a fixed order).
-// wgrad kernel: blocks over (chunk of kWgTokens tokens, 512 columns); each
-//   thread owns 2 columns x E experts and walks its chunk's tokens in order.
-// reduce kernel: the chunk partials of dWg and the block partials of db,
-//   summed in order.  Every sum has a fixed order: bit-reproducible.
+// One pass kernel (rows of at most 2048 16-bit or 1024 fp32 values): CTA b owns
+// a contiguous range of tokens.  Phase 1, one warp per token (the next token's
+// row already loading into registers): logits from the gate weight in shared
+// memory, a fixed xor tree, softmax and dl in every lane, the dx row written
+// (added to the experts' part when asked), dl kept in shared memory.  Phase 2,
+// each thread owns 8 (or 4) columns and adds dl^T x over the CTA's tokens in
+// order (x read again, from L2), giving the CTA's partial dWg.
+// Wider rows use the older three-kernel path (token kernel, chunked wgrad).
+// A reduce kernel sums the partials of dWg and db in order: bit-reproducible.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -103,13 +105,26 @@ __global__ void __launch_bounds__(kBwdThreads) balance_grad_token_kernel(Balance
     for (int e = 0; e < EMAX; ++e)
       if (e < E) { l[e] = expf(l[e] - m); z += l[e]; }
     const float iz = 1.0f / z;
+    // dJ/dP: the balance term c_i on every entry, plus the gates' gradient on the selected slots
+    float dp[EMAX];
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) dp[e] = c_s[e];
+    if (a.dgate) {
+      const int ns = a.n_sel ? a.n_sel[t] : a.K;
+      for (int k = 0; k < a.Kmax && k < ns; ++k) {
+        const int sel = a.topk_idx[(size_t)t * a.Kmax + k];
+        const float gk = a.dgate[(size_t)t * a.Kmax + k];
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) dp[e] += e == sel ? gk : 0.f;
+      }
+    }
     float pc = 0.f;
 #pragma unroll
     for (int e = 0; e < EMAX; ++e)
-      if (e < E) { l[e] *= iz; pc += l[e] * c_s[e]; }
+      if (e < E) { l[e] *= iz; pc += l[e] * dp[e]; }
 #pragma unroll
     for (int e = 0; e < EMAX; ++e) {
-      l[e] = e < E ? l[e] * (c_s[e] - pc) : 0.f;      // dl
+      l[e] = e < E ? l[e] * (dp[e] - pc) : 0.f;       // dl
       dbw[e] += l[e];
     }
     if (lane < E) {
@@ -124,6 +139,7 @@ __global__ void __launch_bounds__(kBwdThreads) balance_grad_token_kernel(Balance
         float o[V::N];
 #pragma unroll
         for (int q = 0; q < V::N; ++q) o[q] = 0.f;
+        if (a.dx_accumulate) V::to_f(dxr[v], o);       // the experts' part of dx, then the router's
 #pragma unroll
         for (int e = 0; e < EMAX; ++e) {
           if (e < E) {
@@ -198,24 +214,218 @@ __global__ void __launch_bounds__(kBwdThreads) balance_grad_wg_kernel(BalanceGra
   }
 }
 
-// Fixed-order sums of the partials: eight interleaved running sums (partial p goes to sum
-// p % 8), added up in order at the end, so eight loads are in flight per thread.
-__device__ __forceinline__ float sum_strided(const float* p, int n, size_t stride) {
-  float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  int k = 0;
-  for (; k + 8 <= n; k += 8) {
-#pragma unroll
-    for (int u = 0; u < 8; ++u) s[u] += __ldcg(p + (size_t)(k + u) * stride);
+constexpr int kRbThreads = 256;
+constexpr int kRbMaxV = 8;                         // 16-byte vectors per lane and row (D <= 2048 16-bit)
+
+template <typename T, int EMAX>
+__global__ void __launch_bounds__(kRbThreads, 2) router_bwd_pass_kernel(BalanceGradArgs a, int tpc) {
+  using V = Vec16<T>;
+  constexpr int NW = kRbThreads / 32;
+  extern __shared__ __align__(16) uint8_t rsm[];    // gate weight [E, D] act, then dl [tpc, EMAX] fp32
+  __shared__ float c_s[EMAX];
+  __shared__ float wdb[NW][EMAX];
+  const int D = a.D, E = a.E, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int nv = D / V::N;
+  const int t0 = blockIdx.x * tpc, t1 = min(a.T, t0 + tpc);
+  float* dls = reinterpret_cast<float*>(rsm + (size_t)E * D * sizeof(T));
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.wg);
+    uint4* dst = reinterpret_cast<uint4*>(rsm);
+    for (int i = tid; i < E * nv; i += kRbThreads) dst[i] = __ldg(src + i);
   }
-  for (int u = 0; k < n; ++k, ++u) s[u] += __ldcg(p + (size_t)k * stride);
-  return ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+  if (tid < EMAX)
+    c_s[tid] = tid < E ? a.scale * a.alpha * ((float)E / ((float)a.K * a.T)) * (float)a.counts[tid] / (float)a.T : 0.f;
+  __syncthreads();
+  const uint4* wv = reinterpret_cast<const uint4*>(rsm);
+  const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+  float dbw[EMAX];
+#pragma unroll
+  for (int e = 0; e < EMAX; ++e) dbw[e] = 0.f;
+  // ---- phase 1: one warp per token
+  uint4 cur[kRbMaxV], nxt[kRbMaxV];
+  int t = t0 + w;
+  if (t < t1) {
+#pragma unroll
+    for (int k = 0; k < kRbMaxV; ++k) {
+      const int v = lane + 32 * k;
+      if (v < nv) cur[k] = __ldg(xv + (size_t)t * nv + v);
+    }
+  }
+  for (; t < t1; t += NW) {
+    const int tn = t + NW;
+    if (tn < t1) {                                   // the next row loads while this one is worked on
+#pragma unroll
+      for (int k = 0; k < kRbMaxV; ++k) {
+        const int v = lane + 32 * k;
+        if (v < nv) nxt[k] = __ldg(xv + (size_t)tn * nv + v);
+      }
+    }
+    float l[EMAX];
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) l[e] = 0.f;
+#pragma unroll
+    for (int k = 0; k < kRbMaxV; ++k) {
+      const int v = lane + 32 * k;
+      if (v < nv) {
+        float xf[V::N];
+        V::to_f(cur[k], xf);
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) {
+          if (e < E) {
+            float wf[V::N];
+            V::to_f(wv[e * nv + v], wf);
+#pragma unroll
+            for (int q = 0; q < V::N; ++q) l[e] = fmaf(xf[q], wf[q], l[e]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l[e] += __shfl_xor_sync(0xffffffffu, l[e], o);
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e)
+      if (e < E) { l[e] += a.bias ? a.bias[e] : 0.f; m = fmaxf(m, l[e]); }
+    float z = 0.f;
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e)
+      if (e < E) { l[e] = expf(l[e] - m); z += l[e]; }
+    const float iz = 1.0f / z;
+    float dp[EMAX];
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) dp[e] = c_s[e];
+    if (a.dgate) {
+      const int ns = a.n_sel ? a.n_sel[t] : a.K;
+      for (int k = 0; k < a.Kmax && k < ns; ++k) {
+        const int sel = a.topk_idx[(size_t)t * a.Kmax + k];
+        const float gk = a.dgate[(size_t)t * a.Kmax + k];
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) dp[e] += e == sel ? gk : 0.f;
+      }
+    }
+    float pc = 0.f;
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e)
+      if (e < E) { l[e] *= iz; pc += l[e] * dp[e]; }
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) {
+      l[e] = e < E ? l[e] * (dp[e] - pc) : 0.f;       // dl
+      dbw[e] += l[e];
+    }
+    if (lane < EMAX) {
+      float v = 0.f;
+#pragma unroll
+      for (int e = 0; e < EMAX; ++e) v = e == lane ? l[e] : v;
+      dls[(size_t)(t - t0) * EMAX + lane] = v;
+    }
+    if (a.dx) {
+      uint4* dxr = reinterpret_cast<uint4*>(a.dx) + (size_t)t * nv;
+#pragma unroll
+      for (int k = 0; k < kRbMaxV; ++k) {
+        const int v = lane + 32 * k;
+        if (v < nv) {
+          float o[V::N];
+#pragma unroll
+          for (int q = 0; q < V::N; ++q) o[q] = 0.f;
+          if (a.dx_accumulate) V::to_f(dxr[v], o);
+#pragma unroll
+          for (int e = 0; e < EMAX; ++e) {
+            if (e < E) {
+              float wf[V::N];
+              V::to_f(wv[e * nv + v], wf);
+#pragma unroll
+              for (int q = 0; q < V::N; ++q) o[q] = fmaf(l[e], wf[q], o[q]);
+            }
+          }
+          dxr[v] = V::from_f(o);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kRbMaxV; ++k) cur[k] = nxt[k];
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int e = 0; e < EMAX; ++e) wdb[w][e] = dbw[e];
+  }
+  __syncthreads();
+  if (tid < E) {
+    float sdb = 0.f;
+    for (int k = 0; k < NW; ++k) sdb += wdb[k][tid];
+    a.db_part[(size_t)blockIdx.x * E + tid] = sdb;
+  }
+  // ---- phase 2: this CTA's dWg partial, column vector v of every expert over the CTA's tokens
+  const int ntok = t1 - t0;
+  float* part = a.partials + (size_t)blockIdx.x * E * D;
+  for (int v = tid; v < nv; v += kRbThreads) {
+    for (int e0 = 0; e0 < E; e0 += 8) {
+      float acc[8][V::N];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int q = 0; q < V::N; ++q) acc[j][q] = 0.f;
+      // eight rows in flight per thread, then their products in token order
+      for (int tb = 0; tb < ntok; tb += 8) {
+        uint4 xr[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (tb + u < ntok) xr[u] = __ldg(xv + (size_t)(t0 + tb + u) * nv + v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (tb + u < ntok) {
+            float xf[V::N];
+            V::to_f(xr[u], xf);
+            const float* dr = dls + (size_t)(tb + u) * EMAX + e0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float d = dr[j];
+#pragma unroll
+              for (int q = 0; q < V::N; ++q) acc[j][q] = fmaf(d, xf[q], acc[j][q]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (e0 + j < E) {
+#pragma unroll
+          for (int q = 0; q < V::N; ++q) part[(size_t)(e0 + j) * D + v * V::N + q] = acc[j][q];
+        }
+    }
+  }
 }
 
+// Block b sums elements [32 b, 32 b + 32) of [dWg, db]: lane = element, warp w takes the partials
+// p = w, w + 8, ... in order (eight loads in flight per lane), then the eight warp sums are added
+// in warp order.  A fixed order throughout.
 __global__ void __launch_bounds__(kBwdThreads) balance_grad_reduce_kernel(BalanceGradArgs a, int nchunks, int nblocks) {
+  constexpr int NW = kBwdThreads / 32;
+  __shared__ float ws[NW][32];
   const int n = a.E * a.D;
-  for (int i = blockIdx.x * kBwdThreads + threadIdx.x; i < n + a.E; i += gridDim.x * kBwdThreads) {
-    if (i < n) a.dwg[i] = sum_strided(a.partials + i, nchunks, (size_t)n);
-    else if (a.dbias) a.dbias[i - n] = sum_strided(a.db_part + (i - n), nblocks, (size_t)a.E);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int i = blockIdx.x * 32 + lane;
+  float s = 0.f;
+  if (i < n + a.E) {
+    const bool wg = i < n;
+    const float* p = wg ? a.partials + i : a.db_part + (i - n);
+    const size_t stride = wg ? (size_t)n : (size_t)a.E;
+    const int cnt = wg ? nchunks : nblocks;
+    float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int k = w, u = 0;
+    for (; k < cnt; k += NW, u = (u + 1) & 7) r[u] += __ldcg(p + (size_t)k * stride);
+    s = ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
+  }
+  ws[w][lane] = s;
+  __syncthreads();
+  if (w == 0 && i < n + a.E) {
+    float t = 0.f;
+#pragma unroll
+    for (int k = 0; k < NW; ++k) t += ws[k][lane];
+    if (i < n) a.dwg[i] = t;
+    else if (a.dbias) a.dbias[i - n] = t;
   }
 }
 
@@ -241,14 +451,59 @@ static cudaError_t launch_bg_t(const BalanceGradArgs& a, int blocks, cudaStream_
   return launch_bg<T, 32>(a, blocks, s);
 }
 
+template <typename T, int EM>
+static cudaError_t launch_rb(const BalanceGradArgs& a, int grid, int tpc, cudaStream_t s) {
+  const size_t smem = (size_t)a.E * a.D * sizeof(T) + (size_t)tpc * EM * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(router_bwd_pass_kernel<T, EM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  router_bwd_pass_kernel<T, EM><<<grid, kRbThreads, smem, s>>>(a, tpc);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_rb_t(const BalanceGradArgs& a, int grid, int tpc, cudaStream_t s) {
+  if (a.E <= 8) return launch_rb<T, 8>(a, grid, tpc, s);
+  if (a.E <= 16) return launch_rb<T, 16>(a, grid, tpc, s);
+  return launch_rb<T, 32>(a, grid, tpc, s);
+}
+
+int router_bwd_pass_grid(int T, int sms, int* tpc) {
+  int g = 2 * sms;                                 // two CTAs per SM
+  if (g > kBwdMaxBlocks) g = kBwdMaxBlocks;
+  if (g > T) g = T > 0 ? T : 1;
+  const int per = (T + g - 1) / g;
+  *tpc = per > 0 ? per : 1;
+  return (T + *tpc - 1) / *tpc;
+}
+
+bool router_bwd_pass_fits(int D, int E, int dtype, int T, int sms) {
+  const int vec = dtype == 0 ? 4 : 8;
+  if (D % vec || D / vec > 32 * kRbMaxV) return false;
+  int tpc = 0;
+  router_bwd_pass_grid(T, sms, &tpc);
+  const int em = E <= 8 ? 8 : (E <= 16 ? 16 : 32);
+  const size_t smem = (size_t)E * D * (dtype == 0 ? 4 : 2) + (size_t)tpc * em * 4;
+  return smem <= 232448 / 2 - 2048;               // two CTAs per SM
+}
+
 cudaError_t launch_balance_grad(const BalanceGradArgs& a, int blocks, cudaStream_t s) {
-  cudaError_t e = a.dtype == 0 ? launch_bg_t<float>(a, blocks, s)
-                  : a.dtype == 2 ? launch_bg_t<__half>(a, blocks, s)
-                                 : launch_bg_t<__nv_bfloat16>(a, blocks, s);
+  cudaError_t e;
+  int nparts = blocks, nchunks = balance_grad_chunks(a.T);
+  if (a.pass_grid > 0) {
+    // one pass: partials of dWg and db per CTA
+    e = a.dtype == 0 ? launch_rb_t<float>(a, a.pass_grid, a.pass_tpc, s)
+        : a.dtype == 2 ? launch_rb_t<__half>(a, a.pass_grid, a.pass_tpc, s)
+                       : launch_rb_t<__nv_bfloat16>(a, a.pass_grid, a.pass_tpc, s);
+    nparts = nchunks = a.pass_grid;
+  } else {
+    e = a.dtype == 0 ? launch_bg_t<float>(a, blocks, s)
+        : a.dtype == 2 ? launch_bg_t<__half>(a, blocks, s)
+                       : launch_bg_t<__nv_bfloat16>(a, blocks, s);
+  }
   if (e != cudaSuccess) return e;
   const int n = a.E * a.D + a.E;
-  balance_grad_reduce_kernel<<<(n + kBwdThreads - 1) / kBwdThreads, kBwdThreads, 0, s>>>(
-      a, balance_grad_chunks(a.T), blocks);
+  balance_grad_reduce_kernel<<<(n + 31) / 32, kBwdThreads, 0, s>>>(a, nchunks, nparts);
   return cudaGetLastError();
 }
 

@@ -255,6 +255,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
   return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
+// The same descriptor for an MN-major operand tile of 128-byte swizzled rows, each row holding 64
+// consecutive M (or N) elements of one k: 8-row groups 1024 B apart (stride byte offset), and the
+// next 64 M (or N) elements in the block 8 KB further on (leading byte offset).  One k16 step of
+// the MMA is 16 rows, 2048 B.
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t addr) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(8192 >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
 // Instruction descriptor, kind::f16: D fp32, A and B of one 16-bit type, both K-major.
 //   bits 4-5 D format (1 = f32), 7-9 A format (0 = f16, 1 = bf16), 10-12 B format,
 //   15/16 A/B major (0 = K), 17-22 N >> 3, 24-28 M >> 4.
@@ -262,6 +270,20 @@ __host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, uint32_t 
   return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) { return idesc_f16kind_f32(M, N, 1u); }
+// bits 15 / 16: A / B MN-major (transposed)
+__host__ __device__ constexpr uint32_t idesc_major_bits(int a_mn, int b_mn) {
+  return ((uint32_t)(a_mn ? 1 : 0) << 15) | ((uint32_t)(b_mn ? 1 : 0) << 16);
+}
+// derivative of the tanh-form GELU: 0.5 (1 + t) + 0.5 u (1 - t^2) c (1 + 3 k u^2),
+// t = tanh(c (u + k u^3)), c = sqrt(2/pi), k = 0.044715; FAST uses tanh.approx.f32
+template <bool FAST>
+__device__ __forceinline__ void gelu_tanh_and_grad(float u, float& g, float& dg) {
+  const float c = 0.7978845608028654f, k = 0.044715f;
+  const float u2 = u * u;
+  const float t = FAST ? tanh_hw(c * (u + k * u2 * u)) : tanhf(c * (u + k * u2 * u));
+  g = 0.5f * u * (1.0f + t);
+  dg = 0.5f * (1.0f + t) + 0.5f * u * (1.0f - t * t) * c * (1.0f + 3.0f * k * u2);
+}
 
 // ---------------------------------------------------------------- CTA pairs (clusters of 2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {

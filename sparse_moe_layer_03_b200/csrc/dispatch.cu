@@ -17,7 +17,10 @@
 //                 rows (group base + rank) and writes pos, row_token and
 //                 row_gate; then one warp per token loads the row and stores
 //                 it once per selected expert with 16-byte vectors (each
-//                 warp's first row loads while the rows are worked out).
+//                 warp's first row loads while the rows are worked out).  Its
+//                 first E blocks write zeros to the padding rows of the E
+//                 segments, so every row of a segment's 256-row tiles holds
+//                 finite values (the weight gradients reduce over them).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -201,11 +204,11 @@ __device__ __forceinline__ void store_row(uint4* dst, int nvec, int lane, const 
 // warp per token: row loads, then one store of the row per selected slot.  Each
 // warp's first row is already loading while phase 1 runs.
 template <typename T, int P>
-__device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos) {
+__device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, int blk) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int Kmax = a.Kmax;
   const int nvec = a.D * (int)sizeof(T) / 16;
-  const int t0 = blockIdx.x * a.tpb;
+  const int t0 = blk * a.tpb;
   const int nt = min(a.tpb, a.T - t0);
   const uint4* xv = reinterpret_cast<const uint4*>(a.x);
   uint4* xp = reinterpret_cast<uint4*>(a.x_perm);
@@ -257,13 +260,33 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos) {
   }
 }
 
+// Zeros on the padding rows [P_e + count_e, P_{e+1}) of segment e of x_perm (offsets from the
+// count kernel).
 template <typename T>
-__global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(DispatchArgs a) {
-  extern __shared__ int spos[];                       // [tpb * Kmax] rows of the block's slots
+__device__ void zero_padding_rows(const DispatchArgs& a, int e) {
   const int nvec = a.D * (int)sizeof(T) / 16;
-  if (nvec <= 4 * 32) gather_block<T, 4>(a, spos);
-  else if (nvec <= 8 * 32) gather_block<T, 8>(a, spos);
-  else gather_block<T, 0>(a, spos);
+  long long p = 0;
+  for (int j = 0; j < e; ++j) p += (a.offsets[j + 1] - a.offsets[j] + kSegAlign - 1) / kSegAlign * kSegAlign;
+  const int c = a.offsets[e + 1] - a.offsets[e];
+  const long long lo = p + c, hi = p + (long long)(c + kSegAlign - 1) / kSegAlign * kSegAlign;
+  if (lo < 0 || hi > a.r_max) return;
+  uint4* xp = reinterpret_cast<uint4*>(a.x_perm);
+  const long long n = (hi - lo) * nvec;
+  for (long long i = threadIdx.x; i < n; i += kDispatchThreads) xp[lo * nvec + i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(DispatchArgs a, int zero_blocks) {
+  extern __shared__ int spos[];                       // [tpb * Kmax] rows of the block's slots
+  if ((int)blockIdx.x < zero_blocks) {
+    zero_padding_rows<T>(a, blockIdx.x);
+    return;
+  }
+  const int blk = blockIdx.x - zero_blocks;
+  const int nvec = a.D * (int)sizeof(T) / 16;
+  if (nvec <= 4 * 32) gather_block<T, 4>(a, spos, blk);
+  else if (nvec <= 8 * 32) gather_block<T, 8>(a, spos, blk);
+  else gather_block<T, 0>(a, spos, blk);
 }
 
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
@@ -273,10 +296,11 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   else dispatch_count_kernel<32><<<cgrid, kDispatchThreads, 0, s>>>(a);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const int ggrid = (a.T + a.tpb - 1) / a.tpb;
+  const int zero_blocks = a.x_perm != nullptr ? a.E : 0;
+  const int ggrid = zero_blocks + (a.T + a.tpb - 1) / a.tpb;
   const size_t smem = (size_t)a.tpb * a.Kmax * sizeof(int);
-  if (a.b16) dispatch_gather_kernel<uint16_t><<<ggrid, kDispatchThreads, smem, s>>>(a);
-  else dispatch_gather_kernel<float><<<ggrid, kDispatchThreads, smem, s>>>(a);
+  if (a.b16) dispatch_gather_kernel<uint16_t><<<ggrid, kDispatchThreads, smem, s>>>(a, zero_blocks);
+  else dispatch_gather_kernel<float><<<ggrid, kDispatchThreads, smem, s>>>(a, zero_blocks);
   return cudaGetLastError();
 }
 

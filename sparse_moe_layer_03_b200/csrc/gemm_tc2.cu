@@ -22,13 +22,17 @@
 // on the leader's "accumulator empty" barrier; both CTAs' TMA loads complete
 // on the leader's "stage full" barrier.  All waits are bounded.
 //
-// Scheduling: persistent pairs claim tiles in increasing order from a counter
-// in global memory (the leader's producer claims one tile ahead and hands each
-// id to the other roles of both CTAs through a small ring in shared memory).
-// Routed tiles are numbered before shared ones, so when the combine is folded
-// into the shared tiles, a shared tile can only wait for routed tiles that
-// resident pairs have already claimed: no wait depends on a pair that is not
-// running, however many pairs the device holds at once.
+// Scheduling: persistent pairs.  Without the folded combine, pair c runs tiles
+// c, c + pairs, c + 2 pairs, ... (consecutive tiles share their A row block and
+// run side by side).  With it, pairs claim tiles in increasing order from a
+// counter in global memory (the leader's producer claims one tile ahead and
+// hands each id to the other roles of both CTAs through a small ring in shared
+// memory).  Routed tiles are numbered before shared ones, so a shared tile can
+// only wait for routed tiles that resident pairs have already claimed: no wait
+// depends on a pair that is not running, however many pairs the device holds
+// at once.  (Bringing the operand boxes of later stages into L2 with TMA
+// prefetches made both GEMMs 1.5x slower: the TMA unit's throughput, not the
+// latency of L2, bounds the loads.)
 #include <cuda.h>
 
 #include <mutex>
@@ -65,6 +69,7 @@ struct PairPlan {
   int poff[33];
   int cnt[32];
   int ntiles[2];
+  int nm[2];          // kgrouped problems: 256-row tiles of each [M, N] output
   int nn[2];          // column tiles per row block: nfull of width BN, then one of width nrem if nrem > 0
   int nfull[2];
   int nrem[2];
@@ -73,6 +78,8 @@ struct PairPlan {
 
 struct PairTile {
   int p, row0, valid, brow, n0, width, e, nk;
+  int k0;             // first K row of the operands held MN-major (rows = K)
+  int bk0;            // first K row of an MN-major B (an expert's block of the weights, or k0)
 };
 
 template <int BN>
@@ -82,6 +89,30 @@ __device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, co
   ti.p = 0;
   if (t >= pl.ntiles[0]) { t -= pl.ntiles[0]; ti.p = 1; }
   const GemmProblem& pr = a.p[ti.p];
+  ti.k0 = 0;
+  ti.bk0 = 0;
+  if (pr.kgrouped) {
+    // weight gradient: tiles of expert e's [M, N] output; the reduction runs over the expert's
+    // rows of the permuted buffers (a dense problem has one segment of K rows)
+    const int per = pl.nm[ti.p] * pl.nn[ti.p];
+    const int e = t / per, r = t % per;
+    const int mt = r / pl.nn[ti.p], nt = r % pl.nn[ti.p];
+    ti.e = e;
+    ti.row0 = mt * kPairBM;
+    ti.n0 = nt * BN;
+    ti.width = nt < pl.nfull[ti.p] ? BN : pl.nrem[ti.p];
+    const int v = pr.M - ti.row0;
+    ti.valid = v < kPairBM ? v : kPairBM;
+    ti.brow = 0;
+    if (pr.routed) {
+      ti.k0 = pl.poff[e];
+      ti.nk = (pl.cnt[e] + kPairBK - 1) / kPairBK;
+    } else {
+      ti.nk = (pr.K + kPairBK - 1) / kPairBK;
+    }
+    ti.bk0 = ti.k0;
+    return ti;
+  }
   const int mt = t / pl.nn[ti.p], nt = t % pl.nn[ti.p];
   ti.row0 = mt * kPairBM;
   ti.n0 = nt * BN;
@@ -94,6 +125,7 @@ __device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, co
     const int v = pl.poff[e] + pl.cnt[e] - ti.row0;
     ti.valid = v < kPairBM ? v : kPairBM;
     ti.brow = e * pr.N + ti.n0;
+    ti.bk0 = e * pr.K;                 // MN-major B: expert e's weights are rows [e K, (e + 1) K)
   } else {
     ti.e = 0;
     const int v = pr.M - ti.row0;
@@ -106,12 +138,13 @@ __device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, co
 // Next tile id of a consumer role (lane 0): wait for the ring slot, read it, and release the
 // slot on the leader.  -1: no tile left (or a wait ran out, recorded in the status word).
 __device__ __forceinline__ int sched_take(uint64_t* sfull, uint64_t* sempty, volatile int* stile, uint32_t& n,
-                                          volatile int* abort_flag, int* status, int where) {
+                                          uint32_t rank, volatile int* abort_flag, int* status, int where) {
   const uint32_t slot = n % kSchedSlots, ph = (n / kSchedSlots) & 1u;
   ++n;
   if (!mbar_wait_cluster(smem_u32(&sfull[slot]), ph, abort_flag, status, where)) return -1;
   const int t = stile[slot];
-  mbar_arrive_release_cluster(map_to_cta(smem_u32(&sempty[slot]), 0));
+  if (rank == 0) mbar_arrive(smem_u32(&sempty[slot]));       // the leader's own roles: CTA scope
+  else mbar_arrive_release_cluster(map_to_cta(smem_u32(&sempty[slot]), 0));
   return t;
 }
 
@@ -159,6 +192,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
 
   const int warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();          // 0 = leader of the pair
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  // tiles claimed in order (the folded combine's guarantee of progress) or a fixed order
+  const bool dyn = a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -188,11 +224,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     }
     if ((long long)p > a.r_max) bad = true;
     for (int q = 0; q < 2; ++q) {
-      if (q >= a.nprob) { pl.ntiles[q] = 0; pl.nn[q] = 1; pl.nfull[q] = 1; pl.nrem[q] = 0; continue; }
+      if (q >= a.nprob) { pl.ntiles[q] = 0; pl.nn[q] = 1; pl.nm[q] = 1; pl.nfull[q] = 1; pl.nrem[q] = 0; continue; }
       const GemmProblem& pr = a.p[q];
       pl.nfull[q] = pr.N / BN;
       pl.nrem[q] = pr.N % BN;
       pl.nn[q] = pl.nfull[q] + (pl.nrem[q] ? 1 : 0);
+      pl.nm[q] = (pr.M + kPairBM - 1) / kPairBM;
+      if (pr.kgrouped) {
+        pl.ntiles[q] = (pr.routed ? (bad ? 0 : a.E) : 1) * pl.nm[q] * pl.nn[q];
+        continue;
+      }
       const int mt = pr.routed ? (bad ? 0 : p / kPairBM) : (pr.M + kPairBM - 1) / kPairBM;
       pl.ntiles[q] = mt * pl.nn[q];
     }
@@ -225,18 +266,23 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     uint32_t phase = 0;
     bool alive = true;
     uint32_t sn = 0;
-    int next = (rank == 0 && lane == 0) ? sched_claim(a.sched_ctr, pl.total) : -1;
+    int next = (dyn && rank == 0 && lane == 0) ? sched_claim(a.sched_ctr, pl.total) : -1;
+    int kstat = 0;                                  // fixed order: this pair's k-th tile is cid + k * ncl
     while (alive) {
       // the leader hands its claimed tile to both CTAs and claims the one after it while the
       // loads go out; the peer takes the tile from its ring
       int tile = -1, ok = 1;
-      if (lane == 0) {
+      if (!dyn) {
+        tile = cid + kstat * ncl;
+        ++kstat;
+        if (tile >= pl.total) tile = -1;
+      } else if (lane == 0) {
         if (rank == 0) {
           tile = next;
           ok = sched_publish(sched_full, sched_empty, sched_tile, sn, tile, abort_flag, a.status) ? 1 : 0;
           if (ok && tile >= 0) next = sched_claim(a.sched_ctr, pl.total);
         } else {
-          tile = sched_take(sched_full, sched_empty, sched_tile, sn, abort_flag, a.status, 508);
+          tile = sched_take(sched_full, sched_empty, sched_tile, sn, rank, abort_flag, a.status, 508);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -274,8 +320,27 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           const int bx = ksplit ? (kb * kPairBK) % ksplit : kb * kPairBK;
           // each CTA holds half of the tile's B rows (a narrower tile's box also brings rows it does not use)
           const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (ti.width / 2);
-          if (!gather) tma_load_2d_pair(smem_u32(sa), tA, kb * kPairBK, ti.row0 + (int)rank * 128, fb_leader, pol_a);
-          tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tB, bx, by, fb_leader, pol_w);
+          if (pr.a_mn) {
+            // A held [K rows, M columns]: this CTA's 128 M columns as two 64-column boxes of 64 K rows
+            const int ax = ti.row0 + (int)rank * 128, ay = ti.k0 + kb * kPairBK;
+            tma_load_2d_pair(smem_u32(sa), tA, ax, ay, fb_leader, pol_a);
+            tma_load_2d_pair(smem_u32(sa) + 8192, tA, ax + 64, ay, fb_leader, pol_a);
+          } else if (!gather) {
+            tma_load_2d_pair(smem_u32(sa), tA, kb * kPairBK, ti.row0 + (int)rank * 128, fb_leader, pol_a);
+          }
+          if (pr.b_mn) {
+            // B held [K rows, N columns]: this CTA's half of the tile's columns as two 64-column boxes
+            // (a narrower tile's second box brings columns it does not use, zeros past the tensor)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int n = ti.n0 + (int)rank * (ti.width / 2) + 64 * i;
+              int x = n, y = ti.bk0 + kb * kPairBK;
+              if (pr.b_split) { x = n % pr.b_split; y += (n / pr.b_split) * pr.K; }
+              tma_load_2d_pair(smem_u32(sa + C::A_BYTES) + 8192 * i, tB, x, y, fb_leader, pol_w);
+            }
+          } else {
+            tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tB, bx, by, fb_leader, pol_w);
+          }
         }
         if (gather) {
           __syncwarp();
@@ -294,7 +359,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       bool issued_any = false;
       uint32_t sn = 0;
       for (int local = 0;; ++local) {
-        const int tile = sched_take(sched_full, sched_empty, sched_tile, sn, abort_flag, a.status, 509);
+        int tile = cid + local * ncl;
+        if (dyn) tile = sched_take(sched_full, sched_empty, sched_tile, sn, rank, abort_flag, a.status, 509);
+        else if (tile >= pl.total) tile = -1;
         if (tile < 0) break;
         const PairTile ti = pair_decode<BN>(tile, pl, a);
         const int acc = local & 1;
@@ -302,16 +369,19 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         if (!mbar_wait(smem_u32(&acc_empty[acc]), accph ^ 1u, abort_flag, a.status, 502)) goto mma_out;
         tc_fence_after();
         const uint32_t d = tmem_base + acc * BN;
-        const uint32_t idesc = idesc_f16kind_f32(kPairBM, ti.width, S::kFmt);
+        const GemmProblem& pr = a.p[ti.p];
+        const uint32_t idesc = idesc_f16kind_f32(kPairBM, ti.width, S::kFmt) | idesc_major_bits(pr.a_mn, pr.b_mn);
+        // a k16 step advances 32 bytes inside a K-major row, or 16 rows (2048 bytes) of an MN-major tile
+        const uint64_t astep = pr.a_mn ? 128 : 2, bstep = pr.b_mn ? 128 : 2;
         for (int kb = 0; kb < ti.nk; ++kb) {
           if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)) goto mma_out;
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * C::STAGE);
-          const uint64_t adesc = smem_desc_sw128(sa);
-          const uint64_t bdesc = smem_desc_sw128(sa + C::A_BYTES);
+          const uint64_t adesc = pr.a_mn ? smem_desc_mn_sw128(sa) : smem_desc_sw128(sa);
+          const uint64_t bdesc = pr.b_mn ? smem_desc_mn_sw128(sa + C::A_BYTES) : smem_desc_sw128(sa + C::A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < kPairBK / 16; ++kk)
-            umma_kindf16_pair(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+            umma_kindf16_pair(d, adesc + astep * kk, bdesc + bstep * kk, idesc, (kb | kk) ? 1u : 0u);
           issued_any = true;
           // stage free in both CTAs once these MMAs finish
           const uint32_t eb = smem_u32(&empty[stage]);
@@ -353,9 +423,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     int nstore = 0;
     uint32_t sn = 0;
     for (int local = 0;; ++local) {
-      int tile = 0;
-      if (lane == 0) tile = sched_take(sched_full, sched_empty, sched_tile, sn, abort_flag, a.status, 510);
-      tile = __shfl_sync(0xffffffffu, tile, 0);
+      int tile = cid + local * ncl;
+      if (dyn) {
+        if (lane == 0) tile = sched_take(sched_full, sched_empty, sched_tile, sn, rank, abort_flag, a.status, 510);
+        tile = __shfl_sync(0xffffffffu, tile, 0);
+      } else if (tile >= pl.total) {
+        tile = -1;
+      }
       if (tile < 0) break;
       const PairTile ti = pair_decode<BN>(tile, pl, a);
       const GemmProblem& pr = a.p[ti.p];
@@ -372,8 +446,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       const uint16_t* bias =
           pr.bias ? reinterpret_cast<const uint16_t*>(pr.bias) + (long long)ti.e * pr.bias_stride : nullptr;
       constexpr int box_cols = 64;                          // 128 bytes of 16-bit h or y
-      // tanh GELU, erf GELU, gate, or the combine (routed rows + shared output)
-      const int mode = pr.epi == 0 ? (a.act == 1 ? 1 : 0) : (pr.epi == 2 ? 3 : 2);
+      // tanh GELU, erf GELU, gate, the combine (routed rows + shared output), or the GELU backward
+      const int mode = pr.epi == 0 ? (a.act == 1 ? 1 : 0) : (pr.epi == 2 ? 3 : (pr.epi == 4 ? 4 : 2));
+      float dgacc = 0.f;
       int ns = 0;
       const int32_t* prow = nullptr;
       if (mode == 3) {
@@ -396,6 +471,40 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         }
       }
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if (pr.out_f32) {
+        // weight gradients: 32 fp32 columns per box through the 3-D output map [z, M, N] (rows past
+        // M are clipped by the map); a tile with no reduction rows (an expert that took no token)
+        // stores zeros
+#pragma unroll 1
+        for (int c0 = 0; c0 < ti.width; c0 += 32) {
+          uint32_t v[32];
+          if (ti.nk > 0) {
+            tmem_ld_32x32b_x32(tbase + c0, v);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0u;
+          }
+          const uint32_t buf = sbuf + (nstore & 1) * 4096;
+          if (lane == 0) bulk_wait_read_le1();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + lane * 128 + ((j ^ (lane & 7)) << 4)),
+                         "r"(v[4 * j]), "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3])
+                         : "memory");
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            const int col = ti.n0 + c0;
+            int x = col, z = (pr.kgrouped && pr.routed) ? ti.e : 0;
+            if (pr.out_split) { z = col / pr.out_split; x = col % pr.out_split; }
+            tma_store_3d(tO, buf, x, box_row, z);
+            bulk_commit();
+          }
+          ++nstore;
+        }
+      } else {
 #pragma unroll 1
       for (int c0 = 0; c0 < ti.width; c0 += box_cols) {
         uint4 o[8];
@@ -441,6 +550,29 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
               ow[j / 2] = S::pack2((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate);
+          } else if (mode == 4) {
+            // GELU backward: acc = dY W (ungated), u the stored pre-activation of these columns;
+            // dU = gate * acc * gelu'(u) (zero on padding rows), and the row's sum of acc * gelu(u)
+            float uf[32];
+            if (rv) {
+              const uint4* up = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(pr.aux) +
+                                                               grow * pr.N + col0);
+#pragma unroll
+              for (int u4 = 0; u4 < 4; ++u4) S::x8_to_f32(__ldcg(up + u4), uf + 8 * u4);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) uf[j] = 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float g0, d0, g1, d1;
+              gelu_tanh_and_grad<true>(uf[j], g0, d0);
+              gelu_tanh_and_grad<true>(uf[j + 1], g1, d1);
+              const float a0 = __uint_as_float(v[j]), a1 = __uint_as_float(v[j + 1]);
+              dgacc = fmaf(a0, g0, dgacc);
+              dgacc = fmaf(a1, g1, dgacc);
+              ow[j / 2] = S::pack2(rv ? gate * a0 * d0 : 0.f, rv ? gate * a1 * d1 : 0.f);
+            }
           } else {
             // out = sum over the token's slots of its routed rows (slot order), plus the shared output
             float y[32];
@@ -498,6 +630,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         }
         ++nstore;
       }
+      if (mode == 4 && pr.dg != nullptr && rv) pr.dg[grow * pr.dg_stride + ti.n0 / BN] = dgacc;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
@@ -520,7 +654,7 @@ done:
   if (warp == 1) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
   if (threadIdx.x == 0) {
     // the last CTA out resets the tile counter and the combine count for the next launch (every
-    // claim of every CTA has returned before its exit is counted)
+    // claim of every CTA has returned before its exit is counted; the fixed order claims nothing)
     __threadfence();
     if (atomicAdd(a.exit_ctr, 1u) == gridDim.x - 1) {
       *a.sched_ctr = 0u;

@@ -96,12 +96,20 @@ struct BalanceGradArgs {
   void* dx;                                           // [T,D] act or null
   float* dwg;                                         // [E,D]
   float* dbias;                                       // [E] or null
+  // the gates' gradient (router backward of the whole layer), or null for the balance loss alone:
+  // dJ/dP[t, topk_idx[t,k]] += dgate[t,k] for the token's selected slots
+  const float* dgate; const int32_t* topk_idx; const int32_t* n_sel; int Kmax;
+  int dx_accumulate;                                  // 1: dx += dl Wg (dx holds the experts' part)
+  int pass_grid, pass_tpc;                             // > 0: the one-pass kernel, CTAs and tokens per CTA
   float* dl;                                          // [T,E] scratch: dL/dlogits
   float* db_part;                                     // [blocks,E] scratch
   float* partials;                                    // [chunks,E,D] scratch
 };
 constexpr int kBwdMaxBlocks = 1024;
 int balance_grad_chunks(int T);
+// the one-pass router backward: whether a row and the CTA's scratch fit, and its grid
+bool router_bwd_pass_fits(int D, int E, int dtype, int T, int sms);
+int router_bwd_pass_grid(int T, int sms, int* tpc);
 cudaError_t launch_balance_grad(const BalanceGradArgs& a, int blocks, cudaStream_t s);
 
 // ---- stats.cu: expert-selection frequency per label
@@ -157,10 +165,25 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
 // ---- gemm (tcgen05 and FFMA)
 struct GemmProblem {
   int routed;               // 1: rows grouped by expert segments (offsets), 0: dense rows
-  int M;                    // dense: rows; routed: unused (from offsets)
-  int N, K;                 // per-expert output width and reduction length
+  int M;                    // dense: rows; routed: unused (from offsets); kgrouped: rows of each output
+  int N, K;                 // per-expert output width and reduction length (kgrouped: K from offsets)
   int epi;                  // 0: bias + GELU -> act store; 1: (bias) * gate -> act store;
-                            // 2 (dense rows, CTA-pair kernel only): out = sum_k y_routed[pos[t,k]] + (acc + bias)
+                            // 2 (dense rows, CTA-pair kernel only): out = sum_k y_routed[pos[t,k]] + (acc + bias);
+                            // 4 (CTA-pair kernel only): out = gate * acc * gelu'(u) with u read from `aux`
+                            //   (same layout as out, may alias it), and dg[row, column tile] = sum acc * gelu(u)
+  // CTA-pair kernel only: operands held MN-major in memory ([K rows, M or N columns] row-major, as
+  // the weights of a backward GEMM or the activations of a weight gradient are), and the weight
+  // gradient's grouping: one [M, N] output per expert whose reduction runs over that expert's rows
+  // of the permuted buffers (segments from offsets, padded to 256; padding rows must be zero)
+  int a_mn, b_mn;
+  int kgrouped;
+  int b_split;              // MN-major B whose N runs over b_split-wide blocks stacked along K (the n_s
+                            // shared W2 [n_s, D, H] seen as [n_s*D, H]): block n / b_split sits K rows lower
+  int out_f32;              // fp32 output through a 3-D map [z, M, N]: z = expert (kgrouped), n / out_split, or 0
+  int out_split;
+  const void* aux;          // epi 4: u [rows, N] act
+  float* dg;                // epi 4: [rows, dg_stride] per-column-tile row dots, or null
+  int dg_stride;
   const void* A;            // [rows,K] act (FFMA path; the TMA path uses tensor maps)
   const void* B;            // [E*N or N, K] act
   void* out; long long ld_out;
@@ -202,6 +225,29 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUt
                              int bn, int num_sms, int max_pairs, cudaStream_t s);
 int gemm_pair_pick_bn(int n0, int n1);
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t s);
+
+// ---- expert_backward.cu: memory-bound parts of the expert MLPs' backward
+struct ExpertBwdArgs {
+  const void* dout;          // [T,D] act: dJ/dMoE(x)
+  const int32_t* row_token;  // [rows] from moe_dispatch (-1 on padding rows)
+  const float* row_gate;     // [rows]
+  long long rows;            // R_max
+  int T, D, E, K, Kmax, f16;
+  void* dout_perm;           // [rows,D] act out: dY in permuted order
+  void* dz_perm;             // [rows,D] act out: g * dY in permuted order
+  // dgate
+  const int32_t* pos; const int32_t* topk_idx; const int32_t* n_sel;
+  const float* dg; int dg_stride;   // [rows, dg_stride] row dots per column tile of the GELU-backward GEMM
+  const void* b2;            // [E,D] act or null
+  float* dgate;              // [T,Kmax] out
+};
+cudaError_t launch_bwd_gather(const ExpertBwdArgs& a, cudaStream_t s);
+cudaError_t launch_dgate(const ExpertBwdArgs& a, cudaStream_t s);
+// column sums of X [nrows, C] (16-bit) per expert segment (offsets) or over all rows (offsets null),
+// each written nrep times: out [nseg * nrep, C] fp32; partial: [colsum_chunks(nrows), C] fp32 scratch
+int colsum_chunks(long long nrows);
+cudaError_t launch_colsum(const void* X, long long nrows, int C, const int32_t* offsets, int E, int nrep,
+                          float* partial, float* out, int f16, cudaStream_t s);
 
 // ---- combine.cu
 struct CombineArgs {

@@ -238,6 +238,41 @@ class MoELayer:
     def check(self):
         B.moe_check_status(self.ws, self.stream())
 
+    # ------------------------------------------------------------ backward
+    def backward(self, x: torch.Tensor, dout: torch.Tensor, aux_scale: float = 1.0) -> dict:
+        """Gradients of J = <dout, MoE(x)> + aux_scale * L_balance after ``forward(x)``.
+
+        Returns fp32 gradients of every weight and bias (dw1, db1, dw2, db2, dws1, dbs1, dws2,
+        dbs2, dwg, dbias), the gates' gradient ``dgate`` [T, Kmax] and ``dx`` (act dtype).  The
+        selection is the forward's (discrete, no gradient).  Needs the forward's x_perm (the
+        default dispatch, not the gathered GEMM1)."""
+        if self.x_perm is None:
+            raise ValueError("the backward reads x_perm: run the forward without gather_rows")
+        s, dev, T = self.s, self.device, self.cfg.T
+        f32 = torch.float32
+        E, D, H, ns = s.E, s.D, s.H, s.n_shared
+        if getattr(self, "_ebws", None) is None:
+            self._ebws_bytes = B.moe_expert_backward_workspace_size(self.cfg)
+            self._ebws = torch.empty(self._ebws_bytes, dtype=torch.uint8, device=dev)
+            self._rbws_bytes = B.moe_backward_workspace_size(self.cfg)
+            self._rbws = torch.empty(self._rbws_bytes, dtype=torch.uint8, device=dev)
+        e = lambda *shape: torch.empty(shape, dtype=f32, device=dev)
+        g = {"dw1": e(E, H, D), "db1": e(E, H), "dw2": e(E, D, H), "db2": e(E, D),
+             "dws1": e(ns, H, D) if ns else None, "dbs1": e(ns, H) if ns else None,
+             "dws2": e(ns, D, H) if ns else None, "dbs2": e(ns, D) if ns else None,
+             "dwg": e(E, D), "dbias": e(E), "dgate": e(T, self.kmax),
+             "dx": torch.empty((T, D), dtype=self.act_dtype, device=dev)}
+        wts = B.make_expert_weights(self.w1, self.b1, self.w2, self.b2, self.ws1, self.bs1, self.ws2, self.bs2)
+        grads = B.make_expert_grads(g["dw1"], g["db1"], g["dw2"], g["db2"], g["dws1"], g["dbs1"], g["dws2"],
+                                    g["dbs2"])
+        B.moe_expert_backward(self.cfg, x, self.x_perm, self.offsets, self.pos, self.topk_idx, self.n_sel,
+                              self.row_token, self.row_gate, wts, self.h_perm, self.h_sh, dout, grads, g["dgate"],
+                              g["dx"], self.ws, self.ws_bytes, self._ebws, self._ebws_bytes, self.stream())
+        B.moe_router_backward(self.cfg, x, self.wg, self.router_bias, self.counts, self.topk_idx, self.n_sel,
+                              g["dgate"], aux_scale, g["dwg"], g["dbias"], g["dx"], 1, self._rbws, self._rbws_bytes,
+                              self.stream())
+        return g
+
     # ------------------------------------------------------------ serving from host memory
     def forward_host_pipelined(self, x_host, out_host, aux_host=None):
         """Run the layer over a sequence of host batches, overlapping transfers with compute.

@@ -178,6 +178,10 @@ def check_permutation(w: Workload, L, r: dict, x_dev: torch.Tensor, rows_to_chec
     assert np.all(r["row_gate"][:Rv][~valid] == 0)
     if L.x_perm is None:             # GEMM1 gathered the rows from x itself: nothing permuted to compare
         return cp
+    # the padding rows inside the expert segments are zero
+    pad = torch.as_tensor(np.nonzero(~valid)[0], device=x_dev.device)
+    if pad.numel():
+        assert int(torch.count_nonzero(L.x_perm.index_select(0, pad))) == 0
     # x_perm rows are exact copies of x rows (sampled rows when large)
     rows = np.nonzero(valid)[0]
     if rows.size > rows_to_check:

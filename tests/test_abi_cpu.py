@@ -191,3 +191,35 @@ def test_negative_gemm_pairs_rejected():
     f = B.lib.moe_expert_gemm1
     assert f(ctypes.byref(cfg), fake, fake, fake, fake, None, fake, None, fake, fake, fake, 1 << 20, None) == \
         B.MOE_ERR_INVALID_ARG
+
+
+def test_expert_backward_arguments_rejected_before_launch():
+    fake = 1 << 40
+    cfg = B.make_config(1024, 384, 1536, 8, 2, 2)
+    n = B.moe_expert_backward_workspace_size(cfg)
+    assert n > 0 and n % 256 == 0
+    wsz = B.moe_workspace_size(cfg)
+    w = B.MoeExpertWeights(*([fake] * 8))
+    g = B.MoeExpertGrads(*([fake] * 8))
+    f = B.lib.moe_expert_backward
+
+    def call(c=cfg, wts=w, grads=g, bws_bytes=n, dgate=fake):
+        return f(ctypes.byref(c), fake, fake, fake, fake, fake, fake, fake, fake,
+                 ctypes.byref(wts) if wts is not None else None, fake, fake, fake,
+                 ctypes.byref(grads) if grads is not None else None, dgate, fake, fake, wsz, fake, bws_bytes, None)
+    f32 = B.make_config(1024, 384, 1536, 8, 2, 2, dtype="f32")
+    assert call(c=f32) == B.MOE_ERR_UNSUPPORTED and b"bf16" in B.lib.moe_last_error()
+    erf = B.make_config(1024, 384, 1536, 8, 2, 2, act="erf")
+    assert call(c=erf) == B.MOE_ERR_UNSUPPORTED
+    assert call(wts=None) == B.MOE_ERR_INVALID_ARG
+    assert call(bws_bytes=n - 256) == B.MOE_ERR_WORKSPACE
+    assert call(dgate=None) == B.MOE_ERR_INVALID_ARG and b"dgate" in B.lib.moe_last_error()
+    bad = B.MoeExpertGrads(None, fake, fake, fake, fake, fake, fake, fake)
+    assert call(grads=bad) == B.MOE_ERR_INVALID_ARG and b"dw1" in B.lib.moe_last_error()
+    rb = B.lib.moe_router_backward
+    nb = B.moe_backward_workspace_size(cfg)
+    # accumulating into dx needs dx; the gates' gradient needs the selection
+    assert rb(ctypes.byref(cfg), fake, fake, None, fake, fake, None, None, ctypes.c_float(1.0), fake, None, None, 1,
+              fake, nb, None) == B.MOE_ERR_INVALID_ARG
+    assert rb(ctypes.byref(cfg), fake, fake, None, fake, None, None, fake, ctypes.c_float(1.0), fake, None, None, 0,
+              fake, nb, None) == B.MOE_ERR_INVALID_ARG

@@ -383,6 +383,27 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
             times.append(b0.elapsed_time(b1))
         bwd_ms = float(np.median(times))
 
+    # the whole layer's backward (experts, gates, router; not part of the forward step): on its own
+    layer_bwd = None
+    if w.dtype in ("bf16", "f16") and not getattr(args, "seq_len", 0) and L.x_perm is not None:
+        L.forward(x)
+        dout = torch.randn((w.T, w.D), generator=torch.Generator().manual_seed(5)).to(device=device, dtype=dt)
+        for _ in range(2):
+            L.backward(x, dout)
+        torch.cuda.synchronize(device)
+        times = []
+        for i in range(5):
+            flush_l2(i)
+            b0 = torch.cuda.Event(enable_timing=True)
+            b1 = torch.cuda.Event(enable_timing=True)
+            b0.record(stream)
+            L.backward(x, dout)
+            b1.record(stream)
+            torch.cuda.synchronize(device)
+            times.append(b0.elapsed_time(b1))
+        L.check()
+        layer_bwd = float(np.median(times))
+
     # expert-selection frequency per patch position of the last routing (not part of the step): on its own
     freq_ms = None
     if w.tokens_per_image and w.T % w.tokens_per_image == 0:
@@ -413,6 +434,15 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local: int) -> dict:
             result["expert_frequency"] = {"ms": round(freq_ms, 4), "GB/s": round(moved / (freq_ms * 1e-3) / 1e9, 1),
                                           "what": "moe_expert_frequency per patch position (selection read once, "
                                                   "[positions, E] counts written), timed separately"}
+        if layer_bwd is not None:
+            # five GEMMs of GEMM1's size: the pre-activations again, dU, dx, dW2, dW1
+            bflops = 5 * M.gemm1_flops(w.T, w.D, w.H, w.K, w.n_shared)
+            result["layer_backward"] = {"ms": round(layer_bwd, 4),
+                                        "gemm_TFLOP/s": round(bflops / (layer_bwd * 1e-3) / 1e12, 1),
+                                        "what": "MoELayer.backward: moe_expert_backward (gather of dY, five "
+                                                "tcgen05 GEMMs with MN-major operands, bias column sums, gate "
+                                                "gradient) + moe_router_backward; timed separately; TFLOP/s counts "
+                                                "the five GEMMs over the whole time"}
         if bwd_ms is not None:
             elem = 2 if w.dtype in ("bf16", "f16") else 4
             moved = 2 * w.T * w.D * elem + w.E * w.D * (elem + 4)

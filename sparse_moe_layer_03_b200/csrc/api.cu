@@ -461,8 +461,14 @@ int router_backward(const moe_config_t* cfg, const void* x, const void* wg, cons
   a.dl = ws_at<float>(bws, BL.dl);
   a.db_part = ws_at<float>(bws, BL.db_part);
   a.partials = ws_at<float>(bws, BL.partials);
-  if (router_bwd_pass_fits(cfg->D, cfg->E, cfg->dtype, cfg->T, num_sms_current()))
+  CUtensorMap tmx;
+  if (router_bwd_mma_fits(cfg->D, cfg->E, cfg->dtype) && make_tmap_rows3d(&tmx, x, cfg->dtype, cfg->T, cfg->D, 16)) {
+    const int nrb = (cfg->T + 15) / 16;
+    a.mma_grid = nrb < num_sms_current() ? nrb : num_sms_current();
+    a.tmap_x = &tmx;
+  } else if (router_bwd_pass_fits(cfg->D, cfg->E, cfg->dtype, cfg->T, num_sms_current())) {
     a.pass_grid = router_bwd_pass_grid(cfg->T, num_sms_current(), &a.pass_tpc);
+  }
   // 8 tokens per block (one per warp) at a time: enough blocks to keep every SM's memory pipe busy
   int blocks = num_sms_current() * 4;
   if (blocks > kBwdMaxBlocks) blocks = kBwdMaxBlocks;

@@ -398,6 +398,287 @@ __global__ void __launch_bounds__(kRbThreads, 2) router_bwd_pass_kernel(BalanceG
   }
 }
 
+// ---------------------------------------------------------------- bf16: on mma.sync
+// Rows of 16 tokens come in by TMA (two half-row boxes per stage, 128-byte swizzle, a ring of
+// kRmStages stages refilled as soon as every warp has left the block).  Per block: each warp
+// takes every kRmWarps-th 64-column block for the partial logits x Wg^T (as the forward router);
+// warp (block mod kRmWarps) adds them in warp order and computes softmax and dl for the 16
+// tokens (one lane each), written to shared memory as two bf16 parts (dl = hi + lo, about 16
+// bits of mantissa); then every warp, on its own contiguous slice of D/8 8-column tiles, forms
+// dx = dl Wg (two MMAs, written to global memory; added to the experts' part when asked) and
+// accumulates dWg += dl^T x in registers over all of the CTA's blocks (x read straight from the
+// stage with transposed ldmatrix).  E <= 16 (zero-padded to 16), D <= 1152.
+constexpr int kRmWarps = 4;
+constexpr int kRmStages = 4;
+constexpr int kRmMaxNT = 36;                      // 8-column tiles per warp: D / 8 / kRmWarps
+
+struct RmSmem {
+  size_t wg, x, dl, lp, db, misc, total;
+  int hc, stage_bytes, wg_stride;
+};
+__host__ __device__ inline RmSmem rm_layout(int D) {
+  RmSmem L;
+  L.hc = (D / 64 + 1) / 2;
+  L.stage_bytes = 16 * 2 * L.hc * 128;
+  L.wg_stride = D * 2 + 16;
+  L.wg = 0;
+  L.x = ((size_t)16 * L.wg_stride + 1023) & ~(size_t)1023;
+  L.dl = L.x + (size_t)kRmStages * L.stage_bytes;
+  L.lp = L.dl + 2 * 16 * 16 * 2;                   // dl hi and lo, [16 tokens][16 experts] bf16 each
+  L.db = L.lp + (size_t)kRmWarps * 16 * 16 * 4;    // partial logits [warp][token][expert] fp32
+  L.misc = L.db + (size_t)kRmWarps * 16 * 16 * 4; // db per selecting lane [warp][lane][expert]
+  L.total = L.misc + 256 + 1024;                   // barriers; 1 KB alignment slack
+  return L;
+}
+
+bool router_bwd_mma_fits(int D, int E, int dtype) {
+  if (dtype != 1 || E > 16 || D % 64 || D / 8 / kRmWarps > kRmMaxNT) return false;
+  return rm_layout(D).total <= 232448;
+}
+size_t router_bwd_mma_smem(int D) { return rm_layout(D).total; }
+
+template <int EMAX>
+__global__ void __launch_bounds__(kRmWarps * 32, 1)
+router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArgs a) {
+  constexpr int NTE = EMAX / 8;                    // expert tiles of the logits
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const RmSmem L = rm_layout(a.D);
+  const int D = a.D, E = a.E, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int g = lane >> 2, c = lane & 3, li = lane >> 3, lj = lane & 7;
+  const int nblk = D / 64, ntw = D / 8 / kRmWarps;
+  uint8_t* wg_s = smem + L.wg;
+  uint8_t* xs = smem + L.x;
+  uint16_t* dlh = reinterpret_cast<uint16_t*>(smem + L.dl);
+  uint16_t* dll = dlh + 16 * 16;
+  float* lp = reinterpret_cast<float*>(smem + L.lp);
+  float* dbs = reinterpret_cast<float*>(smem + L.db);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.misc);
+  __shared__ float c_s[16];
+  const int nrb = (a.T + 15) / 16;
+  const int my_rb = (nrb - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  auto issue = [&](int j) {                        // thread 0: row block j of this CTA into its stage
+    const int st = j % kRmStages;
+    const int rb = blockIdx.x + j * gridDim.x;
+    const uint32_t bar = smem_u32(&full[st]);
+    const uint32_t dst = smem_u32(xs + (size_t)st * L.stage_bytes);
+    mbar_arrive_expect_tx(bar, (uint32_t)L.stage_bytes);
+    tma_load_3d(dst, &tmap_x, 0, rb * 16, 0, bar);
+    tma_load_3d(dst + L.hc * 2048, &tmap_x, 0, rb * 16, L.hc, bar);
+  };
+  if (tid == 0) {
+    for (int st = 0; st < kRmStages; ++st) mbar_init(smem_u32(&full[st]), 1);
+    fence_barrier_init();
+    for (int j = 0; j < kRmStages && j < my_rb; ++j) issue(j);
+  }
+  if (tid < 16)
+    c_s[tid] = tid < E ? a.scale * a.alpha * ((float)E / ((float)a.K * a.T)) * (float)a.counts[tid] / (float)a.T : 0.f;
+  {  // gate weight rows 0..15 (zero past E), padded stride
+    const int vpr = D / 8;
+    const uint4* wv = reinterpret_cast<const uint4*>(a.wg);
+    for (int i = tid; i < 16 * vpr; i += blockDim.x) {
+      const int e = i / vpr, v = i % vpr;
+      const uint4 val = e < E ? __ldg(wv + (size_t)e * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(wg_s + (size_t)e * L.wg_stride + v * 16) = val;
+    }
+  }
+  __syncthreads();
+  const uint32_t wg_base = smem_u32(wg_s);
+  float acc[kRmMaxNT][4];
+#pragma unroll
+  for (int i = 0; i < kRmMaxNT; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+  float dbw[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) dbw[e] = 0.f;
+  bool ok = true;
+  for (int j = 0; j < my_rb; ++j) {
+    const int st = j % kRmStages;
+    const int rb = blockIdx.x + j * gridDim.x;
+    // a wait that ran out once makes every later block skip its work; the barriers still run
+    // (no status word here: the router backward's scratch has none; a wait that ran out still ends the kernel)
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), (j / kRmStages) & 1, nullptr, nullptr, 120));
+    const uint32_t xb = smem_u32(xs + (size_t)st * L.stage_bytes);
+    // ---- partial logits of this warp's 64-column blocks
+    float la[NTE][4];
+#pragma unroll
+    for (int nt = 0; nt < NTE; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) la[nt][q] = 0.f;
+    if (ok) {
+      for (int b = w; b < nblk; b += kRmWarps) {
+        const uint32_t box = xb + b * 2048;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          uint32_t bb[NTE][2];
+          const int kc = b * 64 + ks * 16 + (li & 1) * 8;
+#pragma unroll
+          for (int np = 0; np < NTE; np += 2) {
+            if (np + 1 < NTE) {
+              const int n = (np + (li >> 1)) * 8 + lj;
+              ldsm_x4(wg_base + n * L.wg_stride + kc * 2, bb[np][0], bb[np][1], bb[np + 1][0], bb[np + 1][1]);
+            } else {
+              ldsm_x2(wg_base + (np * 8 + lj) * L.wg_stride + kc * 2, bb[np][0], bb[np][1]);
+            }
+          }
+          const int row = (li & 1) * 8 + lj;
+          const int chunk = ks * 2 + (li >> 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NTE; ++nt) mma_16816<false>(la[nt], a0, a1, a2, a3, bb[nt][0], bb[nt][1]);
+        }
+      }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NTE; ++nt) {
+      float* pw = lp + (size_t)w * 256;
+      pw[g * 16 + nt * 8 + 2 * c] = la[nt][0];
+      pw[g * 16 + nt * 8 + 2 * c + 1] = la[nt][1];
+      pw[(g + 8) * 16 + nt * 8 + 2 * c] = la[nt][2];
+      pw[(g + 8) * 16 + nt * 8 + 2 * c + 1] = la[nt][3];
+    }
+    __syncthreads();
+    // every warp has left block j - 1: its stage takes block j - 1 + kRmStages
+    if (tid == 0 && j >= 1 && j - 1 + kRmStages < my_rb) {
+      fence_async_shared();
+      issue(j - 1 + kRmStages);
+    }
+    // ---- softmax and dl of the block's 16 tokens (one lane each)
+    if (w == j % kRmWarps && lane < 16) {
+      const int t = rb * 16 + lane;
+      float dl[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) dl[e] = 0.f;
+      if (t < a.T && ok) {
+        float l[EMAX];
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) {
+          float v = 0.f;
+#pragma unroll
+          for (int k = 0; k < kRmWarps; ++k) v += lp[k * 256 + lane * 16 + e];
+          l[e] = v;
+        }
+        float m = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e)
+          if (e < E) { l[e] += a.bias ? a.bias[e] : 0.f; m = fmaxf(m, l[e]); }
+        float z = 0.f;
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e)
+          if (e < E) { l[e] = expf(l[e] - m); z += l[e]; }
+        const float iz = 1.0f / z;
+        float dp[EMAX];
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) dp[e] = c_s[e];
+        if (a.dgate) {
+          const int ns = a.n_sel ? a.n_sel[t] : a.K;
+          for (int k = 0; k < a.Kmax && k < ns; ++k) {
+            const int sel = a.topk_idx[(size_t)t * a.Kmax + k];
+            const float gk = a.dgate[(size_t)t * a.Kmax + k];
+#pragma unroll
+            for (int e = 0; e < EMAX; ++e) dp[e] += e == sel ? gk : 0.f;
+          }
+        }
+        float pc = 0.f;
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e)
+          if (e < E) { l[e] *= iz; pc += l[e] * dp[e]; }
+#pragma unroll
+        for (int e = 0; e < EMAX; ++e) {
+          dl[e] = e < E ? l[e] * (dp[e] - pc) : 0.f;
+          dbw[e] += dl[e];
+        }
+      }
+      uint32_t* hp = reinterpret_cast<uint32_t*>(dlh + lane * 16);
+      uint32_t* lo = reinterpret_cast<uint32_t*>(dll + lane * 16);
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(dl[e], dl[e + 1]);
+        const float2 hf = __bfloat1622float2(h2);
+        const __nv_bfloat162 l2 = __floats2bfloat162_rn(dl[e] - hf.x, dl[e + 1] - hf.y);
+        hp[e / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+        lo[e / 2] = *reinterpret_cast<const uint32_t*>(&l2);
+      }
+    }
+    __syncthreads();
+    // ---- dx = dl Wg and dWg += dl^T x on this warp's 8-column tiles
+    if (ok) {
+      uint32_t ah[4], al[4], th[4], tl[4];
+      {
+        const int r = (lane & 7) + ((lane >> 3) & 1) * 8, cb = (lane >> 4) * 8;   // A = dl [t][e]
+        ldsm_x4(smem_u32(dlh + r * 16 + cb), ah[0], ah[1], ah[2], ah[3]);
+        ldsm_x4(smem_u32(dll + r * 16 + cb), al[0], al[1], al[2], al[3]);
+        const int mi = lane >> 3, tt = (mi >> 1) * 8 + (lane & 7), e0 = (mi & 1) * 8;  // A = dl^T [e][t]
+        ldsm_x4_t(smem_u32(dlh + tt * 16 + e0), th[0], th[1], th[2], th[3]);
+        ldsm_x4_t(smem_u32(dll + tt * 16 + e0), tl[0], tl[1], tl[2], tl[3]);
+      }
+      const int t0 = rb * 16 + g, t1 = t0 + 8;
+      const int rr = lane & 15;                    // row of the 8x8 tiles this lane addresses
+#pragma unroll
+      for (int i = 0; i < kRmMaxNT; ++i) {
+        if (i < ntw) {
+          const int col0 = (w * ntw + i) * 8;
+          uint32_t b0, b1, x0, x1;
+          ldsm_x2_t(wg_base + rr * L.wg_stride + col0 * 2, b0, b1);        // B = Wg [e][d]
+          const int blk = col0 >> 6, q = (col0 & 63) >> 3;
+          ldsm_x2_t(xb + blk * 2048 + rr * 128 + ((q ^ (rr & 7)) << 4), x0, x1);   // B = x [t][d]
+          float d4[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_16816<false>(d4, ah[0], ah[1], ah[2], ah[3], b0, b1);
+          mma_16816<false>(d4, al[0], al[1], al[2], al[3], b0, b1);
+          mma_16816<false>(acc[i], th[0], th[1], th[2], th[3], x0, x1);
+          mma_16816<false>(acc[i], tl[0], tl[1], tl[2], tl[3], x0, x1);
+          if (a.dx) {
+            uint32_t* dxp = reinterpret_cast<uint32_t*>(a.dx);
+            const int cc = col0 + 2 * c;
+            if (t0 < a.T) {
+              float o0 = d4[0], o1 = d4[1];
+              const size_t ix = ((size_t)t0 * D + cc) / 2;
+              if (a.dx_accumulate) {
+                const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dxp[ix]));
+                o0 += p.x; o1 += p.y;
+              }
+              const __nv_bfloat162 v = __floats2bfloat162_rn(o0, o1);
+              dxp[ix] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+            if (t1 < a.T) {
+              float o0 = d4[2], o1 = d4[3];
+              const size_t ix = ((size_t)t1 * D + cc) / 2;
+              if (a.dx_accumulate) {
+                const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dxp[ix]));
+                o0 += p.x; o1 += p.y;
+              }
+              const __nv_bfloat162 v = __floats2bfloat162_rn(o0, o1);
+              dxp[ix] = *reinterpret_cast<const uint32_t*>(&v);
+            }
+          }
+        }
+      }
+    }
+  }
+  // ---- this CTA's partial dWg (rows e = g, g + 8 of its fragments) and db (selecting lanes, in order)
+  float* part = a.partials + (size_t)blockIdx.x * E * D;
+#pragma unroll
+  for (int i = 0; i < kRmMaxNT; ++i) {
+    if (i < ntw) {
+      const int col = (w * ntw + i) * 8 + 2 * c;
+      if (g < E) { part[(size_t)g * D + col] = acc[i][0]; part[(size_t)g * D + col + 1] = acc[i][1]; }
+      if (g + 8 < E) { part[(size_t)(g + 8) * D + col] = acc[i][2]; part[(size_t)(g + 8) * D + col + 1] = acc[i][3]; }
+    }
+  }
+  if (lane < 16) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) dbs[(w * 16 + lane) * 16 + e] = dbw[e];
+  }
+  __syncthreads();
+  if (tid < E) {
+    float sdb = 0.f;
+    for (int k = 0; k < kRmWarps * 16; ++k) sdb += dbs[k * 16 + tid];
+    a.db_part[(size_t)blockIdx.x * E + tid] = sdb;
+  }
+}
+
 // Block b sums elements [32 b, 32 b + 32) of [dWg, db]: lane = element, warp w takes the partials
 // p = w, w + 8, ... in order (eight loads in flight per lane), then the eight warp sums are added
 // in warp order.  A fixed order throughout.
@@ -490,7 +771,19 @@ bool router_bwd_pass_fits(int D, int E, int dtype, int T, int sms) {
 cudaError_t launch_balance_grad(const BalanceGradArgs& a, int blocks, cudaStream_t s) {
   cudaError_t e;
   int nparts = blocks, nchunks = balance_grad_chunks(a.T);
-  if (a.pass_grid > 0) {
+  if (a.mma_grid > 0) {
+    // bf16 on mma.sync: partials of dWg and db per CTA
+    const size_t smem = router_bwd_mma_smem(a.D);
+    if (a.E <= 8) {
+      e = cudaFuncSetAttribute(router_bwd_mma_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) router_bwd_mma_kernel<8><<<a.mma_grid, kRmWarps * 32, smem, s>>>(*a.tmap_x, a);
+    } else {
+      e = cudaFuncSetAttribute(router_bwd_mma_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) router_bwd_mma_kernel<16><<<a.mma_grid, kRmWarps * 32, smem, s>>>(*a.tmap_x, a);
+    }
+    if (e == cudaSuccess) e = cudaGetLastError();
+    nparts = nchunks = a.mma_grid;
+  } else if (a.pass_grid > 0) {
     // one pass: partials of dWg and db per CTA
     e = a.dtype == 0 ? launch_rb_t<float>(a, a.pass_grid, a.pass_tpc, s)
         : a.dtype == 2 ? launch_rb_t<__half>(a, a.pass_grid, a.pass_tpc, s)

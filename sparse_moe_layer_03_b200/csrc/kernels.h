@@ -101,6 +101,8 @@ struct BalanceGradArgs {
   const float* dgate; const int32_t* topk_idx; const int32_t* n_sel; int Kmax;
   int dx_accumulate;                                  // 1: dx += dl Wg (dx holds the experts' part)
   int pass_grid, pass_tpc;                             // > 0: the one-pass kernel, CTAs and tokens per CTA
+  int mma_grid;                                       // > 0: the bf16 mma.sync kernel on this many CTAs
+  const CUtensorMap* tmap_x;                          // its x map (3-D half-row boxes of 16 rows)
   float* dl;                                          // [T,E] scratch: dL/dlogits
   float* db_part;                                     // [blocks,E] scratch
   float* partials;                                    // [chunks,E,D] scratch
@@ -109,6 +111,9 @@ constexpr int kBwdMaxBlocks = 1024;
 int balance_grad_chunks(int T);
 // the one-pass router backward: whether a row and the CTA's scratch fit, and its grid
 bool router_bwd_pass_fits(int D, int E, int dtype, int T, int sms);
+// the bf16 router backward on mma.sync: whether it applies, and its shared memory
+bool router_bwd_mma_fits(int D, int E, int dtype);
+size_t router_bwd_mma_smem(int D);
 int router_bwd_pass_grid(int T, int sms, int* tpc);
 cudaError_t launch_balance_grad(const BalanceGradArgs& a, int blocks, cudaStream_t s);
 

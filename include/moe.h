@@ -226,10 +226,11 @@ int moe_expert_gemm1(const moe_config_t* cfg, const int32_t* offsets, const void
 
 /*
  * moe_expert_gemm1_gather -- moe_expert_gemm1 without x_perm: each routed row
- * r of the expert-contiguous layout is row row_token[r] of x, brought into
- * shared memory by TMA tile::gather4 (four rows per load) inside the GEMM, so
- * the dispatch writes positions only and the permuted copy of x never exists.
- * Padding rows (row_token -1) read row 0; their h rows are never used.
+ * r of the expert-contiguous layout is row row_token[r] of x, copied into
+ * shared memory by two gather warps of the GEMM (16-byte cp.async into the
+ * swizzled stage), so the dispatch writes positions only and the permuted copy
+ * of x never exists.  Padding rows (row_token -1) read row 0; their h rows are
+ * never used.
  *   row_token [R_max] int32 from moe_dispatch; other arguments as moe_expert_gemm1.
  * Only for bf16 or fp16 with gemm_impl AUTO (MOE_ERR_UNSUPPORTED otherwise).
  */

@@ -192,7 +192,7 @@ def moe_expert_gemm1(cfg, offsets, x_perm, x, w1, b1, w1s, b1s, h_perm, h_sh, ws
 
 
 def moe_expert_gemm1_gather(cfg, offsets, row_token, x, w1, b1, w1s, b1s, h_perm, h_sh, ws, ws_bytes, stream=0):
-    """GEMM1 reading its routed rows straight from x (TMA gather4 by row_token): no x_perm."""
+    """GEMM1 reading its routed rows straight from x (cp.async by row_token): no x_perm."""
     _check(lib.moe_expert_gemm1_gather(C.byref(cfg), _ptr(offsets), _ptr(row_token), _ptr(x), _ptr(w1), _ptr(b1),
                                        _ptr(w1s), _ptr(b1s), _ptr(h_perm), _ptr(h_sh), _ptr(ws), ws_bytes, stream))
 

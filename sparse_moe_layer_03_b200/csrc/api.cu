@@ -595,9 +595,9 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
   CUtensorMap ta[2], tb[2];
   int rc;
   if (g.p[0].gather_rows) {
-    // gathered A rows: one-row boxes (tile::gather4 brings four rows per load)
+    // gathered A rows: the GEMM's gather warps copy them; the map is not read
     if (!pair) return fail(MOE_ERR_UNSUPPORTED, "row gathering needs the CTA-pair GEMM");
-    if ((rc = make_tmap(&ta[0], A0, cfg->dtype, rows0, K0, 1, "A0 (gathered rows)"))) return rc;
+    if ((rc = make_tmap(&ta[0], A0, cfg->dtype, rows0, K0, 128, "A0 (gathered rows)"))) return rc;
   } else if ((rc = make_tmap(&ta[0], A0, cfg->dtype, rows0, K0, 128, "A0"))) {
     return rc;
   }

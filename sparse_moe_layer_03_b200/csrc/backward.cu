@@ -400,20 +400,22 @@ __global__ void __launch_bounds__(kRbThreads, 2) router_bwd_pass_kernel(BalanceG
 
 // ---------------------------------------------------------------- bf16: on mma.sync
 // Rows of 16 tokens come in by TMA (two half-row boxes per stage, 128-byte swizzle, a ring of
-// kRmStages stages refilled as soon as every warp has left the block).  Per block: each warp
-// takes every kRmWarps-th 64-column block for the partial logits x Wg^T (as the forward router);
-// warp (block mod kRmWarps) adds them in warp order and computes softmax and dl for the 16
-// tokens (one lane each), written to shared memory as two bf16 parts (dl = hi + lo, about 16
-// bits of mantissa); then every warp, on its own contiguous slice of D/8 8-column tiles, forms
-// dx = dl Wg (two MMAs, written to global memory; added to the experts' part when asked) and
-// accumulates dWg += dl^T x in registers over all of the CTA's blocks (x read straight from the
-// stage with transposed ldmatrix).  E <= 16 (zero-padded to 16), D <= 1152.
-constexpr int kRmWarps = 4;
+// kRmStages stages refilled as soon as every warp has left the block).  Per block: each of the
+// 16 warps takes every 16th k16 step for the partial logits x Wg^T (as the forward router); the
+// first 256 threads add the 16 partials in warp order; warp (block mod 16) computes softmax and
+// dl for the 16 tokens (one lane each), written to shared memory as two bf16 parts (dl = hi + lo,
+// about 16 bits of mantissa); then every warp, on its own contiguous slice of the D/8 8-column
+// tiles, forms dx = dl Wg (two MMAs, written to global memory; the experts' part, loaded first
+// for all of the slice's tiles at once, added when asked) and accumulates dWg += dl^T x in
+// registers over all of the CTA's blocks (x read straight from the stage with transposed
+// ldmatrix).  Sixteen warps per SM keep enough MMAs and loads in flight: with four, the SM
+// waited on single dependences most of the time.  E <= 16 (zero-padded to 16), D <= 1152.
+constexpr int kRmWarps = 16;
 constexpr int kRmStages = 4;
-constexpr int kRmMaxNT = 36;                      // 8-column tiles per warp: D / 8 / kRmWarps
+constexpr int kRmMaxNT = 9;                       // 8-column tiles per warp: ceil(D / 8 / kRmWarps)
 
 struct RmSmem {
-  size_t wg, x, dl, lp, db, misc, total;
+  size_t wg, x, dl, lp, ls, db, misc, total;
   int hc, stage_bytes, wg_stride;
 };
 __host__ __device__ inline RmSmem rm_layout(int D) {
@@ -425,14 +427,15 @@ __host__ __device__ inline RmSmem rm_layout(int D) {
   L.x = ((size_t)16 * L.wg_stride + 1023) & ~(size_t)1023;
   L.dl = L.x + (size_t)kRmStages * L.stage_bytes;
   L.lp = L.dl + 2 * 16 * 16 * 2;                   // dl hi and lo, [16 tokens][16 experts] bf16 each
-  L.db = L.lp + (size_t)kRmWarps * 16 * 16 * 4;    // partial logits [warp][token][expert] fp32
+  L.ls = L.lp + (size_t)kRmWarps * 16 * 16 * 4;    // partial logits [warp][token][expert] fp32
+  L.db = L.ls + 16 * 16 * 4;                       // logits [token][expert] fp32
   L.misc = L.db + (size_t)kRmWarps * 16 * 16 * 4; // db per selecting lane [warp][lane][expert]
   L.total = L.misc + 256 + 1024;                   // barriers; 1 KB alignment slack
   return L;
 }
 
 bool router_bwd_mma_fits(int D, int E, int dtype) {
-  if (dtype != 1 || E > 16 || D % 64 || D / 8 / kRmWarps > kRmMaxNT) return false;
+  if (dtype != 1 || E > 16 || D % 64 || (D / 8 + kRmWarps - 1) / kRmWarps > kRmMaxNT) return false;
   return rm_layout(D).total <= 232448;
 }
 size_t router_bwd_mma_smem(int D) { return rm_layout(D).total; }
@@ -446,12 +449,14 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
   const RmSmem L = rm_layout(a.D);
   const int D = a.D, E = a.E, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int g = lane >> 2, c = lane & 3, li = lane >> 3, lj = lane & 7;
-  const int nblk = D / 64, ntw = D / 8 / kRmWarps;
+  const int nks = D / 16, ntiles = D / 8;
+  const int tb = w * ntiles / kRmWarps, te = (w + 1) * ntiles / kRmWarps;   // this warp's 8-column tiles
   uint8_t* wg_s = smem + L.wg;
   uint8_t* xs = smem + L.x;
   uint16_t* dlh = reinterpret_cast<uint16_t*>(smem + L.dl);
   uint16_t* dll = dlh + 16 * 16;
   float* lp = reinterpret_cast<float*>(smem + L.lp);
+  float* ls = reinterpret_cast<float*>(smem + L.ls);
   float* dbs = reinterpret_cast<float*>(smem + L.db);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.misc);
   __shared__ float c_s[16];
@@ -473,6 +478,7 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
   }
   if (tid < 16)
     c_s[tid] = tid < E ? a.scale * a.alpha * ((float)E / ((float)a.K * a.T)) * (float)a.counts[tid] / (float)a.T : 0.f;
+  for (int i = tid; i < kRmWarps * 256; i += blockDim.x) dbs[i] = 0.f;
   {  // gate weight rows 0..15 (zero past E), padded stride
     const int vpr = D / 8;
     const uint4* wv = reinterpret_cast<const uint4*>(a.wg);
@@ -489,9 +495,6 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
   for (int i = 0; i < kRmMaxNT; ++i)
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
-  float dbw[16];
-#pragma unroll
-  for (int e = 0; e < 16; ++e) dbw[e] = 0.f;
   bool ok = true;
   for (int j = 0; j < my_rb; ++j) {
     const int st = j % kRmStages;
@@ -500,35 +503,33 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
     // (no status word here: the router backward's scratch has none; a wait that ran out still ends the kernel)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), (j / kRmStages) & 1, nullptr, nullptr, 120));
     const uint32_t xb = smem_u32(xs + (size_t)st * L.stage_bytes);
-    // ---- partial logits of this warp's 64-column blocks
+    // ---- partial logits of this warp's k16 steps
     float la[NTE][4];
 #pragma unroll
     for (int nt = 0; nt < NTE; ++nt)
 #pragma unroll
       for (int q = 0; q < 4; ++q) la[nt][q] = 0.f;
     if (ok) {
-      for (int b = w; b < nblk; b += kRmWarps) {
-        const uint32_t box = xb + b * 2048;
+      for (int sk = w; sk < nks; sk += kRmWarps) {
+        const int ks = sk & 3;
+        const uint32_t box = xb + (sk >> 2) * 2048;
+        uint32_t bb[NTE][2];
+        const int kc = sk * 16 + (li & 1) * 8;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          uint32_t bb[NTE][2];
-          const int kc = b * 64 + ks * 16 + (li & 1) * 8;
-#pragma unroll
-          for (int np = 0; np < NTE; np += 2) {
-            if (np + 1 < NTE) {
-              const int n = (np + (li >> 1)) * 8 + lj;
-              ldsm_x4(wg_base + n * L.wg_stride + kc * 2, bb[np][0], bb[np][1], bb[np + 1][0], bb[np + 1][1]);
-            } else {
-              ldsm_x2(wg_base + (np * 8 + lj) * L.wg_stride + kc * 2, bb[np][0], bb[np][1]);
-            }
+        for (int np = 0; np < NTE; np += 2) {
+          if (np + 1 < NTE) {
+            const int n = (np + (li >> 1)) * 8 + lj;
+            ldsm_x4(wg_base + n * L.wg_stride + kc * 2, bb[np][0], bb[np][1], bb[np + 1][0], bb[np + 1][1]);
+          } else {
+            ldsm_x2(wg_base + (np * 8 + lj) * L.wg_stride + kc * 2, bb[np][0], bb[np][1]);
           }
-          const int row = (li & 1) * 8 + lj;
-          const int chunk = ks * 2 + (li >> 1);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
-#pragma unroll
-          for (int nt = 0; nt < NTE; ++nt) mma_16816<false>(la[nt], a0, a1, a2, a3, bb[nt][0], bb[nt][1]);
         }
+        const int row = (li & 1) * 8 + lj;
+        const int chunk = ks * 2 + (li >> 1);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(box + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NTE; ++nt) mma_16816<false>(la[nt], a0, a1, a2, a3, bb[nt][0], bb[nt][1]);
       }
     }
 #pragma unroll
@@ -545,6 +546,13 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
       fence_async_shared();
       issue(j - 1 + kRmStages);
     }
+    if (tid < 256) {                               // the logits: the warps' partials in warp order
+      float v = 0.f;
+#pragma unroll
+      for (int k = 0; k < kRmWarps; ++k) v += lp[k * 256 + tid];
+      ls[tid] = v;
+    }
+    __syncthreads();
     // ---- softmax and dl of the block's 16 tokens (one lane each)
     if (w == j % kRmWarps && lane < 16) {
       const int t = rb * 16 + lane;
@@ -554,12 +562,7 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
       if (t < a.T && ok) {
         float l[EMAX];
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-          float v = 0.f;
-#pragma unroll
-          for (int k = 0; k < kRmWarps; ++k) v += lp[k * 256 + lane * 16 + e];
-          l[e] = v;
-        }
+        for (int e = 0; e < EMAX; ++e) l[e] = ls[lane * 16 + e];
         float m = -INFINITY;
 #pragma unroll
         for (int e = 0; e < EMAX; ++e)
@@ -585,10 +588,11 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
 #pragma unroll
         for (int e = 0; e < EMAX; ++e)
           if (e < E) { l[e] *= iz; pc += l[e] * dp[e]; }
+        float* db_lane = dbs + (w * 16 + lane) * 16;
 #pragma unroll
         for (int e = 0; e < EMAX; ++e) {
           dl[e] = e < E ? l[e] * (dp[e] - pc) : 0.f;
-          dbw[e] += dl[e];
+          db_lane[e] += dl[e];
         }
       }
       uint32_t* hp = reinterpret_cast<uint32_t*>(dlh + lane * 16);
@@ -605,6 +609,19 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
     __syncthreads();
     // ---- dx = dl Wg and dWg += dl^T x on this warp's 8-column tiles
     if (ok) {
+      const int t0 = rb * 16 + g, t1 = t0 + 8;
+      uint32_t* dxp = reinterpret_cast<uint32_t*>(a.dx);
+      // the experts' part of dx for every tile of the slice, in flight together
+      uint32_t prev[kRmMaxNT][2];
+#pragma unroll
+      for (int i = 0; i < kRmMaxNT; ++i) {
+        prev[i][0] = prev[i][1] = 0u;
+        if (a.dx && a.dx_accumulate && tb + i < te) {
+          const int cc = (tb + i) * 8 + 2 * c;
+          if (t0 < a.T) prev[i][0] = __ldcg(reinterpret_cast<const unsigned int*>(dxp + ((size_t)t0 * D + cc) / 2));
+          if (t1 < a.T) prev[i][1] = __ldcg(reinterpret_cast<const unsigned int*>(dxp + ((size_t)t1 * D + cc) / 2));
+        }
+      }
       uint32_t ah[4], al[4], th[4], tl[4];
       {
         const int r = (lane & 7) + ((lane >> 3) & 1) * 8, cb = (lane >> 4) * 8;   // A = dl [t][e]
@@ -614,12 +631,11 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
         ldsm_x4_t(smem_u32(dlh + tt * 16 + e0), th[0], th[1], th[2], th[3]);
         ldsm_x4_t(smem_u32(dll + tt * 16 + e0), tl[0], tl[1], tl[2], tl[3]);
       }
-      const int t0 = rb * 16 + g, t1 = t0 + 8;
       const int rr = lane & 15;                    // row of the 8x8 tiles this lane addresses
 #pragma unroll
       for (int i = 0; i < kRmMaxNT; ++i) {
-        if (i < ntw) {
-          const int col0 = (w * ntw + i) * 8;
+        if (tb + i < te) {
+          const int col0 = (tb + i) * 8;
           uint32_t b0, b1, x0, x1;
           ldsm_x2_t(wg_base + rr * L.wg_stride + col0 * 2, b0, b1);        // B = Wg [e][d]
           const int blk = col0 >> 6, q = (col0 & 63) >> 3;
@@ -630,27 +646,16 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
           mma_16816<false>(acc[i], th[0], th[1], th[2], th[3], x0, x1);
           mma_16816<false>(acc[i], tl[0], tl[1], tl[2], tl[3], x0, x1);
           if (a.dx) {
-            uint32_t* dxp = reinterpret_cast<uint32_t*>(a.dx);
             const int cc = col0 + 2 * c;
             if (t0 < a.T) {
-              float o0 = d4[0], o1 = d4[1];
-              const size_t ix = ((size_t)t0 * D + cc) / 2;
-              if (a.dx_accumulate) {
-                const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dxp[ix]));
-                o0 += p.x; o1 += p.y;
-              }
-              const __nv_bfloat162 v = __floats2bfloat162_rn(o0, o1);
-              dxp[ix] = *reinterpret_cast<const uint32_t*>(&v);
+              const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&prev[i][0]));
+              const __nv_bfloat162 v = __floats2bfloat162_rn(d4[0] + p.x, d4[1] + p.y);
+              dxp[((size_t)t0 * D + cc) / 2] = *reinterpret_cast<const uint32_t*>(&v);
             }
             if (t1 < a.T) {
-              float o0 = d4[2], o1 = d4[3];
-              const size_t ix = ((size_t)t1 * D + cc) / 2;
-              if (a.dx_accumulate) {
-                const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&dxp[ix]));
-                o0 += p.x; o1 += p.y;
-              }
-              const __nv_bfloat162 v = __floats2bfloat162_rn(o0, o1);
-              dxp[ix] = *reinterpret_cast<const uint32_t*>(&v);
+              const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&prev[i][1]));
+              const __nv_bfloat162 v = __floats2bfloat162_rn(d4[2] + p.x, d4[3] + p.y);
+              dxp[((size_t)t1 * D + cc) / 2] = *reinterpret_cast<const uint32_t*>(&v);
             }
           }
         }
@@ -661,15 +666,11 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
   float* part = a.partials + (size_t)blockIdx.x * E * D;
 #pragma unroll
   for (int i = 0; i < kRmMaxNT; ++i) {
-    if (i < ntw) {
-      const int col = (w * ntw + i) * 8 + 2 * c;
+    if (tb + i < te) {
+      const int col = (tb + i) * 8 + 2 * c;
       if (g < E) { part[(size_t)g * D + col] = acc[i][0]; part[(size_t)g * D + col + 1] = acc[i][1]; }
       if (g + 8 < E) { part[(size_t)(g + 8) * D + col] = acc[i][2]; part[(size_t)(g + 8) * D + col + 1] = acc[i][3]; }
     }
-  }
-  if (lane < 16) {
-#pragma unroll
-    for (int e = 0; e < 16; ++e) dbs[(w * 16 + lane) * 16 + e] = dbw[e];
   }
   __syncthreads();
   if (tid < E) {

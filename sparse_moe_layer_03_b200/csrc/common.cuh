@@ -379,17 +379,6 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void* tmap,
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar), "l"(policy)
       : "memory");
 }
-// Four rows y0..y3 of a 2-D tensor (columns [x, x + box width)) into four consecutive
-// 128-byte rows of shared memory, completing on the pair leader's barrier.  The
-// tensor map's box is one row high.
-__device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const void* tmap, int32_t x, int32_t y0, int32_t y1,
-                                                 int32_t y2, int32_t y3, uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar), "l"(policy)
-      : "memory");
-}
 // arrive on an mbarrier of any CTA of the cluster, releasing this thread's earlier writes
 // (shared::cluster stores included) at cluster scope
 __device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t bar) {
@@ -398,6 +387,15 @@ __device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t bar) {
 // 32-bit store into the shared memory of any CTA of the cluster (shared::cluster address)
 __device__ __forceinline__ void st_shared_cluster_s32(uint32_t addr, int v) {
   asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// 16-byte asynchronous copy global -> shared through the LSU (L2 only), and its groups
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 // remote arrive.expect_tx on a shared::cluster mbarrier address
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar, uint32_t bytes) {

@@ -11,10 +11,13 @@
 // receives its 128 rows of the accumulator.  Every TMA load fills one CTA's own
 // shared memory (nothing is broadcast to several CTAs).
 //
-// Roles per CTA (6 warps): warp 0 = TMA producer (both CTAs; loads complete on
+// Roles per CTA (8 warps): warp 0 = TMA producer (both CTAs; loads complete on
 // the leader's barrier); warp 1 = TMEM allocation (both) and the MMA issuer
 // (leader only); warps 2-5 = epilogue (both CTAs, one per TMEM lane quadrant),
-// storing through TMA.  (More epilogue warps measured slower: the GEMMs run
+// storing through TMA; warps 6-7 = the row gather of a routed problem whose A
+// rows are rows of x picked by row_token (16-byte cp.async into the swizzled
+// stage, reported on the leader's stage barrier two stages later, after a
+// proxy fence), idle otherwise.  (More epilogue warps measured slower: the GEMMs run
 // at the power cap, where extra epilogue activity costs clock.)
 // Synchronisation: the leader's MMA thread commits MMA completion to the
 // "stage empty" and "accumulator full" barriers of both CTAs (one commit per
@@ -45,7 +48,8 @@ namespace moe {
 constexpr int kPairBM = 256;            // rows of a pair tile (128 per CTA)
 constexpr int kPairBK = 64;             // 16-bit elements per 128-byte swizzle row
 constexpr int kPairEpiWarps = 4;          // one per TMEM lane quadrant
-constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
+constexpr int kPairGatherWarps = 2;
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps + 32 * kPairGatherWarps;
 constexpr int kPairSmemLimit = 232448;
 constexpr int kSchedSlots = 4;                                  // tile ids handed out ahead
 constexpr int kSchedConsumers = 2 + 2 * kPairEpiWarps;          // peer producer, MMA issuer, epilogue warps
@@ -195,10 +199,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
   // tiles claimed in order (the folded combine's guarantee of progress) or a fixed order
   const bool dyn = a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr;
+  // the routed A rows come from x through the gather warps (GEMM1 only: fixed tile order)
+  const bool gather_lsu = a.p[0].gather_rows != nullptr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);             // leader: its producer's expect_tx arrive
+      // leader: its producer's expect_tx arrive (+ one arrive per gather warp of both CTAs)
+      mbar_init(smem_u32(&full[s]), gather_lsu ? 1 + 2 * kPairGatherWarps : 1);
       mbar_init(smem_u32(&empty[s]), 1);            // one MMA-completion commit per phase
     }
     for (int i = 0; i < 2; ++i) {
@@ -255,9 +262,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    // Lane 0 loads the tiles.  When the routed problem gathers its A rows, every lane also
-    // issues one tile::gather4 per stage for 4 of this CTA's 128 rows (indices held for the
-    // whole tile), after lane 0 has seen the stage free and posted the expected bytes.
+    // Lane 0 loads the tiles.  When the routed problem gathers its A rows, it loads only B:
+    // the two gather warps copy this CTA's 128 A rows into the stage with cp.async and
+    // arrive on the leader's full barrier themselves.
     const uint64_t pol_w = policy_evict_last();
     // A tiles are reused by every column tile of their row block (consecutive tiles, run
     // side by side): keep them in L2 normally; evict-first sent them back to DRAM 3.5x
@@ -295,18 +302,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       const CUtensorMap* tB = ti.p ? &tb1 : &tb0;
       const int ksplit = pr.ksplit;
       const int nrows = pr.N;
-      const bool gather = pr.gather_rows != nullptr;      // uniform across the warp
-      int g0 = 0, g1 = 0, g2 = 0, g3 = 0;
-      if (gather) {
-        const long long r0 = (long long)ti.row0 + (int)rank * 128 + lane * 4;
-        int g[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int v = __ldg(pr.gather_rows + r0 + u);
-          g[u] = (v >= 0 && v < pr.gather_nrows) ? v : 0;   // padding rows read row 0; never used
-        }
-        g0 = g[0]; g1 = g[1]; g2 = g[2]; g3 = g[3];
-      }
+      const bool gather = pr.gather_rows != nullptr;      // the gather warps bring this tile's A rows
       for (int kb = 0; kb < ti.nk; ++kb) {
         int ok = 1;
         if (lane == 0) ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.status, 501) ? 1 : 0;
@@ -316,7 +312,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         const uint32_t fb_leader = map_to_cta(fb_local, 0);
         uint8_t* sa = stage_base + stage * C::STAGE;
         if (lane == 0) {
-          if (rank == 0) mbar_arrive_expect_tx(fb_local, 2 * C::STAGE);   // both CTAs' bytes
+          if (rank == 0) mbar_arrive_expect_tx(fb_local, gather ? 2 * C::B_BYTES : 2 * C::STAGE);   // both CTAs' TMA bytes
           const int bx = ksplit ? (kb * kPairBK) % ksplit : kb * kPairBK;
           // each CTA holds half of the tile's B rows (a narrower tile's box also brings rows it does not use)
           const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (ti.width / 2);
@@ -341,10 +337,6 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           } else {
             tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tB, bx, by, fb_leader, pol_w);
           }
-        }
-        if (gather) {
-          __syncwarp();
-          tma_gather4_pair(smem_u32(sa) + lane * 4 * 128, tA, kb * kPairBK, g0, g1, g2, g3, fb_leader, pol_a);
         }
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
       }
@@ -374,7 +366,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         // a k16 step advances 32 bytes inside a K-major row, or 16 rows (2048 bytes) of an MN-major tile
         const uint64_t astep = pr.a_mn ? 128 : 2, bstep = pr.b_mn ? 128 : 2;
         for (int kb = 0; kb < ti.nk; ++kb) {
-          if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)) goto mma_out;
+          // gathered rows arrive from both CTAs' gather warps (cluster scope); else TMA only
+          if (!(gather_lsu ? mbar_wait_cluster(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)
+                           : mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)))
+            goto mma_out;
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * C::STAGE);
           const uint64_t adesc = pr.a_mn ? smem_desc_mn_sw128(sa) : smem_desc_sw128(sa);
@@ -400,7 +395,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < 2 + kPairEpiWarps) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     // Each warp owns 32 TMEM lanes = 32 rows of this CTA's half.  Per 128-byte
     // column box it loads the accumulator, applies the epilogue, writes the
@@ -645,6 +640,73 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       }
     }
     if (lane == 0) bulk_wait_all();            // stores done before the CTA may exit
+  } else if (gather_lsu) {
+    // ------------------------------------------------------------ row gather (both CTAs)
+    // Thread u of the two warps copies 16-byte chunk u % 8 of this CTA's rows u / 8 + 8 i
+    // (i < 16) of every stage of a routed tile: row r of the tile is row row_token[r] of x
+    // (padding rows read row 0; their results are never used).  Each stage is one cp.async
+    // group; when a stage's group is kLag groups old it has landed: fence it for the tensor
+    // cores (async proxy) and arrive on the leader's barrier of that stage.  Stages of the
+    // shared problem (A by TMA) are reported too, with empty groups, so every stage's barrier
+    // counts the same arrivals.  kLag < STAGES: a stage is reported before its ring slot is
+    // needed again.
+    constexpr int kLag = 2;
+    const int u = (warp - 2 - kPairEpiWarps) * 32 + lane;
+    const int cq = u & 7, rq = u >> 3;
+    const GemmProblem& pg = a.p[0];
+    const uint16_t* xa = reinterpret_cast<const uint16_t*>(pg.A);
+    const long long ld = pg.K;
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued = 0;
+    auto report = [&](int s) {
+      fence_async_shared();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_release_cluster(map_to_cta(smem_u32(&full[s]), 0));
+    };
+    for (int k = 0;; ++k) {
+      const int tile = cid + k * ncl;
+      if (tile >= pl.total) break;
+      const PairTile ti = pair_decode<BN>(tile, pl, a);
+      const bool mine = ti.p == 0;
+      int rowid[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        int v = 0;
+        if (mine) {
+          v = __ldg(pg.gather_rows + (long long)ti.row0 + (int)rank * 128 + rq + 8 * i);
+          v = (v >= 0 && v < pg.gather_nrows) ? v : 0;
+        }
+        rowid[i] = v;
+      }
+      for (int kb = 0; kb < ti.nk; ++kb) {
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.status, 511) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) {
+          cp_async_wait<0>();                       // nothing of this warp's left in flight
+          goto gather_out;
+        }
+        if (mine) {
+          const uint32_t sa = smem_u32(stage_base + stage * C::STAGE);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int r = rq + 8 * i;
+            cp_async_16(sa + r * 128 + ((cq ^ (r & 7)) << 4), xa + (long long)rowid[i] * ld + kb * kPairBK + cq * 8);
+          }
+        }
+        cp_async_commit();
+        if (issued >= kLag) {
+          cp_async_wait<kLag>();
+          report((stage - kLag + C::STAGES) % C::STAGES);
+        }
+        ++issued;
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    cp_async_wait<0>();
+    for (int n = issued > kLag ? issued - kLag : 0; n < issued; ++n) report(n % C::STAGES);
+  gather_out:;
   }
 done:
   tc_fence_before();

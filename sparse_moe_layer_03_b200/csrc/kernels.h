@@ -197,7 +197,7 @@ struct GemmProblem {
   int ksplit;               // 0, or: B is [K/ksplit blocks][N][ksplit] (shared W2 stack)
   const float* gate;        // per-row gate or null
   // routed problem on the CTA-pair kernel: A row r is row gather_rows[r] of the A tensor (rows
-  // < 0 read row 0), loaded with TMA tile::gather4 (the A tensor map's box is one row high)
+  // < 0 read row 0), copied into the swizzled A stage by the kernel's cp.async gather warps
   const int32_t* gather_rows;
   int gather_nrows;         // rows of the A tensor
 };

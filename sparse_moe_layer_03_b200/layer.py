@@ -58,8 +58,7 @@ class LayerShape:
     gemm_impl: str = "auto"
     seq_len: int = 0          # tokens per image for the balance loss (0 = the whole call)
     fuse_combine: bool = True  # fold the combine into the shared experts' GEMM2 where supported
-    gather_rows: bool = False  # GEMM1 gathers its routed rows from x by TMA gather4 (no x_perm); measured
-                               # slower at XL (GEMM1 2.37 ms against 1.11 ms): off by default
+    gather_rows: bool = False  # GEMM1 gathers its routed rows from x itself (no x_perm)
     gemm_pairs: int = 0        # CTA pairs the tensor-core GEMMs may occupy at once (0 = as many as fit)
 
 
@@ -105,7 +104,8 @@ class MoELayer:
         self.pos = torch.empty((T, kmax), dtype=i32, device=dev)
         self.row_token = torch.empty((self.R,), dtype=i32, device=dev)
         self.row_gate = torch.empty((self.R,), dtype=f32, device=dev)
-        # GEMM1 reads the routed rows of x itself (TMA gather4) on the 16-bit CTA-pair path: no x_perm
+        # GEMM1 reads the routed rows of x itself (cp.async gather warps) on the 16-bit CTA-pair path:
+        # no x_perm
         self.gathered = bool(s.gather_rows and s.dtype in ("bf16", "f16") and s.gemm_impl == "auto")
         self.x_perm = None if self.gathered else torch.empty((self.R, s.D), dtype=dt, device=dev)
         self.h_perm = torch.empty((self.R, s.H), dtype=dt, device=dev)

@@ -333,7 +333,7 @@ def test_gathered_gemm1_full_size_xl():
 
 @pytest.mark.parametrize("routing", ["topk", "race"])
 def test_gathered_gemm1_rows_equal_permuted_copy(routing):
-    # GEMM1 reading its rows from x by TMA gather4 computes bit for bit what it computes on x_perm
+    # GEMM1 reading its rows from x (cp.async gather warps) computes bit for bit what it computes on x_perm
     from sparse_moe_layer_03_b200.layer import LayerShape, MoELayer
     w = I.small_workload(1500, 384, 768, 16 if routing == "race" else 8, 2, 2, "bf16", routing, seed=61)
     inp = I.make_inputs(w, bias_std=0.2)

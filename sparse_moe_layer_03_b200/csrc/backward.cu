@@ -402,14 +402,17 @@ __global__ void __launch_bounds__(kRbThreads, 2) router_bwd_pass_kernel(BalanceG
 // Rows of 16 tokens come in by TMA (two half-row boxes per stage, 128-byte swizzle, a ring of
 // kRmStages stages refilled as soon as every warp has left the block).  Per block: each of the
 // 16 warps takes every 16th k16 step for the partial logits x Wg^T (as the forward router); the
-// first 256 threads add the 16 partials in warp order; warp (block mod 16) computes softmax and
-// dl for the 16 tokens (one lane each), written to shared memory as two bf16 parts (dl = hi + lo,
-// about 16 bits of mantissa); then every warp, on its own contiguous slice of the D/8 8-column
+// first 256 threads add the 16 partials in warp order; one thread per (token, expert) computes
+// softmax and dl (the token's lanes reduce by shuffles), written to shared memory as two bf16
+// parts (dl = hi + lo, about 16 bits of mantissa); then every warp, on its own contiguous slice of the D/8 8-column
 // tiles, forms dx = dl Wg (two MMAs, written to global memory; the experts' part, loaded first
 // for all of the slice's tiles at once, added when asked) and accumulates dWg += dl^T x in
 // registers over all of the CTA's blocks (x read straight from the stage with transposed
 // ldmatrix).  Sixteen warps per SM keep enough MMAs and loads in flight: with four, the SM
 // waited on single dependences most of the time.  E <= 16 (zero-padded to 16), D <= 1152.
+// With E <= 8 the two parts of dl share one MMA's k = 16: dl is held as [hi | lo] per token and
+// the gate weight as [Wg; Wg], so dx takes one MMA per tile, and dWg's tile gets the hi part in
+// rows 0-7 and the lo part in rows 8-15 (added when the partials are written).
 constexpr int kRmWarps = 16;
 constexpr int kRmStages = 4;
 constexpr int kRmMaxNT = 9;                       // 8-column tiles per warp: ceil(D / 8 / kRmWarps)
@@ -429,7 +432,7 @@ __host__ __device__ inline RmSmem rm_layout(int D) {
   L.lp = L.dl + 2 * 16 * 16 * 2;                   // dl hi and lo, [16 tokens][16 experts] bf16 each
   L.ls = L.lp + (size_t)kRmWarps * 16 * 16 * 4;    // partial logits [warp][token][expert] fp32
   L.db = L.ls + 16 * 16 * 4;                       // logits [token][expert] fp32
-  L.misc = L.db + (size_t)kRmWarps * 16 * 16 * 4; // db per selecting lane [warp][lane][expert]
+  L.misc = L.db + 16 * 16 * 4;                     // db per (token, expert) thread
   L.total = L.misc + 256 + 1024;                   // barriers; 1 KB alignment slack
   return L;
 }
@@ -444,6 +447,7 @@ template <int EMAX>
 __global__ void __launch_bounds__(kRmWarps * 32, 1)
 router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArgs a) {
   constexpr int NTE = EMAX / 8;                    // expert tiles of the logits
+  constexpr bool PACK = EMAX == 8;                 // hi and lo parts of dl in one k16 step
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const RmSmem L = rm_layout(a.D);
@@ -478,13 +482,14 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
   }
   if (tid < 16)
     c_s[tid] = tid < E ? a.scale * a.alpha * ((float)E / ((float)a.K * a.T)) * (float)a.counts[tid] / (float)a.T : 0.f;
-  for (int i = tid; i < kRmWarps * 256; i += blockDim.x) dbs[i] = 0.f;
-  {  // gate weight rows 0..15 (zero past E), padded stride
+  if (tid < 256) dbs[tid] = 0.f;
+  {  // gate weight rows 0..15 (zero past E; rows 8..15 repeat rows 0..7 when packed), padded stride
     const int vpr = D / 8;
     const uint4* wv = reinterpret_cast<const uint4*>(a.wg);
     for (int i = tid; i < 16 * vpr; i += blockDim.x) {
       const int e = i / vpr, v = i % vpr;
-      const uint4 val = e < E ? __ldg(wv + (size_t)e * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
+      const int src = PACK ? (e & 7) : e;
+      const uint4 val = src < E ? __ldg(wv + (size_t)src * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
       *reinterpret_cast<uint4*>(wg_s + (size_t)e * L.wg_stride + v * 16) = val;
     }
   }
@@ -553,129 +558,122 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
       ls[tid] = v;
     }
     __syncthreads();
-    // ---- softmax and dl of the block's 16 tokens (one lane each)
-    if (w == j % kRmWarps && lane < 16) {
-      const int t = rb * 16 + lane;
-      float dl[16];
+    // ---- softmax and dl of the block's 16 tokens: thread (token, expert) of the first 16 * EMAX,
+    // the token's EMAX lanes reducing by shuffles
+    if (tid < 16 * EMAX) {
+      const int tl_ = tid / EMAX, e = tid % EMAX;
+      const int t = rb * 16 + tl_;
+      const bool act = e < E;
+      float l = ls[tl_ * 16 + e] + (act && a.bias ? a.bias[e] : 0.f);
+      float m = act ? l : -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) dl[e] = 0.f;
-      if (t < a.T && ok) {
-        float l[EMAX];
+      for (int o = 1; o < EMAX; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float pe = act ? expf(l - m) : 0.f;
+      float z = pe;
 #pragma unroll
-        for (int e = 0; e < EMAX; ++e) l[e] = ls[lane * 16 + e];
-        float m = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e)
-          if (e < E) { l[e] += a.bias ? a.bias[e] : 0.f; m = fmaxf(m, l[e]); }
-        float z = 0.f;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e)
-          if (e < E) { l[e] = expf(l[e] - m); z += l[e]; }
-        const float iz = 1.0f / z;
-        float dp[EMAX];
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e) dp[e] = c_s[e];
-        if (a.dgate) {
-          const int ns = a.n_sel ? a.n_sel[t] : a.K;
-          for (int k = 0; k < a.Kmax && k < ns; ++k) {
-            const int sel = a.topk_idx[(size_t)t * a.Kmax + k];
-            const float gk = a.dgate[(size_t)t * a.Kmax + k];
-#pragma unroll
-            for (int e = 0; e < EMAX; ++e) dp[e] += e == sel ? gk : 0.f;
-          }
-        }
-        float pc = 0.f;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e)
-          if (e < E) { l[e] *= iz; pc += l[e] * dp[e]; }
-        float* db_lane = dbs + (w * 16 + lane) * 16;
-#pragma unroll
-        for (int e = 0; e < EMAX; ++e) {
-          dl[e] = e < E ? l[e] * (dp[e] - pc) : 0.f;
-          db_lane[e] += dl[e];
-        }
+      for (int o = 1; o < EMAX; o <<= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      pe *= 1.0f / z;
+      float dp = c_s[e];
+      const bool valid = t < a.T && ok;
+      if (a.dgate && valid) {
+        const int ns = a.n_sel ? a.n_sel[t] : a.K;
+        for (int k = 0; k < a.Kmax && k < ns; ++k)
+          if (a.topk_idx[(size_t)t * a.Kmax + k] == e) dp += a.dgate[(size_t)t * a.Kmax + k];
       }
-      uint32_t* hp = reinterpret_cast<uint32_t*>(dlh + lane * 16);
-      uint32_t* lo = reinterpret_cast<uint32_t*>(dll + lane * 16);
+      float pc = pe * dp;
 #pragma unroll
-      for (int e = 0; e < 16; e += 2) {
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(dl[e], dl[e + 1]);
-        const float2 hf = __bfloat1622float2(h2);
-        const __nv_bfloat162 l2 = __floats2bfloat162_rn(dl[e] - hf.x, dl[e + 1] - hf.y);
-        hp[e / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-        lo[e / 2] = *reinterpret_cast<const uint32_t*>(&l2);
-      }
+      for (int o = 1; o < EMAX; o <<= 1) pc += __shfl_xor_sync(0xffffffffu, pc, o);
+      const float dl = (act && valid) ? pe * (dp - pc) : 0.f;
+      dbs[tid] += dl;
+      const __nv_bfloat16 h = __float2bfloat16_rn(dl);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(dl - __bfloat162float(h));
+      // packed: [hi of experts 0..7 | lo of experts 0..7] in one row; else hi and lo rows apart
+      reinterpret_cast<__nv_bfloat16*>(dlh)[tl_ * 16 + e] = h;
+      reinterpret_cast<__nv_bfloat16*>(PACK ? dlh + 8 : dll)[tl_ * 16 + e] = lo;
     }
     __syncthreads();
     // ---- dx = dl Wg and dWg += dl^T x on this warp's 8-column tiles
     if (ok) {
       const int t0 = rb * 16 + g, t1 = t0 + 8;
-      uint32_t* dxp = reinterpret_cast<uint32_t*>(a.dx);
+      const bool v0 = t0 < a.T, v1 = t1 < a.T;
+      // rows t0 and t1 of dx, as bf16 pairs; this lane's pair of each tile sits at (tile * 8 + 2c) / 2
+      uint32_t* dx0 = reinterpret_cast<uint32_t*>(a.dx) + ((size_t)t0 * D + 2 * c) / 2;
+      uint32_t* dx1 = dx0 + (size_t)8 * D / 2;
       // the experts' part of dx for every tile of the slice, in flight together
       uint32_t prev[kRmMaxNT][2];
 #pragma unroll
       for (int i = 0; i < kRmMaxNT; ++i) {
         prev[i][0] = prev[i][1] = 0u;
         if (a.dx && a.dx_accumulate && tb + i < te) {
-          const int cc = (tb + i) * 8 + 2 * c;
-          if (t0 < a.T) prev[i][0] = __ldcg(reinterpret_cast<const unsigned int*>(dxp + ((size_t)t0 * D + cc) / 2));
-          if (t1 < a.T) prev[i][1] = __ldcg(reinterpret_cast<const unsigned int*>(dxp + ((size_t)t1 * D + cc) / 2));
+          if (v0) prev[i][0] = __ldcg(reinterpret_cast<const unsigned int*>(dx0 + (tb + i) * 4));
+          if (v1) prev[i][1] = __ldcg(reinterpret_cast<const unsigned int*>(dx1 + (tb + i) * 4));
         }
       }
       uint32_t ah[4], al[4], th[4], tl[4];
       {
         const int r = (lane & 7) + ((lane >> 3) & 1) * 8, cb = (lane >> 4) * 8;   // A = dl [t][e]
         ldsm_x4(smem_u32(dlh + r * 16 + cb), ah[0], ah[1], ah[2], ah[3]);
-        ldsm_x4(smem_u32(dll + r * 16 + cb), al[0], al[1], al[2], al[3]);
         const int mi = lane >> 3, tt = (mi >> 1) * 8 + (lane & 7), e0 = (mi & 1) * 8;  // A = dl^T [e][t]
         ldsm_x4_t(smem_u32(dlh + tt * 16 + e0), th[0], th[1], th[2], th[3]);
-        ldsm_x4_t(smem_u32(dll + tt * 16 + e0), tl[0], tl[1], tl[2], tl[3]);
+        if (!PACK) {
+          ldsm_x4(smem_u32(dll + r * 16 + cb), al[0], al[1], al[2], al[3]);
+          ldsm_x4_t(smem_u32(dll + tt * 16 + e0), tl[0], tl[1], tl[2], tl[3]);
+        }
       }
       const int rr = lane & 15;                    // row of the 8x8 tiles this lane addresses
+      const uint32_t wrow = wg_base + rr * L.wg_stride;
+      const uint32_t xrow = xb + rr * 128;
 #pragma unroll
       for (int i = 0; i < kRmMaxNT; ++i) {
         if (tb + i < te) {
-          const int col0 = (tb + i) * 8;
+          const int tile = tb + i;
           uint32_t b0, b1, x0, x1;
-          ldsm_x2_t(wg_base + rr * L.wg_stride + col0 * 2, b0, b1);        // B = Wg [e][d]
-          const int blk = col0 >> 6, q = (col0 & 63) >> 3;
-          ldsm_x2_t(xb + blk * 2048 + rr * 128 + ((q ^ (rr & 7)) << 4), x0, x1);   // B = x [t][d]
+          ldsm_x2_t(wrow + tile * 16, b0, b1);                                    // B = Wg [e][d]
+          ldsm_x2_t(xrow + (tile >> 3) * 2048 + (((tile & 7) ^ (rr & 7)) << 4), x0, x1);   // B = x [t][d]
           float d4[4] = {0.f, 0.f, 0.f, 0.f};
           mma_16816<false>(d4, ah[0], ah[1], ah[2], ah[3], b0, b1);
-          mma_16816<false>(d4, al[0], al[1], al[2], al[3], b0, b1);
           mma_16816<false>(acc[i], th[0], th[1], th[2], th[3], x0, x1);
-          mma_16816<false>(acc[i], tl[0], tl[1], tl[2], tl[3], x0, x1);
+          if (!PACK) {
+            mma_16816<false>(d4, al[0], al[1], al[2], al[3], b0, b1);
+            mma_16816<false>(acc[i], tl[0], tl[1], tl[2], tl[3], x0, x1);
+          }
           if (a.dx) {
-            const int cc = col0 + 2 * c;
-            if (t0 < a.T) {
+            if (v0) {
               const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&prev[i][0]));
               const __nv_bfloat162 v = __floats2bfloat162_rn(d4[0] + p.x, d4[1] + p.y);
-              dxp[((size_t)t0 * D + cc) / 2] = *reinterpret_cast<const uint32_t*>(&v);
+              dx0[tile * 4] = *reinterpret_cast<const uint32_t*>(&v);
             }
-            if (t1 < a.T) {
+            if (v1) {
               const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&prev[i][1]));
               const __nv_bfloat162 v = __floats2bfloat162_rn(d4[2] + p.x, d4[3] + p.y);
-              dxp[((size_t)t1 * D + cc) / 2] = *reinterpret_cast<const uint32_t*>(&v);
+              dx1[tile * 4] = *reinterpret_cast<const uint32_t*>(&v);
             }
           }
         }
       }
     }
   }
-  // ---- this CTA's partial dWg (rows e = g, g + 8 of its fragments) and db (selecting lanes, in order)
+  // ---- this CTA's partial dWg (rows e = g, g + 8 of its fragments) and db (tokens in order)
   float* part = a.partials + (size_t)blockIdx.x * E * D;
 #pragma unroll
   for (int i = 0; i < kRmMaxNT; ++i) {
     if (tb + i < te) {
       const int col = (tb + i) * 8 + 2 * c;
-      if (g < E) { part[(size_t)g * D + col] = acc[i][0]; part[(size_t)g * D + col + 1] = acc[i][1]; }
-      if (g + 8 < E) { part[(size_t)(g + 8) * D + col] = acc[i][2]; part[(size_t)(g + 8) * D + col + 1] = acc[i][3]; }
+      if (PACK) {                                  // rows g (hi part) and g + 8 (lo part) of expert g
+        if (g < E) {
+          part[(size_t)g * D + col] = acc[i][0] + acc[i][2];
+          part[(size_t)g * D + col + 1] = acc[i][1] + acc[i][3];
+        }
+      } else {
+        if (g < E) { part[(size_t)g * D + col] = acc[i][0]; part[(size_t)g * D + col + 1] = acc[i][1]; }
+        if (g + 8 < E) { part[(size_t)(g + 8) * D + col] = acc[i][2]; part[(size_t)(g + 8) * D + col + 1] = acc[i][3]; }
+      }
     }
   }
   __syncthreads();
-  if (tid < E) {
+  if (tid < E) {                                   // thread (token, expert) slots of the expert, in order
     float sdb = 0.f;
-    for (int k = 0; k < kRmWarps * 16; ++k) sdb += dbs[k * 16 + tid];
+    for (int k = 0; k < 16; ++k) sdb += dbs[k * EMAX + tid];
     a.db_part[(size_t)blockIdx.x * E + tid] = sdb;
   }
 }

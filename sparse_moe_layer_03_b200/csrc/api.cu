@@ -691,7 +691,7 @@ EbLayout eb_layout(const moe_config_t* c) {
   L.du_perm = take(R * H * eb);
   L.du_sh = take(T * ns * H * eb);
   L.dx_perm = take(R * D * eb);
-  L.dg_stride = (int)((H + 255) / 256);
+  L.dg_stride = (int)((H + 255) / 256) * kPairEpiSplit;   // per 256-column tile and epilogue warp
   L.dg = take(R * (size_t)L.dg_stride * 4);
   size_t cmax = D > H ? D : H;
   if (ns * H > cmax) cmax = ns * H;

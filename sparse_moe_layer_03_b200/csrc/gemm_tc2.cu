@@ -11,14 +11,13 @@
 // receives its 128 rows of the accumulator.  Every TMA load fills one CTA's own
 // shared memory (nothing is broadcast to several CTAs).
 //
-// Roles per CTA (8 warps): warp 0 = TMA producer (both CTAs; loads complete on
+// Roles per CTA (6 warps): warp 0 = TMA producer (both CTAs; loads complete on
 // the leader's barrier); warp 1 = TMEM allocation (both) and the MMA issuer
 // (leader only); warps 2-5 = epilogue (both CTAs, one per TMEM lane quadrant),
-// storing through TMA; warps 6-7 = the row gather of a routed problem whose A
-// rows are rows of x picked by row_token (16-byte cp.async into the swizzled
-// stage, reported on the leader's stage barrier two stages later, after a
-// proxy fence), idle otherwise.  (More epilogue warps measured slower: the GEMMs run
-// at the power cap, where extra epilogue activity costs clock.)
+// storing through TMA.  The gathering instantiation adds warps 6-7: the row
+// gather of a routed problem whose A rows are rows of x picked by row_token
+// (16-byte cp.async into the swizzled stage, reported on the leader's stage
+// barrier two stages later, after a proxy fence).
 // Synchronisation: the leader's MMA thread commits MMA completion to the
 // "stage empty" and "accumulator full" barriers of both CTAs (one commit per
 // CTA, by shared::cluster address); every epilogue warp of both CTAs arrives
@@ -47,9 +46,16 @@ namespace moe {
 
 constexpr int kPairBM = 256;            // rows of a pair tile (128 per CTA)
 constexpr int kPairBK = 64;             // 16-bit elements per 128-byte swizzle row
-constexpr int kPairEpiWarps = 4;          // one per TMEM lane quadrant
+constexpr int kPairEpiWarps = 4 * kPairEpiSplit;   // kPairEpiSplit per TMEM lane quadrant, each on its own column boxes
 constexpr int kPairGatherWarps = 2;
-constexpr int kPairThreads = 64 + 32 * kPairEpiWarps + 32 * kPairGatherWarps;
+// What one instantiation can do, fixed at compile time so that a launch carries only the code
+// its problems use (the forward GEMMs measured 4-10% slower when compiled together with the
+// backward's and the gather's paths):
+constexpr int kFeatClaim = 1;             // tiles claimed in order (the folded combine)
+constexpr int kFeatGather = 2;            // routed A rows copied from x by the gather warps
+constexpr int kFeatBwd = 4;               // MN-major operands, weight-gradient problems, fp32 output, GELU backward
+template <int F>
+constexpr int pair_threads() { return 64 + 32 * kPairEpiWarps + ((F & kFeatGather) ? 32 * kPairGatherWarps : 0); }
 constexpr int kPairSmemLimit = 232448;
 constexpr int kSchedSlots = 4;                                  // tile ids handed out ahead
 constexpr int kSchedConsumers = 2 + 2 * kPairEpiWarps;          // peer producer, MMA issuer, epilogue warps
@@ -63,6 +69,8 @@ struct PairCfg {
   // (a single buffer, trading 16 KB for one more operand stage, measured 1.8x slower on GEMM1)
   static constexpr int EPI_BYTES = kPairEpiWarps * 2 * 4096;
   // keep 4 KB of the 227 KB for barriers, the 1 KB alignment slack and static shared memory
+  // (with 4 epilogue warps this gives 5 stages; a 6th, which fits in 3 KB, measured 3% slower
+  // on GEMM2 + combine at XL)
   static constexpr int FIT = (kPairSmemLimit - 4096 - EPI_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 8 ? 8 : FIT;
   static constexpr int SMEM = STAGES * STAGE + EPI_BYTES + 2048;
@@ -86,7 +94,7 @@ struct PairTile {
   int bk0;            // first K row of an MN-major B (an expert's block of the weights, or k0)
 };
 
-template <int BN>
+template <int BN, bool BWD>
 __device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, const GemmArgs& a) {
   PairTile ti;
   int t = tile;
@@ -95,7 +103,7 @@ __device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, co
   const GemmProblem& pr = a.p[ti.p];
   ti.k0 = 0;
   ti.bk0 = 0;
-  if (pr.kgrouped) {
+  if (BWD && pr.kgrouped) {
     // weight gradient: tiles of expert e's [M, N] output; the reduction runs over the expert's
     // rows of the permuted buffers (a dense problem has one segment of K rows)
     const int per = pl.nm[ti.p] * pl.nn[ti.p];
@@ -172,8 +180,8 @@ __device__ __forceinline__ int sched_claim(unsigned int* ctr, int total) {
   return t < total ? t : -1;
 }
 
-template <int BN, typename S>
-__global__ void __launch_bounds__(kPairThreads, 1)
+template <int BN, typename S, int F>
+__global__ void __launch_bounds__(pair_threads<F>(), 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
                  const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
                  const __grid_constant__ CUtensorMap to0, const __grid_constant__ CUtensorMap to1, GemmArgs a) {
@@ -198,9 +206,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
   const uint32_t rank = cluster_ctarank();          // 0 = leader of the pair
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
   // tiles claimed in order (the folded combine's guarantee of progress) or a fixed order
-  const bool dyn = a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr;
+  constexpr bool kClaim = (F & kFeatClaim) != 0, kGather = (F & kFeatGather) != 0, kBwd = (F & kFeatBwd) != 0;
+  const bool dyn = kClaim && a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr;
   // the routed A rows come from x through the gather warps (GEMM1 only: fixed tile order)
-  const bool gather_lsu = a.p[0].gather_rows != nullptr;
+  const bool gather_lsu = kGather && a.p[0].gather_rows != nullptr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -237,7 +246,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       pl.nrem[q] = pr.N % BN;
       pl.nn[q] = pl.nfull[q] + (pl.nrem[q] ? 1 : 0);
       pl.nm[q] = (pr.M + kPairBM - 1) / kPairBM;
-      if (pr.kgrouped) {
+      if (kBwd && pr.kgrouped) {
         pl.ntiles[q] = (pr.routed ? (bad ? 0 : a.E) : 1) * pl.nm[q] * pl.nn[q];
         continue;
       }
@@ -296,13 +305,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       tile = __shfl_sync(0xffffffffu, tile, 0);
       if (!ok) { alive = false; break; }
       if (tile < 0) break;
-      const PairTile ti = pair_decode<BN>(tile, pl, a);
+      const PairTile ti = pair_decode<BN, kBwd>(tile, pl, a);
       const GemmProblem& pr = a.p[ti.p];
       const CUtensorMap* tA = ti.p ? &ta1 : &ta0;
       const CUtensorMap* tB = ti.p ? &tb1 : &tb0;
       const int ksplit = pr.ksplit;
       const int nrows = pr.N;
-      const bool gather = pr.gather_rows != nullptr;      // the gather warps bring this tile's A rows
+      const bool gather = kGather && pr.gather_rows != nullptr;   // the gather warps bring this tile's A rows
       for (int kb = 0; kb < ti.nk; ++kb) {
         int ok = 1;
         if (lane == 0) ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.status, 501) ? 1 : 0;
@@ -316,7 +325,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           const int bx = ksplit ? (kb * kPairBK) % ksplit : kb * kPairBK;
           // each CTA holds half of the tile's B rows (a narrower tile's box also brings rows it does not use)
           const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (ti.width / 2);
-          if (pr.a_mn) {
+          if (kBwd && pr.a_mn) {
             // A held [K rows, M columns]: this CTA's 128 M columns as two 64-column boxes of 64 K rows
             const int ax = ti.row0 + (int)rank * 128, ay = ti.k0 + kb * kPairBK;
             tma_load_2d_pair(smem_u32(sa), tA, ax, ay, fb_leader, pol_a);
@@ -324,7 +333,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           } else if (!gather) {
             tma_load_2d_pair(smem_u32(sa), tA, kb * kPairBK, ti.row0 + (int)rank * 128, fb_leader, pol_a);
           }
-          if (pr.b_mn) {
+          if (kBwd && pr.b_mn) {
             // B held [K rows, N columns]: this CTA's half of the tile's columns as two 64-column boxes
             // (a narrower tile's second box brings columns it does not use, zeros past the tensor)
 #pragma unroll
@@ -355,16 +364,17 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         if (dyn) tile = sched_take(sched_full, sched_empty, sched_tile, sn, rank, abort_flag, a.status, 509);
         else if (tile >= pl.total) tile = -1;
         if (tile < 0) break;
-        const PairTile ti = pair_decode<BN>(tile, pl, a);
+        const PairTile ti = pair_decode<BN, kBwd>(tile, pl, a);
         const int acc = local & 1;
         const uint32_t accph = (local >> 1) & 1;
         if (!mbar_wait(smem_u32(&acc_empty[acc]), accph ^ 1u, abort_flag, a.status, 502)) goto mma_out;
         tc_fence_after();
         const uint32_t d = tmem_base + acc * BN;
         const GemmProblem& pr = a.p[ti.p];
-        const uint32_t idesc = idesc_f16kind_f32(kPairBM, ti.width, S::kFmt) | idesc_major_bits(pr.a_mn, pr.b_mn);
+        const bool amn = kBwd && pr.a_mn, bmn = kBwd && pr.b_mn;
+        const uint32_t idesc = idesc_f16kind_f32(kPairBM, ti.width, S::kFmt) | (kBwd ? idesc_major_bits(amn, bmn) : 0u);
         // a k16 step advances 32 bytes inside a K-major row, or 16 rows (2048 bytes) of an MN-major tile
-        const uint64_t astep = pr.a_mn ? 128 : 2, bstep = pr.b_mn ? 128 : 2;
+        const uint64_t astep = amn ? 128 : 2, bstep = bmn ? 128 : 2;
         for (int kb = 0; kb < ti.nk; ++kb) {
           // gathered rows arrive from both CTAs' gather warps (cluster scope); else TMA only
           if (!(gather_lsu ? mbar_wait_cluster(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)
@@ -372,8 +382,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
             goto mma_out;
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * C::STAGE);
-          const uint64_t adesc = pr.a_mn ? smem_desc_mn_sw128(sa) : smem_desc_sw128(sa);
-          const uint64_t bdesc = pr.b_mn ? smem_desc_mn_sw128(sa + C::A_BYTES) : smem_desc_sw128(sa + C::A_BYTES);
+          const uint64_t adesc = amn ? smem_desc_mn_sw128(sa) : smem_desc_sw128(sa);
+          const uint64_t bdesc = bmn ? smem_desc_mn_sw128(sa + C::A_BYTES) : smem_desc_sw128(sa + C::A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < kPairBK / 16; ++kk)
             umma_kindf16_pair(d, adesc + astep * kk, bdesc + bstep * kk, idesc, (kb | kk) ? 1u : 0u);
@@ -397,11 +407,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     __syncwarp();
   } else if (warp < 2 + kPairEpiWarps) {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    // Each warp owns 32 TMEM lanes = 32 rows of this CTA's half.  Per 128-byte
-    // column box it loads the accumulator, applies the epilogue, writes the
-    // 32 x 128-byte box into a swizzled shared buffer and hands it to a TMA
-    // store (two buffers per warp, so a store overlaps the next box).
+    // Each warp owns 32 TMEM lanes = 32 rows of this CTA's half, and every
+    // kPairEpiSplit-th column box of the tile (the warps of one lane quadrant
+    // share its boxes).  Per 128-byte column box it loads the accumulator,
+    // applies the epilogue, writes the 32 x 128-byte box into a swizzled shared
+    // buffer and hands it to a TMA store (two buffers per warp, so a store
+    // overlaps the next box).
     const int q = warp & 3;
+    const int grp = (warp - 2) >> 2;               // which of the quadrant's warps
     const int r = q * 32 + lane;                   // row inside this CTA's 128-row half
     const uint32_t acc_empty_leader0 = map_to_cta(smem_u32(&acc_empty[0]), 0);
     const uint32_t acc_empty_leader1 = map_to_cta(smem_u32(&acc_empty[1]), 0);
@@ -426,7 +439,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         tile = -1;
       }
       if (tile < 0) break;
-      const PairTile ti = pair_decode<BN>(tile, pl, a);
+      const PairTile ti = pair_decode<BN, kBwd>(tile, pl, a);
       const GemmProblem& pr = a.p[ti.p];
       const CUtensorMap* tO = ti.p ? &to1 : &to0;
       const int acc = local & 1;
@@ -442,7 +455,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           pr.bias ? reinterpret_cast<const uint16_t*>(pr.bias) + (long long)ti.e * pr.bias_stride : nullptr;
       constexpr int box_cols = 64;                          // 128 bytes of 16-bit h or y
       // tanh GELU, erf GELU, gate, the combine (routed rows + shared output), or the GELU backward
-      const int mode = pr.epi == 0 ? (a.act == 1 ? 1 : 0) : (pr.epi == 2 ? 3 : (pr.epi == 4 ? 4 : 2));
+      const int mode = pr.epi == 0 ? (a.act == 1 ? 1 : 0) : (pr.epi == 2 ? 3 : ((kBwd && pr.epi == 4) ? 4 : 2));
       float dgacc = 0.f;
       int ns = 0;
       const int32_t* prow = nullptr;
@@ -466,12 +479,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         }
       }
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-      if (pr.out_f32) {
+      if (kBwd && pr.out_f32) {
         // weight gradients: 32 fp32 columns per box through the 3-D output map [z, M, N] (rows past
         // M are clipped by the map); a tile with no reduction rows (an expert that took no token)
         // stores zeros
 #pragma unroll 1
-        for (int c0 = 0; c0 < ti.width; c0 += 32) {
+        for (int c0 = grp * 32; c0 < ti.width; c0 += 32 * kPairEpiSplit) {
           uint32_t v[32];
           if (ti.nk > 0) {
             tmem_ld_32x32b_x32(tbase + c0, v);
@@ -501,7 +514,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         }
       } else {
 #pragma unroll 1
-      for (int c0 = 0; c0 < ti.width; c0 += box_cols) {
+      for (int c0 = grp * box_cols; c0 < ti.width; c0 += box_cols * kPairEpiSplit) {
         uint4 o[8];
         uint32_t vv[2][32];
         tmem_ld_32x32b_x32(tbase + c0, vv[0]);
@@ -511,21 +524,21 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         for (int half = 0; half < 2; ++half) {
           if (half * 32 >= box_cols) break;
           const int cc = c0 + half * 32;
-          const uint32_t* v = vv[half];
+          uint32_t* v = vv[half];
           const int col0 = ti.n0 + cc;
-          float b[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) b[j] = 0.f;
           if (bias) {
-            for (int br = 0; br < pr.bias_rows; ++br) {
-              const uint4* bp = reinterpret_cast<const uint4*>(bias + (long long)br * pr.N + col0);
+            // acc + (the bias rows' sum, in row order): one fp32 add per element, kept in v
 #pragma unroll
-              for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 4; ++u) {
+              float bs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+              for (int br = 0; br < pr.bias_rows; ++br) {
                 float t8[8];
-                S::x8_to_f32(__ldg(bp + u), t8);
+                S::x8_to_f32(__ldg(reinterpret_cast<const uint4*>(bias + (long long)br * pr.N + col0) + u), t8);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) b[8 * u + j] += t8[j];
+                for (int j = 0; j < 8; ++j) bs[j] += t8[j];
               }
+#pragma unroll
+              for (int j = 0; j < 8; ++j) v[8 * u + j] = __float_as_uint(__uint_as_float(v[8 * u + j]) + bs[j]);
             }
           }
           // GEMM1: gelu(acc + b1); GEMM2: gate * (acc + b2); both rounded once to 16 bits.  The
@@ -534,18 +547,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           if (mode == 0) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = S::pack2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 0),
-                                      gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], 0));
+              ow[j / 2] = S::pack2(gelu_act<true>(__uint_as_float(v[j]), 0), gelu_act<true>(__uint_as_float(v[j + 1]), 0));
           } else if (mode == 1) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = S::pack2(gelu_act<true>(__uint_as_float(v[j]) + b[j], 1),
-                                      gelu_act<true>(__uint_as_float(v[j + 1]) + b[j + 1], 1));
+              ow[j / 2] = S::pack2(gelu_act<true>(__uint_as_float(v[j]), 1), gelu_act<true>(__uint_as_float(v[j + 1]), 1));
           } else if (mode == 2) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-              ow[j / 2] = S::pack2((__uint_as_float(v[j]) + b[j]) * gate, (__uint_as_float(v[j + 1]) + b[j + 1]) * gate);
-          } else if (mode == 4) {
+              ow[j / 2] = S::pack2(__uint_as_float(v[j]) * gate, __uint_as_float(v[j + 1]) * gate);
+          } else if (kBwd && mode == 4) {
             // GELU backward: acc = dY W (ungated), u the stored pre-activation of these columns;
             // dU = gate * acc * gelu'(u) (zero on padding rows), and the row's sum of acc * gelu(u)
             float uf[32];
@@ -587,7 +598,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
               }
             }
 #pragma unroll
-            for (int j = 0; j < 32; ++j) y[j] += __uint_as_float(v[j]) + b[j];
+            for (int j = 0; j < 32; ++j) y[j] += __uint_as_float(v[j]);
             if (a.x_res != nullptr && rv) {
               // adaLN-Zero residual: x_res + alpha[image] * (layer output)
               const uint4* xp = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.x_res) +
@@ -625,7 +636,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         }
         ++nstore;
       }
-      if (mode == 4 && pr.dg != nullptr && rv) pr.dg[grow * pr.dg_stride + ti.n0 / BN] = dgacc;
+      if (kBwd && mode == 4 && pr.dg != nullptr && rv) pr.dg[grow * pr.dg_stride + (ti.n0 / BN) * kPairEpiSplit + grp] = dgacc;
       }
       tc_fence_before();
       __syncwarp();
@@ -640,7 +651,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       }
     }
     if (lane == 0) bulk_wait_all();            // stores done before the CTA may exit
-  } else if (gather_lsu) {
+  } else if (kGather && gather_lsu) {
     // ------------------------------------------------------------ row gather (both CTAs)
     // Thread u of the two warps copies 16-byte chunk u % 8 of this CTA's rows u / 8 + 8 i
     // (i < 16) of every stage of a routed tile: row r of the tile is row row_token[r] of x
@@ -667,7 +678,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     for (int k = 0;; ++k) {
       const int tile = cid + k * ncl;
       if (tile >= pl.total) break;
-      const PairTile ti = pair_decode<BN>(tile, pl, a);
+      const PairTile ti = pair_decode<BN, kBwd>(tile, pl, a);
       const bool mine = ti.p == 0;
       int rowid[16];
 #pragma unroll
@@ -727,15 +738,15 @@ done:
   }
 }
 
-template <int BN, typename S>
+template <int BN, typename S, int F>
 static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb,
                                   const CUtensorMap* to, int num_sms, int max_pairs, cudaStream_t s) {
   using C = PairCfg<BN>;
-  cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<BN, S>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<BN, S, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms & ~1, 1, 1);
-  cfg.blockDim = dim3(kPairThreads, 1, 1);
+  cfg.blockDim = dim3(pair_threads<F>(), 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -757,7 +768,7 @@ static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, cons
     if (dev >= 0 && dev < kMaxDevicesCached && fit[dev] > 0) {
       pairs = fit[dev];
     } else {
-      err = cudaOccupancyMaxActiveClusters(&pairs, gemm_pair_kernel<BN, S>, &cfg);
+      err = cudaOccupancyMaxActiveClusters(&pairs, gemm_pair_kernel<BN, S, F>, &cfg);
       if (err != cudaSuccess) return err;
       if (pairs < 1) return cudaErrorInvalidConfiguration;
       if (dev >= 0 && dev < kMaxDevicesCached) fit[dev] = pairs;
@@ -766,7 +777,7 @@ static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, cons
   const int grid = pair_grid(num_sms, pairs, max_pairs);
   if (grid < 2) return cudaErrorInvalidConfiguration;
   cfg.gridDim = dim3(grid, 1, 1);
-  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, S>, ta[0], tb[0], ta[1], tb[1], to[0], to[1], a);
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, S, F>, ta[0], tb[0], ta[1], tb[1], to[0], to[1], a);
 }
 
 // Tiles are 256 columns wide, with one narrower tile (a multiple of 64 columns)
@@ -780,8 +791,27 @@ int gemm_pair_pick_bn(int n0, int n1) {
 cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, const CUtensorMap* to,
                              int bn, int num_sms, int max_pairs, cudaStream_t s) {
   if (bn != 256) return cudaErrorInvalidValue;
-  return a.f16 ? launch_pair_bn<256, StoreF16>(a, ta, tb, to, num_sms, max_pairs, s)
-               : launch_pair_bn<256, StoreBF16>(a, ta, tb, to, num_sms, max_pairs, s);
+  int f = 0;
+  if (a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr) f |= kFeatClaim;
+  if (a.p[0].gather_rows != nullptr) f |= kFeatGather;
+  for (int q = 0; q < a.nprob && q < 2; ++q) {
+    const GemmProblem& p = a.p[q];
+    if (p.a_mn || p.b_mn || p.kgrouped || p.out_f32 || p.epi == 4) f |= kFeatBwd;
+  }
+#define MOE_PAIR_LAUNCH(FEAT)                                                                    \
+  case FEAT:                                                                                     \
+    return a.f16 ? launch_pair_bn<256, StoreF16, FEAT>(a, ta, tb, to, num_sms, max_pairs, s)    \
+                 : launch_pair_bn<256, StoreBF16, FEAT>(a, ta, tb, to, num_sms, max_pairs, s);
+  switch (f) {
+    MOE_PAIR_LAUNCH(0)
+    MOE_PAIR_LAUNCH(kFeatClaim)
+    MOE_PAIR_LAUNCH(kFeatGather)
+    MOE_PAIR_LAUNCH(kFeatBwd)
+    MOE_PAIR_LAUNCH(kFeatBwd | kFeatClaim)
+    default:
+      return cudaErrorNotSupported;                 // no instantiation gathers rows and claims tiles
+  }
+#undef MOE_PAIR_LAUNCH
 }
 
 }  // namespace moe

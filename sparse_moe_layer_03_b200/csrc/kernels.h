@@ -12,6 +12,11 @@ void set_last_error_message(const char* msg);
 // every expert segment of the permuted buffers starts on a multiple of this many rows
 constexpr int kSegAlign = 256;
 
+// CTA-pair GEMM: epilogue warps per TMEM lane quadrant (each takes every kPairEpiSplit-th column
+// box of a tile); the GELU-backward row dots come per column tile and warp: kPairEpiSplit slots.
+// Two per quadrant measured no faster on GEMM1 and 5% slower on GEMM2 + combine at XL.
+constexpr int kPairEpiSplit = 1;
+
 // per-device values cached by the launchers (devices 0 .. kMaxDevicesCached-1)
 constexpr int kMaxDevicesCached = 64;
 
@@ -187,7 +192,7 @@ struct GemmProblem {
   int out_f32;              // fp32 output through a 3-D map [z, M, N]: z = expert (kgrouped), n / out_split, or 0
   int out_split;
   const void* aux;          // epi 4: u [rows, N] act
-  float* dg;                // epi 4: [rows, dg_stride] per-column-tile row dots, or null
+  float* dg;                // epi 4: [rows, dg_stride] row dots per column tile and epilogue warp, or null
   int dg_stride;
   const void* A;            // [rows,K] act (FFMA path; the TMA path uses tensor maps)
   const void* B;            // [E*N or N, K] act

@@ -348,9 +348,6 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
       // one box of hc blocks; blocks past D come back zero-filled and count as bytes
       mbar_arrive_expect_tx(bar, stage_bytes);
       tma_load_3d(dst, &tmap_x, 0, rb * kMmaRB, z0, bar);
-      // the same half of this warp's next row block into L2, so that its load (issued once this
-      // block is done) finds it there: two row blocks per warp in flight towards the SM
-      if (j + NC < my_rb) tma_prefetch_3d(&tmap_x, 0, (rb + NC * (int)gridDim.x) * kMmaRB, z0);
     } else {
       mbar_arrive_expect_tx(bar, (uint32_t)nb * kMmaRB * 128);
       for (int c = 0; c < nb; ++c) tma_load_2d(dst + c * (kMmaRB * 128), &tmap_x, (z0 + c) * 64, rb * kMmaRB, bar);

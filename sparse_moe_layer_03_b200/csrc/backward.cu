@@ -475,11 +475,6 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
     tma_load_3d(dst, &tmap_x, 0, rb * 16, 0, bar);
     tma_load_3d(dst + L.hc * 2048, &tmap_x, 0, rb * 16, L.hc, bar);
   };
-  if (tid == 0) {
-    for (int st = 0; st < kRmStages; ++st) mbar_init(smem_u32(&full[st]), 1);
-    fence_barrier_init();
-    for (int j = 0; j < kRmStages && j < my_rb; ++j) issue(j);
-  }
   if (tid < 16)
     c_s[tid] = tid < E ? a.scale * a.alpha * ((float)E / ((float)a.K * a.T)) * (float)a.counts[tid] / (float)a.T : 0.f;
   if (tid < 256) dbs[tid] = 0.f;
@@ -492,6 +487,12 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
       const uint4 val = src < E ? __ldg(wv + (size_t)src * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
       *reinterpret_cast<uint4*>(wg_s + (size_t)e * L.wg_stride + v * 16) = val;
     }
+  }
+  // x after the gate weight: issued first, every CTA's x loads delayed the weight's reads
+  if (tid == 0) {
+    for (int st = 0; st < kRmStages; ++st) mbar_init(smem_u32(&full[st]), 1);
+    fence_barrier_init();
+    for (int j = 0; j < kRmStages && j < my_rb; ++j) issue(j);
   }
   __syncthreads();
   const uint32_t wg_base = smem_u32(wg_s);

@@ -51,7 +51,8 @@ NOMINAL_HBM_GBS = 8000.0         # HBM3e bandwidth named by the workload's targe
 # DRAM read + write bytes of one launch of each expert GEMM at the default workload (ncu, one pass,
 # full size), valid only for the GEMM sources they were measured on: GEMM_SOURCES hashed to
 # TRAFFIC_SOURCES_SHA.  Any change to those files makes the reported traffic null until re-measured.
-GEMM_SOURCES = ("sparse_moe_layer_03_b200/csrc/gemm_tc2.cu", "sparse_moe_layer_03_b200/csrc/common.cuh")
+GEMM_SOURCES = ("sparse_moe_layer_03_b200/csrc/gemm_tc2.cu", "sparse_moe_layer_03_b200/csrc/common.cuh",
+                "sparse_moe_layer_03_b200/csrc/kernels.h")
 TRAFFIC_SOURCES_SHA = ""
 MEASURED_TRAFFIC = {}
 EXTRA_STEPS = 10                 # timed steps of each other workload in the ``workloads`` key

@@ -203,6 +203,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int3
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
 }
+// Programmatic dependent launch: the next kernel of the stream, launched with programmatic
+// stream serialization, may start once every block of this one has signalled (or exited); it
+// waits in grid_dependency_wait until this grid has completed and its writes are visible.
+// Without that launch attribute the wait returns at once.
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const void* tmap, int32_t x, int32_t y,
                                                  uint32_t bar, uint64_t policy) {
   asm volatile(

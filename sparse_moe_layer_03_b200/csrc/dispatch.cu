@@ -127,6 +127,8 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_count_kernel(Dispat
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int g = blockIdx.x;
   const int Kmax = a.Kmax, E = a.E;
+  grid_dependency_wait();                               // the router's selection
+  launch_dependents();                                  // the gather kernel may start loading x rows
   const int t = g * kGroup + tid;
   const bool valid = t < a.T;
   const int ns = valid ? (a.n_sel ? a.n_sel[t] : a.K) : 0;
@@ -202,7 +204,9 @@ __device__ __forceinline__ void store_row(uint4* dst, int nvec, int lane, const 
 // slots of the block at once: row = group base + rank inside the group; writes
 // pos, row_token, row_gate and keeps the row in shared memory.  Phase 2, one
 // warp per token: row loads, then one store of the row per selected slot.  Each
-// warp's first row is already loading while phase 1 runs.
+// warp's first row is loaded before the kernel waits for the count kernel
+// (programmatic dependent launch), so it loads while the counts are scanned (two
+// rows per warp measured the same, with half the blocks resident per SM).
 template <typename T, int P>
 __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, int blk) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -212,9 +216,12 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, i
   const int nt = min(a.tpb, a.T - t0);
   const uint4* xv = reinterpret_cast<const uint4*>(a.x);
   uint4* xp = reinterpret_cast<uint4*>(a.x_perm);
+  constexpr int NW = kDispatchThreads / 32;
   uint4 buf[P > 0 ? P : 1];
   const bool copy = a.x_perm != nullptr;               // else positions only
+  // each warp's first row loads before the wait (x only: it overlaps the count kernel)
   if (P > 0 && copy && w < nt) load_row<P>(xv + (size_t)(t0 + w) * nvec, nvec, lane, buf);
+  grid_dependency_wait();                              // the count kernel's ranks and bases from here on
 
   for (int i = tid; i < nt * Kmax; i += kDispatchThreads) {
     const int t = t0 + i / Kmax, k = i % Kmax;
@@ -239,7 +246,7 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, i
   if (!copy) return;
   __syncthreads();
 
-  for (int l = w; l < nt; l += kDispatchThreads / 32) {
+  for (int l = w; l < nt; l += NW) {
     const uint4* src = xv + (size_t)(t0 + l) * nvec;
     if (P > 0) {
       if (l != w) load_row<P>(src, nvec, lane, buf);
@@ -279,6 +286,7 @@ template <typename T>
 __global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(DispatchArgs a, int zero_blocks) {
   extern __shared__ int spos[];                       // [tpb * Kmax] rows of the block's slots
   if ((int)blockIdx.x < zero_blocks) {
+    grid_dependency_wait();
     zero_padding_rows<T>(a, blockIdx.x);
     return;
   }
@@ -290,18 +298,35 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(Dispa
 }
 
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
-  const int cgrid = a.ngroups;
-  if (a.E <= 8) dispatch_count_kernel<8><<<cgrid, kDispatchThreads, 0, s>>>(a);
-  else if (a.E <= 16) dispatch_count_kernel<16><<<cgrid, kDispatchThreads, 0, s>>>(a);
-  else dispatch_count_kernel<32><<<cgrid, kDispatchThreads, 0, s>>>(a);
-  cudaError_t err = cudaGetLastError();
+  // both kernels launch as programmatic dependents of the kernel before them (they wait for it
+  // inside, before reading what it wrote), so their launches overlap its tail
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cc = {};
+  cc.gridDim = dim3(a.ngroups, 1, 1);
+  cc.blockDim = dim3(kDispatchThreads, 1, 1);
+  cc.stream = s;
+  cc.attrs = attr;
+  cc.numAttrs = 1;
+  cudaError_t err = a.E <= 8 ? cudaLaunchKernelEx(&cc, dispatch_count_kernel<8>, a)
+                    : a.E <= 16 ? cudaLaunchKernelEx(&cc, dispatch_count_kernel<16>, a)
+                                : cudaLaunchKernelEx(&cc, dispatch_count_kernel<32>, a);
   if (err != cudaSuccess) return err;
   const int zero_blocks = a.x_perm != nullptr ? a.E : 0;
   const int ggrid = zero_blocks + (a.T + a.tpb - 1) / a.tpb;
   const size_t smem = (size_t)a.tpb * a.Kmax * sizeof(int);
-  if (a.b16) dispatch_gather_kernel<uint16_t><<<ggrid, kDispatchThreads, smem, s>>>(a, zero_blocks);
-  else dispatch_gather_kernel<float><<<ggrid, kDispatchThreads, smem, s>>>(a, zero_blocks);
-  return cudaGetLastError();
+  // the gather's first row loads (x only) overlap the count kernel; everything the count kernel
+  // writes is read after the wait
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ggrid, 1, 1);
+  cfg.blockDim = dim3(kDispatchThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (a.b16) return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<uint16_t>, a, zero_blocks);
+  return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<float>, a, zero_blocks);
 }
 
 }  // namespace moe

@@ -210,6 +210,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
   const bool dyn = kClaim && a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr;
   // the routed A rows come from x through the gather warps (GEMM1 only: fixed tile order)
   const bool gather_lsu = kGather && a.p[0].gather_rows != nullptr;
+  // launched as a programmatic dependent: wait here for the kernel before (its rows, offsets and
+  // outputs), and let the next one get resident as this grid's CTAs finish
+  grid_dependency_wait();
+  launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -749,13 +753,15 @@ static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, cons
   cfg.blockDim = dim3(pair_threads<F>(), 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   // pairs the device can hold at once (one per TPC normally; fewer on a partitioned device):
   // asked once per device, then at most that many are launched
   static std::mutex mu;

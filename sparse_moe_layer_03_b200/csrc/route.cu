@@ -320,6 +320,7 @@ __global__ void __launch_bounds__(kMmaMaxConsumers * 32, 1)
 route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_m, RouteArgs a,
                  FinalizeArgs fin) {
   constexpr int NT = EMAX / 8;
+  launch_dependents();                              // the dispatch count kernel may get resident
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const MmaSmem L = mma_layout(a.D, a.E);

@@ -1031,36 +1031,38 @@ int moe_expert_backward(const moe_config_t* cfg, const void* x, const void* x_pe
     }
   }
   // 5. dW2 = sum over the expert's rows of (g dY)^T h; dW2s_j = dY^T h_sh_j
-  {
-    GemmArgs g = base_args(np);
-    GemmProblem& p0 = g.p[0];
-    p0.routed = 1; p0.kgrouped = 1; p0.M = (int)D; p0.N = (int)H; p0.K = 0; p0.a_mn = 1; p0.b_mn = 1;
-    p0.out_f32 = 1; p0.out = grads->dw2;
-    GemmProblem& p1 = g.p[1];
-    if (ns > 0) {
-      p1.routed = 0; p1.kgrouped = 1; p1.M = (int)D; p1.N = ns * (int)H; p1.K = (int)T; p1.a_mn = 1; p1.b_mn = 1;
-      p1.out_f32 = 1; p1.out_split = (int)H; p1.out = grads->dws2;
-    }
-    const OperandMap A[2] = {{dz_perm, R, D, 64}, {dout, T, D, 64}};
-    const OperandMap B[2] = {{h_perm, R, H, 64}, {h_sh, T, (long long)ns * H, 64}};
-    const OutputMap O[2] = {{grads->dw2, 1, E, D, H}, {grads->dws2, 1, ns, D, H}};
-    if ((rc = launch_pair_problems(cfg, g, A, B, O, ws, s))) return rc;
-  }
   // 6. dW1 = sum over the expert's rows of dU^T x_perm; dW1s = dU_sh^T x
-  {
+  // The shared problem (K = T reduction rows per tile, the longest tiles) goes first: the tiles
+  // are claimed in order, so the last ones to start are the short routed tiles.
+  for (int step = 0; step < 2; ++step) {
     GemmArgs g = base_args(np);
-    GemmProblem& p0 = g.p[0];
-    p0.routed = 1; p0.kgrouped = 1; p0.M = (int)H; p0.N = (int)D; p0.K = 0; p0.a_mn = 1; p0.b_mn = 1;
-    p0.out_f32 = 1; p0.out = grads->dw1;
-    GemmProblem& p1 = g.p[1];
-    if (ns > 0) {
-      p1.routed = 0; p1.kgrouped = 1; p1.M = ns * (int)H; p1.N = (int)D; p1.K = (int)T; p1.a_mn = 1; p1.b_mn = 1;
-      p1.out_f32 = 1; p1.out = grads->dws1;
+    GemmProblem routed{}, shared{};
+    OperandMap Ar, Br, As, Bs;
+    OutputMap Or, Os;
+    routed.routed = 1; routed.kgrouped = 1; routed.K = 0; routed.a_mn = 1; routed.b_mn = 1; routed.out_f32 = 1;
+    shared.routed = 0; shared.kgrouped = 1; shared.K = (int)T; shared.a_mn = 1; shared.b_mn = 1; shared.out_f32 = 1;
+    if (step == 0) {
+      routed.M = (int)D; routed.N = (int)H; routed.out = grads->dw2;
+      shared.M = (int)D; shared.N = ns * (int)H; shared.out_split = (int)H; shared.out = grads->dws2;
+      Ar = {dz_perm, R, D, 64}; Br = {h_perm, R, H, 64}; Or = {grads->dw2, 1, E, D, H};
+      As = {dout, T, D, 64}; Bs = {h_sh, T, (long long)ns * H, 64}; Os = {grads->dws2, 1, ns, D, H};
+    } else {
+      routed.M = (int)H; routed.N = (int)D; routed.out = grads->dw1;
+      shared.M = ns * (int)H; shared.N = (int)D; shared.out = grads->dws1;
+      Ar = {du_perm, R, H, 64}; Br = {x_perm, R, D, 64}; Or = {grads->dw1, 1, E, H, D};
+      As = {du_sh, T, (long long)ns * H, 64}; Bs = {x, T, D, 64}; Os = {grads->dws1, 1, 1, (long long)ns * H, D};
     }
-    const OperandMap A[2] = {{du_perm, R, H, 64}, {du_sh, T, (long long)ns * H, 64}};
-    const OperandMap B[2] = {{x_perm, R, D, 64}, {x, T, D, 64}};
-    const OutputMap O[2] = {{grads->dw1, 1, E, H, D}, {grads->dws1, 1, 1, (long long)ns * H, D}};
-    if ((rc = launch_pair_problems(cfg, g, A, B, O, ws, s))) return rc;
+    if (ns > 0) {
+      g.p[0] = shared; g.p[1] = routed;
+      const OperandMap A[2] = {As, Ar}, B[2] = {Bs, Br};
+      const OutputMap O[2] = {Os, Or};
+      if ((rc = launch_pair_problems(cfg, g, A, B, O, ws, s))) return rc;
+    } else {
+      g.p[0] = routed;
+      const OperandMap A[2] = {Ar, Ar}, B[2] = {Br, Br};
+      const OutputMap O[2] = {Or, Or};
+      if ((rc = launch_pair_problems(cfg, g, A, B, O, ws, s))) return rc;
+    }
   }
   // 7. bias gradients: column sums of g dY and dU over each expert's rows, of dY and dU_sh over all tokens
   if (grads->db2 && (e = launch_colsum(dz_perm, R, (int)D, offsets, (int)E, 1, partial, grads->db2, f16, s)) != cudaSuccess)

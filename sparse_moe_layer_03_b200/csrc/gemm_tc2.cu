@@ -80,6 +80,7 @@ struct PairCfg {
 struct PairPlan {
   int poff[33];
   int cnt[32];
+  int eorder[32];     // weight-gradient problems: experts by row count, largest first (ties: lower id)
   int ntiles[2];
   int nm[2];          // kgrouped problems: 256-row tiles of each [M, N] output
   int nn[2];          // column tiles per row block: nfull of width BN, then one of width nrem if nrem > 0
@@ -107,7 +108,7 @@ __device__ __forceinline__ PairTile pair_decode(int tile, const PairPlan& pl, co
     // weight gradient: tiles of expert e's [M, N] output; the reduction runs over the expert's
     // rows of the permuted buffers (a dense problem has one segment of K rows)
     const int per = pl.nm[ti.p] * pl.nn[ti.p];
-    const int e = t / per, r = t % per;
+    const int e = pr.routed ? pl.eorder[t / per] : t / per, r = t % per;
     const int mt = r / pl.nn[ti.p], nt = r % pl.nn[ti.p];
     ti.e = e;
     ti.row0 = mt * kPairBM;
@@ -207,7 +208,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
   // tiles claimed in order (the folded combine's guarantee of progress) or a fixed order
   constexpr bool kClaim = (F & kFeatClaim) != 0, kGather = (F & kFeatGather) != 0, kBwd = (F & kFeatBwd) != 0;
-  const bool dyn = kClaim && a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr;
+  // claimed in order: the folded combine (its guarantee of progress) and the weight-gradient
+  // launches (tiles of very different lengths, longest first)
+  const bool dyn = kClaim && a.sched_ctr != nullptr;
   // the routed A rows come from x through the gather warps (GEMM1 only: fixed tile order)
   const bool gather_lsu = kGather && a.p[0].gather_rows != nullptr;
   // launched as a programmatic dependent: wait here for the kernel before (its rows, offsets and
@@ -243,6 +246,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       pl.poff[e + 1] = p;
     }
     if ((long long)p > a.r_max) bad = true;
+    for (int e = 0; e < a.E; ++e) {                 // insertion sort, stable: largest count first
+      int j = e;
+      while (j > 0 && pl.cnt[pl.eorder[j - 1]] < pl.cnt[e]) {
+        pl.eorder[j] = pl.eorder[j - 1];
+        --j;
+      }
+      pl.eorder[j] = e;
+    }
     for (int q = 0; q < 2; ++q) {
       if (q >= a.nprob) { pl.ntiles[q] = 0; pl.nn[q] = 1; pl.nm[q] = 1; pl.nfull[q] = 1; pl.nrem[q] = 0; continue; }
       const GemmProblem& pr = a.p[q];
@@ -517,9 +528,30 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           ++nstore;
         }
       } else {
+      // GELU backward: the stored pre-activation u of the row's next box (64 columns), loaded one
+      // box ahead so that its latency hides behind the current box's work
+      const uint16_t* urow = (kBwd && mode == 4 && rv)
+                                 ? reinterpret_cast<const uint16_t*>(pr.aux) + grow * pr.N + ti.n0 : nullptr;
+      uint4 unext[8];
+      if (kBwd && mode == 4) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          unext[u] = (urow && grp * box_cols < ti.width)
+                         ? __ldcg(reinterpret_cast<const uint4*>(urow + grp * box_cols) + u) : make_uint4(0u, 0u, 0u, 0u);
+      }
 #pragma unroll 1
       for (int c0 = grp * box_cols; c0 < ti.width; c0 += box_cols * kPairEpiSplit) {
         uint4 o[8];
+        uint4 ucur[8];
+        if (kBwd && mode == 4) {
+          const int cn = c0 + box_cols * kPairEpiSplit;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            ucur[u] = unext[u];
+            unext[u] = (urow && cn < ti.width) ? __ldcg(reinterpret_cast<const uint4*>(urow + cn) + u)
+                                               : make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
         uint32_t vv[2][32];
         tmem_ld_32x32b_x32(tbase + c0, vv[0]);
         tmem_ld_32x32b_x32(tbase + c0 + 32, vv[1]);
@@ -563,16 +595,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
           } else if (kBwd && mode == 4) {
             // GELU backward: acc = dY W (ungated), u the stored pre-activation of these columns;
             // dU = gate * acc * gelu'(u) (zero on padding rows), and the row's sum of acc * gelu(u)
-            float uf[32];
-            if (rv) {
-              const uint4* up = reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(pr.aux) +
-                                                               grow * pr.N + col0);
+            float uf[32];                            // zeros on padding rows (ucur is zero there)
 #pragma unroll
-              for (int u4 = 0; u4 < 4; ++u4) S::x8_to_f32(__ldcg(up + u4), uf + 8 * u4);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) uf[j] = 0.f;
-            }
+            for (int u4 = 0; u4 < 4; ++u4) S::x8_to_f32(ucur[half * 4 + u4], uf + 8 * u4);
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
               float g0, d0, g1, d1;
@@ -803,7 +828,9 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUt
   for (int q = 0; q < a.nprob && q < 2; ++q) {
     const GemmProblem& p = a.p[q];
     if (p.a_mn || p.b_mn || p.kgrouped || p.out_f32 || p.epi == 4) f |= kFeatBwd;
+    if (p.kgrouped) f |= kFeatClaim;
   }
+  if ((f & kFeatClaim) && a.sched_ctr == nullptr) return cudaErrorInvalidValue;
 #define MOE_PAIR_LAUNCH(FEAT)                                                                    \
   case FEAT:                                                                                     \
     return a.f16 ? launch_pair_bn<256, StoreF16, FEAT>(a, ta, tb, to, num_sms, max_pairs, s)    \

@@ -261,38 +261,45 @@ __device__ __forceinline__ void route_modulate(const RouteArgs& a, uint8_t* xs, 
 
 // The last block to finish turns the per-block partials into counts and the loss
 // (and, where asked, leaves the per-expert score sums for cross-call statistics).
-// Warp w reduces experts w, w + nwarps, ...: its lanes stride over the tiles
-// (independent loads), then a fixed xor tree; a fixed expert order for the
-// loss.  Bit-reproducible.  scratch: 2 x 32 x 8 bytes of shared memory.
+// Thread (chunk, expert) of the first nch * E sums tiles chunk, chunk + nch, ... of
+// its expert (all of its loads independent, so the block's loads are in flight
+// together: one round trip instead of one per expert); then thread e adds the
+// chunks' sums in chunk order, and a fixed tree over the experts gives the loss.
+// Bit-reproducible.  scratch: 16 bytes per (chunk, expert), at most blockDim of them.
 constexpr int kFinalizeScratch = 2 * 32 * 32 * 8;
 template <int EMAX>
 __device__ void finalize_counts_loss(const FinalizeArgs& a, uint8_t* scratch) {
-  long long* wc = reinterpret_cast<long long*>(scratch);
-  double* wp = reinterpret_cast<double*>(scratch + 32 * 8);
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  const int tid = threadIdx.x;
   const int E = a.E;
-  for (int e = w; e < E; e += nw) {
+  const int nch = (int)blockDim.x / E;               // E <= 32 <= blockDim
+  long long* cc = reinterpret_cast<long long*>(scratch);
+  double* pp = reinterpret_cast<double*>(scratch + (size_t)nch * E * sizeof(long long));
+  if (tid < nch * E) {
+    const int e = tid % E, ch = tid / E;
+    const int nt = a.ntiles_counts > a.ntiles_psum ? a.ntiles_counts : a.ntiles_psum;
     long long c = 0;
     double p = 0.0;
-#pragma unroll 4
-    for (int t = lane; t < a.ntiles_counts; t += 32) c += __ldcg(a.tile_counts + (size_t)t * E + e);
-#pragma unroll 4
-    for (int t = lane; t < a.ntiles_psum; t += 32) p += (double)__ldcg(a.tile_psum + (size_t)t * E + e);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      c += __shfl_xor_sync(0xffffffffu, c, o);
-      p += __shfl_xor_sync(0xffffffffu, p, o);
+#pragma unroll 8
+    for (int t = ch; t < nt; t += nch) {
+      if (t < a.ntiles_counts) c += __ldcg(a.tile_counts + (size_t)t * E + e);
+      if (t < a.ntiles_psum) p += (double)__ldcg(a.tile_psum + (size_t)t * E + e);
     }
-    if (lane == 0) { wc[e] = c; wp[e] = p; }
+    cc[ch * E + e] = c;
+    pp[ch * E + e] = p;
   }
   __syncthreads();
   if (tid < 32) {
     double term = 0.0;
     if (tid < E) {
-      const long long cc = wc[tid];
-      a.counts[tid] = (int32_t)cc;
-      if (a.score_sum) a.score_sum[tid] = wp[tid];
-      term = ((double)E / ((double)a.K * a.T)) * (double)cc * (wp[tid] / a.T);
+      long long c = 0;
+      double p = 0.0;
+      for (int ch = 0; ch < nch; ++ch) {
+        c += cc[ch * E + tid];
+        p += pp[ch * E + tid];
+      }
+      a.counts[tid] = (int32_t)c;
+      if (a.score_sum) a.score_sum[tid] = p;
+      term = ((double)E / ((double)a.K * a.T)) * (double)c * (p / a.T);
     }
     for (int o = 16; o > 0; o >>= 1) term += __shfl_down_sync(0xffffffffu, term, o);
     if (tid == 0) *a.aux_loss = (float)(a.alpha * term);

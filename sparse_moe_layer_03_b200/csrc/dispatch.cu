@@ -9,18 +9,24 @@
 //
 //   count kernel  (one block per group of 256 tokens): the group's count per
 //                 expert, and each slot's rank among the group's slots of the
-//                 same expert (warp ballots), parked in `pos`.  The block that
-//                 finishes last scans the group counts into each group's first
-//                 row in every segment, writes the offsets and marks the
-//                 padding rows.
-//   gather kernel (64 tokens per block): one thread per slot turns ranks into
-//                 rows (group base + rank) and writes pos, row_token and
-//                 row_gate; then one warp per token loads the row and stores
-//                 it once per selected expert with 16-byte vectors (each
-//                 warp's first row loads while the rows are worked out).  Its
-//                 first E blocks write zeros to the padding rows of the E
-//                 segments, so every row of a segment's 256-row tiles holds
-//                 finite values (the weight gradients reduce over them).
+//                 same expert (warp ballots), parked in `pos`.  No scan, no
+//                 grid-wide step: it ends as soon as its counts are written.
+//   gather kernel (launched as a programmatic dependent of the count kernel):
+//                 every block first reads all group counts (4 KB at XL, one
+//                 round of loads) and works out the segment starts and its
+//                 own group's first row in every segment, redundantly.
+//                 Blocks 0..E: block e < E marks the padding rows of segment
+//                 e (row_token -1, gate 0, zero rows in x_perm: every row of a
+//                 segment's 256-row tiles then holds finite values, which the
+//                 weight gradients reduce over); block E marks the rows after
+//                 the last segment; block 0 writes the offsets.  The other
+//                 blocks take 64 tokens each: one thread per slot turns ranks
+//                 into rows (group base + rank) and writes pos, row_token and
+//                 row_gate; then one warp per token stores its row once per
+//                 selected expert with 16-byte vectors (each warp's first row
+//                 loads before the wait, while the count kernel runs).
+//   A last-block scan inside the count kernel (fence, counter, two rounds of
+//   loads) took half of its 8.6 us, measured with a timer probe.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -44,75 +50,48 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane) {
   return v;
 }
 
-// Segment bases from the group counts; run by the last block of the count kernel.
-// cnt[e * ngroups + g] (counts in, first row of group g in segment e out).
-// Warp w takes experts w, w + 8, ...; its lanes read 32 consecutive groups per
-// load (coalesced), eight loads in flight.
-__device__ void dispatch_scan_groups(const DispatchArgs& a) {
-  __shared__ int total_s[32], poff_s[33];
+// The segment plan from the group counts cnt[e * ngroups + g], computed by every gather block:
+// total_s[e] = expert e's rows, before_s[e] = its rows in groups before g0, poff_s[e] = the first
+// row of segment e (poff_s[E] = rows of all segments).  Warp w takes experts w, w + 8, ...; its
+// lanes read 32 consecutive groups per load (coalesced), eight loads in flight.  Every thread
+// of the block calls it.
+__device__ void segment_plan(const DispatchArgs& a, int g0, int* total_s, int* before_s, long long* poff_s) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, NW = kDispatchThreads / 32;
   const int E = a.E, ng = a.ngroups;
-  int32_t* cnt = a.group_base;
-  // 1. per-expert totals
   for (int e = w; e < E; e += NW) {
-    const int32_t* row = cnt + (size_t)e * ng;
-    int sum = 0;
-    for (int g0 = 0; g0 < ng; g0 += 8 * 32) {
+    const int32_t* row = a.group_base + (size_t)e * ng;
+    int tot = 0, bef = 0;
+    for (int c0 = 0; c0 < ng; c0 += 8 * 32) {
       int v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int g = g0 + u * 32 + lane;
+        const int g = c0 + u * 32 + lane;
         v[u] = g < ng ? __ldcg(row + g) : 0;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) sum += v[u];
+      for (int u = 0; u < 8; ++u) {
+        const int g = c0 + u * 32 + lane;
+        tot += v[u];
+        bef += g < g0 ? v[u] : 0;
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) total_s[e] = sum;
+    for (int o = 16; o > 0; o >>= 1) {
+      tot += __shfl_xor_sync(0xffffffffu, tot, o);
+      bef += __shfl_xor_sync(0xffffffffu, bef, o);
+    }
+    if (lane == 0) { total_s[e] = tot; before_s[e] = bef; }
   }
   __syncthreads();
   if (tid == 0) {
-    int p = 0, u = 0;
+    long long p = 0;
     for (int e = 0; e < E; ++e) {
       poff_s[e] = p;
-      a.offsets[e] = u;
-      u += total_s[e];
       p += (total_s[e] + kSegAlign - 1) / kSegAlign * kSegAlign;
     }
     poff_s[E] = p;
-    a.offsets[E] = u;
   }
   __syncthreads();
-  // 2. exclusive scan over the groups of each segment, from the segment's start
-  for (int e = w; e < E; e += NW) {
-    int32_t* row = cnt + (size_t)e * ng;
-    int carry = poff_s[e];
-    for (int g0 = 0; g0 < ng; g0 += 8 * 32) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int g = g0 + u * 32 + lane;
-        v[u] = g < ng ? __ldcg(row + g) : 0;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int g = g0 + u * 32 + lane;
-        const int incl = warp_incl_scan(v[u], lane);
-        if (g < ng) row[g] = carry + incl - v[u];
-        carry += __shfl_sync(0xffffffffu, incl, 31);
-      }
-    }
-  }
-  // 3. padding rows: segment e's tail (e < E) or the rows after the last segment (e = E)
-  for (int e = 0; e <= E; ++e) {
-    const long long lo = e < E ? (long long)poff_s[e] + total_s[e] : poff_s[E];
-    const long long hi = e < E ? (long long)poff_s[e + 1] : a.r_max;
-    for (long long r = lo + tid; r < hi; r += kDispatchThreads) {
-      a.row_token[r] = -1;
-      a.row_gate[r] = 0.f;
-    }
-  }
 }
 
 // One group of kGroup tokens per block, one token per thread: the group's count
@@ -123,7 +102,6 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_count_kernel(Dispat
   constexpr int NW = kDispatchThreads / 32;
   __shared__ uint32_t bal[NW][EMAX];
   __shared__ int wbase[NW][EMAX];
-  __shared__ bool last;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int g = blockIdx.x;
   const int Kmax = a.Kmax, E = a.E;
@@ -160,7 +138,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_count_kernel(Dispat
       wbase[v][tid] = run;
       run += __popc(bal[v][tid]);
     }
-    a.group_base[(size_t)tid * a.ngroups + g] = run;
+    a.group_base[(size_t)tid * a.ngroups + g] = run;     // the group's count of expert tid
   }
   __syncthreads();
   const uint32_t lt = lanemask_lt();
@@ -168,18 +146,6 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_count_kernel(Dispat
   for (int k = 0; k < EMAX; ++k)
     if (k < Kmax && valid)
       a.pos[(size_t)t * Kmax + k] = ek[k] >= 0 ? wbase[w][ek[k]] + __popc(bal[w][ek[k]] & lt) : -1;
-  // the last block to finish turns the counts into segment bases
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const unsigned int prev = atomicAdd(a.ctr, 1u);
-    last = prev == gridDim.x - 1;
-  }
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  dispatch_scan_groups(a);
-  if (tid == 0) *a.ctr = 0u;                            // ready for the next call
 }
 
 // One row copy: P x 32 lanes x 16 bytes covers up to P*32 vectors of the row.
@@ -200,8 +166,9 @@ __device__ __forceinline__ void store_row(uint4* dst, int nvec, int lane, const 
   }
 }
 
-// Gather block: tokens [t0, t0 + tpb).  Phase 1, one thread per slot, all
-// slots of the block at once: row = group base + rank inside the group; writes
+// Gather block: tokens [t0, t0 + tpb), all in group g0 = t0 / 256.  Phase 1, one thread per slot,
+// all slots of the block at once: row = segment start + the expert's rows in earlier groups +
+// rank inside the group; writes
 // pos, row_token, row_gate and keeps the row in shared memory.  Phase 2, one
 // warp per token: row loads, then one store of the row per selected slot.  Each
 // warp's first row is loaded before the kernel waits for the count kernel
@@ -221,7 +188,10 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, i
   const bool copy = a.x_perm != nullptr;               // else positions only
   // each warp's first row loads before the wait (x only: it overlaps the count kernel)
   if (P > 0 && copy && w < nt) load_row<P>(xv + (size_t)(t0 + w) * nvec, nvec, lane, buf);
-  grid_dependency_wait();                              // the count kernel's ranks and bases from here on
+  grid_dependency_wait();                              // the count kernel's counts and ranks from here on
+  __shared__ int total_s[32], before_s[32];
+  __shared__ long long poff_s[33];
+  segment_plan(a, t0 / kGroup, total_s, before_s, poff_s);
 
   for (int i = tid; i < nt * Kmax; i += kDispatchThreads) {
     const int t = t0 + i / Kmax, k = i % Kmax;
@@ -232,8 +202,9 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, i
       const int e = a.topk_idx[slot];
       const int r = a.pos[slot];
       if (e >= 0 && e < a.E && r >= 0) {
-        p = a.group_base[(size_t)e * a.ngroups + t / kGroup] + r;
-        if (p < 0 || p >= a.r_max) { set_status(a.status, DEV_BAD_INDEX, 201); p = -1; }
+        const long long q = poff_s[e] + before_s[e] + r;
+        p = (int)q;
+        if (q < 0 || q >= a.r_max) { set_status(a.status, DEV_BAD_INDEX, 201); p = -1; }
         else {
           a.row_token[p] = t;
           a.row_gate[p] = a.topk_w[slot];
@@ -267,30 +238,51 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, i
   }
 }
 
-// Zeros on the padding rows [P_e + count_e, P_{e+1}) of segment e of x_perm (offsets from the
-// count kernel).
+// Segment block e <= E: the rows of no token.  e < E: segment e's padding rows [P_e + count_e,
+// P_{e+1}) get row_token -1, gate 0 and (with x_perm) zero rows; e = E: the rows after the last
+// segment, [P_E, r_max), get row_token -1 and gate 0.  Block 0 also writes the offsets.
 template <typename T>
-__device__ void zero_padding_rows(const DispatchArgs& a, int e) {
-  const int nvec = a.D * (int)sizeof(T) / 16;
-  long long p = 0;
-  for (int j = 0; j < e; ++j) p += (a.offsets[j + 1] - a.offsets[j] + kSegAlign - 1) / kSegAlign * kSegAlign;
-  const int c = a.offsets[e + 1] - a.offsets[e];
-  const long long lo = p + c, hi = p + (long long)(c + kSegAlign - 1) / kSegAlign * kSegAlign;
-  if (lo < 0 || hi > a.r_max) return;
-  uint4* xp = reinterpret_cast<uint4*>(a.x_perm);
-  const long long n = (hi - lo) * nvec;
-  for (long long i = threadIdx.x; i < n; i += kDispatchThreads) xp[lo * nvec + i] = make_uint4(0u, 0u, 0u, 0u);
+__device__ void segment_block(const DispatchArgs& a, int e) {
+  __shared__ int total_s[32], before_s[32];
+  __shared__ long long poff_s[33];
+  segment_plan(a, 0, total_s, before_s, poff_s);
+  const int tid = threadIdx.x;
+  const int E = a.E;
+  if (e == 0 && tid == 0) {
+    int u = 0;
+    for (int j = 0; j < E; ++j) {
+      a.offsets[j] = u;
+      u += total_s[j];
+    }
+    a.offsets[E] = u;
+  }
+  const long long lo = e < E ? poff_s[e] + total_s[e] : poff_s[E];
+  const long long hi = e < E ? poff_s[e + 1] : a.r_max;
+  if (lo < 0 || hi > a.r_max) {
+    if (tid == 0) set_status(a.status, DEV_BAD_INDEX, 203);
+    return;
+  }
+  for (long long r = lo + tid; r < hi; r += kDispatchThreads) {
+    a.row_token[r] = -1;
+    a.row_gate[r] = 0.f;
+  }
+  if (e < E && a.x_perm != nullptr) {
+    const int nvec = a.D * (int)sizeof(T) / 16;
+    uint4* xp = reinterpret_cast<uint4*>(a.x_perm);
+    const long long n = (hi - lo) * nvec;
+    for (long long i = tid; i < n; i += kDispatchThreads) xp[lo * nvec + i] = make_uint4(0u, 0u, 0u, 0u);
+  }
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(DispatchArgs a, int zero_blocks) {
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(DispatchArgs a, int seg_blocks) {
   extern __shared__ int spos[];                       // [tpb * Kmax] rows of the block's slots
-  if ((int)blockIdx.x < zero_blocks) {
+  if ((int)blockIdx.x < seg_blocks) {
     grid_dependency_wait();
-    zero_padding_rows<T>(a, blockIdx.x);
+    segment_block<T>(a, blockIdx.x);
     return;
   }
-  const int blk = blockIdx.x - zero_blocks;
+  const int blk = blockIdx.x - seg_blocks;
   const int nvec = a.D * (int)sizeof(T) / 16;
   if (nvec <= 4 * 32) gather_block<T, 4>(a, spos, blk);
   else if (nvec <= 8 * 32) gather_block<T, 8>(a, spos, blk);
@@ -313,8 +305,9 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
                     : a.E <= 16 ? cudaLaunchKernelEx(&cc, dispatch_count_kernel<16>, a)
                                 : cudaLaunchKernelEx(&cc, dispatch_count_kernel<32>, a);
   if (err != cudaSuccess) return err;
-  const int zero_blocks = a.x_perm != nullptr ? a.E : 0;
-  const int ggrid = zero_blocks + (a.T + a.tpb - 1) / a.tpb;
+  if (a.tpb <= 0 || kGroup % a.tpb) return cudaErrorInvalidValue;   // a gather block stays inside one group
+  const int seg_blocks = a.E + 1;
+  const int ggrid = seg_blocks + (a.T + a.tpb - 1) / a.tpb;
   const size_t smem = (size_t)a.tpb * a.Kmax * sizeof(int);
   // the gather's first row loads (x only) overlap the count kernel; everything the count kernel
   // writes is read after the wait
@@ -325,8 +318,8 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.b16) return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<uint16_t>, a, zero_blocks);
-  return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<float>, a, zero_blocks);
+  if (a.b16) return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<uint16_t>, a, seg_blocks);
+  return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<float>, a, seg_blocks);
 }
 
 }  // namespace moe

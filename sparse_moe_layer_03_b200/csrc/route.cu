@@ -361,26 +361,31 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
       for (int c = 0; c < nb; ++c) tma_load_2d(dst + c * (kMmaRB * 128), &tmap_x, (z0 + c) * 64, rb * kMmaRB, bar);
     }
   };
-  if (lane == 0) {
-    mbar_init(smem_u32(&full[2 * w]), 1);
-    mbar_init(smem_u32(&full[2 * w + 1]), 1);
+  // The gate weight's rows come in by bulk copies issued before any x load, so that they are not
+  // queued behind every CTA's x stream (loaded by the threads after the x loads were issued,
+  // setup took about 8 us at XL, measured with a timer probe); the x loads follow at once.
+  uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + L.misc + 1536);
+  if (tid == 0) {
+    mbar_init(smem_u32(wbar), 1);
+    for (int i = 0; i < 2 * NC; ++i) mbar_init(smem_u32(&full[i]), 1);
     fence_barrier_init();
-    if (w < my_rb) { issue(w, 0); issue(w, 1); }   // x streams in while the gate weight loads
+    mbar_arrive_expect_tx(smem_u32(wbar), (uint32_t)(E * D * 2));
+    for (int e = 0; e < E; ++e)
+      bulk_load(smem_u32(wg_s + (size_t)e * wg_stride), reinterpret_cast<const uint8_t*>(a.wg) + (size_t)e * D * 2,
+                (uint32_t)(D * 2), smem_u32(wbar));
   }
+  __syncthreads();
+  if (lane == 0 && w < my_rb) { issue(w, 0); issue(w, 1); }
   if (tid < 32) cnt_s[tid] = 0;
   if (blockIdx.x == 0 && a.zero)
     for (int i = tid; i < a.nzero; i += blockDim.x) a.zero[i] = 0u;
-  {  // gate weight (16-bit) -> padded rows; rows E..EMAX-1 are zero
+  {  // rows E..EMAX-1 of the padded gate weight are zero
     const int vpr = D / 8;
-    const uint4* wv = reinterpret_cast<const uint4*>(a.wg);
-#pragma unroll 4
-    for (int i = tid; i < EMAX * vpr; i += blockDim.x) {
-      const int e = i / vpr, v = i % vpr;
-      const uint4 val = e < E ? __ldg(wv + (size_t)e * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(wg_s + (size_t)e * wg_stride + v * 16) = val;
-    }
+    for (int i = E * vpr + tid; i < EMAX * vpr; i += blockDim.x)
+      *reinterpret_cast<uint4*>(wg_s + (size_t)(i / vpr) * wg_stride + (i % vpr) * 16) = make_uint4(0u, 0u, 0u, 0u);
   }
   __syncthreads();
+  if (!mbar_wait(smem_u32(wbar), 0, nullptr, a.status, 104)) set_status(a.status, DEV_TIMEOUT, 104);
 
   float psum[EMAX];
 #pragma unroll

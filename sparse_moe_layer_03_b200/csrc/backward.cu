@@ -478,23 +478,34 @@ router_bwd_mma_kernel(const __grid_constant__ CUtensorMap tmap_x, BalanceGradArg
   if (tid < 16)
     c_s[tid] = tid < E ? a.scale * a.alpha * ((float)E / ((float)a.K * a.T)) * (float)a.counts[tid] / (float)a.T : 0.f;
   if (tid < 256) dbs[tid] = 0.f;
-  {  // gate weight rows 0..15 (zero past E; rows 8..15 repeat rows 0..7 when packed), padded stride
-    const int vpr = D / 8;
-    const uint4* wv = reinterpret_cast<const uint4*>(a.wg);
-    for (int i = tid; i < 16 * vpr; i += blockDim.x) {
-      const int e = i / vpr, v = i % vpr;
-      const int src = PACK ? (e & 7) : e;
-      const uint4 val = src < E ? __ldg(wv + (size_t)src * vpr + v) : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(wg_s + (size_t)e * L.wg_stride + v * 16) = val;
-    }
-  }
-  // x after the gate weight: issued first, every CTA's x loads delayed the weight's reads
+  // Gate weight rows 0..15 (zero past E; rows 8..15 repeat rows 0..7 when packed), padded stride:
+  // bulk copies of whole rows, issued before any x load (loaded by the threads after the x loads,
+  // the weight's reads queued behind every CTA's x stream); then the x stages.
+  uint64_t* wbar = full + 8;
   if (tid == 0) {
+    mbar_init(smem_u32(wbar), 1);
     for (int st = 0; st < kRmStages; ++st) mbar_init(smem_u32(&full[st]), 1);
     fence_barrier_init();
+    int nrows = 0;
+    for (int e = 0; e < 16; ++e) nrows += (PACK ? (e & 7) : e) < E ? 1 : 0;
+    mbar_arrive_expect_tx(smem_u32(wbar), (uint32_t)(nrows * D * 2));
+    for (int e = 0; e < 16; ++e) {
+      const int src = PACK ? (e & 7) : e;
+      if (src < E)
+        bulk_load(smem_u32(wg_s + (size_t)e * L.wg_stride), reinterpret_cast<const uint8_t*>(a.wg) + (size_t)src * D * 2,
+                  (uint32_t)(D * 2), smem_u32(wbar));
+    }
     for (int j = 0; j < kRmStages && j < my_rb; ++j) issue(j);
   }
+  {  // the rows of no expert are zero
+    const int vpr = D / 8;
+    for (int i = tid; i < 16 * vpr; i += blockDim.x) {
+      const int e = i / vpr;
+      if ((PACK ? (e & 7) : e) >= E) *reinterpret_cast<uint4*>(wg_s + (size_t)e * L.wg_stride + (i % vpr) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   __syncthreads();
+  mbar_wait(smem_u32(wbar), 0, nullptr, nullptr, 121);
   const uint32_t wg_base = smem_u32(wg_s);
   float acc[kRmMaxNT][4];
 #pragma unroll

@@ -65,8 +65,8 @@ int validate(const moe_config_t* c) {
   if (c->gemm_pairs < 0) return fail(MOE_ERR_INVALID_ARG, "gemm_pairs=%d < 0", c->gemm_pairs);
   if (c->seq_len > 0 && c->T % c->seq_len)
     return fail(MOE_ERR_INVALID_ARG, "seq_len=%d does not divide T=%d", c->seq_len, c->T);
-  if (route_smem_total(c->D, c->E, 32, is16(c)) > 232448 ||
-      (is16(c) && route_mma_stages(c->D, c->E) < 1))
+  if (route_smem_total(c->D, c->E, 32, is16(c), 1) > 232448 ||
+      (is16(c) && route_mma_stages(c->D, c->E, 1) < 1))
     return fail(MOE_ERR_UNSUPPORTED, "E=%d x D=%d too large for the router's shared memory", c->E, c->D);
   return MOE_OK;
 }
@@ -191,12 +191,14 @@ int make_tmap(CUtensorMap* m, const void* base, int dtype, long long rows, long 
 // `box_rows` rows x ceil(cols/128) swizzled 128-byte blocks (half of each row),
 // block-major.  Returns false when the driver does not accept the layout (the
 // caller then uses 2-D boxes).
-bool make_tmap_rows3d(CUtensorMap* m, const void* base, int dtype, long long rows, long long cols, int box_rows) {
+bool make_tmap_rows3d(CUtensorMap* m, const void* base, int dtype, long long rows, long long cols, int box_rows,
+                      int box_blocks = 0) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)(rows > 0 ? rows : 1), (cuuint64_t)(cols / 64)};
   cuuint64_t strides[2] = {(cuuint64_t)cols * 2, 128};
-  const cuuint32_t blocks = (cuuint32_t)((cols / 64 + 1) / 2);    // one box = half of a row block
+  // one box = box_blocks 64-column blocks (default: half of a row block)
+  const cuuint32_t blocks = (cuuint32_t)(box_blocks > 0 ? box_blocks : (cols / 64 + 1) / 2);
   cuuint32_t box[3] = {64, (cuuint32_t)box_rows, blocks};
   cuuint32_t estr[3] = {1, 1, 1};
   if (blocks > 256) return false;
@@ -290,20 +292,21 @@ int moe_route(const moe_config_t* cfg, const void* x, const void* wg, const floa
   const int sms = num_sms_current();
   int tile = 0, threads = 0;
   const bool b16 = is16(cfg);
-  route_plan(cfg->T, cfg->D, cfg->E, b16, sms, &tile, &threads);
+  route_plan(cfg->T, cfg->D, cfg->E, b16, mod != nullptr, sms, &tile, &threads);
   const int ntiles = (cfg->T + tile - 1) / tile;
   const int grid = ntiles < sms ? ntiles : sms;
   // partial sums: one row per CTA (16-bit kernel) or per token tile (fp32 kernel)
   const int nparts = b16 ? grid : ntiles;
   CUtensorMap tm, tmm;
   int tmap3d = 0;
-  if (b16 && make_tmap_rows3d(&tm, x, cfg->dtype, cfg->T, cfg->D, tile)) tmap3d = 1;
+  const int box_blocks = b16 ? route_box_blocks(cfg->D, cfg->E, mod != nullptr) : 0;
+  if (b16 && make_tmap_rows3d(&tm, x, cfg->dtype, cfg->T, cfg->D, tile, box_blocks)) tmap3d = 1;
   else if ((rc = make_tmap(&tm, x, cfg->dtype, cfg->T, cfg->D, tile, "x"))) return rc;
   // the modulated rows go out with the same box geometry as x comes in
   tmm = tm;
   if (mod) {
     if (tmap3d) {
-      if (!make_tmap_rows3d(&tmm, mod->x_mod, cfg->dtype, cfg->T, cfg->D, tile))
+      if (!make_tmap_rows3d(&tmm, mod->x_mod, cfg->dtype, cfg->T, cfg->D, tile, box_blocks))
         return fail(MOE_ERR_CUDA, "tensor map for mod->x_mod failed");
     } else if ((rc = make_tmap(&tmm, mod->x_mod, cfg->dtype, cfg->T, cfg->D, tile, "x_mod"))) {
       return rc;

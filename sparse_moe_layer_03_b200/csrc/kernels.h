@@ -37,7 +37,7 @@ struct RouteArgs {
   int T, D, E, K;
   int b16, f16;             // 16-bit storage (bf16 or fp16); fp16
   int tile_rows, ntiles, grid;
-  int tmap3d;               // 16-bit router: 1 = one 3-D box {64, 16 rows, D/64} per unit, 0 = D/64 2-D boxes
+  int tmap3d;               // 16-bit router: 1 = one 3-D box {64, 16 rows, blocks} per part, 0 = 2-D boxes
   int32_t* topk_idx;        // top-K mode: [T,K]
   float* topk_w;
   int32_t* n_sel;           // may be null (top-K)
@@ -56,9 +56,10 @@ struct RouteArgs {
   int* status;
 };
 size_t route_smem_bytes(int D, int E, int tile_rows, int b16);
-size_t route_smem_total(int D, int E, int tile_rows, int b16);
-int route_mma_stages(int D, int E);
-void route_plan(int T, int D, int E, int b16, int sms, int* tile_rows, int* threads);
+size_t route_smem_total(int D, int E, int tile_rows, int b16, int modulate);
+int route_mma_stages(int D, int E, int modulate);
+int route_box_blocks(int D, int E, int modulate);   // 16-bit router: 64-column blocks per TMA box
+void route_plan(int T, int D, int E, int b16, int modulate, int sms, int* tile_rows, int* threads);
 
 // partial counts / score sums -> counts[E] and the balance loss
 struct FinalizeArgs {

@@ -125,46 +125,56 @@ __device__ __forceinline__ void tile_partials(const float* psum, int tile, const
 
 // ---------------------------------------------------------------- 16-bit: tensor-core logits
 // Work unit = a block of 16 consecutive tokens: their full rows (16 x D 16-bit,
-// one contiguous stretch of HBM, so DRAM pages are read whole) land in one
-// pair of shared-memory stages (one per half of the row, each one 3-D TMA box of
-// 64-column blocks x 16 rows, 128-byte swizzle).  Each warp owns two stages,
-// takes every NC-th row block and issues its own loads: wait for a half,
-// compute its part of the 16 x E logits with mma.sync m16n8k16 (A via ldmatrix
-// from the swizzled stage, B = gate weight in shared memory with rows padded by
-// 16 bytes), refill that stage with the next row block's half (the load
-// overlaps the other half's MMAs and the epilogue), then run softmax and
-// selection (one lane per token).  No block-wide barrier inside the loop and no
-// warp waits on another warp's progress.
+// one contiguous stretch of HBM, so DRAM pages are read whole) arrive in P parts,
+// each one 3-D TMA box of 64-column blocks x 16 rows (128-byte swizzle) into one
+// of the warp's two stages.  Each warp takes every NC-th row block and issues its
+// own loads: wait for a part, compute its share of the 16 x E logits with
+// mma.sync m16n8k16 (A via ldmatrix from the swizzled stage, B = gate weight in
+// shared memory with rows padded by 16 bytes), refill that stage with the part
+// after next (the load overlaps the other stage's MMAs and the epilogue), then
+// run softmax and selection (one lane per token).  No block-wide barrier inside
+// the loop and no warp waits on another warp's progress.
 constexpr int kMmaRB = 16;        // tokens per row block
-constexpr int kMmaMaxConsumers = 6;
+constexpr int kMmaMaxConsumers = 8;
 
-// A row block is loaded as two halves (column blocks [0, hc) and [hc, 2hc), hc =
-// ceil(D/128)), each into its own stage; warp c owns stages 2c and 2c+1, issues
-// their loads itself and waits on their phases strictly in order.  As many warps
-// (<= 6) as the shared memory allows.
+// A row block is loaded in P parts of cpq = ceil(D/64 / P) column blocks (one 3-D TMA box each);
+// warp c owns stages 2c and 2c+1, which take the parts of its row blocks in turn (part n of the
+// warp's sequence goes to stage n mod 2), issues their loads itself and waits on their phases
+// strictly in order.  P is chosen for the most consumer warps (<= 8) that shared memory holds:
+// more warps leave fewer row blocks per warp (at XL, 8 warps with P = 3 give each warp at most
+// 2 of the 2048 blocks, where 5 warps with halves gave most warps 3).  The adaLN modulation needs
+// the whole row in the warp's two stages: P = 2.
 struct MmaSmem {
   size_t wg, x, logits, misc, total;
-  int consumers, hc;
+  int consumers, parts, cpq;
 };
-__host__ __device__ inline MmaSmem mma_layout(int D, int E) {
-  MmaSmem L;
+__host__ __device__ inline MmaSmem mma_layout(int D, int E, bool modulate) {
+  MmaSmem best{};
   const int em = route_emax(E);
-  L.hc = (D / 64 + 1) / 2;
-  L.wg = 0;
-  L.x = align1k((size_t)em * (D * 2 + 16));
-  const size_t stage = (size_t)kMmaRB * L.hc * 128;
-  L.consumers = 0;
-  for (int nc = kMmaMaxConsumers; nc >= 1; --nc) {
+  const int nchunks = D / 64;
+  for (int parts = 2; parts <= (modulate ? 2 : 4); ++parts) {
+    if (parts > 2 && parts > nchunks) break;
+    MmaSmem L;
+    L.parts = parts;
+    L.cpq = (nchunks + parts - 1) / parts;
+    if (parts > 2 && (parts - 1) * L.cpq >= nchunks) continue;   // no part without columns
+    L.wg = 0;
+    L.x = align1k((size_t)em * (D * 2 + 16));
+    const size_t stage = (size_t)kMmaRB * L.cpq * 128;
+    L.consumers = 0;
+    for (int nc = kMmaMaxConsumers; nc >= 1; --nc) {
+      const size_t xb = 2 * nc * stage;
+      const size_t total = L.x + (xb > 16896 ? xb : 16896) + (size_t)nc * kMmaRB * em * 4 + 2048 + 1024;
+      if (total + 1024 <= 232448) { L.consumers = nc; break; }
+    }
+    const int nc = L.consumers > 0 ? L.consumers : 1;
     const size_t xb = 2 * nc * stage;
-    const size_t total = L.x + (xb > 16896 ? xb : 16896) + (size_t)nc * kMmaRB * em * 4 + 2048 + 1024;
-    if (total + 1024 <= 232448) { L.consumers = nc; break; }
+    L.logits = L.x + (xb > 16896 ? xb : 16896);   // x stages double as the finalize scratch
+    L.misc = L.logits + (size_t)nc * kMmaRB * em * 4;
+    L.total = L.misc + 2048 + 1024;
+    if (parts == 2 || L.consumers > best.consumers) best = L;
   }
-  const int nc = L.consumers > 0 ? L.consumers : 1;
-  const size_t xb = 2 * nc * stage;
-  L.logits = L.x + (xb > 16896 ? xb : 16896);   // x stages double as the finalize scratch
-  L.misc = L.logits + (size_t)nc * kMmaRB * em * 4;
-  L.total = L.misc + 2048 + 1024;
-  return L;
+  return best;
 }
 
 // adaLN modulation of one row block held in a warp's two stages, in place:
@@ -180,7 +190,7 @@ __host__ __device__ inline MmaSmem mma_layout(int D, int E) {
 // the 32 lanes spread over the 8 chunk positions (4 wavefronts per access).
 template <bool F16>
 __device__ __forceinline__ void route_modulate(const RouteArgs& a, uint8_t* xs, int stage_bytes, int w, int hc,
-                                               int nchunks, int rb, int lane) {
+                                               int nchunks, int rb, int lane) {   // hc: blocks per half (P = 2)
   using S = typename std::conditional<F16, StoreF16, StoreBF16>::type;
   const int r = lane & 15, p = lane >> 4;
   const int z0 = p * hc;
@@ -330,8 +340,9 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
   launch_dependents();                              // the dispatch count kernel may get resident
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  const MmaSmem L = mma_layout(a.D, a.E);
-  const int NC = L.consumers, hc = L.hc;
+  const bool modulate = a.gamma != nullptr;
+  const MmaSmem L = mma_layout(a.D, a.E, modulate);
+  const int NC = L.consumers, P = L.parts, hc = L.cpq;
   const int E = a.E, D = a.D, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int wg_stride = D * 2 + 16;
   const int nchunks = D / 64;
@@ -344,10 +355,9 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
 
   const int nrb = (a.T + kMmaRB - 1) / kMmaRB;
   const int my_rb = (nrb - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-  // lane 0 of warp w: half h of this CTA's j-th row block into the warp's stage 2w + h
-  auto issue = [&](int j, int h) {
+  // lane 0 of warp w: part h of this CTA's j-th row block into stage st (2w or 2w + 1)
+  auto issue = [&](int j, int h, int st) {
     const int rb = blockIdx.x + j * gridDim.x;
-    const int st = 2 * w + h;
     const int z0 = h * hc;
     const int nb = (nchunks - z0) < hc ? (nchunks - z0) : hc;     // blocks inside D
     const uint32_t bar = smem_u32(&full[st]);
@@ -375,7 +385,7 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
                 (uint32_t)(D * 2), smem_u32(wbar));
   }
   __syncthreads();
-  if (lane == 0 && w < my_rb) { issue(w, 0); issue(w, 1); }
+  if (lane == 0 && w < my_rb) { issue(w, 0, 2 * w); issue(w, 1, 2 * w + 1); }
   if (tid < 32) cnt_s[tid] = 0;
   if (blockIdx.x == 0 && a.zero)
     for (int i = tid; i < a.nzero; i += blockDim.x) a.zero[i] = 0u;
@@ -391,10 +401,10 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
 #pragma unroll
   for (int e = 0; e < EMAX; ++e) psum[e] = 0.f;
   bool ok = true;
-  const bool modulate = a.gamma != nullptr;
   float* logit_w = reinterpret_cast<float*>(smem + L.logits) + (size_t)w * kMmaRB * EMAX;
   const uint32_t wg_base = smem_u32(wg_s);
   const int li = lane >> 3, lj = lane & 7;
+  int n = 0;                                        // this warp's part count: part n uses stage 2w + n % 2
   for (int j = w, k = 0; j < my_rb; j += NC, ++k) {
     const int rb = blockIdx.x + j * gridDim.x;
     // four independent accumulator chains (one per k16 step of a 64-column block)
@@ -426,9 +436,9 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
         bulk_commit();
       }
     }
-    for (int h = 0; h < 2; ++h) {
-      const int st = 2 * w + h;
-      if (!modulate) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), k & 1, nullptr, a.status, 100));
+    for (int h = 0; h < P; ++h, ++n) {
+      const int st = 2 * w + (n & 1);
+      if (!modulate) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&full[st]), (n >> 1) & 1, nullptr, a.status, 100));
       if (!ok) break;
       const uint32_t buf = smem_u32(xs + (size_t)st * stage_bytes);
       const int z0 = h * hc;
@@ -458,10 +468,11 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
         }
       }
       __syncwarp();                                  // every lane is done reading the stage
-      if (lane == 0 && j + NC < my_rb) {             // refill it with the next row block's half
+      const int n2 = n + 2, j2 = w + (n2 / P) * NC;  // the stage's next part: this warp's part n + 2
+      if (lane == 0 && j2 < my_rb) {
         if (modulate) bulk_wait_read_all();          // the x_mod store has read the stage
         fence_async_shared();
-        issue(j + NC, h);
+        issue(j2, n2 % P, st);
       }
     }
     if (!ok) break;
@@ -590,10 +601,10 @@ route_kernel_ffma(const __grid_constant__ CUtensorMap tmap_x, RouteArgs a, Final
   if (fin.counts != nullptr && last_block_done(fin.ctr)) finalize_counts_loss<EMAX>(fin, xs);
 }
 
-void route_plan(int T, int D, int E, int b16, int sms, int* tile_rows, int* threads) {
+void route_plan(int T, int D, int E, int b16, int modulate, int sms, int* tile_rows, int* threads) {
   if (b16) {
     *tile_rows = kMmaRB;
-    *threads = mma_layout(D, E).consumers * 32;
+    *threads = mma_layout(D, E, modulate != 0).consumers * 32;
   } else {
     int tile = (T + sms - 1) / sms;
     tile = (tile + 31) / 32 * 32;
@@ -604,22 +615,25 @@ void route_plan(int T, int D, int E, int b16, int sms, int* tile_rows, int* thre
   }
 }
 
-size_t route_smem_total(int D, int E, int tile_rows, int b16) {
-  return b16 ? mma_layout(D, E).total : route_smem_bytes(D, E, tile_rows, 0);
+size_t route_smem_total(int D, int E, int tile_rows, int b16, int modulate) {
+  return b16 ? mma_layout(D, E, modulate != 0).total : route_smem_bytes(D, E, tile_rows, 0);
 }
 
-int route_mma_stages(int D, int E) { return mma_layout(D, E).consumers; }
+int route_mma_stages(int D, int E, int modulate) { return mma_layout(D, E, modulate != 0).consumers; }
+
+int route_box_blocks(int D, int E, int modulate) { return mma_layout(D, E, modulate != 0).cpq; }
 
 cudaError_t launch_route(const RouteArgs& a, const FinalizeArgs& fin, const CUtensorMap* tm, const CUtensorMap* tmm,
                          cudaStream_t s) {
-  const size_t smem = route_smem_total(a.D, a.E, a.tile_rows, a.b16);
+  const bool modulate = a.gamma != nullptr;
+  const size_t smem = route_smem_total(a.D, a.E, a.tile_rows, a.b16, modulate);
   cudaError_t err;
   if (a.b16) {
 #define MOE_ROUTE_MMA(EM, F)                                                                            \
   if (a.E <= EM && (a.f16 != 0) == F) {                                                                 \
     err = cudaFuncSetAttribute(route_kernel_mma<EM, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
     if (err != cudaSuccess) return err;                                                                 \
-    route_kernel_mma<EM, F><<<a.grid, mma_layout(a.D, a.E).consumers * 32, smem, s>>>(*tm, *tmm, a, fin); \
+    route_kernel_mma<EM, F><<<a.grid, mma_layout(a.D, a.E, modulate).consumers * 32, smem, s>>>(*tm, *tmm, a, fin); \
     return cudaGetLastError();                                                                          \
   }
     MOE_ROUTE_MMA(8, false)

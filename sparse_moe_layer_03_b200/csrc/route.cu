@@ -355,6 +355,7 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
 
   const int nrb = (a.T + kMmaRB - 1) / kMmaRB;
   const int my_rb = (nrb - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+  const uint64_t pol_x = policy_evict_last();
   // lane 0 of warp w: part h of this CTA's j-th row block into stage st (2w or 2w + 1)
   auto issue = [&](int j, int h, int st) {
     const int rb = blockIdx.x + j * gridDim.x;
@@ -365,7 +366,8 @@ route_kernel_mma(const __grid_constant__ CUtensorMap tmap_x, const __grid_consta
     if (a.tmap3d) {
       // one box of hc blocks; blocks past D come back zero-filled and count as bytes
       mbar_arrive_expect_tx(bar, stage_bytes);
-      tma_load_3d(dst, &tmap_x, 0, rb * kMmaRB, z0, bar);
+      // x stays in L2 for the dispatch gather, which reads it again right after (75 MB at XL)
+      tma_load_3d_hint(dst, &tmap_x, 0, rb * kMmaRB, z0, bar, pol_x);
     } else {
       mbar_arrive_expect_tx(bar, (uint32_t)nb * kMmaRB * 128);
       for (int c = 0; c < nb; ++c) tma_load_2d(dst + c * (kMmaRB * 128), &tmap_x, (z0 + c) * 64, rb * kMmaRB, bar);

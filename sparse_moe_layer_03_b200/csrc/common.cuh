@@ -455,6 +455,10 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int
                "r"(src), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
+// bring the 128-byte line holding p into L2 (no register result, no completion to wait for)
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 // untiled bulk copy from global memory into this CTA's shared memory, completing on an mbarrier
 // (both addresses 16-byte aligned, the size a multiple of 16)
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

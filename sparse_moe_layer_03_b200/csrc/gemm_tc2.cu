@@ -457,6 +457,20 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       const PairTile ti = pair_decode<BN, kBwd>(tile, pl, a);
       const GemmProblem& pr = a.p[ti.p];
       const CUtensorMap* tO = ti.p ? &to1 : &to0;
+      if (kBwd && !dyn) {
+        // GELU backward: bring this lane's row of u for the pair's next tile (fixed order) into L2
+        // now, a tile ahead of its loads; the epilogue's own loads reach only one box ahead
+        const int nt_ = tile + ncl;
+        if (nt_ < pl.total) {
+          const PairTile tn = pair_decode<BN, kBwd>(nt_, pl, a);
+          const GemmProblem& pn = a.p[tn.p];
+          if (pn.epi == 4 && pn.aux != nullptr && r < tn.valid - (int)rank * 128) {
+            const uint16_t* un = reinterpret_cast<const uint16_t*>(pn.aux) +
+                                 ((long long)tn.row0 + (int)rank * 128 + r) * pn.N + tn.n0;
+            for (int c = 0; c < tn.width; c += 64) prefetch_l2(un + c);
+          }
+        }
+      }
       const int acc = local & 1;
       const uint32_t accph = (local >> 1) & 1;
       if (!mbar_wait(smem_u32(&acc_full[acc]), accph, abort_flag, a.status, 505)) break;

@@ -543,7 +543,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         }
       } else {
       // GELU backward: the stored pre-activation u of the row's next box (64 columns), loaded one
-      // box ahead so that its latency hides behind the current box's work
+      // box ahead so that its latency hides behind the current box's work.  Plain (L1-cached) loads:
+      // a lane's eight 16-byte loads of a box share its row's 128-byte line, which each address
+      // is read once before dU overwrites it (L1 holds no stale copy a later load could see)
       const uint16_t* urow = (kBwd && mode == 4 && rv)
                                  ? reinterpret_cast<const uint16_t*>(pr.aux) + grow * pr.N + ti.n0 : nullptr;
       uint4 unext[8];
@@ -551,7 +553,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
 #pragma unroll
         for (int u = 0; u < 8; ++u)
           unext[u] = (urow && grp * box_cols < ti.width)
-                         ? __ldcg(reinterpret_cast<const uint4*>(urow + grp * box_cols) + u) : make_uint4(0u, 0u, 0u, 0u);
+                         ? *(reinterpret_cast<const uint4*>(urow + grp * box_cols) + u) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll 1
       for (int c0 = grp * box_cols; c0 < ti.width; c0 += box_cols * kPairEpiSplit) {
@@ -562,7 +564,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             ucur[u] = unext[u];
-            unext[u] = (urow && cn < ti.width) ? __ldcg(reinterpret_cast<const uint4*>(urow + cn) + u)
+            unext[u] = (urow && cn < ti.width) ? *(reinterpret_cast<const uint4*>(urow + cn) + u)
                                                : make_uint4(0u, 0u, 0u, 0u);
           }
         }

@@ -37,6 +37,8 @@ SMALL = [
     (1000, 256, 512, 8, 2, 2, "f16", "topk"),     # fp16 storage (DiT inference default)
     (900, 320, 640, 16, 3, 2, "f16", "race"),
     (999, 128, 256, 4, 1, 0, "f16", "topk"),       # no shared experts: separate combine
+    (1200, 640, 1280, 8, 2, 2, "bf16", "topk"),     # 512 + 128-wide column tiles in GEMM2 + combine
+    (900, 1152, 768, 8, 2, 1, "f16", "topk"),      # 2 x 512 + 128
 ]
 
 

@@ -142,7 +142,7 @@ int64_t moe_max_rows(const moe_config_t* cfg);
 /* Zero the first 256 bytes of `ws`: the status word and the counters the kernels keep
  * between launches (asynchronous on `stream`).  Once before first use.
  * Layout of those bytes: status word and error site (0, 4); blocks-done counters of the
- * router (64), the dispatch (128) and the per-image loss (192); the fused GEMM2's count of
+ * router (64) and the per-image loss (192); bytes 128..191 reserved; the fused GEMM2's count of
  * finished routed tiles (224); the CTA-pair GEMM's exit and tile-claim counters (228, 232).
  * Every kernel leaves its counters at zero when it ends.
  * Bytes 240..247 are two test words that only the host writes (zero in normal use); they let a

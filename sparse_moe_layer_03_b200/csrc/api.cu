@@ -553,7 +553,6 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx
   da.tpb = kGatherTokens;
   da.r_max = R;
   da.group_base = ws_at<int32_t>(ws, L.group_base);
-  da.ctr = ws_at<unsigned int>(ws, 128);
   da.offsets = offsets; da.pos = pos; da.row_token = row_token; da.row_gate = row_gate;
   da.x_perm = x_perm;
   da.status = status_ptr(ws);

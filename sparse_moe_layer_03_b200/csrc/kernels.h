@@ -165,7 +165,6 @@ struct DispatchArgs {
   int tpb;                  // tokens per gather block
   long long r_max;
   int32_t* group_base;      // [E,ngroups] scratch: counts, then each group's first row in every segment
-  unsigned int* ctr;        // blocks-done counter in ws (zero between calls)
   int32_t* offsets;         // [E+1]
   int32_t* pos; int32_t* row_token; float* row_gate;
   void* x_perm;             // null: positions only (GEMM1 gathers the rows itself)

@@ -53,11 +53,11 @@ NOMINAL_HBM_GBS = 8000.0         # HBM3e bandwidth named by the workload's targe
 # TRAFFIC_SOURCES_SHA.  Any change to those files makes the reported traffic null until re-measured.
 GEMM_SOURCES = ("sparse_moe_layer_03_b200/csrc/gemm_tc2.cu", "sparse_moe_layer_03_b200/csrc/common.cuh",
                 "sparse_moe_layer_03_b200/csrc/kernels.h")
-TRAFFIC_SOURCES_SHA = "60ff5b37cbaf01e6"
+TRAFFIC_SOURCES_SHA = "e11855240a9a7abd"
 MEASURED_TRAFFIC = {
     # second forward pass of profile_layer at XL (ncu, gpu__time_duration + dram__bytes_read/write)
-    ("xl2_8e2a_512", "gemm1"): 348069888 + 1169803520,
-    ("xl2_8e2a_512", "gemm2_combine"): 1490263040 + 220073728,
+    ("xl2_8e2a_512", "gemm1"): 337147904 + 1168617216,
+    ("xl2_8e2a_512", "gemm2_combine"): 1552899840 + 220297728,
 }
 EXTRA_STEPS = 10                 # timed steps of each other workload in the ``workloads`` key
 

@@ -22,9 +22,10 @@
 //                 the last segment; block 0 writes the offsets.  The other
 //                 blocks take 64 tokens each: one thread per slot turns ranks
 //                 into rows (group base + rank) and writes pos, row_token and
-//                 row_gate; then one warp per token stores its row once per
-//                 selected expert with 16-byte vectors (each warp's first row
-//                 loads before the wait, while the count kernel runs).
+//                 row_gate; then each warp's lane 0 moves its tokens' rows by
+//                 bulk copies through two shared-memory row buffers, storing
+//                 each row once per selected expert (each warp's first row is
+//                 requested before the wait, while the count kernel runs).
 //   A last-block scan inside the count kernel (fence, counter, two rounds of
 //   loads) took half of its 8.6 us, measured with a timer probe.
 #include "common.cuh"
@@ -148,6 +149,13 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_count_kernel(Dispat
       a.pos[(size_t)t * Kmax + k] = ek[k] >= 0 ? wbase[w][ek[k]] + __popc(bal[w][ek[k]] & lt) : -1;
 }
 
+// untiled bulk copy from this CTA's shared memory to global memory, completing in a bulk group
+// (both addresses 16-byte aligned, the size a multiple of 16)
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+}
+
 // One row copy: P x 32 lanes x 16 bytes covers up to P*32 vectors of the row.
 template <int P>
 __device__ __forceinline__ void load_row(const uint4* src, int nvec, int lane, uint4* buf) {
@@ -174,9 +182,15 @@ __device__ __forceinline__ void store_row(uint4* dst, int nvec, int lane, const 
 // warp's first row is loaded before the kernel waits for the count kernel
 // (programmatic dependent launch), so it loads while the counts are scanned (two
 // rows per warp measured the same, with half the blocks resident per SM).
+// P = -1: rows move by bulk copies (TMA): lane 0 of each warp loads a row into one of the warp's
+// two shared-memory row buffers and stores it from there once per selected expert, the next row
+// loading while the current one is stored.  P > 0: 16-byte vectors through registers.
 template <typename T, int P>
 __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, int blk) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  __shared__ uint64_t rbar[kDispatchThreads / 32][2];
+  const uint32_t row_bytes = (uint32_t)a.D * (uint32_t)sizeof(T);
+  uint8_t* rbuf = reinterpret_cast<uint8_t*>(spos) + ((a.tpb * a.Kmax * 4 + 127) & ~127) + (size_t)w * 2 * row_bytes;
   const int Kmax = a.Kmax;
   const int nvec = a.D * (int)sizeof(T) / 16;
   const int t0 = blk * a.tpb;
@@ -188,6 +202,15 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, i
   const bool copy = a.x_perm != nullptr;               // else positions only
   // each warp's first row loads before the wait (x only: it overlaps the count kernel)
   if (P > 0 && copy && w < nt) load_row<P>(xv + (size_t)(t0 + w) * nvec, nvec, lane, buf);
+  if (P < 0 && copy && lane == 0) {
+    mbar_init(smem_u32(&rbar[w][0]), 1);
+    mbar_init(smem_u32(&rbar[w][1]), 1);
+    fence_barrier_init();
+    if (w < nt) {
+      mbar_arrive_expect_tx(smem_u32(&rbar[w][0]), row_bytes);
+      bulk_load(smem_u32(rbuf), xv + (size_t)(t0 + w) * nvec, row_bytes, smem_u32(&rbar[w][0]));
+    }
+  }
   grid_dependency_wait();                              // the count kernel's counts and ranks from here on
   __shared__ int total_s[32], before_s[32];
   __shared__ long long poff_s[33];
@@ -216,6 +239,29 @@ __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, i
   }
   if (!copy) return;
   __syncthreads();
+
+  if (P < 0) {
+    if (lane == 0) {
+      int it = 0;
+      for (int l = w; l < nt; l += NW, ++it) {
+        const int b = it & 1;
+        if (l + NW < nt) {
+          bulk_wait_read_all();                      // the stores out of the other buffer have read it
+          mbar_arrive_expect_tx(smem_u32(&rbar[w][b ^ 1]), row_bytes);
+          bulk_load(smem_u32(rbuf + (b ^ 1) * row_bytes), xv + (size_t)(t0 + l + NW) * nvec, row_bytes,
+                    smem_u32(&rbar[w][b ^ 1]));
+        }
+        if (!mbar_wait(smem_u32(&rbar[w][b]), (uint32_t)(it >> 1) & 1u, nullptr, a.status, 204)) break;
+        for (int k = 0; k < Kmax; ++k) {
+          const int p = spos[l * Kmax + k];
+          if (p >= 0) bulk_store(xp + (size_t)p * nvec, smem_u32(rbuf + b * row_bytes), row_bytes);
+        }
+        bulk_commit();
+      }
+      bulk_wait_all();                               // every row stored before the block ends
+    }
+    return;
+  }
 
   for (int l = w; l < nt; l += NW) {
     const uint4* src = xv + (size_t)(t0 + l) * nvec;
@@ -275,7 +321,7 @@ __device__ void segment_block(const DispatchArgs& a, int e) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(DispatchArgs a, int seg_blocks) {
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(DispatchArgs a, int seg_blocks, int bulk) {
   extern __shared__ int spos[];                       // [tpb * Kmax] rows of the block's slots
   if ((int)blockIdx.x < seg_blocks) {
     grid_dependency_wait();
@@ -284,7 +330,8 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_gather_kernel(Dispa
   }
   const int blk = blockIdx.x - seg_blocks;
   const int nvec = a.D * (int)sizeof(T) / 16;
-  if (nvec <= 4 * 32) gather_block<T, 4>(a, spos, blk);
+  if (bulk) gather_block<T, -1>(a, spos, blk);
+  else if (nvec <= 4 * 32) gather_block<T, 4>(a, spos, blk);
   else if (nvec <= 8 * 32) gather_block<T, 8>(a, spos, blk);
   else gather_block<T, 0>(a, spos, blk);
 }
@@ -308,7 +355,17 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   if (a.tpb <= 0 || kGroup % a.tpb) return cudaErrorInvalidValue;   // a gather block stays inside one group
   const int seg_blocks = a.E + 1;
   const int ggrid = seg_blocks + (a.T + a.tpb - 1) / a.tpb;
-  const size_t smem = (size_t)a.tpb * a.Kmax * sizeof(int);
+  // bulk row copies when the warps' row buffers fit (two rows per warp after the slots' rows)
+  const size_t row_bytes = (size_t)a.D * (a.b16 ? 2 : 4);
+  const size_t smem_bulk = (((size_t)a.tpb * a.Kmax * sizeof(int) + 127) & ~(size_t)127) +
+                           (size_t)(kDispatchThreads / 32) * 2 * row_bytes;
+  const int bulk = a.x_perm != nullptr && smem_bulk <= 160 * 1024 ? 1 : 0;
+  const size_t smem = bulk ? smem_bulk : (size_t)a.tpb * a.Kmax * sizeof(int);
+  if (smem > 48 * 1024) {
+    cudaError_t e2 = a.b16 ? cudaFuncSetAttribute(dispatch_gather_kernel<uint16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
+                           : cudaFuncSetAttribute(dispatch_gather_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e2 != cudaSuccess) return e2;
+  }
   // the gather's first row loads (x only) overlap the count kernel; everything the count kernel
   // writes is read after the wait
   cudaLaunchConfig_t cfg = {};
@@ -318,8 +375,8 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.b16) return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<uint16_t>, a, seg_blocks);
-  return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<float>, a, seg_blocks);
+  if (a.b16) return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<uint16_t>, a, seg_blocks, bulk);
+  return cudaLaunchKernelEx(&cfg, dispatch_gather_kernel<float>, a, seg_blocks, bulk);
 }
 
 }  // namespace moe

@@ -176,15 +176,14 @@ __device__ __forceinline__ void store_row(uint4* dst, int nvec, int lane, const 
 
 // Gather block: tokens [t0, t0 + tpb), all in group g0 = t0 / 256.  Phase 1, one thread per slot,
 // all slots of the block at once: row = segment start + the expert's rows in earlier groups +
-// rank inside the group; writes
-// pos, row_token, row_gate and keeps the row in shared memory.  Phase 2, one
-// warp per token: row loads, then one store of the row per selected slot.  Each
-// warp's first row is loaded before the kernel waits for the count kernel
-// (programmatic dependent launch), so it loads while the counts are scanned (two
-// rows per warp measured the same, with half the blocks resident per SM).
-// P = -1: rows move by bulk copies (TMA): lane 0 of each warp loads a row into one of the warp's
-// two shared-memory row buffers and stores it from there once per selected expert, the next row
-// loading while the current one is stored.  P > 0: 16-byte vectors through registers.
+// rank inside the group; writes pos, row_token, row_gate and keeps the row in shared memory.
+// Phase 2 copies the rows, token l of the block by warp l mod 8, once per selected slot:
+//   P = -1 (when the row buffers fit): bulk copies (TMA); lane 0 of each warp loads a row into one
+//          of the warp's two shared-memory row buffers and stores it from there, the warp's next
+//          row loading while the current one is stored;
+//   P > 0: 16-byte vectors through registers (P per lane; P = 0: wide rows in pieces).
+// Each warp's first row is requested before the kernel waits for the count kernel (programmatic
+// dependent launch), so it loads while the counts are worked out.
 template <typename T, int P>
 __device__ __forceinline__ void gather_block(const DispatchArgs& a, int* spos, int blk) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;

@@ -335,7 +335,16 @@ template <bool FAST>
 __device__ __forceinline__ void gelu_tanh_and_grad(float u, float& g, float& dg) {
   const float c = 0.7978845608028654f, k = 0.044715f;
   const float u2 = u * u;
-  const float t = FAST ? tanh_hw(c * (u + k * u2 * u)) : tanhf(c * (u + k * u2 * u));
+  if (FAST) {
+    // g = u/2 (1 + t), g' = (1 + t)/2 + u/2 (1 - t^2) c (1 + 3 k u^2), t = tanh(u (c k u^2 + c)),
+    // with the products folded into fused multiply-adds
+    const float hu = 0.5f * u;
+    const float t = tanh_hw(u * fmaf(c * k, u2, c));
+    g = fmaf(hu, t, hu);
+    dg = fmaf(hu * fmaf(-t, t, 1.0f), fmaf(3.0f * c * k, u2, c), fmaf(0.5f, t, 0.5f));
+    return;
+  }
+  const float t = tanhf(c * (u + k * u2 * u));
   g = 0.5f * u * (1.0f + t);
   dg = 0.5f * (1.0f + t) + 0.5f * u * (1.0f - t * t) * c * (1.0f + 3.0f * k * u2);
 }

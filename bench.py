@@ -53,11 +53,11 @@ NOMINAL_HBM_GBS = 8000.0         # HBM3e bandwidth named by the workload's targe
 # TRAFFIC_SOURCES_SHA.  Any change to those files makes the reported traffic null until re-measured.
 GEMM_SOURCES = ("sparse_moe_layer_03_b200/csrc/gemm_tc2.cu", "sparse_moe_layer_03_b200/csrc/common.cuh",
                 "sparse_moe_layer_03_b200/csrc/kernels.h")
-TRAFFIC_SOURCES_SHA = "e11855240a9a7abd"
+TRAFFIC_SOURCES_SHA = "ef9625b7a421c62f"
 MEASURED_TRAFFIC = {
     # second forward pass of profile_layer at XL (ncu, gpu__time_duration + dram__bytes_read/write)
-    ("xl2_8e2a_512", "gemm1"): 337147904 + 1168617216,
-    ("xl2_8e2a_512", "gemm2_combine"): 1552899840 + 220297728,
+    ("xl2_8e2a_512", "gemm1"): 364092928 + 1170012928,
+    ("xl2_8e2a_512", "gemm2_combine"): 1505018112 + 221867264,
 }
 EXTRA_STEPS = 10                 # timed steps of each other workload in the ``workloads`` key
 

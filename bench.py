@@ -52,12 +52,13 @@ NOMINAL_HBM_GBS = 8000.0         # HBM3e bandwidth named by the workload's targe
 # full size), valid only for the GEMM sources they were measured on: GEMM_SOURCES hashed to
 # TRAFFIC_SOURCES_SHA.  Any change to those files makes the reported traffic null until re-measured.
 GEMM_SOURCES = ("sparse_moe_layer_03_b200/csrc/gemm_tc2.cu", "sparse_moe_layer_03_b200/csrc/common.cuh",
-                "sparse_moe_layer_03_b200/csrc/kernels.h")
-TRAFFIC_SOURCES_SHA = "ef9625b7a421c62f"
+                "sparse_moe_layer_03_b200/csrc/kernels.h",
+                "sparse_moe_layer_03_b200/csrc/api.cu")      # api.cu builds the tensor maps the GEMMs load through
+TRAFFIC_SOURCES_SHA = "37acbc2e8c9b76aa"
 MEASURED_TRAFFIC = {
     # second forward pass of profile_layer at XL (ncu, gpu__time_duration + dram__bytes_read/write)
-    ("xl2_8e2a_512", "gemm1"): 364092928 + 1170012928,
-    ("xl2_8e2a_512", "gemm2_combine"): 1505018112 + 221867264,
+    ("xl2_8e2a_512", "gemm1"): 346237696 + 1170529024,
+    ("xl2_8e2a_512", "gemm2_combine"): 1496586752 + 220761344,
 }
 EXTRA_STEPS = 10                 # timed steps of each other workload in the ``workloads`` key
 

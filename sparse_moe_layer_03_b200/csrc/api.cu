@@ -626,7 +626,15 @@ int run_gemm(const moe_config_t* cfg, GemmArgs& g, const void* A0, long long row
     g.sched_ctr = ws_at<unsigned int>(ws, kWsSchedCtr);
     g.exit_ctr = ws_at<unsigned int>(ws, kWsExitCtr);
     g.test = ws_at<const uint32_t>(ws, kWsTestWords);
-    if ((e = launch_gemm_pair(g, ta, tb, to, bn, num_sms_current(), cfg->gemm_pairs, s)) != cudaSuccess)
+    // B maps with half-height boxes for the narrower column tile (N = 1152: the last 128 columns)
+    CUtensorMap tbn[2];
+    if ((rc = make_tmap(&tbn[0], B0, cfg->dtype, brows0, K0, brows_box / 2, "B0 (narrow tiles)"))) return rc;
+    if (g.nprob > 1) {
+      if ((rc = make_tmap(&tbn[1], B1, cfg->dtype, brows1, bcols1, brows_box / 2, "B1 (narrow tiles)"))) return rc;
+    } else {
+      tbn[1] = tbn[0];
+    }
+    if ((e = launch_gemm_pair(g, ta, tb, to, tbn, bn, num_sms_current(), cfg->gemm_pairs, s)) != cudaSuccess)
       return cuda_fail(e, "tcgen05 CTA-pair expert GEMM");
     return ok();
   }
@@ -675,7 +683,7 @@ int launch_pair_problems(const moe_config_t* cfg, GemmArgs& g, const OperandMap*
   g.sched_ctr = ws_at<unsigned int>(ws, kWsSchedCtr);
   g.exit_ctr = ws_at<unsigned int>(ws, kWsExitCtr);
   g.test = ws_at<const uint32_t>(ws, kWsTestWords);
-  const cudaError_t e = launch_gemm_pair(g, ta, tb, to, 256, num_sms_current(), cfg->gemm_pairs, s);
+  const cudaError_t e = launch_gemm_pair(g, ta, tb, to, nullptr, 256, num_sms_current(), cfg->gemm_pairs, s);
   if (e != cudaSuccess) return cuda_fail(e, "tcgen05 CTA-pair GEMM (backward)");
   return MOE_OK;
 }

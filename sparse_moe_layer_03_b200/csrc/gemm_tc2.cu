@@ -185,7 +185,8 @@ template <int BN, typename S, int F>
 __global__ void __launch_bounds__(pair_threads<F>(), 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant__ CUtensorMap tb0,
                  const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
-                 const __grid_constant__ CUtensorMap to0, const __grid_constant__ CUtensorMap to1, GemmArgs a) {
+                 const __grid_constant__ CUtensorMap to0, const __grid_constant__ CUtensorMap to1,
+                 const __grid_constant__ CUtensorMap tbn0, const __grid_constant__ CUtensorMap tbn1, GemmArgs a) {
   using C = PairCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -276,6 +277,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
     prefetch_tmap(&tb1);
     prefetch_tmap(&to0);
     prefetch_tmap(&to1);
+    if (a.b_half) {
+      prefetch_tmap(&tbn0);
+      prefetch_tmap(&tbn1);
+    }
   }
   if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
   tc_fence_before();
@@ -327,6 +332,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       const int ksplit = pr.ksplit;
       const int nrows = pr.N;
       const bool gather = kGather && pr.gather_rows != nullptr;   // the gather warps bring this tile's A rows
+      // a tile at most BN/2 wide reads BN/4 B rows per CTA: load only those (a 16 KB box would bring
+      // twice the B bytes the MMAs use, and these tiles are bound by their operand loads)
+      const bool half_b = a.b_half && 2 * ti.width <= BN && !(kBwd && pr.b_mn);
+      const CUtensorMap* tBk = half_b ? (ti.p ? &tbn1 : &tbn0) : tB;
+      const uint32_t bbytes = half_b ? C::B_BYTES / 2 : C::B_BYTES;
       for (int kb = 0; kb < ti.nk; ++kb) {
         int ok = 1;
         if (lane == 0) ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.status, 501) ? 1 : 0;
@@ -336,9 +346,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         const uint32_t fb_leader = map_to_cta(fb_local, 0);
         uint8_t* sa = stage_base + stage * C::STAGE;
         if (lane == 0) {
-          if (rank == 0) mbar_arrive_expect_tx(fb_local, gather ? 2 * C::B_BYTES : 2 * C::STAGE);   // both CTAs' TMA bytes
+          if (rank == 0) mbar_arrive_expect_tx(fb_local, gather ? 2 * bbytes : 2 * (C::A_BYTES + bbytes));   // both CTAs' TMA bytes
           const int bx = ksplit ? (kb * kPairBK) % ksplit : kb * kPairBK;
-          // each CTA holds half of the tile's B rows (a narrower tile's box also brings rows it does not use)
+          // each CTA holds half of the tile's B rows (for a tile between BN/2 and BN wide, the box also
+          // brings rows it does not use)
           const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (ti.width / 2);
           if (kBwd && pr.a_mn) {
             // A held [K rows, M columns]: this CTA's 128 M columns as two 64-column boxes of 64 K rows
@@ -359,7 +370,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
               tma_load_2d_pair(smem_u32(sa + C::A_BYTES) + 8192 * i, tB, x, y, fb_leader, pol_w);
             }
           } else {
-            tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tB, bx, by, fb_leader, pol_w);
+            tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tBk, bx, by, fb_leader, pol_w);
           }
         }
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -785,7 +796,8 @@ done:
 
 template <int BN, typename S, int F>
 static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb,
-                                  const CUtensorMap* to, int num_sms, int max_pairs, cudaStream_t s) {
+                                  const CUtensorMap* to, const CUtensorMap* tbn, int num_sms, int max_pairs,
+                                  cudaStream_t s) {
   using C = PairCfg<BN>;
   cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<BN, S, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (err != cudaSuccess) return err;
@@ -824,7 +836,11 @@ static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, cons
   const int grid = pair_grid(num_sms, pairs, max_pairs);
   if (grid < 2) return cudaErrorInvalidConfiguration;
   cfg.gridDim = dim3(grid, 1, 1);
-  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, S, F>, ta[0], tb[0], ta[1], tb[1], to[0], to[1], a);
+  GemmArgs ak = a;
+  ak.b_half = tbn != nullptr ? 1 : 0;
+  const CUtensorMap* tn = tbn != nullptr ? tbn : tb;
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<BN, S, F>, ta[0], tb[0], ta[1], tb[1], to[0], to[1], tn[0], tn[1],
+                            ak);
 }
 
 // Tiles are 256 columns wide, with one narrower tile (a multiple of 64 columns)
@@ -836,7 +852,7 @@ int gemm_pair_pick_bn(int n0, int n1) {
 }
 
 cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, const CUtensorMap* to,
-                             int bn, int num_sms, int max_pairs, cudaStream_t s) {
+                             const CUtensorMap* tbn, int bn, int num_sms, int max_pairs, cudaStream_t s) {
   if (bn != 256) return cudaErrorInvalidValue;
   int f = 0;
   if (a.nprob > 1 && a.p[1].epi == 2 && a.done_ctr != nullptr) f |= kFeatClaim;
@@ -849,8 +865,8 @@ cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUt
   if ((f & kFeatClaim) && a.sched_ctr == nullptr) return cudaErrorInvalidValue;
 #define MOE_PAIR_LAUNCH(FEAT)                                                                    \
   case FEAT:                                                                                     \
-    return a.f16 ? launch_pair_bn<256, StoreF16, FEAT>(a, ta, tb, to, num_sms, max_pairs, s)    \
-                 : launch_pair_bn<256, StoreBF16, FEAT>(a, ta, tb, to, num_sms, max_pairs, s);
+    return a.f16 ? launch_pair_bn<256, StoreF16, FEAT>(a, ta, tb, to, tbn, num_sms, max_pairs, s)    \
+                 : launch_pair_bn<256, StoreBF16, FEAT>(a, ta, tb, to, tbn, num_sms, max_pairs, s);
   switch (f) {
     MOE_PAIR_LAUNCH(0)
     MOE_PAIR_LAUNCH(kFeatClaim)

@@ -227,12 +227,16 @@ struct GemmArgs {
   const void* x_res;        // adaLN-Zero residual in the epi-2 output: x_res + alpha[t / img_len] * sum, or null
   const void* alpha;
   int img_len;
+  int b_half;               // CTA-pair kernel (set by its launcher): tiles at most BN/2 wide load their B rows
+                            // through the half-height boxes of the tbn maps
 };
 cudaError_t launch_gemm_tc(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, int bn,
                            int num_sms, cudaStream_t s);
 int gemm_tc_pick_bn(int n0, int n1);
+// tbn: the two problems' B maps with boxes of bn/4 rows (half of a CTA's usual B box), used by the
+// tiles at most bn/2 wide so that they do not load rows they never read; null: every tile uses tb
 cudaError_t launch_gemm_pair(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb, const CUtensorMap* to,
-                             int bn, int num_sms, int max_pairs, cudaStream_t s);
+                             const CUtensorMap* tbn, int bn, int num_sms, int max_pairs, cudaStream_t s);
 int gemm_pair_pick_bn(int n0, int n1);
 cudaError_t launch_gemm_simt(const GemmArgs& a, cudaStream_t s);
 

@@ -56,22 +56,27 @@ constexpr int kFeatGather = 2;            // routed A rows copied from x by the 
 constexpr int kFeatBwd = 4;               // MN-major operands, weight-gradient problems, fp32 output, GELU backward
 template <int F>
 constexpr int pair_threads() { return 64 + 32 * kPairEpiWarps + ((F & kFeatGather) ? 32 * kPairGatherWarps : 0); }
+// 64-wide k-blocks per pipeline stage: two in the forward instantiations, one where the backward's
+// operand forms or the gather warps fill the stages
+template <int F>
+constexpr int pair_kps() { return (F & (kFeatBwd | kFeatGather)) ? 1 : 2; }
 constexpr int kPairSmemLimit = 232448;
 constexpr int kSchedSlots = 4;                                  // tile ids handed out ahead
 constexpr int kSchedConsumers = 2 + 2 * kPairEpiWarps;          // peer producer, MMA issuer, epilogue warps
 
-template <int BN>
+template <int BN, int KPS = 1>
 struct PairCfg {
-  static constexpr int A_BYTES = 128 * kPairBK * 2;
+  static constexpr int A_BYTES = 128 * kPairBK * 2;     // one k-block of this CTA's A rows
   static constexpr int B_BYTES = (BN / 2) * kPairBK * 2;
-  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int KB_BYTES = A_BYTES + B_BYTES;    // one k-block: its A box, then its B box
+  static constexpr int STAGE = KPS * KB_BYTES;
   // epilogue staging: two 32 rows x 128 bytes buffers per epilogue warp for TMA stores
   // (a single buffer, trading 16 KB for one more operand stage, measured 1.8x slower on GEMM1)
   static constexpr int EPI_BYTES = kPairEpiWarps * 2 * 4096;
   // keep 4 KB of the 227 KB for barriers, the 1 KB alignment slack and static shared memory
-  // (with 4 epilogue warps this gives 5 stages; a 6th, which fits in 3 KB, measured 3% slower
-  // on GEMM2 + combine at XL)
-  static constexpr int FIT = (kPairSmemLimit - 4096 - EPI_BYTES) / STAGE;
+  // (with 4 epilogue warps and one k-block per stage this gives 5 stages; a 6th, which fits in 3 KB,
+  // measured 3% slower on GEMM2 + combine at XL); with two k-blocks per stage, 3 stages fit in 3 KB
+  static constexpr int FIT = (kPairSmemLimit - (KPS > 1 ? 3072 : 4096) - EPI_BYTES) / STAGE;
   static constexpr int STAGES = FIT > 8 ? 8 : FIT;
   static constexpr int SMEM = STAGES * STAGE + EPI_BYTES + 2048;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
@@ -187,7 +192,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
                  const __grid_constant__ CUtensorMap ta1, const __grid_constant__ CUtensorMap tb1,
                  const __grid_constant__ CUtensorMap to0, const __grid_constant__ CUtensorMap to1,
                  const __grid_constant__ CUtensorMap tbn0, const __grid_constant__ CUtensorMap tbn1, GemmArgs a) {
-  using C = PairCfg<BN>;
+  constexpr int kKps = pair_kps<F>();
+  using C = PairCfg<BN, kKps>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* stage_base = smem;
@@ -337,40 +343,46 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
       const bool half_b = a.b_half && 2 * ti.width <= BN && !(kBwd && pr.b_mn);
       const CUtensorMap* tBk = half_b ? (ti.p ? &tbn1 : &tbn0) : tB;
       const uint32_t bbytes = half_b ? C::B_BYTES / 2 : C::B_BYTES;
-      for (int kb = 0; kb < ti.nk; ++kb) {
+      for (int kb0 = 0; kb0 < ti.nk; kb0 += kKps) {
         int ok = 1;
         if (lane == 0) ok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag, a.status, 501) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { alive = false; break; }
         const uint32_t fb_local = smem_u32(&full[stage]);
         const uint32_t fb_leader = map_to_cta(fb_local, 0);
-        uint8_t* sa = stage_base + stage * C::STAGE;
+        // the stage's k-blocks (the last stage of a tile may hold fewer), each an A box then a B box
+        const int nkb = ti.nk - kb0 < kKps ? ti.nk - kb0 : kKps;
         if (lane == 0) {
-          if (rank == 0) mbar_arrive_expect_tx(fb_local, gather ? 2 * bbytes : 2 * (C::A_BYTES + bbytes));   // both CTAs' TMA bytes
-          const int bx = ksplit ? (kb * kPairBK) % ksplit : kb * kPairBK;
-          // each CTA holds half of the tile's B rows (for a tile between BN/2 and BN wide, the box also
-          // brings rows it does not use)
-          const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (ti.width / 2);
-          if (kBwd && pr.a_mn) {
-            // A held [K rows, M columns]: this CTA's 128 M columns as two 64-column boxes of 64 K rows
-            const int ax = ti.row0 + (int)rank * 128, ay = ti.k0 + kb * kPairBK;
-            tma_load_2d_pair(smem_u32(sa), tA, ax, ay, fb_leader, pol_a);
-            tma_load_2d_pair(smem_u32(sa) + 8192, tA, ax + 64, ay, fb_leader, pol_a);
-          } else if (!gather) {
-            tma_load_2d_pair(smem_u32(sa), tA, kb * kPairBK, ti.row0 + (int)rank * 128, fb_leader, pol_a);
-          }
-          if (kBwd && pr.b_mn) {
-            // B held [K rows, N columns]: this CTA's half of the tile's columns as two 64-column boxes
-            // (a narrower tile's second box brings columns it does not use, zeros past the tensor)
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const int n = ti.n0 + (int)rank * (ti.width / 2) + 64 * i;
-              int x = n, y = ti.bk0 + kb * kPairBK;
-              if (pr.b_split) { x = n % pr.b_split; y += (n / pr.b_split) * pr.K; }
-              tma_load_2d_pair(smem_u32(sa + C::A_BYTES) + 8192 * i, tB, x, y, fb_leader, pol_w);
+          if (rank == 0)                                  // both CTAs' TMA bytes
+            mbar_arrive_expect_tx(fb_local, (uint32_t)nkb * (gather ? 2 * bbytes : 2 * (C::A_BYTES + bbytes)));
+          for (int j = 0; j < nkb; ++j) {
+            const int kb = kb0 + j;
+            uint8_t* sa = stage_base + stage * C::STAGE + j * C::KB_BYTES;
+            const int bx = ksplit ? (kb * kPairBK) % ksplit : kb * kPairBK;
+            // each CTA holds half of the tile's B rows (for a tile between BN/2 and BN wide, the box also
+            // brings rows it does not use)
+            const int by = (ksplit ? ((kb * kPairBK) / ksplit) * nrows : 0) + ti.brow + (int)rank * (ti.width / 2);
+            if (kBwd && pr.a_mn) {
+              // A held [K rows, M columns]: this CTA's 128 M columns as two 64-column boxes of 64 K rows
+              const int ax = ti.row0 + (int)rank * 128, ay = ti.k0 + kb * kPairBK;
+              tma_load_2d_pair(smem_u32(sa), tA, ax, ay, fb_leader, pol_a);
+              tma_load_2d_pair(smem_u32(sa) + 8192, tA, ax + 64, ay, fb_leader, pol_a);
+            } else if (!gather) {
+              tma_load_2d_pair(smem_u32(sa), tA, kb * kPairBK, ti.row0 + (int)rank * 128, fb_leader, pol_a);
             }
-          } else {
-            tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tBk, bx, by, fb_leader, pol_w);
+            if (kBwd && pr.b_mn) {
+              // B held [K rows, N columns]: this CTA's half of the tile's columns as two 64-column boxes
+              // (a narrower tile's second box brings columns it does not use, zeros past the tensor)
+#pragma unroll
+              for (int i = 0; i < 2; ++i) {
+                const int n = ti.n0 + (int)rank * (ti.width / 2) + 64 * i;
+                int x = n, y = ti.bk0 + kb * kPairBK;
+                if (pr.b_split) { x = n % pr.b_split; y += (n / pr.b_split) * pr.K; }
+                tma_load_2d_pair(smem_u32(sa + C::A_BYTES) + 8192 * i, tB, x, y, fb_leader, pol_w);
+              }
+            } else {
+              tma_load_2d_pair(smem_u32(sa + C::A_BYTES), tBk, bx, by, fb_leader, pol_w);
+            }
           }
         }
         if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -401,18 +413,21 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap ta0, const __grid_constant_
         const uint32_t idesc = idesc_f16kind_f32(kPairBM, ti.width, S::kFmt) | (kBwd ? idesc_major_bits(amn, bmn) : 0u);
         // a k16 step advances 32 bytes inside a K-major row, or 16 rows (2048 bytes) of an MN-major tile
         const uint64_t astep = amn ? 128 : 2, bstep = bmn ? 128 : 2;
-        for (int kb = 0; kb < ti.nk; ++kb) {
+        for (int kb0 = 0; kb0 < ti.nk; kb0 += kKps) {
           // gathered rows arrive from both CTAs' gather warps (cluster scope); else TMA only
           if (!(gather_lsu ? mbar_wait_cluster(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)
                            : mbar_wait(smem_u32(&full[stage]), phase, abort_flag, a.status, 503)))
             goto mma_out;
           tc_fence_after();
-          const uint32_t sa = smem_u32(stage_base + stage * C::STAGE);
-          const uint64_t adesc = amn ? smem_desc_mn_sw128(sa) : smem_desc_sw128(sa);
-          const uint64_t bdesc = bmn ? smem_desc_mn_sw128(sa + C::A_BYTES) : smem_desc_sw128(sa + C::A_BYTES);
+          const int nkb = ti.nk - kb0 < kKps ? ti.nk - kb0 : kKps;
+          for (int j = 0; j < nkb; ++j) {
+            const uint32_t sa = smem_u32(stage_base + stage * C::STAGE + j * C::KB_BYTES);
+            const uint64_t adesc = amn ? smem_desc_mn_sw128(sa) : smem_desc_sw128(sa);
+            const uint64_t bdesc = bmn ? smem_desc_mn_sw128(sa + C::A_BYTES) : smem_desc_sw128(sa + C::A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < kPairBK / 16; ++kk)
-            umma_kindf16_pair(d, adesc + astep * kk, bdesc + bstep * kk, idesc, (kb | kk) ? 1u : 0u);
+            for (int kk = 0; kk < kPairBK / 16; ++kk)
+              umma_kindf16_pair(d, adesc + astep * kk, bdesc + bstep * kk, idesc, ((kb0 + j) | kk) ? 1u : 0u);
+          }
           issued_any = true;
           // stage free in both CTAs once these MMAs finish
           const uint32_t eb = smem_u32(&empty[stage]);
@@ -798,7 +813,7 @@ template <int BN, typename S, int F>
 static cudaError_t launch_pair_bn(const GemmArgs& a, const CUtensorMap* ta, const CUtensorMap* tb,
                                   const CUtensorMap* to, const CUtensorMap* tbn, int num_sms, int max_pairs,
                                   cudaStream_t s) {
-  using C = PairCfg<BN>;
+  using C = PairCfg<BN, pair_kps<F>()>;
   cudaError_t err = cudaFuncSetAttribute(gemm_pair_kernel<BN, S, F>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};

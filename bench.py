@@ -54,11 +54,11 @@ NOMINAL_HBM_GBS = 8000.0         # HBM3e bandwidth named by the workload's targe
 GEMM_SOURCES = ("sparse_moe_layer_03_b200/csrc/gemm_tc2.cu", "sparse_moe_layer_03_b200/csrc/common.cuh",
                 "sparse_moe_layer_03_b200/csrc/kernels.h",
                 "sparse_moe_layer_03_b200/csrc/api.cu")      # api.cu builds the tensor maps the GEMMs load through
-TRAFFIC_SOURCES_SHA = "37acbc2e8c9b76aa"
+TRAFFIC_SOURCES_SHA = "739292302fa1c5d8"
 MEASURED_TRAFFIC = {
     # second forward pass of profile_layer at XL (ncu, gpu__time_duration + dram__bytes_read/write)
-    ("xl2_8e2a_512", "gemm1"): 346237696 + 1170529024,
-    ("xl2_8e2a_512", "gemm2_combine"): 1496586752 + 220761344,
+    ("xl2_8e2a_512", "gemm1"): 335237888 + 1167026432,
+    ("xl2_8e2a_512", "gemm2_combine"): 1499219968 + 220247296,
 }
 EXTRA_STEPS = 10                 # timed steps of each other workload in the ``workloads`` key
 

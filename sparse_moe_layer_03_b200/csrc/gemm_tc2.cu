@@ -56,10 +56,9 @@ constexpr int kFeatGather = 2;            // routed A rows copied from x by the 
 constexpr int kFeatBwd = 4;               // MN-major operands, weight-gradient problems, fp32 output, GELU backward
 template <int F>
 constexpr int pair_threads() { return 64 + 32 * kPairEpiWarps + ((F & kFeatGather) ? 32 * kPairGatherWarps : 0); }
-// 64-wide k-blocks per pipeline stage: two in the forward instantiations, one where the backward's
-// operand forms or the gather warps fill the stages
+// 64-wide k-blocks per pipeline stage: two, or one where the gather warps fill the stages' A rows
 template <int F>
-constexpr int pair_kps() { return (F & (kFeatBwd | kFeatGather)) ? 1 : 2; }
+constexpr int pair_kps() { return (F & kFeatGather) ? 1 : 2; }
 constexpr int kPairSmemLimit = 232448;
 constexpr int kSchedSlots = 4;                                  // tile ids handed out ahead
 constexpr int kSchedConsumers = 2 + 2 * kPairEpiWarps;          // peer producer, MMA issuer, epilogue warps

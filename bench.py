@@ -54,11 +54,11 @@ NOMINAL_HBM_GBS = 8000.0         # HBM3e bandwidth named by the workload's targe
 GEMM_SOURCES = ("sparse_moe_layer_03_b200/csrc/gemm_tc2.cu", "sparse_moe_layer_03_b200/csrc/common.cuh",
                 "sparse_moe_layer_03_b200/csrc/kernels.h",
                 "sparse_moe_layer_03_b200/csrc/api.cu")      # api.cu builds the tensor maps the GEMMs load through
-TRAFFIC_SOURCES_SHA = "7fa12267e91d0916"
+TRAFFIC_SOURCES_SHA = "e092bedd6c63be57"
 MEASURED_TRAFFIC = {
     # second forward pass of profile_layer at XL (ncu, gpu__time_duration + dram__bytes_read/write)
-    ("xl2_8e2a_512", "gemm1"): 335875584 + 1168662272,
-    ("xl2_8e2a_512", "gemm2_combine"): 1493750016 + 221108736,
+    ("xl2_8e2a_512", "gemm1"): 335233536 + 1166943488,
+    ("xl2_8e2a_512", "gemm2_combine"): 1487715840 + 219694080,
 }
 EXTRA_STEPS = 10                 # timed steps of each other workload in the ``workloads`` key
 

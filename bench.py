@@ -54,11 +54,11 @@ NOMINAL_HBM_GBS = 8000.0         # HBM3e bandwidth named by the workload's targe
 GEMM_SOURCES = ("sparse_moe_layer_03_b200/csrc/gemm_tc2.cu", "sparse_moe_layer_03_b200/csrc/common.cuh",
                 "sparse_moe_layer_03_b200/csrc/kernels.h",
                 "sparse_moe_layer_03_b200/csrc/api.cu")      # api.cu builds the tensor maps the GEMMs load through
-TRAFFIC_SOURCES_SHA = "e092bedd6c63be57"
+TRAFFIC_SOURCES_SHA = "a7f379751030705b"
 MEASURED_TRAFFIC = {
     # second forward pass of profile_layer at XL (ncu, gpu__time_duration + dram__bytes_read/write)
-    ("xl2_8e2a_512", "gemm1"): 335233536 + 1166943488,
-    ("xl2_8e2a_512", "gemm2_combine"): 1487715840 + 219694080,
+    ("xl2_8e2a_512", "gemm1"): 335290112 + 1168311040,
+    ("xl2_8e2a_512", "gemm2_combine"): 1495313920 + 220181760,
 }
 EXTRA_STEPS = 10                 # timed steps of each other workload in the ``workloads`` key
 

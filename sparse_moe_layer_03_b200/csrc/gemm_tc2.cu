@@ -83,6 +83,9 @@ struct PairCfg {
   static constexpr int STAGES = FIT > 8 ? 8 : FIT;
   static constexpr int SMEM = STAGES * STAGE + EPI_BYTES + 2048;
   static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+  static_assert(STAGES >= 2, "the operand ring needs two stages at least");
+  static_assert(SMEM <= kPairSmemLimit, "shared memory above the per-block limit");
+  static_assert(STAGE % 1024 == 0, "stages must keep the 1024-byte alignment of the 128-byte swizzle");
 };
 
 struct PairPlan {
